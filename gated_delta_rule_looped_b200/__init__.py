@@ -1,0 +1,206 @@
+"""Python binding of liblt2gdr.so, the B200 looped gated-delta-rule mixer.
+
+Thin ctypes layer over the C ABI of include/lt2_gdr.h with the same names
+(lt2_gdr_prefill, lt2_gdr_decode, lt2_gdr_prefill_workspace_bytes, lt2_gdr_last_device_error,
+lt2_status_string).  It only marshals arguments: torch tensors are passed as raw device
+pointers together with the current CUDA stream, and every step of the computation runs in
+the library's kernels.  ``prefill`` and ``decode`` are conveniences that allocate outputs
+with torch and raise on a non-OK status.
+
+The shared library is loaded on first use; if it is missing the call raises (there is no
+fallback implementation).
+"""
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblt2gdr.so")
+
+LT2_OK = 0
+LT2_ERR_INVALID_ARGUMENT = 1
+LT2_ERR_UNSUPPORTED = 2
+LT2_ERR_WORKSPACE = 3
+LT2_ERR_CUDA = 4
+LT2_ERR_DEVICE_TIMEOUT = 5
+
+LT2_DTYPE_F32 = 0
+LT2_DTYPE_BF16 = 1
+LT2_GATE_SCALAR = 0
+LT2_GATE_PER_KEY = 1
+LT2_ALGO_AUTO = 0
+LT2_ALGO_TENSOR_CORE = 1
+LT2_ALGO_CUDA_CORE = 2
+LT2_OUT_SAME = 0
+LT2_OUT_F32 = 1
+LT2_OUT_BF16 = 2
+
+# Every symbol include/lt2_gdr.h declares.
+EXPORTS = (
+    "lt2_gdr_prefill_workspace_bytes",
+    "lt2_gdr_prefill",
+    "lt2_gdr_decode",
+    "lt2_gdr_last_device_error",
+    "lt2_status_string",
+    "lt2_last_cuda_error_string",
+    "lt2_gdr_version",
+)
+
+
+class lt2_gdr_dims(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("B", ctypes.c_int64), ("H", ctypes.c_int64),
+                ("L", ctypes.c_int64), ("dk", ctypes.c_int64), ("dv", ctypes.c_int64),
+                ("dtype", ctypes.c_int32), ("gate", ctypes.c_int32), ("algo", ctypes.c_int32),
+                ("out_dtype", ctypes.c_int32)]
+
+
+class Lt2Error(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        extra = ""
+        if status == LT2_ERR_CUDA:
+            extra = ": " + lib().lt2_last_cuda_error_string().decode()
+        super().__init__(f"{where} returned {lt2_status_string(status)}{extra}")
+
+
+_LIB = None
+
+
+def lib():
+    """The loaded liblt2gdr.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m gated_delta_rule_looped_b200.build` (no fallback exists)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, fp = ctypes.c_void_p, ctypes.c_void_p
+        dims_p = ctypes.POINTER(lt2_gdr_dims)
+        L.lt2_gdr_prefill_workspace_bytes.argtypes = [dims_p]
+        L.lt2_gdr_prefill_workspace_bytes.restype = ctypes.c_size_t
+        L.lt2_gdr_prefill.argtypes = [dims_p, vp, vp, vp, fp, fp, fp, vp, fp, vp,
+                                      ctypes.c_size_t, vp]
+        L.lt2_gdr_prefill.restype = ctypes.c_int
+        L.lt2_gdr_decode.argtypes = [dims_p, vp, vp, vp, fp, fp, fp, vp, vp]
+        L.lt2_gdr_decode.restype = ctypes.c_int
+        L.lt2_gdr_last_device_error.argtypes = []
+        L.lt2_gdr_last_device_error.restype = ctypes.c_int
+        L.lt2_status_string.argtypes = [ctypes.c_int]
+        L.lt2_status_string.restype = ctypes.c_char_p
+        L.lt2_last_cuda_error_string.argtypes = []
+        L.lt2_last_cuda_error_string.restype = ctypes.c_char_p
+        L.lt2_gdr_version.argtypes = []
+        L.lt2_gdr_version.restype = ctypes.c_int
+        _LIB = L
+    return _LIB
+
+
+def make_dims(T, B, H, L, dk, dv, dtype=LT2_DTYPE_BF16, gate=LT2_GATE_SCALAR,
+              algo=LT2_ALGO_AUTO, out_dtype=LT2_OUT_SAME):
+    return lt2_gdr_dims(T, B, H, L, dk, dv, dtype, gate, algo, out_dtype)
+
+
+def _p(x):
+    """Raw pointer of a tensor (or None / an int address passed through)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# --- the C ABI, same names ---------------------------------------------------------------
+
+def lt2_gdr_prefill_workspace_bytes(dims):
+    return lib().lt2_gdr_prefill_workspace_bytes(ctypes.byref(dims))
+
+
+def lt2_gdr_prefill(dims, q, k, v, alpha, beta, S0, o, S_out, workspace=None,
+                    workspace_bytes=0, stream=None):
+    return lib().lt2_gdr_prefill(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(alpha), _p(beta),
+                                 _p(S0), _p(o), _p(S_out), _p(workspace), int(workspace_bytes),
+                                 _stream(stream))
+
+
+def lt2_gdr_decode(dims, q, k, v, alpha, beta, S, o, stream=None):
+    return lib().lt2_gdr_decode(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(alpha), _p(beta),
+                                _p(S), _p(o), _stream(stream))
+
+
+def lt2_gdr_last_device_error():
+    return lib().lt2_gdr_last_device_error()
+
+
+def lt2_status_string(status):
+    return lib().lt2_status_string(int(status)).decode()
+
+
+# --- conveniences on torch tensors ---------------------------------------------------------
+
+_OUT = {None: LT2_OUT_SAME, "same": LT2_OUT_SAME, "f32": LT2_OUT_F32, "bf16": LT2_OUT_BF16}
+
+
+def _out_torch_dtype(in_dtype, out):
+    import torch
+    if out in (None, "same"):
+        return in_dtype
+    return torch.float32 if out == "f32" else torch.bfloat16
+
+
+def _dims_from(q, v, alpha, per_key, algo, out=None):
+    import torch
+    if q.dim() != 5 or v.dim() != 5:
+        raise ValueError("q, k, v must be [T, B, H, L, d]")
+    T, B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    dt = {torch.float32: LT2_DTYPE_F32, torch.bfloat16: LT2_DTYPE_BF16}.get(q.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    if per_key is None:
+        per_key = alpha.dim() == 5
+    return make_dims(T, B, H, L, dk, dv, dt, LT2_GATE_PER_KEY if per_key else LT2_GATE_SCALAR,
+                     algo, _OUT[out])
+
+
+def prefill(q, k, v, alpha, beta, S0=None, per_key=None, algo=LT2_ALGO_AUTO, o=None,
+            S_out=None, out=None, stream=None):
+    """Run the looped prefill on CUDA tensors; returns (o, S_out).  ``out`` selects the
+    storage type of o: None/"same" (as the inputs), "f32" or "bf16"."""
+    import torch
+    dims = _dims_from(q, v, alpha, per_key, algo, out)
+    if o is None:
+        o = torch.empty(v.shape, dtype=_out_torch_dtype(q.dtype, out), device=v.device)
+    if S_out is None:
+        S_out = torch.empty(tuple(q.shape[:3]) + (q.shape[-1], v.shape[-1]),
+                            dtype=torch.float32, device=q.device)
+    ws_bytes = lt2_gdr_prefill_workspace_bytes(dims)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device) if ws_bytes else None
+    st = lt2_gdr_prefill(dims, q, k, v, alpha, beta, S0, o, S_out, ws, ws_bytes, stream)
+    if st != LT2_OK:
+        raise Lt2Error(st, "lt2_gdr_prefill")
+    return o, S_out
+
+
+def decode(q, k, v, alpha, beta, S, per_key=None, o=None, out=None, stream=None):
+    """One decode token per (loop, batch, head); q/k/v [T,B,H,d]; S updated in place."""
+    import torch
+    per_key = (alpha.dim() == 4) if per_key is None else per_key
+    T, B, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = {torch.float32: LT2_DTYPE_F32, torch.bfloat16: LT2_DTYPE_BF16}[q.dtype]
+    dims = make_dims(T, B, H, 1, dk, dv, dt, LT2_GATE_PER_KEY if per_key else LT2_GATE_SCALAR,
+                     out_dtype=_OUT[out])
+    if o is None:
+        o = torch.empty(v.shape, dtype=_out_torch_dtype(q.dtype, out), device=v.device)
+    st = lt2_gdr_decode(dims, q, k, v, alpha, beta, S, o, stream)
+    if st != LT2_OK:
+        raise Lt2Error(st, "lt2_gdr_decode")
+    return o

@@ -1,0 +1,66 @@
+// gdr_common.cuh -- small device/host helpers shared by the looped gated-delta-rule kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lt2 {
+
+// Device-side status word written by bounded waits (see lt2_gdr_last_device_error).
+enum : unsigned int {
+    kDevOk = 0u,
+    kDevTimeout = 1u,
+};
+
+// Per-launch view of one loop's slice: base pointers already offset to loop tau.
+struct LoopSlice {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* alpha;
+    const float* beta;
+    const float* S0;     // nullable: zero initial state
+    void* o;
+    float* S_out;        // nullable (prefill) / in-out state (decode)
+    int64_t units;       // B * H head-units in this loop
+    int64_t L;
+    int dk;
+    int dv;
+    int per_key;
+    int out_bf16;        // o stored as bf16 (else fp32)
+    unsigned int* err;   // device status word
+};
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Programmatic dependent launch: let the next kernel on the stream start now.  Loops are
+// independent recurrences, so a loop's kernel never waits on the previous loop's results.
+__device__ __forceinline__ void allow_next_loop_to_start() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ float4 ld_stream_f4(const float* p) {
+    float4 r;
+    asm volatile("ld.global.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void st_stream_f4(float* p, float4 v) {
+    asm volatile("st.global.cs.v4.f32 [%0], {%1,%2,%3,%4};"
+                 :: "l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
+}
+
+}  // namespace lt2

@@ -1,0 +1,287 @@
+// lt2_gdr_api.cu -- the C ABI declared in include/lt2_gdr.h: argument validation, path
+// selection and the loop orchestration (T launches back to back on one stream).
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "gdr_common.cuh"
+#include "gdr_launch.h"
+#include "lt2_gdr.h"
+
+namespace {
+
+// Status word of bounded in-kernel waits; one instance per device that loads the library.
+__device__ unsigned int g_lt2_device_status = 0u;
+
+thread_local char t_cuda_error[256] = {0};
+
+lt2_status cuda_fail(cudaError_t e, const char* where)
+{
+    std::snprintf(t_cuda_error, sizeof(t_cuda_error), "%s: %s (%d)", where,
+                  cudaGetErrorString(e), (int)e);
+    return LT2_ERR_CUDA;
+}
+
+// Device address of the status word for the current device (cached per device).
+constexpr int kMaxDevices = 64;
+std::atomic<unsigned int*> g_status_ptr[kMaxDevices];
+std::mutex g_status_mu;
+
+lt2_status status_word(unsigned int** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return LT2_ERR_UNSUPPORTED;
+    unsigned int* p = g_status_ptr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        std::lock_guard<std::mutex> lock(g_status_mu);
+        p = g_status_ptr[dev].load(std::memory_order_acquire);
+        if (!p) {
+            e = cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_lt2_device_status);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+            g_status_ptr[dev].store(p, std::memory_order_release);
+        }
+    }
+    *out = p;
+    return LT2_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Byte ranges for the aliasing checks.
+struct Range {
+    uintptr_t lo, hi;
+};
+Range range_of(const void* p, int64_t bytes)
+{
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return {a, a + static_cast<uintptr_t>(bytes)};
+}
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.hi > a.lo && b.hi > b.lo; }
+
+constexpr int64_t kMaxDim = int64_t(1) << 31;
+
+bool out_is_bf16(const lt2_gdr_dims* d)
+{
+    return d->out_dtype == LT2_OUT_BF16 || (d->out_dtype == LT2_OUT_SAME && d->dtype == LT2_DTYPE_BF16);
+}
+
+struct Sizes {
+    int64_t units;        // T*B*H
+    int64_t per_loop;     // B*H
+    int64_t qk, vo, al, be, st;   // element counts over all loops
+    int esz;              // bytes per q/k/v element
+    int osz;              // bytes per o element
+};
+
+lt2_status validate_dims(const lt2_gdr_dims* d, Sizes* sz)
+{
+    if (!d) return LT2_ERR_INVALID_ARGUMENT;
+    if (d->T < 0 || d->B < 0 || d->H < 0 || d->L < 0 || d->dk <= 0 || d->dv <= 0)
+        return LT2_ERR_INVALID_ARGUMENT;
+    if (d->T >= kMaxDim || d->B >= kMaxDim || d->H >= kMaxDim || d->L >= kMaxDim ||
+        d->dk >= kMaxDim || d->dv >= kMaxDim)
+        return LT2_ERR_INVALID_ARGUMENT;
+    if (d->dtype != LT2_DTYPE_F32 && d->dtype != LT2_DTYPE_BF16) return LT2_ERR_INVALID_ARGUMENT;
+    if (d->gate != LT2_GATE_SCALAR && d->gate != LT2_GATE_PER_KEY) return LT2_ERR_INVALID_ARGUMENT;
+    if (d->algo < LT2_ALGO_AUTO || d->algo > LT2_ALGO_CUDA_CORE) return LT2_ERR_INVALID_ARGUMENT;
+    if (d->out_dtype < LT2_OUT_SAME || d->out_dtype > LT2_OUT_BF16) return LT2_ERR_INVALID_ARGUMENT;
+    if (d->dk > 128 || d->dv > 128 || (d->dk % 8) != 0 || (d->dv % 8) != 0)
+        return LT2_ERR_UNSUPPORTED;
+    // Overflow-safe element counts (each factor < 2^31; check the running products).
+    __int128 units = (__int128)d->T * d->B * d->H;
+    __int128 tok = units * d->L;
+    __int128 big = tok * 128;
+    if (big > ((__int128)1 << 62)) return LT2_ERR_INVALID_ARGUMENT;
+    sz->units = (int64_t)units;
+    sz->per_loop = d->B * d->H;
+    sz->qk = (int64_t)(tok * d->dk);
+    sz->vo = (int64_t)(tok * d->dv);
+    sz->al = (int64_t)(d->gate == LT2_GATE_PER_KEY ? tok * d->dk : tok);
+    sz->be = (int64_t)tok;
+    sz->st = (int64_t)(units * d->dk * d->dv);
+    sz->esz = d->dtype == LT2_DTYPE_BF16 ? 2 : 4;
+    sz->osz = out_is_bf16(d) ? 2 : 4;
+    if (sz->units > 0 && sz->per_loop >= kMaxDim) return LT2_ERR_UNSUPPORTED;
+    return LT2_OK;
+}
+
+// Null / alignment checks for a tensor of `count` elements.
+bool tensor_ok(const void* p, int64_t count)
+{
+    if (count == 0) return true;
+    return p != nullptr && aligned16(p);
+}
+
+bool use_tensor_core(const lt2_gdr_dims* d)
+{
+    const bool ok = lt2::prefill_tc_supports(d->dtype == LT2_DTYPE_BF16, (int)d->dk, (int)d->dv,
+                                             d->gate == LT2_GATE_PER_KEY);
+    if (d->algo == LT2_ALGO_CUDA_CORE) return false;
+    return ok;
+}
+
+lt2::LoopSlice loop_slice(const lt2_gdr_dims* d, const Sizes& sz, int64_t tau,
+                          const void* q, const void* k, const void* v, const float* alpha,
+                          const float* beta, const float* S0, void* o, float* S_out,
+                          unsigned int* err)
+{
+    const int64_t U = sz.per_loop, L = d->L, dk = d->dk, dv = d->dv;
+    const int64_t na = d->gate == LT2_GATE_PER_KEY ? dk : 1;
+    lt2::LoopSlice s;
+    s.q = static_cast<const char*>(q) + tau * U * L * dk * sz.esz;
+    s.k = static_cast<const char*>(k) + tau * U * L * dk * sz.esz;
+    s.v = static_cast<const char*>(v) + tau * U * L * dv * sz.esz;
+    s.alpha = alpha + tau * U * L * na;
+    s.beta = beta + tau * U * L;
+    s.S0 = S0 ? S0 + tau * U * dk * dv : nullptr;
+    s.o = static_cast<char*>(o) + tau * U * L * dv * sz.osz;
+    s.S_out = S_out ? S_out + tau * U * dk * dv : nullptr;
+    s.units = U;
+    s.L = L;
+    s.dk = (int)dk;
+    s.dv = (int)dv;
+    s.per_key = d->gate == LT2_GATE_PER_KEY;
+    s.out_bf16 = out_is_bf16(d) ? 1 : 0;
+    s.err = err;
+    return s;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t lt2_gdr_prefill_workspace_bytes(const lt2_gdr_dims* dims)
+{
+    Sizes sz;
+    if (validate_dims(dims, &sz) != LT2_OK) return 0;
+    return 0;
+}
+
+lt2_status lt2_gdr_prefill(const lt2_gdr_dims* dims, const void* q, const void* k, const void* v,
+                           const float* alpha, const float* beta, const float* S0, void* o,
+                           float* S_out, void* workspace, size_t workspace_bytes, void* stream)
+{
+    Sizes sz;
+    lt2_status st = validate_dims(dims, &sz);
+    if (st != LT2_OK) return st;
+    if (dims->algo == LT2_ALGO_TENSOR_CORE &&
+        !lt2::prefill_tc_supports(dims->dtype == LT2_DTYPE_BF16, (int)dims->dk, (int)dims->dv,
+                                  dims->gate == LT2_GATE_PER_KEY))
+        return LT2_ERR_UNSUPPORTED;
+    if (!tensor_ok(q, sz.qk) || !tensor_ok(k, sz.qk) || !tensor_ok(v, sz.vo) ||
+        !tensor_ok(alpha, sz.al) || !tensor_ok(beta, sz.be) || !tensor_ok(o, sz.vo))
+        return LT2_ERR_INVALID_ARGUMENT;
+    if ((S0 && !aligned16(S0)) || (S_out && !aligned16(S_out))) return LT2_ERR_INVALID_ARGUMENT;
+    const size_t need = lt2_gdr_prefill_workspace_bytes(dims);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+        return LT2_ERR_WORKSPACE;
+    // Aliasing: o and S_out are written; neither may overlap an input or each other
+    // (S_out == S0 exactly is the documented in-place resume).
+    const Range ro = range_of(o, sz.vo * sz.osz);
+    const Range rin[5] = {range_of(q, sz.qk * sz.esz), range_of(k, sz.qk * sz.esz),
+                          range_of(v, sz.vo * sz.esz), range_of(alpha, sz.al * 4),
+                          range_of(beta, sz.be * 4)};
+    for (const Range& r : rin)
+        if (overlap(ro, r)) return LT2_ERR_INVALID_ARGUMENT;
+    if (S0 && overlap(ro, range_of(S0, sz.st * 4))) return LT2_ERR_INVALID_ARGUMENT;
+    if (S_out) {
+        const Range rs = range_of(S_out, sz.st * 4);
+        if (overlap(rs, ro)) return LT2_ERR_INVALID_ARGUMENT;
+        for (const Range& r : rin)
+            if (overlap(rs, r)) return LT2_ERR_INVALID_ARGUMENT;
+        if (S0 && S0 != S_out && overlap(rs, range_of(S0, sz.st * 4)))
+            return LT2_ERR_INVALID_ARGUMENT;
+    }
+    if (sz.units == 0) return LT2_OK;
+
+    unsigned int* err = nullptr;
+    st = status_word(&err);
+    if (st != LT2_OK) return st;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool tc = use_tensor_core(dims);
+    for (int64_t tau = 0; tau < dims->T; ++tau) {
+        const lt2::LoopSlice ls = loop_slice(dims, sz, tau, q, k, v, alpha, beta, S0, o, S_out, err);
+        // Loop 0 waits for all earlier work on the stream; later loops may start as soon as
+        // the previous loop's grid is running (the loops share no data).
+        const bool pdl = tau > 0;
+        cudaError_t e = tc ? lt2::launch_prefill_tc(ls, s, pdl)
+                           : lt2::launch_prefill_seq(ls, dims->dtype == LT2_DTYPE_BF16, s, pdl);
+        if (e == cudaSuccess) e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, tc ? "prefill (tensor core)" : "prefill (cuda core)");
+    }
+    return LT2_OK;
+}
+
+lt2_status lt2_gdr_decode(const lt2_gdr_dims* dims, const void* q, const void* k, const void* v,
+                          const float* alpha, const float* beta, float* S, void* o, void* stream)
+{
+    Sizes sz;
+    lt2_status st = validate_dims(dims, &sz);
+    if (st != LT2_OK) return st;
+    if (dims->L != 1) return LT2_ERR_INVALID_ARGUMENT;
+    if (!tensor_ok(q, sz.qk) || !tensor_ok(k, sz.qk) || !tensor_ok(v, sz.vo) ||
+        !tensor_ok(alpha, sz.al) || !tensor_ok(beta, sz.be) || !tensor_ok(o, sz.vo) ||
+        !tensor_ok(S, sz.st))
+        return LT2_ERR_INVALID_ARGUMENT;
+    const Range ro = range_of(o, sz.vo * sz.osz), rs = range_of(S, sz.st * 4);
+    const Range rin[5] = {range_of(q, sz.qk * sz.esz), range_of(k, sz.qk * sz.esz),
+                          range_of(v, sz.vo * sz.esz), range_of(alpha, sz.al * 4),
+                          range_of(beta, sz.be * 4)};
+    if (overlap(ro, rs)) return LT2_ERR_INVALID_ARGUMENT;
+    for (const Range& r : rin)
+        if (overlap(ro, r) || overlap(rs, r)) return LT2_ERR_INVALID_ARGUMENT;
+    if (sz.units == 0) return LT2_OK;
+
+    unsigned int* err = nullptr;
+    st = status_word(&err);
+    if (st != LT2_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    for (int64_t tau = 0; tau < dims->T; ++tau) {
+        lt2::LoopSlice ls = loop_slice(dims, sz, tau, q, k, v, alpha, beta, nullptr, o, S, err);
+        cudaError_t e = lt2::launch_decode(ls, dims->dtype == LT2_DTYPE_BF16, s, tau > 0);
+        if (e == cudaSuccess) e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "decode");
+    }
+    return LT2_OK;
+}
+
+lt2_status lt2_gdr_last_device_error(void)
+{
+    unsigned int* p = nullptr;
+    lt2_status st = status_word(&p);
+    if (st != LT2_OK) return st;
+    unsigned int h = 0;
+    cudaError_t e = cudaMemcpy(&h, p, sizeof(h), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "read device status");
+    if (h == lt2::kDevOk) return LT2_OK;
+    const unsigned int zero = 0;
+    e = cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "clear device status");
+    return LT2_ERR_DEVICE_TIMEOUT;
+}
+
+const char* lt2_status_string(lt2_status s)
+{
+    switch (s) {
+        case LT2_OK: return "LT2_OK";
+        case LT2_ERR_INVALID_ARGUMENT: return "LT2_ERR_INVALID_ARGUMENT";
+        case LT2_ERR_UNSUPPORTED: return "LT2_ERR_UNSUPPORTED";
+        case LT2_ERR_WORKSPACE: return "LT2_ERR_WORKSPACE";
+        case LT2_ERR_CUDA: return "LT2_ERR_CUDA";
+        case LT2_ERR_DEVICE_TIMEOUT: return "LT2_ERR_DEVICE_TIMEOUT";
+    }
+    return "LT2_STATUS_UNKNOWN";
+}
+
+const char* lt2_last_cuda_error_string(void) { return t_cuda_error; }
+
+int lt2_gdr_version(void) { return 100; }
+
+}  // extern "C"

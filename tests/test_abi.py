@@ -1,0 +1,162 @@
+"""The C-ABI library on the CPU: it loads, exports every symbol include/lt2_gdr.h declares,
+and rejects bad arguments synchronously with the documented status, before touching the GPU
+(every call below fails validation, so nothing is launched; pointers are fake addresses).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_looped_b200 as lt2
+from gated_delta_rule_looped_b200 import build as lbuild
+
+HEADER_DIR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+
+
+@pytest.fixture(scope="module")
+def L():
+    if lbuild.needs_build():
+        lbuild.build()
+    return lt2.lib()
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(HEADER_DIR):
+        if fn.endswith(".h"):
+            with open(os.path.join(HEADER_DIR, fn)) as f:
+                text = f.read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(lt2_\w+)\s*\(", text))
+    return names
+
+
+def test_exports_every_declared_symbol(L):
+    declared = _declared_functions()
+    assert declared, "no declarations found"
+    assert declared == set(lt2.EXPORTS)
+    for name in declared:
+        assert hasattr(L, name), f"{name} not exported"
+
+
+def test_status_strings(L):
+    for code, name in [(0, "LT2_OK"), (1, "LT2_ERR_INVALID_ARGUMENT"), (2, "LT2_ERR_UNSUPPORTED"),
+                       (3, "LT2_ERR_WORKSPACE"), (4, "LT2_ERR_CUDA"),
+                       (5, "LT2_ERR_DEVICE_TIMEOUT")]:
+        assert lt2.lt2_status_string(code) == name
+    assert lt2.lt2_status_string(99) == "LT2_STATUS_UNKNOWN"
+    assert L.lt2_gdr_version() >= 100
+
+
+def test_dims_struct_layout():
+    assert ctypes.sizeof(lt2.lt2_gdr_dims) == 6 * 8 + 4 * 4
+
+
+# Fake, 16-byte aligned, non-overlapping "device" addresses (never dereferenced).
+BASE = 1 << 40
+SPAN = 1 << 34
+
+
+def addrs(n):
+    return [BASE + i * SPAN for i in range(n)]
+
+
+def call_prefill(dims, **over):
+    q, k, v, a, b, s0, o, so = addrs(8)
+    args = dict(q=q, k=k, v=v, alpha=a, beta=b, S0=s0, o=o, S_out=so)
+    args.update(over)
+    return lt2.lt2_gdr_prefill(dims, args["q"], args["k"], args["v"], args["alpha"], args["beta"],
+                               args["S0"], args["o"], args["S_out"], None, 0, 0)
+
+
+def call_decode(dims, **over):
+    q, k, v, a, b, S, o = addrs(7)
+    args = dict(q=q, k=k, v=v, alpha=a, beta=b, S=S, o=o)
+    args.update(over)
+    return lt2.lt2_gdr_decode(dims, args["q"], args["k"], args["v"], args["alpha"], args["beta"],
+                              args["S"], args["o"], 0)
+
+
+def D(**kw):
+    base = dict(T=2, B=1, H=2, L=64, dk=32, dv=32, dtype=lt2.LT2_DTYPE_F32,
+                gate=lt2.LT2_GATE_SCALAR, algo=lt2.LT2_ALGO_AUTO)
+    base.update(kw)
+    return lt2.make_dims(**base)
+
+
+def test_null_dims_rejected(L):
+    st = L.lt2_gdr_prefill(None, 1, 1, 1, 1, 1, None, 1, None, None, 0, None)
+    assert st == lt2.LT2_ERR_INVALID_ARGUMENT
+    assert L.lt2_gdr_prefill_workspace_bytes(None) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=256, dv=256), lt2.LT2_ERR_UNSUPPORTED),
+    (dict(dk=12), lt2.LT2_ERR_UNSUPPORTED),
+    (dict(dv=130), lt2.LT2_ERR_UNSUPPORTED),
+    (dict(dk=0), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(L=-1), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(T=-2), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(dtype=7), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(gate=3), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(algo=9), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(algo=lt2.LT2_ALGO_TENSOR_CORE), lt2.LT2_ERR_UNSUPPORTED),   # fp32, d=32
+    (dict(T=1 << 30, B=1 << 30, H=1 << 30), lt2.LT2_ERR_INVALID_ARGUMENT),
+])
+def test_bad_dims(L, kw, status):
+    assert call_prefill(D(**kw)) == status
+
+
+def test_bad_out_dtype(L):
+    d = D()
+    d.out_dtype = 3
+    assert call_prefill(d) == lt2.LT2_ERR_INVALID_ARGUMENT
+    d.out_dtype = -1
+    assert call_prefill(d) == lt2.LT2_ERR_INVALID_ARGUMENT
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "alpha", "beta", "o"])
+def test_null_pointer_rejected(L, field):
+    assert call_prefill(D(), **{field: None}) == lt2.LT2_ERR_INVALID_ARGUMENT
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "alpha", "beta", "o", "S0", "S_out"])
+def test_misaligned_pointer_rejected(L, field):
+    assert call_prefill(D(), **{field: BASE + 20 * SPAN + 8}) == lt2.LT2_ERR_INVALID_ARGUMENT
+
+
+def test_aliasing_rejected(L):
+    q = addrs(1)[0]
+    assert call_prefill(D(), o=q + 64) == lt2.LT2_ERR_INVALID_ARGUMENT        # o inside q
+    s0 = addrs(6)[5]
+    assert call_prefill(D(), S_out=s0 + 256) == lt2.LT2_ERR_INVALID_ARGUMENT  # partial overlap
+    o = addrs(7)[6]
+    assert call_prefill(D(), S_out=o) == lt2.LT2_ERR_INVALID_ARGUMENT
+
+
+def test_empty_problem_is_a_noop(L):
+    # No head-units: valid, nothing to launch, no GPU needed.
+    assert call_prefill(D(T=0)) == lt2.LT2_OK
+    assert call_prefill(D(B=0), q=None, k=None, v=None, alpha=None, beta=None, o=None) == lt2.LT2_OK
+
+
+def test_workspace_query(L):
+    assert lt2.lt2_gdr_prefill_workspace_bytes(D()) == 0
+    assert lt2.lt2_gdr_prefill_workspace_bytes(D(dk=7)) == 0
+
+
+def test_decode_validation(L):
+    assert call_decode(D(L=64)) == lt2.LT2_ERR_INVALID_ARGUMENT
+    assert call_decode(D(L=1), S=None) == lt2.LT2_ERR_INVALID_ARGUMENT
+    S = addrs(7)[5]
+    assert call_decode(D(L=1), o=S) == lt2.LT2_ERR_INVALID_ARGUMENT
+    assert call_decode(D(L=1, dk=136)) == lt2.LT2_ERR_UNSUPPORTED
+    assert call_decode(D(L=1, B=0)) == lt2.LT2_OK
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(lt2, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(lt2, "_LIB", None)
+    with pytest.raises(ImportError):
+        lt2.lib()
