@@ -44,8 +44,10 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
-// Programmatic dependent launch: let the next kernel on the stream start now.  Loops are
-// independent recurrences, so a loop's kernel never waits on the previous loop's results.
+// Programmatic dependent launch: let the next kernel on the stream start now.  Only the
+// library's own launches of later loops carry the attribute that honours this trigger, and
+// loops are independent recurrences, so none of them waits on the previous loop's results;
+// any other kernel launched after these still waits for their completion.
 __device__ __forceinline__ void allow_next_loop_to_start() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }

@@ -24,7 +24,8 @@ namespace lt2 {
 template <typename T, typename To>
 __global__ void __launch_bounds__(256, 2) gdr_decode_kernel(LoopSlice p, int use_pdl)
 {
-    if (use_pdl) allow_next_loop_to_start();
+    (void)use_pdl;
+    allow_next_loop_to_start();
 
     __shared__ __align__(16) float sk[128];
     __shared__ __align__(16) float saq[128];

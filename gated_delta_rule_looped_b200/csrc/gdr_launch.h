@@ -13,8 +13,24 @@ cudaError_t launch_decode(const LoopSlice& s, int dtype_bf16, cudaStream_t strea
 // Token-sequential CUDA-core prefill of one loop (fp32 arithmetic, any supported shape).
 cudaError_t launch_prefill_seq(const LoopSlice& s, int dtype_bf16, cudaStream_t stream, bool pdl);
 
-// Tensor-core chunked prefill of one loop (bf16 inputs, dk = dv = 128).
+// Tensor-core chunked prefill (bf16 inputs, dk = dv = 128), all T loops: one launch per loop,
+// back to back on `stream`, loops after the first allowed to start early (they share no data).
+struct TcCall {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* alpha;
+    const float* beta;
+    const float* S0;       // nullable
+    void* o;
+    float* S_out;          // nullable
+    int64_t T;
+    int64_t units_per_loop;  // B * H
+    int64_t L;               // >= 1
+    int out_bf16;
+    unsigned int* err;
+};
 bool prefill_tc_supports(int dtype_bf16, int dk, int dv, int per_key);
-cudaError_t launch_prefill_tc(const LoopSlice& s, cudaStream_t stream, bool pdl);
+cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream);
 
 }  // namespace lt2

@@ -27,7 +27,8 @@ constexpr int kCols = 32;    // d_v columns per CTA
 template <typename T, typename To>
 __global__ void __launch_bounds__(256) gdr_prefill_seq_kernel(LoopSlice p, int use_pdl)
 {
-    if (use_pdl) allow_next_loop_to_start();
+    (void)use_pdl;
+    allow_next_loop_to_start();
 
     extern __shared__ __align__(16) float smem[];
     const int dk = p.dk, dv = p.dv;

@@ -1,12 +1,857 @@
-// gdr_prefill_tc.cu -- tensor-core (tcgen05 + TMA) chunked prefill.  Placeholder until the
-// kernel lands: reports no supported shape, so every call takes the CUDA-core path.
+// gdr_prefill_tc.cu -- chunked prefill of the gated delta rule on Blackwell tensor cores
+// (tcgen05 MMA with TMEM accumulators, operands staged by TMA), scalar gating, d_k = d_v = 128.
+//
+// The recurrence ("LT2 transformer looped a tempo lineare", section "Sostituire il motore",
+// displayed equation)  S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T  with
+// the readout o_t = S_t^T q_t is evaluated 64 tokens ("a chunk") at a time.  With the chunk's
+// incoming state S, G_r = sum_{s<=r} log alpha_s, g_r = exp(G_r):
+//
+//   A_rs = beta_s e^{G_r-G_s} k_r.k_s  (s < r),   P_rs = beta_s e^{G_r-G_s} q_r.k_s  (s <= r)
+//   T    = (I + A)^{-1}                              (unit lower triangular, 64 x 64)
+//   X    = V - diag(g) K S                           (64 x d_v)
+//   U    = T X,     o = diag(g) Q S + (P T) X
+//   S'   = g_63 S + K^T diag(beta_s e^{G_63-G_s}) U
+//
+// (u_r = v_r - alpha_r S_{r-1}^T k_r unrolls the chunk; the identity is checked in fp64 by
+// the test suite's chunked oracle.)  Everything that does not involve S -- the Gram
+// products K K^T and Q K^T, the solve, P T -- is done one chunk ahead, overlapped with the
+// S-dependent chain of the current chunk:
+//
+//   MMA_A  [K; Q] S           (M=128, N=64, K=128)     -> TMEM  (K S | Q S)
+//   MMA_B  [T; PT] X          (M=128, N=64, K=64)      -> TMEM  (U   | P T X)
+//   MMA_C  S += K^T U~        (M=128, N=64, K=64)      -> TMEM  (the fp32 state)
+//
+// for each half of d_v (two independent 64-column chains, so one half's CUDA-core epilogue
+// overlaps the other half's MMAs).  The state lives in TMEM in fp32 for the whole sequence;
+// its fp16 copy in shared memory is the B operand of MMA_A.
+//
+// Precision.  All MMA operands are fp16 (10-bit mantissa), not bf16: with bf16
+// intermediates (S, X, [T;PT], U~ rounded to 8 significant bits) the error against the
+// fp64 oracle reaches ~3% of rms(o) at the largest outputs, while fp16 keeps it near 0.5%.
+// q, k arrive in bf16; converting a bf16 tile to fp16 in shared memory is exact for the
+// magnitudes involved (|x| in [2^-14, 2^15]), so the inputs are not rounded again.
+//
+// CTA = one (loop, batch, head) unit, 16 warps:
+//   warp 0       TMA producer (and TMEM allocation)
+//   warp 1       tcgen05.mma issuer (one thread)
+//   warps 2-3    chunk gates (log-decay prefix sums) and bf16 -> fp16 conversion of K, Q
+//   warps 4-7    "prep": Gram epilogue, the 64x64 triangular solve (16x16 blocks with
+//                warp-level mma.sync), P T; writes [T; PT] for MMA_B
+//   warps 8-11   chain of d_v columns 0..63;  warps 12-15  chain of columns 64..127
+// Every wait is bounded (see mbar_wait); on a timeout the CTA records it in the device
+// status word, drains its in-flight copies and MMAs, frees TMEM and exits.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
 #include "gdr_common.cuh"
 #include "gdr_launch.h"
+#include "sm100_primitives.cuh"
 
 namespace lt2 {
+namespace tc {
 
-bool prefill_tc_supports(int, int, int, int) { return false; }
+using namespace sm100;
 
-cudaError_t launch_prefill_tc(const LoopSlice&, cudaStream_t, bool) { return cudaErrorNotSupported; }
+constexpr int kC = 64;                 // tokens per chunk
+constexpr int kD = 128;                // d_k = d_v
+constexpr int kThreads = 512;
+constexpr uint64_t kTimeoutNs = 4000000000ull;   // 4 s
+
+// Shared memory map (offsets from a 1024-byte aligned base).
+constexpr uint32_t KQ_STAGE = 32768;   // K|Q, two 64-column panels: [K rows 0-63 | Q rows 0-63]
+constexpr uint32_t V_STAGE = 16384;    // V, two 64-column panels (bf16, read by CUDA cores)
+constexpr uint32_t TP_STAGE = 16384;   // [T; PT], 128 rows x 64 fp16
+constexpr uint32_t OFF_KQ = 0;
+constexpr uint32_t OFF_V = OFF_KQ + 2 * KQ_STAGE;
+constexpr uint32_t OFF_TP = OFF_V + 2 * V_STAGE;
+constexpr uint32_t OFF_SOP = OFF_TP + 2 * TP_STAGE;   // per half: S (fp16) [128 rows][64]
+constexpr uint32_t OFF_XOP = OFF_SOP + 2 * 16384;     // per half: X (fp16) [64 tokens][64]
+constexpr uint32_t OFF_UOP = OFF_XOP + 2 * 8192;      // per half: U~ (fp16) [64 tokens][64]
+constexpr uint32_t OFF_AS = OFF_UOP + 2 * 8192;       // A (fp16) [64][64]
+constexpr uint32_t OFF_PS = OFF_AS + 8192;            // P (fp16) [64][64]
+constexpr uint32_t OFF_ADIAG = OFF_PS + 8192;         // diagonal 16x16 blocks of A, fp32
+constexpr uint32_t OFF_GATES = OFF_ADIAG + 4096;
+constexpr uint32_t GATE_STAGE = 1536;
+constexpr uint32_t OFF_BAR = OFF_GATES + 2 * GATE_STAGE;
+constexpr uint32_t BAR_BYTES = 512;
+constexpr uint32_t SMEM_USED = OFF_BAR + BAR_BYTES;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;     // slack for aligning the base
+
+struct Gates {
+    float G[kC];       // chunk-local cumulative log-decay
+    float gam[kC];     // e^{G_r}
+    float einv[kC];    // e^{-G_s} (valid when `safe`)
+    float beta[kC];    // beta_s (0 beyond the sequence end)
+    float bgc[kC];     // beta_s e^{G_63 - G_s}
+    float gC;          // e^{G_63}
+    int safe;          // e^{-G} representable: A/P use the factored decay
+};
+static_assert(sizeof(Gates) <= GATE_STAGE, "gate stage too small");
+
+// Barrier slots (8 bytes each) inside the OFF_BAR area.
+enum Bar : uint32_t {
+    B_KQ_FULL = 0,     // [2] TMA landed (tx count)
+    B_KQ_CONV = 2,     // [2] K, Q converted to fp16
+    B_KQ_EMPTY = 4,    // [2] MMAs done with the K|Q stage
+    B_V_EMPTY = 6,     // [2] chains done with the V stage
+    B_GATE_FULL = 8,   // [2]
+    B_GATE_EMPTY = 10, // [2]
+    B_TP_FULL = 12,    // [2]
+    B_TP_EMPTY = 14,   // [2]
+    B_G_FULL = 16,     // Gram in TMEM
+    B_G_EMPTY = 17,    // Gram read out
+    B_A_FULL = 18,     // [2] per half
+    B_B_FULL = 20,     // [2]
+    B_X_FULL = 22,     // [2]
+    B_U_FULL = 24,     // [2]
+    B_S_FULL = 26,     // [2]
+    B_SOP_FULL = 28,   // [2]
+    B_PREP_SYNC = 30,  // prep-group barrier (reused phase by phase)
+    B_DRAIN = 31,      // MMA drain on abort
+    B_COUNT = 32
+};
+constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + B_COUNT * 8;        // tcgen05.alloc result
+constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 16;
+
+// TMEM columns (fp32 accumulators, 128 lanes each).
+constexpr uint32_t TM_G = 0;                     // Gram [K;Q] K^T, 64 columns
+constexpr uint32_t TM_A = 64;                    // + 64*h : [K;Q] S per half
+constexpr uint32_t TM_B = 192;                   // + 64*h : [T;PT] X per half
+constexpr uint32_t TM_S = 320;                   // + 64*h : state per half
+constexpr uint32_t TM_COLS = 512;
+
+constexpr uint32_t ID_KK = idesc_f16_f32(128, 64, 0, 0);  // A K-major, B K-major
+constexpr uint32_t ID_KM = idesc_f16_f32(128, 64, 0, 1);  // A K-major, B MN-major
+constexpr uint32_t ID_MM = idesc_f16_f32(128, 64, 1, 1);  // A MN-major, B MN-major
+
+struct Params {
+    const float* alpha;    // [units_total][L]
+    const float* beta;
+    const float* S0;       // [units_total][128][128] or null
+    void* o;               // [units_total][L][128]
+    float* S_out;          // nullable
+    int64_t L;
+    int unit0;             // first unit of this loop in the flattened [T*B*H] order
+    int out_bf16;
+    unsigned int* err;
+};
+
+__device__ __forceinline__ uint32_t bar_addr(uint32_t base, uint32_t i) { return base + OFF_BAR + 8u * i; }
+
+// Prep-group (warps 4-7) barrier on a shared mbarrier; bounded like every other wait.
+struct GroupSync {
+    uint32_t bar;
+    uint32_t phase;
+    __device__ bool sync(volatile int* abort_flag, unsigned int* err)
+    {
+        mbar_arrive(bar);
+        const bool ok = mbar_wait(bar, phase & 1u, abort_flag, err, kTimeoutNs);
+        ++phase;
+        return ok;
+    }
+};
+
+// --- prep helpers: 16x16 fp16 blocks of row-major 128B-swizzled tiles --------------------
+__device__ __forceinline__ void frag_a(uint32_t tile, int row0, int col0, int lane, uint32_t (&a)[4])
+{
+    const uint32_t row = row0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+    const uint32_t chunk = (col0 >> 3) + (lane >> 4);
+    ldsm_x4(sw128(tile, row, chunk), a);
+}
+__device__ __forceinline__ void frag_b(uint32_t tile, int k0, int n0, int lane, uint32_t (&b)[4])
+{
+    const uint32_t row = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+    const uint32_t chunk = (n0 >> 3) + (lane >> 4);
+    ldsm_x4_trans(sw128(tile, row, chunk), b);
+}
+__device__ __forceinline__ void mma_block(float (&c)[2][4], const uint32_t (&a)[4], const uint32_t (&b)[4])
+{
+    mma16816(c[0], a, b[0], b[1]);
+    mma16816(c[1], a, b[2], b[3]);
+}
+__device__ __forceinline__ void c_to_a(const float (&c)[2][4], uint32_t (&a)[4])
+{
+    a[0] = pack_half2(c[0][0], c[0][1]);
+    a[1] = pack_half2(c[0][2], c[0][3]);
+    a[2] = pack_half2(c[1][0], c[1][1]);
+    a[3] = pack_half2(c[1][2], c[1][3]);
+}
+__device__ __forceinline__ void store_block(uint32_t tile, int row0, int col0, int lane,
+                                            const float (&c)[2][4], float sign)
+{
+    const uint32_t g = lane >> 2, tq = lane & 3;
+    #pragma unroll
+    for (int nb = 0; nb < 2; ++nb) {
+        const uint32_t chunk = (col0 >> 3) + nb;
+        sts32(sw128(tile, row0 + g, chunk) + tq * 4, pack_half2(sign * c[nb][0], sign * c[nb][1]));
+        sts32(sw128(tile, row0 + g + 8, chunk) + tq * 4, pack_half2(sign * c[nb][2], sign * c[nb][3]));
+    }
+}
+__device__ __forceinline__ void zero_c(float (&c)[2][4])
+{
+    #pragma unroll
+    for (int i = 0; i < 2; ++i)
+        #pragma unroll
+        for (int j = 0; j < 4; ++j) c[i][j] = 0.f;
+}
+
+// T_ij = -sum_{k=j}^{i-1} (D_i^{-1} A_ik) T_kj, with D_i^{-1} = T_ii already in TP.
+__device__ void t_block(uint32_t tp, uint32_t as, int i, int j, int lane)
+{
+    float acc[2][4];
+    zero_c(acc);
+    uint32_t dinv[4];
+    frag_a(tp, 16 * i, 16 * i, lane, dinv);
+    for (int k = j; k < i; ++k) {
+        uint32_t b[4];
+        frag_b(as, 16 * i, 16 * k, lane, b);
+        float n[2][4];
+        zero_c(n);
+        mma_block(n, dinv, b);           // N_ik = D_i^{-1} A_ik
+        uint32_t na[4];
+        c_to_a(n, na);
+        frag_b(tp, 16 * k, 16 * j, lane, b);
+        mma_block(acc, na, b);           // += N_ik T_kj
+    }
+    store_block(tp, 16 * i, 16 * j, lane, acc, -1.f);
+}
+
+// PT_qj = sum_{k=j}^{q} P_qk T_kj for j = 0..q, stored in rows 64.. of TP.
+__device__ void pt_row(uint32_t tp, uint32_t ps, int q, int lane)
+{
+    for (int j = 0; j <= q; ++j) {
+        float acc[2][4];
+        zero_c(acc);
+        for (int k = j; k <= q; ++k) {
+            uint32_t a[4], b[4];
+            frag_a(ps, 16 * q, 16 * k, lane, a);
+            frag_b(tp, 16 * k, 16 * j, lane, b);
+            mma_block(acc, a, b);
+        }
+        store_block(tp, 64 + 16 * q, 16 * j, lane, acc, 1.f);
+    }
+}
+
+__device__ __forceinline__ void st_global_v4(void* p, uint4 v)
+{
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};"
+                 ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, Params p, int use_pdl)
+{
+    (void)use_pdl;
+    allow_next_loop_to_start();
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t sb = (raw + 1023u) & ~1023u;        // 1024-aligned base (swizzle atoms)
+    uint8_t* sbase = smem_raw + (sb - raw);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + OFF_ABORT);
+    Gates* gates = reinterpret_cast<Gates*>(sbase + OFF_GATES);   // [2], GATE_STAGE apart
+    auto gate = [&](int s) -> Gates* {
+        return reinterpret_cast<Gates*>(sbase + OFF_GATES + s * GATE_STAGE);
+    };
+    (void)gates;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t L = p.L;
+    const int nchunks = static_cast<int>((L + kC - 1) / kC);
+    const int ug = p.unit0 + blockIdx.x;               // global head-unit index
+    unsigned int* err = p.err;
+
+    // ---- set-up: barriers, TMEM ----
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar_addr(sb, B_KQ_FULL + s), 1);
+            mbar_init(bar_addr(sb, B_KQ_CONV + s), 64);
+            mbar_init(bar_addr(sb, B_KQ_EMPTY + s), 1);
+            mbar_init(bar_addr(sb, B_V_EMPTY + s), 256);
+            mbar_init(bar_addr(sb, B_GATE_FULL + s), 1);
+            mbar_init(bar_addr(sb, B_GATE_EMPTY + s), 384);
+            mbar_init(bar_addr(sb, B_TP_FULL + s), 128);
+            mbar_init(bar_addr(sb, B_TP_EMPTY + s), 1);
+            mbar_init(bar_addr(sb, B_A_FULL + s), 1);
+            mbar_init(bar_addr(sb, B_B_FULL + s), 1);
+            mbar_init(bar_addr(sb, B_X_FULL + s), 128);
+            mbar_init(bar_addr(sb, B_U_FULL + s), 128);
+            mbar_init(bar_addr(sb, B_S_FULL + s), 1);
+            mbar_init(bar_addr(sb, B_SOP_FULL + s), 128);
+        }
+        mbar_init(bar_addr(sb, B_G_FULL), 1);
+        mbar_init(bar_addr(sb, B_G_EMPTY), 128);
+        mbar_init(bar_addr(sb, B_PREP_SYNC), 128);
+        mbar_init(bar_addr(sb, B_DRAIN), 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(sb + OFF_TMEM_SLOT, TM_COLS);
+        tmem_relinquish();
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+        }
+    }
+    if (warp >= 4 && warp < 8) {
+        // zero both [T; PT] stages once: the blocks above the diagonal are never written
+        const int t = threadIdx.x - 128;
+        for (uint32_t off = t * 16; off < 2 * TP_STAGE; off += 128 * 16)
+            sts128(sb + OFF_TP + off, make_uint4(0, 0, 0, 0));
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + OFF_TMEM_SLOT);
+
+    if (warp == 0) {
+        // ================= TMA producer =================
+        if (lane == 0) {
+            int issued = 0;
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c & 1;
+                const uint32_t ph = ((c >> 1) & 1) ^ 1;
+                if (!mbar_wait(bar_addr(sb, B_KQ_EMPTY + s), ph, abort_flag, err, kTimeoutNs)) break;
+                if (!mbar_wait(bar_addr(sb, B_V_EMPTY + s), ph, abort_flag, err, kTimeoutNs)) break;
+                const uint32_t fb = bar_addr(sb, B_KQ_FULL + s);
+                mbar_arrive_expect_tx(fb, KQ_STAGE + V_STAGE);
+                const uint32_t kq = sb + OFF_KQ + s * KQ_STAGE, vv = sb + OFF_V + s * V_STAGE;
+                const int32_t y = c * kC;
+                tma_load_3d(kq, &tm_k, 0, y, ug, fb);
+                tma_load_3d(kq + 16384, &tm_k, 64, y, ug, fb);
+                tma_load_3d(kq + 8192, &tm_q, 0, y, ug, fb);
+                tma_load_3d(kq + 24576, &tm_q, 64, y, ug, fb);
+                tma_load_3d(vv, &tm_v, 0, y, ug, fb);
+                tma_load_3d(vv + 8192, &tm_v, 64, y, ug, fb);
+                issued = c + 1;
+            }
+            if (*abort_flag) {
+                // let the copies already in flight land before the CTA's memory goes away
+                for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c)
+                    mbar_wait(bar_addr(sb, B_KQ_FULL + (c & 1)), (c >> 1) & 1, abort_flag, err, kTimeoutNs / 4);
+            }
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer =================
+        if (lane == 0) {
+            bool ok = true;
+            if (nchunks > 0) {
+                ok = mbar_wait(bar_addr(sb, B_KQ_CONV + 0), 0, abort_flag, err, kTimeoutNs);
+                if (ok) {
+                    tc_fence_after();
+                    const uint32_t kq = sb + OFF_KQ;
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+                        umma_f16(tmem + TM_G, smem_desc_sw128(kq + off, 16, 1024),
+                                 smem_desc_sw128(kq + off, 16, 1024), ID_KK, k > 0);
+                    }
+                    umma_commit(bar_addr(sb, B_G_FULL));
+                }
+            }
+            for (int c = 0; ok && c < nchunks; ++c) {
+                const int s = c & 1;
+                const uint32_t kq = sb + OFF_KQ + s * KQ_STAGE;
+                for (int h = 0; h < 2 && ok; ++h) {
+                    ok = mbar_wait(bar_addr(sb, B_SOP_FULL + h), c & 1, abort_flag, err, kTimeoutNs);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t sop = sb + OFF_SOP + h * 16384;
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t aoff = (k >> 2) * 16384 + (k & 3) * 32;
+                        umma_f16(tmem + TM_A + 64 * h, smem_desc_sw128(kq + aoff, 16, 1024),
+                                 smem_desc_sw128(sop + k * 2048, 8192, 1024), ID_KM, k > 0);
+                    }
+                    umma_commit(bar_addr(sb, B_A_FULL + h));
+                }
+                if (!ok) break;
+                if (c + 1 < nchunks) {
+                    const int s1 = (c + 1) & 1;
+                    ok = mbar_wait(bar_addr(sb, B_KQ_CONV + s1), ((c + 1) >> 1) & 1, abort_flag, err, kTimeoutNs) &&
+                         mbar_wait(bar_addr(sb, B_G_EMPTY), c & 1, abort_flag, err, kTimeoutNs);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t kq1 = sb + OFF_KQ + s1 * KQ_STAGE;
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+                        umma_f16(tmem + TM_G, smem_desc_sw128(kq1 + off, 16, 1024),
+                                 smem_desc_sw128(kq1 + off, 16, 1024), ID_KK, k > 0);
+                    }
+                    umma_commit(bar_addr(sb, B_G_FULL));
+                }
+                ok = mbar_wait(bar_addr(sb, B_TP_FULL + s), (c >> 1) & 1, abort_flag, err, kTimeoutNs);
+                if (!ok) break;
+                const uint32_t tp = sb + OFF_TP + s * TP_STAGE;
+                for (int h = 0; h < 2 && ok; ++h) {
+                    ok = mbar_wait(bar_addr(sb, B_X_FULL + h), c & 1, abort_flag, err, kTimeoutNs);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t xop = sb + OFF_XOP + h * 8192;
+                    for (int k = 0; k < 4; ++k)
+                        umma_f16(tmem + TM_B + 64 * h, smem_desc_sw128(tp + k * 32, 16, 1024),
+                                 smem_desc_sw128(xop + k * 2048, 8192, 1024), ID_KM, k > 0);
+                    umma_commit(bar_addr(sb, B_B_FULL + h));
+                }
+                if (!ok) break;
+                umma_commit(bar_addr(sb, B_TP_EMPTY + s));
+                for (int h = 0; h < 2 && ok; ++h) {
+                    ok = mbar_wait(bar_addr(sb, B_U_FULL + h), c & 1, abort_flag, err, kTimeoutNs);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t uop = sb + OFF_UOP + h * 8192;
+                    for (int k = 0; k < 4; ++k)
+                        umma_f16(tmem + TM_S + 64 * h, smem_desc_sw128(kq + k * 2048, 16384, 1024),
+                                 smem_desc_sw128(uop + k * 2048, 8192, 1024), ID_MM, 1);
+                    umma_commit(bar_addr(sb, B_S_FULL + h));
+                }
+                if (!ok) break;
+                umma_commit(bar_addr(sb, B_KQ_EMPTY + s));
+            }
+            if (!ok) {
+                // wait for every MMA issued so far before TMEM is released
+                umma_commit(bar_addr(sb, B_DRAIN));
+                mbar_wait(bar_addr(sb, B_DRAIN), 0, abort_flag, err, kTimeoutNs / 4);
+            }
+        }
+    } else if (warp == 2 || warp == 3) {
+        // ================= gates (warp 2) and fp16 conversion of K (warp 2) / Q (warp 3) ====
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c & 1;
+            const uint32_t ph = (c >> 1) & 1;
+            if (warp == 2) {
+                if (!mbar_wait(bar_addr(sb, B_GATE_EMPTY + s), ph ^ 1, abort_flag, err, kTimeoutNs)) break;
+                Gates* gs = gate(s);
+                const int64_t t0 = static_cast<int64_t>(c) * kC;
+                float g[2], b[2];
+                #pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int64_t tok = t0 + lane + 32 * i;
+                    const bool valid = tok < L;
+                    const float a = valid ? p.alpha[ug * L + tok] : 1.f;
+                    b[i] = valid ? p.beta[ug * L + tok] : 0.f;
+                    g[i] = __logf(fmaxf(a, 1e-30f));
+                }
+                // inclusive prefix sums over the 64 tokens
+                #pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    #pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float y = __shfl_up_sync(0xffffffffu, g[i], off);
+                        if (lane >= off) g[i] += y;
+                    }
+                }
+                g[1] += __shfl_sync(0xffffffffu, g[0], 31);
+                const float GC = __shfl_sync(0xffffffffu, g[1], 31);
+                const bool safe = GC > -80.f;
+                #pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int r = lane + 32 * i;
+                    gs->G[r] = g[i];
+                    gs->gam[r] = __expf(g[i]);
+                    gs->einv[r] = safe ? __expf(-g[i]) : 0.f;
+                    gs->beta[r] = b[i];
+                    gs->bgc[r] = b[i] * __expf(GC - g[i]);
+                }
+                if (lane == 0) {
+                    gs->gC = __expf(GC);
+                    gs->safe = safe ? 1 : 0;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_addr(sb, B_GATE_FULL + s));
+            }
+            if (!mbar_wait(bar_addr(sb, B_KQ_FULL + s), ph, abort_flag, err, kTimeoutNs)) break;
+            const uint32_t base = sb + OFF_KQ + s * KQ_STAGE + (warp == 3 ? 8192u : 0u);
+            #pragma unroll 4
+            for (int i = 0; i < 32; ++i) {
+                const int v = i * 32 + lane;
+                const uint32_t a = base + (v < 512 ? v * 16 : 16384 + (v - 512) * 16);
+                const uint4 w = lds128(a);
+                uint4 h;
+                h.x = pack_half2(bf16_lo(w.x), bf16_hi(w.x));
+                h.y = pack_half2(bf16_lo(w.y), bf16_hi(w.y));
+                h.z = pack_half2(bf16_lo(w.z), bf16_hi(w.z));
+                h.w = pack_half2(bf16_lo(w.w), bf16_hi(w.w));
+                sts128(a, h);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bar_addr(sb, B_KQ_CONV + s));
+        }
+    } else if (warp < 8) {
+        // ================= prep: Gram epilogue, solve, P T =================
+        const int t = threadIdx.x - 128;            // 0..127 = TMEM lane
+        const int q = warp - 4;                     // warp within the group
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+        GroupSync gsync{bar_addr(sb, B_PREP_SYNC), 0};
+        const uint32_t as = sb + OFF_AS, ps = sb + OFF_PS;
+        float* adiag = reinterpret_cast<float*>(sbase + OFF_ADIAG);
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c & 1;
+            const uint32_t ph = (c >> 1) & 1;
+            if (!mbar_wait(bar_addr(sb, B_G_FULL), c & 1, abort_flag, err, kTimeoutNs)) break;
+            if (!mbar_wait(bar_addr(sb, B_GATE_FULL + s), ph, abort_flag, err, kTimeoutNs)) break;
+            tc_fence_after();
+            const Gates* gs = gate(s);
+            const int r = t & 63;
+            const bool is_a = t < 64;               // rows of K K^T (A) or Q K^T (P)
+            const float Gr = gs->G[r], gr = gs->gam[r];
+            const bool safe = gs->safe != 0;
+            const uint32_t dst = is_a ? as : ps;
+            #pragma unroll
+            for (int piece = 0; piece < 2; ++piece) {
+                float v[32];
+                tmem_ld32(tmem + TM_G + lane_addr + 32 * piece, v);
+                tmem_wait_ld();
+                #pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int sc = 32 * piece + j;
+                    const bool keep = is_a ? (sc < r) : (sc <= r);
+                    const float dec = safe ? gr * gs->einv[sc] : __expf(Gr - gs->G[sc]);
+                    v[j] = keep ? gs->beta[sc] * dec * v[j] : 0.f;
+                }
+                if (is_a) {
+                    const int b = r >> 4;
+                    if ((b >> 1) == piece) {
+                        const int j0 = (b & 1) * 16;
+                        #pragma unroll
+                        for (int j = 0; j < 16; ++j) adiag[b * 256 + (r & 15) * 16 + j] = v[j0 + j];
+                    }
+                }
+                #pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint4 w;
+                    w.x = pack_half2(v[8 * ch + 0], v[8 * ch + 1]);
+                    w.y = pack_half2(v[8 * ch + 2], v[8 * ch + 3]);
+                    w.z = pack_half2(v[8 * ch + 4], v[8 * ch + 5]);
+                    w.w = pack_half2(v[8 * ch + 6], v[8 * ch + 7]);
+                    sts128(sw128(dst, r, 4 * piece + ch), w);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar_addr(sb, B_G_EMPTY));
+            mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
+            // the [T; PT] stage must be free (MMA_B two chunks back has completed)
+            if (!mbar_wait(bar_addr(sb, B_TP_EMPTY + s), ph ^ 1, abort_flag, err, kTimeoutNs)) break;
+            if (!gsync.sync(abort_flag, err)) break;
+            const uint32_t tp = sb + OFF_TP + s * TP_STAGE;
+            if (is_a) {
+                // row r of D_b^{-1} = (I + A_bb)^{-1} by the column recurrence within the block
+                const int b = r >> 4, i = r & 15;
+                const float* ad = adiag + b * 256;
+                float x[16];
+                #pragma unroll
+                for (int j = 15; j >= 0; --j) {
+                    float acc = 0.f;
+                    #pragma unroll
+                    for (int m = j + 1; m < 16; ++m) acc += x[m] * ad[m * 16 + j];
+                    x[j] = (j == i) ? 1.f : ((j < i) ? -acc : 0.f);
+                }
+                #pragma unroll
+                for (int ch = 0; ch < 2; ++ch) {
+                    uint4 w;
+                    w.x = pack_half2(x[8 * ch + 0], x[8 * ch + 1]);
+                    w.y = pack_half2(x[8 * ch + 2], x[8 * ch + 3]);
+                    w.z = pack_half2(x[8 * ch + 4], x[8 * ch + 5]);
+                    w.w = pack_half2(x[8 * ch + 6], x[8 * ch + 7]);
+                    sts128(sw128(tp, r, 2 * b + ch), w);
+                }
+            }
+            if (!gsync.sync(abort_flag, err)) break;
+            if (q < 3) t_block(tp, as, q + 1, q, lane);          // T_{q+1,q}
+            if (!gsync.sync(abort_flag, err)) break;
+            if (q < 2) t_block(tp, as, q + 2, q, lane);          // T_{q+2,q}
+            if (!gsync.sync(abort_flag, err)) break;
+            if (q == 0) t_block(tp, as, 3, 0, lane);             // T_30
+            if (!gsync.sync(abort_flag, err)) break;
+            pt_row(tp, ps, q, lane);                             // PT block-row q
+            fence_proxy_async_smem();
+            mbar_arrive(bar_addr(sb, B_TP_FULL + s));
+        }
+    } else {
+        // ================= chain of one d_v half =================
+        const int h = (warp - 8) >> 2;              // 0: columns 0-63, 1: columns 64-127
+        const int t = (threadIdx.x - 256) & 127;    // 0..127 = TMEM lane
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+        const uint32_t tA = tmem + TM_A + 64 * h + lane_addr;
+        const uint32_t tB = tmem + TM_B + 64 * h + lane_addr;
+        const uint32_t tS = tmem + TM_S + 64 * h + lane_addr;
+        const uint32_t sop = sb + OFF_SOP + h * 16384;
+        const uint32_t xop = sb + OFF_XOP + h * 8192;
+        const uint32_t uop = sb + OFF_UOP + h * 8192;
+        bool ok = nchunks > 0;
+        // initial state: S0 (fp32 master in TMEM pre-scaled by the first chunk's decay,
+        // fp16 copy in shared memory)
+        if (ok) ok = mbar_wait(bar_addr(sb, B_GATE_FULL + 0), 0, abort_flag, err, kTimeoutNs);
+        if (ok) {
+            const float g0 = gate(0)->gC;
+            const float* s0row = p.S0 ? p.S0 + (static_cast<int64_t>(ug) * kD + t) * kD + 64 * h : nullptr;
+            #pragma unroll
+            for (int piece = 0; piece < 2; ++piece) {
+                float v[32];
+                #pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    float4 f = s0row ? *reinterpret_cast<const float4*>(s0row + 32 * piece + j)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[j] = f.x; v[j + 1] = f.y; v[j + 2] = f.z; v[j + 3] = f.w;
+                }
+                #pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint4 w;
+                    w.x = pack_half2(v[8 * ch + 0], v[8 * ch + 1]);
+                    w.y = pack_half2(v[8 * ch + 2], v[8 * ch + 3]);
+                    w.z = pack_half2(v[8 * ch + 4], v[8 * ch + 5]);
+                    w.w = pack_half2(v[8 * ch + 6], v[8 * ch + 7]);
+                    sts128(sw128(sop, t, 4 * piece + ch), w);
+                }
+                #pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] *= g0;
+                tmem_st32(tS + 32 * piece, v);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            fence_proxy_async_smem();
+            mbar_arrive(bar_addr(sb, B_SOP_FULL + h));
+        }
+        for (int c = 0; ok && c < nchunks; ++c) {
+            const int s = c & 1;
+            const uint32_t ph = (c >> 1) & 1;
+            const int64_t t0 = static_cast<int64_t>(c) * kC;
+            const Gates* gs = gate(s);
+            // --- step 1: X = V - g (K S) ---
+            ok = mbar_wait(bar_addr(sb, B_A_FULL + h), c & 1, abort_flag, err, kTimeoutNs) &&
+                 mbar_wait(bar_addr(sb, B_KQ_FULL + s), ph, abort_flag, err, kTimeoutNs);
+            if (!ok) break;
+            tc_fence_after();
+            if (t < 64) {
+                const float g = gs->gam[t];
+                const uint32_t vt = sb + OFF_V + s * V_STAGE + h * 8192;
+                #pragma unroll
+                for (int piece = 0; piece < 2; ++piece) {
+                    float ks[32];
+                    tmem_ld32(tA + 32 * piece, ks);
+                    tmem_wait_ld();
+                    #pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        const uint4 w = lds128(sw128(vt, t, 4 * piece + ch));
+                        const float* kc = ks + 8 * ch;
+                        uint4 x;
+                        x.x = pack_half2(bf16_lo(w.x) - g * kc[0], bf16_hi(w.x) - g * kc[1]);
+                        x.y = pack_half2(bf16_lo(w.y) - g * kc[2], bf16_hi(w.y) - g * kc[3]);
+                        x.z = pack_half2(bf16_lo(w.z) - g * kc[4], bf16_hi(w.z) - g * kc[5]);
+                        x.w = pack_half2(bf16_lo(w.w) - g * kc[6], bf16_hi(w.w) - g * kc[7]);
+                        sts128(sw128(xop, t, 4 * piece + ch), x);
+                    }
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            mbar_arrive(bar_addr(sb, B_X_FULL + h));
+            mbar_arrive(bar_addr(sb, B_V_EMPTY + s));
+            // --- step 2: U~ for the state update; o = g (Q S) + P T X ---
+            ok = mbar_wait(bar_addr(sb, B_B_FULL + h), c & 1, abort_flag, err, kTimeoutNs);
+            if (!ok) break;
+            tc_fence_after();
+            if (t < 64) {
+                const float bg = gs->bgc[t];
+                #pragma unroll
+                for (int piece = 0; piece < 2; ++piece) {
+                    float u[32];
+                    tmem_ld32(tB + 32 * piece, u);
+                    tmem_wait_ld();
+                    #pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        const float* uc = u + 8 * ch;
+                        uint4 w;
+                        w.x = pack_half2(bg * uc[0], bg * uc[1]);
+                        w.y = pack_half2(bg * uc[2], bg * uc[3]);
+                        w.z = pack_half2(bg * uc[4], bg * uc[5]);
+                        w.w = pack_half2(bg * uc[6], bg * uc[7]);
+                        sts128(sw128(uop, t, 4 * piece + ch), w);
+                    }
+                }
+            } else {
+                const int r = t - 64;
+                const int64_t tok = t0 + r;
+                const float g = gs->gam[r];
+                #pragma unroll
+                for (int piece = 0; piece < 2; ++piece) {
+                    float qs[32], pu[32];
+                    tmem_ld32(tA + 32 * piece, qs);
+                    tmem_ld32(tB + 32 * piece, pu);
+                    tmem_wait_ld();
+                    if (tok < L) {
+                        const int64_t col = static_cast<int64_t>(ug) * L * kD + tok * kD + 64 * h + 32 * piece;
+                        if (p.out_bf16) {
+                            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + col;
+                            #pragma unroll
+                            for (int ch = 0; ch < 4; ++ch) {
+                                uint32_t wv[4];
+                                #pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int j = 8 * ch + 2 * e;
+                                    __nv_bfloat162 b2 = __floats2bfloat162_rn(g * qs[j] + pu[j], g * qs[j + 1] + pu[j + 1]);
+                                    wv[e] = *reinterpret_cast<uint32_t*>(&b2);
+                                }
+                                st_global_v4(orow + 8 * ch, make_uint4(wv[0], wv[1], wv[2], wv[3]));
+                            }
+                        } else {
+                            float* orow = static_cast<float*>(p.o) + col;
+                            #pragma unroll
+                            for (int ch = 0; ch < 8; ++ch) {
+                                const int j = 4 * ch;
+                                st_global_v4(orow + j, make_uint4(__float_as_uint(g * qs[j] + pu[j]),
+                                                                  __float_as_uint(g * qs[j + 1] + pu[j + 1]),
+                                                                  __float_as_uint(g * qs[j + 2] + pu[j + 2]),
+                                                                  __float_as_uint(g * qs[j + 3] + pu[j + 3])));
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            mbar_arrive(bar_addr(sb, B_U_FULL + h));
+            mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
+            // --- step 3: the new state ---
+            ok = mbar_wait(bar_addr(sb, B_S_FULL + h), c & 1, abort_flag, err, kTimeoutNs);
+            if (!ok) break;
+            tc_fence_after();
+            if (c + 1 == nchunks) {
+                if (p.S_out) {
+                    float* so = p.S_out + (static_cast<int64_t>(ug) * kD + t) * kD + 64 * h;
+                    #pragma unroll
+                    for (int piece = 0; piece < 2; ++piece) {
+                        float v[32];
+                        tmem_ld32(tS + 32 * piece, v);
+                        tmem_wait_ld();
+                        #pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            st_global_v4(so + 32 * piece + j, make_uint4(__float_as_uint(v[j]), __float_as_uint(v[j + 1]),
+                                                                         __float_as_uint(v[j + 2]), __float_as_uint(v[j + 3])));
+                    }
+                }
+            } else {
+                const int s1 = (c + 1) & 1;
+                ok = mbar_wait(bar_addr(sb, B_GATE_FULL + s1), ((c + 1) >> 1) & 1, abort_flag, err, kTimeoutNs);
+                if (!ok) break;
+                const float gn = gate(s1)->gC;
+                #pragma unroll
+                for (int piece = 0; piece < 2; ++piece) {
+                    float v[32];
+                    tmem_ld32(tS + 32 * piece, v);
+                    tmem_wait_ld();
+                    #pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint4 w;
+                        w.x = pack_half2(v[8 * ch + 0], v[8 * ch + 1]);
+                        w.y = pack_half2(v[8 * ch + 2], v[8 * ch + 3]);
+                        w.z = pack_half2(v[8 * ch + 4], v[8 * ch + 5]);
+                        w.w = pack_half2(v[8 * ch + 6], v[8 * ch + 7]);
+                        sts128(sw128(sop, t, 4 * piece + ch), w);
+                    }
+                    #pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] *= gn;
+                    tmem_st32(tS + 32 * piece, v);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                fence_proxy_async_smem();
+                mbar_arrive(bar_addr(sb, B_SOP_FULL + h));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, TM_COLS);
+}
+
+// ---- host side ----------------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// 3-D view [units][L][128] of a bf16 tensor, boxes of 64 columns x 64 tokens x 1 unit,
+// 128-byte swizzle.  Rows past a unit's L are filled with zeros by the TMA unit.
+static bool make_map(CUtensorMap* m, const void* base, int64_t units, int64_t L)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(L),
+                                static_cast<cuuint64_t>(units)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * 2, static_cast<cuuint64_t>(L) * kD * 2};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kC), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace tc
+
+bool prefill_tc_supports(int dtype_bf16, int dk, int dv, int per_key)
+{
+    return dtype_bf16 && dk == tc::kD && dv == tc::kD && !per_key;
+}
+
+cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
+{
+    using namespace tc;
+    if (call.units_per_loop == 0 || call.T == 0) return cudaSuccess;
+    const int64_t units = call.T * call.units_per_loop;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, call.q, units, call.L) || !make_map(&mk, call.k, units, call.L) ||
+        !make_map(&mv, call.v, units, call.L))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(gdr_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(SMEM_BYTES));
+    if (e != cudaSuccess) return e;
+    for (int64_t tau = 0; tau < call.T; ++tau) {
+        Params p;
+        p.alpha = call.alpha;
+        p.beta = call.beta;
+        p.S0 = call.S0;
+        p.o = call.o;
+        p.S_out = call.S_out;
+        p.L = call.L;
+        p.unit0 = static_cast<int>(tau * call.units_per_loop);
+        p.out_bf16 = call.out_bf16;
+        p.err = call.err;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(call.units_per_loop), 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = SMEM_BYTES;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = tau > 0 ? 1 : 0;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const int use_pdl = tau > 0 ? 1 : 0;
+        e = cudaLaunchKernelEx(&cfg, gdr_prefill_tc_kernel, mq, mk, mv, p, use_pdl);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
 
 }  // namespace lt2

@@ -205,16 +205,35 @@ lt2_status lt2_gdr_prefill(const lt2_gdr_dims* dims, const void* q, const void* 
     if (st != LT2_OK) return st;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const bool tc = use_tensor_core(dims);
+    const bool tc = use_tensor_core(dims) && dims->L > 0;
+    if (tc) {
+        lt2::TcCall call;
+        call.q = q;
+        call.k = k;
+        call.v = v;
+        call.alpha = alpha;
+        call.beta = beta;
+        call.S0 = S0;
+        call.o = o;
+        call.S_out = S_out;
+        call.T = dims->T;
+        call.units_per_loop = sz.per_loop;
+        call.L = dims->L;
+        call.out_bf16 = out_is_bf16(dims) ? 1 : 0;
+        call.err = err;
+        cudaError_t e = lt2::launch_prefill_tc_all(call, s);
+        if (e == cudaSuccess) e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "prefill (tensor core)");
+        return LT2_OK;
+    }
     for (int64_t tau = 0; tau < dims->T; ++tau) {
         const lt2::LoopSlice ls = loop_slice(dims, sz, tau, q, k, v, alpha, beta, S0, o, S_out, err);
         // Loop 0 waits for all earlier work on the stream; later loops may start as soon as
         // the previous loop's grid is running (the loops share no data).
         const bool pdl = tau > 0;
-        cudaError_t e = tc ? lt2::launch_prefill_tc(ls, s, pdl)
-                           : lt2::launch_prefill_seq(ls, dims->dtype == LT2_DTYPE_BF16, s, pdl);
+        cudaError_t e = lt2::launch_prefill_seq(ls, dims->dtype == LT2_DTYPE_BF16, s, pdl);
         if (e == cudaSuccess) e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, tc ? "prefill (tensor core)" : "prefill (cuda core)");
+        if (e != cudaSuccess) return cuda_fail(e, "prefill (cuda core)");
     }
     return LT2_OK;
 }
