@@ -21,9 +21,10 @@
 //   MMA_B  [T; PT] X          (M=128, N=64, K=64)      -> TMEM  (U   | P T X)
 //   MMA_C  S += K^T U~        (M=128, N=64, K=64)      -> TMEM  (the fp32 state)
 //
-// for each half of d_v (two independent 64-column chains, so one half's CUDA-core epilogue
-// overlaps the other half's MMAs).  The state lives in TMEM in fp32 for the whole sequence;
-// its fp16 copy in shared memory is the B operand of MMA_A.
+// for each half of d_v: two independent 64-column chains, each with its own MMA-issuing
+// thread, so one half's CUDA-core epilogue overlaps the other half's MMAs.  The state lives
+// in TMEM in fp32 for the whole sequence; its fp16 copy in shared memory is the B operand
+// of MMA_A.
 //
 // Precision.  All MMA operands are fp16 (10-bit mantissa), not bf16: with bf16
 // intermediates (S, X, [T;PT], U~ rounded to 8 significant bits) the error against the
@@ -33,13 +34,17 @@
 //
 // CTA = one (loop, batch, head) unit, 16 warps:
 //   warp 0       TMA producer (and TMEM allocation)
-//   warp 1       tcgen05.mma issuer (one thread)
-//   warps 2-3    chunk gates (log-decay prefix sums) and bf16 -> fp16 conversion of K, Q
+//   warp 1       tcgen05.mma issuer for the d_v half 0 chain
+//   warp 2       chunk gates (log-decay prefix sums), bf16 -> fp16 conversion of K and Q,
+//                and the Gram products [K; Q] K^T as soon as a chunk is converted
+//   warp 3       tcgen05.mma issuer for the d_v half 1 chain
 //   warps 4-7    "prep": Gram epilogue, the 64x64 triangular solve (16x16 blocks with
 //                warp-level mma.sync), P T; writes [T; PT] for MMA_B
 //   warps 8-11   chain of d_v columns 0..63;  warps 12-15  chain of columns 64..127
-// Every wait is bounded (see mbar_wait); on a timeout the CTA records it in the device
-// status word, drains its in-flight copies and MMAs, frees TMEM and exits.
+// Every wait on an mbarrier is bounded (see mbar_wait) and made by one thread per group;
+// the group then meets at a named barrier and reads the outcome from shared memory, so a
+// timeout leaves every thread of the group on the same path.  On a timeout the CTA records
+// it in the device status word, drains its in-flight copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -71,8 +76,9 @@ constexpr uint32_t OFF_XOP = OFF_SOP + 2 * 16384;     // per half: X (fp16) [64 
 constexpr uint32_t OFF_UOP = OFF_XOP + 2 * 8192;      // per half: U~ (fp16) [64 tokens][64]
 constexpr uint32_t OFF_AS = OFF_UOP + 2 * 8192;       // A (fp16) [64][64]
 constexpr uint32_t OFF_PS = OFF_AS + 8192;            // P (fp16) [64][64]
-constexpr uint32_t OFF_ADIAG = OFF_PS + 8192;         // diagonal 16x16 blocks of A, fp32
-constexpr uint32_t OFF_GATES = OFF_ADIAG + 4096;
+constexpr uint32_t OFF_ADIAG = OFF_PS + 8192;         // diagonal 16x16 blocks of A, fp32, rows padded to 17
+constexpr uint32_t ADIAG_BLOCK = 16 * 17;
+constexpr uint32_t OFF_GATES = OFF_ADIAG + 4608;
 constexpr uint32_t GATE_STAGE = 1536;
 constexpr uint32_t OFF_BAR = OFF_GATES + 2 * GATE_STAGE;
 constexpr uint32_t BAR_BYTES = 512;
@@ -82,7 +88,7 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;     // slack for aligning the 
 struct Gates {
     float G[kC];       // chunk-local cumulative log-decay
     float gam[kC];     // e^{G_r}
-    float einv[kC];    // e^{-G_s} (valid when `safe`)
+    float bein[kC];    // beta_s e^{-G_s} (valid when `safe`)
     float beta[kC];    // beta_s (0 beyond the sequence end)
     float bgc[kC];     // beta_s e^{G_63 - G_s}
     float gC;          // e^{G_63}
@@ -90,12 +96,12 @@ struct Gates {
 };
 static_assert(sizeof(Gates) <= GATE_STAGE, "gate stage too small");
 
-// Barrier slots (8 bytes each) inside the OFF_BAR area.
+// Barrier slots (8 bytes each) inside the OFF_BAR area.  [2] = per stage or per half.
 enum Bar : uint32_t {
     B_KQ_FULL = 0,     // [2] TMA landed (tx count)
     B_KQ_CONV = 2,     // [2] K, Q converted to fp16
-    B_KQ_EMPTY = 4,    // [2] MMAs done with the K|Q stage
-    B_V_EMPTY = 6,     // [2] chains done with the V stage
+    B_KQ_EMPTY = 4,    // [2] both chains' MMAs done with the K|Q stage
+    B_V_EMPTY = 6,     // [2] both chains done with the V stage
     B_GATE_FULL = 8,   // [2]
     B_GATE_EMPTY = 10, // [2]
     B_TP_FULL = 12,    // [2]
@@ -108,12 +114,17 @@ enum Bar : uint32_t {
     B_U_FULL = 24,     // [2]
     B_S_FULL = 26,     // [2]
     B_SOP_FULL = 28,   // [2]
-    B_PREP_SYNC = 30,  // prep-group barrier (reused phase by phase)
-    B_DRAIN = 31,      // MMA drain on abort
-    B_COUNT = 32
+    B_DRAIN = 30,      // [3] per MMA-issuing thread, drain on abort
+    B_COUNT = 33
 };
 constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + B_COUNT * 8;        // tcgen05.alloc result
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 16;
+constexpr uint32_t OFF_OKFLAG = OFF_ABORT + 16;                  // [3 groups][2] wait outcomes
+
+// Named barriers (bar.sync ids; 0 is __syncthreads).
+constexpr int NB_PREP = 1;             // warps 4-7
+constexpr int NB_CHAIN = 2;            // + 2*h : warps of chain h (128 threads)
+constexpr int NB_LOW = 3;              // + 2*h : first two warps of chain h (64 threads)
 
 // TMEM columns (fp32 accumulators, 128 lanes each).
 constexpr uint32_t TM_G = 0;                     // Gram [K;Q] K^T, 64 columns
@@ -140,17 +151,38 @@ struct Params {
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t base, uint32_t i) { return base + OFF_BAR + 8u * i; }
 
-// Prep-group (warps 4-7) barrier on a shared mbarrier; bounded like every other wait.
-struct GroupSync {
-    uint32_t bar;
-    uint32_t phase;
-    __device__ bool sync(volatile int* abort_flag, unsigned int* err)
+__device__ __forceinline__ void named_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// A group of warps that waits through one leader: the leader makes the bounded waits, the
+// group meets at its named barrier and every thread reads the outcome.  Two outcome slots
+// alternate, so the leader never overwrites a slot another thread has yet to read.
+struct Group {
+    int nb;             // named barrier id
+    int nthreads;
+    bool leader;
+    volatile int* slots;
+    uint32_t k;
+    volatile int* abort_flag;
+    unsigned int* err;
+
+    __device__ bool wait(uint32_t bar0, uint32_t par0, uint32_t bar1 = 0, uint32_t par1 = 0,
+                         uint32_t bar2 = 0, uint32_t par2 = 0)
     {
-        mbar_arrive(bar);
-        const bool ok = mbar_wait(bar, phase & 1u, abort_flag, err, kTimeoutNs);
-        ++phase;
-        return ok;
+        volatile int* slot = slots + (k & 1u);
+        ++k;
+        if (leader) {
+            bool ok = mbar_wait(bar0, par0, abort_flag, err, kTimeoutNs);
+            if (ok && bar1) ok = mbar_wait(bar1, par1, abort_flag, err, kTimeoutNs);
+            if (ok && bar2) ok = mbar_wait(bar2, par2, abort_flag, err, kTimeoutNs);
+            *slot = ok ? 1 : 0;
+        }
+        named_sync(nb, nthreads);
+        return *slot != 0;
     }
+    __device__ void sync() { named_sync(nb, nthreads); }
 };
 
 // --- prep helpers: 16x16 fp16 blocks of row-major 128B-swizzled tiles --------------------
@@ -218,26 +250,96 @@ __device__ void t_block(uint32_t tp, uint32_t as, int i, int j, int lane)
     store_block(tp, 16 * i, 16 * j, lane, acc, -1.f);
 }
 
-// PT_qj = sum_{k=j}^{q} P_qk T_kj for j = 0..q, stored in rows 64.. of TP.
-__device__ void pt_row(uint32_t tp, uint32_t ps, int q, int lane)
+// PT_qj = sum_{k=j}^{q} P_qk T_kj, stored in rows 64.. of TP (column j of T must be final).
+__device__ void pt_block(uint32_t tp, uint32_t ps, int q, int j, int lane)
 {
-    for (int j = 0; j <= q; ++j) {
-        float acc[2][4];
-        zero_c(acc);
-        for (int k = j; k <= q; ++k) {
-            uint32_t a[4], b[4];
-            frag_a(ps, 16 * q, 16 * k, lane, a);
-            frag_b(tp, 16 * k, 16 * j, lane, b);
-            mma_block(acc, a, b);
-        }
-        store_block(tp, 64 + 16 * q, 16 * j, lane, acc, 1.f);
+    float acc[2][4];
+    zero_c(acc);
+    for (int k = j; k <= q; ++k) {
+        uint32_t a[4], b[4];
+        frag_a(ps, 16 * q, 16 * k, lane, a);
+        frag_b(tp, 16 * k, 16 * j, lane, b);
+        mma_block(acc, a, b);
     }
+    store_block(tp, 64 + 16 * q, 16 * j, lane, acc, 1.f);
 }
 
 __device__ __forceinline__ void st_global_v4(void* p, uint4 v)
 {
     asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};"
                  ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+__device__ __forceinline__ uint4 pack8_half(const float* v)
+{
+    uint4 w;
+    w.x = pack_half2(v[0], v[1]);
+    w.y = pack_half2(v[2], v[3]);
+    w.z = pack_half2(v[4], v[5]);
+    w.w = pack_half2(v[6], v[7]);
+    return w;
+}
+
+// Gram products [K; Q] K^T of chunk c (M=128, N=64, K=128) into TMEM, then commit.
+__device__ __forceinline__ void issue_gram(uint32_t sb, uint32_t tmem, int c)
+{
+    const uint32_t kq = sb + OFF_KQ + (c & 1) * KQ_STAGE;
+    for (int k = 0; k < 8; ++k) {
+        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+        umma_f16(tmem + TM_G, smem_desc_sw128(kq + off, 16, 1024), smem_desc_sw128(kq + off, 16, 1024),
+                 ID_KK, k > 0);
+    }
+    umma_commit(bar_addr(sb, B_G_FULL));
+}
+
+// Issues the chain MMAs of d_v half h.
+__device__ void mma_issuer(int h, uint32_t sb, uint32_t tmem, int nchunks, volatile int* abort_flag,
+                           unsigned int* err)
+{
+    auto wait = [&](uint32_t b, uint32_t par) { return mbar_wait(bar_addr(sb, b), par, abort_flag, err, kTimeoutNs); };
+    bool ok = true;
+    const uint32_t sop = sb + OFF_SOP + h * 16384;
+    const uint32_t xop = sb + OFF_XOP + h * 8192;
+    const uint32_t uop = sb + OFF_UOP + h * 8192;
+    for (int c = 0; ok && c < nchunks; ++c) {
+        const int s = c & 1;
+        const uint32_t ph = (c >> 1) & 1;
+        const uint32_t kq = sb + OFF_KQ + s * KQ_STAGE;
+        // MMA_A: [K; Q] S
+        ok = wait(B_KQ_CONV + s, ph) && wait(B_SOP_FULL + h, c & 1);
+        if (!ok) break;
+        tc_fence_after();
+        for (int k = 0; k < 8; ++k) {
+            const uint32_t aoff = (k >> 2) * 16384 + (k & 3) * 32;
+            umma_f16(tmem + TM_A + 64 * h, smem_desc_sw128(kq + aoff, 16, 1024),
+                     smem_desc_sw128(sop + k * 2048, 8192, 1024), ID_KM, k > 0);
+        }
+        umma_commit(bar_addr(sb, B_A_FULL + h));
+        // MMA_B: [T; PT] X
+        ok = wait(B_TP_FULL + s, ph) && wait(B_X_FULL + h, c & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tp = sb + OFF_TP + s * TP_STAGE;
+        for (int k = 0; k < 4; ++k)
+            umma_f16(tmem + TM_B + 64 * h, smem_desc_sw128(tp + k * 32, 16, 1024),
+                     smem_desc_sw128(xop + k * 2048, 8192, 1024), ID_KM, k > 0);
+        umma_commit(bar_addr(sb, B_B_FULL + h));
+        umma_commit(bar_addr(sb, B_TP_EMPTY + s));
+        // MMA_C: S += K^T U~
+        ok = wait(B_U_FULL + h, c & 1);
+        if (!ok) break;
+        tc_fence_after();
+        for (int k = 0; k < 4; ++k)
+            umma_f16(tmem + TM_S + 64 * h, smem_desc_sw128(kq + k * 2048, 16384, 1024),
+                     smem_desc_sw128(uop + k * 2048, 8192, 1024), ID_MM, 1);
+        umma_commit(bar_addr(sb, B_S_FULL + h));
+        umma_commit(bar_addr(sb, B_KQ_EMPTY + s));
+    }
+    if (!ok) {
+        // wait for every MMA this thread issued before TMEM is released
+        umma_commit(bar_addr(sb, B_DRAIN + h));
+        mbar_wait(bar_addr(sb, B_DRAIN + h), 0, abort_flag, err, kTimeoutNs / 4);
+    }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -252,11 +354,15 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t sb = (raw + 1023u) & ~1023u;        // 1024-aligned base (swizzle atoms)
     uint8_t* sbase = smem_raw + (sb - raw);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + OFF_ABORT);
-    Gates* gates = reinterpret_cast<Gates*>(sbase + OFF_GATES);   // [2], GATE_STAGE apart
+    volatile int* okflags = reinterpret_cast<volatile int*>(sbase + OFF_OKFLAG);
     auto gate = [&](int s) -> Gates* {
         return reinterpret_cast<Gates*>(sbase + OFF_GATES + s * GATE_STAGE);
     };
-    (void)gates;
+    // Plain shared-memory accesses by absolute shared address (so the compiler can batch and
+    // schedule them); ordering with other threads and with the async proxy comes from the
+    // barriers and proxy fences, which are memory-clobbering asm statements.
+    auto lds = [&](uint32_t addr) -> uint4 { return *reinterpret_cast<const uint4*>(sbase + (addr - sb)); };
+    auto sts = [&](uint32_t addr, uint4 v) { *reinterpret_cast<uint4*>(sbase + (addr - sb)) = v; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -270,24 +376,24 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         *abort_flag = 0;
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar_addr(sb, B_KQ_FULL + s), 1);
-            mbar_init(bar_addr(sb, B_KQ_CONV + s), 64);
-            mbar_init(bar_addr(sb, B_KQ_EMPTY + s), 1);
-            mbar_init(bar_addr(sb, B_V_EMPTY + s), 256);
+            mbar_init(bar_addr(sb, B_KQ_CONV + s), 1);
+            mbar_init(bar_addr(sb, B_KQ_EMPTY + s), 2);
+            mbar_init(bar_addr(sb, B_V_EMPTY + s), 2);
             mbar_init(bar_addr(sb, B_GATE_FULL + s), 1);
-            mbar_init(bar_addr(sb, B_GATE_EMPTY + s), 384);
-            mbar_init(bar_addr(sb, B_TP_FULL + s), 128);
-            mbar_init(bar_addr(sb, B_TP_EMPTY + s), 1);
+            mbar_init(bar_addr(sb, B_GATE_EMPTY + s), 3);
+            mbar_init(bar_addr(sb, B_TP_FULL + s), 1);
+            mbar_init(bar_addr(sb, B_TP_EMPTY + s), 2);
             mbar_init(bar_addr(sb, B_A_FULL + s), 1);
             mbar_init(bar_addr(sb, B_B_FULL + s), 1);
-            mbar_init(bar_addr(sb, B_X_FULL + s), 128);
-            mbar_init(bar_addr(sb, B_U_FULL + s), 128);
+            mbar_init(bar_addr(sb, B_X_FULL + s), 1);
+            mbar_init(bar_addr(sb, B_U_FULL + s), 1);
             mbar_init(bar_addr(sb, B_S_FULL + s), 1);
-            mbar_init(bar_addr(sb, B_SOP_FULL + s), 128);
+            mbar_init(bar_addr(sb, B_SOP_FULL + s), 1);
+            mbar_init(bar_addr(sb, B_DRAIN + s), 1);
         }
         mbar_init(bar_addr(sb, B_G_FULL), 1);
-        mbar_init(bar_addr(sb, B_G_EMPTY), 128);
-        mbar_init(bar_addr(sb, B_PREP_SYNC), 128);
-        mbar_init(bar_addr(sb, B_DRAIN), 1);
+        mbar_init(bar_addr(sb, B_G_EMPTY), 1);
+        mbar_init(bar_addr(sb, B_DRAIN + 2), 1);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -303,7 +409,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // zero both [T; PT] stages once: the blocks above the diagonal are never written
         const int t = threadIdx.x - 128;
         for (uint32_t off = t * 16; off < 2 * TP_STAGE; off += 128 * 16)
-            sts128(sb + OFF_TP + off, make_uint4(0, 0, 0, 0));
+            sts(sb + OFF_TP + off, make_uint4(0, 0, 0, 0));
     }
     tc_fence_before();
     __syncthreads();
@@ -337,163 +443,102 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     mbar_wait(bar_addr(sb, B_KQ_FULL + (c & 1)), (c >> 1) & 1, abort_flag, err, kTimeoutNs / 4);
             }
         }
-    } else if (warp == 1) {
-        // ================= MMA issuer =================
-        if (lane == 0) {
-            bool ok = true;
-            if (nchunks > 0) {
-                ok = mbar_wait(bar_addr(sb, B_KQ_CONV + 0), 0, abort_flag, err, kTimeoutNs);
-                if (ok) {
-                    tc_fence_after();
-                    const uint32_t kq = sb + OFF_KQ;
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                        umma_f16(tmem + TM_G, smem_desc_sw128(kq + off, 16, 1024),
-                                 smem_desc_sw128(kq + off, 16, 1024), ID_KK, k > 0);
-                    }
-                    umma_commit(bar_addr(sb, B_G_FULL));
-                }
-            }
-            for (int c = 0; ok && c < nchunks; ++c) {
-                const int s = c & 1;
-                const uint32_t kq = sb + OFF_KQ + s * KQ_STAGE;
-                for (int h = 0; h < 2 && ok; ++h) {
-                    ok = mbar_wait(bar_addr(sb, B_SOP_FULL + h), c & 1, abort_flag, err, kTimeoutNs);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t sop = sb + OFF_SOP + h * 16384;
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t aoff = (k >> 2) * 16384 + (k & 3) * 32;
-                        umma_f16(tmem + TM_A + 64 * h, smem_desc_sw128(kq + aoff, 16, 1024),
-                                 smem_desc_sw128(sop + k * 2048, 8192, 1024), ID_KM, k > 0);
-                    }
-                    umma_commit(bar_addr(sb, B_A_FULL + h));
-                }
-                if (!ok) break;
-                if (c + 1 < nchunks) {
-                    const int s1 = (c + 1) & 1;
-                    ok = mbar_wait(bar_addr(sb, B_KQ_CONV + s1), ((c + 1) >> 1) & 1, abort_flag, err, kTimeoutNs) &&
-                         mbar_wait(bar_addr(sb, B_G_EMPTY), c & 1, abort_flag, err, kTimeoutNs);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t kq1 = sb + OFF_KQ + s1 * KQ_STAGE;
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                        umma_f16(tmem + TM_G, smem_desc_sw128(kq1 + off, 16, 1024),
-                                 smem_desc_sw128(kq1 + off, 16, 1024), ID_KK, k > 0);
-                    }
-                    umma_commit(bar_addr(sb, B_G_FULL));
-                }
-                ok = mbar_wait(bar_addr(sb, B_TP_FULL + s), (c >> 1) & 1, abort_flag, err, kTimeoutNs);
-                if (!ok) break;
-                const uint32_t tp = sb + OFF_TP + s * TP_STAGE;
-                for (int h = 0; h < 2 && ok; ++h) {
-                    ok = mbar_wait(bar_addr(sb, B_X_FULL + h), c & 1, abort_flag, err, kTimeoutNs);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t xop = sb + OFF_XOP + h * 8192;
-                    for (int k = 0; k < 4; ++k)
-                        umma_f16(tmem + TM_B + 64 * h, smem_desc_sw128(tp + k * 32, 16, 1024),
-                                 smem_desc_sw128(xop + k * 2048, 8192, 1024), ID_KM, k > 0);
-                    umma_commit(bar_addr(sb, B_B_FULL + h));
-                }
-                if (!ok) break;
-                umma_commit(bar_addr(sb, B_TP_EMPTY + s));
-                for (int h = 0; h < 2 && ok; ++h) {
-                    ok = mbar_wait(bar_addr(sb, B_U_FULL + h), c & 1, abort_flag, err, kTimeoutNs);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t uop = sb + OFF_UOP + h * 8192;
-                    for (int k = 0; k < 4; ++k)
-                        umma_f16(tmem + TM_S + 64 * h, smem_desc_sw128(kq + k * 2048, 16384, 1024),
-                                 smem_desc_sw128(uop + k * 2048, 8192, 1024), ID_MM, 1);
-                    umma_commit(bar_addr(sb, B_S_FULL + h));
-                }
-                if (!ok) break;
-                umma_commit(bar_addr(sb, B_KQ_EMPTY + s));
-            }
-            if (!ok) {
-                // wait for every MMA issued so far before TMEM is released
-                umma_commit(bar_addr(sb, B_DRAIN));
-                mbar_wait(bar_addr(sb, B_DRAIN), 0, abort_flag, err, kTimeoutNs / 4);
-            }
-        }
-    } else if (warp == 2 || warp == 3) {
-        // ================= gates (warp 2) and fp16 conversion of K (warp 2) / Q (warp 3) ====
+    } else if (warp == 1 || warp == 3) {
+        // ================= MMA issuers (one thread per d_v half) =================
+        if (lane == 0) mma_issuer(warp == 1 ? 0 : 1, sb, tmem, nchunks, abort_flag, err);
+    } else if (warp == 2) {
+        // ================= gates and fp16 conversion of K, Q =================
         for (int c = 0; c < nchunks; ++c) {
             const int s = c & 1;
             const uint32_t ph = (c >> 1) & 1;
-            if (warp == 2) {
-                if (!mbar_wait(bar_addr(sb, B_GATE_EMPTY + s), ph ^ 1, abort_flag, err, kTimeoutNs)) break;
-                Gates* gs = gate(s);
-                const int64_t t0 = static_cast<int64_t>(c) * kC;
-                float g[2], b[2];
-                #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int64_t tok = t0 + lane + 32 * i;
-                    const bool valid = tok < L;
-                    const float a = valid ? p.alpha[ug * L + tok] : 1.f;
-                    b[i] = valid ? p.beta[ug * L + tok] : 0.f;
-                    g[i] = __logf(fmaxf(a, 1e-30f));
-                }
-                // inclusive prefix sums over the 64 tokens
-                #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    #pragma unroll
-                    for (int off = 1; off < 32; off <<= 1) {
-                        const float y = __shfl_up_sync(0xffffffffu, g[i], off);
-                        if (lane >= off) g[i] += y;
-                    }
-                }
-                g[1] += __shfl_sync(0xffffffffu, g[0], 31);
-                const float GC = __shfl_sync(0xffffffffu, g[1], 31);
-                const bool safe = GC > -80.f;
-                #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int r = lane + 32 * i;
-                    gs->G[r] = g[i];
-                    gs->gam[r] = __expf(g[i]);
-                    gs->einv[r] = safe ? __expf(-g[i]) : 0.f;
-                    gs->beta[r] = b[i];
-                    gs->bgc[r] = b[i] * __expf(GC - g[i]);
-                }
-                if (lane == 0) {
-                    gs->gC = __expf(GC);
-                    gs->safe = safe ? 1 : 0;
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_addr(sb, B_GATE_FULL + s));
+            if (!mbar_wait(bar_addr(sb, B_GATE_EMPTY + s), ph ^ 1, abort_flag, err, kTimeoutNs)) break;
+            Gates* gs = gate(s);
+            const int64_t t0 = static_cast<int64_t>(c) * kC;
+            float g[2], b[2];
+            #pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int64_t tok = t0 + lane + 32 * i;
+                const bool valid = tok < L;
+                const float a = valid ? p.alpha[ug * L + tok] : 1.f;
+                b[i] = valid ? p.beta[ug * L + tok] : 0.f;
+                g[i] = __logf(fmaxf(a, 1e-30f));
             }
+            // inclusive prefix sums over the 64 tokens
+            #pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                #pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, g[i], off);
+                    if (lane >= off) g[i] += y;
+                }
+            }
+            g[1] += __shfl_sync(0xffffffffu, g[0], 31);
+            const float GC = __shfl_sync(0xffffffffu, g[1], 31);
+            const bool safe = GC > -80.f;
+            #pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int r = lane + 32 * i;
+                gs->G[r] = g[i];
+                gs->gam[r] = __expf(g[i]);
+                gs->bein[r] = safe ? b[i] * __expf(-g[i]) : 0.f;
+                gs->beta[r] = b[i];
+                gs->bgc[r] = b[i] * __expf(GC - g[i]);
+            }
+            if (lane == 0) {
+                gs->gC = __expf(GC);
+                gs->safe = safe ? 1 : 0;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_addr(sb, B_GATE_FULL + s));
             if (!mbar_wait(bar_addr(sb, B_KQ_FULL + s), ph, abort_flag, err, kTimeoutNs)) break;
-            const uint32_t base = sb + OFF_KQ + s * KQ_STAGE + (warp == 3 ? 8192u : 0u);
-            #pragma unroll 4
-            for (int i = 0; i < 32; ++i) {
-                const int v = i * 32 + lane;
-                const uint32_t a = base + (v < 512 ? v * 16 : 16384 + (v - 512) * 16);
-                const uint4 w = lds128(a);
-                uint4 h;
-                h.x = pack_half2(bf16_lo(w.x), bf16_hi(w.x));
-                h.y = pack_half2(bf16_lo(w.y), bf16_hi(w.y));
-                h.z = pack_half2(bf16_lo(w.z), bf16_hi(w.z));
-                h.w = pack_half2(bf16_lo(w.w), bf16_hi(w.w));
-                sts128(a, h);
+            const uint32_t base = sb + OFF_KQ + s * KQ_STAGE;
+            for (int i0 = 0; i0 < 64; i0 += 8) {
+                uint4 w[8];
+                #pragma unroll
+                for (int i = 0; i < 8; ++i) w[i] = lds(base + static_cast<uint32_t>((i0 + i) * 32 + lane) * 16u);
+                #pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    uint4 hv;
+                    hv.x = pack_half2(bf16_lo(w[i].x), bf16_hi(w[i].x));
+                    hv.y = pack_half2(bf16_lo(w[i].y), bf16_hi(w[i].y));
+                    hv.z = pack_half2(bf16_lo(w[i].z), bf16_hi(w[i].z));
+                    hv.w = pack_half2(bf16_lo(w[i].w), bf16_hi(w[i].w));
+                    sts(base + static_cast<uint32_t>((i0 + i) * 32 + lane) * 16u, hv);
+                }
             }
             fence_proxy_async_smem();
-            mbar_arrive(bar_addr(sb, B_KQ_CONV + s));
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar_addr(sb, B_KQ_CONV + s));
+                // Gram products of this chunk, as soon as its K and Q are in fp16 and the
+                // prep group has read the previous chunk's
+                if (c == 0 || mbar_wait(bar_addr(sb, B_G_EMPTY), (c - 1) & 1, abort_flag, err, kTimeoutNs)) {
+                    tc_fence_after();
+                    issue_gram(sb, tmem, c);
+                }
+            }
+            if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
+        }
+        if (lane == 0 && *abort_flag && nchunks > 0) {
+            // wait for the Gram MMAs this thread issued before TMEM is released
+            umma_commit(bar_addr(sb, B_DRAIN + 2));
+            mbar_wait(bar_addr(sb, B_DRAIN + 2), 0, abort_flag, err, kTimeoutNs / 4);
         }
     } else if (warp < 8) {
         // ================= prep: Gram epilogue, solve, P T =================
         const int t = threadIdx.x - 128;            // 0..127 = TMEM lane
         const int q = warp - 4;                     // warp within the group
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-        GroupSync gsync{bar_addr(sb, B_PREP_SYNC), 0};
+        Group grp{NB_PREP, 128, t == 0, okflags + 0, 0, abort_flag, err};
         const uint32_t as = sb + OFF_AS, ps = sb + OFF_PS;
         float* adiag = reinterpret_cast<float*>(sbase + OFF_ADIAG);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c & 1;
             const uint32_t ph = (c >> 1) & 1;
-            if (!mbar_wait(bar_addr(sb, B_G_FULL), c & 1, abort_flag, err, kTimeoutNs)) break;
-            if (!mbar_wait(bar_addr(sb, B_GATE_FULL + s), ph, abort_flag, err, kTimeoutNs)) break;
+            // Gram of chunk c in TMEM, its gates, and a free [T; PT] stage
+            if (!grp.wait(bar_addr(sb, B_G_FULL), c & 1, bar_addr(sb, B_GATE_FULL + s), ph,
+                          bar_addr(sb, B_TP_EMPTY + s), ph ^ 1))
+                break;
             tc_fence_after();
             const Gates* gs = gate(s);
             const int r = t & 63;
@@ -501,75 +546,74 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const float Gr = gs->G[r], gr = gs->gam[r];
             const bool safe = gs->safe != 0;
             const uint32_t dst = is_a ? as : ps;
-            #pragma unroll
-            for (int piece = 0; piece < 2; ++piece) {
-                float v[32];
-                tmem_ld32(tmem + TM_G + lane_addr + 32 * piece, v);
-                tmem_wait_ld();
+            float v[64];
+            tmem_ld32(tmem + TM_G + lane_addr, *reinterpret_cast<float(*)[32]>(v));
+            tmem_ld32(tmem + TM_G + lane_addr + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+            tmem_wait_ld();
+            const int lim = is_a ? r : r + 1;         // keep columns s < lim
+            if (safe) {
                 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int sc = 32 * piece + j;
-                    const bool keep = is_a ? (sc < r) : (sc <= r);
-                    const float dec = safe ? gr * gs->einv[sc] : __expf(Gr - gs->G[sc]);
-                    v[j] = keep ? gs->beta[sc] * dec * v[j] : 0.f;
+                for (int j4 = 0; j4 < 64; j4 += 4) {
+                    const float4 be = *reinterpret_cast<const float4*>(&gs->bein[j4]);
+                    v[j4 + 0] = (j4 + 0 < lim) ? gr * be.x * v[j4 + 0] : 0.f;
+                    v[j4 + 1] = (j4 + 1 < lim) ? gr * be.y * v[j4 + 1] : 0.f;
+                    v[j4 + 2] = (j4 + 2 < lim) ? gr * be.z * v[j4 + 2] : 0.f;
+                    v[j4 + 3] = (j4 + 3 < lim) ? gr * be.w * v[j4 + 3] : 0.f;
                 }
-                if (is_a) {
-                    const int b = r >> 4;
-                    if ((b >> 1) == piece) {
-                        const int j0 = (b & 1) * 16;
-                        #pragma unroll
-                        for (int j = 0; j < 16; ++j) adiag[b * 256 + (r & 15) * 16 + j] = v[j0 + j];
-                    }
-                }
+            } else {
                 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint4 w;
-                    w.x = pack_half2(v[8 * ch + 0], v[8 * ch + 1]);
-                    w.y = pack_half2(v[8 * ch + 2], v[8 * ch + 3]);
-                    w.z = pack_half2(v[8 * ch + 4], v[8 * ch + 5]);
-                    w.w = pack_half2(v[8 * ch + 6], v[8 * ch + 7]);
-                    sts128(sw128(dst, r, 4 * piece + ch), w);
-                }
+                for (int sc = 0; sc < 64; ++sc)
+                    v[sc] = (sc < lim) ? gs->beta[sc] * __expf(Gr - gs->G[sc]) * v[sc] : 0.f;
             }
+            if (is_a) {
+                const int b = r >> 4;
+                #pragma unroll
+                for (int bb = 0; bb < 4; ++bb)
+                    if (b == bb) {
+                        #pragma unroll
+                        for (int j = 0; j < 16; ++j) adiag[b * ADIAG_BLOCK + (r & 15) * 17 + j] = v[16 * bb + j];
+                    }
+            }
+            #pragma unroll
+            for (int ch = 0; ch < 8; ++ch) sts(sw128(dst, r, ch), pack8_half(v + 8 * ch));
             tc_fence_before();
-            mbar_arrive(bar_addr(sb, B_G_EMPTY));
-            mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
-            // the [T; PT] stage must be free (MMA_B two chunks back has completed)
-            if (!mbar_wait(bar_addr(sb, B_TP_EMPTY + s), ph ^ 1, abort_flag, err, kTimeoutNs)) break;
-            if (!gsync.sync(abort_flag, err)) break;
+            grp.sync();
+            if (t == 0) {
+                mbar_arrive(bar_addr(sb, B_G_EMPTY));
+                mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
+            }
             const uint32_t tp = sb + OFF_TP + s * TP_STAGE;
             if (is_a) {
                 // row r of D_b^{-1} = (I + A_bb)^{-1} by the column recurrence within the block
                 const int b = r >> 4, i = r & 15;
-                const float* ad = adiag + b * 256;
+                const float* ad = adiag + b * ADIAG_BLOCK;
                 float x[16];
                 #pragma unroll
                 for (int j = 15; j >= 0; --j) {
                     float acc = 0.f;
                     #pragma unroll
-                    for (int m = j + 1; m < 16; ++m) acc += x[m] * ad[m * 16 + j];
+                    for (int m = j + 1; m < 16; ++m) acc += x[m] * ad[m * 17 + j];
                     x[j] = (j == i) ? 1.f : ((j < i) ? -acc : 0.f);
                 }
-                #pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
-                    uint4 w;
-                    w.x = pack_half2(x[8 * ch + 0], x[8 * ch + 1]);
-                    w.y = pack_half2(x[8 * ch + 2], x[8 * ch + 3]);
-                    w.z = pack_half2(x[8 * ch + 4], x[8 * ch + 5]);
-                    w.w = pack_half2(x[8 * ch + 6], x[8 * ch + 7]);
-                    sts128(sw128(tp, r, 2 * b + ch), w);
-                }
+                sts(sw128(tp, r, 2 * b), pack8_half(x));
+                sts(sw128(tp, r, 2 * b + 1), pack8_half(x + 8));
             }
-            if (!gsync.sync(abort_flag, err)) break;
-            if (q < 3) t_block(tp, as, q + 1, q, lane);          // T_{q+1,q}
-            if (!gsync.sync(abort_flag, err)) break;
-            if (q < 2) t_block(tp, as, q + 2, q, lane);          // T_{q+2,q}
-            if (!gsync.sync(abort_flag, err)) break;
-            if (q == 0) t_block(tp, as, 3, 0, lane);             // T_30
-            if (!gsync.sync(abort_flag, err)) break;
-            pt_row(tp, ps, q, lane);                             // PT block-row q
+            grp.sync();
+            // level 1 of the block inverse, and the first column of P T that is ready
+            if (q < 3) t_block(tp, as, q + 1, q, lane);         // T_{q+1,q}
+            else pt_block(tp, ps, 3, 3, lane);                  // PT_33
+            grp.sync();
+            if (q < 2) t_block(tp, as, q + 2, q, lane);         // T_{q+2,q}
+            else if (q == 2) pt_block(tp, ps, 2, 2, lane);      // PT_22
+            else pt_block(tp, ps, 3, 2, lane);                  // PT_32
+            grp.sync();
+            if (q == 0) t_block(tp, as, 3, 0, lane);            // T_30
+            else pt_block(tp, ps, q, 1, lane);                  // PT_11, PT_21, PT_31
+            grp.sync();
+            pt_block(tp, ps, 3 - q, 0, lane);                   // PT_30, PT_20, PT_10, PT_00
             fence_proxy_async_smem();
-            mbar_arrive(bar_addr(sb, B_TP_FULL + s));
+            grp.sync();
+            if (t == 0) mbar_arrive(bar_addr(sb, B_TP_FULL + s));
         }
     } else {
         // ================= chain of one d_v half =================
@@ -582,10 +626,12 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const uint32_t sop = sb + OFF_SOP + h * 16384;
         const uint32_t xop = sb + OFF_XOP + h * 8192;
         const uint32_t uop = sb + OFF_UOP + h * 8192;
+        const int nb_low = NB_LOW + 2 * h;
+        Group grp{NB_CHAIN + 2 * h, 128, t == 0, okflags + 2 + 2 * h, 0, abort_flag, err};
         bool ok = nchunks > 0;
         // initial state: S0 (fp32 master in TMEM pre-scaled by the first chunk's decay,
         // fp16 copy in shared memory)
-        if (ok) ok = mbar_wait(bar_addr(sb, B_GATE_FULL + 0), 0, abort_flag, err, kTimeoutNs);
+        if (ok) ok = grp.wait(bar_addr(sb, B_GATE_FULL + 0), 0);
         if (ok) {
             const float g0 = gate(0)->gC;
             const float* s0row = p.S0 ? p.S0 + (static_cast<int64_t>(ug) * kD + t) * kD + 64 * h : nullptr;
@@ -599,14 +645,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     v[j] = f.x; v[j + 1] = f.y; v[j + 2] = f.z; v[j + 3] = f.w;
                 }
                 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint4 w;
-                    w.x = pack_half2(v[8 * ch + 0], v[8 * ch + 1]);
-                    w.y = pack_half2(v[8 * ch + 2], v[8 * ch + 3]);
-                    w.z = pack_half2(v[8 * ch + 4], v[8 * ch + 5]);
-                    w.w = pack_half2(v[8 * ch + 6], v[8 * ch + 7]);
-                    sts128(sw128(sop, t, 4 * piece + ch), w);
-                }
+                for (int ch = 0; ch < 4; ++ch) sts(sw128(sop, t, 4 * piece + ch), pack8_half(v + 8 * ch));
                 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] *= g0;
                 tmem_st32(tS + 32 * piece, v);
@@ -614,65 +653,62 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tmem_wait_st();
             tc_fence_before();
             fence_proxy_async_smem();
-            mbar_arrive(bar_addr(sb, B_SOP_FULL + h));
+            grp.sync();
+            if (t == 0) mbar_arrive(bar_addr(sb, B_SOP_FULL + h));
         }
         for (int c = 0; ok && c < nchunks; ++c) {
             const int s = c & 1;
             const uint32_t ph = (c >> 1) & 1;
             const int64_t t0 = static_cast<int64_t>(c) * kC;
             const Gates* gs = gate(s);
-            // --- step 1: X = V - g (K S) ---
-            ok = mbar_wait(bar_addr(sb, B_A_FULL + h), c & 1, abort_flag, err, kTimeoutNs) &&
-                 mbar_wait(bar_addr(sb, B_KQ_FULL + s), ph, abort_flag, err, kTimeoutNs);
+            // --- step 1: X = V - g (K S), by the first 64 threads (token rows) ---
+            ok = grp.wait(bar_addr(sb, B_A_FULL + h), c & 1, bar_addr(sb, B_KQ_FULL + s), ph);
             if (!ok) break;
             tc_fence_after();
             if (t < 64) {
                 const float g = gs->gam[t];
                 const uint32_t vt = sb + OFF_V + s * V_STAGE + h * 8192;
+                float ks[64];
+                tmem_ld32(tA, *reinterpret_cast<float(*)[32]>(ks));
+                tmem_ld32(tA + 32, *reinterpret_cast<float(*)[32]>(ks + 32));
+                tmem_wait_ld();
+                uint4 vw[8];
                 #pragma unroll
-                for (int piece = 0; piece < 2; ++piece) {
-                    float ks[32];
-                    tmem_ld32(tA + 32 * piece, ks);
-                    tmem_wait_ld();
-                    #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        const uint4 w = lds128(sw128(vt, t, 4 * piece + ch));
-                        const float* kc = ks + 8 * ch;
-                        uint4 x;
-                        x.x = pack_half2(bf16_lo(w.x) - g * kc[0], bf16_hi(w.x) - g * kc[1]);
-                        x.y = pack_half2(bf16_lo(w.y) - g * kc[2], bf16_hi(w.y) - g * kc[3]);
-                        x.z = pack_half2(bf16_lo(w.z) - g * kc[4], bf16_hi(w.z) - g * kc[5]);
-                        x.w = pack_half2(bf16_lo(w.w) - g * kc[6], bf16_hi(w.w) - g * kc[7]);
-                        sts128(sw128(xop, t, 4 * piece + ch), x);
-                    }
+                for (int ch = 0; ch < 8; ++ch) vw[ch] = lds(sw128(vt, t, ch));
+                #pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint4 w = vw[ch];
+                    const float* kc = ks + 8 * ch;
+                    float x[8] = {bf16_lo(w.x) - g * kc[0], bf16_hi(w.x) - g * kc[1],
+                                  bf16_lo(w.y) - g * kc[2], bf16_hi(w.y) - g * kc[3],
+                                  bf16_lo(w.z) - g * kc[4], bf16_hi(w.z) - g * kc[5],
+                                  bf16_lo(w.w) - g * kc[6], bf16_hi(w.w) - g * kc[7]};
+                    sts(sw128(xop, t, ch), pack8_half(x));
+                }
+                fence_proxy_async_smem();
+                named_sync(nb_low, 64);
+                if (t == 0) {
+                    mbar_arrive(bar_addr(sb, B_X_FULL + h));
+                    mbar_arrive(bar_addr(sb, B_V_EMPTY + s));
                 }
             }
-            tc_fence_before();
-            fence_proxy_async_smem();
-            mbar_arrive(bar_addr(sb, B_X_FULL + h));
-            mbar_arrive(bar_addr(sb, B_V_EMPTY + s));
-            // --- step 2: U~ for the state update; o = g (Q S) + P T X ---
-            ok = mbar_wait(bar_addr(sb, B_B_FULL + h), c & 1, abort_flag, err, kTimeoutNs);
+            // --- step 2: U~ for the state update (first 64 threads); o = g (Q S) + P T X ---
+            ok = grp.wait(bar_addr(sb, B_B_FULL + h), c & 1);
             if (!ok) break;
             tc_fence_after();
             if (t < 64) {
                 const float bg = gs->bgc[t];
+                float u[64];
+                tmem_ld32(tB, *reinterpret_cast<float(*)[32]>(u));
+                tmem_ld32(tB + 32, *reinterpret_cast<float(*)[32]>(u + 32));
+                tmem_wait_ld();
                 #pragma unroll
-                for (int piece = 0; piece < 2; ++piece) {
-                    float u[32];
-                    tmem_ld32(tB + 32 * piece, u);
-                    tmem_wait_ld();
-                    #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        const float* uc = u + 8 * ch;
-                        uint4 w;
-                        w.x = pack_half2(bg * uc[0], bg * uc[1]);
-                        w.y = pack_half2(bg * uc[2], bg * uc[3]);
-                        w.z = pack_half2(bg * uc[4], bg * uc[5]);
-                        w.w = pack_half2(bg * uc[6], bg * uc[7]);
-                        sts128(sw128(uop, t, 4 * piece + ch), w);
-                    }
-                }
+                for (int j = 0; j < 64; ++j) u[j] *= bg;
+                #pragma unroll
+                for (int ch = 0; ch < 8; ++ch) sts(sw128(uop, t, ch), pack8_half(u + 8 * ch));
+                fence_proxy_async_smem();
+                named_sync(nb_low, 64);
+                if (t == 0) mbar_arrive(bar_addr(sb, B_U_FULL + h));
             } else {
                 const int r = t - 64;
                 const int64_t tok = t0 + r;
@@ -713,54 +749,40 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
             }
             tc_fence_before();
-            fence_proxy_async_smem();
-            mbar_arrive(bar_addr(sb, B_U_FULL + h));
-            mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
             // --- step 3: the new state ---
-            ok = mbar_wait(bar_addr(sb, B_S_FULL + h), c & 1, abort_flag, err, kTimeoutNs);
+            const bool last = c + 1 == nchunks;
+            const int s1 = (c + 1) & 1;
+            ok = last ? grp.wait(bar_addr(sb, B_S_FULL + h), c & 1)
+                      : grp.wait(bar_addr(sb, B_S_FULL + h), c & 1, bar_addr(sb, B_GATE_FULL + s1),
+                                 ((c + 1) >> 1) & 1);
             if (!ok) break;
             tc_fence_after();
-            if (c + 1 == nchunks) {
+            if (t == 0) mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));   // gates of chunk c consumed
+            float v[64];
+            tmem_ld32(tS, *reinterpret_cast<float(*)[32]>(v));
+            tmem_ld32(tS + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+            tmem_wait_ld();
+            if (last) {
                 if (p.S_out) {
                     float* so = p.S_out + (static_cast<int64_t>(ug) * kD + t) * kD + 64 * h;
                     #pragma unroll
-                    for (int piece = 0; piece < 2; ++piece) {
-                        float v[32];
-                        tmem_ld32(tS + 32 * piece, v);
-                        tmem_wait_ld();
-                        #pragma unroll
-                        for (int j = 0; j < 32; j += 4)
-                            st_global_v4(so + 32 * piece + j, make_uint4(__float_as_uint(v[j]), __float_as_uint(v[j + 1]),
-                                                                         __float_as_uint(v[j + 2]), __float_as_uint(v[j + 3])));
-                    }
+                    for (int j = 0; j < 64; j += 4)
+                        st_global_v4(so + j, make_uint4(__float_as_uint(v[j]), __float_as_uint(v[j + 1]),
+                                                        __float_as_uint(v[j + 2]), __float_as_uint(v[j + 3])));
                 }
             } else {
-                const int s1 = (c + 1) & 1;
-                ok = mbar_wait(bar_addr(sb, B_GATE_FULL + s1), ((c + 1) >> 1) & 1, abort_flag, err, kTimeoutNs);
-                if (!ok) break;
                 const float gn = gate(s1)->gC;
                 #pragma unroll
-                for (int piece = 0; piece < 2; ++piece) {
-                    float v[32];
-                    tmem_ld32(tS + 32 * piece, v);
-                    tmem_wait_ld();
-                    #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint4 w;
-                        w.x = pack_half2(v[8 * ch + 0], v[8 * ch + 1]);
-                        w.y = pack_half2(v[8 * ch + 2], v[8 * ch + 3]);
-                        w.z = pack_half2(v[8 * ch + 4], v[8 * ch + 5]);
-                        w.w = pack_half2(v[8 * ch + 6], v[8 * ch + 7]);
-                        sts128(sw128(sop, t, 4 * piece + ch), w);
-                    }
-                    #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] *= gn;
-                    tmem_st32(tS + 32 * piece, v);
-                }
+                for (int ch = 0; ch < 8; ++ch) sts(sw128(sop, t, ch), pack8_half(v + 8 * ch));
+                #pragma unroll
+                for (int j = 0; j < 64; ++j) v[j] *= gn;
+                tmem_st32(tS, *reinterpret_cast<float(*)[32]>(v));
+                tmem_st32(tS + 32, *reinterpret_cast<float(*)[32]>(v + 32));
                 tmem_wait_st();
                 tc_fence_before();
                 fence_proxy_async_smem();
-                mbar_arrive(bar_addr(sb, B_SOP_FULL + h));
+                grp.sync();
+                if (t == 0) mbar_arrive(bar_addr(sb, B_SOP_FULL + h));
             }
         }
     }
