@@ -547,9 +547,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const bool safe = gs->safe != 0;
             const uint32_t dst = is_a ? as : ps;
             float v[64];
-            tmem_ld32(tmem + TM_G + lane_addr, *reinterpret_cast<float(*)[32]>(v));
-            tmem_ld32(tmem + TM_G + lane_addr + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-            tmem_wait_ld();
+            tmem_load_2x32(tmem + TM_G + lane_addr, tmem + TM_G + lane_addr + 32, v);
             const int lim = is_a ? r : r + 1;         // keep columns s < lim
             if (safe) {
                 #pragma unroll
@@ -668,13 +666,11 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (t < 64) {
                 const float g = gs->gam[t];
                 const uint32_t vt = sb + OFF_V + s * V_STAGE + h * 8192;
-                float ks[64];
-                tmem_ld32(tA, *reinterpret_cast<float(*)[32]>(ks));
-                tmem_ld32(tA + 32, *reinterpret_cast<float(*)[32]>(ks + 32));
-                tmem_wait_ld();
                 uint4 vw[8];
                 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) vw[ch] = lds(sw128(vt, t, ch));
+                float ks[64];
+                tmem_load_2x32(tA, tA + 32, ks);
                 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
                     const uint4 w = vw[ch];
@@ -699,9 +695,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (t < 64) {
                 const float bg = gs->bgc[t];
                 float u[64];
-                tmem_ld32(tB, *reinterpret_cast<float(*)[32]>(u));
-                tmem_ld32(tB + 32, *reinterpret_cast<float(*)[32]>(u + 32));
-                tmem_wait_ld();
+                tmem_load_2x32(tB, tB + 32, u);
                 #pragma unroll
                 for (int j = 0; j < 64; ++j) u[j] *= bg;
                 #pragma unroll
@@ -715,10 +709,10 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 const float g = gs->gam[r];
                 #pragma unroll
                 for (int piece = 0; piece < 2; ++piece) {
-                    float qs[32], pu[32];
-                    tmem_ld32(tA + 32 * piece, qs);
-                    tmem_ld32(tB + 32 * piece, pu);
-                    tmem_wait_ld();
+                    float qp[64];
+                    tmem_load_2x32(tA + 32 * piece, tB + 32 * piece, qp);
+                    const float* qs = qp;
+                    const float* pu = qp + 32;
                     if (tok < L) {
                         const int64_t col = static_cast<int64_t>(ug) * L * kD + tok * kD + 64 * h + 32 * piece;
                         if (p.out_bf16) {
@@ -759,9 +753,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tc_fence_after();
             if (t == 0) mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));   // gates of chunk c consumed
             float v[64];
-            tmem_ld32(tS, *reinterpret_cast<float(*)[32]>(v));
-            tmem_ld32(tS + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-            tmem_wait_ld();
+            tmem_load_2x32(tS, tS + 32, v);
             if (last) {
                 if (p.S_out) {
                     float* so = p.S_out + (static_cast<int64_t>(ug) * kD + t) * kD + 64 * h;
