@@ -1,5 +1,6 @@
 // gdr_prefill_tc.cu -- chunked prefill of the gated delta rule on Blackwell tensor cores
-// (tcgen05 MMA with TMEM accumulators, operands staged by TMA), scalar gating, d_k = d_v = 128.
+// (tcgen05 MMA with TMEM accumulators and TMEM operands, tiles staged by TMA), scalar gating,
+// d_k = d_v = 128.
 //
 // The recurrence ("LT2 transformer looped a tempo lineare", section "Sostituire il motore",
 // displayed equation)  S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T  with
@@ -13,34 +14,34 @@
 //   S'   = g_63 S + K^T diag(beta_s e^{G_63-G_s}) U
 //
 // (u_r = v_r - alpha_r S_{r-1}^T k_r unrolls the chunk; the identity is checked in fp64 by
-// the test suite's chunked oracle.)  Everything that does not involve S -- the Gram
-// products K K^T and Q K^T, the solve, P T -- is done one chunk ahead, overlapped with the
-// S-dependent chain of the current chunk:
+// the test suite's chunked oracle.)  Everything that does not involve S -- the Gram products
+// K K^T and Q K^T, the solve, P T -- is done ahead of the S-dependent chain.
 //
-//   MMA_A  [K; Q] S           (M=128, N=64, K=128)     -> TMEM  (K S | Q S)
-//   MMA_B  [T; PT] X          (M=128, N=64, K=64)      -> TMEM  (U   | P T X)
-//   MMA_C  S += K^T U~        (M=128, N=64, K=64)      -> TMEM  (the fp32 state)
+// The chain works on the transposed quantities, one d_v column per TMEM lane, so that every
+// S-dependent MMA operand is produced in tensor memory and never goes through shared memory:
 //
-// for each half of d_v: two independent 64-column chains, each with its own MMA-issuing
-// thread, so one half's CUDA-core epilogue overlaps the other half's MMAs.  The state lives
-// in TMEM in fp32 for the whole sequence; its fp16 copy in shared memory is the B operand
-// of MMA_A.
+//   MMA_A  (KQ S)^T  = S^T [K;Q]^T          A = S^T (TMEM, fp16)     B = [K;Q] tile
+//   MMA_B  ([T;PT] X)^T = V^T [T;PT]^T + (-g K S)^T [T;PT]^T
+//                                           A = V^T (smem) then (-g K S)^T (TMEM)   B = [T;PT]
+//   MMA_C  S^T += U~^T K                    A = U~^T (TMEM, fp16)    B = K tile
+//
+// all M = 128 (d_v), N = 128.  The fp32 state S^T stays in TMEM for the whole sequence; its
+// fp16 copy (the A operand of MMA_A) is rewritten once per chunk.
 //
 // Precision.  All MMA operands are fp16 (10-bit mantissa), not bf16: with bf16
 // intermediates (S, X, [T;PT], U~ rounded to 8 significant bits) the error against the
 // fp64 oracle reaches ~3% of rms(o) at the largest outputs, while fp16 keeps it near 0.5%.
-// q, k arrive in bf16; converting a bf16 tile to fp16 in shared memory is exact for the
+// q, k, v arrive in bf16; converting a bf16 tile to fp16 in shared memory is exact for the
 // magnitudes involved (|x| in [2^-14, 2^15]), so the inputs are not rounded again.
 //
 // CTA = one (loop, batch, head) unit, 16 warps:
 //   warp 0       TMA producer (and TMEM allocation)
-//   warp 1       tcgen05.mma issuer for the d_v half 0 chain
-//   warp 2       chunk gates (log-decay prefix sums), bf16 -> fp16 conversion of K and Q,
-//                and the Gram products [K; Q] K^T as soon as a chunk is converted
-//   warp 3       tcgen05.mma issuer for the d_v half 1 chain
+//   warp 1       chunk gates, fp16 conversion of K, and the Gram MMA [K; Q] K^T
+//   warps 2, 3   fp16 conversion of Q and of V
 //   warps 4-7    "prep": Gram epilogue, the 64x64 triangular solve (16x16 blocks with
 //                warp-level mma.sync), P T; writes [T; PT] for MMA_B
-//   warps 8-11   chain of d_v columns 0..63;  warps 12-15  chain of columns 64..127
+//   warps 8-11   the S-dependent chain (its first thread issues MMA_A, MMA_B, MMA_C)
+//   warps 12-15  output epilogue: o = g (Q S) + P T X from TMEM to global memory
 // Every wait on an mbarrier is bounded (see mbar_wait) and made by one thread per group;
 // the group then meets at a named barrier and reads the outcome from shared memory, so a
 // timeout leaves every thread of the group on the same path.  On a timeout the CTA records
@@ -62,25 +63,26 @@ using namespace sm100;
 constexpr int kC = 64;                 // tokens per chunk
 constexpr int kD = 128;                // d_k = d_v
 constexpr int kThreads = 512;
+constexpr int kStages = 3;             // K/Q/V tile stages (and gate stages)
 constexpr uint64_t kTimeoutNs = 4000000000ull;   // 4 s
 
-// Shared memory map (offsets from a 1024-byte aligned base).
-constexpr uint32_t KQ_STAGE = 32768;   // K|Q, two 64-column panels: [K rows 0-63 | Q rows 0-63]
-constexpr uint32_t V_STAGE = 16384;    // V, two 64-column panels (bf16, read by CUDA cores)
+// Shared memory map (offsets from a 1024-byte aligned base).  A K/Q/V stage holds, as fp16
+// after conversion, [K panel 0 | Q panel 0 | K panel 1 | Q panel 1 | V panel 0 | V panel 1],
+// each panel 64 rows x 128 bytes with the 128-byte swizzle.
+constexpr uint32_t KQ_BYTES = 32768;
+constexpr uint32_t V_BYTES = 16384;
+constexpr uint32_t STAGE_BYTES = KQ_BYTES + V_BYTES;
 constexpr uint32_t TP_STAGE = 16384;   // [T; PT], 128 rows x 64 fp16
-constexpr uint32_t OFF_KQ = 0;
-constexpr uint32_t OFF_V = OFF_KQ + 2 * KQ_STAGE;
-constexpr uint32_t OFF_TP = OFF_V + 2 * V_STAGE;
-constexpr uint32_t OFF_SOP = OFF_TP + 2 * TP_STAGE;   // per half: S (fp16) [128 rows][64]
-constexpr uint32_t OFF_XOP = OFF_SOP + 2 * 16384;     // per half: X (fp16) [64 tokens][64]
-constexpr uint32_t OFF_UOP = OFF_XOP + 2 * 8192;      // per half: U~ (fp16) [64 tokens][64]
-constexpr uint32_t OFF_AS = OFF_UOP + 2 * 8192;       // A (fp16) [64][64]
+constexpr uint32_t OFF_KQV = 0;
+constexpr uint32_t OFF_TP = OFF_KQV + kStages * STAGE_BYTES;
+constexpr uint32_t OFF_OST = OFF_TP + 2 * TP_STAGE;   // o staging for the TMA store: 2 x [64 tokens][64] bf16
+constexpr uint32_t OFF_AS = OFF_OST + 16384;          // A (fp16) [64][64]
 constexpr uint32_t OFF_PS = OFF_AS + 8192;            // P (fp16) [64][64]
 constexpr uint32_t OFF_ADIAG = OFF_PS + 8192;         // diagonal 16x16 blocks of A, fp32, rows padded to 17
 constexpr uint32_t ADIAG_BLOCK = 16 * 17;
 constexpr uint32_t OFF_GATES = OFF_ADIAG + 4608;
 constexpr uint32_t GATE_STAGE = 1536;
-constexpr uint32_t OFF_BAR = OFF_GATES + 2 * GATE_STAGE;
+constexpr uint32_t OFF_BAR = OFF_GATES + kStages * GATE_STAGE;
 constexpr uint32_t BAR_BYTES = 512;
 constexpr uint32_t SMEM_USED = OFF_BAR + BAR_BYTES;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;     // slack for aligning the base
@@ -96,26 +98,24 @@ struct Gates {
 };
 static_assert(sizeof(Gates) <= GATE_STAGE, "gate stage too small");
 
-// Barrier slots (8 bytes each) inside the OFF_BAR area.  [2] = per stage or per half.
+// Barrier slots (8 bytes each) inside the OFF_BAR area.
 enum Bar : uint32_t {
-    B_KQ_FULL = 0,     // [2] TMA landed (tx count)
-    B_KQ_CONV = 2,     // [2] K, Q converted to fp16
-    B_KQ_EMPTY = 4,    // [2] both chains' MMAs done with the K|Q stage
-    B_V_EMPTY = 6,     // [2] both chains done with the V stage
-    B_GATE_FULL = 8,   // [2]
-    B_GATE_EMPTY = 10, // [2]
-    B_TP_FULL = 12,    // [2]
-    B_TP_EMPTY = 14,   // [2]
-    B_G_FULL = 16,     // Gram in TMEM
-    B_G_EMPTY = 17,    // Gram read out
-    B_A_FULL = 18,     // [2] per half
-    B_B_FULL = 20,     // [2]
-    B_X_FULL = 22,     // [2]
-    B_U_FULL = 24,     // [2]
-    B_S_FULL = 26,     // [2]
-    B_SOP_FULL = 28,   // [2]
-    B_DRAIN = 30,      // [3] per MMA-issuing thread, drain on abort
-    B_COUNT = 33
+    B_FULL = 0,        // [3] TMA of a K/Q/V stage landed (tx count)
+    B_CONV = 3,        // [3] K, Q, V of a stage converted to fp16 (3 arrivals)
+    B_EMPTY = 6,       // [3] MMAs done with a K/Q/V stage
+    B_GATE_FULL = 9,   // [3]
+    B_GATE_EMPTY = 12, // [3] prep, chain and output epilogue done with a gate stage
+    B_TP_FULL = 15,    // [2]
+    B_TP_EMPTY = 17,   // [2]
+    B_G_FULL = 19,     // Gram in TMEM
+    B_G_EMPTY = 20,    // Gram read out
+    B_A_FULL = 21,     // MMA_A done
+    B_B_FULL = 22,     // MMA_B done
+    B_S_FULL = 23,     // MMA_C done
+    B_O_READY = 24,    // output epilogue may read its TMEM columns
+    B_O_DONE = 25,     // output epilogue has read them
+    B_DRAIN = 26,      // [2] drain on abort (chain, Gram issuer)
+    B_COUNT = 28
 };
 constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + B_COUNT * 8;        // tcgen05.alloc result
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 16;
@@ -123,19 +123,23 @@ constexpr uint32_t OFF_OKFLAG = OFF_ABORT + 16;                  // [3 groups][2
 
 // Named barriers (bar.sync ids; 0 is __syncthreads).
 constexpr int NB_PREP = 1;             // warps 4-7
-constexpr int NB_CHAIN = 2;            // + 2*h : warps of chain h (128 threads)
-constexpr int NB_LOW = 3;              // + 2*h : first two warps of chain h (64 threads)
+constexpr int NB_CHAIN = 2;            // warps 8-11
+constexpr int NB_OUT = 3;              // warps 12-15
 
-// TMEM columns (fp32 accumulators, 128 lanes each).
-constexpr uint32_t TM_G = 0;                     // Gram [K;Q] K^T, 64 columns
-constexpr uint32_t TM_A = 64;                    // + 64*h : [K;Q] S per half
-constexpr uint32_t TM_B = 192;                   // + 64*h : [T;PT] X per half
-constexpr uint32_t TM_S = 320;                   // + 64*h : state per half
+// TMEM columns (128 lanes; lane j = d_v index in the chain's regions).
+constexpr uint32_t TM_G = 0;           // Gram [K;Q] K^T (fp32, 64 columns; lane = token row)
+constexpr uint32_t TM_S = 64;          // S^T, fp32 (128 columns)
+constexpr uint32_t TM_SH = 192;        // S^T, fp16 pairs (64 columns): A operand of MMA_A
+constexpr uint32_t TM_AB = 256;        // (KQ S)^T fp32 (128 columns); later the A operands:
+constexpr uint32_t TM_Y = 256;         //   (-g K S)^T fp16 pairs (32 columns), MMA_B
+constexpr uint32_t TM_U = 288;         //   U~^T fp16 pairs (32 columns), MMA_C
+constexpr uint32_t TM_B = 384;         // ([T;PT] X)^T fp32 (128 columns)
 constexpr uint32_t TM_COLS = 512;
 
-constexpr uint32_t ID_KK = idesc_f16_f32(128, 64, 0, 0);  // A K-major, B K-major
-constexpr uint32_t ID_KM = idesc_f16_f32(128, 64, 0, 1);  // A K-major, B MN-major
-constexpr uint32_t ID_MM = idesc_f16_f32(128, 64, 1, 1);  // A MN-major, B MN-major
+constexpr uint32_t ID_GRAM = idesc_f16_f32(128, 64, 0, 0);    // A, B K-major
+constexpr uint32_t ID_TK = idesc_f16_f32(128, 128, 0, 0);     // A in TMEM, B K-major
+constexpr uint32_t ID_MK = idesc_f16_f32(128, 128, 1, 0);     // A MN-major (smem), B K-major
+constexpr uint32_t ID_TM = idesc_f16_f32(128, 128, 0, 1);     // A in TMEM, B MN-major
 
 struct Params {
     const float* alpha;    // [units_total][L]
@@ -230,7 +234,7 @@ __device__ __forceinline__ void zero_c(float (&c)[2][4])
 }
 
 // T_ij = -sum_{k=j}^{i-1} (D_i^{-1} A_ik) T_kj, with D_i^{-1} = T_ii already in TP.
-__device__ void t_block(uint32_t tp, uint32_t as, int i, int j, int lane)
+__device__ __noinline__ void t_block(uint32_t tp, uint32_t as, int i, int j, int lane)
 {
     float acc[2][4];
     zero_c(acc);
@@ -251,7 +255,7 @@ __device__ void t_block(uint32_t tp, uint32_t as, int i, int j, int lane)
 }
 
 // PT_qj = sum_{k=j}^{q} P_qk T_kj, stored in rows 64.. of TP (column j of T must be final).
-__device__ void pt_block(uint32_t tp, uint32_t ps, int q, int j, int lane)
+__device__ __noinline__ void pt_block(uint32_t tp, uint32_t ps, int q, int j, int lane)
 {
     float acc[2][4];
     zero_c(acc);
@@ -264,12 +268,6 @@ __device__ void pt_block(uint32_t tp, uint32_t ps, int q, int j, int lane)
     store_block(tp, 64 + 16 * q, 16 * j, lane, acc, 1.f);
 }
 
-__device__ __forceinline__ void st_global_v4(void* p, uint4 v)
-{
-    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};"
-                 ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
-}
-
 __device__ __forceinline__ uint4 pack8_half(const float* v)
 {
     uint4 w;
@@ -280,71 +278,42 @@ __device__ __forceinline__ uint4 pack8_half(const float* v)
     return w;
 }
 
-// Gram products [K; Q] K^T of chunk c (M=128, N=64, K=128) into TMEM, then commit.
-__device__ __forceinline__ void issue_gram(uint32_t sb, uint32_t tmem, int c)
+// Gram products [K; Q] K^T of stage s (M=128, N=64, K=128) into TMEM, then commit.
+__device__ __forceinline__ void issue_gram(uint32_t sb, uint32_t tmem, int s)
 {
-    const uint32_t kq = sb + OFF_KQ + (c & 1) * KQ_STAGE;
+    const uint32_t kq = sb + OFF_KQV + s * STAGE_BYTES;
     for (int k = 0; k < 8; ++k) {
         const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
         umma_f16(tmem + TM_G, smem_desc_sw128(kq + off, 16, 1024), smem_desc_sw128(kq + off, 16, 1024),
-                 ID_KK, k > 0);
+                 ID_GRAM, k > 0);
     }
     umma_commit(bar_addr(sb, B_G_FULL));
 }
 
-// Issues the chain MMAs of d_v half h.
-__device__ void mma_issuer(int h, uint32_t sb, uint32_t tmem, int nchunks, volatile int* abort_flag,
-                           unsigned int* err)
+// bf16 -> fp16, in place, for `n16` 16-byte vectors starting at shared address `base`.
+template <typename LdFn, typename StFn>
+__device__ __forceinline__ void convert_tile(uint32_t base, int n16, int lane, LdFn lds, StFn sts)
 {
-    auto wait = [&](uint32_t b, uint32_t par) { return mbar_wait(bar_addr(sb, b), par, abort_flag, err, kTimeoutNs); };
-    bool ok = true;
-    const uint32_t sop = sb + OFF_SOP + h * 16384;
-    const uint32_t xop = sb + OFF_XOP + h * 8192;
-    const uint32_t uop = sb + OFF_UOP + h * 8192;
-    for (int c = 0; ok && c < nchunks; ++c) {
-        const int s = c & 1;
-        const uint32_t ph = (c >> 1) & 1;
-        const uint32_t kq = sb + OFF_KQ + s * KQ_STAGE;
-        // MMA_A: [K; Q] S
-        ok = wait(B_KQ_CONV + s, ph) && wait(B_SOP_FULL + h, c & 1);
-        if (!ok) break;
-        tc_fence_after();
-        for (int k = 0; k < 8; ++k) {
-            const uint32_t aoff = (k >> 2) * 16384 + (k & 3) * 32;
-            umma_f16(tmem + TM_A + 64 * h, smem_desc_sw128(kq + aoff, 16, 1024),
-                     smem_desc_sw128(sop + k * 2048, 8192, 1024), ID_KM, k > 0);
+    for (int i0 = 0; i0 < n16; i0 += 8 * 32) {
+        uint4 w[8];
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = lds(base + static_cast<uint32_t>(i0 + i * 32 + lane) * 16u);
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            uint4 hv;
+            hv.x = pack_half2(bf16_lo(w[i].x), bf16_hi(w[i].x));
+            hv.y = pack_half2(bf16_lo(w[i].y), bf16_hi(w[i].y));
+            hv.z = pack_half2(bf16_lo(w[i].z), bf16_hi(w[i].z));
+            hv.w = pack_half2(bf16_lo(w[i].w), bf16_hi(w[i].w));
+            sts(base + static_cast<uint32_t>(i0 + i * 32 + lane) * 16u, hv);
         }
-        umma_commit(bar_addr(sb, B_A_FULL + h));
-        // MMA_B: [T; PT] X
-        ok = wait(B_TP_FULL + s, ph) && wait(B_X_FULL + h, c & 1);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t tp = sb + OFF_TP + s * TP_STAGE;
-        for (int k = 0; k < 4; ++k)
-            umma_f16(tmem + TM_B + 64 * h, smem_desc_sw128(tp + k * 32, 16, 1024),
-                     smem_desc_sw128(xop + k * 2048, 8192, 1024), ID_KM, k > 0);
-        umma_commit(bar_addr(sb, B_B_FULL + h));
-        umma_commit(bar_addr(sb, B_TP_EMPTY + s));
-        // MMA_C: S += K^T U~
-        ok = wait(B_U_FULL + h, c & 1);
-        if (!ok) break;
-        tc_fence_after();
-        for (int k = 0; k < 4; ++k)
-            umma_f16(tmem + TM_S + 64 * h, smem_desc_sw128(kq + k * 2048, 16384, 1024),
-                     smem_desc_sw128(uop + k * 2048, 8192, 1024), ID_MM, 1);
-        umma_commit(bar_addr(sb, B_S_FULL + h));
-        umma_commit(bar_addr(sb, B_KQ_EMPTY + s));
-    }
-    if (!ok) {
-        // wait for every MMA this thread issued before TMEM is released
-        umma_commit(bar_addr(sb, B_DRAIN + h));
-        mbar_wait(bar_addr(sb, B_DRAIN + h), 0, abort_flag, err, kTimeoutNs / 4);
     }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, Params p, int use_pdl)
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                      Params p, int use_pdl)
 {
     (void)use_pdl;
     allow_next_loop_to_start();
@@ -374,26 +343,25 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // ---- set-up: barriers, TMEM ----
     if (threadIdx.x == 0) {
         *abort_flag = 0;
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(bar_addr(sb, B_KQ_FULL + s), 1);
-            mbar_init(bar_addr(sb, B_KQ_CONV + s), 1);
-            mbar_init(bar_addr(sb, B_KQ_EMPTY + s), 2);
-            mbar_init(bar_addr(sb, B_V_EMPTY + s), 2);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar_addr(sb, B_FULL + s), 1);
+            mbar_init(bar_addr(sb, B_CONV + s), 3);
+            mbar_init(bar_addr(sb, B_EMPTY + s), 1);
             mbar_init(bar_addr(sb, B_GATE_FULL + s), 1);
             mbar_init(bar_addr(sb, B_GATE_EMPTY + s), 3);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(bar_addr(sb, B_TP_FULL + s), 1);
-            mbar_init(bar_addr(sb, B_TP_EMPTY + s), 2);
-            mbar_init(bar_addr(sb, B_A_FULL + s), 1);
-            mbar_init(bar_addr(sb, B_B_FULL + s), 1);
-            mbar_init(bar_addr(sb, B_X_FULL + s), 1);
-            mbar_init(bar_addr(sb, B_U_FULL + s), 1);
-            mbar_init(bar_addr(sb, B_S_FULL + s), 1);
-            mbar_init(bar_addr(sb, B_SOP_FULL + s), 1);
+            mbar_init(bar_addr(sb, B_TP_EMPTY + s), 1);
             mbar_init(bar_addr(sb, B_DRAIN + s), 1);
         }
         mbar_init(bar_addr(sb, B_G_FULL), 1);
         mbar_init(bar_addr(sb, B_G_EMPTY), 1);
-        mbar_init(bar_addr(sb, B_DRAIN + 2), 1);
+        mbar_init(bar_addr(sb, B_A_FULL), 1);
+        mbar_init(bar_addr(sb, B_B_FULL), 1);
+        mbar_init(bar_addr(sb, B_S_FULL), 1);
+        mbar_init(bar_addr(sb, B_O_READY), 1);
+        mbar_init(bar_addr(sb, B_O_DONE), 1);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -403,6 +371,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
+            prefetch_tmap(&tm_o);
         }
     }
     if (warp >= 4 && warp < 8) {
@@ -410,6 +379,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const int t = threadIdx.x - 128;
         for (uint32_t off = t * 16; off < 2 * TP_STAGE; off += 128 * 16)
             sts(sb + OFF_TP + off, make_uint4(0, 0, 0, 0));
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -421,108 +391,101 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (lane == 0) {
             int issued = 0;
             for (int c = 0; c < nchunks; ++c) {
-                const int s = c & 1;
-                const uint32_t ph = ((c >> 1) & 1) ^ 1;
-                if (!mbar_wait(bar_addr(sb, B_KQ_EMPTY + s), ph, abort_flag, err, kTimeoutNs)) break;
-                if (!mbar_wait(bar_addr(sb, B_V_EMPTY + s), ph, abort_flag, err, kTimeoutNs)) break;
-                const uint32_t fb = bar_addr(sb, B_KQ_FULL + s);
-                mbar_arrive_expect_tx(fb, KQ_STAGE + V_STAGE);
-                const uint32_t kq = sb + OFF_KQ + s * KQ_STAGE, vv = sb + OFF_V + s * V_STAGE;
+                const int s = c % kStages;
+                const uint32_t ph = ((c / kStages) & 1) ^ 1;
+                if (!mbar_wait(bar_addr(sb, B_EMPTY + s), ph, abort_flag, err, kTimeoutNs)) break;
+                const uint32_t fb = bar_addr(sb, B_FULL + s);
+                mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                const uint32_t st = sb + OFF_KQV + s * STAGE_BYTES;
                 const int32_t y = c * kC;
-                tma_load_3d(kq, &tm_k, 0, y, ug, fb);
-                tma_load_3d(kq + 16384, &tm_k, 64, y, ug, fb);
-                tma_load_3d(kq + 8192, &tm_q, 0, y, ug, fb);
-                tma_load_3d(kq + 24576, &tm_q, 64, y, ug, fb);
-                tma_load_3d(vv, &tm_v, 0, y, ug, fb);
-                tma_load_3d(vv + 8192, &tm_v, 64, y, ug, fb);
+                tma_load_3d(st, &tm_k, 0, y, ug, fb);
+                tma_load_3d(st + 16384, &tm_k, 64, y, ug, fb);
+                tma_load_3d(st + 8192, &tm_q, 0, y, ug, fb);
+                tma_load_3d(st + 24576, &tm_q, 64, y, ug, fb);
+                tma_load_3d(st + KQ_BYTES, &tm_v, 0, y, ug, fb);
+                tma_load_3d(st + KQ_BYTES + 8192, &tm_v, 64, y, ug, fb);
                 issued = c + 1;
             }
             if (*abort_flag) {
                 // let the copies already in flight land before the CTA's memory goes away
-                for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c)
-                    mbar_wait(bar_addr(sb, B_KQ_FULL + (c & 1)), (c >> 1) & 1, abort_flag, err, kTimeoutNs / 4);
+                for (int c = issued - kStages < 0 ? 0 : issued - kStages; c < issued; ++c)
+                    mbar_wait(bar_addr(sb, B_FULL + c % kStages), (c / kStages) & 1, abort_flag, err, kTimeoutNs / 4);
             }
         }
-    } else if (warp == 1 || warp == 3) {
-        // ================= MMA issuers (one thread per d_v half) =================
-        if (lane == 0) mma_issuer(warp == 1 ? 0 : 1, sb, tmem, nchunks, abort_flag, err);
-    } else if (warp == 2) {
-        // ================= gates and fp16 conversion of K, Q =================
+    } else if (warp < 4) {
+        // ================= gates (warp 1), conversion of K / Q / V (warps 1 / 2 / 3), Gram ===
         for (int c = 0; c < nchunks; ++c) {
-            const int s = c & 1;
-            const uint32_t ph = (c >> 1) & 1;
-            if (!mbar_wait(bar_addr(sb, B_GATE_EMPTY + s), ph ^ 1, abort_flag, err, kTimeoutNs)) break;
-            Gates* gs = gate(s);
-            const int64_t t0 = static_cast<int64_t>(c) * kC;
-            float g[2], b[2];
-            #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int64_t tok = t0 + lane + 32 * i;
-                const bool valid = tok < L;
-                const float a = valid ? p.alpha[ug * L + tok] : 1.f;
-                b[i] = valid ? p.beta[ug * L + tok] : 0.f;
-                g[i] = __logf(fmaxf(a, 1e-30f));
-            }
-            // inclusive prefix sums over the 64 tokens
-            #pragma unroll
-            for (int i = 0; i < 2; ++i) {
+            const int s = c % kStages;
+            const uint32_t ph = (c / kStages) & 1;
+            if (warp == 1) {
+                if (!mbar_wait(bar_addr(sb, B_GATE_EMPTY + s), ph ^ 1, abort_flag, err, kTimeoutNs)) break;
+                Gates* gs = gate(s);
+                const int64_t t0 = static_cast<int64_t>(c) * kC;
+                float g[2], b[2];
                 #pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, g[i], off);
-                    if (lane >= off) g[i] += y;
+                for (int i = 0; i < 2; ++i) {
+                    const int64_t tok = t0 + lane + 32 * i;
+                    const bool valid = tok < L;
+                    const float a = valid ? p.alpha[ug * L + tok] : 1.f;
+                    b[i] = valid ? p.beta[ug * L + tok] : 0.f;
+                    g[i] = __logf(fmaxf(a, 1e-30f));
                 }
-            }
-            g[1] += __shfl_sync(0xffffffffu, g[0], 31);
-            const float GC = __shfl_sync(0xffffffffu, g[1], 31);
-            const bool safe = GC > -80.f;
-            #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int r = lane + 32 * i;
-                gs->G[r] = g[i];
-                gs->gam[r] = __expf(g[i]);
-                gs->bein[r] = safe ? b[i] * __expf(-g[i]) : 0.f;
-                gs->beta[r] = b[i];
-                gs->bgc[r] = b[i] * __expf(GC - g[i]);
-            }
-            if (lane == 0) {
-                gs->gC = __expf(GC);
-                gs->safe = safe ? 1 : 0;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_addr(sb, B_GATE_FULL + s));
-            if (!mbar_wait(bar_addr(sb, B_KQ_FULL + s), ph, abort_flag, err, kTimeoutNs)) break;
-            const uint32_t base = sb + OFF_KQ + s * KQ_STAGE;
-            for (int i0 = 0; i0 < 64; i0 += 8) {
-                uint4 w[8];
+                // inclusive prefix sums over the 64 tokens
                 #pragma unroll
-                for (int i = 0; i < 8; ++i) w[i] = lds(base + static_cast<uint32_t>((i0 + i) * 32 + lane) * 16u);
-                #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    uint4 hv;
-                    hv.x = pack_half2(bf16_lo(w[i].x), bf16_hi(w[i].x));
-                    hv.y = pack_half2(bf16_lo(w[i].y), bf16_hi(w[i].y));
-                    hv.z = pack_half2(bf16_lo(w[i].z), bf16_hi(w[i].z));
-                    hv.w = pack_half2(bf16_lo(w[i].w), bf16_hi(w[i].w));
-                    sts(base + static_cast<uint32_t>((i0 + i) * 32 + lane) * 16u, hv);
+                for (int i = 0; i < 2; ++i) {
+                    #pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float y = __shfl_up_sync(0xffffffffu, g[i], off);
+                        if (lane >= off) g[i] += y;
+                    }
                 }
+                g[1] += __shfl_sync(0xffffffffu, g[0], 31);
+                const float GC = __shfl_sync(0xffffffffu, g[1], 31);
+                const bool safe = GC > -80.f;
+                #pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int r = lane + 32 * i;
+                    gs->G[r] = g[i];
+                    gs->gam[r] = __expf(g[i]);
+                    gs->bein[r] = safe ? b[i] * __expf(-g[i]) : 0.f;
+                    gs->beta[r] = b[i];
+                    gs->bgc[r] = b[i] * __expf(GC - g[i]);
+                }
+                if (lane == 0) {
+                    gs->gC = __expf(GC);
+                    gs->safe = safe ? 1 : 0;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_addr(sb, B_GATE_FULL + s));
+            }
+            if (!mbar_wait(bar_addr(sb, B_FULL + s), ph, abort_flag, err, kTimeoutNs)) break;
+            const uint32_t st = sb + OFF_KQV + s * STAGE_BYTES;
+            // K panels (warp 1) at +0 and +16 KB, Q panels (warp 2) at +8 and +24 KB, both V panels
+            // (warp 3) at +32 KB: one copy of the conversion loop for all three
+            #pragma unroll 1
+            for (int panel = 0; panel < 2; ++panel) {
+                const uint32_t src = warp == 3 ? st + KQ_BYTES + panel * 8192
+                                               : st + (warp - 1) * 8192 + panel * 16384;
+                convert_tile(src, 512, lane, lds, sts);
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar_addr(sb, B_KQ_CONV + s));
-                // Gram products of this chunk, as soon as its K and Q are in fp16 and the
-                // prep group has read the previous chunk's
-                if (c == 0 || mbar_wait(bar_addr(sb, B_G_EMPTY), (c - 1) & 1, abort_flag, err, kTimeoutNs)) {
+            if (lane == 0) mbar_arrive(bar_addr(sb, B_CONV + s));
+            if (warp == 1 && lane == 0) {
+                // Gram products of this chunk, once all of its tiles are in fp16 and the prep
+                // group has read the previous chunk's
+                if (mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs) &&
+                    (c == 0 || mbar_wait(bar_addr(sb, B_G_EMPTY), (c - 1) & 1, abort_flag, err, kTimeoutNs))) {
                     tc_fence_after();
-                    issue_gram(sb, tmem, c);
+                    issue_gram(sb, tmem, s);
                 }
             }
             if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
         }
-        if (lane == 0 && *abort_flag && nchunks > 0) {
+        if (warp == 1 && lane == 0 && *abort_flag && nchunks > 0) {
             // wait for the Gram MMAs this thread issued before TMEM is released
-            umma_commit(bar_addr(sb, B_DRAIN + 2));
-            mbar_wait(bar_addr(sb, B_DRAIN + 2), 0, abort_flag, err, kTimeoutNs / 4);
+            umma_commit(bar_addr(sb, B_DRAIN + 1));
+            mbar_wait(bar_addr(sb, B_DRAIN + 1), 0, abort_flag, err, kTimeoutNs / 4);
         }
     } else if (warp < 8) {
         // ================= prep: Gram epilogue, solve, P T =================
@@ -533,11 +496,11 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const uint32_t as = sb + OFF_AS, ps = sb + OFF_PS;
         float* adiag = reinterpret_cast<float*>(sbase + OFF_ADIAG);
         for (int c = 0; c < nchunks; ++c) {
-            const int s = c & 1;
-            const uint32_t ph = (c >> 1) & 1;
+            const int s = c % kStages;
+            const int tps = c & 1;
             // Gram of chunk c in TMEM, its gates, and a free [T; PT] stage
-            if (!grp.wait(bar_addr(sb, B_G_FULL), c & 1, bar_addr(sb, B_GATE_FULL + s), ph,
-                          bar_addr(sb, B_TP_EMPTY + s), ph ^ 1))
+            if (!grp.wait(bar_addr(sb, B_G_FULL), c & 1, bar_addr(sb, B_GATE_FULL + s), (c / kStages) & 1,
+                          bar_addr(sb, B_TP_EMPTY + tps), ((c >> 1) & 1) ^ 1))
                 break;
             tc_fence_after();
             const Gates* gs = gate(s);
@@ -580,7 +543,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 mbar_arrive(bar_addr(sb, B_G_EMPTY));
                 mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
             }
-            const uint32_t tp = sb + OFF_TP + s * TP_STAGE;
+            const uint32_t tp = sb + OFF_TP + tps * TP_STAGE;
             if (is_a) {
                 // row r of D_b^{-1} = (I + A_bb)^{-1} by the column recurrence within the block
                 const int b = r >> 4, i = r & 15;
@@ -611,172 +574,229 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             pt_block(tp, ps, 3 - q, 0, lane);                   // PT_30, PT_20, PT_10, PT_00
             fence_proxy_async_smem();
             grp.sync();
-            if (t == 0) mbar_arrive(bar_addr(sb, B_TP_FULL + s));
+            if (t == 0) mbar_arrive(bar_addr(sb, B_TP_FULL + tps));
         }
-    } else {
-        // ================= chain of one d_v half =================
-        const int h = (warp - 8) >> 2;              // 0: columns 0-63, 1: columns 64-127
-        const int t = (threadIdx.x - 256) & 127;    // 0..127 = TMEM lane
+    } else if (warp < 12) {
+        // ================= the S-dependent chain (lane j = d_v column j of S) =================
+        const int j = threadIdx.x - 256;            // 0..127 = TMEM lane = d_v index
         const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-        const uint32_t tA = tmem + TM_A + 64 * h + lane_addr;
-        const uint32_t tB = tmem + TM_B + 64 * h + lane_addr;
-        const uint32_t tS = tmem + TM_S + 64 * h + lane_addr;
-        const uint32_t sop = sb + OFF_SOP + h * 16384;
-        const uint32_t xop = sb + OFF_XOP + h * 8192;
-        const uint32_t uop = sb + OFF_UOP + h * 8192;
-        const int nb_low = NB_LOW + 2 * h;
-        Group grp{NB_CHAIN + 2 * h, 128, t == 0, okflags + 2 + 2 * h, 0, abort_flag, err};
+        const bool leader = j == 0;
+        Group grp{NB_CHAIN, 128, leader, okflags + 2, 0, abort_flag, err};
         bool ok = nchunks > 0;
-        // initial state: S0 (fp32 master in TMEM pre-scaled by the first chunk's decay,
-        // fp16 copy in shared memory)
+        // initial state: S0^T (fp32 in TMEM, pre-scaled by the first chunk's decay; fp16 copy)
         if (ok) ok = grp.wait(bar_addr(sb, B_GATE_FULL + 0), 0);
         if (ok) {
             const float g0 = gate(0)->gC;
-            const float* s0row = p.S0 ? p.S0 + (static_cast<int64_t>(ug) * kD + t) * kD + 64 * h : nullptr;
+            const float* s0 = p.S0 ? p.S0 + static_cast<int64_t>(ug) * kD * kD + j : nullptr;
             #pragma unroll
-            for (int piece = 0; piece < 2; ++piece) {
+            for (int piece = 0; piece < 4; ++piece) {
                 float v[32];
                 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    float4 f = s0row ? *reinterpret_cast<const float4*>(s0row + 32 * piece + j)
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
-                    v[j] = f.x; v[j + 1] = f.y; v[j + 2] = f.z; v[j + 3] = f.w;
-                }
+                for (int d = 0; d < 32; ++d) v[d] = s0 ? s0[(32 * piece + d) * kD] : 0.f;
+                uint32_t hpk[16];
                 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) sts(sw128(sop, t, 4 * piece + ch), pack8_half(v + 8 * ch));
+                for (int e = 0; e < 16; ++e) hpk[e] = pack_half2(v[2 * e], v[2 * e + 1]);
+                tmem_st16(tmem + TM_SH + lane_addr + 16 * piece, hpk);
                 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] *= g0;
-                tmem_st32(tS + 32 * piece, v);
+                for (int d = 0; d < 32; ++d) v[d] *= g0;
+                tmem_st32(tmem + TM_S + lane_addr + 32 * piece, v);
             }
             tmem_wait_st();
             tc_fence_before();
-            fence_proxy_async_smem();
-            grp.sync();
-            if (t == 0) mbar_arrive(bar_addr(sb, B_SOP_FULL + h));
         }
+        uint32_t drain_needed = 0;
         for (int c = 0; ok && c < nchunks; ++c) {
-            const int s = c & 1;
-            const uint32_t ph = (c >> 1) & 1;
-            const int64_t t0 = static_cast<int64_t>(c) * kC;
+            const int s = c % kStages;
+            const uint32_t ph = (c / kStages) & 1;
             const Gates* gs = gate(s);
-            // --- step 1: X = V - g (K S), by the first 64 threads (token rows) ---
-            ok = grp.wait(bar_addr(sb, B_A_FULL + h), c & 1, bar_addr(sb, B_KQ_FULL + s), ph);
-            if (!ok) break;
-            tc_fence_after();
-            if (t < 64) {
-                const float g = gs->gam[t];
-                const uint32_t vt = sb + OFF_V + s * V_STAGE + h * 8192;
-                uint4 vw[8];
-                #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) vw[ch] = lds(sw128(vt, t, ch));
-                float ks[64];
-                tmem_load_2x32(tA, tA + 32, ks);
-                #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const uint4 w = vw[ch];
-                    const float* kc = ks + 8 * ch;
-                    float x[8] = {bf16_lo(w.x) - g * kc[0], bf16_hi(w.x) - g * kc[1],
-                                  bf16_lo(w.y) - g * kc[2], bf16_hi(w.y) - g * kc[3],
-                                  bf16_lo(w.z) - g * kc[4], bf16_hi(w.z) - g * kc[5],
-                                  bf16_lo(w.w) - g * kc[6], bf16_hi(w.w) - g * kc[7]};
-                    sts(sw128(xop, t, ch), pack8_half(x));
-                }
-                fence_proxy_async_smem();
-                named_sync(nb_low, 64);
-                if (t == 0) {
-                    mbar_arrive(bar_addr(sb, B_X_FULL + h));
-                    mbar_arrive(bar_addr(sb, B_V_EMPTY + s));
+            const uint32_t st = sb + OFF_KQV + s * STAGE_BYTES;
+            // --- MMA_A: (KQ S)^T = S^T [K;Q]^T ---
+            grp.sync();
+            if (leader) {
+                bool lok = mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs) &&
+                           (c == 0 || mbar_wait(bar_addr(sb, B_O_DONE), (c - 1) & 1, abort_flag, err, kTimeoutNs));
+                if (lok) {
+                    tc_fence_after();
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t boff = (k >> 2) * 16384 + (k & 3) * 32;
+                        umma_f16_tmem_a(tmem + TM_AB, tmem + TM_SH + 8 * k, smem_desc_sw128(st + boff, 16, 1024),
+                                        ID_TK, k > 0);
+                    }
+                    umma_commit(bar_addr(sb, B_A_FULL));
+                    drain_needed = 1;
                 }
             }
-            // --- step 2: U~ for the state update (first 64 threads); o = g (Q S) + P T X ---
-            ok = grp.wait(bar_addr(sb, B_B_FULL + h), c & 1);
+            ok = grp.wait(bar_addr(sb, B_A_FULL), c & 1);
             if (!ok) break;
             tc_fence_after();
-            if (t < 64) {
-                const float bg = gs->bgc[t];
-                float u[64];
-                tmem_load_2x32(tB, tB + 32, u);
+            // --- Y^T = -g (K S)^T, fp16, into TMEM as the second A operand of MMA_B ---
+            {
+                float ks[64];
+                tmem_load_2x32(tmem + TM_AB + lane_addr, tmem + TM_AB + lane_addr + 32, ks);
+                uint32_t hpk[32];
                 #pragma unroll
-                for (int j = 0; j < 64; ++j) u[j] *= bg;
-                #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) sts(sw128(uop, t, ch), pack8_half(u + 8 * ch));
-                fence_proxy_async_smem();
-                named_sync(nb_low, 64);
-                if (t == 0) mbar_arrive(bar_addr(sb, B_U_FULL + h));
-            } else {
-                const int r = t - 64;
-                const int64_t tok = t0 + r;
-                const float g = gs->gam[r];
-                #pragma unroll
-                for (int piece = 0; piece < 2; ++piece) {
-                    float qp[64];
-                    tmem_load_2x32(tA + 32 * piece, tB + 32 * piece, qp);
-                    const float* qs = qp;
-                    const float* pu = qp + 32;
-                    if (tok < L) {
-                        const int64_t col = static_cast<int64_t>(ug) * L * kD + tok * kD + 64 * h + 32 * piece;
-                        if (p.out_bf16) {
-                            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + col;
-                            #pragma unroll
-                            for (int ch = 0; ch < 4; ++ch) {
-                                uint32_t wv[4];
-                                #pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const int j = 8 * ch + 2 * e;
-                                    __nv_bfloat162 b2 = __floats2bfloat162_rn(g * qs[j] + pu[j], g * qs[j + 1] + pu[j + 1]);
-                                    wv[e] = *reinterpret_cast<uint32_t*>(&b2);
-                                }
-                                st_global_v4(orow + 8 * ch, make_uint4(wv[0], wv[1], wv[2], wv[3]));
-                            }
-                        } else {
-                            float* orow = static_cast<float*>(p.o) + col;
-                            #pragma unroll
-                            for (int ch = 0; ch < 8; ++ch) {
-                                const int j = 4 * ch;
-                                st_global_v4(orow + j, make_uint4(__float_as_uint(g * qs[j] + pu[j]),
-                                                                  __float_as_uint(g * qs[j + 1] + pu[j + 1]),
-                                                                  __float_as_uint(g * qs[j + 2] + pu[j + 2]),
-                                                                  __float_as_uint(g * qs[j + 3] + pu[j + 3])));
-                            }
-                        }
-                    }
+                for (int e4 = 0; e4 < 64; e4 += 4) {
+                    const float4 g4 = *reinterpret_cast<const float4*>(&gs->gam[e4]);
+                    hpk[e4 / 2] = pack_half2(-g4.x * ks[e4], -g4.y * ks[e4 + 1]);
+                    hpk[e4 / 2 + 1] = pack_half2(-g4.z * ks[e4 + 2], -g4.w * ks[e4 + 3]);
                 }
+                tmem_st16(tmem + TM_Y + lane_addr, *reinterpret_cast<uint32_t(*)[16]>(hpk));
+                tmem_st16(tmem + TM_Y + lane_addr + 16, *reinterpret_cast<uint32_t(*)[16]>(hpk + 16));
+                tmem_wait_st();
             }
             tc_fence_before();
-            // --- step 3: the new state ---
-            const bool last = c + 1 == nchunks;
-            const int s1 = (c + 1) & 1;
-            ok = last ? grp.wait(bar_addr(sb, B_S_FULL + h), c & 1)
-                      : grp.wait(bar_addr(sb, B_S_FULL + h), c & 1, bar_addr(sb, B_GATE_FULL + s1),
-                                 ((c + 1) >> 1) & 1);
+            grp.sync();
+            // --- MMA_B: ([T;PT] X)^T = V^T [T;PT]^T + Y^T [T;PT]^T ---
+            if (leader) {
+                const int tps = c & 1;
+                if (mbar_wait(bar_addr(sb, B_TP_FULL + tps), (c >> 1) & 1, abort_flag, err, kTimeoutNs)) {
+                    tc_fence_after();
+                    const uint32_t tp = sb + OFF_TP + tps * TP_STAGE;
+                    const uint32_t vt = st + KQ_BYTES;
+                    for (int k = 0; k < 4; ++k)
+                        umma_f16(tmem + TM_B, smem_desc_sw128(vt + k * 2048, 8192, 1024),
+                                 smem_desc_sw128(tp + k * 32, 16, 1024), ID_MK, k > 0);
+                    for (int k = 0; k < 4; ++k)
+                        umma_f16_tmem_a(tmem + TM_B, tmem + TM_Y + 8 * k, smem_desc_sw128(tp + k * 32, 16, 1024),
+                                        ID_TK, 1);
+                    umma_commit(bar_addr(sb, B_B_FULL));
+                    umma_commit(bar_addr(sb, B_TP_EMPTY + tps));
+                }
+            }
+            ok = grp.wait(bar_addr(sb, B_B_FULL), c & 1);
             if (!ok) break;
             tc_fence_after();
-            if (t == 0) mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));   // gates of chunk c consumed
-            float v[64];
-            tmem_load_2x32(tS, tS + 32, v);
+            if (leader) mbar_arrive(bar_addr(sb, B_O_READY));
+            // --- U~^T = diag(beta e^{G_63 - G}) U^T, fp16, into TMEM for MMA_C ---
+            {
+                float u[64];
+                tmem_load_2x32(tmem + TM_B + lane_addr, tmem + TM_B + lane_addr + 32, u);
+                uint32_t hpk[32];
+                #pragma unroll
+                for (int e4 = 0; e4 < 64; e4 += 4) {
+                    const float4 b4 = *reinterpret_cast<const float4*>(&gs->bgc[e4]);
+                    hpk[e4 / 2] = pack_half2(b4.x * u[e4], b4.y * u[e4 + 1]);
+                    hpk[e4 / 2 + 1] = pack_half2(b4.z * u[e4 + 2], b4.w * u[e4 + 3]);
+                }
+                tmem_st16(tmem + TM_U + lane_addr, *reinterpret_cast<uint32_t(*)[16]>(hpk));
+                tmem_st16(tmem + TM_U + lane_addr + 16, *reinterpret_cast<uint32_t(*)[16]>(hpk + 16));
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            grp.sync();
+            // --- MMA_C: S^T += U~^T K ---
+            if (leader) {
+                tc_fence_after();
+                for (int k = 0; k < 4; ++k)
+                    umma_f16_tmem_a(tmem + TM_S, tmem + TM_U + 8 * k, smem_desc_sw128(st + k * 2048, 16384, 1024),
+                                    ID_TM, 1);
+                umma_commit(bar_addr(sb, B_S_FULL));
+                umma_commit(bar_addr(sb, B_EMPTY + s));
+                mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));     // gates of chunk c consumed
+            }
+            // --- the new state ---
+            const bool last = c + 1 == nchunks;
+            const int s1 = (c + 1) % kStages;
+            ok = last ? grp.wait(bar_addr(sb, B_S_FULL), c & 1)
+                      : grp.wait(bar_addr(sb, B_S_FULL), c & 1, bar_addr(sb, B_GATE_FULL + s1),
+                                 ((c + 1) / kStages) & 1);
+            if (!ok) break;
+            tc_fence_after();
             if (last) {
                 if (p.S_out) {
-                    float* so = p.S_out + (static_cast<int64_t>(ug) * kD + t) * kD + 64 * h;
+                    float* so = p.S_out + static_cast<int64_t>(ug) * kD * kD + j;
                     #pragma unroll
-                    for (int j = 0; j < 64; j += 4)
-                        st_global_v4(so + j, make_uint4(__float_as_uint(v[j]), __float_as_uint(v[j + 1]),
-                                                        __float_as_uint(v[j + 2]), __float_as_uint(v[j + 3])));
+                    for (int piece = 0; piece < 4; piece += 2) {
+                        float v[64];
+                        tmem_load_2x32(tmem + TM_S + lane_addr + 32 * piece, tmem + TM_S + lane_addr + 32 * piece + 32, v);
+                        #pragma unroll
+                        for (int d = 0; d < 64; ++d) so[(32 * piece + d) * kD] = v[d];
+                    }
                 }
+                drain_needed = 0;
             } else {
                 const float gn = gate(s1)->gC;
-                #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) sts(sw128(sop, t, ch), pack8_half(v + 8 * ch));
-                #pragma unroll
-                for (int j = 0; j < 64; ++j) v[j] *= gn;
-                tmem_st32(tS, *reinterpret_cast<float(*)[32]>(v));
-                tmem_st32(tS + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                #pragma unroll 1
+                for (int piece = 0; piece < 4; piece += 2) {
+                    float v[64];
+                    tmem_load_2x32(tmem + TM_S + lane_addr + 32 * piece, tmem + TM_S + lane_addr + 32 * piece + 32, v);
+                    uint32_t hpk[32];
+                    #pragma unroll
+                    for (int e = 0; e < 32; ++e) hpk[e] = pack_half2(v[2 * e], v[2 * e + 1]);
+                    tmem_st16(tmem + TM_SH + lane_addr + 16 * piece, *reinterpret_cast<uint32_t(*)[16]>(hpk));
+                    tmem_st16(tmem + TM_SH + lane_addr + 16 * piece + 16, *reinterpret_cast<uint32_t(*)[16]>(hpk + 16));
+                    #pragma unroll
+                    for (int d = 0; d < 64; ++d) v[d] *= gn;
+                    tmem_st32(tmem + TM_S + lane_addr + 32 * piece, *reinterpret_cast<float(*)[32]>(v));
+                    tmem_st32(tmem + TM_S + lane_addr + 32 * piece + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                }
                 tmem_wait_st();
                 tc_fence_before();
-                fence_proxy_async_smem();
-                grp.sync();
-                if (t == 0) mbar_arrive(bar_addr(sb, B_SOP_FULL + h));
             }
         }
+        if (leader && drain_needed && !ok) {
+            // wait for every MMA this thread issued before TMEM is released
+            umma_commit(bar_addr(sb, B_DRAIN + 0));
+            mbar_wait(bar_addr(sb, B_DRAIN + 0), 0, abort_flag, err, kTimeoutNs / 4);
+        }
+    } else {
+        // ================= output epilogue: o = g (Q S) + P T X =================
+        const int j = threadIdx.x - 384;            // TMEM lane = d_v index
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+        Group grp{NB_OUT, 128, j == 0, okflags + 4, 0, abort_flag, err};
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % kStages;
+            if (!grp.wait(bar_addr(sb, B_O_READY), c & 1)) break;
+            tc_fence_after();
+            const Gates* gs = gate(s);
+            const int64_t t0 = static_cast<int64_t>(c) * kC;
+            const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
+            const int64_t base = (static_cast<int64_t>(ug) * L + t0) * kD + j;
+            float res[64];                           // o[r][j] for the chunk's 64 tokens
+            #pragma unroll
+            for (int piece = 0; piece < 2; ++piece) {
+                float qp[64];                        // (Q S)^T, then (P T X)^T, for 32 tokens
+                tmem_load_2x32(tmem + TM_AB + lane_addr + 64 + 32 * piece,
+                               tmem + TM_B + lane_addr + 64 + 32 * piece, qp);
+                #pragma unroll
+                for (int e4 = 0; e4 < 32; e4 += 4) {
+                    const float4 g4 = *reinterpret_cast<const float4*>(&gs->gam[32 * piece + e4]);
+                    res[32 * piece + e4 + 0] = g4.x * qp[e4 + 0] + qp[32 + e4 + 0];
+                    res[32 * piece + e4 + 1] = g4.y * qp[e4 + 1] + qp[32 + e4 + 1];
+                    res[32 * piece + e4 + 2] = g4.z * qp[e4 + 2] + qp[32 + e4 + 2];
+                    res[32 * piece + e4 + 3] = g4.w * qp[e4 + 3] + qp[32 + e4 + 3];
+                }
+            }
+            // the TMEM columns are free for the next chunk's MMAs before the stores go out
+            tc_fence_before();
+            if (p.out_bf16 && j == 0) bulk_wait_read_all();   // staging tile free again
+            grp.sync();
+            if (j == 0) {
+                mbar_arrive(bar_addr(sb, B_O_DONE));
+                mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
+            }
+            if (p.out_bf16) {
+                // transpose through shared memory (a warp writes 64 contiguous bytes per token)
+                // and let the TMA unit write the 64 x 128 tile; rows past L are clipped
+                uint8_t* ost = sbase + OFF_OST + (j >> 6) * 8192 + (j & 63) * 2;
+                #pragma unroll
+                for (int r = 0; r < 64; ++r)
+                    *reinterpret_cast<__nv_bfloat16*>(ost + r * 128) = __float2bfloat16_rn(res[r]);
+                fence_proxy_async_smem();
+                grp.sync();
+                if (j == 0) {
+                    tma_store_3d(&tm_o, sb + OFF_OST, 0, static_cast<int32_t>(t0), ug);
+                    tma_store_3d(&tm_o, sb + OFF_OST + 8192, 64, static_cast<int32_t>(t0), ug);
+                    bulk_commit_group();
+                }
+            } else {
+                float* o = static_cast<float*>(p.o) + base;
+                #pragma unroll
+                for (int r = 0; r < 64; ++r)
+                    if (r < n) o[r * kD] = res[r];
+            }
+        }
+        if (j == 0) bulk_wait_all();     // every output tile written before the CTA exits
     }
 
     tc_fence_before();
@@ -807,7 +827,8 @@ static EncodeTiledFn encode_fn()
 
 // 3-D view [units][L][128] of a bf16 tensor, boxes of 64 columns x 64 tokens x 1 unit,
 // 128-byte swizzle.  Rows past a unit's L are filled with zeros by the TMA unit.
-static bool make_map(CUtensorMap* m, const void* base, int64_t units, int64_t L)
+static bool make_map(CUtensorMap* m, const void* base, int64_t units, int64_t L,
+                     CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
@@ -817,7 +838,7 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t units, int64_t L)
     const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kC), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -833,9 +854,12 @@ cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
     using namespace tc;
     if (call.units_per_loop == 0 || call.T == 0) return cudaSuccess;
     const int64_t units = call.T * call.units_per_loop;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, call.q, units, call.L) || !make_map(&mk, call.k, units, call.L) ||
         !make_map(&mv, call.v, units, call.L))
+        return cudaErrorInvalidValue;
+    // o (bf16 output only): plain row-major tile, written by the TMA store from shared memory
+    if (call.out_bf16 && !make_map(&mo, call.o, units, call.L, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(gdr_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM_BYTES));
@@ -862,7 +886,7 @@ cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         const int use_pdl = tau > 0 ? 1 : 0;
-        e = cudaLaunchKernelEx(&cfg, gdr_prefill_tc_kernel, mq, mk, mv, p, use_pdl);
+        e = cudaLaunchKernelEx(&cfg, gdr_prefill_tc_kernel, mq, mk, mv, call.out_bf16 ? mo : mv, p, use_pdl);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
