@@ -233,39 +233,57 @@ __device__ __forceinline__ void zero_c(float (&c)[2][4])
         for (int j = 0; j < 4; ++j) c[i][j] = 0.f;
 }
 
-// T_ij = -sum_{k=j}^{i-1} (D_i^{-1} A_ik) T_kj, with D_i^{-1} = T_ii already in TP.
-__device__ __noinline__ void t_block(uint32_t tp, uint32_t as, int i, int j, int lane)
+// Zeroes the entries above the diagonal of a diagonal 16x16 block held as an m16n8k16 A
+// fragment (a0: row g, columns 2tq..2tq+1; a1: row g+8, same columns; a2/a3: columns +8).
+__device__ __forceinline__ void keep_lower(uint32_t (&a)[4], int lane)
 {
-    float acc[2][4];
-    zero_c(acc);
-    uint32_t dinv[4];
-    frag_a(tp, 16 * i, 16 * i, lane, dinv);
-    for (int k = j; k < i; ++k) {
-        uint32_t b[4];
-        frag_b(as, 16 * i, 16 * k, lane, b);
-        float n[2][4];
-        zero_c(n);
-        mma_block(n, dinv, b);           // N_ik = D_i^{-1} A_ik
-        uint32_t na[4];
-        c_to_a(n, na);
-        frag_b(tp, 16 * k, 16 * j, lane, b);
-        mma_block(acc, na, b);           // += N_ik T_kj
-    }
-    store_block(tp, 16 * i, 16 * j, lane, acc, -1.f);
+    const int g = lane >> 2, c0 = 2 * (lane & 3);
+    const uint32_t m = (c0 + 1 <= g) ? 0xffffffffu : ((c0 <= g) ? 0x0000ffffu : 0u);
+    a[0] &= m;
+    a[2] = 0u;
+    a[3] &= m;
 }
 
-// PT_qj = sum_{k=j}^{q} P_qk T_kj, stored in rows 64.. of TP (column j of T must be final).
-__device__ __noinline__ void pt_block(uint32_t tp, uint32_t ps, int q, int j, int lane)
+// One 16-row block `rb` of X = [T; PT] (T = (I + A)^{-1}, rows 0..63; PT, rows 64..127).
+// X solves X (I + A) = [I; P]; with A strictly lower triangular this is a back substitution
+// over the 16-column blocks j = 3, 2, 1, 0:
+//     X_j = (E_j + sum_{k>j} X_k (-A)_{kj}) D_j,      D_j = (I + A_jj)^{-1}  (already in TP)
+// where E = I for the T rows and E = P for the PT rows, and X_j = 0 right of the diagonal
+// block (T_jj = D_j itself).  AS holds -A.  Each X_j goes to TP as soon as it is known and is
+// read back from there by the warp's later steps, so both loops stay rolled.
+__device__ __noinline__ void solve_row_block(uint32_t tp, uint32_t as, uint32_t ps, int rb, int lane)
 {
-    float acc[2][4];
-    zero_c(acc);
-    for (int k = j; k <= q; ++k) {
-        uint32_t a[4], b[4];
-        frag_a(ps, 16 * q, 16 * k, lane, a);
-        frag_b(tp, 16 * k, 16 * j, lane, b);
-        mma_block(acc, a, b);
+    const bool is_t = rb < 4;
+    const int qd = is_t ? rb : rb - 4;          // diagonal column block of this row block
+    #pragma unroll 1
+    for (int j = is_t ? qd - 1 : qd; j >= 0; --j) {
+        float acc[2][4];
+        zero_c(acc);
+        #pragma unroll 1
+        for (int k = j + 1; k <= qd; ++k) {
+            uint32_t xa[4], b[4];
+            frag_a(tp, 16 * rb, 16 * k, lane, xa);
+            frag_b(as, 16 * k, 16 * j, lane, b);
+            mma_block(acc, xa, b);              // += X_k (-A)_kj
+        }
+        uint32_t dj[4];
+        frag_b(tp, 16 * j, 16 * j, lane, dj);
+        float x[2][4];
+        zero_c(x);
+        if (!is_t) {
+            uint32_t pa[4];
+            frag_a(ps, 16 * qd, 16 * j, lane, pa);
+            if (j == qd) keep_lower(pa, lane);
+            mma_block(x, pa, dj);               // P_qj D_j
+        }
+        if (j < qd) {
+            uint32_t aa[4];
+            c_to_a(acc, aa);
+            mma_block(x, aa, dj);
+        }
+        store_block(tp, 16 * rb, 16 * j, lane, x, 1.f);
+        __syncwarp();                           // X_j is read back by this warp's next steps
     }
-    store_block(tp, 64 + 16 * q, 16 * j, lane, acc, 1.f);
 }
 
 __device__ __forceinline__ uint4 pack8_half(const float* v)
@@ -307,6 +325,81 @@ __device__ __forceinline__ void convert_tile(uint32_t base, int n16, int lane, L
             hv.w = pack_half2(bf16_lo(w[i].w), bf16_hi(w[i].w));
             sts(base + static_cast<uint32_t>(i0 + i * 32 + lane) * 16u, hv);
         }
+    }
+}
+
+// ---- cold paths, kept out of line so that the per-chunk code stays compact ----------------
+
+// Chain thread j: S0^T row j (column j of S0, or zeros) into TMEM, as fp16 pairs for MMA_A and
+// as fp32 pre-scaled by the first chunk's decay g0.
+__device__ __noinline__ void load_initial_state(uint32_t tm_s, uint32_t tm_sh, const float* s0, float g0)
+{
+    #pragma unroll 1
+    for (int piece = 0; piece < 4; ++piece) {
+        float v[32];
+        #pragma unroll
+        for (int d = 0; d < 32; ++d) v[d] = s0 ? s0[(32 * piece + d) * kD] : 0.f;
+        uint32_t hpk[16];
+        #pragma unroll
+        for (int e = 0; e < 16; ++e) hpk[e] = pack_half2(v[2 * e], v[2 * e + 1]);
+        tmem_st16(tm_sh + 16 * piece, hpk);
+        #pragma unroll
+        for (int d = 0; d < 32; ++d) v[d] *= g0;
+        tmem_st32(tm_s + 32 * piece, v);
+    }
+    tmem_wait_st();
+}
+
+// Chain thread j: column j of the final state (row j of S^T in TMEM) to S_out.
+__device__ __noinline__ void store_final_state(uint32_t tm_s, float* so)
+{
+    #pragma unroll 1
+    for (int piece = 0; piece < 4; piece += 2) {
+        float v[64];
+        tmem_load_2x32(tm_s + 32 * piece, tm_s + 32 * piece + 32, v);
+        #pragma unroll
+        for (int d = 0; d < 64; ++d) so[(32 * piece + d) * kD] = v[d];
+    }
+}
+
+// Output thread j, fp32 output: o[r][j] = g_r (Q S)_rj + (P T X)_rj for the chunk's n tokens.
+__device__ __noinline__ void store_o_f32(uint32_t tm_qs, uint32_t tm_ptx, const float* gam, float* o, int n)
+{
+    #pragma unroll 1
+    for (int piece = 0; piece < 2; ++piece) {
+        float qp[64];
+        tmem_load_2x32(tm_qs + 32 * piece, tm_ptx + 32 * piece, qp);
+        #pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int r = 32 * piece + e;
+            if (r < n) o[r * kD] = gam[r] * qp[e] + qp[32 + e];
+        }
+    }
+}
+
+// Prep thread t, chunks whose decay e^{-G} is not representable: row r of -A (t < 64) or of P
+// with the unfactored e^{G_r - G_s}, masked to s < r (A) or s <= r (P), 8 columns at a time,
+// to the fp16 tile `dst` and (A rows) the fp32 diagonal-block copy.
+__device__ __noinline__ void gram_epilogue_unfactored(uint32_t tm_row, const Gates* gs, int r, bool is_a,
+                                                      uint8_t* dst_ptr, uint32_t dst, float* adiag_row)
+{
+    const int lim = is_a ? r : r + 1;
+    const float sg = is_a ? -1.f : 1.f;
+    const float Gr = gs->G[r];
+    #pragma unroll 1
+    for (int ch = 0; ch < 8; ++ch) {
+        float v[8];
+        tmem_load8(tm_row + 8 * ch, v);
+        #pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int sc = 8 * ch + e;
+            v[e] = (sc < lim) ? sg * gs->beta[sc] * __expf(Gr - gs->G[sc]) * v[e] : 0.f;
+        }
+        if (is_a && (ch >> 1) == (r >> 4)) {
+            #pragma unroll
+            for (int e = 0; e < 8; ++e) adiag_row[(ch & 1) * 8 + e] = v[e];
+        }
+        *reinterpret_cast<uint4*>(dst_ptr + (sw128(dst, r, ch) - dst)) = pack8_half(v);
     }
 }
 
@@ -388,12 +481,15 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
     if (warp == 0) {
         // ================= TMA producer =================
-        if (lane == 0) {
-            int issued = 0;
-            for (int c = 0; c < nchunks; ++c) {
-                const int s = c % kStages;
-                const uint32_t ph = ((c / kStages) & 1) ^ 1;
-                if (!mbar_wait(bar_addr(sb, B_EMPTY + s), ph, abort_flag, err, kTimeoutNs)) break;
+        int issued = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % kStages;
+            const uint32_t ph = ((c / kStages) & 1) ^ 1;
+            int free_ok = 0;
+            if (lane == 0) free_ok = mbar_wait(bar_addr(sb, B_EMPTY + s), ph, abort_flag, err, kTimeoutNs);
+            if (!__shfl_sync(0xffffffffu, free_ok, 0)) break;
+            uint32_t leader;
+            if (elect_one(leader)) {
                 const uint32_t fb = bar_addr(sb, B_FULL + s);
                 mbar_arrive_expect_tx(fb, STAGE_BYTES);
                 const uint32_t st = sb + OFF_KQV + s * STAGE_BYTES;
@@ -404,16 +500,19 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 tma_load_3d(st + 24576, &tm_q, 64, y, ug, fb);
                 tma_load_3d(st + KQ_BYTES, &tm_v, 0, y, ug, fb);
                 tma_load_3d(st + KQ_BYTES + 8192, &tm_v, 64, y, ug, fb);
-                issued = c + 1;
             }
-            if (*abort_flag) {
-                // let the copies already in flight land before the CTA's memory goes away
-                for (int c = issued - kStages < 0 ? 0 : issued - kStages; c < issued; ++c)
-                    mbar_wait(bar_addr(sb, B_FULL + c % kStages), (c / kStages) & 1, abort_flag, err, kTimeoutNs / 4);
-            }
+            __syncwarp();
+            issued = c + 1;
+        }
+        if (lane == 0 && *abort_flag) {
+            // let the copies already in flight land before the CTA's memory goes away
+            for (int c = issued - kStages < 0 ? 0 : issued - kStages; c < issued; ++c)
+                mbar_wait(bar_addr(sb, B_FULL + c % kStages), (c / kStages) & 1, abort_flag, err, kTimeoutNs / 4);
         }
     } else if (warp < 4) {
         // ================= gates (warp 1), conversion of K / Q / V (warps 1 / 2 / 3), Gram ===
+        uint32_t gram_issuer = 0;
+        int gram_issued = 0;
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;
             const uint32_t ph = (c / kStages) & 1;
@@ -471,18 +570,23 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_addr(sb, B_CONV + s));
-            if (warp == 1 && lane == 0) {
+            if (warp == 1) {
                 // Gram products of this chunk, once all of its tiles are in fp16 and the prep
                 // group has read the previous chunk's
-                if (mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs) &&
-                    (c == 0 || mbar_wait(bar_addr(sb, B_G_EMPTY), (c - 1) & 1, abort_flag, err, kTimeoutNs))) {
+                int gram_ok = 0;
+                if (lane == 0)
+                    gram_ok = mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs) &&
+                              (c == 0 || mbar_wait(bar_addr(sb, B_G_EMPTY), (c - 1) & 1, abort_flag, err, kTimeoutNs));
+                if (__shfl_sync(0xffffffffu, gram_ok, 0)) {
                     tc_fence_after();
-                    issue_gram(sb, tmem, s);
+                    if (elect_one(gram_issuer)) issue_gram(sb, tmem, s);
+                    __syncwarp();
+                    gram_issued = 1;
                 }
             }
             if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
         }
-        if (warp == 1 && lane == 0 && *abort_flag && nchunks > 0) {
+        if (warp == 1 && lane == gram_issuer && gram_issued && *abort_flag) {
             // wait for the Gram MMAs this thread issued before TMEM is released
             umma_commit(bar_addr(sb, B_DRAIN + 1));
             mbar_wait(bar_addr(sb, B_DRAIN + 1), 0, abort_flag, err, kTimeoutNs / 4);
@@ -506,37 +610,42 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const Gates* gs = gate(s);
             const int r = t & 63;
             const bool is_a = t < 64;               // rows of K K^T (A) or Q K^T (P)
-            const float Gr = gs->G[r], gr = gs->gam[r];
+            const float gr = gs->gam[r];
             const bool safe = gs->safe != 0;
             const uint32_t dst = is_a ? as : ps;
-            float v[64];
-            tmem_load_2x32(tmem + TM_G + lane_addr, tmem + TM_G + lane_addr + 32, v);
-            const int lim = is_a ? r : r + 1;         // keep columns s < lim
             if (safe) {
-                #pragma unroll
-                for (int j4 = 0; j4 < 64; j4 += 4) {
-                    const float4 be = *reinterpret_cast<const float4*>(&gs->bein[j4]);
-                    v[j4 + 0] = (j4 + 0 < lim) ? gr * be.x * v[j4 + 0] : 0.f;
-                    v[j4 + 1] = (j4 + 1 < lim) ? gr * be.y * v[j4 + 1] : 0.f;
-                    v[j4 + 2] = (j4 + 2 < lim) ? gr * be.z * v[j4 + 2] : 0.f;
-                    v[j4 + 3] = (j4 + 3 < lim) ? gr * be.w * v[j4 + 3] : 0.f;
+                // A is kept negated (the solve only accumulates).  Entries on or above the
+                // diagonal (s >= r in A, s > r in P) are never read, apart from the diagonal P
+                // block, which the solve masks in registers, so no mask is applied here.
+                const float sg = is_a ? -gr : gr;
+                #pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    float v[32];
+                    tmem_load32(tmem + TM_G + lane_addr + 32 * h, v);
+                    const float* be = gs->bein + 32 * h;
+                    #pragma unroll
+                    for (int j4 = 0; j4 < 32; j4 += 4) {
+                        const float4 b4 = *reinterpret_cast<const float4*>(be + j4);
+                        v[j4 + 0] *= sg * b4.x;
+                        v[j4 + 1] *= sg * b4.y;
+                        v[j4 + 2] *= sg * b4.z;
+                        v[j4 + 3] *= sg * b4.w;
+                    }
+                    if (is_a && h == q) {
+                        // this warp's rows r = 32q..32q+31 have their diagonal blocks in columns
+                        // 32h..32h+31: keep the fp32 copy for the diagonal inverses
+                        const bool upper = (r & 16) != 0;
+                        float* ad = adiag + (r >> 4) * ADIAG_BLOCK + (r & 15) * 17;
+                        #pragma unroll
+                        for (int jj = 0; jj < 16; ++jj) ad[jj] = upper ? v[16 + jj] : v[jj];
+                    }
+                    #pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) sts(sw128(dst, r, 4 * h + ch), pack8_half(v + 8 * ch));
                 }
             } else {
-                #pragma unroll
-                for (int sc = 0; sc < 64; ++sc)
-                    v[sc] = (sc < lim) ? gs->beta[sc] * __expf(Gr - gs->G[sc]) * v[sc] : 0.f;
+                gram_epilogue_unfactored(tmem + TM_G + lane_addr, gs, r, is_a, sbase + (dst - sb), dst,
+                                         adiag + (r >> 4) * ADIAG_BLOCK + (r & 15) * 17);
             }
-            if (is_a) {
-                const int b = r >> 4;
-                #pragma unroll
-                for (int bb = 0; bb < 4; ++bb)
-                    if (b == bb) {
-                        #pragma unroll
-                        for (int j = 0; j < 16; ++j) adiag[b * ADIAG_BLOCK + (r & 15) * 17 + j] = v[16 * bb + j];
-                    }
-            }
-            #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) sts(sw128(dst, r, ch), pack8_half(v + 8 * ch));
             tc_fence_before();
             grp.sync();
             if (t == 0) {
@@ -545,7 +654,8 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             const uint32_t tp = sb + OFF_TP + tps * TP_STAGE;
             if (is_a) {
-                // row r of D_b^{-1} = (I + A_bb)^{-1} by the column recurrence within the block
+                // row i of D_b = (I + A_bb)^{-1}:  x_j = delta_ij + sum_{m>j} x_m (-A)_mj, j = 15..0;
+                // the sum runs from m = 15 down so that only its last term waits for x_{j+1}
                 const int b = r >> 4, i = r & 15;
                 const float* ad = adiag + b * ADIAG_BLOCK;
                 float x[16];
@@ -553,25 +663,16 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int j = 15; j >= 0; --j) {
                     float acc = 0.f;
                     #pragma unroll
-                    for (int m = j + 1; m < 16; ++m) acc += x[m] * ad[m * 17 + j];
-                    x[j] = (j == i) ? 1.f : ((j < i) ? -acc : 0.f);
+                    for (int m = 15; m > j; --m) acc = fmaf(x[m], ad[m * 17 + j], acc);
+                    x[j] = (j == i) ? 1.f : ((j < i) ? acc : 0.f);
                 }
                 sts(sw128(tp, r, 2 * b), pack8_half(x));
                 sts(sw128(tp, r, 2 * b + 1), pack8_half(x + 8));
             }
             grp.sync();
-            // level 1 of the block inverse, and the first column of P T that is ready
-            if (q < 3) t_block(tp, as, q + 1, q, lane);         // T_{q+1,q}
-            else pt_block(tp, ps, 3, 3, lane);                  // PT_33
-            grp.sync();
-            if (q < 2) t_block(tp, as, q + 2, q, lane);         // T_{q+2,q}
-            else if (q == 2) pt_block(tp, ps, 2, 2, lane);      // PT_22
-            else pt_block(tp, ps, 3, 2, lane);                  // PT_32
-            grp.sync();
-            if (q == 0) t_block(tp, as, 3, 0, lane);            // T_30
-            else pt_block(tp, ps, q, 1, lane);                  // PT_11, PT_21, PT_31
-            grp.sync();
-            pt_block(tp, ps, 3 - q, 0, lane);                   // PT_30, PT_20, PT_10, PT_00
+            // warp q: the T rows of block q and the PT rows of block 3 - q
+            solve_row_block(tp, as, ps, q, lane);
+            solve_row_block(tp, as, ps, 7 - q, lane);
             fence_proxy_async_smem();
             grp.sync();
             if (t == 0) mbar_arrive(bar_addr(sb, B_TP_FULL + tps));
@@ -586,25 +687,12 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // initial state: S0^T (fp32 in TMEM, pre-scaled by the first chunk's decay; fp16 copy)
         if (ok) ok = grp.wait(bar_addr(sb, B_GATE_FULL + 0), 0);
         if (ok) {
-            const float g0 = gate(0)->gC;
-            const float* s0 = p.S0 ? p.S0 + static_cast<int64_t>(ug) * kD * kD + j : nullptr;
-            #pragma unroll
-            for (int piece = 0; piece < 4; ++piece) {
-                float v[32];
-                #pragma unroll
-                for (int d = 0; d < 32; ++d) v[d] = s0 ? s0[(32 * piece + d) * kD] : 0.f;
-                uint32_t hpk[16];
-                #pragma unroll
-                for (int e = 0; e < 16; ++e) hpk[e] = pack_half2(v[2 * e], v[2 * e + 1]);
-                tmem_st16(tmem + TM_SH + lane_addr + 16 * piece, hpk);
-                #pragma unroll
-                for (int d = 0; d < 32; ++d) v[d] *= g0;
-                tmem_st32(tmem + TM_S + lane_addr + 32 * piece, v);
-            }
-            tmem_wait_st();
+            load_initial_state(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr,
+                               p.S0 ? p.S0 + static_cast<int64_t>(ug) * kD * kD + j : nullptr, gate(0)->gC);
             tc_fence_before();
         }
         uint32_t drain_needed = 0;
+        uint32_t mma_issuer = 0;
         for (int c = 0; ok && c < nchunks; ++c) {
             const int s = c % kStages;
             const uint32_t ph = (c / kStages) & 1;
@@ -612,17 +700,22 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const uint32_t st = sb + OFF_KQV + s * STAGE_BYTES;
             // --- MMA_A: (KQ S)^T = S^T [K;Q]^T ---
             grp.sync();
-            if (leader) {
-                bool lok = mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs) &&
-                           (c == 0 || mbar_wait(bar_addr(sb, B_O_DONE), (c - 1) & 1, abort_flag, err, kTimeoutNs));
-                if (lok) {
+            if (warp == 8) {
+                int lok = 0;
+                if (leader)
+                    lok = mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs) &&
+                          (c == 0 || mbar_wait(bar_addr(sb, B_O_DONE), (c - 1) & 1, abort_flag, err, kTimeoutNs));
+                if (__shfl_sync(0xffffffffu, lok, 0)) {
                     tc_fence_after();
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t boff = (k >> 2) * 16384 + (k & 3) * 32;
-                        umma_f16_tmem_a(tmem + TM_AB, tmem + TM_SH + 8 * k, smem_desc_sw128(st + boff, 16, 1024),
-                                        ID_TK, k > 0);
+                    if (elect_one(mma_issuer)) {
+                        for (int k = 0; k < 8; ++k) {
+                            const uint32_t boff = (k >> 2) * 16384 + (k & 3) * 32;
+                            umma_f16_tmem_a(tmem + TM_AB, tmem + TM_SH + 8 * k,
+                                            smem_desc_sw128(st + boff, 16, 1024), ID_TK, k > 0);
+                        }
+                        umma_commit(bar_addr(sb, B_A_FULL));
                     }
-                    umma_commit(bar_addr(sb, B_A_FULL));
+                    __syncwarp();
                     drain_needed = 1;
                 }
             }
@@ -647,20 +740,25 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tc_fence_before();
             grp.sync();
             // --- MMA_B: ([T;PT] X)^T = V^T [T;PT]^T + Y^T [T;PT]^T ---
-            if (leader) {
+            if (warp == 8) {
                 const int tps = c & 1;
-                if (mbar_wait(bar_addr(sb, B_TP_FULL + tps), (c >> 1) & 1, abort_flag, err, kTimeoutNs)) {
+                int tok = 0;
+                if (leader) tok = mbar_wait(bar_addr(sb, B_TP_FULL + tps), (c >> 1) & 1, abort_flag, err, kTimeoutNs);
+                if (__shfl_sync(0xffffffffu, tok, 0)) {
                     tc_fence_after();
-                    const uint32_t tp = sb + OFF_TP + tps * TP_STAGE;
-                    const uint32_t vt = st + KQ_BYTES;
-                    for (int k = 0; k < 4; ++k)
-                        umma_f16(tmem + TM_B, smem_desc_sw128(vt + k * 2048, 8192, 1024),
-                                 smem_desc_sw128(tp + k * 32, 16, 1024), ID_MK, k > 0);
-                    for (int k = 0; k < 4; ++k)
-                        umma_f16_tmem_a(tmem + TM_B, tmem + TM_Y + 8 * k, smem_desc_sw128(tp + k * 32, 16, 1024),
-                                        ID_TK, 1);
-                    umma_commit(bar_addr(sb, B_B_FULL));
-                    umma_commit(bar_addr(sb, B_TP_EMPTY + tps));
+                    if (elect_one(mma_issuer)) {
+                        const uint32_t tp = sb + OFF_TP + tps * TP_STAGE;
+                        const uint32_t vt = st + KQ_BYTES;
+                        for (int k = 0; k < 4; ++k)
+                            umma_f16(tmem + TM_B, smem_desc_sw128(vt + k * 2048, 8192, 1024),
+                                     smem_desc_sw128(tp + k * 32, 16, 1024), ID_MK, k > 0);
+                        for (int k = 0; k < 4; ++k)
+                            umma_f16_tmem_a(tmem + TM_B, tmem + TM_Y + 8 * k, smem_desc_sw128(tp + k * 32, 16, 1024),
+                                            ID_TK, 1);
+                        umma_commit(bar_addr(sb, B_B_FULL));
+                        umma_commit(bar_addr(sb, B_TP_EMPTY + tps));
+                    }
+                    __syncwarp();
                 }
             }
             ok = grp.wait(bar_addr(sb, B_B_FULL), c & 1);
@@ -685,14 +783,17 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tc_fence_before();
             grp.sync();
             // --- MMA_C: S^T += U~^T K ---
-            if (leader) {
+            if (warp == 8) {
                 tc_fence_after();
-                for (int k = 0; k < 4; ++k)
-                    umma_f16_tmem_a(tmem + TM_S, tmem + TM_U + 8 * k, smem_desc_sw128(st + k * 2048, 16384, 1024),
-                                    ID_TM, 1);
-                umma_commit(bar_addr(sb, B_S_FULL));
-                umma_commit(bar_addr(sb, B_EMPTY + s));
-                mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));     // gates of chunk c consumed
+                if (elect_one(mma_issuer)) {
+                    for (int k = 0; k < 4; ++k)
+                        umma_f16_tmem_a(tmem + TM_S, tmem + TM_U + 8 * k, smem_desc_sw128(st + k * 2048, 16384, 1024),
+                                        ID_TM, 1);
+                    umma_commit(bar_addr(sb, B_S_FULL));
+                    umma_commit(bar_addr(sb, B_EMPTY + s));
+                    mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));     // gates of chunk c consumed
+                }
+                __syncwarp();
             }
             // --- the new state ---
             const bool last = c + 1 == nchunks;
@@ -703,16 +804,8 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (!ok) break;
             tc_fence_after();
             if (last) {
-                if (p.S_out) {
-                    float* so = p.S_out + static_cast<int64_t>(ug) * kD * kD + j;
-                    #pragma unroll
-                    for (int piece = 0; piece < 4; piece += 2) {
-                        float v[64];
-                        tmem_load_2x32(tmem + TM_S + lane_addr + 32 * piece, tmem + TM_S + lane_addr + 32 * piece + 32, v);
-                        #pragma unroll
-                        for (int d = 0; d < 64; ++d) so[(32 * piece + d) * kD] = v[d];
-                    }
-                }
+                if (p.S_out)
+                    store_final_state(tmem + TM_S + lane_addr, p.S_out + static_cast<int64_t>(ug) * kD * kD + j);
                 drain_needed = 0;
             } else {
                 const float gn = gate(s1)->gC;
@@ -734,7 +827,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 tc_fence_before();
             }
         }
-        if (leader && drain_needed && !ok) {
+        if (warp == 8 && lane == mma_issuer && drain_needed && !ok) {
             // wait for every MMA this thread issued before TMEM is released
             umma_commit(bar_addr(sb, B_DRAIN + 0));
             mbar_wait(bar_addr(sb, B_DRAIN + 0), 0, abort_flag, err, kTimeoutNs / 4);
@@ -746,54 +839,53 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         Group grp{NB_OUT, 128, j == 0, okflags + 4, 0, abort_flag, err};
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;
+            if (j == 0) bulk_wait_read_all();        // the staging tile is free again
             if (!grp.wait(bar_addr(sb, B_O_READY), c & 1)) break;
             tc_fence_after();
             const Gates* gs = gate(s);
             const int64_t t0 = static_cast<int64_t>(c) * kC;
-            const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
-            const int64_t base = (static_cast<int64_t>(ug) * L + t0) * kD + j;
-            float res[64];                           // o[r][j] for the chunk's 64 tokens
-            #pragma unroll
+            if (!p.out_bf16) {
+                // fp32 output: plain stores, done before the TMEM columns are released
+                const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
+                store_o_f32(tmem + TM_AB + lane_addr + 64, tmem + TM_B + lane_addr + 64, gs->gam,
+                            static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, n);
+                tc_fence_before();
+                grp.sync();
+                if (j == 0) {
+                    mbar_arrive(bar_addr(sb, B_O_DONE));
+                    mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
+                }
+                continue;
+            }
+            // o[r][j] = g_r (Q S)^T[j][r] + (P T X)^T[j][r], transposed through the staging tile
+            // (a warp writes 64 contiguous bytes per token) and written by the TMA unit as two
+            // 64 x 64 boxes; rows past L are clipped
+            uint8_t* ost = sbase + OFF_OST + (j >> 6) * 8192 + (j & 63) * 2;
+            #pragma unroll 1
             for (int piece = 0; piece < 2; ++piece) {
                 float qp[64];                        // (Q S)^T, then (P T X)^T, for 32 tokens
                 tmem_load_2x32(tmem + TM_AB + lane_addr + 64 + 32 * piece,
                                tmem + TM_B + lane_addr + 64 + 32 * piece, qp);
+                const float* gam = gs->gam + 32 * piece;
+                uint8_t* orow = ost + piece * 32 * 128;
                 #pragma unroll
                 for (int e4 = 0; e4 < 32; e4 += 4) {
-                    const float4 g4 = *reinterpret_cast<const float4*>(&gs->gam[32 * piece + e4]);
-                    res[32 * piece + e4 + 0] = g4.x * qp[e4 + 0] + qp[32 + e4 + 0];
-                    res[32 * piece + e4 + 1] = g4.y * qp[e4 + 1] + qp[32 + e4 + 1];
-                    res[32 * piece + e4 + 2] = g4.z * qp[e4 + 2] + qp[32 + e4 + 2];
-                    res[32 * piece + e4 + 3] = g4.w * qp[e4 + 3] + qp[32 + e4 + 3];
+                    const float4 g4 = *reinterpret_cast<const float4*>(gam + e4);
+                    *reinterpret_cast<__nv_bfloat16*>(orow + (e4 + 0) * 128) = __float2bfloat16_rn(g4.x * qp[e4 + 0] + qp[32 + e4 + 0]);
+                    *reinterpret_cast<__nv_bfloat16*>(orow + (e4 + 1) * 128) = __float2bfloat16_rn(g4.y * qp[e4 + 1] + qp[32 + e4 + 1]);
+                    *reinterpret_cast<__nv_bfloat16*>(orow + (e4 + 2) * 128) = __float2bfloat16_rn(g4.z * qp[e4 + 2] + qp[32 + e4 + 2]);
+                    *reinterpret_cast<__nv_bfloat16*>(orow + (e4 + 3) * 128) = __float2bfloat16_rn(g4.w * qp[e4 + 3] + qp[32 + e4 + 3]);
                 }
             }
-            // the TMEM columns are free for the next chunk's MMAs before the stores go out
             tc_fence_before();
-            if (p.out_bf16 && j == 0) bulk_wait_read_all();   // staging tile free again
+            fence_proxy_async_smem();
             grp.sync();
             if (j == 0) {
                 mbar_arrive(bar_addr(sb, B_O_DONE));
                 mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
-            }
-            if (p.out_bf16) {
-                // transpose through shared memory (a warp writes 64 contiguous bytes per token)
-                // and let the TMA unit write the 64 x 128 tile; rows past L are clipped
-                uint8_t* ost = sbase + OFF_OST + (j >> 6) * 8192 + (j & 63) * 2;
-                #pragma unroll
-                for (int r = 0; r < 64; ++r)
-                    *reinterpret_cast<__nv_bfloat16*>(ost + r * 128) = __float2bfloat16_rn(res[r]);
-                fence_proxy_async_smem();
-                grp.sync();
-                if (j == 0) {
-                    tma_store_3d(&tm_o, sb + OFF_OST, 0, static_cast<int32_t>(t0), ug);
-                    tma_store_3d(&tm_o, sb + OFF_OST + 8192, 64, static_cast<int32_t>(t0), ug);
-                    bulk_commit_group();
-                }
-            } else {
-                float* o = static_cast<float*>(p.o) + base;
-                #pragma unroll
-                for (int r = 0; r < 64; ++r)
-                    if (r < n) o[r * kD] = res[r];
+                tma_store_3d(&tm_o, sb + OFF_OST, 0, static_cast<int32_t>(t0), ug);
+                tma_store_3d(&tm_o, sb + OFF_OST + 8192, 64, static_cast<int32_t>(t0), ug);
+                bulk_commit_group();
             }
         }
         if (j == 0) bulk_wait_all();     // every output tile written before the CTA exits

@@ -78,3 +78,17 @@ def test_tc_in_place_state_and_no_final_state():
     torch.cuda.synchronize()
     assert st == lt2.LT2_OK and lt2.lt2_gdr_last_device_error() == lt2.LT2_OK
     assert torch.equal(o2, o)
+
+
+@pytest.mark.parametrize("power", [30.0, 3.0])
+def test_tc_strong_decay(power):
+    # alpha^30 gives a chunk decay far below e^-80, where e^{-G} is not representable and the
+    # chunk matrices take the unfactored e^{G_r - G_s}; alpha^3 mixes both kinds of chunk.
+    w = inputs.workload("gdn_prefill", T=1, B=1, H=3, L=450, s0="normal")
+    x = inputs.make_inputs(w, seed=21)
+    x["alpha"] = x["alpha"].double().pow(power).float()
+    x = to_device(x)
+    o, S = run_prefill(x, per_key=False, algo=TC)
+    o_ref, S_ref = oracle_prefill(x, False)
+    check("o", o, o_ref, TOL["bf16"])
+    check("S_T", S, S_ref, TOL["bf16"])
