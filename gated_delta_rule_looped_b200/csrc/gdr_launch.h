@@ -30,7 +30,11 @@ struct TcCall {
     int out_bf16;
     unsigned int* err;
 };
+// Scalar gating: 64-token chunks.  Per-key gating: 32-token chunks in the e-form (chunks whose
+// per-key decay is out of the tensor-core range run token by token inside the same kernel).
 bool prefill_tc_supports(int dtype_bf16, int dk, int dv, int per_key);
 cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream);
+bool prefill_kda_tc_supports(int dtype_bf16, int dk, int dv);
+cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream);
 
 }  // namespace lt2

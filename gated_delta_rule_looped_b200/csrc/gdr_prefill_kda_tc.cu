@@ -1,0 +1,892 @@
+// gdr_prefill_kda_tc.cu -- chunked prefill of the gated delta rule with per-key gating
+// (alpha_t a d_k vector) on Blackwell tensor cores, d_k = d_v = 128, bf16 q/k/v.
+//
+// The recurrence ("LT2 transformer looped a tempo lineare", section "Sostituire il motore",
+// displayed equation)  S_t = Diag(alpha_t) (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T,
+// read out as o_t = S_t^T q_t, is taken 32 tokens ("a chunk") at a time in its e-form: with the
+// chunk's incoming state S, G_r = sum_{s<=r} log alpha_s (a d_k vector, G_{-1} = 0),
+// Gamma_r = Diag(e^{G_r}) and e_r = k_r^T S_{r-1},
+//
+//   (I + M_ke) E = K^ S + M_kv V                                    (E: rows e_r)
+//   O  = Q^ S + N_qv V - N_qe E
+//   S' = Gamma_31 S + Kv^T V - Ke^T E
+//
+//   K^_r = Gamma_{r-1} k_r,  Q^_r = Gamma_r q_r,  Kv_s = beta_s Gamma_31 Gamma_s^{-1} k_s,
+//   Ke_s = beta_s Gamma_31 Gamma_{s-1}^{-1} k_s,
+//   M_ke[r,s] = beta_s k_r^T Gamma_{r-1} Gamma_{s-1}^{-1} k_s  (s < r),  M_kv: Gamma_s^{-1} (s < r),
+//   N_qe[r,s] = beta_s q_r^T Gamma_r Gamma_{s-1}^{-1} k_s  (s <= r),     N_qv: Gamma_s^{-1} (s <= r).
+//
+// (Checked in fp64 against the sequential definition by the test suite's chunked oracle.)
+// Every factor in the state-side operands K^, Q^, Kv, Ke is at most 1, so they are always
+// representable in fp16.  The four chunk Gram matrices are products of two fp16 tiles that
+// carry e^{G - R} and e^{R - G} around a per-key reference R = G_31 / 2, which stays in
+// range while a key decays by at most e^-19 over the chunk.  A chunk beyond that (or with any
+// alpha outside (0, 1]) is instead run token by token, exactly, on the fp32 state in TMEM.
+//
+// With the solve X = [T; N_qe T], T = (I + M_ke)^{-1}, and Z = X M_kv - [0; N_qv]:
+//   [E; -(O - Q^ S)] = X (K^ S) + Z V,
+// so one MMA (MMA_B) gives both E and the non-state part of O.  Per chunk, on transposed
+// quantities (one d_v column per TMEM lane):
+//   MMA_A  (K^ S, Q^ S)^T    = S^T [K^; Q^]^T          A = S^T (TMEM, fp16)   N = 64
+//   MMA_B  ([E; -O'])^T      = V^T Z^T + (K^ S)^T X^T  A = V^T (smem), then (K^ S)^T (TMEM)
+//   MMA_C  S^T (pre-scaled by Gamma_31) += V^T Kv - E^T Ke
+//
+// CTA = one (loop, batch, head) unit, 16 warps:
+//   warp 0       TMA producer (and TMEM allocation)
+//   warps 1, 2   per-key decay factors; K and Q tiles for keys 0..63 / 64..127 (eight fp16 tiles)
+//   warp 3       fp16 conversion of V, and the Gram MMA
+//   warps 4-7    prep: Gram epilogue, diagonal-block inverses, back substitution, Z
+//   warps 8-11   the S-dependent chain (warp 8 issues MMA_A, MMA_B, MMA_C)
+//   warps 12-15  output epilogue
+// Every mbarrier wait is bounded (see mbar_wait); a timeout is recorded in the device status
+// word and the CTA drains its copies and MMAs, frees TMEM and exits.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "gdr_common.cuh"
+#include "gdr_launch.h"
+#include "gdr_tc_common.cuh"
+#include "gdr_tma_host.h"
+#include "sm100_primitives.cuh"
+
+namespace lt2 {
+namespace kda {
+
+using namespace sm100;
+using namespace tcc;
+
+constexpr int kC = 32;                 // tokens per chunk
+constexpr int kThreads = 512;
+constexpr int kStages = 3;
+constexpr uint64_t kTimeoutNs = kWaitTimeoutNs;
+// Gram tiles carry factors e^{+-(G - G_31/2)}: in range while they stay within [2^-14, 2^14].
+constexpr float kFactorMax = 16384.f;
+constexpr float kFactorMin = 1.f / 16384.f;
+
+// Shared memory map (offsets from a 1024-byte aligned base).  Tiles are fp16, 128-byte rows
+// (64 elements) under the 128-byte swizzle; a 128-wide operand is two panels.
+// Chunk stage (3): [K^ | Q^] x 2 panels (rows 0-31 K^, 32-63 Q^), [Kv | Ke] x 2 panels, V x 2.
+constexpr uint32_t ST_KQ = 0;          // + panel * 8192
+constexpr uint32_t ST_KVE = 16384;     // + panel * 8192
+constexpr uint32_t ST_V = 32768;       // + panel * 4096
+constexpr uint32_t STAGE_BYTES = 40960;
+constexpr uint32_t STAGE_TX = 6 * 4096;   // K, Q, V boxes of 64 columns x 32 tokens (bf16)
+constexpr uint32_t OFF_STG = 0;
+// Gram stage (1): per panel [Kt (0-31) | Qt (32-63) | Be (64-95) | Bv (96-127)].
+constexpr uint32_t OFF_GRAM = OFF_STG + kStages * STAGE_BYTES;
+constexpr uint32_t GRAM_PANEL = 16384;
+// [X; Z] stages (2): X = [T; N_qe T] 64 rows, Z 64 rows, both 32 columns in 128-byte rows.
+constexpr uint32_t OFF_TP = OFF_GRAM + 2 * GRAM_PANEL;
+constexpr uint32_t TP_STAGE = 16384;
+constexpr uint32_t TP_Z = 8192;
+// Gram blocks for the solve (32 rows each): -M_ke, N_qe, M_kv, N_qv.
+constexpr uint32_t OFF_MKE = OFF_TP + 2 * TP_STAGE;
+constexpr uint32_t OFF_NQE = OFF_MKE + 4096;
+constexpr uint32_t OFF_MKV = OFF_NQE + 4096;
+constexpr uint32_t OFF_NQV = OFF_MKV + 4096;
+constexpr uint32_t OFF_ADIAG = OFF_NQV + 4096;   // fp32 diagonal blocks of -M_ke
+constexpr uint32_t ADIAG_BLOCK = 16 * kAdiagRow;
+constexpr uint32_t OFF_OST = OFF_ADIAG + 2304;   // o staging: 2 x [32 tokens][64] bf16
+constexpr uint32_t OFF_GATES = OFF_OST + 8192;
+constexpr uint32_t GATE_STAGE = 640;
+constexpr uint32_t OFF_BAR = OFF_GATES + kStages * GATE_STAGE;
+constexpr uint32_t BAR_BYTES = 512;
+constexpr uint32_t SMEM_USED = OFF_BAR + BAR_BYTES;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
+
+struct Gates {
+    float decay[kD];   // e^{G_31}: the chunk's decay per key
+    int in_range[2];   // per conversion warp: Gram factors within range for its 64 keys
+};
+static_assert(sizeof(Gates) <= GATE_STAGE, "gate stage too small");
+
+enum Bar : uint32_t {
+    B_FULL = 0,        // [3] TMA of a stage landed
+    B_CONV = 3,        // [3] stage and Gram tiles converted (warps 1, 2, 3)
+    B_EMPTY = 6,       // [3] chain done with a stage
+    B_GATE_FULL = 9,   // [3] decay factors written (warps 1, 2)
+    B_GATE_EMPTY = 12, // [3] chain and output epilogue done with a gate stage
+    B_TP_FULL = 15,    // [2]
+    B_TP_EMPTY = 17,   // [2]
+    B_G_FULL = 19,     // Gram in TMEM
+    B_G_EMPTY = 20,    // Gram read out
+    B_GFREE = 21,      // Gram MMA done reading the Gram tiles
+    B_A_FULL = 22,
+    B_B_FULL = 23,
+    B_S_FULL = 24,
+    B_O_READY = 25,
+    B_O_DONE = 26,
+    B_DRAIN = 27,      // [2]
+    B_COUNT = 29
+};
+constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + B_COUNT * 8;
+constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 16;
+constexpr uint32_t OFF_OKFLAG = OFF_ABORT + 16;
+static_assert(OFF_OKFLAG + 32 <= OFF_BAR + BAR_BYTES, "barrier area too small");
+
+constexpr int NB_PREP = 1, NB_CHAIN = 2, NB_OUT = 3;
+
+// TMEM columns (lane j = d_v index in the chain's regions).
+constexpr uint32_t TM_G = 0;           // Gram (64 columns; lanes 0-31 Kt rows, 32-63 Qt rows)
+constexpr uint32_t TM_S = 64;          // S^T fp32, pre-scaled by the chunk decay (128)
+constexpr uint32_t TM_SH = 192;        // S^T fp16 pairs (64): A operand of MMA_A
+constexpr uint32_t TM_AB = 256;        // (K^ S)^T 256..287, (Q^ S)^T 288..319
+constexpr uint32_t TM_Y = 256;         //   (K^ S)^T as fp16 pairs (16), A operand of MMA_B
+constexpr uint32_t TM_E = 272;         //   -E^T as fp16 pairs (16), A operand of MMA_C
+constexpr uint32_t TM_B = 320;         // E^T 320..351, -(O - Q^ S)^T 352..383
+constexpr uint32_t TM_COLS = 512;
+
+constexpr uint32_t ID_GRAM = idesc_f16_f32(128, 64, 0, 0);
+constexpr uint32_t ID_T64 = idesc_f16_f32(128, 64, 0, 0);     // A in TMEM, B K-major, N = 64
+constexpr uint32_t ID_M64 = idesc_f16_f32(128, 64, 1, 0);     // A MN-major (smem), B K-major
+constexpr uint32_t ID_MM = idesc_f16_f32(128, 128, 1, 1);     // A MN-major (smem), B MN-major
+constexpr uint32_t ID_TM = idesc_f16_f32(128, 128, 0, 1);     // A in TMEM, B MN-major
+
+struct Params {
+    const __nv_bfloat16* q;    // [units_total][L][128] (the exact path of out-of-range chunks)
+    const __nv_bfloat16* k;
+    const __nv_bfloat16* v;
+    const float* alpha;        // [units_total][L][128]
+    const float* beta;         // [units_total][L]
+    const float* S0;           // [units_total][128][128] or null
+    void* o;
+    float* S_out;              // nullable
+    int64_t L;
+    int unit0;
+    int out_bf16;
+    unsigned int* err;
+};
+
+__device__ __forceinline__ uint32_t bar_addr(uint32_t base, uint32_t i) { return base + OFF_BAR + 8u * i; }
+
+__device__ __forceinline__ uint32_t pack_half2_scaled(uint32_t bf2, float f0, float f1)
+{
+    return pack_half2(bf16_lo(bf2) * f0, bf16_hi(bf2) * f1);
+}
+
+// ---- conversion: per-key decay factors and the eight fp16 tiles of one chunk --------------
+// Lane l of conversion warp w (1 or 2) owns keys i = 64 (w-1) + 2l, +1, i.e. 4 bytes of every
+// 128-byte row of panel w-1.  With P_t = e^{G_t} (P_-1 = 1), sq = sqrt(P_31), F_t = P_t / sq:
+//   K^_t = P_{t-1} k_t,  Q^_t = P_t q_t,  Kv_t = b_t (P_31 / P_t) k_t,  Ke_t = b_t (P_31 / P_{t-1}) k_t,
+//   Kt_t = F_{t-1} k_t,  Qt_t = F_t q_t,  Bv_t = b_t k_t / F_t,          Be_t = b_t k_t / F_{t-1}.
+// Returns the chunk decay P_31 of the lane's two keys, and whether every F_t lies in
+// [kFactorMin, kFactorMax] for both.
+struct ConvOut {
+    float2 decay;
+    bool in_range;
+};
+__device__ __noinline__ ConvOut convert_kq(uint32_t st, uint32_t gram, const float* alpha_u, const float* beta_u,
+                                           int n, int panel, int lane, uint8_t* sbase, uint32_t sb)
+{
+    // beta of token `lane` (0 beyond the chunk's end)
+    const float bl = lane < n ? beta_u[lane] : 0.f;
+    const int koff = 64 * panel + 2 * lane;
+    // pass 1: the chunk's total decay per key
+    float2 P31 = make_float2(1.f, 1.f);
+    #pragma unroll 4
+    for (int t = 0; t < n; ++t) {
+        const float2 a = *reinterpret_cast<const float2*>(alpha_u + static_cast<int64_t>(t) * kD + koff);
+        P31.x *= a.x;
+        P31.y *= a.y;
+    }
+    const float2 sq = make_float2(sqrtf(P31.x), sqrtf(P31.y));
+    const float2 isq = make_float2(1.f / sq.x, 1.f / sq.y);
+    float2 P = make_float2(1.f, 1.f);          // P_{t-1}
+    float2 F = isq;                            // F_{t-1}
+    float2 R = sq;                             // 1 / F_{t-1}
+    float fmax_ = fmaxf(isq.x, isq.y), fmin_ = fminf(isq.x, isq.y);
+    const uint32_t chunk = static_cast<uint32_t>(lane >> 2);
+    const uint32_t within = static_cast<uint32_t>(lane & 3) * 4u;
+    auto at = [&](uint32_t tile, int row) -> uint32_t* {
+        return reinterpret_cast<uint32_t*>(sbase + (sw128(tile, row, chunk) + within - sb));
+    };
+    const uint32_t kq = st + ST_KQ + panel * 8192, kve = st + ST_KVE + panel * 8192;
+    const uint32_t gp = gram + panel * GRAM_PANEL;
+    #pragma unroll 1
+    for (int t = 0; t < kC; ++t) {
+        const float2 a = t < n ? *reinterpret_cast<const float2*>(alpha_u + static_cast<int64_t>(t) * kD + koff)
+                               : make_float2(1.f, 1.f);
+        const float b = __shfl_sync(0xffffffffu, bl, t);
+        const float2 Pn = make_float2(P.x * a.x, P.y * a.y);          // P_t
+        const float2 Fn = make_float2(Pn.x * isq.x, Pn.y * isq.y);    // F_t
+        const float2 Rn = make_float2(1.f / Fn.x, 1.f / Fn.y);        // 1 / F_t
+        fmax_ = fmaxf(fmax_, fmaxf(Fn.x, Fn.y));
+        fmin_ = fminf(fmin_, fminf(Fn.x, Fn.y));
+        uint32_t* kp = at(kq, t);
+        uint32_t* qp = at(kq, 32 + t);
+        const uint32_t k2 = *kp, q2 = *qp;
+        *kp = pack_half2_scaled(k2, P.x, P.y);                              // K^ (in place)
+        *qp = pack_half2_scaled(q2, Pn.x, Pn.y);                            // Q^ (in place)
+        *at(kve, t) = pack_half2_scaled(k2, b * sq.x * Rn.x, b * sq.y * Rn.y);       // Kv
+        *at(kve, 32 + t) = pack_half2_scaled(k2, b * sq.x * R.x, b * sq.y * R.y);    // Ke
+        *at(gp, t) = pack_half2_scaled(k2, F.x, F.y);                       // Kt
+        *at(gp, 32 + t) = pack_half2_scaled(q2, Fn.x, Fn.y);                // Qt
+        *at(gp, 64 + t) = pack_half2_scaled(k2, b * R.x, b * R.y);          // Be
+        *at(gp, 96 + t) = pack_half2_scaled(k2, b * Rn.x, b * Rn.y);        // Bv
+        P = Pn;
+        F = Fn;
+        R = Rn;
+    }
+    return ConvOut{P, fmax_ <= kFactorMax && fmin_ >= kFactorMin};
+}
+
+// ---- prep helpers (32-token chunk: two 16-token blocks) -----------------------------------
+
+// Gram epilogue, row r of the Kt rows (warp 4) or Qt rows (warp 5): the two 32-column halves
+// of the Gram row (against Be, against Bv), masked to s < r (Kt rows) or s <= r (Qt rows),
+// as fp16 rows of -M_ke / M_kv or N_qe / N_qv; the Kt rows also keep fp32 copies of the
+// diagonal 16x16 blocks of -M_ke.
+__device__ __forceinline__ void gram_epilogue_row(const float (&v)[64], int r, bool kt_rows, uint8_t* sbase,
+                                                  uint32_t sb, float* adiag)
+{
+    const int lim = kt_rows ? r : r + 1;
+    const float sg = kt_rows ? -1.f : 1.f;
+    const uint32_t t_e = sb + (kt_rows ? OFF_MKE : OFF_NQE);
+    const uint32_t t_v = sb + (kt_rows ? OFF_MKV : OFF_NQV);
+    float e[32], w[32];
+    #pragma unroll
+    for (int s = 0; s < 32; ++s) {
+        e[s] = s < lim ? sg * v[s] : 0.f;
+        w[s] = s < lim ? v[32 + s] : 0.f;
+    }
+    #pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+        *reinterpret_cast<uint4*>(sbase + (sw128(t_e, r, ch) - sb)) = pack8_half(e + 8 * ch);
+        *reinterpret_cast<uint4*>(sbase + (sw128(t_v, r, ch) - sb)) = pack8_half(w + 8 * ch);
+    }
+    if (kt_rows) {
+        const bool upper = (r & 16) != 0;
+        float* ad = adiag + (r >> 4) * ADIAG_BLOCK + (r & 15) * kAdiagRow;
+        #pragma unroll
+        for (int j = 0; j < 16; ++j) ad[j] = upper ? e[16 + j] : e[j];
+    }
+}
+
+// Row block rb of Z = X M_kv - [0; N_qv] (X from TP, rows 0..63; M_kv strictly lower).
+__device__ __noinline__ void z_row_block(uint32_t tp, uint32_t mkv, uint32_t nqv, int rb, int lane)
+{
+    const bool is_t = rb < 2;
+    const uint32_t g = lane >> 2, tq = lane & 3;
+    #pragma unroll 1
+    for (int j = 0; j < 2; ++j) {
+        float acc[2][4];
+        zero_c(acc);
+        if (!is_t) {
+            // -N_qv block (rb - 2, j) in the accumulator layout: rows g, g+8; columns 2tq, 2tq+1
+            const int row0 = 16 * (rb - 2);
+            #pragma unroll
+            for (int nb = 0; nb < 2; ++nb) {
+                const uint32_t c0 = lds32(sw128(nqv, row0 + g, 2 * j + nb) + tq * 4);
+                const uint32_t c1 = lds32(sw128(nqv, row0 + g + 8, 2 * j + nb) + tq * 4);
+                acc[nb][0] = -half_lo(c0);
+                acc[nb][1] = -half_hi(c0);
+                acc[nb][2] = -half_lo(c1);
+                acc[nb][3] = -half_hi(c1);
+            }
+        }
+        const int kmax = is_t ? rb : 1;
+        #pragma unroll 1
+        for (int k = j; k <= kmax; ++k) {
+            uint32_t a[4], b[4];
+            frag_a(tp, 16 * rb, 16 * k, lane, a);
+            frag_b(mkv, 16 * k, 16 * j, lane, b);
+            mma_block(acc, a, b);
+        }
+        store_block(tp + TP_Z, 16 * rb, 16 * j, lane, acc, 1.f);
+    }
+}
+
+// ---- chain helpers --------------------------------------------------------------------------
+
+// Chain thread j: S0^T row j into TMEM, as fp16 pairs (unscaled) and as fp32 scaled per
+// column i (= key) by decay[i] (nullptr: unscaled).
+__device__ __noinline__ void load_initial_state(uint32_t tm_s, uint32_t tm_sh, const float* s0, const float* decay)
+{
+    #pragma unroll 1
+    for (int piece = 0; piece < 4; ++piece) {
+        float v[32];
+        #pragma unroll
+        for (int d = 0; d < 32; ++d) v[d] = s0 ? s0[(32 * piece + d) * kD] : 0.f;
+        uint32_t hpk[16];
+        #pragma unroll
+        for (int e = 0; e < 16; ++e) hpk[e] = pack_half2(v[2 * e], v[2 * e + 1]);
+        tmem_st16(tm_sh + 16 * piece, hpk);
+        if (decay) {
+            #pragma unroll
+            for (int d = 0; d < 32; ++d) v[d] *= decay[32 * piece + d];
+        }
+        tmem_st32(tm_s + 32 * piece, v);
+    }
+    tmem_wait_st();
+}
+
+// Chain thread j: the new state's fp16 copy (for MMA_A) and the fp32 state scaled per column
+// by the next chunk's decay (nullptr: unscaled, the next chunk runs token by token).
+__device__ __forceinline__ void state_update(uint32_t tm_s, uint32_t tm_sh, const float* decay)
+{
+    #pragma unroll 1
+    for (int piece = 0; piece < 4; piece += 2) {
+        float v[64];
+        tmem_load_2x32(tm_s + 32 * piece, tm_s + 32 * piece + 32, v);
+        uint32_t hpk[32];
+        #pragma unroll
+        for (int e = 0; e < 32; ++e) hpk[e] = pack_half2(v[2 * e], v[2 * e + 1]);
+        tmem_st16(tm_sh + 16 * piece, *reinterpret_cast<uint32_t(*)[16]>(hpk));
+        tmem_st16(tm_sh + 16 * piece + 16, *reinterpret_cast<uint32_t(*)[16]>(hpk + 16));
+        if (decay) {
+            #pragma unroll
+            for (int d4 = 0; d4 < 64; d4 += 4) {
+                const float4 f = *reinterpret_cast<const float4*>(decay + 32 * piece + d4);
+                v[d4 + 0] *= f.x;
+                v[d4 + 1] *= f.y;
+                v[d4 + 2] *= f.z;
+                v[d4 + 3] *= f.w;
+            }
+            tmem_st32(tm_s + 32 * piece, *reinterpret_cast<float(*)[32]>(v));
+            tmem_st32(tm_s + 32 * piece + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+        }
+    }
+    tmem_wait_st();
+}
+
+// Chain thread j: the chunk's n tokens run one at a time on column j of the fp32 state in
+// TMEM (the definition, in fp32): e = k^T S, S <- Diag(alpha) (S - beta k e) + beta k v^T,
+// o = S^T q.  Inputs are read from global memory (the same 256-byte rows for every thread).
+struct ExactIn {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* k;
+    const __nv_bfloat16* v;
+    const float* alpha;
+    const float* beta;
+    void* o;
+    int out_bf16;
+};
+__device__ __noinline__ void exact_chunk(uint32_t tm_s, ExactIn p, int64_t row0, int n, int j)
+{
+    #pragma unroll 1
+    for (int t = 0; t < n; ++t) {
+        const int64_t row = row0 + t;
+        const __nv_bfloat16* kr = p.k + row * kD;
+        const __nv_bfloat16* qr = p.q + row * kD;
+        const float* ar = p.alpha + row * kD;
+        const float b = p.beta[row];
+        const float vj = __bfloat162float(p.v[row * kD + j]);
+        float e = 0.f;
+        #pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+            float sv[64];
+            tmem_load_2x32(tm_s + 64 * h, tm_s + 64 * h + 32, sv);
+            #pragma unroll
+            for (int d8 = 0; d8 < 64; d8 += 8) {
+                const uint4 kw = *reinterpret_cast<const uint4*>(kr + 64 * h + d8);
+                const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w};
+                #pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    e = fmaf(bf16_lo(kk[u]), sv[d8 + 2 * u], e);
+                    e = fmaf(bf16_hi(kk[u]), sv[d8 + 2 * u + 1], e);
+                }
+            }
+        }
+        float o = 0.f;
+        #pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+            float sv[64];
+            tmem_load_2x32(tm_s + 64 * h, tm_s + 64 * h + 32, sv);
+            #pragma unroll
+            for (int d8 = 0; d8 < 64; d8 += 8) {
+                const uint4 kw = *reinterpret_cast<const uint4*>(kr + 64 * h + d8);
+                const uint4 qw = *reinterpret_cast<const uint4*>(qr + 64 * h + d8);
+                const float4 a0 = *reinterpret_cast<const float4*>(ar + 64 * h + d8);
+                const float4 a1 = *reinterpret_cast<const float4*>(ar + 64 * h + d8 + 4);
+                const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w};
+                const uint32_t qq[4] = {qw.x, qw.y, qw.z, qw.w};
+                const float aa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                #pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float k0 = bf16_lo(kk[u]), k1 = bf16_hi(kk[u]);
+                    float& s0 = sv[d8 + 2 * u];
+                    float& s1 = sv[d8 + 2 * u + 1];
+                    s0 = aa[2 * u] * (s0 - b * k0 * e) + b * k0 * vj;
+                    s1 = aa[2 * u + 1] * (s1 - b * k1 * e) + b * k1 * vj;
+                    o = fmaf(bf16_lo(qq[u]), s0, o);
+                    o = fmaf(bf16_hi(qq[u]), s1, o);
+                }
+            }
+            tmem_st32(tm_s + 64 * h, *reinterpret_cast<float(*)[32]>(sv));
+            tmem_st32(tm_s + 64 * h + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
+            tmem_wait_st();
+        }
+        if (p.out_bf16)
+            static_cast<__nv_bfloat16*>(p.o)[row * kD + j] = __float2bfloat16_rn(o);
+        else
+            static_cast<float*>(p.o)[row * kD + j] = o;
+    }
+}
+
+// Output thread j, fp32 output: o[r][j] = (Q^ S)_rj - B_rj for the chunk's n tokens.
+__device__ __noinline__ void store_o_f32(uint32_t tm_qs, uint32_t tm_b, float* o, int n)
+{
+    float qp[64];
+    tmem_load_2x32(tm_qs, tm_b, qp);
+    #pragma unroll
+    for (int r = 0; r < 32; ++r)
+        if (r < n) o[r * kD] = qp[r] - qp[32 + r];
+}
+
+// Gram [Kt; Qt; Be; Bv] [Be; Bv]^T (M = 128, N = 64, K = 128) into TMEM; only lanes 0-63 are
+// used.  Commits the Gram barrier and the release of the Gram tiles.
+__device__ __forceinline__ void issue_gram(uint32_t sb, uint32_t tmem)
+{
+    const uint32_t g = sb + OFF_GRAM;
+    for (int k = 0; k < 8; ++k) {
+        const uint32_t off = (k >> 2) * GRAM_PANEL + (k & 3) * 32;
+        umma_f16(tmem + TM_G, smem_desc_sw128(g + off, 16, 1024), smem_desc_sw128(g + 8192 + off, 16, 1024),
+                 ID_GRAM, k > 0);
+    }
+    umma_commit(bar_addr(sb, B_G_FULL));
+    umma_commit(bar_addr(sb, B_GFREE));
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                          Params p)
+{
+    allow_next_loop_to_start();
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t sb = (raw + 1023u) & ~1023u;
+    uint8_t* sbase = smem_raw + (sb - raw);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + OFF_ABORT);
+    volatile int* okflags = reinterpret_cast<volatile int*>(sbase + OFF_OKFLAG);
+    auto gate = [&](int s) -> Gates* { return reinterpret_cast<Gates*>(sbase + OFF_GATES + s * GATE_STAGE); };
+    auto lds = [&](uint32_t addr) -> uint4 { return *reinterpret_cast<const uint4*>(sbase + (addr - sb)); };
+    auto sts = [&](uint32_t addr, uint4 v) { *reinterpret_cast<uint4*>(sbase + (addr - sb)) = v; };
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t L = p.L;
+    const int nchunks = static_cast<int>((L + kC - 1) / kC);
+    const int ug = p.unit0 + blockIdx.x;
+    unsigned int* err = p.err;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar_addr(sb, B_FULL + s), 1);
+            mbar_init(bar_addr(sb, B_CONV + s), 3);
+            mbar_init(bar_addr(sb, B_EMPTY + s), 1);
+            mbar_init(bar_addr(sb, B_GATE_FULL + s), 2);
+            mbar_init(bar_addr(sb, B_GATE_EMPTY + s), 2);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar_addr(sb, B_TP_FULL + s), 1);
+            mbar_init(bar_addr(sb, B_TP_EMPTY + s), 1);
+            mbar_init(bar_addr(sb, B_DRAIN + s), 1);
+        }
+        mbar_init(bar_addr(sb, B_G_FULL), 1);
+        mbar_init(bar_addr(sb, B_G_EMPTY), 1);
+        mbar_init(bar_addr(sb, B_GFREE), 1);
+        mbar_init(bar_addr(sb, B_A_FULL), 1);
+        mbar_init(bar_addr(sb, B_B_FULL), 1);
+        mbar_init(bar_addr(sb, B_S_FULL), 1);
+        mbar_init(bar_addr(sb, B_O_READY), 1);
+        mbar_init(bar_addr(sb, B_O_DONE), 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(sb + OFF_TMEM_SLOT, TM_COLS);
+        tmem_relinquish();
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+            prefetch_tmap(&tm_o);
+        }
+    }
+    if (warp >= 4 && warp < 8) {
+        // zero both [X; Z] stages once: blocks right of the diagonal and the unused columns
+        // 32..63 of every row are never written
+        const int t = threadIdx.x - 128;
+        for (uint32_t off = t * 16; off < 2 * TP_STAGE; off += 128 * 16) sts(sb + OFF_TP + off, make_uint4(0, 0, 0, 0));
+        fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + OFF_TMEM_SLOT);
+
+    if (warp == 0) {
+        // ================= TMA producer =================
+        int issued = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % kStages;
+            const uint32_t ph = ((c / kStages) & 1) ^ 1;
+            int free_ok = 0;
+            if (lane == 0) free_ok = mbar_wait(bar_addr(sb, B_EMPTY + s), ph, abort_flag, err, kTimeoutNs);
+            if (!__shfl_sync(0xffffffffu, free_ok, 0)) break;
+            uint32_t leader;
+            if (elect_one(leader)) {
+                const uint32_t fb = bar_addr(sb, B_FULL + s);
+                mbar_arrive_expect_tx(fb, STAGE_TX);
+                const uint32_t st = sb + OFF_STG + s * STAGE_BYTES;
+                const int32_t y = c * kC;
+                tma_load_3d(st + ST_KQ, &tm_k, 0, y, ug, fb);
+                tma_load_3d(st + ST_KQ + 8192, &tm_k, 64, y, ug, fb);
+                tma_load_3d(st + ST_KQ + 4096, &tm_q, 0, y, ug, fb);
+                tma_load_3d(st + ST_KQ + 8192 + 4096, &tm_q, 64, y, ug, fb);
+                tma_load_3d(st + ST_V, &tm_v, 0, y, ug, fb);
+                tma_load_3d(st + ST_V + 4096, &tm_v, 64, y, ug, fb);
+            }
+            __syncwarp();
+            issued = c + 1;
+        }
+        if (lane == 0 && *abort_flag) {
+            for (int c = issued - kStages < 0 ? 0 : issued - kStages; c < issued; ++c)
+                mbar_wait(bar_addr(sb, B_FULL + c % kStages), (c / kStages) & 1, abort_flag, err, kTimeoutNs / 4);
+        }
+    } else if (warp < 4) {
+        // ================= decay factors and K/Q tiles (warps 1, 2), V and the Gram (warp 3) =====
+        uint32_t gram_issuer = 0;
+        int gram_issued = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % kStages;
+            const uint32_t ph = (c / kStages) & 1;
+            const uint32_t st = sb + OFF_STG + s * STAGE_BYTES;
+            const int64_t t0 = static_cast<int64_t>(c) * kC;
+            const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
+            int ok = 0;
+            if (lane == 0) {
+                ok = mbar_wait(bar_addr(sb, B_FULL + s), ph, abort_flag, err, kTimeoutNs);
+                if (ok && warp != 3) {
+                    ok = mbar_wait(bar_addr(sb, B_GATE_EMPTY + s), ph ^ 1, abort_flag, err, kTimeoutNs) &&
+                         (c == 0 || mbar_wait(bar_addr(sb, B_GFREE), (c - 1) & 1, abort_flag, err, kTimeoutNs));
+                }
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            if (warp != 3) {
+                const int panel = warp - 1;
+                const int64_t urow = static_cast<int64_t>(ug) * L + t0;
+                const ConvOut cv = convert_kq(st, sb + OFF_GRAM, p.alpha + urow * kD, p.beta + urow, n, panel, lane,
+                                              sbase, sb);
+                Gates* gs = gate(s);
+                *reinterpret_cast<float2*>(&gs->decay[64 * panel + 2 * lane]) = cv.decay;
+                const bool all_in = __all_sync(0xffffffffu, cv.in_range);
+                if (lane == 0) gs->in_range[panel] = all_in ? 1 : 0;
+            } else {
+                #pragma unroll 1
+                for (int panel = 0; panel < 2; ++panel) convert_tile(st + ST_V + panel * 4096, 256, lane, lds, sts);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar_addr(sb, B_CONV + s));
+                if (warp != 3) mbar_arrive(bar_addr(sb, B_GATE_FULL + s));
+            }
+            if (warp == 3) {
+                int gram_ok = 0;
+                if (lane == 0)
+                    gram_ok = mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs) &&
+                              (c == 0 || mbar_wait(bar_addr(sb, B_G_EMPTY), (c - 1) & 1, abort_flag, err, kTimeoutNs));
+                if (__shfl_sync(0xffffffffu, gram_ok, 0)) {
+                    tc_fence_after();
+                    if (elect_one(gram_issuer)) issue_gram(sb, tmem);
+                    __syncwarp();
+                    gram_issued = 1;
+                }
+            }
+            if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
+        }
+        if (warp == 3 && lane == gram_issuer && gram_issued && *abort_flag) {
+            umma_commit(bar_addr(sb, B_DRAIN + 1));
+            mbar_wait(bar_addr(sb, B_DRAIN + 1), 0, abort_flag, err, kTimeoutNs / 4);
+        }
+    } else if (warp < 8) {
+        // ================= prep: Gram epilogue, diagonal inverses, back substitution, Z =========
+        const int t = threadIdx.x - 128;
+        const int q = warp - 4;
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+        Group grp{NB_PREP, 128, t == 0, okflags + 0, 0, abort_flag, err};
+        float* adiag = reinterpret_cast<float*>(sbase + OFF_ADIAG);
+        for (int c = 0; c < nchunks; ++c) {
+            const int tps = c & 1;
+            if (!grp.wait(bar_addr(sb, B_G_FULL), c & 1, bar_addr(sb, B_TP_EMPTY + tps), ((c >> 1) & 1) ^ 1)) break;
+            tc_fence_after();
+            if (q < 2) {
+                float v[64];
+                tmem_load_2x32(tmem + TM_G + lane_addr, tmem + TM_G + lane_addr + 32, v);
+                gram_epilogue_row(v, lane, q == 0, sbase, sb, adiag);
+            }
+            tc_fence_before();
+            grp.sync();
+            if (t == 0) mbar_arrive(bar_addr(sb, B_G_EMPTY));
+            const uint32_t tp = sb + OFF_TP + tps * TP_STAGE;
+            if (q == 0) diag_block_inverse_row(tp, lane, adiag + (lane >> 4) * ADIAG_BLOCK);
+            grp.sync();
+            // warp q: row block q of X = [T; N_qe T] (T rows 0..31, then 32..63), then of Z
+            solve_row_block(tp, sb + OFF_MKE, sb + OFF_NQE, q, 2, lane);
+            z_row_block(tp, sb + OFF_MKV, sb + OFF_NQV, q, lane);
+            fence_proxy_async_smem();
+            grp.sync();
+            if (t == 0) mbar_arrive(bar_addr(sb, B_TP_FULL + tps));
+        }
+    } else if (warp < 12) {
+        // ================= the S-dependent chain (lane j = d_v column j of S) =================
+        const int j = threadIdx.x - 256;
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+        const bool leader = j == 0;
+        Group grp{NB_CHAIN, 128, leader, okflags + 2, 0, abort_flag, err};
+        bool ok = nchunks > 0;
+        uint32_t ph_a = 0, ph_b = 0, ph_s = 0;
+        if (ok) ok = grp.wait(bar_addr(sb, B_GATE_FULL + 0), 0);
+        if (ok) {
+            const Gates* g0 = gate(0);
+            const bool exact0 = !(g0->in_range[0] && g0->in_range[1]);
+            load_initial_state(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr,
+                               p.S0 ? p.S0 + static_cast<int64_t>(ug) * kD * kD + j : nullptr,
+                               exact0 ? nullptr : g0->decay);
+            tc_fence_before();
+        }
+        uint32_t drain_needed = 0;
+        uint32_t mma_issuer = 0;
+        for (int c = 0; ok && c < nchunks; ++c) {
+            const int s = c % kStages;
+            const uint32_t ph = (c / kStages) & 1;
+            const int tps = c & 1;
+            const uint32_t st = sb + OFF_STG + s * STAGE_BYTES;
+            const uint32_t tp = sb + OFF_TP + tps * TP_STAGE;
+            const int64_t t0 = static_cast<int64_t>(c) * kC;
+            const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
+            const Gates* gs = gate(s);
+            const bool exact = !(gs->in_range[0] && gs->in_range[1]);
+            if (!exact) {
+                // --- MMA_A: (K^ S, Q^ S)^T = S^T [K^; Q^]^T ---
+                grp.sync();
+                if (warp == 8) {
+                    int lok = 0;
+                    if (leader)
+                        lok = mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs) &&
+                              (c == 0 || mbar_wait(bar_addr(sb, B_O_DONE), (c - 1) & 1, abort_flag, err, kTimeoutNs));
+                    if (__shfl_sync(0xffffffffu, lok, 0)) {
+                        tc_fence_after();
+                        if (elect_one(mma_issuer)) {
+                            for (int k = 0; k < 8; ++k) {
+                                const uint32_t boff = ST_KQ + (k >> 2) * 8192 + (k & 3) * 32;
+                                umma_f16_tmem_a(tmem + TM_AB, tmem + TM_SH + 8 * k,
+                                                smem_desc_sw128(st + boff, 16, 1024), ID_T64, k > 0);
+                            }
+                            umma_commit(bar_addr(sb, B_A_FULL));
+                        }
+                        __syncwarp();
+                        drain_needed = 1;
+                    }
+                }
+                ok = grp.wait(bar_addr(sb, B_A_FULL), ph_a);
+                ph_a ^= 1u;
+                if (!ok) break;
+                tc_fence_after();
+                // --- (K^ S)^T as fp16 pairs: the second A operand of MMA_B ---
+                {
+                    float ks[32];
+                    tmem_load32(tmem + TM_AB + lane_addr, ks);
+                    uint32_t hpk[16];
+                    #pragma unroll
+                    for (int e = 0; e < 16; ++e) hpk[e] = pack_half2(ks[2 * e], ks[2 * e + 1]);
+                    tmem_st16(tmem + TM_Y + lane_addr, hpk);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                grp.sync();
+                // --- MMA_B: ([E; -O'])^T = V^T Z^T + (K^ S)^T X^T ---
+                if (warp == 8) {
+                    int tok = 0;
+                    if (leader) tok = mbar_wait(bar_addr(sb, B_TP_FULL + tps), (c >> 1) & 1, abort_flag, err, kTimeoutNs);
+                    if (__shfl_sync(0xffffffffu, tok, 0)) {
+                        tc_fence_after();
+                        if (elect_one(mma_issuer)) {
+                            for (int k = 0; k < 2; ++k)
+                                umma_f16(tmem + TM_B, smem_desc_sw128(st + ST_V + k * 2048, 4096, 1024),
+                                         smem_desc_sw128(tp + TP_Z + k * 32, 16, 1024), ID_M64, k > 0);
+                            for (int k = 0; k < 2; ++k)
+                                umma_f16_tmem_a(tmem + TM_B, tmem + TM_Y + 8 * k, smem_desc_sw128(tp + k * 32, 16, 1024),
+                                                ID_T64, 1);
+                            umma_commit(bar_addr(sb, B_B_FULL));
+                            umma_commit(bar_addr(sb, B_O_READY));
+                            umma_commit(bar_addr(sb, B_TP_EMPTY + tps));
+                        }
+                        __syncwarp();
+                    }
+                }
+                ok = grp.wait(bar_addr(sb, B_B_FULL), ph_b);
+                ph_b ^= 1u;
+                if (!ok) break;
+                tc_fence_after();
+                // --- -E^T as fp16 pairs: the A operand of the E half of MMA_C ---
+                {
+                    float ev[32];
+                    tmem_load32(tmem + TM_B + lane_addr, ev);
+                    uint32_t hpk[16];
+                    #pragma unroll
+                    for (int e = 0; e < 16; ++e) hpk[e] = pack_half2(-ev[2 * e], -ev[2 * e + 1]);
+                    tmem_st16(tmem + TM_E + lane_addr, hpk);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                grp.sync();
+                // --- MMA_C: S^T += V^T Kv - E^T Ke ---
+                if (warp == 8) {
+                    tc_fence_after();
+                    if (elect_one(mma_issuer)) {
+                        for (int k = 0; k < 2; ++k)
+                            umma_f16(tmem + TM_S, smem_desc_sw128(st + ST_V + k * 2048, 4096, 1024),
+                                     smem_desc_sw128(st + ST_KVE + k * 2048, 8192, 1024), ID_MM, 1);
+                        for (int k = 0; k < 2; ++k)
+                            umma_f16_tmem_a(tmem + TM_S, tmem + TM_E + 8 * k,
+                                            smem_desc_sw128(st + ST_KVE + 4096 + k * 2048, 8192, 1024), ID_TM, 1);
+                        umma_commit(bar_addr(sb, B_S_FULL));
+                        umma_commit(bar_addr(sb, B_EMPTY + s));
+                    }
+                    __syncwarp();
+                }
+                ok = grp.wait(bar_addr(sb, B_S_FULL), ph_s);
+                ph_s ^= 1u;
+                if (!ok) break;
+                tc_fence_after();
+            } else {
+                // --- out-of-range chunk: the definition, token by token, on the fp32 state ---
+                exact_chunk(tmem + TM_S + lane_addr, ExactIn{p.q, p.k, p.v, p.alpha, p.beta, p.o, p.out_bf16},
+                            static_cast<int64_t>(ug) * L + t0, n, j);
+                tc_fence_before();
+                // keep every hand-off in step: the stage and the [X; Z] stage are released
+                // once their producers are done with them, the output epilogue is released
+                ok = grp.wait(bar_addr(sb, B_CONV + s), ph, bar_addr(sb, B_TP_FULL + tps), (c >> 1) & 1);
+                if (!ok) break;
+                if (leader) {
+                    mbar_arrive(bar_addr(sb, B_EMPTY + s));
+                    mbar_arrive(bar_addr(sb, B_TP_EMPTY + tps));
+                    mbar_arrive(bar_addr(sb, B_O_READY));
+                }
+            }
+            // --- the new state ---
+            if (c + 1 == nchunks) {
+                if (p.S_out) store_final_state(tmem + TM_S + lane_addr, p.S_out + static_cast<int64_t>(ug) * kD * kD + j);
+                drain_needed = 0;
+            } else {
+                const int s1 = (c + 1) % kStages;
+                ok = grp.wait(bar_addr(sb, B_GATE_FULL + s1), ((c + 1) / kStages) & 1);
+                if (!ok) break;
+                const Gates* g1 = gate(s1);
+                const bool exact1 = !(g1->in_range[0] && g1->in_range[1]);
+                state_update(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr, exact1 ? nullptr : g1->decay);
+                tc_fence_before();
+            }
+            grp.sync();
+            if (leader) mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
+        }
+        if (warp == 8 && lane == mma_issuer && drain_needed && !ok) {
+            umma_commit(bar_addr(sb, B_DRAIN + 0));
+            mbar_wait(bar_addr(sb, B_DRAIN + 0), 0, abort_flag, err, kTimeoutNs / 4);
+        }
+    } else {
+        // ================= output epilogue: o = Q^ S - (the -O' half of MMA_B) =================
+        const int j = threadIdx.x - 384;
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+        Group grp{NB_OUT, 128, j == 0, okflags + 4, 0, abort_flag, err};
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % kStages;
+            if (j == 0) bulk_wait_read_all();
+            if (!grp.wait(bar_addr(sb, B_O_READY), c & 1)) break;
+            tc_fence_after();
+            const Gates* gs = gate(s);
+            const bool exact = !(gs->in_range[0] && gs->in_range[1]);
+            const int64_t t0 = static_cast<int64_t>(c) * kC;
+            if (!exact) {
+                if (!p.out_bf16) {
+                    const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
+                    store_o_f32(tmem + TM_AB + lane_addr + 32, tmem + TM_B + lane_addr + 32,
+                                static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, n);
+                } else {
+                    float qp[64];
+                    tmem_load_2x32(tmem + TM_AB + lane_addr + 32, tmem + TM_B + lane_addr + 32, qp);
+                    uint8_t* ost = sbase + OFF_OST + (j >> 6) * 4096 + (j & 63) * 2;
+                    #pragma unroll
+                    for (int r = 0; r < 32; ++r)
+                        *reinterpret_cast<__nv_bfloat16*>(ost + r * 128) = __float2bfloat16_rn(qp[r] - qp[32 + r]);
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            grp.sync();
+            if (j == 0) {
+                mbar_arrive(bar_addr(sb, B_O_DONE));
+                mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
+                if (!exact && p.out_bf16) {
+                    tma_store_3d(&tm_o, sb + OFF_OST, 0, static_cast<int32_t>(t0), ug);
+                    tma_store_3d(&tm_o, sb + OFF_OST + 4096, 64, static_cast<int32_t>(t0), ug);
+                    bulk_commit_group();
+                }
+            }
+        }
+        if (j == 0) bulk_wait_all();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, TM_COLS);
+}
+
+}  // namespace kda
+
+bool prefill_kda_tc_supports(int dtype_bf16, int dk, int dv)
+{
+    return dtype_bf16 && dk == kda::kD && dv == kda::kD;
+}
+
+cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream)
+{
+    using namespace kda;
+    if (call.units_per_loop == 0 || call.T == 0) return cudaSuccess;
+    const int64_t units = call.T * call.units_per_loop;
+    CUtensorMap mq, mk, mv, mo;
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!make_bf16_map_3d(&mq, call.q, units, call.L, kC, sw) || !make_bf16_map_3d(&mk, call.k, units, call.L, kC, sw) ||
+        !make_bf16_map_3d(&mv, call.v, units, call.L, kC, sw))
+        return cudaErrorInvalidValue;
+    if (call.out_bf16 && !make_bf16_map_3d(&mo, call.o, units, call.L, kC, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(gdr_prefill_kda_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(SMEM_BYTES));
+    if (e != cudaSuccess) return e;
+    for (int64_t tau = 0; tau < call.T; ++tau) {
+        Params p;
+        p.q = static_cast<const __nv_bfloat16*>(call.q);
+        p.k = static_cast<const __nv_bfloat16*>(call.k);
+        p.v = static_cast<const __nv_bfloat16*>(call.v);
+        p.alpha = call.alpha;
+        p.beta = call.beta;
+        p.S0 = call.S0;
+        p.o = call.o;
+        p.S_out = call.S_out;
+        p.L = call.L;
+        p.unit0 = static_cast<int>(tau * call.units_per_loop);
+        p.out_bf16 = call.out_bf16;
+        p.err = call.err;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(call.units_per_loop), 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = SMEM_BYTES;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = tau > 0 ? 1 : 0;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, gdr_prefill_kda_tc_kernel, mq, mk, mv, call.out_bf16 ? mo : mv, p);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace lt2

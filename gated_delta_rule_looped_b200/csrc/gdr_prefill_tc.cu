@@ -49,22 +49,22 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "gdr_common.cuh"
 #include "gdr_launch.h"
+#include "gdr_tc_common.cuh"
+#include "gdr_tma_host.h"
 #include "sm100_primitives.cuh"
 
 namespace lt2 {
 namespace tc {
 
 using namespace sm100;
+using namespace tcc;
 
 constexpr int kC = 64;                 // tokens per chunk
-constexpr int kD = 128;                // d_k = d_v
 constexpr int kThreads = 512;
 constexpr int kStages = 3;             // K/Q/V tile stages (and gate stages)
-constexpr uint64_t kTimeoutNs = 4000000000ull;   // 4 s
+constexpr uint64_t kTimeoutNs = kWaitTimeoutNs;
 
 // Shared memory map (offsets from a 1024-byte aligned base).  A K/Q/V stage holds, as fp16
 // after conversion, [K panel 0 | Q panel 0 | K panel 1 | Q panel 1 | V panel 0 | V panel 1],
@@ -79,7 +79,7 @@ constexpr uint32_t OFF_OST = OFF_TP + 2 * TP_STAGE;   // o staging for the TMA s
 constexpr uint32_t OFF_AS = OFF_OST + 16384;          // A (fp16) [64][64]
 constexpr uint32_t OFF_PS = OFF_AS + 8192;            // P (fp16) [64][64]
 constexpr uint32_t OFF_ADIAG = OFF_PS + 8192;         // diagonal 16x16 blocks of A, fp32, rows padded to 17
-constexpr uint32_t ADIAG_BLOCK = 16 * 17;
+constexpr uint32_t ADIAG_BLOCK = 16 * kAdiagRow;
 constexpr uint32_t OFF_GATES = OFF_ADIAG + 4608;
 constexpr uint32_t GATE_STAGE = 1536;
 constexpr uint32_t OFF_BAR = OFF_GATES + kStages * GATE_STAGE;
@@ -155,147 +155,6 @@ struct Params {
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t base, uint32_t i) { return base + OFF_BAR + 8u * i; }
 
-__device__ __forceinline__ void named_sync(int id, int nthreads)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// A group of warps that waits through one leader: the leader makes the bounded waits, the
-// group meets at its named barrier and every thread reads the outcome.  Two outcome slots
-// alternate, so the leader never overwrites a slot another thread has yet to read.
-struct Group {
-    int nb;             // named barrier id
-    int nthreads;
-    bool leader;
-    volatile int* slots;
-    uint32_t k;
-    volatile int* abort_flag;
-    unsigned int* err;
-
-    __device__ bool wait(uint32_t bar0, uint32_t par0, uint32_t bar1 = 0, uint32_t par1 = 0,
-                         uint32_t bar2 = 0, uint32_t par2 = 0)
-    {
-        volatile int* slot = slots + (k & 1u);
-        ++k;
-        if (leader) {
-            bool ok = mbar_wait(bar0, par0, abort_flag, err, kTimeoutNs);
-            if (ok && bar1) ok = mbar_wait(bar1, par1, abort_flag, err, kTimeoutNs);
-            if (ok && bar2) ok = mbar_wait(bar2, par2, abort_flag, err, kTimeoutNs);
-            *slot = ok ? 1 : 0;
-        }
-        named_sync(nb, nthreads);
-        return *slot != 0;
-    }
-    __device__ void sync() { named_sync(nb, nthreads); }
-};
-
-// --- prep helpers: 16x16 fp16 blocks of row-major 128B-swizzled tiles --------------------
-__device__ __forceinline__ void frag_a(uint32_t tile, int row0, int col0, int lane, uint32_t (&a)[4])
-{
-    const uint32_t row = row0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-    const uint32_t chunk = (col0 >> 3) + (lane >> 4);
-    ldsm_x4(sw128(tile, row, chunk), a);
-}
-__device__ __forceinline__ void frag_b(uint32_t tile, int k0, int n0, int lane, uint32_t (&b)[4])
-{
-    const uint32_t row = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-    const uint32_t chunk = (n0 >> 3) + (lane >> 4);
-    ldsm_x4_trans(sw128(tile, row, chunk), b);
-}
-__device__ __forceinline__ void mma_block(float (&c)[2][4], const uint32_t (&a)[4], const uint32_t (&b)[4])
-{
-    mma16816(c[0], a, b[0], b[1]);
-    mma16816(c[1], a, b[2], b[3]);
-}
-__device__ __forceinline__ void c_to_a(const float (&c)[2][4], uint32_t (&a)[4])
-{
-    a[0] = pack_half2(c[0][0], c[0][1]);
-    a[1] = pack_half2(c[0][2], c[0][3]);
-    a[2] = pack_half2(c[1][0], c[1][1]);
-    a[3] = pack_half2(c[1][2], c[1][3]);
-}
-__device__ __forceinline__ void store_block(uint32_t tile, int row0, int col0, int lane,
-                                            const float (&c)[2][4], float sign)
-{
-    const uint32_t g = lane >> 2, tq = lane & 3;
-    #pragma unroll
-    for (int nb = 0; nb < 2; ++nb) {
-        const uint32_t chunk = (col0 >> 3) + nb;
-        sts32(sw128(tile, row0 + g, chunk) + tq * 4, pack_half2(sign * c[nb][0], sign * c[nb][1]));
-        sts32(sw128(tile, row0 + g + 8, chunk) + tq * 4, pack_half2(sign * c[nb][2], sign * c[nb][3]));
-    }
-}
-__device__ __forceinline__ void zero_c(float (&c)[2][4])
-{
-    #pragma unroll
-    for (int i = 0; i < 2; ++i)
-        #pragma unroll
-        for (int j = 0; j < 4; ++j) c[i][j] = 0.f;
-}
-
-// Zeroes the entries above the diagonal of a diagonal 16x16 block held as an m16n8k16 A
-// fragment (a0: row g, columns 2tq..2tq+1; a1: row g+8, same columns; a2/a3: columns +8).
-__device__ __forceinline__ void keep_lower(uint32_t (&a)[4], int lane)
-{
-    const int g = lane >> 2, c0 = 2 * (lane & 3);
-    const uint32_t m = (c0 + 1 <= g) ? 0xffffffffu : ((c0 <= g) ? 0x0000ffffu : 0u);
-    a[0] &= m;
-    a[2] = 0u;
-    a[3] &= m;
-}
-
-// One 16-row block `rb` of X = [T; PT] (T = (I + A)^{-1}, rows 0..63; PT, rows 64..127).
-// X solves X (I + A) = [I; P]; with A strictly lower triangular this is a back substitution
-// over the 16-column blocks j = 3, 2, 1, 0:
-//     X_j = (E_j + sum_{k>j} X_k (-A)_{kj}) D_j,      D_j = (I + A_jj)^{-1}  (already in TP)
-// where E = I for the T rows and E = P for the PT rows, and X_j = 0 right of the diagonal
-// block (T_jj = D_j itself).  AS holds -A.  Each X_j goes to TP as soon as it is known and is
-// read back from there by the warp's later steps, so both loops stay rolled.
-__device__ __noinline__ void solve_row_block(uint32_t tp, uint32_t as, uint32_t ps, int rb, int lane)
-{
-    const bool is_t = rb < 4;
-    const int qd = is_t ? rb : rb - 4;          // diagonal column block of this row block
-    #pragma unroll 1
-    for (int j = is_t ? qd - 1 : qd; j >= 0; --j) {
-        float acc[2][4];
-        zero_c(acc);
-        #pragma unroll 1
-        for (int k = j + 1; k <= qd; ++k) {
-            uint32_t xa[4], b[4];
-            frag_a(tp, 16 * rb, 16 * k, lane, xa);
-            frag_b(as, 16 * k, 16 * j, lane, b);
-            mma_block(acc, xa, b);              // += X_k (-A)_kj
-        }
-        uint32_t dj[4];
-        frag_b(tp, 16 * j, 16 * j, lane, dj);
-        float x[2][4];
-        zero_c(x);
-        if (!is_t) {
-            uint32_t pa[4];
-            frag_a(ps, 16 * qd, 16 * j, lane, pa);
-            if (j == qd) keep_lower(pa, lane);
-            mma_block(x, pa, dj);               // P_qj D_j
-        }
-        if (j < qd) {
-            uint32_t aa[4];
-            c_to_a(acc, aa);
-            mma_block(x, aa, dj);
-        }
-        store_block(tp, 16 * rb, 16 * j, lane, x, 1.f);
-        __syncwarp();                           // X_j is read back by this warp's next steps
-    }
-}
-
-__device__ __forceinline__ uint4 pack8_half(const float* v)
-{
-    uint4 w;
-    w.x = pack_half2(v[0], v[1]);
-    w.y = pack_half2(v[2], v[3]);
-    w.z = pack_half2(v[4], v[5]);
-    w.w = pack_half2(v[6], v[7]);
-    return w;
-}
-
 // Gram products [K; Q] K^T of stage s (M=128, N=64, K=128) into TMEM, then commit.
 __device__ __forceinline__ void issue_gram(uint32_t sb, uint32_t tmem, int s)
 {
@@ -306,26 +165,6 @@ __device__ __forceinline__ void issue_gram(uint32_t sb, uint32_t tmem, int s)
                  ID_GRAM, k > 0);
     }
     umma_commit(bar_addr(sb, B_G_FULL));
-}
-
-// bf16 -> fp16, in place, for `n16` 16-byte vectors starting at shared address `base`.
-template <typename LdFn, typename StFn>
-__device__ __forceinline__ void convert_tile(uint32_t base, int n16, int lane, LdFn lds, StFn sts)
-{
-    for (int i0 = 0; i0 < n16; i0 += 8 * 32) {
-        uint4 w[8];
-        #pragma unroll
-        for (int i = 0; i < 8; ++i) w[i] = lds(base + static_cast<uint32_t>(i0 + i * 32 + lane) * 16u);
-        #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            uint4 hv;
-            hv.x = pack_half2(bf16_lo(w[i].x), bf16_hi(w[i].x));
-            hv.y = pack_half2(bf16_lo(w[i].y), bf16_hi(w[i].y));
-            hv.z = pack_half2(bf16_lo(w[i].z), bf16_hi(w[i].z));
-            hv.w = pack_half2(bf16_lo(w[i].w), bf16_hi(w[i].w));
-            sts(base + static_cast<uint32_t>(i0 + i * 32 + lane) * 16u, hv);
-        }
-    }
 }
 
 // ---- cold paths, kept out of line so that the per-chunk code stays compact ----------------
@@ -348,18 +187,6 @@ __device__ __noinline__ void load_initial_state(uint32_t tm_s, uint32_t tm_sh, c
         tmem_st32(tm_s + 32 * piece, v);
     }
     tmem_wait_st();
-}
-
-// Chain thread j: column j of the final state (row j of S^T in TMEM) to S_out.
-__device__ __noinline__ void store_final_state(uint32_t tm_s, float* so)
-{
-    #pragma unroll 1
-    for (int piece = 0; piece < 4; piece += 2) {
-        float v[64];
-        tmem_load_2x32(tm_s + 32 * piece, tm_s + 32 * piece + 32, v);
-        #pragma unroll
-        for (int d = 0; d < 64; ++d) so[(32 * piece + d) * kD] = v[d];
-    }
 }
 
 // Output thread j, fp32 output: o[r][j] = g_r (Q S)_rj + (P T X)_rj for the chunk's n tokens.
@@ -635,7 +462,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         // this warp's rows r = 32q..32q+31 have their diagonal blocks in columns
                         // 32h..32h+31: keep the fp32 copy for the diagonal inverses
                         const bool upper = (r & 16) != 0;
-                        float* ad = adiag + (r >> 4) * ADIAG_BLOCK + (r & 15) * 17;
+                        float* ad = adiag + (r >> 4) * ADIAG_BLOCK + (r & 15) * kAdiagRow;
                         #pragma unroll
                         for (int jj = 0; jj < 16; ++jj) ad[jj] = upper ? v[16 + jj] : v[jj];
                     }
@@ -644,7 +471,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
             } else {
                 gram_epilogue_unfactored(tmem + TM_G + lane_addr, gs, r, is_a, sbase + (dst - sb), dst,
-                                         adiag + (r >> 4) * ADIAG_BLOCK + (r & 15) * 17);
+                                         adiag + (r >> 4) * ADIAG_BLOCK + (r & 15) * kAdiagRow);
             }
             tc_fence_before();
             grp.sync();
@@ -654,25 +481,12 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             const uint32_t tp = sb + OFF_TP + tps * TP_STAGE;
             if (is_a) {
-                // row i of D_b = (I + A_bb)^{-1}:  x_j = delta_ij + sum_{m>j} x_m (-A)_mj, j = 15..0;
-                // the sum runs from m = 15 down so that only its last term waits for x_{j+1}
-                const int b = r >> 4, i = r & 15;
-                const float* ad = adiag + b * ADIAG_BLOCK;
-                float x[16];
-                #pragma unroll
-                for (int j = 15; j >= 0; --j) {
-                    float acc = 0.f;
-                    #pragma unroll
-                    for (int m = 15; m > j; --m) acc = fmaf(x[m], ad[m * 17 + j], acc);
-                    x[j] = (j == i) ? 1.f : ((j < i) ? acc : 0.f);
-                }
-                sts(sw128(tp, r, 2 * b), pack8_half(x));
-                sts(sw128(tp, r, 2 * b + 1), pack8_half(x + 8));
+                diag_block_inverse_row(tp, r, adiag + (r >> 4) * ADIAG_BLOCK);
             }
             grp.sync();
             // warp q: the T rows of block q and the PT rows of block 3 - q
-            solve_row_block(tp, as, ps, q, lane);
-            solve_row_block(tp, as, ps, 7 - q, lane);
+            solve_row_block(tp, as, ps, q, 4, lane);
+            solve_row_block(tp, as, ps, 7 - q, 4, lane);
             fence_proxy_async_smem();
             grp.sync();
             if (t == 0) mbar_arrive(bar_addr(sb, B_TP_FULL + tps));
@@ -899,46 +713,12 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
 // ---- host side ----------------------------------------------------------------------------
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(f);
-    });
-    return fn;
-}
-
-// 3-D view [units][L][128] of a bf16 tensor, boxes of 64 columns x 64 tokens x 1 unit,
-// 128-byte swizzle.  Rows past a unit's L are filled with zeros by the TMA unit.
-static bool make_map(CUtensorMap* m, const void* base, int64_t units, int64_t L,
-                     CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(L),
-                                static_cast<cuuint64_t>(units)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * 2, static_cast<cuuint64_t>(L) * kD * 2};
-    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kC), 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace tc
 
 bool prefill_tc_supports(int dtype_bf16, int dk, int dv, int per_key)
 {
-    return dtype_bf16 && dk == tc::kD && dv == tc::kD && !per_key;
+    if (per_key) return prefill_kda_tc_supports(dtype_bf16, dk, dv);
+    return dtype_bf16 && dk == tc::kD && dv == tc::kD;
 }
 
 cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
@@ -947,11 +727,12 @@ cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
     if (call.units_per_loop == 0 || call.T == 0) return cudaSuccess;
     const int64_t units = call.T * call.units_per_loop;
     CUtensorMap mq, mk, mv, mo;
-    if (!make_map(&mq, call.q, units, call.L) || !make_map(&mk, call.k, units, call.L) ||
-        !make_map(&mv, call.v, units, call.L))
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!make_bf16_map_3d(&mq, call.q, units, call.L, kC, sw) || !make_bf16_map_3d(&mk, call.k, units, call.L, kC, sw) ||
+        !make_bf16_map_3d(&mv, call.v, units, call.L, kC, sw))
         return cudaErrorInvalidValue;
     // o (bf16 output only): plain row-major tile, written by the TMA store from shared memory
-    if (call.out_bf16 && !make_map(&mo, call.o, units, call.L, CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (call.out_bf16 && !make_bf16_map_3d(&mo, call.o, units, call.L, kC, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(gdr_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM_BYTES));

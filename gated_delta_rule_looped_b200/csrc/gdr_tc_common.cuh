@@ -1,0 +1,215 @@
+// gdr_tc_common.cuh -- pieces shared by the tensor-core chunked prefills (scalar and per-key
+// gating): group waits, the 16x16-block helpers of the triangular solve on warp-level fp16
+// mma, the solve itself, the diagonal-block inverse and the in-place bf16 -> fp16 conversion.
+//
+// All tiles here are row-major fp16 with 128-byte rows under the 128-byte swizzle (`sw128`),
+// the layout the tcgen05 descriptors of both kernels use.
+#pragma once
+
+#include <cstdint>
+
+#include "sm100_primitives.cuh"
+
+namespace lt2 {
+namespace tcc {
+
+using namespace sm100;
+
+constexpr int kD = 128;                          // d_k = d_v
+constexpr uint64_t kWaitTimeoutNs = 4000000000ull;   // bound of every mbarrier wait (4 s)
+constexpr int kAdiagRow = 17;                    // fp32 diagonal blocks: rows padded to 17
+
+__device__ __forceinline__ void named_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// A group of warps that waits through one leader: the leader makes the bounded waits, the
+// group meets at its named barrier and every thread reads the outcome.  Two outcome slots
+// alternate, so the leader never overwrites a slot another thread has yet to read.
+struct Group {
+    int nb;             // named barrier id
+    int nthreads;
+    bool leader;
+    volatile int* slots;
+    uint32_t k;
+    volatile int* abort_flag;
+    unsigned int* err;
+
+    __device__ bool wait(uint32_t bar0, uint32_t par0, uint32_t bar1 = 0, uint32_t par1 = 0,
+                         uint32_t bar2 = 0, uint32_t par2 = 0)
+    {
+        volatile int* slot = slots + (k & 1u);
+        ++k;
+        if (leader) {
+            bool ok = mbar_wait(bar0, par0, abort_flag, err, kWaitTimeoutNs);
+            if (ok && bar1) ok = mbar_wait(bar1, par1, abort_flag, err, kWaitTimeoutNs);
+            if (ok && bar2) ok = mbar_wait(bar2, par2, abort_flag, err, kWaitTimeoutNs);
+            *slot = ok ? 1 : 0;
+        }
+        named_sync(nb, nthreads);
+        return *slot != 0;
+    }
+    __device__ void sync() { named_sync(nb, nthreads); }
+};
+
+// --- 16x16 fp16 blocks of row-major 128B-swizzled tiles, as m16n8k16 fragments ------------
+__device__ __forceinline__ void frag_a(uint32_t tile, int row0, int col0, int lane, uint32_t (&a)[4])
+{
+    const uint32_t row = row0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+    const uint32_t chunk = (col0 >> 3) + (lane >> 4);
+    ldsm_x4(sw128(tile, row, chunk), a);
+}
+__device__ __forceinline__ void frag_b(uint32_t tile, int k0, int n0, int lane, uint32_t (&b)[4])
+{
+    const uint32_t row = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+    const uint32_t chunk = (n0 >> 3) + (lane >> 4);
+    ldsm_x4_trans(sw128(tile, row, chunk), b);
+}
+__device__ __forceinline__ void mma_block(float (&c)[2][4], const uint32_t (&a)[4], const uint32_t (&b)[4])
+{
+    mma16816(c[0], a, b[0], b[1]);
+    mma16816(c[1], a, b[2], b[3]);
+}
+__device__ __forceinline__ void c_to_a(const float (&c)[2][4], uint32_t (&a)[4])
+{
+    a[0] = pack_half2(c[0][0], c[0][1]);
+    a[1] = pack_half2(c[0][2], c[0][3]);
+    a[2] = pack_half2(c[1][0], c[1][1]);
+    a[3] = pack_half2(c[1][2], c[1][3]);
+}
+__device__ __forceinline__ void store_block(uint32_t tile, int row0, int col0, int lane,
+                                            const float (&c)[2][4], float sign)
+{
+    const uint32_t g = lane >> 2, tq = lane & 3;
+    #pragma unroll
+    for (int nb = 0; nb < 2; ++nb) {
+        const uint32_t chunk = (col0 >> 3) + nb;
+        sts32(sw128(tile, row0 + g, chunk) + tq * 4, pack_half2(sign * c[nb][0], sign * c[nb][1]));
+        sts32(sw128(tile, row0 + g + 8, chunk) + tq * 4, pack_half2(sign * c[nb][2], sign * c[nb][3]));
+    }
+}
+__device__ __forceinline__ void zero_c(float (&c)[2][4])
+{
+    #pragma unroll
+    for (int i = 0; i < 2; ++i)
+        #pragma unroll
+        for (int j = 0; j < 4; ++j) c[i][j] = 0.f;
+}
+
+// Zeroes the entries above the diagonal of a diagonal 16x16 block held as an m16n8k16 A
+// fragment (a0: row g, columns 2tq..2tq+1; a1: row g+8, same columns; a2/a3: columns +8).
+__device__ __forceinline__ void keep_lower(uint32_t (&a)[4], int lane)
+{
+    const int g = lane >> 2, c0 = 2 * (lane & 3);
+    const uint32_t m = (c0 + 1 <= g) ? 0xffffffffu : ((c0 <= g) ? 0x0000ffffu : 0u);
+    a[0] &= m;
+    a[2] = 0u;
+    a[3] &= m;
+}
+
+__device__ __forceinline__ uint4 pack8_half(const float* v)
+{
+    uint4 w;
+    w.x = pack_half2(v[0], v[1]);
+    w.y = pack_half2(v[2], v[3]);
+    w.z = pack_half2(v[4], v[5]);
+    w.w = pack_half2(v[6], v[7]);
+    return w;
+}
+
+// One 16-row block `rb` of X = [T; PT] for a chunk of 16*nblk tokens: T = (I + A)^{-1} in rows
+// 0..16*nblk-1, PT below it.  X solves X (I + A) = [I; P]; with A strictly lower triangular
+// this is a back substitution over the 16-column blocks j = nblk-1, ..., 0:
+//     X_j = (E_j + sum_{k>j} X_k (-A)_{kj}) D_j,      D_j = (I + A_jj)^{-1}  (already in TP)
+// where E = I for the T rows and E = P for the PT rows, and X_j = 0 right of the diagonal
+// block (T_jj = D_j itself).  AS holds -A.  Each X_j goes to TP as soon as it is known and is
+// read back from there by the warp's later steps, so both loops stay rolled.
+static __device__ __noinline__ void solve_row_block(uint32_t tp, uint32_t as, uint32_t ps, int rb, int nblk, int lane)
+{
+    const bool is_t = rb < nblk;
+    const int qd = is_t ? rb : rb - nblk;       // diagonal column block of this row block
+    #pragma unroll 1
+    for (int j = is_t ? qd - 1 : qd; j >= 0; --j) {
+        float acc[2][4];
+        zero_c(acc);
+        #pragma unroll 1
+        for (int k = j + 1; k <= qd; ++k) {
+            uint32_t xa[4], b[4];
+            frag_a(tp, 16 * rb, 16 * k, lane, xa);
+            frag_b(as, 16 * k, 16 * j, lane, b);
+            mma_block(acc, xa, b);              // += X_k (-A)_kj
+        }
+        uint32_t dj[4];
+        frag_b(tp, 16 * j, 16 * j, lane, dj);
+        float x[2][4];
+        zero_c(x);
+        if (!is_t) {
+            uint32_t pa[4];
+            frag_a(ps, 16 * qd, 16 * j, lane, pa);
+            if (j == qd) keep_lower(pa, lane);
+            mma_block(x, pa, dj);               // P_qj D_j
+        }
+        if (j < qd) {
+            uint32_t aa[4];
+            c_to_a(acc, aa);
+            mma_block(x, aa, dj);
+        }
+        store_block(tp, 16 * rb, 16 * j, lane, x, 1.f);
+        __syncwarp();                           // X_j is read back by this warp's next steps
+    }
+}
+
+// Row i = r & 15 of D_b = (I + A_bb)^{-1}, b = r >> 4, from the fp32 copy `ad` of -A_bb (rows
+// padded to kAdiagRow): x_j = delta_ij + sum_{m>j} x_m (-A)_mj for j = 15..0.  The sum runs from
+// m = 15 down so that only its last term waits for x_{j+1}.  Written to row r, columns
+// 16b..16b+15 of the fp16 tile `tp`.
+__device__ __forceinline__ void diag_block_inverse_row(uint32_t tp, int r, const float* ad)
+{
+    const int b = r >> 4, i = r & 15;
+    float x[16];
+    #pragma unroll
+    for (int j = 15; j >= 0; --j) {
+        float acc = 0.f;
+        #pragma unroll
+        for (int m = 15; m > j; --m) acc = fmaf(x[m], ad[m * kAdiagRow + j], acc);
+        x[j] = (j == i) ? 1.f : ((j < i) ? acc : 0.f);
+    }
+    sts128(sw128(tp, r, 2 * b), pack8_half(x));
+    sts128(sw128(tp, r, 2 * b + 1), pack8_half(x + 8));
+}
+
+// bf16 -> fp16, in place, for `n16` 16-byte vectors starting at shared address `base`.
+template <typename LdFn, typename StFn>
+__device__ __forceinline__ void convert_tile(uint32_t base, int n16, int lane, LdFn lds, StFn sts)
+{
+    for (int i0 = 0; i0 < n16; i0 += 8 * 32) {
+        uint4 w[8];
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = lds(base + static_cast<uint32_t>(i0 + i * 32 + lane) * 16u);
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            uint4 hv;
+            hv.x = pack_half2(bf16_lo(w[i].x), bf16_hi(w[i].x));
+            hv.y = pack_half2(bf16_lo(w[i].y), bf16_hi(w[i].y));
+            hv.z = pack_half2(bf16_lo(w[i].z), bf16_hi(w[i].z));
+            hv.w = pack_half2(bf16_lo(w[i].w), bf16_hi(w[i].w));
+            sts(base + static_cast<uint32_t>(i0 + i * 32 + lane) * 16u, hv);
+        }
+    }
+}
+
+// Chain thread j: column j of the final state (row j of S^T in TMEM) to S_out.
+static __device__ __noinline__ void store_final_state(uint32_t tm_s, float* so)
+{
+    #pragma unroll 1
+    for (int piece = 0; piece < 4; piece += 2) {
+        float v[64];
+        tmem_load_2x32(tm_s + 32 * piece, tm_s + 32 * piece + 32, v);
+        #pragma unroll
+        for (int d = 0; d < 64; ++d) so[(32 * piece + d) * kD] = v[d];
+    }
+}
+
+}  // namespace tcc
+}  // namespace lt2

@@ -221,7 +221,8 @@ lt2_status lt2_gdr_prefill(const lt2_gdr_dims* dims, const void* q, const void* 
         call.L = dims->L;
         call.out_bf16 = out_is_bf16(dims) ? 1 : 0;
         call.err = err;
-        cudaError_t e = lt2::launch_prefill_tc_all(call, s);
+        cudaError_t e = dims->gate == LT2_GATE_PER_KEY ? lt2::launch_prefill_kda_tc_all(call, s)
+                                                       : lt2::launch_prefill_tc_all(call, s);
         if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "prefill (tensor core)");
         return LT2_OK;
