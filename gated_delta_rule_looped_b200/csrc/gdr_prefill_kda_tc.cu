@@ -33,7 +33,7 @@
 //
 // CTA = one (loop, batch, head) unit, 16 warps:
 //   warp 0       TMA producer (and TMEM allocation)
-//   warps 1, 2   per-key decay factors; K and Q tiles for keys 0..63 / 64..127 (eight fp16 tiles)
+//   warps 1, 2   per-key decay factors; K and Q tiles of tokens 0..15 / 16..31 (eight fp16 tiles)
 //   warp 3       fp16 conversion of V, and the Gram MMA
 //   warps 4-7    prep: Gram epilogue, diagonal-block inverses, back substitution, Z
 //   warps 8-11   the S-dependent chain (warp 8 issues MMA_A, MMA_B, MMA_C)
@@ -75,16 +75,17 @@ constexpr uint32_t OFF_STG = 0;
 // Gram stage (1): per panel [Kt (0-31) | Qt (32-63) | Be (64-95) | Bv (96-127)].
 constexpr uint32_t OFF_GRAM = OFF_STG + kStages * STAGE_BYTES;
 constexpr uint32_t GRAM_PANEL = 16384;
-// [X; Z] stages (2): X = [T; N_qe T] 64 rows, Z 64 rows, both 32 columns in 128-byte rows.
+// [X | Z] stages (2): 64 rows; X = [T; N_qe T] in columns 0-31, Z in columns 32-63.
 constexpr uint32_t OFF_TP = OFF_GRAM + 2 * GRAM_PANEL;
-constexpr uint32_t TP_STAGE = 16384;
-constexpr uint32_t TP_Z = 8192;
-// Gram blocks for the solve (32 rows each): -M_ke, N_qe, M_kv, N_qv.
-constexpr uint32_t OFF_MKE = OFF_TP + 2 * TP_STAGE;
-constexpr uint32_t OFF_NQE = OFF_MKE + 4096;
-constexpr uint32_t OFF_MKV = OFF_NQE + 4096;
-constexpr uint32_t OFF_NQV = OFF_MKV + 4096;
-constexpr uint32_t OFF_ADIAG = OFF_NQV + 4096;   // fp32 diagonal blocks of -M_ke
+constexpr uint32_t TP_STAGE = 8192;
+constexpr int TP_ZCOL = 32;
+// Gram blocks for the solve (32 rows each): [-M_ke | N_qe] and [M_kv | N_qv].
+constexpr uint32_t OFF_MA = OFF_TP + 2 * TP_STAGE;
+constexpr uint32_t OFF_MB = OFF_MA + 4096;
+// alpha of a chunk, [32 tokens][128] fp32, landed by TMA (2 stages).
+constexpr uint32_t OFF_ALPHA = OFF_MB + 4096;
+constexpr uint32_t ALPHA_STAGE = 16384;
+constexpr uint32_t OFF_ADIAG = OFF_ALPHA + 2 * ALPHA_STAGE;   // fp32 diagonal blocks of -M_ke
 constexpr uint32_t ADIAG_BLOCK = 16 * kAdiagRow;
 constexpr uint32_t OFF_OST = OFF_ADIAG + 2304;   // o staging: 2 x [32 tokens][64] bf16
 constexpr uint32_t OFF_GATES = OFF_OST + 8192;
@@ -96,7 +97,7 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 
 struct Gates {
     float decay[kD];   // e^{G_31}: the chunk's decay per key
-    int in_range[2];   // per conversion warp: Gram factors within range for its 64 keys
+    int in_range[2];   // per conversion warp: Gram factors within range for its 16 tokens
 };
 static_assert(sizeof(Gates) <= GATE_STAGE, "gate stage too small");
 
@@ -117,7 +118,9 @@ enum Bar : uint32_t {
     B_O_READY = 25,
     B_O_DONE = 26,
     B_DRAIN = 27,      // [2]
-    B_COUNT = 29
+    B_AL_FULL = 29,    // [2] TMA of a chunk's alpha landed
+    B_AL_EMPTY = 31,   // [2] conversion warps done with it
+    B_COUNT = 33
 };
 constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + B_COUNT * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 16;
@@ -159,90 +162,104 @@ struct Params {
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t base, uint32_t i) { return base + OFF_BAR + 8u * i; }
 
-__device__ __forceinline__ uint32_t pack_half2_scaled(uint32_t bf2, float f0, float f1)
+// ---- conversion: per-key decay factors and the eight fp16 tiles of one chunk --------------
+// Conversion warp w (1 or 2) converts tokens 16 (w-1) .. +15 of the chunk for all 128 keys;
+// lane l owns keys 4l .. 4l+3 (8 bytes of a row of panel l >> 4 of every 128-wide tile).
+// With P_t = e^{G_t} (P_-1 = 1), sq = sqrt(P_31), F_t = P_t / sq and R_t = 1 / F_t:
+//   K^_t = P_{t-1} k_t,  Q^_t = P_t q_t,  Kv_t = b_t sq R_t k_t,  Ke_t = b_t sq R_{t-1} k_t,
+//   Kt_t = F_{t-1} k_t,  Qt_t = F_t q_t,  Bv_t = b_t R_t k_t,      Be_t = b_t R_{t-1} k_t
+// (sq R_t = P_31 / P_t).  The loops stay rolled: this code runs once per chunk per warp and
+// would otherwise be fetched afresh every time.  Warp 1 writes the chunk decay P_31 of every
+// key to `decay`; the return value says whether every F_t of the warp's tokens lies in
+// [kFactorMin, kFactorMax].
+__device__ __forceinline__ float4 mul4(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
+__device__ __forceinline__ float4 scale4(float4 a, float s) { return make_float4(a.x * s, a.y * s, a.z * s, a.w * s); }
+__device__ __forceinline__ float4 rcp4(float4 a)
 {
-    return pack_half2(bf16_lo(bf2) * f0, bf16_hi(bf2) * f1);
+    return make_float4(rcp_approx(a.x), rcp_approx(a.y), rcp_approx(a.z), rcp_approx(a.w));
+}
+__device__ __forceinline__ float4 unpack4_bf16(uint2 w)
+{
+    return make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+}
+__device__ __forceinline__ uint2 pack4_scaled(float4 x, float4 f)
+{
+    return make_uint2(pack_half2(x.x * f.x, x.y * f.y), pack_half2(x.z * f.z, x.w * f.w));
+}
+__device__ __forceinline__ bool in_factor_range(float4 f)
+{
+    return fminf(fminf(f.x, f.y), fminf(f.z, f.w)) >= kFactorMin && fmaxf(fmaxf(f.x, f.y), fmaxf(f.z, f.w)) <= kFactorMax;
 }
 
-// ---- conversion: per-key decay factors and the eight fp16 tiles of one chunk --------------
-// Lane l of conversion warp w (1 or 2) owns keys i = 64 (w-1) + 2l, +1, i.e. 4 bytes of every
-// 128-byte row of panel w-1.  With P_t = e^{G_t} (P_-1 = 1), sq = sqrt(P_31), F_t = P_t / sq:
-//   K^_t = P_{t-1} k_t,  Q^_t = P_t q_t,  Kv_t = b_t (P_31 / P_t) k_t,  Ke_t = b_t (P_31 / P_{t-1}) k_t,
-//   Kt_t = F_{t-1} k_t,  Qt_t = F_t q_t,  Bv_t = b_t k_t / F_t,          Be_t = b_t k_t / F_{t-1}.
-// Returns the chunk decay P_31 of the lane's two keys, and whether every F_t lies in
-// [kFactorMin, kFactorMax] for both.
-struct ConvOut {
-    float2 decay;
-    bool in_range;
-};
-__device__ __noinline__ ConvOut convert_kq(uint32_t st, uint32_t gram, const float* alpha_u, const float* beta_u,
-                                           int n, int panel, int lane, uint8_t* sbase, uint32_t sb)
+// `alpha_c` is the chunk's alpha tile in shared memory ([32][128]); `bl` the beta of token
+// `lane` (0 beyond the chunk's end).
+__device__ __forceinline__ bool convert_kq(uint32_t st, uint32_t gram, const float* alpha_c, float bl, int n, int half,
+                                           int lane, uint8_t* sbase, uint32_t sb, float* decay)
 {
-    // beta of token `lane` (0 beyond the chunk's end)
-    const float bl = lane < n ? beta_u[lane] : 0.f;
-    const int koff = 64 * panel + 2 * lane;
-    // pass 1: the chunk's total decay per key
-    float2 P31 = make_float2(1.f, 1.f);
-    #pragma unroll 4
-    for (int t = 0; t < n; ++t) {
-        const float2 a = *reinterpret_cast<const float2*>(alpha_u + static_cast<int64_t>(t) * kD + koff);
-        P31.x *= a.x;
-        P31.y *= a.y;
-    }
-    const float2 sq = make_float2(sqrtf(P31.x), sqrtf(P31.y));
-    const float2 isq = make_float2(1.f / sq.x, 1.f / sq.y);
-    float2 P = make_float2(1.f, 1.f);          // P_{t-1}
-    float2 F = isq;                            // F_{t-1}
-    float2 R = sq;                             // 1 / F_{t-1}
-    float fmax_ = fmaxf(isq.x, isq.y), fmin_ = fminf(isq.x, isq.y);
-    const uint32_t chunk = static_cast<uint32_t>(lane >> 2);
-    const uint32_t within = static_cast<uint32_t>(lane & 3) * 4u;
-    auto at = [&](uint32_t tile, int row) -> uint32_t* {
-        return reinterpret_cast<uint32_t*>(sbase + (sw128(tile, row, chunk) + within - sb));
+    const float* arow = alpha_c + 4 * lane;
+    auto alpha4 = [&](int t) -> float4 {
+        return t < n ? *reinterpret_cast<const float4*>(arow + t * kD) : make_float4(1.f, 1.f, 1.f, 1.f);
     };
-    const uint32_t kq = st + ST_KQ + panel * 8192, kve = st + ST_KVE + panel * 8192;
-    const uint32_t gp = gram + panel * GRAM_PANEL;
+    const int t0 = 16 * half;
+    // products of alpha over the tokens before this half and over the whole chunk
+    float4 Pt = make_float4(1.f, 1.f, 1.f, 1.f), Ph = Pt;
     #pragma unroll 1
     for (int t = 0; t < kC; ++t) {
-        const float2 a = t < n ? *reinterpret_cast<const float2*>(alpha_u + static_cast<int64_t>(t) * kD + koff)
-                               : make_float2(1.f, 1.f);
+        if (t == t0) Ph = Pt;
+        Pt = mul4(Pt, alpha4(t));
+    }
+    const float4 isq = make_float4(rsqrt_approx(Pt.x), rsqrt_approx(Pt.y), rsqrt_approx(Pt.z), rsqrt_approx(Pt.w));
+    const float4 sq = mul4(Pt, isq);
+    if (half == 0) *reinterpret_cast<float4*>(decay + 4 * lane) = Pt;
+    float4 P = Ph;                               // P_{t-1}
+    float4 F = mul4(P, isq);                     // F_{t-1}
+    float4 R = rcp4(F);                          // 1 / F_{t-1}
+    bool ok = in_factor_range(F);
+    const int panel = lane >> 4;
+    const uint32_t chunk = static_cast<uint32_t>((lane & 15) >> 1), within = static_cast<uint32_t>(lane & 1) * 8u;
+    const uint32_t kq = st + ST_KQ + panel * 8192, kve = st + ST_KVE + panel * 8192;
+    const uint32_t gp = gram + panel * GRAM_PANEL;
+    auto at = [&](uint32_t tile, int row) -> uint2* {
+        return reinterpret_cast<uint2*>(sbase + (sw128(tile, row, chunk) + within - sb));
+    };
+    #pragma unroll 1
+    for (int t = t0; t < t0 + 16; ++t) {
+        const float4 a = alpha4(t);
         const float b = __shfl_sync(0xffffffffu, bl, t);
-        const float2 Pn = make_float2(P.x * a.x, P.y * a.y);          // P_t
-        const float2 Fn = make_float2(Pn.x * isq.x, Pn.y * isq.y);    // F_t
-        const float2 Rn = make_float2(1.f / Fn.x, 1.f / Fn.y);        // 1 / F_t
-        fmax_ = fmaxf(fmax_, fmaxf(Fn.x, Fn.y));
-        fmin_ = fminf(fmin_, fminf(Fn.x, Fn.y));
-        uint32_t* kp = at(kq, t);
-        uint32_t* qp = at(kq, 32 + t);
-        const uint32_t k2 = *kp, q2 = *qp;
-        *kp = pack_half2_scaled(k2, P.x, P.y);                              // K^ (in place)
-        *qp = pack_half2_scaled(q2, Pn.x, Pn.y);                            // Q^ (in place)
-        *at(kve, t) = pack_half2_scaled(k2, b * sq.x * Rn.x, b * sq.y * Rn.y);       // Kv
-        *at(kve, 32 + t) = pack_half2_scaled(k2, b * sq.x * R.x, b * sq.y * R.y);    // Ke
-        *at(gp, t) = pack_half2_scaled(k2, F.x, F.y);                       // Kt
-        *at(gp, 32 + t) = pack_half2_scaled(q2, Fn.x, Fn.y);                // Qt
-        *at(gp, 64 + t) = pack_half2_scaled(k2, b * R.x, b * R.y);          // Be
-        *at(gp, 96 + t) = pack_half2_scaled(k2, b * Rn.x, b * Rn.y);        // Bv
+        uint2* kp = at(kq, t);
+        uint2* qp = at(kq, 32 + t);
+        const float4 k = unpack4_bf16(*kp), q = unpack4_bf16(*qp);
+        const float4 Pn = mul4(P, a), Fn = mul4(Pn, isq), Rn = rcp4(Fn);
+        ok = ok && in_factor_range(Fn);
+        const float4 bRn = scale4(Rn, b), bR = scale4(R, b);
+        *kp = pack4_scaled(k, P);                               // K^ (in place)
+        *qp = pack4_scaled(q, Pn);                              // Q^ (in place)
+        *at(kve, t) = pack4_scaled(k, mul4(bRn, sq));           // Kv
+        *at(kve, 32 + t) = pack4_scaled(k, mul4(bR, sq));       // Ke
+        *at(gp, t) = pack4_scaled(k, F);                        // Kt
+        *at(gp, 32 + t) = pack4_scaled(q, Fn);                  // Qt
+        *at(gp, 64 + t) = pack4_scaled(k, bR);                  // Be
+        *at(gp, 96 + t) = pack4_scaled(k, bRn);                 // Bv
         P = Pn;
         F = Fn;
         R = Rn;
     }
-    return ConvOut{P, fmax_ <= kFactorMax && fmin_ >= kFactorMin};
+    return __all_sync(0xffffffffu, ok);
 }
 
 // ---- prep helpers (32-token chunk: two 16-token blocks) -----------------------------------
 
 // Gram epilogue, row r of the Kt rows (warp 4) or Qt rows (warp 5): the two 32-column halves
 // of the Gram row (against Be, against Bv), masked to s < r (Kt rows) or s <= r (Qt rows),
-// as fp16 rows of -M_ke / M_kv or N_qe / N_qv; the Kt rows also keep fp32 copies of the
-// diagonal 16x16 blocks of -M_ke.
+// as fp16 rows of -M_ke / M_kv (columns 0-31 of the MA / MB tiles) or N_qe / N_qv (columns
+// 32-63); the Kt rows also keep fp32 copies of the diagonal 16x16 blocks of -M_ke.
 __device__ __forceinline__ void gram_epilogue_row(const float (&v)[64], int r, bool kt_rows, uint8_t* sbase,
                                                   uint32_t sb, float* adiag)
 {
     const int lim = kt_rows ? r : r + 1;
     const float sg = kt_rows ? -1.f : 1.f;
-    const uint32_t t_e = sb + (kt_rows ? OFF_MKE : OFF_NQE);
-    const uint32_t t_v = sb + (kt_rows ? OFF_MKV : OFF_NQV);
+    const uint32_t t_e = sb + OFF_MA, t_v = sb + OFF_MB;
+    const int c0 = kt_rows ? 0 : 4;             // Kt rows in columns 0-31, Qt rows in 32-63
     float e[32], w[32];
     #pragma unroll
     for (int s = 0; s < 32; ++s) {
@@ -251,8 +268,8 @@ __device__ __forceinline__ void gram_epilogue_row(const float (&v)[64], int r, b
     }
     #pragma unroll
     for (int ch = 0; ch < 4; ++ch) {
-        *reinterpret_cast<uint4*>(sbase + (sw128(t_e, r, ch) - sb)) = pack8_half(e + 8 * ch);
-        *reinterpret_cast<uint4*>(sbase + (sw128(t_v, r, ch) - sb)) = pack8_half(w + 8 * ch);
+        *reinterpret_cast<uint4*>(sbase + (sw128(t_e, r, c0 + ch) - sb)) = pack8_half(e + 8 * ch);
+        *reinterpret_cast<uint4*>(sbase + (sw128(t_v, r, c0 + ch) - sb)) = pack8_half(w + 8 * ch);
     }
     if (kt_rows) {
         const bool upper = (r & 16) != 0;
@@ -262,8 +279,9 @@ __device__ __forceinline__ void gram_epilogue_row(const float (&v)[64], int r, b
     }
 }
 
-// Row block rb of Z = X M_kv - [0; N_qv] (X from TP, rows 0..63; M_kv strictly lower).
-__device__ __noinline__ void z_row_block(uint32_t tp, uint32_t mkv, uint32_t nqv, int rb, int lane)
+// Row block rb of Z = X M_kv - [0; N_qv] (X in columns 0-31 of TP, Z to columns 32-63; M_kv
+// and N_qv in columns 0-31 and 32-63 of MB; M_kv strictly lower).
+__device__ __noinline__ void z_row_block(uint32_t tp, uint32_t mb, int rb, int lane)
 {
     const bool is_t = rb < 2;
     const uint32_t g = lane >> 2, tq = lane & 3;
@@ -276,8 +294,8 @@ __device__ __noinline__ void z_row_block(uint32_t tp, uint32_t mkv, uint32_t nqv
             const int row0 = 16 * (rb - 2);
             #pragma unroll
             for (int nb = 0; nb < 2; ++nb) {
-                const uint32_t c0 = lds32(sw128(nqv, row0 + g, 2 * j + nb) + tq * 4);
-                const uint32_t c1 = lds32(sw128(nqv, row0 + g + 8, 2 * j + nb) + tq * 4);
+                const uint32_t c0 = lds32(sw128(mb, row0 + g, 4 + 2 * j + nb) + tq * 4);
+                const uint32_t c1 = lds32(sw128(mb, row0 + g + 8, 4 + 2 * j + nb) + tq * 4);
                 acc[nb][0] = -half_lo(c0);
                 acc[nb][1] = -half_hi(c0);
                 acc[nb][2] = -half_lo(c1);
@@ -289,10 +307,10 @@ __device__ __noinline__ void z_row_block(uint32_t tp, uint32_t mkv, uint32_t nqv
         for (int k = j; k <= kmax; ++k) {
             uint32_t a[4], b[4];
             frag_a(tp, 16 * rb, 16 * k, lane, a);
-            frag_b(mkv, 16 * k, 16 * j, lane, b);
+            frag_b(mb, 16 * k, 16 * j, lane, b);
             mma_block(acc, a, b);
         }
-        store_block(tp + TP_Z, 16 * rb, 16 * j, lane, acc, 1.f);
+        store_block(tp, 16 * rb, TP_ZCOL + 16 * j, lane, acc, 1.f);
     }
 }
 
@@ -450,7 +468,7 @@ __device__ __forceinline__ void issue_gram(uint32_t sb, uint32_t tmem)
 __global__ void __launch_bounds__(kThreads, 1)
 gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                          Params p)
+                          const __grid_constant__ CUtensorMap tm_a, Params p)
 {
     allow_next_loop_to_start();
 
@@ -484,6 +502,8 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             mbar_init(bar_addr(sb, B_TP_FULL + s), 1);
             mbar_init(bar_addr(sb, B_TP_EMPTY + s), 1);
             mbar_init(bar_addr(sb, B_DRAIN + s), 1);
+            mbar_init(bar_addr(sb, B_AL_FULL + s), 1);
+            mbar_init(bar_addr(sb, B_AL_EMPTY + s), 2);
         }
         mbar_init(bar_addr(sb, B_G_FULL), 1);
         mbar_init(bar_addr(sb, B_G_EMPTY), 1);
@@ -503,11 +523,11 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
             prefetch_tmap(&tm_o);
+            prefetch_tmap(&tm_a);
         }
     }
     if (warp >= 4 && warp < 8) {
-        // zero both [X; Z] stages once: blocks right of the diagonal and the unused columns
-        // 32..63 of every row are never written
+        // zero both [X | Z] stages once: the blocks of X right of its diagonal are never written
         const int t = threadIdx.x - 128;
         for (uint32_t off = t * 16; off < 2 * TP_STAGE; off += 128 * 16) sts(sb + OFF_TP + off, make_uint4(0, 0, 0, 0));
         fence_proxy_async_smem();
@@ -524,7 +544,9 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             const int s = c % kStages;
             const uint32_t ph = ((c / kStages) & 1) ^ 1;
             int free_ok = 0;
-            if (lane == 0) free_ok = mbar_wait(bar_addr(sb, B_EMPTY + s), ph, abort_flag, err, kTimeoutNs);
+            if (lane == 0)
+                free_ok = mbar_wait(bar_addr(sb, B_EMPTY + s), ph, abort_flag, err, kTimeoutNs) &&
+                          mbar_wait(bar_addr(sb, B_AL_EMPTY + (c & 1)), ((c >> 1) & 1) ^ 1, abort_flag, err, kTimeoutNs);
             if (!__shfl_sync(0xffffffffu, free_ok, 0)) break;
             uint32_t leader;
             if (elect_one(leader)) {
@@ -538,6 +560,9 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 tma_load_3d(st + ST_KQ + 8192 + 4096, &tm_q, 64, y, ug, fb);
                 tma_load_3d(st + ST_V, &tm_v, 0, y, ug, fb);
                 tma_load_3d(st + ST_V + 4096, &tm_v, 64, y, ug, fb);
+                const uint32_t ab = bar_addr(sb, B_AL_FULL + (c & 1));
+                mbar_arrive_expect_tx(ab, ALPHA_STAGE);
+                tma_load_3d(sb + OFF_ALPHA + (c & 1) * ALPHA_STAGE, &tm_a, 0, y, ug, ab);
             }
             __syncwarp();
             issued = c + 1;
@@ -545,6 +570,8 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         if (lane == 0 && *abort_flag) {
             for (int c = issued - kStages < 0 ? 0 : issued - kStages; c < issued; ++c)
                 mbar_wait(bar_addr(sb, B_FULL + c % kStages), (c / kStages) & 1, abort_flag, err, kTimeoutNs / 4);
+            for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c)
+                mbar_wait(bar_addr(sb, B_AL_FULL + (c & 1)), (c >> 1) & 1, abort_flag, err, kTimeoutNs / 4);
         }
     } else if (warp < 4) {
         // ================= decay factors and K/Q tiles (warps 1, 2), V and the Gram (warp 3) =====
@@ -556,24 +583,26 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             const uint32_t st = sb + OFF_STG + s * STAGE_BYTES;
             const int64_t t0 = static_cast<int64_t>(c) * kC;
             const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
+            // beta of token `lane` of this chunk: the load is issued before the waits below, which
+            // hide its latency
+            const float bl = (warp != 3 && lane < n) ? p.beta[static_cast<int64_t>(ug) * L + t0 + lane] : 0.f;
             int ok = 0;
             if (lane == 0) {
                 ok = mbar_wait(bar_addr(sb, B_FULL + s), ph, abort_flag, err, kTimeoutNs);
                 if (ok && warp != 3) {
                     ok = mbar_wait(bar_addr(sb, B_GATE_EMPTY + s), ph ^ 1, abort_flag, err, kTimeoutNs) &&
+                         mbar_wait(bar_addr(sb, B_AL_FULL + (c & 1)), (c >> 1) & 1, abort_flag, err, kTimeoutNs) &&
                          (c == 0 || mbar_wait(bar_addr(sb, B_GFREE), (c - 1) & 1, abort_flag, err, kTimeoutNs));
                 }
             }
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             if (warp != 3) {
                 const int panel = warp - 1;
-                const int64_t urow = static_cast<int64_t>(ug) * L + t0;
-                const ConvOut cv = convert_kq(st, sb + OFF_GRAM, p.alpha + urow * kD, p.beta + urow, n, panel, lane,
-                                              sbase, sb);
                 Gates* gs = gate(s);
-                *reinterpret_cast<float2*>(&gs->decay[64 * panel + 2 * lane]) = cv.decay;
-                const bool all_in = __all_sync(0xffffffffu, cv.in_range);
-                if (lane == 0) gs->in_range[panel] = all_in ? 1 : 0;
+                const bool in_range =
+                    convert_kq(st, sb + OFF_GRAM, reinterpret_cast<const float*>(sbase + OFF_ALPHA + (c & 1) * ALPHA_STAGE),
+                               bl, n, panel, lane, sbase, sb, gs->decay);
+                if (lane == 0) gs->in_range[panel] = in_range ? 1 : 0;
             } else {
                 #pragma unroll 1
                 for (int panel = 0; panel < 2; ++panel) convert_tile(st + ST_V + panel * 4096, 256, lane, lds, sts);
@@ -582,7 +611,10 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(bar_addr(sb, B_CONV + s));
-                if (warp != 3) mbar_arrive(bar_addr(sb, B_GATE_FULL + s));
+                if (warp != 3) {
+                    mbar_arrive(bar_addr(sb, B_GATE_FULL + s));
+                    mbar_arrive(bar_addr(sb, B_AL_EMPTY + (c & 1)));
+                }
             }
             if (warp == 3) {
                 int gram_ok = 0;
@@ -625,8 +657,8 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             if (q == 0) diag_block_inverse_row(tp, lane, adiag + (lane >> 4) * ADIAG_BLOCK);
             grp.sync();
             // warp q: row block q of X = [T; N_qe T] (T rows 0..31, then 32..63), then of Z
-            solve_row_block(tp, sb + OFF_MKE, sb + OFF_NQE, q, 2, lane);
-            z_row_block(tp, sb + OFF_MKV, sb + OFF_NQV, q, lane);
+            solve_row_block(tp, sb + OFF_MA, 0, sb + OFF_MA, 32, q, 2, lane);
+            z_row_block(tp, sb + OFF_MB, q, lane);
             fence_proxy_async_smem();
             grp.sync();
             if (t == 0) mbar_arrive(bar_addr(sb, B_TP_FULL + tps));
@@ -707,7 +739,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                         if (elect_one(mma_issuer)) {
                             for (int k = 0; k < 2; ++k)
                                 umma_f16(tmem + TM_B, smem_desc_sw128(st + ST_V + k * 2048, 4096, 1024),
-                                         smem_desc_sw128(tp + TP_Z + k * 32, 16, 1024), ID_M64, k > 0);
+                                         smem_desc_sw128(tp + 2 * TP_ZCOL + k * 32, 16, 1024), ID_M64, k > 0);
                             for (int k = 0; k < 2; ++k)
                                 umma_f16_tmem_a(tmem + TM_B, tmem + TM_Y + 8 * k, smem_desc_sw128(tp + k * 32, 16, 1024),
                                                 ID_T64, 1);
@@ -856,6 +888,8 @@ cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream)
         return cudaErrorInvalidValue;
     if (call.out_bf16 && !make_bf16_map_3d(&mo, call.o, units, call.L, kC, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
+    CUtensorMap ma;
+    if (!make_f32_map_3d(&ma, call.alpha, units, call.L, kC)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(gdr_prefill_kda_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess) return e;
@@ -883,7 +917,7 @@ cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream)
         attr[0].val.programmaticStreamSerializationAllowed = tau > 0 ? 1 : 0;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, gdr_prefill_kda_tc_kernel, mq, mk, mv, call.out_bf16 ? mo : mv, p);
+        e = cudaLaunchKernelEx(&cfg, gdr_prefill_kda_tc_kernel, mq, mk, mv, call.out_bf16 ? mo : mv, ma, p);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -485,8 +485,8 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             grp.sync();
             // warp q: the T rows of block q and the PT rows of block 3 - q
-            solve_row_block(tp, as, ps, q, 4, lane);
-            solve_row_block(tp, as, ps, 7 - q, 4, lane);
+            solve_row_block(tp, as, 0, ps, 0, q, 4, lane);
+            solve_row_block(tp, as, 0, ps, 0, 7 - q, 4, lane);
             fence_proxy_async_smem();
             grp.sync();
             if (t == 0) mbar_arrive(bar_addr(sb, B_TP_FULL + tps));

@@ -124,8 +124,10 @@ __device__ __forceinline__ uint4 pack8_half(const float* v)
 //     X_j = (E_j + sum_{k>j} X_k (-A)_{kj}) D_j,      D_j = (I + A_jj)^{-1}  (already in TP)
 // where E = I for the T rows and E = P for the PT rows, and X_j = 0 right of the diagonal
 // block (T_jj = D_j itself).  AS holds -A.  Each X_j goes to TP as soon as it is known and is
-// read back from there by the warp's later steps, so both loops stay rolled.
-static __device__ __noinline__ void solve_row_block(uint32_t tp, uint32_t as, uint32_t ps, int rb, int nblk, int lane)
+// read back from there by the warp's later steps, so both loops stay rolled.  -A and P start
+// at columns as_col / ps_col of their tiles (two 32-column matrices may share 128-byte rows).
+static __device__ __noinline__ void solve_row_block(uint32_t tp, uint32_t as, int as_col, uint32_t ps, int ps_col,
+                                                    int rb, int nblk, int lane)
 {
     const bool is_t = rb < nblk;
     const int qd = is_t ? rb : rb - nblk;       // diagonal column block of this row block
@@ -137,7 +139,7 @@ static __device__ __noinline__ void solve_row_block(uint32_t tp, uint32_t as, ui
         for (int k = j + 1; k <= qd; ++k) {
             uint32_t xa[4], b[4];
             frag_a(tp, 16 * rb, 16 * k, lane, xa);
-            frag_b(as, 16 * k, 16 * j, lane, b);
+            frag_b(as, 16 * k, as_col + 16 * j, lane, b);
             mma_block(acc, xa, b);              // += X_k (-A)_kj
         }
         uint32_t dj[4];
@@ -146,7 +148,7 @@ static __device__ __noinline__ void solve_row_block(uint32_t tp, uint32_t as, ui
         zero_c(x);
         if (!is_t) {
             uint32_t pa[4];
-            frag_a(ps, 16 * qd, 16 * j, lane, pa);
+            frag_a(ps, 16 * qd, ps_col + 16 * j, lane, pa);
             if (j == qd) keep_lower(pa, lane);
             mma_block(x, pa, dj);               // P_qj D_j
         }

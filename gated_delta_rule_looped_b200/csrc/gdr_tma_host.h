@@ -47,4 +47,19 @@ inline bool make_bf16_map_3d(CUtensorMap* m, const void* base, int64_t units, in
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D view [units][L][128] of an fp32 tensor (per-key gates), boxes of all 128 columns x
+// `box_rows` tokens x 1 unit, no swizzle (a 512-byte row per token).
+inline bool make_f32_map_3d(CUtensorMap* m, const void* base, int64_t units, int64_t L, uint32_t box_rows)
+{
+    EncodeTiledFn fn = tma_encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(units)};
+    const cuuint64_t strides[2] = {128 * 4, static_cast<cuuint64_t>(L) * 128 * 4};
+    const cuuint32_t box[3] = {128, box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace lt2

@@ -353,6 +353,20 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
 }
 
 // Two bf16 in one 32-bit word -> two floats (exact).
+// Approximate reciprocal (one MUFU instruction, relative error ~2^-22; denormals flush to 0).
+__device__ __forceinline__ float rcp_approx(float x)
+{
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// Approximate reciprocal square root (one MUFU instruction, relative error ~2^-22).
+__device__ __forceinline__ float rsqrt_approx(float x)
+{
+    float y;
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __device__ __forceinline__ uint32_t lds32(uint32_t addr)
 {
     uint32_t v;
