@@ -17,11 +17,12 @@
 //   N_qe[r,s] = beta_s q_r^T Gamma_r Gamma_{s-1}^{-1} k_s  (s <= r),     N_qv: Gamma_s^{-1} (s <= r).
 //
 // (Checked in fp64 against the sequential definition by the test suite's chunked oracle.)
-// Every factor in the state-side operands K^, Q^, Kv, Ke is at most 1, so they are always
-// representable in fp16.  The four chunk Gram matrices are products of two fp16 tiles that
-// carry e^{G - R} and e^{R - G} around a per-key reference R = G_31 / 2, which stays in
-// range while a key decays by at most e^-19 over the chunk.  A chunk beyond that (or with any
-// alpha outside (0, 1]) is instead run token by token, exactly, on the fp32 state in TMEM.
+// K^ and Q^ carry factors of at most 1.  The four chunk Gram matrices are products of fp16
+// tiles Kt, Qt and Be, Bv that carry e^{G - R} and e^{R - G} around a per-key reference
+// R = G_31 / 2; Be and Bv also serve the state update (Kv = sq Bv, Ke = sq Be, sq = e^{G_31/2}).
+// The tiles stay in range while a key decays by at most e^-19 over the chunk.  A chunk beyond
+// that (or with any alpha outside (0, 1]) is instead run token by token, exactly, on the fp32
+// state in TMEM.
 //
 // With the solve X = [T; N_qe T], T = (I + M_ke)^{-1}, and Z = X M_kv - [0; N_qv]:
 //   [E; -(O - Q^ S)] = X (K^ S) + Z V,
@@ -29,11 +30,13 @@
 // quantities (one d_v column per TMEM lane):
 //   MMA_A  (K^ S, Q^ S)^T    = S^T [K^; Q^]^T          A = S^T (TMEM, fp16)   N = 64
 //   MMA_B  ([E; -O'])^T      = V^T Z^T + (K^ S)^T X^T  A = V^T (smem), then (K^ S)^T (TMEM)
-//   MMA_C  S^T (pre-scaled by Gamma_31) += V^T Kv - E^T Ke
+//   MMA_C  (sq S)^T += V^T Bv - E^T Be, giving (S' / sq)^T
+// where sq = sqrt(P_31) per key and Bv, Be are the Gram tiles below: Kv = sq Bv, Ke = sq Be, so
+// the fp32 state in TMEM is kept scaled by sq (per key, i.e. per TMEM column) around MMA_C.
 //
 // CTA = one (loop, batch, head) unit, 16 warps:
 //   warp 0       TMA producer (and TMEM allocation)
-//   warps 1, 2   per-key decay factors; K and Q tiles of tokens 0..15 / 16..31 (eight fp16 tiles)
+//   warps 1, 2   per-key decay factors; K and Q tiles of tokens 0..15 / 16..31 (six fp16 tiles)
 //   warp 3       fp16 conversion of V, and the Gram MMA
 //   warps 4-7    prep: Gram epilogue, diagonal-block inverses, back substitution, Z
 //   warps 8-11   the S-dependent chain (warp 8 issues MMA_A, MMA_B, MMA_C)
@@ -65,14 +68,15 @@ constexpr float kFactorMin = 1.f / 16384.f;
 
 // Shared memory map (offsets from a 1024-byte aligned base).  Tiles are fp16, 128-byte rows
 // (64 elements) under the 128-byte swizzle; a 128-wide operand is two panels.
-// Chunk stage (3): [K^ | Q^] x 2 panels (rows 0-31 K^, 32-63 Q^), [Kv | Ke] x 2 panels, V x 2.
+// Chunk stage (3): [K^ | Q^] x 2 panels (rows 0-31 K^, 32-63 Q^), [Be | Bv] x 2 panels, V x 2.
 constexpr uint32_t ST_KQ = 0;          // + panel * 8192
 constexpr uint32_t ST_KVE = 16384;     // + panel * 8192
 constexpr uint32_t ST_V = 32768;       // + panel * 4096
 constexpr uint32_t STAGE_BYTES = 40960;
 constexpr uint32_t STAGE_TX = 6 * 4096;   // K, Q, V boxes of 64 columns x 32 tokens (bf16)
 constexpr uint32_t OFF_STG = 0;
-// Gram stage (1): per panel [Kt (0-31) | Qt (32-63) | Be (64-95) | Bv (96-127)].
+// Gram stage (1): per panel [Kt (0-31) | Qt (32-63)]; the Gram reads 128 rows (the other 64 are
+// never written and only reach TMEM lanes that are not read).
 constexpr uint32_t OFF_GRAM = OFF_STG + kStages * STAGE_BYTES;
 constexpr uint32_t GRAM_PANEL = 16384;
 // [X | Z] stages (2): 64 rows; X = [T; N_qe T] in columns 0-31, Z in columns 32-63.
@@ -96,7 +100,7 @@ constexpr uint32_t SMEM_USED = OFF_BAR + BAR_BYTES;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 
 struct Gates {
-    float decay[kD];   // e^{G_31}: the chunk's decay per key
+    float sq[kD];      // sqrt(e^{G_31}): square root of the chunk's decay per key
     int in_range[2];   // per conversion warp: Gram factors within range for its 16 tokens
 };
 static_assert(sizeof(Gates) <= GATE_STAGE, "gate stage too small");
@@ -131,7 +135,7 @@ constexpr int NB_PREP = 1, NB_CHAIN = 2, NB_OUT = 3;
 
 // TMEM columns (lane j = d_v index in the chain's regions).
 constexpr uint32_t TM_G = 0;           // Gram (64 columns; lanes 0-31 Kt rows, 32-63 Qt rows)
-constexpr uint32_t TM_S = 64;          // S^T fp32, pre-scaled by the chunk decay (128)
+constexpr uint32_t TM_S = 64;          // S^T fp32, scaled per key by sq around MMA_C (128)
 constexpr uint32_t TM_SH = 192;        // S^T fp16 pairs (64): A operand of MMA_A
 constexpr uint32_t TM_AB = 256;        // (K^ S)^T 256..287, (Q^ S)^T 288..319
 constexpr uint32_t TM_Y = 256;         //   (K^ S)^T as fp16 pairs (16), A operand of MMA_B
@@ -162,16 +166,16 @@ struct Params {
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t base, uint32_t i) { return base + OFF_BAR + 8u * i; }
 
-// ---- conversion: per-key decay factors and the eight fp16 tiles of one chunk --------------
+// ---- conversion: per-key decay factors and the six fp16 tiles of one chunk ----------------
 // Conversion warp w (1 or 2) converts tokens 16 (w-1) .. +15 of the chunk for all 128 keys;
 // lane l owns keys 4l .. 4l+3 (8 bytes of a row of panel l >> 4 of every 128-wide tile).
 // With P_t = e^{G_t} (P_-1 = 1), sq = sqrt(P_31), F_t = P_t / sq and R_t = 1 / F_t:
-//   K^_t = P_{t-1} k_t,  Q^_t = P_t q_t,  Kv_t = b_t sq R_t k_t,  Ke_t = b_t sq R_{t-1} k_t,
-//   Kt_t = F_{t-1} k_t,  Qt_t = F_t q_t,  Bv_t = b_t R_t k_t,      Be_t = b_t R_{t-1} k_t
-// (sq R_t = P_31 / P_t).  The loops stay rolled: this code runs once per chunk per warp and
-// would otherwise be fetched afresh every time.  Warp 1 writes the chunk decay P_31 of every
-// key to `decay`; the return value says whether every F_t of the warp's tokens lies in
-// [kFactorMin, kFactorMax].
+//   K^_t = P_{t-1} k_t,  Q^_t = P_t q_t,  Kt_t = F_{t-1} k_t,  Qt_t = F_t q_t,
+//   Bv_t = b_t R_t k_t,  Be_t = b_t R_{t-1} k_t
+// (the state products need Kv = sq Bv and Ke = sq Be: sq R_t = P_31 / P_t).  The loops stay
+// rolled: this code runs once per chunk per warp and would otherwise be fetched afresh every
+// time.  Warp 1 writes sq of every key to `sq_out`; the return value says whether every F_t of
+// the warp's tokens lies in [kFactorMin, kFactorMax].
 __device__ __forceinline__ float4 mul4(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
 __device__ __forceinline__ float4 scale4(float4 a, float s) { return make_float4(a.x * s, a.y * s, a.z * s, a.w * s); }
 __device__ __forceinline__ float4 rcp4(float4 a)
@@ -194,7 +198,7 @@ __device__ __forceinline__ bool in_factor_range(float4 f)
 // `alpha_c` is the chunk's alpha tile in shared memory ([32][128]); `bl` the beta of token
 // `lane` (0 beyond the chunk's end).
 __device__ __forceinline__ bool convert_kq(uint32_t st, uint32_t gram, const float* alpha_c, float bl, int n, int half,
-                                           int lane, uint8_t* sbase, uint32_t sb, float* decay)
+                                           int lane, uint8_t* sbase, uint32_t sb, float* sq_out)
 {
     const float* arow = alpha_c + 4 * lane;
     auto alpha4 = [&](int t) -> float4 {
@@ -204,42 +208,42 @@ __device__ __forceinline__ bool convert_kq(uint32_t st, uint32_t gram, const flo
     // products of alpha over the tokens before this half and over the whole chunk
     float4 Pt = make_float4(1.f, 1.f, 1.f, 1.f), Ph = Pt;
     #pragma unroll 1
-    for (int t = 0; t < kC; ++t) {
-        if (t == t0) Ph = Pt;
-        Pt = mul4(Pt, alpha4(t));
+    for (int t8 = 0; t8 < kC; t8 += 8) {
+        if (t8 == t0) Ph = Pt;
+        float4 a[8];
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = alpha4(t8 + i);    // the eight loads issue together
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) Pt = mul4(Pt, a[i]);
     }
     const float4 isq = make_float4(rsqrt_approx(Pt.x), rsqrt_approx(Pt.y), rsqrt_approx(Pt.z), rsqrt_approx(Pt.w));
-    const float4 sq = mul4(Pt, isq);
-    if (half == 0) *reinterpret_cast<float4*>(decay + 4 * lane) = Pt;
+    if (half == 0) *reinterpret_cast<float4*>(sq_out + 4 * lane) = mul4(Pt, isq);
     float4 P = Ph;                               // P_{t-1}
     float4 F = mul4(P, isq);                     // F_{t-1}
     float4 R = rcp4(F);                          // 1 / F_{t-1}
     bool ok = in_factor_range(F);
+    // the eight bytes of row t this lane owns, in every tile (rows 32 + t: +4096 bytes)
     const int panel = lane >> 4;
     const uint32_t chunk = static_cast<uint32_t>((lane & 15) >> 1), within = static_cast<uint32_t>(lane & 1) * 8u;
-    const uint32_t kq = st + ST_KQ + panel * 8192, kve = st + ST_KVE + panel * 8192;
-    const uint32_t gp = gram + panel * GRAM_PANEL;
-    auto at = [&](uint32_t tile, int row) -> uint2* {
-        return reinterpret_cast<uint2*>(sbase + (sw128(tile, row, chunk) + within - sb));
-    };
+    uint8_t* kq = sbase + (st + ST_KQ + panel * 8192 - sb);
+    uint8_t* bve = sbase + (st + ST_KVE + panel * 8192 - sb);
+    uint8_t* gp = sbase + (gram + panel * GRAM_PANEL - sb);
     #pragma unroll 1
     for (int t = t0; t < t0 + 16; ++t) {
         const float4 a = alpha4(t);
         const float b = __shfl_sync(0xffffffffu, bl, t);
-        uint2* kp = at(kq, t);
-        uint2* qp = at(kq, 32 + t);
+        const uint32_t off = sw128(0u, t, chunk) + within;
+        uint2* kp = reinterpret_cast<uint2*>(kq + off);
+        uint2* qp = reinterpret_cast<uint2*>(kq + off + 4096);
         const float4 k = unpack4_bf16(*kp), q = unpack4_bf16(*qp);
         const float4 Pn = mul4(P, a), Fn = mul4(Pn, isq), Rn = rcp4(Fn);
         ok = ok && in_factor_range(Fn);
-        const float4 bRn = scale4(Rn, b), bR = scale4(R, b);
-        *kp = pack4_scaled(k, P);                               // K^ (in place)
-        *qp = pack4_scaled(q, Pn);                              // Q^ (in place)
-        *at(kve, t) = pack4_scaled(k, mul4(bRn, sq));           // Kv
-        *at(kve, 32 + t) = pack4_scaled(k, mul4(bR, sq));       // Ke
-        *at(gp, t) = pack4_scaled(k, F);                        // Kt
-        *at(gp, 32 + t) = pack4_scaled(q, Fn);                  // Qt
-        *at(gp, 64 + t) = pack4_scaled(k, bR);                  // Be
-        *at(gp, 96 + t) = pack4_scaled(k, bRn);                 // Bv
+        *kp = pack4_scaled(k, P);                                               // K^ (in place)
+        *qp = pack4_scaled(q, Pn);                                              // Q^ (in place)
+        *reinterpret_cast<uint2*>(gp + off) = pack4_scaled(k, F);               // Kt
+        *reinterpret_cast<uint2*>(gp + off + 4096) = pack4_scaled(q, Fn);       // Qt
+        *reinterpret_cast<uint2*>(bve + off) = pack4_scaled(k, scale4(R, b));   // Be
+        *reinterpret_cast<uint2*>(bve + off + 4096) = pack4_scaled(k, scale4(Rn, b));   // Bv
         P = Pn;
         F = Fn;
         R = Rn;
@@ -317,8 +321,8 @@ __device__ __noinline__ void z_row_block(uint32_t tp, uint32_t mb, int rb, int l
 // ---- chain helpers --------------------------------------------------------------------------
 
 // Chain thread j: S0^T row j into TMEM, as fp16 pairs (unscaled) and as fp32 scaled per
-// column i (= key) by decay[i] (nullptr: unscaled).
-__device__ __noinline__ void load_initial_state(uint32_t tm_s, uint32_t tm_sh, const float* s0, const float* decay)
+// column i (= key) by f[i] (nullptr: unscaled).
+__device__ __noinline__ void load_initial_state(uint32_t tm_s, uint32_t tm_sh, const float* s0, const float* f)
 {
     #pragma unroll 1
     for (int piece = 0; piece < 4; ++piece) {
@@ -329,42 +333,67 @@ __device__ __noinline__ void load_initial_state(uint32_t tm_s, uint32_t tm_sh, c
         #pragma unroll
         for (int e = 0; e < 16; ++e) hpk[e] = pack_half2(v[2 * e], v[2 * e + 1]);
         tmem_st16(tm_sh + 16 * piece, hpk);
-        if (decay) {
+        if (f) {
             #pragma unroll
-            for (int d = 0; d < 32; ++d) v[d] *= decay[32 * piece + d];
+            for (int d = 0; d < 32; ++d) v[d] *= f[32 * piece + d];
         }
         tmem_st32(tm_s + 32 * piece, v);
     }
     tmem_wait_st();
 }
 
-// Chain thread j: the new state's fp16 copy (for MMA_A) and the fp32 state scaled per column
-// by the next chunk's decay (nullptr: unscaled, the next chunk runs token by token).
-__device__ __forceinline__ void state_update(uint32_t tm_s, uint32_t tm_sh, const float* decay)
+// Chain thread j, after a chunk: the state S' = f_sh (.) TM_S (per column i = key; nullptr: 1)
+// as fp16 pairs for MMA_A, and TM_S <- f_s (.) S' (nullptr: 1), the pre-scaled state the next
+// chunk's MMA_C accumulates into.
+__device__ __forceinline__ void state_update(uint32_t tm_s, uint32_t tm_sh, const float* f_sh, const float* f_s)
 {
     #pragma unroll 1
     for (int piece = 0; piece < 4; piece += 2) {
         float v[64];
         tmem_load_2x32(tm_s + 32 * piece, tm_s + 32 * piece + 32, v);
-        uint32_t hpk[32];
-        #pragma unroll
-        for (int e = 0; e < 32; ++e) hpk[e] = pack_half2(v[2 * e], v[2 * e + 1]);
-        tmem_st16(tm_sh + 16 * piece, *reinterpret_cast<uint32_t(*)[16]>(hpk));
-        tmem_st16(tm_sh + 16 * piece + 16, *reinterpret_cast<uint32_t(*)[16]>(hpk + 16));
-        if (decay) {
+        if (f_sh) {
             #pragma unroll
             for (int d4 = 0; d4 < 64; d4 += 4) {
-                const float4 f = *reinterpret_cast<const float4*>(decay + 32 * piece + d4);
+                const float4 f = *reinterpret_cast<const float4*>(f_sh + 32 * piece + d4);
                 v[d4 + 0] *= f.x;
                 v[d4 + 1] *= f.y;
                 v[d4 + 2] *= f.z;
                 v[d4 + 3] *= f.w;
             }
+        }
+        uint32_t hpk[32];
+        #pragma unroll
+        for (int e = 0; e < 32; ++e) hpk[e] = pack_half2(v[2 * e], v[2 * e + 1]);
+        tmem_st16(tm_sh + 16 * piece, *reinterpret_cast<uint32_t(*)[16]>(hpk));
+        tmem_st16(tm_sh + 16 * piece + 16, *reinterpret_cast<uint32_t(*)[16]>(hpk + 16));
+        if (f_s) {
+            #pragma unroll
+            for (int d4 = 0; d4 < 64; d4 += 4) {
+                const float4 f = *reinterpret_cast<const float4*>(f_s + 32 * piece + d4);
+                v[d4 + 0] *= f.x;
+                v[d4 + 1] *= f.y;
+                v[d4 + 2] *= f.z;
+                v[d4 + 3] *= f.w;
+            }
+        }
+        if (f_sh || f_s) {
             tmem_st32(tm_s + 32 * piece, *reinterpret_cast<float(*)[32]>(v));
             tmem_st32(tm_s + 32 * piece + 32, *reinterpret_cast<float(*)[32]>(v + 32));
         }
     }
     tmem_wait_st();
+}
+
+// Chain thread j: column j of the final state, f (.) TM_S (nullptr: 1), to S_out.
+__device__ __noinline__ void store_final_state_scaled(uint32_t tm_s, float* so, const float* f)
+{
+    #pragma unroll 1
+    for (int piece = 0; piece < 4; piece += 2) {
+        float v[64];
+        tmem_load_2x32(tm_s + 32 * piece, tm_s + 32 * piece + 32, v);
+        #pragma unroll
+        for (int d = 0; d < 64; ++d) so[(32 * piece + d) * kD] = f ? v[d] * f[32 * piece + d] : v[d];
+    }
 }
 
 // Chain thread j: the chunk's n tokens run one at a time on column j of the fp32 state in
@@ -451,15 +480,15 @@ __device__ __noinline__ void store_o_f32(uint32_t tm_qs, uint32_t tm_b, float* o
         if (r < n) o[r * kD] = qp[r] - qp[32 + r];
 }
 
-// Gram [Kt; Qt; Be; Bv] [Be; Bv]^T (M = 128, N = 64, K = 128) into TMEM; only lanes 0-63 are
-// used.  Commits the Gram barrier and the release of the Gram tiles.
-__device__ __forceinline__ void issue_gram(uint32_t sb, uint32_t tmem)
+// Gram [Kt; Qt; -] [Be; Bv]^T (M = 128, N = 64, K = 128) into TMEM, Be and Bv from the chunk
+// stage `st`; only lanes 0-63 are read.  Commits the Gram barrier and the release of the Gram
+// tiles.
+__device__ __forceinline__ void issue_gram(uint32_t sb, uint32_t tmem, uint32_t st)
 {
     const uint32_t g = sb + OFF_GRAM;
     for (int k = 0; k < 8; ++k) {
-        const uint32_t off = (k >> 2) * GRAM_PANEL + (k & 3) * 32;
-        umma_f16(tmem + TM_G, smem_desc_sw128(g + off, 16, 1024), smem_desc_sw128(g + 8192 + off, 16, 1024),
-                 ID_GRAM, k > 0);
+        umma_f16(tmem + TM_G, smem_desc_sw128(g + (k >> 2) * GRAM_PANEL + (k & 3) * 32, 16, 1024),
+                 smem_desc_sw128(st + ST_KVE + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), ID_GRAM, k > 0);
     }
     umma_commit(bar_addr(sb, B_G_FULL));
     umma_commit(bar_addr(sb, B_GFREE));
@@ -601,7 +630,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 Gates* gs = gate(s);
                 const bool in_range =
                     convert_kq(st, sb + OFF_GRAM, reinterpret_cast<const float*>(sbase + OFF_ALPHA + (c & 1) * ALPHA_STAGE),
-                               bl, n, panel, lane, sbase, sb, gs->decay);
+                               bl, n, panel, lane, sbase, sb, gs->sq);
                 if (lane == 0) gs->in_range[panel] = in_range ? 1 : 0;
             } else {
                 #pragma unroll 1
@@ -623,7 +652,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                               (c == 0 || mbar_wait(bar_addr(sb, B_G_EMPTY), (c - 1) & 1, abort_flag, err, kTimeoutNs));
                 if (__shfl_sync(0xffffffffu, gram_ok, 0)) {
                     tc_fence_after();
-                    if (elect_one(gram_issuer)) issue_gram(sb, tmem);
+                    if (elect_one(gram_issuer)) issue_gram(sb, tmem, st);
                     __syncwarp();
                     gram_issued = 1;
                 }
@@ -677,7 +706,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             const bool exact0 = !(g0->in_range[0] && g0->in_range[1]);
             load_initial_state(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr,
                                p.S0 ? p.S0 + static_cast<int64_t>(ug) * kD * kD + j : nullptr,
-                               exact0 ? nullptr : g0->decay);
+                               exact0 ? nullptr : g0->sq);
             tc_fence_before();
         }
         uint32_t drain_needed = 0;
@@ -766,16 +795,16 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 }
                 tc_fence_before();
                 grp.sync();
-                // --- MMA_C: S^T += V^T Kv - E^T Ke ---
+                // --- MMA_C: (sq S)^T += V^T Bv - E^T Be ---
                 if (warp == 8) {
                     tc_fence_after();
                     if (elect_one(mma_issuer)) {
                         for (int k = 0; k < 2; ++k)
                             umma_f16(tmem + TM_S, smem_desc_sw128(st + ST_V + k * 2048, 4096, 1024),
-                                     smem_desc_sw128(st + ST_KVE + k * 2048, 8192, 1024), ID_MM, 1);
+                                     smem_desc_sw128(st + ST_KVE + 4096 + k * 2048, 8192, 1024), ID_MM, 1);
                         for (int k = 0; k < 2; ++k)
                             umma_f16_tmem_a(tmem + TM_S, tmem + TM_E + 8 * k,
-                                            smem_desc_sw128(st + ST_KVE + 4096 + k * 2048, 8192, 1024), ID_TM, 1);
+                                            smem_desc_sw128(st + ST_KVE + k * 2048, 8192, 1024), ID_TM, 1);
                         umma_commit(bar_addr(sb, B_S_FULL));
                         umma_commit(bar_addr(sb, B_EMPTY + s));
                     }
@@ -801,8 +830,11 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 }
             }
             // --- the new state ---
+            // TM_S holds S' / sq after a tensor-core chunk, S' itself after an exact one
+            const float* f_sh = exact ? nullptr : gs->sq;
             if (c + 1 == nchunks) {
-                if (p.S_out) store_final_state(tmem + TM_S + lane_addr, p.S_out + static_cast<int64_t>(ug) * kD * kD + j);
+                if (p.S_out)
+                    store_final_state_scaled(tmem + TM_S + lane_addr, p.S_out + static_cast<int64_t>(ug) * kD * kD + j, f_sh);
                 drain_needed = 0;
             } else {
                 const int s1 = (c + 1) % kStages;
@@ -810,7 +842,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 if (!ok) break;
                 const Gates* g1 = gate(s1);
                 const bool exact1 = !(g1->in_range[0] && g1->in_range[1]);
-                state_update(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr, exact1 ? nullptr : g1->decay);
+                state_update(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr, f_sh, exact1 ? nullptr : g1->sq);
                 tc_fence_before();
             }
             grp.sync();
