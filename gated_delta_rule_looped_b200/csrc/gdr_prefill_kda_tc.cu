@@ -36,8 +36,8 @@
 //
 // CTA = one (loop, batch, head) unit, 16 warps:
 //   warp 0       TMA producer (and TMEM allocation)
-//   warps 1, 2   per-key decay factors; K and Q tiles of tokens 0..15 / 16..31 (six fp16 tiles)
-//   warp 3       fp16 conversion of V, and the Gram MMA
+//   warps 1-3    per-key decay factors; K and Q tiles of tokens 0-10 / 11-21 / 22-31 (six fp16
+//                tiles); warp 3 also converts V to fp16 and issues the Gram MMA
 //   warps 4-7    prep: Gram epilogue, diagonal-block inverses, back substitution, Z
 //   warps 8-11   the S-dependent chain (warp 8 issues MMA_A, MMA_B, MMA_C)
 //   warps 12-15  output epilogue
@@ -101,7 +101,7 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 
 struct Gates {
     float sq[kD];      // sqrt(e^{G_31}): square root of the chunk's decay per key
-    int in_range[2];   // per conversion warp: Gram factors within range for its 16 tokens
+    int in_range[3];   // per conversion warp: Gram factors within range for its tokens
 };
 static_assert(sizeof(Gates) <= GATE_STAGE, "gate stage too small");
 
@@ -109,7 +109,7 @@ enum Bar : uint32_t {
     B_FULL = 0,        // [3] TMA of a stage landed
     B_CONV = 3,        // [3] stage and Gram tiles converted (warps 1, 2, 3)
     B_EMPTY = 6,       // [3] chain done with a stage
-    B_GATE_FULL = 9,   // [3] decay factors written (warps 1, 2)
+    B_GATE_FULL = 9,   // [3] decay factors written (warps 1, 2, 3)
     B_GATE_EMPTY = 12, // [3] chain and output epilogue done with a gate stage
     B_TP_FULL = 15,    // [2]
     B_TP_EMPTY = 17,   // [2]
@@ -167,15 +167,16 @@ struct Params {
 __device__ __forceinline__ uint32_t bar_addr(uint32_t base, uint32_t i) { return base + OFF_BAR + 8u * i; }
 
 // ---- conversion: per-key decay factors and the six fp16 tiles of one chunk ----------------
-// Conversion warp w (1 or 2) converts tokens 16 (w-1) .. +15 of the chunk for all 128 keys;
-// lane l owns keys 4l .. 4l+3 (8 bytes of a row of panel l >> 4 of every 128-wide tile).
+// Conversion warp w (1, 2, 3) converts tokens [t_begin, t_end) of the chunk (11, 11 and 10
+// tokens) for all 128 keys; lane l owns keys 4l .. 4l+3 (8 bytes of a row of panel l >> 4 of
+// every 128-wide tile).
 // With P_t = e^{G_t} (P_-1 = 1), sq = sqrt(P_31), F_t = P_t / sq and R_t = 1 / F_t:
 //   K^_t = P_{t-1} k_t,  Q^_t = P_t q_t,  Kt_t = F_{t-1} k_t,  Qt_t = F_t q_t,
 //   Bv_t = b_t R_t k_t,  Be_t = b_t R_{t-1} k_t
 // (the state products need Kv = sq Bv and Ke = sq Be: sq R_t = P_31 / P_t).  The loops stay
 // rolled: this code runs once per chunk per warp and would otherwise be fetched afresh every
-// time.  Warp 1 writes sq of every key to `sq_out`; the return value says whether every F_t of
-// the warp's tokens lies in [kFactorMin, kFactorMax].
+// time.  The warp starting at token 0 writes sq of every key to `sq_out`; the return value says
+// whether every F_t of the warp's tokens lies in [kFactorMin, kFactorMax].
 __device__ __forceinline__ float4 mul4(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
 __device__ __forceinline__ float4 scale4(float4 a, float s) { return make_float4(a.x * s, a.y * s, a.z * s, a.w * s); }
 __device__ __forceinline__ float4 rcp4(float4 a)
@@ -197,27 +198,28 @@ __device__ __forceinline__ bool in_factor_range(float4 f)
 
 // `alpha_c` is the chunk's alpha tile in shared memory ([32][128]); `bl` the beta of token
 // `lane` (0 beyond the chunk's end).
-__device__ __forceinline__ bool convert_kq(uint32_t st, uint32_t gram, const float* alpha_c, float bl, int n, int half,
-                                           int lane, uint8_t* sbase, uint32_t sb, float* sq_out)
+__device__ __forceinline__ bool convert_kq(uint32_t st, uint32_t gram, const float* alpha_c, float bl, int n,
+                                           int t_begin, int t_end, int lane, uint8_t* sbase, uint32_t sb, float* sq_out)
 {
     const float* arow = alpha_c + 4 * lane;
     auto alpha4 = [&](int t) -> float4 {
         return t < n ? *reinterpret_cast<const float4*>(arow + t * kD) : make_float4(1.f, 1.f, 1.f, 1.f);
     };
-    const int t0 = 16 * half;
-    // products of alpha over the tokens before this half and over the whole chunk
+    // products of alpha over the tokens before t_begin and over the whole chunk
     float4 Pt = make_float4(1.f, 1.f, 1.f, 1.f), Ph = Pt;
     #pragma unroll 1
     for (int t8 = 0; t8 < kC; t8 += 8) {
-        if (t8 == t0) Ph = Pt;
         float4 a[8];
         #pragma unroll
         for (int i = 0; i < 8; ++i) a[i] = alpha4(t8 + i);    // the eight loads issue together
         #pragma unroll
-        for (int i = 0; i < 8; ++i) Pt = mul4(Pt, a[i]);
+        for (int i = 0; i < 8; ++i) {
+            if (t8 + i == t_begin) Ph = Pt;
+            Pt = mul4(Pt, a[i]);
+        }
     }
     const float4 isq = make_float4(rsqrt_approx(Pt.x), rsqrt_approx(Pt.y), rsqrt_approx(Pt.z), rsqrt_approx(Pt.w));
-    if (half == 0) *reinterpret_cast<float4*>(sq_out + 4 * lane) = mul4(Pt, isq);
+    if (t_begin == 0) *reinterpret_cast<float4*>(sq_out + 4 * lane) = mul4(Pt, isq);
     float4 P = Ph;                               // P_{t-1}
     float4 F = mul4(P, isq);                     // F_{t-1}
     float4 R = rcp4(F);                          // 1 / F_{t-1}
@@ -229,7 +231,7 @@ __device__ __forceinline__ bool convert_kq(uint32_t st, uint32_t gram, const flo
     uint8_t* bve = sbase + (st + ST_KVE + panel * 8192 - sb);
     uint8_t* gp = sbase + (gram + panel * GRAM_PANEL - sb);
     #pragma unroll 1
-    for (int t = t0; t < t0 + 16; ++t) {
+    for (int t = t_begin; t < t_end; ++t) {
         const float4 a = alpha4(t);
         const float b = __shfl_sync(0xffffffffu, bl, t);
         const uint32_t off = sw128(0u, t, chunk) + within;
@@ -524,7 +526,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             mbar_init(bar_addr(sb, B_FULL + s), 1);
             mbar_init(bar_addr(sb, B_CONV + s), 3);
             mbar_init(bar_addr(sb, B_EMPTY + s), 1);
-            mbar_init(bar_addr(sb, B_GATE_FULL + s), 2);
+            mbar_init(bar_addr(sb, B_GATE_FULL + s), 3);
             mbar_init(bar_addr(sb, B_GATE_EMPTY + s), 2);
         }
         for (int s = 0; s < 2; ++s) {
@@ -532,7 +534,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             mbar_init(bar_addr(sb, B_TP_EMPTY + s), 1);
             mbar_init(bar_addr(sb, B_DRAIN + s), 1);
             mbar_init(bar_addr(sb, B_AL_FULL + s), 1);
-            mbar_init(bar_addr(sb, B_AL_EMPTY + s), 2);
+            mbar_init(bar_addr(sb, B_AL_EMPTY + s), 3);
         }
         mbar_init(bar_addr(sb, B_G_FULL), 1);
         mbar_init(bar_addr(sb, B_G_EMPTY), 1);
@@ -603,9 +605,11 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 mbar_wait(bar_addr(sb, B_AL_FULL + (c & 1)), (c >> 1) & 1, abort_flag, err, kTimeoutNs / 4);
         }
     } else if (warp < 4) {
-        // ================= decay factors and K/Q tiles (warps 1, 2), V and the Gram (warp 3) =====
+        // ================= decay factors and K/Q tiles (warps 1-3), V and the Gram (warp 3) ======
         uint32_t gram_issuer = 0;
         int gram_issued = 0;
+        const int w = warp - 1;                     // 0, 1, 2: tokens [11w, min(11w + 11, 32))
+        const int t_begin = 11 * w, t_end = w == 2 ? kC : 11 * w + 11;
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;
             const uint32_t ph = (c / kStages) & 1;
@@ -614,25 +618,20 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
             // beta of token `lane` of this chunk: the load is issued before the waits below, which
             // hide its latency
-            const float bl = (warp != 3 && lane < n) ? p.beta[static_cast<int64_t>(ug) * L + t0 + lane] : 0.f;
+            const float bl = lane < n ? p.beta[static_cast<int64_t>(ug) * L + t0 + lane] : 0.f;
             int ok = 0;
-            if (lane == 0) {
-                ok = mbar_wait(bar_addr(sb, B_FULL + s), ph, abort_flag, err, kTimeoutNs);
-                if (ok && warp != 3) {
-                    ok = mbar_wait(bar_addr(sb, B_GATE_EMPTY + s), ph ^ 1, abort_flag, err, kTimeoutNs) &&
-                         mbar_wait(bar_addr(sb, B_AL_FULL + (c & 1)), (c >> 1) & 1, abort_flag, err, kTimeoutNs) &&
-                         (c == 0 || mbar_wait(bar_addr(sb, B_GFREE), (c - 1) & 1, abort_flag, err, kTimeoutNs));
-                }
-            }
+            if (lane == 0)
+                ok = mbar_wait(bar_addr(sb, B_FULL + s), ph, abort_flag, err, kTimeoutNs) &&
+                     mbar_wait(bar_addr(sb, B_GATE_EMPTY + s), ph ^ 1, abort_flag, err, kTimeoutNs) &&
+                     mbar_wait(bar_addr(sb, B_AL_FULL + (c & 1)), (c >> 1) & 1, abort_flag, err, kTimeoutNs) &&
+                     (c == 0 || mbar_wait(bar_addr(sb, B_GFREE), (c - 1) & 1, abort_flag, err, kTimeoutNs));
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            if (warp != 3) {
-                const int panel = warp - 1;
-                Gates* gs = gate(s);
-                const bool in_range =
-                    convert_kq(st, sb + OFF_GRAM, reinterpret_cast<const float*>(sbase + OFF_ALPHA + (c & 1) * ALPHA_STAGE),
-                               bl, n, panel, lane, sbase, sb, gs->sq);
-                if (lane == 0) gs->in_range[panel] = in_range ? 1 : 0;
-            } else {
+            Gates* gs = gate(s);
+            const bool in_range =
+                convert_kq(st, sb + OFF_GRAM, reinterpret_cast<const float*>(sbase + OFF_ALPHA + (c & 1) * ALPHA_STAGE),
+                           bl, n, t_begin, t_end, lane, sbase, sb, gs->sq);
+            if (lane == 0) gs->in_range[w] = in_range ? 1 : 0;
+            if (warp == 3) {
                 #pragma unroll 1
                 for (int panel = 0; panel < 2; ++panel) convert_tile(st + ST_V + panel * 4096, 256, lane, lds, sts);
             }
@@ -640,10 +639,8 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(bar_addr(sb, B_CONV + s));
-                if (warp != 3) {
-                    mbar_arrive(bar_addr(sb, B_GATE_FULL + s));
-                    mbar_arrive(bar_addr(sb, B_AL_EMPTY + (c & 1)));
-                }
+                mbar_arrive(bar_addr(sb, B_GATE_FULL + s));
+                mbar_arrive(bar_addr(sb, B_AL_EMPTY + (c & 1)));
             }
             if (warp == 3) {
                 int gram_ok = 0;
@@ -703,7 +700,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         if (ok) ok = grp.wait(bar_addr(sb, B_GATE_FULL + 0), 0);
         if (ok) {
             const Gates* g0 = gate(0);
-            const bool exact0 = !(g0->in_range[0] && g0->in_range[1]);
+            const bool exact0 = !(g0->in_range[0] && g0->in_range[1] && g0->in_range[2]);
             load_initial_state(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr,
                                p.S0 ? p.S0 + static_cast<int64_t>(ug) * kD * kD + j : nullptr,
                                exact0 ? nullptr : g0->sq);
@@ -720,7 +717,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             const int64_t t0 = static_cast<int64_t>(c) * kC;
             const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
             const Gates* gs = gate(s);
-            const bool exact = !(gs->in_range[0] && gs->in_range[1]);
+            const bool exact = !(gs->in_range[0] && gs->in_range[1] && gs->in_range[2]);
             if (!exact) {
                 // --- MMA_A: (K^ S, Q^ S)^T = S^T [K^; Q^]^T ---
                 grp.sync();
@@ -841,7 +838,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 ok = grp.wait(bar_addr(sb, B_GATE_FULL + s1), ((c + 1) / kStages) & 1);
                 if (!ok) break;
                 const Gates* g1 = gate(s1);
-                const bool exact1 = !(g1->in_range[0] && g1->in_range[1]);
+                const bool exact1 = !(g1->in_range[0] && g1->in_range[1] && g1->in_range[2]);
                 state_update(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr, f_sh, exact1 ? nullptr : g1->sq);
                 tc_fence_before();
             }
@@ -863,7 +860,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             if (!grp.wait(bar_addr(sb, B_O_READY), c & 1)) break;
             tc_fence_after();
             const Gates* gs = gate(s);
-            const bool exact = !(gs->in_range[0] && gs->in_range[1]);
+            const bool exact = !(gs->in_range[0] && gs->in_range[1] && gs->in_range[2]);
             const int64_t t0 = static_cast<int64_t>(c) * kC;
             if (!exact) {
                 if (!p.out_bf16) {
