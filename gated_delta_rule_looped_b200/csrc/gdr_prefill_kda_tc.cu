@@ -75,10 +75,12 @@ constexpr uint32_t ST_V = 32768;       // + panel * 4096
 constexpr uint32_t STAGE_BYTES = 40960;
 constexpr uint32_t STAGE_TX = 6 * 4096;   // K, Q, V boxes of 64 columns x 32 tokens (bf16)
 constexpr uint32_t OFF_STG = 0;
-// Gram stage (1): per panel [Kt (0-31) | Qt (32-63)]; the Gram reads 128 rows (the other 64 are
-// never written and only reach TMEM lanes that are not read).
+// Gram tiles, two buffers: buffer b holds [Kt (rows 64b + 0-31) | Qt (64b + 32-63)] of each panel.
+// The Gram reads 128 rows from its buffer's first row; the 64 rows past the buffer (the other
+// buffer, or the next region) reach only TMEM lanes that are never read.
 constexpr uint32_t OFF_GRAM = OFF_STG + kStages * STAGE_BYTES;
 constexpr uint32_t GRAM_PANEL = 16384;
+constexpr uint32_t GRAM_BUF = 8192;
 // [X | Z] stages (2): 64 rows; X = [T; N_qe T] in columns 0-31, Z in columns 32-63.
 constexpr uint32_t OFF_TP = OFF_GRAM + 2 * GRAM_PANEL;
 constexpr uint32_t TP_STAGE = 8192;
@@ -115,16 +117,16 @@ enum Bar : uint32_t {
     B_TP_EMPTY = 17,   // [2]
     B_G_FULL = 19,     // Gram in TMEM
     B_G_EMPTY = 20,    // Gram read out
-    B_GFREE = 21,      // Gram MMA done reading the Gram tiles
-    B_A_FULL = 22,
-    B_B_FULL = 23,
-    B_S_FULL = 24,
-    B_O_READY = 25,
-    B_O_DONE = 26,
-    B_DRAIN = 27,      // [2]
-    B_AL_FULL = 29,    // [2] TMA of a chunk's alpha landed
-    B_AL_EMPTY = 31,   // [2] conversion warps done with it
-    B_COUNT = 33
+    B_GFREE = 21,      // [2] Gram MMA done reading a Gram tile buffer
+    B_A_FULL = 23,
+    B_B_FULL = 24,
+    B_S_FULL = 25,
+    B_O_READY = 26,
+    B_O_DONE = 27,
+    B_DRAIN = 28,      // [2]
+    B_AL_FULL = 30,    // [2] TMA of a chunk's alpha landed
+    B_AL_EMPTY = 32,   // [2] conversion warps done with it
+    B_COUNT = 34
 };
 constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + B_COUNT * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 16;
@@ -485,15 +487,15 @@ __device__ __noinline__ void store_o_f32(uint32_t tm_qs, uint32_t tm_b, float* o
 // Gram [Kt; Qt; -] [Be; Bv]^T (M = 128, N = 64, K = 128) into TMEM, Be and Bv from the chunk
 // stage `st`; only lanes 0-63 are read.  Commits the Gram barrier and the release of the Gram
 // tiles.
-__device__ __forceinline__ void issue_gram(uint32_t sb, uint32_t tmem, uint32_t st)
+__device__ __forceinline__ void issue_gram(uint32_t sb, uint32_t tmem, uint32_t st, int gbuf)
 {
-    const uint32_t g = sb + OFF_GRAM;
+    const uint32_t g = sb + OFF_GRAM + gbuf * GRAM_BUF;
     for (int k = 0; k < 8; ++k) {
         umma_f16(tmem + TM_G, smem_desc_sw128(g + (k >> 2) * GRAM_PANEL + (k & 3) * 32, 16, 1024),
                  smem_desc_sw128(st + ST_KVE + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), ID_GRAM, k > 0);
     }
     umma_commit(bar_addr(sb, B_G_FULL));
-    umma_commit(bar_addr(sb, B_GFREE));
+    umma_commit(bar_addr(sb, B_GFREE + gbuf));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -538,7 +540,8 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         }
         mbar_init(bar_addr(sb, B_G_FULL), 1);
         mbar_init(bar_addr(sb, B_G_EMPTY), 1);
-        mbar_init(bar_addr(sb, B_GFREE), 1);
+        mbar_init(bar_addr(sb, B_GFREE + 0), 1);
+        mbar_init(bar_addr(sb, B_GFREE + 1), 1);
         mbar_init(bar_addr(sb, B_A_FULL), 1);
         mbar_init(bar_addr(sb, B_B_FULL), 1);
         mbar_init(bar_addr(sb, B_S_FULL), 1);
@@ -624,11 +627,12 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 ok = mbar_wait(bar_addr(sb, B_FULL + s), ph, abort_flag, err, kTimeoutNs) &&
                      mbar_wait(bar_addr(sb, B_GATE_EMPTY + s), ph ^ 1, abort_flag, err, kTimeoutNs) &&
                      mbar_wait(bar_addr(sb, B_AL_FULL + (c & 1)), (c >> 1) & 1, abort_flag, err, kTimeoutNs) &&
-                     (c == 0 || mbar_wait(bar_addr(sb, B_GFREE), (c - 1) & 1, abort_flag, err, kTimeoutNs));
+                     mbar_wait(bar_addr(sb, B_GFREE + (c & 1)), ((c >> 1) & 1) ^ 1, abort_flag, err, kTimeoutNs);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             Gates* gs = gate(s);
             const bool in_range =
-                convert_kq(st, sb + OFF_GRAM, reinterpret_cast<const float*>(sbase + OFF_ALPHA + (c & 1) * ALPHA_STAGE),
+                convert_kq(st, sb + OFF_GRAM + (c & 1) * GRAM_BUF,
+                           reinterpret_cast<const float*>(sbase + OFF_ALPHA + (c & 1) * ALPHA_STAGE),
                            bl, n, t_begin, t_end, lane, sbase, sb, gs->sq);
             if (lane == 0) gs->in_range[w] = in_range ? 1 : 0;
             if (warp == 3) {
@@ -649,7 +653,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                               (c == 0 || mbar_wait(bar_addr(sb, B_G_EMPTY), (c - 1) & 1, abort_flag, err, kTimeoutNs));
                 if (__shfl_sync(0xffffffffu, gram_ok, 0)) {
                     tc_fence_after();
-                    if (elect_one(gram_issuer)) issue_gram(sb, tmem, st);
+                    if (elect_one(gram_issuer)) issue_gram(sb, tmem, st, c & 1);
                     __syncwarp();
                     gram_issued = 1;
                 }
