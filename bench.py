@@ -47,7 +47,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "gated_delta_rule_looped_b200", "csrc", f)
-                  for f in ("gdr_prefill_tc.cu", "gdr_decode.cu", "sm100_primitives.cuh")]
+                  for f in ("gdr_prefill_tc.cu", "gdr_prefill_kda_tc.cu", "gdr_decode.cu", "sm100_primitives.cuh")]
 
 
 def kernel_source_hash(name):
@@ -329,7 +329,8 @@ def metric_of(w):
 
 def config_of(w, n_gpus):
     return {"workload": w.name, "T": w.T, "B": w.B, "H": w.H, "L": w.L, "d_k": w.d, "d_v": w.d,
-            "gate": w.gate, "chunk": 64, "io_dtype": w.dtype, "state_dtype": "f32",
+            "gate": w.gate, "chunk": 32 if w.gate == "per_key" else 64, "io_dtype": w.dtype,
+            "state_dtype": "f32",
             "parallelism": f"replicas x{n_gpus} (independent head-units, no collective)",
             "l2": "inputs larger than L2 (no flush needed)"}
 
@@ -373,13 +374,13 @@ def main():
     launch_s = ms * 1e-3 / w.T
     flops_launch = units_per_launch * w.L * FLOP_PER_TOKEN_HEAD[gate]
     bytes_launch = units_per_launch * w.L * BYTES_PER_TOKEN_HEAD[gate]
-    tc_path = gate == "scalar"
-    kernel = "gdr_prefill_tc_kernel" if tc_path else "gdr_prefill_seq_kernel"
+    kernel, source = (("gdr_prefill_tc_kernel", "gdr_prefill_tc.cu") if gate == "scalar"
+                      else ("gdr_prefill_kda_tc_kernel", "gdr_prefill_kda_tc.cu"))
     achieved_tf = flops_launch / launch_s / 1e12
     peak_tf = peaks["bf16_tflops"]
     roofline = {"bound": "tensor", "kernel": kernel, "achieved": achieved_tf, "peak": peak_tf,
                 "unit": "TFLOP/s", "frac": achieved_tf / peak_tf,
-                "traffic": traffic_for(kernel, "gdr_prefill_tc.cu") if tc_path else None,
+                "traffic": traffic_for(kernel, source),
                 "peak_source": f"{peak_src} bf16 dense (fp16 operands run at the same rate)",
                 "algorithmic_per_launch": {"flop": flops_launch, "bytes": bytes_launch},
                 "hbm": {"achieved": bytes_launch / launch_s / 1e9, "peak": peaks["hbm_gbs"],

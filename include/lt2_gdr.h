@@ -37,8 +37,11 @@
  * lt2_gdr_last_device_error() reads (and clears) it.  No C++ exception crosses the ABI.
  *
  * Supported set.
- *   The tensor-core chunked prefill serves bf16 inputs with dk = dv = 128; every other
- *   supported shape runs on the CUDA-core path.
+ *   The tensor-core chunked prefills serve bf16 inputs with dk = dv = 128, for scalar gating
+ *   (64-token chunks) and per-key gating (32-token chunks); every other supported shape runs
+ *   on the CUDA-core path.  With per-key gating, a chunk in which some key decays by more than
+ *   ~e^-19, or with any alpha outside (0, 1], is evaluated token by token inside the same
+ *   kernel (exact, slower); alpha is expected in (0, 1] and |q|, |k| entries of order 1.
  *   fp32 inputs: dk, dv multiples of 8 up to 128 (CUDA-core fp32 arithmetic throughout).
  *   bf16 inputs: dk, dv multiples of 8 up to 128.
  *   Any L >= 0 (a ragged final chunk is fine; L = 0 copies S0 to S_out).
