@@ -32,6 +32,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import gated_delta_rule_looped_b200 as lt2  # noqa: E402
+from gated_delta_rule_looped_b200 import dist as gdist  # noqa: E402
 from gated_delta_rule_looped_b200 import inputs  # noqa: E402
 
 # Algorithmic work per token-head (chunk 64, d = 128; scalar gating): three d x d state
@@ -145,36 +146,21 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-# ---- distributed plumbing ----------------------------------------------------------------
+# ---- distributed plumbing (gated_delta_rule_looped_b200.dist) -----------------------------
 
 def dist_setup(n_gpus):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
+    world, rank, local = gdist.env_ranks()
+    torch.cuda.set_device(local if world > 1 else 0)
+    gdist.init("nccl", timeout_s=120, device=torch.device("cuda", local))
     return world, rank, local
 
 
 def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    gdist.barrier(world)
 
 
 def max_over_ranks(x, world):
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return gdist.max_over_ranks(x, world, device="cuda")
 
 
 # ---- timed regions -----------------------------------------------------------------------
@@ -367,7 +353,7 @@ def main():
         raise RuntimeError("device-side timeout during the benchmark")
     clocks = sampler.stop() if sampler else None
     tok_loops = w.T * w.B * w.L * world
-    value = tok_loops / (ms * 1e-3)
+    value = gdist.whole_job_rate(w.T * w.B * w.L, world, ms)
 
     gate = w.gate
     units_per_launch = w.B * w.H
