@@ -17,6 +17,7 @@ sample), "clocks" (nvidia-smi sampled during the timed region), "gpu_launches".
 """
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -51,10 +52,26 @@ KERNEL_SOURCES = [os.path.join(ROOT, "gated_delta_rule_looped_b200", "csrc", f)
                   for f in ("gdr_prefill_tc.cu", "gdr_prefill_kda_tc.cu", "gdr_decode.cu", "sm100_primitives.cuh")]
 
 
+def kernel_sources(name):
+    """The kernel's source file and every local header it includes, directly or not, in a fixed
+    order: kernel code that lives in a shared header changes the kernel as much as its own file."""
+    csrc = os.path.join(ROOT, "gated_delta_rule_looped_b200", "csrc")
+    seen, todo = [], [name]
+    while todo:
+        f = todo.pop(0)
+        if f in seen or not os.path.exists(os.path.join(csrc, f)):
+            continue
+        seen.append(f)
+        with open(os.path.join(csrc, f)) as fh:
+            todo.extend(re.findall(r'^\s*#\s*include\s+"([^"]+)"', fh.read(), re.M))
+    return seen
+
+
 def kernel_source_hash(name):
     h = hashlib.sha256()
-    with open(os.path.join(ROOT, "gated_delta_rule_looped_b200", "csrc", name), "rb") as f:
-        h.update(f.read())
+    for f in kernel_sources(name):
+        with open(os.path.join(ROOT, "gated_delta_rule_looped_b200", "csrc", f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
 
 
