@@ -36,11 +36,12 @@
 //
 // CTA = one (loop, batch, head) unit, 16 warps:
 //   warp 0       TMA producer (and TMEM allocation)
-//   warps 1-3    per-key decay factors; K and Q tiles of tokens 0-10 / 11-21 / 22-31 (six fp16
-//                tiles); warp 3 also converts V to fp16 and issues the Gram MMA
+//   warps 1-3, 12-15  conversion, seven warps of 5, 5, 5, 5, 4, 4, 4 tokens: per-key decay
+//                factors, the six fp16 tiles of K and Q, and V to fp16; warp 3 also issues the
+//                Gram MMA
 //   warps 4-7    prep: Gram epilogue, diagonal-block inverses, back substitution, Z
-//   warps 8-11   the S-dependent chain (warp 8 issues MMA_A, MMA_B, MMA_C)
-//   warps 12-15  output epilogue
+//   warps 8-11   the S-dependent chain (warp 8 issues MMA_A, MMA_B, MMA_C) and the output
+//                epilogue, which runs while MMA_C does
 // Every mbarrier wait is bounded (see mbar_wait); a timeout is recorded in the device status
 // word and the CTA drains its copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
@@ -60,6 +61,7 @@ using namespace tcc;
 
 constexpr int kC = 32;                 // tokens per chunk
 constexpr int kThreads = 512;
+constexpr int kConv = 7;               // conversion warps
 constexpr int kStages = 3;
 constexpr uint64_t kTimeoutNs = kWaitTimeoutNs;
 // Gram tiles carry factors e^{+-(G - G_31/2)}: in range while they stay within [2^-14, 2^14].
@@ -103,16 +105,24 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 
 struct Gates {
     float sq[kD];      // sqrt(e^{G_31}): square root of the chunk's decay per key
-    int in_range[3];   // per conversion warp: Gram factors within range for its tokens
+    int in_range[8];   // per conversion warp: Gram factors within range for its tokens
 };
 static_assert(sizeof(Gates) <= GATE_STAGE, "gate stage too small");
 
+__device__ __forceinline__ bool gates_in_range(const Gates* g)
+{
+    int all = 1;
+    #pragma unroll
+    for (int w = 0; w < kConv; ++w) all &= g->in_range[w];
+    return all != 0;
+}
+
 enum Bar : uint32_t {
     B_FULL = 0,        // [3] TMA of a stage landed
-    B_CONV = 3,        // [3] stage and Gram tiles converted (warps 1, 2, 3)
+    B_CONV = 3,        // [3] stage and Gram tiles converted (the conversion warps)
     B_EMPTY = 6,       // [3] chain done with a stage
-    B_GATE_FULL = 9,   // [3] decay factors written (warps 1, 2, 3)
-    B_GATE_EMPTY = 12, // [3] chain and output epilogue done with a gate stage
+    B_GATE_FULL = 9,   // [3] decay factors written (the conversion warps)
+    B_GATE_EMPTY = 12, // [3] chain done with a gate stage
     B_TP_FULL = 15,    // [2]
     B_TP_EMPTY = 17,   // [2]
     B_G_FULL = 19,     // Gram in TMEM
@@ -121,19 +131,17 @@ enum Bar : uint32_t {
     B_A_FULL = 23,
     B_B_FULL = 24,
     B_S_FULL = 25,
-    B_O_READY = 26,
-    B_O_DONE = 27,
-    B_DRAIN = 28,      // [2]
-    B_AL_FULL = 30,    // [2] TMA of a chunk's alpha landed
-    B_AL_EMPTY = 32,   // [2] conversion warps done with it
-    B_COUNT = 34
+    B_DRAIN = 26,      // [2]
+    B_AL_FULL = 28,    // [2] TMA of a chunk's alpha landed
+    B_AL_EMPTY = 30,   // [2] conversion warps done with it
+    B_COUNT = 32
 };
 constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + B_COUNT * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 16;
 constexpr uint32_t OFF_OKFLAG = OFF_ABORT + 16;
 static_assert(OFF_OKFLAG + 32 <= OFF_BAR + BAR_BYTES, "barrier area too small");
 
-constexpr int NB_PREP = 1, NB_CHAIN = 2, NB_OUT = 3;
+constexpr int NB_PREP = 1, NB_CHAIN = 2, NB_CONV = 3;
 
 // TMEM columns (lane j = d_v index in the chain's regions).
 constexpr uint32_t TM_G = 0;           // Gram (64 columns; lanes 0-31 Kt rows, 32-63 Qt rows)
@@ -169,16 +177,20 @@ struct Params {
 __device__ __forceinline__ uint32_t bar_addr(uint32_t base, uint32_t i) { return base + OFF_BAR + 8u * i; }
 
 // ---- conversion: per-key decay factors and the six fp16 tiles of one chunk ----------------
-// Conversion warp w (1, 2, 3) converts tokens [t_begin, t_end) of the chunk (11, 11 and 10
-// tokens) for all 128 keys; lane l owns keys 4l .. 4l+3 (8 bytes of a row of panel l >> 4 of
-// every 128-wide tile).
-// With P_t = e^{G_t} (P_-1 = 1), sq = sqrt(P_31), F_t = P_t / sq and R_t = 1 / F_t:
+// Conversion warp w (0 .. 6) converts tokens [conv_begin(w), conv_begin(w + 1)) of the chunk for
+// all 128 keys; lane l owns keys 4l .. 4l+3 (8 bytes of a row of panel l >> 4 of every 128-wide
+// tile).  With P_t = e^{G_t} (P_-1 = 1), sq = sqrt(P_31), F_t = P_t / sq and R_t = 1 / F_t:
 //   K^_t = P_{t-1} k_t,  Q^_t = P_t q_t,  Kt_t = F_{t-1} k_t,  Qt_t = F_t q_t,
 //   Bv_t = b_t R_t k_t,  Be_t = b_t R_{t-1} k_t
-// (the state products need Kv = sq Bv and Ke = sq Be: sq R_t = P_31 / P_t).  The loops stay
-// rolled: this code runs once per chunk per warp and would otherwise be fetched afresh every
-// time.  The warp starting at token 0 writes sq of every key to `sq_out`; the return value says
-// whether every F_t of the warp's tokens lies in [kFactorMin, kFactorMax].
+// (the state products need Kv = sq Bv and Ke = sq Be: sq R_t = P_31 / P_t), and V_t to fp16.
+// P_t comes in two steps: each warp first overwrites the alpha rows of its own tokens with the
+// running product over them (local_products); after a barrier of the conversion warps, row
+// conv_begin(v + 1) - 1 holds the product over warp v's tokens, from which a warp takes the
+// product over the tokens before its own and over the whole chunk (chunk_products).  The loops
+// stay rolled: this code runs once per chunk per warp and would otherwise be fetched afresh
+// every time.
+__device__ __forceinline__ int conv_begin(int w) { return w < 4 ? 5 * w : 20 + 4 * (w - 4); }
+
 __device__ __forceinline__ float4 mul4(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
 __device__ __forceinline__ float4 scale4(float4 a, float s) { return make_float4(a.x * s, a.y * s, a.z * s, a.w * s); }
 __device__ __forceinline__ float4 rcp4(float4 a)
@@ -198,28 +210,46 @@ __device__ __forceinline__ bool in_factor_range(float4 f)
     return fminf(fminf(f.x, f.y), fminf(f.z, f.w)) >= kFactorMin && fmaxf(fmaxf(f.x, f.y), fmaxf(f.z, f.w)) <= kFactorMax;
 }
 
-// `alpha_c` is the chunk's alpha tile in shared memory ([32][128]); `bl` the beta of token
-// `lane` (0 beyond the chunk's end).
-__device__ __forceinline__ bool convert_kq(uint32_t st, uint32_t gram, const float* alpha_c, float bl, int n,
-                                           int t_begin, int t_end, int lane, uint8_t* sbase, uint32_t sb, float* sq_out)
+// Row t of the chunk's alpha (t in [t_begin, t_end), at most 5 tokens) becomes
+// prod_{t_begin <= u <= t} alpha_u, alpha taken as 1 past the chunk's last token n - 1.
+__device__ __forceinline__ void local_products(float* alpha_c, int n, int t_begin, int t_end, int lane)
 {
-    const float* arow = alpha_c + 4 * lane;
-    auto alpha4 = [&](int t) -> float4 {
-        return t < n ? *reinterpret_cast<const float4*>(arow + t * kD) : make_float4(1.f, 1.f, 1.f, 1.f);
-    };
-    // products of alpha over the tokens before t_begin and over the whole chunk
-    float4 Pt = make_float4(1.f, 1.f, 1.f, 1.f), Ph = Pt;
-    #pragma unroll 1
-    for (int t8 = 0; t8 < kC; t8 += 8) {
-        float4 a[8];
-        #pragma unroll
-        for (int i = 0; i < 8; ++i) a[i] = alpha4(t8 + i);    // the eight loads issue together
-        #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (t8 + i == t_begin) Ph = Pt;
-            Pt = mul4(Pt, a[i]);
-        }
+    float4* row = reinterpret_cast<float4*>(alpha_c + t_begin * kD + 4 * lane);
+    float4 a[5];
+    #pragma unroll
+    for (int i = 0; i < 5; ++i)
+        a[i] = t_begin + i < n && t_begin + i < t_end ? row[i * (kD / 4)] : make_float4(1.f, 1.f, 1.f, 1.f);
+    float4 p = a[0];
+    #pragma unroll
+    for (int i = 0; i < 5; ++i) {
+        if (i > 0) p = mul4(p, a[i]);
+        if (t_begin + i < t_end) row[i * (kD / 4)] = p;
     }
+}
+
+// After local_products of every conversion warp: the product over the tokens before warp w's
+// (Ph) and over the whole chunk (returned).
+__device__ __forceinline__ float4 chunk_products(const float* alpha_c, int w, int lane, float4& Ph)
+{
+    float4 Pt = make_float4(1.f, 1.f, 1.f, 1.f);
+    Ph = Pt;
+    #pragma unroll
+    for (int v = 0; v < kConv; ++v) {
+        const float4 tot = *reinterpret_cast<const float4*>(alpha_c + (conv_begin(v + 1) - 1) * kD + 4 * lane);
+        if (v == w) Ph = Pt;
+        Pt = mul4(Pt, tot);
+    }
+    return Pt;
+}
+
+// The tiles of tokens [t_begin, t_end), given Ph and the chunk's product Pt; alpha_c holds the
+// running products of local_products.  The warp starting at token 0 writes sq of every key to
+// `sq_out`; the return value says whether every F_t of the warp's tokens lies in
+// [kFactorMin, kFactorMax].
+__device__ __forceinline__ bool convert_kqv(uint32_t st, uint32_t gram, const float* alpha_c, float bl, float4 Ph,
+                                            float4 Pt, int t_begin, int t_end, int lane, uint8_t* sbase, uint32_t sb,
+                                            float* sq_out)
+{
     const float4 isq = make_float4(rsqrt_approx(Pt.x), rsqrt_approx(Pt.y), rsqrt_approx(Pt.z), rsqrt_approx(Pt.w));
     if (t_begin == 0) *reinterpret_cast<float4*>(sq_out + 4 * lane) = mul4(Pt, isq);
     float4 P = Ph;                               // P_{t-1}
@@ -231,19 +261,24 @@ __device__ __forceinline__ bool convert_kq(uint32_t st, uint32_t gram, const flo
     const uint32_t chunk = static_cast<uint32_t>((lane & 15) >> 1), within = static_cast<uint32_t>(lane & 1) * 8u;
     uint8_t* kq = sbase + (st + ST_KQ + panel * 8192 - sb);
     uint8_t* bve = sbase + (st + ST_KVE + panel * 8192 - sb);
+    uint8_t* vt = sbase + (st + ST_V + panel * 4096 - sb);
     uint8_t* gp = sbase + (gram + panel * GRAM_PANEL - sb);
+    const float* arow = alpha_c + 4 * lane;
     #pragma unroll 1
     for (int t = t_begin; t < t_end; ++t) {
-        const float4 a = alpha4(t);
+        const float4 lp = *reinterpret_cast<const float4*>(arow + t * kD);
         const float b = __shfl_sync(0xffffffffu, bl, t);
         const uint32_t off = sw128(0u, t, chunk) + within;
         uint2* kp = reinterpret_cast<uint2*>(kq + off);
         uint2* qp = reinterpret_cast<uint2*>(kq + off + 4096);
+        uint2* vp = reinterpret_cast<uint2*>(vt + off);
         const float4 k = unpack4_bf16(*kp), q = unpack4_bf16(*qp);
-        const float4 Pn = mul4(P, a), Fn = mul4(Pn, isq), Rn = rcp4(Fn);
+        const uint2 vb = *vp;
+        const float4 Pn = mul4(Ph, lp), Fn = mul4(Pn, isq), Rn = rcp4(Fn);
         ok = ok && in_factor_range(Fn);
         *kp = pack4_scaled(k, P);                                               // K^ (in place)
         *qp = pack4_scaled(q, Pn);                                              // Q^ (in place)
+        *vp = make_uint2(pack_half2(bf16_lo(vb.x), bf16_hi(vb.x)), pack_half2(bf16_lo(vb.y), bf16_hi(vb.y)));
         *reinterpret_cast<uint2*>(gp + off) = pack4_scaled(k, F);               // Kt
         *reinterpret_cast<uint2*>(gp + off + 4096) = pack4_scaled(q, Fn);       // Qt
         *reinterpret_cast<uint2*>(bve + off) = pack4_scaled(k, scale4(R, b));   // Be
@@ -512,7 +547,6 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + OFF_ABORT);
     volatile int* okflags = reinterpret_cast<volatile int*>(sbase + OFF_OKFLAG);
     auto gate = [&](int s) -> Gates* { return reinterpret_cast<Gates*>(sbase + OFF_GATES + s * GATE_STAGE); };
-    auto lds = [&](uint32_t addr) -> uint4 { return *reinterpret_cast<const uint4*>(sbase + (addr - sb)); };
     auto sts = [&](uint32_t addr, uint4 v) { *reinterpret_cast<uint4*>(sbase + (addr - sb)) = v; };
 
     const int warp = threadIdx.x >> 5;
@@ -526,17 +560,17 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         *abort_flag = 0;
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar_addr(sb, B_FULL + s), 1);
-            mbar_init(bar_addr(sb, B_CONV + s), 3);
+            mbar_init(bar_addr(sb, B_CONV + s), kConv);
             mbar_init(bar_addr(sb, B_EMPTY + s), 1);
-            mbar_init(bar_addr(sb, B_GATE_FULL + s), 3);
-            mbar_init(bar_addr(sb, B_GATE_EMPTY + s), 2);
+            mbar_init(bar_addr(sb, B_GATE_FULL + s), kConv);
+            mbar_init(bar_addr(sb, B_GATE_EMPTY + s), 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar_addr(sb, B_TP_FULL + s), 1);
             mbar_init(bar_addr(sb, B_TP_EMPTY + s), 1);
             mbar_init(bar_addr(sb, B_DRAIN + s), 1);
             mbar_init(bar_addr(sb, B_AL_FULL + s), 1);
-            mbar_init(bar_addr(sb, B_AL_EMPTY + s), 3);
+            mbar_init(bar_addr(sb, B_AL_EMPTY + s), kConv);
         }
         mbar_init(bar_addr(sb, B_G_FULL), 1);
         mbar_init(bar_addr(sb, B_G_EMPTY), 1);
@@ -545,8 +579,6 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         mbar_init(bar_addr(sb, B_A_FULL), 1);
         mbar_init(bar_addr(sb, B_B_FULL), 1);
         mbar_init(bar_addr(sb, B_S_FULL), 1);
-        mbar_init(bar_addr(sb, B_O_READY), 1);
-        mbar_init(bar_addr(sb, B_O_DONE), 1);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -607,12 +639,14 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c)
                 mbar_wait(bar_addr(sb, B_AL_FULL + (c & 1)), (c >> 1) & 1, abort_flag, err, kTimeoutNs / 4);
         }
-    } else if (warp < 4) {
-        // ================= decay factors and K/Q tiles (warps 1-3), V and the Gram (warp 3) ======
+    } else if (warp < 4 || warp >= 12) {
+        // ======= conversion (warps 1-3, 12-15): decay factors, K/Q/V tiles; warp 3 issues the Gram ======
         uint32_t gram_issuer = 0;
         int gram_issued = 0;
-        const int w = warp - 1;                     // 0, 1, 2: tokens [11w, min(11w + 11, 32))
-        const int t_begin = 11 * w, t_end = w == 2 ? kC : 11 * w + 11;
+        const int w = warp < 4 ? warp - 1 : warp - 9;
+        const int t_begin = conv_begin(w), t_end = conv_begin(w + 1);
+        // one leader waits for the chunk's inputs; all seven warps leave the loop together
+        Group grp{NB_CONV, 32 * kConv, warp == 1 && lane == 0, okflags + 4, 0, abort_flag, err};
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;
             const uint32_t ph = (c / kStages) & 1;
@@ -622,23 +656,19 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             // beta of token `lane` of this chunk: the load is issued before the waits below, which
             // hide its latency
             const float bl = lane < n ? p.beta[static_cast<int64_t>(ug) * L + t0 + lane] : 0.f;
-            int ok = 0;
-            if (lane == 0)
-                ok = mbar_wait(bar_addr(sb, B_FULL + s), ph, abort_flag, err, kTimeoutNs) &&
-                     mbar_wait(bar_addr(sb, B_GATE_EMPTY + s), ph ^ 1, abort_flag, err, kTimeoutNs) &&
-                     mbar_wait(bar_addr(sb, B_AL_FULL + (c & 1)), (c >> 1) & 1, abort_flag, err, kTimeoutNs) &&
-                     mbar_wait(bar_addr(sb, B_GFREE + (c & 1)), ((c >> 1) & 1) ^ 1, abort_flag, err, kTimeoutNs);
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            if (!grp.wait(bar_addr(sb, B_FULL + s), ph, bar_addr(sb, B_GATE_EMPTY + s), ph ^ 1,
+                          bar_addr(sb, B_AL_FULL + (c & 1)), (c >> 1) & 1))
+                break;
+            if (!grp.wait(bar_addr(sb, B_GFREE + (c & 1)), ((c >> 1) & 1) ^ 1)) break;
+            float* alpha_c = reinterpret_cast<float*>(sbase + OFF_ALPHA + (c & 1) * ALPHA_STAGE);
+            local_products(alpha_c, n, t_begin, t_end, lane);
+            grp.sync();
+            float4 Ph;
+            const float4 Pt = chunk_products(alpha_c, w, lane, Ph);
             Gates* gs = gate(s);
-            const bool in_range =
-                convert_kq(st, sb + OFF_GRAM + (c & 1) * GRAM_BUF,
-                           reinterpret_cast<const float*>(sbase + OFF_ALPHA + (c & 1) * ALPHA_STAGE),
-                           bl, n, t_begin, t_end, lane, sbase, sb, gs->sq);
+            const bool in_range = convert_kqv(st, sb + OFF_GRAM + (c & 1) * GRAM_BUF, alpha_c, bl, Ph, Pt,
+                                              t_begin, t_end, lane, sbase, sb, gs->sq);
             if (lane == 0) gs->in_range[w] = in_range ? 1 : 0;
-            if (warp == 3) {
-                #pragma unroll 1
-                for (int panel = 0; panel < 2; ++panel) convert_tile(st + ST_V + panel * 4096, 256, lane, lds, sts);
-            }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -658,7 +688,6 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                     gram_issued = 1;
                 }
             }
-            if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
         }
         if (warp == 3 && lane == gram_issuer && gram_issued && *abort_flag) {
             umma_commit(bar_addr(sb, B_DRAIN + 1));
@@ -693,7 +722,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             grp.sync();
             if (t == 0) mbar_arrive(bar_addr(sb, B_TP_FULL + tps));
         }
-    } else if (warp < 12) {
+    } else {
         // ================= the S-dependent chain (lane j = d_v column j of S) =================
         const int j = threadIdx.x - 256;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
@@ -704,7 +733,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         if (ok) ok = grp.wait(bar_addr(sb, B_GATE_FULL + 0), 0);
         if (ok) {
             const Gates* g0 = gate(0);
-            const bool exact0 = !(g0->in_range[0] && g0->in_range[1] && g0->in_range[2]);
+            const bool exact0 = !gates_in_range(g0);
             load_initial_state(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr,
                                p.S0 ? p.S0 + static_cast<int64_t>(ug) * kD * kD + j : nullptr,
                                exact0 ? nullptr : g0->sq);
@@ -721,15 +750,14 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             const int64_t t0 = static_cast<int64_t>(c) * kC;
             const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
             const Gates* gs = gate(s);
-            const bool exact = !(gs->in_range[0] && gs->in_range[1] && gs->in_range[2]);
+            const bool exact = !gates_in_range(gs);
             if (!exact) {
                 // --- MMA_A: (K^ S, Q^ S)^T = S^T [K^; Q^]^T ---
                 grp.sync();
                 if (warp == 8) {
                     int lok = 0;
                     if (leader)
-                        lok = mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs) &&
-                              (c == 0 || mbar_wait(bar_addr(sb, B_O_DONE), (c - 1) & 1, abort_flag, err, kTimeoutNs));
+                        lok = mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs);
                     if (__shfl_sync(0xffffffffu, lok, 0)) {
                         tc_fence_after();
                         if (elect_one(mma_issuer)) {
@@ -774,7 +802,6 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                                 umma_f16_tmem_a(tmem + TM_B, tmem + TM_Y + 8 * k, smem_desc_sw128(tp + k * 32, 16, 1024),
                                                 ID_T64, 1);
                             umma_commit(bar_addr(sb, B_B_FULL));
-                            umma_commit(bar_addr(sb, B_O_READY));
                             umma_commit(bar_addr(sb, B_TP_EMPTY + tps));
                         }
                         __syncwarp();
@@ -794,6 +821,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                     tmem_st16(tmem + TM_E + lane_addr, hpk);
                     tmem_wait_st();
                 }
+                if (leader) bulk_wait_read_all();      // the previous chunk's o store has left the staging
                 tc_fence_before();
                 grp.sync();
                 // --- MMA_C: (sq S)^T += V^T Bv - E^T Be ---
@@ -811,10 +839,28 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                     }
                     __syncwarp();
                 }
+                // --- while MMA_C runs: o = Q^ S - (the -O' half of MMA_B) ---
+                if (!p.out_bf16) {
+                    store_o_f32(tmem + TM_AB + lane_addr + 32, tmem + TM_B + lane_addr + 32,
+                                static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, n);
+                } else {
+                    float qp[64];
+                    tmem_load_2x32(tmem + TM_AB + lane_addr + 32, tmem + TM_B + lane_addr + 32, qp);
+                    uint8_t* ost = sbase + OFF_OST + (j >> 6) * 4096 + (j & 63) * 2;
+                    #pragma unroll
+                    for (int r = 0; r < 32; ++r)
+                        *reinterpret_cast<__nv_bfloat16*>(ost + r * 128) = __float2bfloat16_rn(qp[r] - qp[32 + r]);
+                    fence_proxy_async_smem();
+                }
                 ok = grp.wait(bar_addr(sb, B_S_FULL), ph_s);
                 ph_s ^= 1u;
                 if (!ok) break;
                 tc_fence_after();
+                if (leader && p.out_bf16) {
+                    tma_store_3d(&tm_o, sb + OFF_OST, 0, static_cast<int32_t>(t0), ug);
+                    tma_store_3d(&tm_o, sb + OFF_OST + 4096, 64, static_cast<int32_t>(t0), ug);
+                    bulk_commit_group();
+                }
             } else {
                 // --- out-of-range chunk: the definition, token by token, on the fp32 state ---
                 exact_chunk(tmem + TM_S + lane_addr, ExactIn{p.q, p.k, p.v, p.alpha, p.beta, p.o, p.out_bf16},
@@ -827,7 +873,6 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 if (leader) {
                     mbar_arrive(bar_addr(sb, B_EMPTY + s));
                     mbar_arrive(bar_addr(sb, B_TP_EMPTY + tps));
-                    mbar_arrive(bar_addr(sb, B_O_READY));
                 }
             }
             // --- the new state ---
@@ -842,7 +887,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 ok = grp.wait(bar_addr(sb, B_GATE_FULL + s1), ((c + 1) / kStages) & 1);
                 if (!ok) break;
                 const Gates* g1 = gate(s1);
-                const bool exact1 = !(g1->in_range[0] && g1->in_range[1] && g1->in_range[2]);
+                const bool exact1 = !gates_in_range(g1);
                 state_update(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr, f_sh, exact1 ? nullptr : g1->sq);
                 tc_fence_before();
             }
@@ -853,47 +898,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             umma_commit(bar_addr(sb, B_DRAIN + 0));
             mbar_wait(bar_addr(sb, B_DRAIN + 0), 0, abort_flag, err, kTimeoutNs / 4);
         }
-    } else {
-        // ================= output epilogue: o = Q^ S - (the -O' half of MMA_B) =================
-        const int j = threadIdx.x - 384;
-        const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-        Group grp{NB_OUT, 128, j == 0, okflags + 4, 0, abort_flag, err};
-        for (int c = 0; c < nchunks; ++c) {
-            const int s = c % kStages;
-            if (j == 0) bulk_wait_read_all();
-            if (!grp.wait(bar_addr(sb, B_O_READY), c & 1)) break;
-            tc_fence_after();
-            const Gates* gs = gate(s);
-            const bool exact = !(gs->in_range[0] && gs->in_range[1] && gs->in_range[2]);
-            const int64_t t0 = static_cast<int64_t>(c) * kC;
-            if (!exact) {
-                if (!p.out_bf16) {
-                    const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
-                    store_o_f32(tmem + TM_AB + lane_addr + 32, tmem + TM_B + lane_addr + 32,
-                                static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, n);
-                } else {
-                    float qp[64];
-                    tmem_load_2x32(tmem + TM_AB + lane_addr + 32, tmem + TM_B + lane_addr + 32, qp);
-                    uint8_t* ost = sbase + OFF_OST + (j >> 6) * 4096 + (j & 63) * 2;
-                    #pragma unroll
-                    for (int r = 0; r < 32; ++r)
-                        *reinterpret_cast<__nv_bfloat16*>(ost + r * 128) = __float2bfloat16_rn(qp[r] - qp[32 + r]);
-                }
-            }
-            tc_fence_before();
-            fence_proxy_async_smem();
-            grp.sync();
-            if (j == 0) {
-                mbar_arrive(bar_addr(sb, B_O_DONE));
-                mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
-                if (!exact && p.out_bf16) {
-                    tma_store_3d(&tm_o, sb + OFF_OST, 0, static_cast<int32_t>(t0), ug);
-                    tma_store_3d(&tm_o, sb + OFF_OST + 4096, 64, static_cast<int32_t>(t0), ug);
-                    bulk_commit_group();
-                }
-            }
-        }
-        if (j == 0) bulk_wait_all();
+        if (leader) bulk_wait_all();
     }
 
     tc_fence_before();
