@@ -36,12 +36,13 @@
 //
 // CTA = one (loop, batch, head) unit, 16 warps:
 //   warp 0       TMA producer (and TMEM allocation)
-//   warps 1-3, 12-15  conversion, seven warps of 5, 5, 5, 5, 4, 4, 4 tokens: per-key decay
-//                factors, the six fp16 tiles of K and Q, and V to fp16; warp 3 also issues the
-//                Gram MMA
+//   warps 1-3    conversion of tokens 0-10 / 11-21 / 22-31: per-key decay factors, the six
+//                fp16 tiles of K and Q, and V to fp16; warp 3 also issues the Gram MMA
 //   warps 4-7    prep: Gram epilogue, diagonal-block inverses, back substitution, Z
-//   warps 8-11   the S-dependent chain (warp 8 issues MMA_A, MMA_B, MMA_C) and the output
-//                epilogue, which runs while MMA_C does
+//   warps 8-15   the S-dependent chain (warp 8 issues MMA_A, MMA_B, MMA_C) and the output
+//                epilogue, which runs while MMA_C does.  Warps w and w + 4 share TMEM lanes
+//                32 (w & 3) .. + 31 (d_v columns) and split every epilogue by TMEM column: keys
+//                0-63 / 64-127 of the state, tokens 0-15 / 16-31 of the chunk
 // Every mbarrier wait is bounded (see mbar_wait); a timeout is recorded in the device status
 // word and the CTA drains its copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
@@ -61,7 +62,7 @@ using namespace tcc;
 
 constexpr int kC = 32;                 // tokens per chunk
 constexpr int kThreads = 512;
-constexpr int kConv = 7;               // conversion warps
+constexpr int kConv = 3;               // conversion warps
 constexpr int kStages = 3;
 constexpr uint64_t kTimeoutNs = kWaitTimeoutNs;
 // Gram tiles carry factors e^{+-(G - G_31/2)}: in range while they stay within [2^-14, 2^14].
@@ -148,8 +149,8 @@ constexpr uint32_t TM_G = 0;           // Gram (64 columns; lanes 0-31 Kt rows, 
 constexpr uint32_t TM_S = 64;          // S^T fp32, scaled per key by sq around MMA_C (128)
 constexpr uint32_t TM_SH = 192;        // S^T fp16 pairs (64): A operand of MMA_A
 constexpr uint32_t TM_AB = 256;        // (K^ S)^T 256..287, (Q^ S)^T 288..319
-constexpr uint32_t TM_Y = 256;         //   (K^ S)^T as fp16 pairs (16), A operand of MMA_B
-constexpr uint32_t TM_E = 272;         //   -E^T as fp16 pairs (16), A operand of MMA_C
+constexpr uint32_t TM_Y = 384;         // (K^ S)^T as fp16 pairs (16), A operand of MMA_B
+constexpr uint32_t TM_E = 400;         // -E^T as fp16 pairs (16), A operand of MMA_C
 constexpr uint32_t TM_B = 320;         // E^T 320..351, -(O - Q^ S)^T 352..383
 constexpr uint32_t TM_COLS = 512;
 
@@ -176,8 +177,48 @@ struct Params {
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t base, uint32_t i) { return base + OFF_BAR + 8u * i; }
 
+// ---- 16-column TMEM access (one half of the chain's warps each) -----------------------------
+__device__ __forceinline__ void tmem_load16(uint32_t a, float (&v)[16])
+{
+    uint32_t* r = reinterpret_cast<uint32_t*>(v);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(a)
+        : "memory");
+}
+// Two 16-column loads (a0 into v[0..15], a1 into v[16..31]) and the wait for both.
+__device__ __forceinline__ void tmem_load_2x16(uint32_t a0, uint32_t a1, float (&v)[32])
+{
+    uint32_t* r = reinterpret_cast<uint32_t*>(v);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(a0), "r"(a1)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t a, const uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 ::"r"(a), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                   "r"(r[7])
+                 : "memory");
+}
+
 // ---- conversion: per-key decay factors and the six fp16 tiles of one chunk ----------------
-// Conversion warp w (0 .. 6) converts tokens [conv_begin(w), conv_begin(w + 1)) of the chunk for
+// Conversion warp w (0 .. 2) converts tokens [conv_begin(w), conv_begin(w + 1)) of the chunk for
 // all 128 keys; lane l owns keys 4l .. 4l+3 (8 bytes of a row of panel l >> 4 of every 128-wide
 // tile).  With P_t = e^{G_t} (P_-1 = 1), sq = sqrt(P_31), F_t = P_t / sq and R_t = 1 / F_t:
 //   K^_t = P_{t-1} k_t,  Q^_t = P_t q_t,  Kt_t = F_{t-1} k_t,  Qt_t = F_t q_t,
@@ -189,7 +230,7 @@ __device__ __forceinline__ uint32_t bar_addr(uint32_t base, uint32_t i) { return
 // product over the tokens before its own and over the whole chunk (chunk_products).  The loops
 // stay rolled: this code runs once per chunk per warp and would otherwise be fetched afresh
 // every time.
-__device__ __forceinline__ int conv_begin(int w) { return w < 4 ? 5 * w : 20 + 4 * (w - 4); }
+__device__ __forceinline__ int conv_begin(int w) { return w < kConv ? 11 * w : kC; }
 
 __device__ __forceinline__ float4 mul4(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
 __device__ __forceinline__ float4 scale4(float4 a, float s) { return make_float4(a.x * s, a.y * s, a.z * s, a.w * s); }
@@ -210,20 +251,23 @@ __device__ __forceinline__ bool in_factor_range(float4 f)
     return fminf(fminf(f.x, f.y), fminf(f.z, f.w)) >= kFactorMin && fmaxf(fmaxf(f.x, f.y), fmaxf(f.z, f.w)) <= kFactorMax;
 }
 
-// Row t of the chunk's alpha (t in [t_begin, t_end), at most 5 tokens) becomes
-// prod_{t_begin <= u <= t} alpha_u, alpha taken as 1 past the chunk's last token n - 1.
+// Row t of the chunk's alpha (t in [t_begin, t_end)) becomes prod_{t_begin <= u <= t} alpha_u,
+// alpha taken as 1 past the chunk's last token n - 1.
 __device__ __forceinline__ void local_products(float* alpha_c, int n, int t_begin, int t_end, int lane)
 {
-    float4* row = reinterpret_cast<float4*>(alpha_c + t_begin * kD + 4 * lane);
-    float4 a[5];
-    #pragma unroll
-    for (int i = 0; i < 5; ++i)
-        a[i] = t_begin + i < n && t_begin + i < t_end ? row[i * (kD / 4)] : make_float4(1.f, 1.f, 1.f, 1.f);
-    float4 p = a[0];
-    #pragma unroll
-    for (int i = 0; i < 5; ++i) {
-        if (i > 0) p = mul4(p, a[i]);
-        if (t_begin + i < t_end) row[i * (kD / 4)] = p;
+    float4 p = make_float4(1.f, 1.f, 1.f, 1.f);
+    #pragma unroll 1
+    for (int t4 = t_begin; t4 < t_end; t4 += 4) {
+        float4* row = reinterpret_cast<float4*>(alpha_c + t4 * kD + 4 * lane);
+        float4 a[4];
+        #pragma unroll
+        for (int i = 0; i < 4; ++i)
+            a[i] = t4 + i < n && t4 + i < t_end ? row[i * (kD / 4)] : make_float4(1.f, 1.f, 1.f, 1.f);
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            p = mul4(p, a[i]);
+            if (t4 + i < t_end) row[i * (kD / 4)] = p;
+        }
     }
 }
 
@@ -359,12 +403,14 @@ __device__ __noinline__ void z_row_block(uint32_t tp, uint32_t mb, int rb, int l
 
 // ---- chain helpers --------------------------------------------------------------------------
 
-// Chain thread j: S0^T row j into TMEM, as fp16 pairs (unscaled) and as fp32 scaled per
-// column i (= key) by f[i] (nullptr: unscaled).
-__device__ __noinline__ void load_initial_state(uint32_t tm_s, uint32_t tm_sh, const float* s0, const float* f)
+// Chain thread (d_v column j, key half piece0 / 2): keys 32 piece0 .. + 63 of S0^T row j into
+// TMEM, as fp16 pairs (unscaled) and as fp32 scaled per column i (= key) by f[i] (nullptr:
+// unscaled).
+__device__ __noinline__ void load_initial_state(uint32_t tm_s, uint32_t tm_sh, const float* s0, const float* f,
+                                                int piece0)
 {
     #pragma unroll 1
-    for (int piece = 0; piece < 4; ++piece) {
+    for (int piece = piece0; piece < piece0 + 2; ++piece) {
         float v[32];
         #pragma unroll
         for (int d = 0; d < 32; ++d) v[d] = s0 ? s0[(32 * piece + d) * kD] : 0.f;
@@ -381,13 +427,13 @@ __device__ __noinline__ void load_initial_state(uint32_t tm_s, uint32_t tm_sh, c
     tmem_wait_st();
 }
 
-// Chain thread j, after a chunk: the state S' = f_sh (.) TM_S (per column i = key; nullptr: 1)
-// as fp16 pairs for MMA_A, and TM_S <- f_s (.) S' (nullptr: 1), the pre-scaled state the next
-// chunk's MMA_C accumulates into.
-__device__ __forceinline__ void state_update(uint32_t tm_s, uint32_t tm_sh, const float* f_sh, const float* f_s)
+// Chain thread (d_v column j, keys 32 piece .. + 63), after a chunk: the state
+// S' = f_sh (.) TM_S (per column i = key; nullptr: 1) as fp16 pairs for MMA_A, and
+// TM_S <- f_s (.) S' (nullptr: 1), the pre-scaled state the next chunk's MMA_C accumulates into.
+__device__ __forceinline__ void state_update(uint32_t tm_s, uint32_t tm_sh, const float* f_sh, const float* f_s,
+                                             int piece)
 {
-    #pragma unroll 1
-    for (int piece = 0; piece < 4; piece += 2) {
+    {
         float v[64];
         tmem_load_2x32(tm_s + 32 * piece, tm_s + 32 * piece + 32, v);
         if (f_sh) {
@@ -423,11 +469,11 @@ __device__ __forceinline__ void state_update(uint32_t tm_s, uint32_t tm_sh, cons
     tmem_wait_st();
 }
 
-// Chain thread j: column j of the final state, f (.) TM_S (nullptr: 1), to S_out.
-__device__ __noinline__ void store_final_state_scaled(uint32_t tm_s, float* so, const float* f)
+// Chain thread (d_v column j, keys 32 piece .. + 63): that part of column j of the final state,
+// f (.) TM_S (nullptr: 1), to S_out.
+__device__ __noinline__ void store_final_state_scaled(uint32_t tm_s, float* so, const float* f, int piece)
 {
-    #pragma unroll 1
-    for (int piece = 0; piece < 4; piece += 2) {
+    {
         float v[64];
         tmem_load_2x32(tm_s + 32 * piece, tm_s + 32 * piece + 32, v);
         #pragma unroll
@@ -509,14 +555,15 @@ __device__ __noinline__ void exact_chunk(uint32_t tm_s, ExactIn p, int64_t row0,
     }
 }
 
-// Output thread j, fp32 output: o[r][j] = (Q^ S)_rj - B_rj for the chunk's n tokens.
-__device__ __noinline__ void store_o_f32(uint32_t tm_qs, uint32_t tm_b, float* o, int n)
+// Chain thread j, fp32 output: o[r][j] = (Q^ S)_rj - B_rj for tokens r = r0 .. r0 + 15 below n
+// (tm_qs and tm_b address token r0).
+__device__ __noinline__ void store_o_f32(uint32_t tm_qs, uint32_t tm_b, float* o, int r0, int n)
 {
-    float qp[64];
-    tmem_load_2x32(tm_qs, tm_b, qp);
+    float qp[32];
+    tmem_load_2x16(tm_qs, tm_b, qp);
     #pragma unroll
-    for (int r = 0; r < 32; ++r)
-        if (r < n) o[r * kD] = qp[r] - qp[32 + r];
+    for (int r = 0; r < 16; ++r)
+        if (r0 + r < n) o[(r0 + r) * kD] = qp[r] - qp[16 + r];
 }
 
 // Gram [Kt; Qt; -] [Be; Bv]^T (M = 128, N = 64, K = 128) into TMEM, Be and Bv from the chunk
@@ -639,13 +686,13 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c)
                 mbar_wait(bar_addr(sb, B_AL_FULL + (c & 1)), (c >> 1) & 1, abort_flag, err, kTimeoutNs / 4);
         }
-    } else if (warp < 4 || warp >= 12) {
-        // ======= conversion (warps 1-3, 12-15): decay factors, K/Q/V tiles; warp 3 issues the Gram ======
+    } else if (warp < 4) {
+        // ================= conversion (warps 1-3): decay factors, K/Q/V tiles; warp 3 issues the Gram ======
         uint32_t gram_issuer = 0;
         int gram_issued = 0;
-        const int w = warp < 4 ? warp - 1 : warp - 9;
+        const int w = warp - 1;
         const int t_begin = conv_begin(w), t_end = conv_begin(w + 1);
-        // one leader waits for the chunk's inputs; all seven warps leave the loop together
+        // one leader waits for the chunk's inputs; the conversion warps leave the loop together
         Group grp{NB_CONV, 32 * kConv, warp == 1 && lane == 0, okflags + 4, 0, abort_flag, err};
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;
@@ -723,11 +770,12 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             if (t == 0) mbar_arrive(bar_addr(sb, B_TP_FULL + tps));
         }
     } else {
-        // ================= the S-dependent chain (lane j = d_v column j of S) =================
-        const int j = threadIdx.x - 256;
+        // ======= the S-dependent chain (lane j = d_v column j of S; half h of the TMEM columns) =======
+        const int j = 32 * (warp & 3) + lane;
+        const int h = (warp - 8) >> 2;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-        const bool leader = j == 0;
-        Group grp{NB_CHAIN, 128, leader, okflags + 2, 0, abort_flag, err};
+        const bool leader = warp == 8 && lane == 0;
+        Group grp{NB_CHAIN, 256, leader, okflags + 2, 0, abort_flag, err};
         bool ok = nchunks > 0;
         uint32_t ph_a = 0, ph_b = 0, ph_s = 0;
         if (ok) ok = grp.wait(bar_addr(sb, B_GATE_FULL + 0), 0);
@@ -736,7 +784,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             const bool exact0 = !gates_in_range(g0);
             load_initial_state(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr,
                                p.S0 ? p.S0 + static_cast<int64_t>(ug) * kD * kD + j : nullptr,
-                               exact0 ? nullptr : g0->sq);
+                               exact0 ? nullptr : g0->sq, 2 * h);
             tc_fence_before();
         }
         uint32_t drain_needed = 0;
@@ -776,14 +824,14 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 ph_a ^= 1u;
                 if (!ok) break;
                 tc_fence_after();
-                // --- (K^ S)^T as fp16 pairs: the second A operand of MMA_B ---
+                // --- (K^ S)^T as fp16 pairs: the second A operand of MMA_B (tokens 16h .. + 15) ---
                 {
-                    float ks[32];
-                    tmem_load32(tmem + TM_AB + lane_addr, ks);
-                    uint32_t hpk[16];
+                    float ks[16];
+                    tmem_load16(tmem + TM_AB + lane_addr + 16 * h, ks);
+                    uint32_t hpk[8];
                     #pragma unroll
-                    for (int e = 0; e < 16; ++e) hpk[e] = pack_half2(ks[2 * e], ks[2 * e + 1]);
-                    tmem_st16(tmem + TM_Y + lane_addr, hpk);
+                    for (int e = 0; e < 8; ++e) hpk[e] = pack_half2(ks[2 * e], ks[2 * e + 1]);
+                    tmem_st8(tmem + TM_Y + lane_addr + 8 * h, hpk);
                     tmem_wait_st();
                 }
                 tc_fence_before();
@@ -811,14 +859,14 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 ph_b ^= 1u;
                 if (!ok) break;
                 tc_fence_after();
-                // --- -E^T as fp16 pairs: the A operand of the E half of MMA_C ---
+                // --- -E^T as fp16 pairs: the A operand of the E half of MMA_C (tokens 16h .. + 15) ---
                 {
-                    float ev[32];
-                    tmem_load32(tmem + TM_B + lane_addr, ev);
-                    uint32_t hpk[16];
+                    float ev[16];
+                    tmem_load16(tmem + TM_B + lane_addr + 16 * h, ev);
+                    uint32_t hpk[8];
                     #pragma unroll
-                    for (int e = 0; e < 16; ++e) hpk[e] = pack_half2(-ev[2 * e], -ev[2 * e + 1]);
-                    tmem_st16(tmem + TM_E + lane_addr, hpk);
+                    for (int e = 0; e < 8; ++e) hpk[e] = pack_half2(-ev[2 * e], -ev[2 * e + 1]);
+                    tmem_st8(tmem + TM_E + lane_addr + 8 * h, hpk);
                     tmem_wait_st();
                 }
                 if (leader) bulk_wait_read_all();      // the previous chunk's o store has left the staging
@@ -839,17 +887,17 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                     }
                     __syncwarp();
                 }
-                // --- while MMA_C runs: o = Q^ S - (the -O' half of MMA_B) ---
+                // --- while MMA_C runs: o = Q^ S - (the -O' half of MMA_B), tokens 16h .. + 15 ---
                 if (!p.out_bf16) {
-                    store_o_f32(tmem + TM_AB + lane_addr + 32, tmem + TM_B + lane_addr + 32,
-                                static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, n);
+                    store_o_f32(tmem + TM_AB + lane_addr + 32 + 16 * h, tmem + TM_B + lane_addr + 32 + 16 * h,
+                                static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, 16 * h, n);
                 } else {
-                    float qp[64];
-                    tmem_load_2x32(tmem + TM_AB + lane_addr + 32, tmem + TM_B + lane_addr + 32, qp);
-                    uint8_t* ost = sbase + OFF_OST + (j >> 6) * 4096 + (j & 63) * 2;
+                    float qp[32];
+                    tmem_load_2x16(tmem + TM_AB + lane_addr + 32 + 16 * h, tmem + TM_B + lane_addr + 32 + 16 * h, qp);
+                    uint8_t* ost = sbase + OFF_OST + (j >> 6) * 4096 + (j & 63) * 2 + 16 * h * 128;
                     #pragma unroll
-                    for (int r = 0; r < 32; ++r)
-                        *reinterpret_cast<__nv_bfloat16*>(ost + r * 128) = __float2bfloat16_rn(qp[r] - qp[32 + r]);
+                    for (int r = 0; r < 16; ++r)
+                        *reinterpret_cast<__nv_bfloat16*>(ost + r * 128) = __float2bfloat16_rn(qp[r] - qp[16 + r]);
                     fence_proxy_async_smem();
                 }
                 ok = grp.wait(bar_addr(sb, B_S_FULL), ph_s);
@@ -862,9 +910,11 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                     bulk_commit_group();
                 }
             } else {
-                // --- out-of-range chunk: the definition, token by token, on the fp32 state ---
-                exact_chunk(tmem + TM_S + lane_addr, ExactIn{p.q, p.k, p.v, p.alpha, p.beta, p.o, p.out_bf16},
-                            static_cast<int64_t>(ug) * L + t0, n, j);
+                // --- out-of-range chunk: the definition, token by token, on the fp32 state (the
+                // first half of the chain's warps; every key of a column takes part in k^T S) ---
+                if (h == 0)
+                    exact_chunk(tmem + TM_S + lane_addr, ExactIn{p.q, p.k, p.v, p.alpha, p.beta, p.o, p.out_bf16},
+                                static_cast<int64_t>(ug) * L + t0, n, j);
                 tc_fence_before();
                 // keep every hand-off in step: the stage and the [X; Z] stage are released
                 // once their producers are done with them, the output epilogue is released
@@ -880,7 +930,8 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             const float* f_sh = exact ? nullptr : gs->sq;
             if (c + 1 == nchunks) {
                 if (p.S_out)
-                    store_final_state_scaled(tmem + TM_S + lane_addr, p.S_out + static_cast<int64_t>(ug) * kD * kD + j, f_sh);
+                    store_final_state_scaled(tmem + TM_S + lane_addr, p.S_out + static_cast<int64_t>(ug) * kD * kD + j, f_sh,
+                                             2 * h);
                 drain_needed = 0;
             } else {
                 const int s1 = (c + 1) % kStages;
@@ -888,7 +939,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 if (!ok) break;
                 const Gates* g1 = gate(s1);
                 const bool exact1 = !gates_in_range(g1);
-                state_update(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr, f_sh, exact1 ? nullptr : g1->sq);
+                state_update(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr, f_sh, exact1 ? nullptr : g1->sq, 2 * h);
                 tc_fence_before();
             }
             grp.sync();
