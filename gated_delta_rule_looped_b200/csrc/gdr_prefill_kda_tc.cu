@@ -37,8 +37,9 @@
 // CTA = one (loop, batch, head) unit, 16 warps:
 //   warp 0       TMA producer (and TMEM allocation)
 //   warps 1-3    conversion of tokens 0-10 / 11-21 / 22-31: per-key decay factors, the six
-//                fp16 tiles of K and Q, and V to fp16; warp 3 also issues the Gram MMA
-//   warps 4-7    prep: Gram epilogue, diagonal-block inverses, back substitution, Z
+//                fp16 tiles of K and Q, and V to fp16
+//   warps 4-7    prep: Gram epilogue, diagonal-block inverses, back substitution, Z; warp 4
+//                then issues the next chunk's Gram MMA
 //   warps 8-15   the S-dependent chain (warp 8 issues MMA_A, MMA_B, MMA_C) and the output
 //                epilogue, which runs while MMA_C does.  Warps w and w + 4 share TMEM lanes
 //                32 (w & 3) .. + 31 (d_v columns) and split every epilogue by TMEM column: keys
@@ -127,7 +128,6 @@ enum Bar : uint32_t {
     B_TP_FULL = 15,    // [2]
     B_TP_EMPTY = 17,   // [2]
     B_G_FULL = 19,     // Gram in TMEM
-    B_G_EMPTY = 20,    // Gram read out
     B_GFREE = 21,      // [2] Gram MMA done reading a Gram tile buffer
     B_A_FULL = 23,
     B_B_FULL = 24,
@@ -580,6 +580,21 @@ __device__ __forceinline__ void issue_gram(uint32_t sb, uint32_t tmem, uint32_t 
     umma_commit(bar_addr(sb, B_GFREE + gbuf));
 }
 
+// Prep warp 4: the Gram of chunk k once its tiles are converted (prep has read the previous
+// Gram out of TMEM before it gets here).  Returns 1 if issued; `issuer` is the issuing lane.
+__device__ __noinline__ int issue_gram_of(int k, uint32_t sb, uint32_t tmem, int lane, volatile int* abort_flag,
+                                          unsigned int* err, uint32_t& issuer)
+{
+    int gok = 0;
+    if (lane == 0)
+        gok = mbar_wait(bar_addr(sb, B_CONV + k % kStages), (k / kStages) & 1, abort_flag, err, kTimeoutNs);
+    if (!__shfl_sync(0xffffffffu, gok, 0)) return 0;
+    tc_fence_after();
+    if (elect_one(issuer)) issue_gram(sb, tmem, sb + OFF_STG + (k % kStages) * STAGE_BYTES, k & 1);
+    __syncwarp();
+    return 1;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -620,7 +635,6 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             mbar_init(bar_addr(sb, B_AL_EMPTY + s), kConv);
         }
         mbar_init(bar_addr(sb, B_G_FULL), 1);
-        mbar_init(bar_addr(sb, B_G_EMPTY), 1);
         mbar_init(bar_addr(sb, B_GFREE + 0), 1);
         mbar_init(bar_addr(sb, B_GFREE + 1), 1);
         mbar_init(bar_addr(sb, B_A_FULL), 1);
@@ -687,9 +701,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 mbar_wait(bar_addr(sb, B_AL_FULL + (c & 1)), (c >> 1) & 1, abort_flag, err, kTimeoutNs / 4);
         }
     } else if (warp < 4) {
-        // ================= conversion (warps 1-3): decay factors, K/Q/V tiles; warp 3 issues the Gram ======
-        uint32_t gram_issuer = 0;
-        int gram_issued = 0;
+        // ================= conversion (warps 1-3): decay factors, K/Q/V tiles =================
         const int w = warp - 1;
         const int t_begin = conv_begin(w), t_end = conv_begin(w + 1);
         // one leader waits for the chunk's inputs; the conversion warps leave the loop together
@@ -723,30 +735,17 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 mbar_arrive(bar_addr(sb, B_GATE_FULL + s));
                 mbar_arrive(bar_addr(sb, B_AL_EMPTY + (c & 1)));
             }
-            if (warp == 3) {
-                int gram_ok = 0;
-                if (lane == 0)
-                    gram_ok = mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs) &&
-                              (c == 0 || mbar_wait(bar_addr(sb, B_G_EMPTY), (c - 1) & 1, abort_flag, err, kTimeoutNs));
-                if (__shfl_sync(0xffffffffu, gram_ok, 0)) {
-                    tc_fence_after();
-                    if (elect_one(gram_issuer)) issue_gram(sb, tmem, st, c & 1);
-                    __syncwarp();
-                    gram_issued = 1;
-                }
-            }
-        }
-        if (warp == 3 && lane == gram_issuer && gram_issued && *abort_flag) {
-            umma_commit(bar_addr(sb, B_DRAIN + 1));
-            mbar_wait(bar_addr(sb, B_DRAIN + 1), 0, abort_flag, err, kTimeoutNs / 4);
         }
     } else if (warp < 8) {
-        // ================= prep: Gram epilogue, diagonal inverses, back substitution, Z =========
+        // ======= prep: Gram epilogue, diagonal inverses, back substitution, Z; the next Gram =======
         const int t = threadIdx.x - 128;
         const int q = warp - 4;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
         Group grp{NB_PREP, 128, t == 0, okflags + 0, 0, abort_flag, err};
         float* adiag = reinterpret_cast<float*>(sbase + OFF_ADIAG);
+        uint32_t gram_issuer = 0;
+        int gram_issued = 0;
+        if (warp == 4 && nchunks > 0) gram_issued |= issue_gram_of(0, sb, tmem, lane, abort_flag, err, gram_issuer);
         for (int c = 0; c < nchunks; ++c) {
             const int tps = c & 1;
             if (!grp.wait(bar_addr(sb, B_G_FULL), c & 1, bar_addr(sb, B_TP_EMPTY + tps), ((c >> 1) & 1) ^ 1)) break;
@@ -758,7 +757,6 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             }
             tc_fence_before();
             grp.sync();
-            if (t == 0) mbar_arrive(bar_addr(sb, B_G_EMPTY));
             const uint32_t tp = sb + OFF_TP + tps * TP_STAGE;
             if (q == 0) diag_block_inverse_row(tp, lane, adiag + (lane >> 4) * ADIAG_BLOCK);
             grp.sync();
@@ -768,6 +766,11 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             fence_proxy_async_smem();
             grp.sync();
             if (t == 0) mbar_arrive(bar_addr(sb, B_TP_FULL + tps));
+            if (warp == 4 && c + 1 < nchunks) gram_issued |= issue_gram_of(c + 1, sb, tmem, lane, abort_flag, err, gram_issuer);
+        }
+        if (warp == 4 && lane == gram_issuer && gram_issued && *abort_flag) {
+            umma_commit(bar_addr(sb, B_DRAIN + 1));
+            mbar_wait(bar_addr(sb, B_DRAIN + 1), 0, abort_flag, err, kTimeoutNs / 4);
         }
     } else {
         // ======= the S-dependent chain (lane j = d_v column j of S; half h of the TMEM columns) =======
@@ -789,6 +792,8 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         }
         uint32_t drain_needed = 0;
         uint32_t mma_issuer = 0;
+        // the previous chunk's gate stage, released after the next group barrier (-1: none)
+        int pend_gate = -1;
         for (int c = 0; ok && c < nchunks; ++c) {
             const int s = c % kStages;
             const uint32_t ph = (c / kStages) & 1;
@@ -799,9 +804,13 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
             const Gates* gs = gate(s);
             const bool exact = !gates_in_range(gs);
+            const bool last = c + 1 == nchunks;
+            const int s1 = (c + 1) % kStages;
             if (!exact) {
                 // --- MMA_A: (K^ S, Q^ S)^T = S^T [K^; Q^]^T ---
                 grp.sync();
+                if (leader && pend_gate >= 0) mbar_arrive(bar_addr(sb, B_GATE_EMPTY + pend_gate));
+                pend_gate = -1;
                 if (warp == 8) {
                     int lok = 0;
                     if (leader)
@@ -900,7 +909,9 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                         *reinterpret_cast<__nv_bfloat16*>(ost + r * 128) = __float2bfloat16_rn(qp[r] - qp[16 + r]);
                     fence_proxy_async_smem();
                 }
-                ok = grp.wait(bar_addr(sb, B_S_FULL), ph_s);
+                // MMA_C done, and the next chunk's gates written
+                ok = grp.wait(bar_addr(sb, B_S_FULL), ph_s, last ? 0u : bar_addr(sb, B_GATE_FULL + s1),
+                              ((c + 1) / kStages) & 1);
                 ph_s ^= 1u;
                 if (!ok) break;
                 tc_fence_after();
@@ -918,32 +929,31 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 tc_fence_before();
                 // keep every hand-off in step: the stage and the [X; Z] stage are released
                 // once their producers are done with them, the output epilogue is released
-                ok = grp.wait(bar_addr(sb, B_CONV + s), ph, bar_addr(sb, B_TP_FULL + tps), (c >> 1) & 1);
+                ok = grp.wait(bar_addr(sb, B_CONV + s), ph, bar_addr(sb, B_TP_FULL + tps), (c >> 1) & 1,
+                              last ? 0u : bar_addr(sb, B_GATE_FULL + s1), ((c + 1) / kStages) & 1);
                 if (!ok) break;
                 if (leader) {
                     mbar_arrive(bar_addr(sb, B_EMPTY + s));
                     mbar_arrive(bar_addr(sb, B_TP_EMPTY + tps));
+                    if (pend_gate >= 0) mbar_arrive(bar_addr(sb, B_GATE_EMPTY + pend_gate));
                 }
+                pend_gate = -1;
             }
             // --- the new state ---
             // TM_S holds S' / sq after a tensor-core chunk, S' itself after an exact one
             const float* f_sh = exact ? nullptr : gs->sq;
-            if (c + 1 == nchunks) {
+            if (last) {
                 if (p.S_out)
                     store_final_state_scaled(tmem + TM_S + lane_addr, p.S_out + static_cast<int64_t>(ug) * kD * kD + j, f_sh,
                                              2 * h);
                 drain_needed = 0;
             } else {
-                const int s1 = (c + 1) % kStages;
-                ok = grp.wait(bar_addr(sb, B_GATE_FULL + s1), ((c + 1) / kStages) & 1);
-                if (!ok) break;
                 const Gates* g1 = gate(s1);
                 const bool exact1 = !gates_in_range(g1);
                 state_update(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr, f_sh, exact1 ? nullptr : g1->sq, 2 * h);
                 tc_fence_before();
+                pend_gate = s;
             }
-            grp.sync();
-            if (leader) mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
         }
         if (warp == 8 && lane == mma_issuer && drain_needed && !ok) {
             umma_commit(bar_addr(sb, B_DRAIN + 0));
