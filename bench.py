@@ -52,10 +52,10 @@ KERNEL_SOURCES = [os.path.join(ROOT, "gated_delta_rule_looped_b200", "csrc", f)
                   for f in ("gdr_prefill_tc.cu", "gdr_prefill_kda_tc.cu", "gdr_decode.cu", "sm100_primitives.cuh")]
 
 
-def kernel_sources(name):
+def kernel_sources(name, csrc=None):
     """The kernel's source file and every local header it includes, directly or not, in a fixed
     order: kernel code that lives in a shared header changes the kernel as much as its own file."""
-    csrc = os.path.join(ROOT, "gated_delta_rule_looped_b200", "csrc")
+    csrc = csrc or os.path.join(ROOT, "gated_delta_rule_looped_b200", "csrc")
     seen, todo = [], [name]
     while todo:
         f = todo.pop(0)
@@ -67,10 +67,11 @@ def kernel_sources(name):
     return seen
 
 
-def kernel_source_hash(name):
+def kernel_source_hash(name, csrc=None):
+    csrc = csrc or os.path.join(ROOT, "gated_delta_rule_looped_b200", "csrc")
     h = hashlib.sha256()
-    for f in kernel_sources(name):
-        with open(os.path.join(ROOT, "gated_delta_rule_looped_b200", "csrc", f), "rb") as fh:
+    for f in kernel_sources(name, csrc):
+        with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
 
@@ -84,17 +85,25 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def traffic_for(kernel, source):
+def traffic_for(kernel, source, bytes_launch=None, path=None):
     """DRAM bytes per launch from the committed ncu summary, if the kernel source still
-    matches the one that was profiled; else None."""
-    if not os.path.exists(PROFILE_TRAFFIC):
-        return None
-    with open(PROFILE_TRAFFIC) as f:
+    matches the one that was profiled; else None.  When the benchmarked launch moves a different
+    number of algorithmic bytes than the captured one (another workload of the same kernel), the
+    captured traffic is scaled by that ratio, since a launch's traffic grows with the token-heads
+    it processes.  Returns (bytes or None, a note saying how it was obtained or None)."""
+    path = path or PROFILE_TRAFFIC
+    if not os.path.exists(path):
+        return None, None
+    with open(path) as f:
         d = json.load(f)
     e = d.get(kernel)
     if not e or e.get("source_hash") != kernel_source_hash(source):
-        return None
-    return e.get("dram_bytes_per_launch_scaled")
+        return None, None
+    t = e.get("dram_bytes_per_launch_scaled")
+    a = e.get("algorithmic_bytes_per_launch")
+    if t is None or bytes_launch is None or not a or a == bytes_launch:
+        return t, None
+    return t * bytes_launch / a, f"scaled from the capture on {e.get('workload')} by algorithmic bytes per launch"
 
 
 # ---- clocks during the timed region ------------------------------------------------------
@@ -381,15 +390,18 @@ def main():
                       else ("gdr_prefill_kda_tc_kernel", "gdr_prefill_kda_tc.cu"))
     achieved_tf = flops_launch / launch_s / 1e12
     peak_tf = peaks["bf16_tflops"]
+    traffic, traffic_note = traffic_for(kernel, source, bytes_launch)
     roofline = {"bound": "tensor", "kernel": kernel, "achieved": achieved_tf, "peak": peak_tf,
                 "unit": "TFLOP/s", "frac": achieved_tf / peak_tf,
-                "traffic": traffic_for(kernel, source),
+                "traffic": traffic,
                 "peak_source": f"{peak_src} bf16 dense (fp16 operands run at the same rate)",
                 "algorithmic_per_launch": {"flop": flops_launch, "bytes": bytes_launch},
                 "hbm": {"achieved": bytes_launch / launch_s / 1e9, "peak": peaks["hbm_gbs"],
                         "unit": "GB/s", "frac": bytes_launch / launch_s / 1e9 / peaks["hbm_gbs"]},
                 "launch_time": "step time / T launches (the T loop launches of a step run back "
                                "to back and overlap through programmatic dependent launch)"}
+    if traffic_note:
+        roofline["traffic_note"] = traffic_note
 
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -411,7 +423,7 @@ def main():
                           "roofline": {"bound": "hbm", "kernel": "gdr_decode_kernel",
                                        "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                        "frac": gbs / peaks["hbm_gbs"],
-                                       "traffic": traffic_for("gdr_decode_kernel", "gdr_decode.cu"),
+                                       "traffic": traffic_for("gdr_decode_kernel", "gdr_decode.cu")[0],
                                        "peak_source": f"{peak_src} HBM copy"}}
 
     if not args.no_e2e:
