@@ -18,6 +18,12 @@ independent head-units), up-cast everything to fp64 and return fp64 results:
     decode_step          one token, state updated and returned
 
 ``oracle.twin`` holds a second, pure numpy implementation for tiny cases.
+
+Order of the per-key factors.  ``order="delta_first"`` (the default) is the equation as printed,
+A_t = Diag(alpha_t)(I - beta_t k_t k_t^T).  ``order="decay_first"`` takes
+A_t = (I - beta_t k_t k_t^T) Diag(alpha_t), the order a right-multiplying convention for the
+state would give; the page's equation fixes the first, the second is the other reading of the
+same symbols.  For scalar gating both are the same matrix.
 """
 import ctypes
 import os
@@ -68,6 +74,15 @@ def _ptr(a):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
 
 
+def _gate_code(per_key, order):
+    """Gate code of the C oracle: 0 scalar, 1 per-key delta first, 2 per-key decay first."""
+    if order not in ("delta_first", "decay_first"):
+        raise ValueError(f"order must be 'delta_first' or 'decay_first', got {order!r}")
+    if not per_key:
+        return 0
+    return 2 if order == "decay_first" else 1
+
+
 def _prep(q, k, v, alpha, beta, S0, per_key):
     q, k, v, alpha, beta = map(_f64, (q, k, v, alpha, beta))
     if q.shape != k.shape or q.ndim < 2:
@@ -92,10 +107,12 @@ def _prep(q, k, v, alpha, beta, S0, per_key):
     return q, k, v, alpha, beta, S0, o, S, U, L, dk, dv
 
 
-def prefill_sequential(q, k, v, alpha, beta, S0=None, per_key=False, nthreads=0, lib=None):
+def prefill_sequential(q, k, v, alpha, beta, S0=None, per_key=False, nthreads=0, lib=None,
+                       order="delta_first"):
     """Token-by-token recurrence. Returns (o [..., L, d_v], S_L [..., d_k, d_v]) in fp64."""
+    g = _gate_code(per_key, order)
     q, k, v, alpha, beta, S0, o, S, U, L, dk, dv = _prep(q, k, v, alpha, beta, S0, per_key)
-    rc = _lib(lib).gdr_ref_sequential(U, L, dk, dv, int(per_key), _ptr(q), _ptr(k), _ptr(v),
+    rc = _lib(lib).gdr_ref_sequential(U, L, dk, dv, g, _ptr(q), _ptr(k), _ptr(v),
                                    _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(o), _ptr(S),
                                    int(nthreads))
     if rc != 0:
@@ -103,10 +120,11 @@ def prefill_sequential(q, k, v, alpha, beta, S0=None, per_key=False, nthreads=0,
     return o, S
 
 
-def prefill_dense(q, k, v, alpha, beta, S0=None, per_key=False, nthreads=0):
+def prefill_dense(q, k, v, alpha, beta, S0=None, per_key=False, nthreads=0, order="delta_first"):
     """Same recurrence with A_t materialised as a d_k x d_k matrix (brute force)."""
+    g = _gate_code(per_key, order)
     q, k, v, alpha, beta, S0, o, S, U, L, dk, dv = _prep(q, k, v, alpha, beta, S0, per_key)
-    rc = _lib().gdr_ref_dense(U, L, dk, dv, int(per_key), _ptr(q), _ptr(k), _ptr(v),
+    rc = _lib().gdr_ref_dense(U, L, dk, dv, g, _ptr(q), _ptr(k), _ptr(v),
                               _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(o), _ptr(S),
                               int(nthreads))
     if rc != 0:
@@ -115,11 +133,12 @@ def prefill_dense(q, k, v, alpha, beta, S0=None, per_key=False, nthreads=0):
 
 
 def prefill_chunked(q, k, v, alpha, beta, S0=None, per_key=False, chunk=64, form="e",
-                    nthreads=0):
+                    nthreads=0, order="delta_first"):
     """Chunk-parallel rewriting; ``form`` is "u" (scalar gating only) or "e" (either)."""
+    g = _gate_code(per_key, order)
     q, k, v, alpha, beta, S0, o, S, U, L, dk, dv = _prep(q, k, v, alpha, beta, S0, per_key)
     f = {"u": 0, "e": 1}[form]
-    rc = _lib().gdr_ref_chunked(U, L, dk, dv, int(per_key), int(chunk), f, _ptr(q), _ptr(k),
+    rc = _lib().gdr_ref_chunked(U, L, dk, dv, g, int(chunk), f, _ptr(q), _ptr(k),
                                 _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(o), _ptr(S),
                                 int(nthreads))
     if rc != 0:
@@ -127,7 +146,7 @@ def prefill_chunked(q, k, v, alpha, beta, S0=None, per_key=False, chunk=64, form
     return o, S
 
 
-def decode_step(q, k, v, alpha, beta, S, per_key=False, nthreads=0, lib=None):
+def decode_step(q, k, v, alpha, beta, S, per_key=False, nthreads=0, lib=None, order="delta_first"):
     """One token per unit. q, k: [..., d_k]; v: [..., d_v]; alpha: [...] or [..., d_k];
     beta: [...]; S: [..., d_k, d_v].  Returns (o [..., d_v], S_new)."""
     q = _f64(q)[..., None, :]
@@ -137,7 +156,7 @@ def decode_step(q, k, v, alpha, beta, S, per_key=False, nthreads=0, lib=None):
     alpha = alpha[..., None, :] if per_key else alpha[..., None]
     beta = _f64(beta)[..., None]
     o, S_new = prefill_sequential(q, k, v, alpha, beta, S0=S, per_key=per_key,
-                                  nthreads=nthreads, lib=lib)
+                                  nthreads=nthreads, lib=lib, order=order)
     return o[..., 0, :], S_new
 
 

@@ -15,6 +15,12 @@
  * after token t's update, with no extra scale.  alpha_t is either one scalar per token
  * (GDN gating: Diag(alpha) = alpha I) or one value per key channel (a d_k vector).
  *
+ * The gate code `per_key` of every entry point: 0 scalar gating; 1 per-key gating in the
+ * order the equation is printed (delta, then decay: A_t = Diag(alpha_t)(I - beta_t k_t k_t^T));
+ * 2 per-key gating with the decay first, A_t = (I - beta_t k_t k_t^T) Diag(alpha_t), the
+ * order a right-multiplying convention for S would give.  For scalar alpha the two orders
+ * are the same matrix.
+ *
  * Loops.  Section "Profondita presa in prestito" of the same page applies one weight-tied
  * block T times; the section "Dove il quadro si incrina" lists carrying the recurrent
  * state from one loop to the next as unexplored.  So every (loop, batch, head) triple is
@@ -66,17 +72,32 @@ static void seq_unit(int64_t L, int64_t dk, int64_t dv, int per_key,
         const double* vt = v + t * dv;
         const double  bt = beta[t];
 
-        /* e = k_t^T S_{t-1}  (a d_v row vector) */
+        if (per_key == 2) {
+            /* decay first: S <- Diag(alpha_t) S_{t-1}, then the delta step on it */
+            for (int64_t i = 0; i < dk; ++i) {
+                const double ai = gate_at(alpha, per_key, t, i, dk);
+                for (int64_t j = 0; j < dv; ++j) S[IDX2(i, j, dv)] *= ai;
+            }
+        }
+
+        /* e = k_t^T S  (a d_v row vector; S = S_{t-1}, or its decayed copy) */
         for (int64_t j = 0; j < dv; ++j) e[j] = 0.0;
         for (int64_t i = 0; i < dk; ++i)
             for (int64_t j = 0; j < dv; ++j)
                 e[j] += kt[i] * S[IDX2(i, j, dv)];
 
-        /* S_t = Diag(alpha_t) (S_{t-1} - beta_t k_t e) + beta_t k_t v_t^T */
-        for (int64_t i = 0; i < dk; ++i) {
-            const double ai = gate_at(alpha, per_key, t, i, dk);
-            for (int64_t j = 0; j < dv; ++j)
-                S[IDX2(i, j, dv)] = ai * (S[IDX2(i, j, dv)] - bt * kt[i] * e[j]) + bt * kt[i] * vt[j];
+        if (per_key == 2) {
+            /* S_t = S - beta_t k_t e + beta_t k_t v_t^T */
+            for (int64_t i = 0; i < dk; ++i)
+                for (int64_t j = 0; j < dv; ++j)
+                    S[IDX2(i, j, dv)] += bt * kt[i] * (vt[j] - e[j]);
+        } else {
+            /* S_t = Diag(alpha_t) (S_{t-1} - beta_t k_t e) + beta_t k_t v_t^T */
+            for (int64_t i = 0; i < dk; ++i) {
+                const double ai = gate_at(alpha, per_key, t, i, dk);
+                for (int64_t j = 0; j < dv; ++j)
+                    S[IDX2(i, j, dv)] = ai * (S[IDX2(i, j, dv)] - bt * kt[i] * e[j]) + bt * kt[i] * vt[j];
+            }
         }
 
         /* o_t = S_t^T q_t */
@@ -105,12 +126,13 @@ static void dense_unit(int64_t L, int64_t dk, int64_t dv, int per_key,
         const double* vt = v + t * dv;
         const double  bt = beta[t];
 
-        /* A_t[i][m] = alpha_t[i] * (delta_im - beta_t k_t[i] k_t[m]) */
-        for (int64_t i = 0; i < dk; ++i) {
-            const double ai = gate_at(alpha, per_key, t, i, dk);
-            for (int64_t m = 0; m < dk; ++m)
-                A[IDX2(i, m, dk)] = ai * ((i == m ? 1.0 : 0.0) - bt * kt[i] * kt[m]);
-        }
+        /* A_t[i][m] = alpha_t[i] (delta_im - beta_t k_t[i] k_t[m]);
+           decay first: A_t[i][m] = (delta_im - beta_t k_t[i] k_t[m]) alpha_t[m] */
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t m = 0; m < dk; ++m) {
+                const double a = gate_at(alpha, per_key, t, per_key == 2 ? m : i, dk);
+                A[IDX2(i, m, dk)] = a * ((i == m ? 1.0 : 0.0) - bt * kt[i] * kt[m]);
+            }
         /* Snew = A_t S + beta_t k_t v_t^T */
         for (int64_t i = 0; i < dk; ++i)
             for (int64_t j = 0; j < dv; ++j) {
@@ -139,6 +161,13 @@ static void dense_unit(int64_t L, int64_t dk, int64_t dv, int per_key,
 /* (the delta term of token s is hit by its own alpha_s, the write term is not).  Taking */
 /* k_r^T S_{r-1} of that expression gives a unit lower-triangular system for the e_r,    */
 /* solved by forward substitution; o_r = S_r^T q_r and the chunk's final state follow.   */
+/* With the decay first (gate code 2), e_r = k_r^T Diag(alpha_r) S_{r-1} and token s's    */
+/* delta term is decayed like its write term:                                            */
+/*                                                                                        */
+/*   S_r = decay(r,-1) S0 + sum_{s<=r} beta_s (decay(r,s) k_s) (v_s - e_s)^T             */
+/*                                                                                        */
+/* so every decay(., s-1) below becomes decay(., s) and the k_r-side decay(r-1, .) of    */
+/* the e system becomes decay(r, .).                                                      */
 /* This "e-form" covers both gatings.  For scalar gating the same algebra with           */
 /* u_r = v_r - alpha_r e_r collapses the two terms into one ("u-form"):                  */
 /*                                                                                        */
@@ -164,6 +193,7 @@ static void chunked_unit_eform(int64_t L, int64_t dk, int64_t dv, int per_key, i
 {
     if (S0) memcpy(S, S0, sizeof(double) * dk * dv);
     else    memset(S, 0, sizeof(double) * dk * dv);
+    const int64_t df = per_key == 2 ? 1 : 0;    /* decay first: shift the e-side indices */
 
     for (int64_t t0 = 0; t0 < L; t0 += C) {
         const int64_t n = (L - t0 < C) ? (L - t0) : C;
@@ -177,8 +207,8 @@ static void chunked_unit_eform(int64_t L, int64_t dk, int64_t dv, int per_key, i
             for (int64_t s = 0; s < r; ++s) {
                 double ke = 0.0, kv = 0.0;
                 for (int64_t i = 0; i < dk; ++i) {
-                    ke += kc[r * dk + i] * decay(alpha, per_key, t0, r - 1, s - 1, i, dk) * kc[s * dk + i];
-                    kv += kc[r * dk + i] * decay(alpha, per_key, t0, r - 1, s, i, dk) * kc[s * dk + i];
+                    ke += kc[r * dk + i] * decay(alpha, per_key, t0, r - 1 + df, s - 1 + df, i, dk) * kc[s * dk + i];
+                    kv += kc[r * dk + i] * decay(alpha, per_key, t0, r - 1 + df, s, i, dk) * kc[s * dk + i];
                 }
                 Mke[r * C + s] = bc[s] * ke;
                 Mkv[r * C + s] = bc[s] * kv;
@@ -189,7 +219,7 @@ static void chunked_unit_eform(int64_t L, int64_t dk, int64_t dv, int per_key, i
             for (int64_t j = 0; j < dv; ++j) {
                 double acc = 0.0;
                 for (int64_t i = 0; i < dk; ++i)
-                    acc += kc[r * dk + i] * decay(alpha, per_key, t0, r - 1, -1, i, dk) * S[IDX2(i, j, dv)];
+                    acc += kc[r * dk + i] * decay(alpha, per_key, t0, r - 1 + df, -1, i, dk) * S[IDX2(i, j, dv)];
                 for (int64_t s = 0; s < r; ++s)
                     acc += Mkv[r * C + s] * vc[s * dv + j] - Mke[r * C + s] * E[s * dv + j];
                 E[r * dv + j] = acc;
@@ -207,7 +237,7 @@ static void chunked_unit_eform(int64_t L, int64_t dk, int64_t dv, int per_key, i
                 double qv = 0.0, qe = 0.0;
                 for (int64_t i = 0; i < dk; ++i) {
                     qv += qc[r * dk + i] * decay(alpha, per_key, t0, r, s, i, dk) * kc[s * dk + i];
-                    qe += qc[r * dk + i] * decay(alpha, per_key, t0, r, s - 1, i, dk) * kc[s * dk + i];
+                    qe += qc[r * dk + i] * decay(alpha, per_key, t0, r, s - 1 + df, i, dk) * kc[s * dk + i];
                 }
                 for (int64_t j = 0; j < dv; ++j)
                     o[(t0 + r) * dv + j] += bc[s] * (qv * vc[s * dv + j] - qe * E[s * dv + j]);
@@ -220,7 +250,7 @@ static void chunked_unit_eform(int64_t L, int64_t dk, int64_t dv, int per_key, i
             for (int64_t j = 0; j < dv; ++j) Snew[IDX2(i, j, dv)] = g * S[IDX2(i, j, dv)];
             for (int64_t s = 0; s < n; ++s) {
                 const double wv = bc[s] * decay(alpha, per_key, t0, n - 1, s, i, dk) * kc[s * dk + i];
-                const double we = bc[s] * decay(alpha, per_key, t0, n - 1, s - 1, i, dk) * kc[s * dk + i];
+                const double we = bc[s] * decay(alpha, per_key, t0, n - 1, s - 1 + df, i, dk) * kc[s * dk + i];
                 for (int64_t j = 0; j < dv; ++j)
                     Snew[IDX2(i, j, dv)] += wv * vc[s * dv + j] - we * E[s * dv + j];
             }

@@ -9,7 +9,8 @@ equation), one head-unit at a time with Python loops.
 import numpy as np
 
 
-def prefill(q, k, v, alpha, beta, S0=None, per_key=False):
+def prefill(q, k, v, alpha, beta, S0=None, per_key=False, order="delta_first"):
+    """``order="decay_first"`` takes A_t = (I - beta_t k_t k_t^T) Diag(alpha_t) instead."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -33,7 +34,8 @@ def prefill(q, k, v, alpha, beta, S0=None, per_key=False):
         for t in range(L):
             kt = kf[u, t]
             diag = af[u, t] if per_key else np.full(dk, af[u, t])
-            A = np.diag(diag) @ (eye - bf[u, t] * np.outer(kt, kt))
+            delta = eye - bf[u, t] * np.outer(kt, kt)
+            A = delta @ np.diag(diag) if order == "decay_first" else np.diag(diag) @ delta
             S = A @ S + bf[u, t] * np.outer(kt, vf[u, t])
             o[u, t] = S.T @ qf[u, t]
         S_out[u] = S

@@ -59,12 +59,12 @@ def pin_overwrite(lib=None, seed=1):
 
 
 # --- P2: beta = 0 leaves only the decay: S_t = Diag(prod_{s<=t} a_s) S_0, o_t = S_t^T q_t.
-def pin_beta_zero(lib=None, per_key=False, seed=2):
+def pin_beta_zero(lib=None, per_key=False, seed=2, order="delta_first"):
     rng = np.random.default_rng(seed)
     U, L, dk, dv = 3, 25, 9, 5
     q, k, v, alpha, _, S0 = rand_case(rng, U, L, dk, dv, per_key, alpha_lo=0.5)
     beta = np.zeros((U, L))
-    o, S = oracle.prefill_sequential(q, k, v, alpha, beta, S0=S0, per_key=per_key, lib=lib)
+    o, S = oracle.prefill_sequential(q, k, v, alpha, beta, S0=S0, per_key=per_key, lib=lib, order=order)
     a = alpha if per_key else np.repeat(alpha[..., None], dk, axis=-1)
     g = np.cumprod(a, axis=1)                                 # [U, L, dk]
     St = g[..., :, None] * S0[:, None, :, :]                  # [U, L, dk, dv]
@@ -77,7 +77,7 @@ def pin_beta_zero(lib=None, per_key=False, seed=2):
 
 # --- P3: mutually orthogonal unit keys and S_0 = 0 make every delta term vanish, so the
 # mixer is decayed linear attention: o_t = sum_{s<=t} b_s (prod_{s<s'<=t} a_s') (q_t.k_s) v_s.
-def pin_orthogonal_keys(lib=None, per_key=False, seed=3):
+def pin_orthogonal_keys(lib=None, per_key=False, seed=3, order="delta_first"):
     rng = np.random.default_rng(seed)
     U, dk, dv = 2, 12, 6
     L = dk
@@ -95,7 +95,7 @@ def pin_orthogonal_keys(lib=None, per_key=False, seed=3):
     else:
         k = np.stack([np.linalg.qr(rng.standard_normal((dk, dk)))[0].T[:L] for _ in range(U)])
         alpha = rng.uniform(0.5, 1.0, size=(U, L))
-    o, _ = oracle.prefill_sequential(q, k, v, alpha, beta, S0=None, per_key=per_key, lib=lib)
+    o, _ = oracle.prefill_sequential(q, k, v, alpha, beta, S0=None, per_key=per_key, lib=lib, order=order)
     o_ref = np.zeros_like(o)
     for u in range(U):
         for t in range(L):
@@ -167,6 +167,38 @@ def pin_overwrite_identity(lib=None, seed=10):
     return 0.0
 
 
+# --- P7 (decay-first order, A_t = (I - b_t k_t k_t^T) Diag(a_t)): the delta step acts on the
+# already decayed state, so with b = 1 and unit keys the write is an exact overwrite whatever
+# the per-key decay: S_t^T k_t = v_t.  (In the printed order the decay comes after the write
+# and breaks this as soon as a != 1.)
+def pin_overwrite_decay_first(lib=None, seed=11):
+    rng = np.random.default_rng(seed)
+    U, L, dk, dv = 2, 30, 12, 5
+    k = _unit(rng.standard_normal((U, L, dk)))
+    v = rng.standard_normal((U, L, dv))
+    S0 = rng.standard_normal((U, dk, dv))
+    alpha = rng.uniform(0.3, 1.0, size=(U, L, dk))
+    ones = np.ones((U, L))
+    o, _ = oracle.prefill_sequential(k, k, v, alpha, ones, S0=S0, per_key=True, lib=lib, order="decay_first")
+    err = np.max(np.abs(o - v)) / np.max(np.abs(v))
+    assert err < 1e-12, f"decay-first overwrite broken: {err}"
+    return err
+
+
+# --- P8: per-key decay equal on every key is scalar gating, for which both orders are the
+# same matrix; the decay-first per-key path must then agree with the scalar path.
+def pin_uniform_alpha_decay_first(lib=None, seed=12):
+    rng = np.random.default_rng(seed)
+    U, L, dk, dv = 2, 23, 8, 6
+    q, k, v, alpha, beta, S0 = rand_case(rng, U, L, dk, dv, per_key=False, alpha_lo=0.5)
+    o_s, S_s = oracle.prefill_sequential(q, k, v, alpha, beta, S0=S0, per_key=False, lib=lib)
+    a_vec = np.repeat(alpha[..., None], dk, axis=-1)
+    o_d, S_d = oracle.prefill_sequential(q, k, v, a_vec, beta, S0=S0, per_key=True, lib=lib, order="decay_first")
+    err = max(np.max(np.abs(o_d - o_s)) / np.max(np.abs(o_s)), np.max(np.abs(S_d - S_s)) / np.max(np.abs(S_s)))
+    assert err < 1e-12, f"uniform per-key decay-first differs from scalar gating: {err}"
+    return err
+
+
 ALL_PINS = [
     ("overwrite", lambda lib: pin_overwrite(lib)),
     ("beta_zero", lambda lib: pin_beta_zero(lib, per_key=False)),
@@ -177,4 +209,8 @@ ALL_PINS = [
     ("non_expansive", lambda lib: pin_non_expansive(lib, per_key=False)),
     ("non_expansive_per_key", lambda lib: pin_non_expansive(lib, per_key=True)),
     ("overwrite_identity", lambda lib: pin_overwrite_identity(lib)),
+    ("overwrite_decay_first", lambda lib: pin_overwrite_decay_first(lib)),
+    ("uniform_alpha_decay_first", lambda lib: pin_uniform_alpha_decay_first(lib)),
+    ("beta_zero_decay_first", lambda lib: pin_beta_zero(lib, per_key=True, order="decay_first")),
+    ("orthogonal_decay_first", lambda lib: pin_orthogonal_keys(lib, per_key=True, order="decay_first")),
 ]

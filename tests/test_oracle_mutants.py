@@ -43,6 +43,15 @@ MUTANTS = [
     ("per_key_gate_reversed", "gate_at",
      "return per_key ? alpha[t * dk + i] : alpha[t];",
      "return per_key ? alpha[t * dk + (dk - 1 - i)] : alpha[t];"),
+    # decay-first order: the decay skipped, or applied to the write term as well
+    ("decay_first_decay_skipped", "seq_unit",
+     "for (int64_t j = 0; j < dv; ++j) S[IDX2(i, j, dv)] *= ai;",
+     "for (int64_t j = 0; j < dv; ++j) S[IDX2(i, j, dv)] *= 1.0;"),
+    ("decay_first_projects_undecayed", "seq_unit",
+     "S[IDX2(i, j, dv)] += bt * kt[i] * (vt[j] - e[j]);",
+     "S[IDX2(i, j, dv)] += bt * kt[i] * (vt[j] - e[j] / gate_at(alpha, per_key, t, i, dk));"),
+    ("decay_first_delta_first", "seq_unit",
+     "if (per_key == 2) {\n            /* decay first", "if (0) {\n            /* decay first"),
 ]
 
 

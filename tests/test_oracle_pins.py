@@ -18,27 +18,28 @@ def test_pin(name, check):
     check(None)
 
 
-@pytest.mark.parametrize("per_key", [False, True])
-def test_sequential_dense_twin_agree(per_key):
+@pytest.mark.parametrize("per_key,order", [(False, "delta_first"), (True, "delta_first"), (True, "decay_first")])
+def test_sequential_dense_twin_agree(per_key, order):
     # c2: the transition matrix built densely (C code and an independent numpy twin).
     rng = np.random.default_rng(11)
     q, k, v, a, b, S0 = rand_case(rng, 3, 13, 6, 5, per_key)
-    o1, S1 = oracle.prefill_sequential(q, k, v, a, b, S0=S0, per_key=per_key)
-    o2, S2 = oracle.prefill_dense(q, k, v, a, b, S0=S0, per_key=per_key)
-    o3, S3 = twin.prefill(q, k, v, a, b, S0=S0, per_key=per_key)
+    o1, S1 = oracle.prefill_sequential(q, k, v, a, b, S0=S0, per_key=per_key, order=order)
+    o2, S2 = oracle.prefill_dense(q, k, v, a, b, S0=S0, per_key=per_key, order=order)
+    o3, S3 = twin.prefill(q, k, v, a, b, S0=S0, per_key=per_key, order=order)
     for x, y in ((o2, o1), (S2, S1), (o3, o1), (S3, S1)):
         assert np.max(np.abs(x - y)) <= 1e-13 * max(1.0, np.max(np.abs(y)))
 
 
 @pytest.mark.parametrize("C", [1, 2, 8, 16, 64])
 @pytest.mark.parametrize("L", [1, 5, 63, 64, 65, 200])
-@pytest.mark.parametrize("per_key,form", [(False, "u"), (False, "e"), (True, "e")])
-def test_chunked_equals_sequential(C, L, per_key, form):
+@pytest.mark.parametrize("per_key,form,order", [(False, "u", "delta_first"), (False, "e", "delta_first"),
+                                                (True, "e", "delta_first"), (True, "e", "decay_first")])
+def test_chunked_equals_sequential(C, L, per_key, form, order):
     # P4: the chunk-parallel rewriting used by the GPU equals the token-by-token equation.
     rng = np.random.default_rng(1000 + C + 7 * L + (13 if per_key else 0))
     q, k, v, a, b, S0 = rand_case(rng, 2, L, 8, 5, per_key)
-    o1, S1 = oracle.prefill_sequential(q, k, v, a, b, S0=S0, per_key=per_key)
-    o2, S2 = oracle.prefill_chunked(q, k, v, a, b, S0=S0, per_key=per_key, chunk=C, form=form)
+    o1, S1 = oracle.prefill_sequential(q, k, v, a, b, S0=S0, per_key=per_key, order=order)
+    o2, S2 = oracle.prefill_chunked(q, k, v, a, b, S0=S0, per_key=per_key, chunk=C, form=form, order=order)
     assert oracle.rel_max_err(o2, o1) < 1e-12
     assert oracle.rel_max_err(S2, S1) < 1e-12
 
@@ -108,3 +109,19 @@ def test_empty_sequence_returns_initial_state():
 def test_parity_metric():
     ref = np.array([3.0, -4.0])          # rms = sqrt(12.5)
     assert abs(oracle.rel_max_err(ref + [0.5, 0.0], ref) - 0.5 / np.sqrt(12.5)) < 1e-15
+
+
+def test_orders_differ_per_key_and_agree_for_scalar_decay():
+    # The two readings of the per-key equation are different recurrences (so the pins above
+    # tell them apart), except when the decay is the same on every key.
+    rng = np.random.default_rng(13)
+    q, k, v, a, b, S0 = rand_case(rng, 2, 17, 6, 4, True, alpha_lo=0.5)
+    o1, _ = oracle.prefill_sequential(q, k, v, a, b, S0=S0, per_key=True)
+    o2, _ = oracle.prefill_sequential(q, k, v, a, b, S0=S0, per_key=True, order="decay_first")
+    assert oracle.rel_max_err(o2, o1) > 1e-2
+    a1 = np.repeat(a[..., :1], 6, axis=-1)
+    o1, _ = oracle.prefill_sequential(q, k, v, a1, b, S0=S0, per_key=True)
+    o2, _ = oracle.prefill_sequential(q, k, v, a1, b, S0=S0, per_key=True, order="decay_first")
+    assert oracle.rel_max_err(o2, o1) < 1e-13
+    with pytest.raises(ValueError):
+        oracle.prefill_sequential(q, k, v, a, b, S0=S0, per_key=True, order="sideways")
