@@ -216,12 +216,17 @@ def timed(fn, steps, warmup, world, sampler=None):
     return max_over_ranks(ms, world)
 
 
-def prefill_case(w, device):
+def gate_of(w, order):
+    if w.gate != "per_key":
+        return lt2.LT2_GATE_SCALAR
+    return lt2.LT2_GATE_PER_KEY_DECAY_FIRST if order == "decay_first" else lt2.LT2_GATE_PER_KEY
+
+
+def prefill_case(w, device, order="delta_first"):
     x = inputs.make_inputs(w, seed=0, device=device)
     o = torch.empty(x["v"].shape, dtype=torch.bfloat16, device=device)
     S = torch.empty((w.T, w.B, w.H, w.d, w.d), dtype=torch.float32, device=device)
-    dims = lt2.make_dims(w.T, w.B, w.H, w.L, w.d, w.d, lt2.LT2_DTYPE_BF16,
-                         lt2.LT2_GATE_PER_KEY if w.gate == "per_key" else lt2.LT2_GATE_SCALAR)
+    dims = lt2.make_dims(w.T, w.B, w.H, w.L, w.d, w.d, lt2.LT2_DTYPE_BF16, gate_of(w, order))
     ws_bytes = lt2.lt2_gdr_prefill_workspace_bytes(dims)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device) if ws_bytes else None
 
@@ -281,7 +286,7 @@ def run_decode(world, steps, warmup):
 
 # ---- CPU oracle (reported baseline / reference arm) -----------------------------------------
 
-def oracle_sample(w, target_s=15.0):
+def oracle_sample(w, target_s=15.0, order="delta_first"):
     """Time the fp64 oracle on a bounded sample of workload w's head-units on this host.
     Returns (tokens*loops per second, threads used, description)."""
     import oracle
@@ -296,7 +301,7 @@ def oracle_sample(w, target_s=15.0):
     # calibrate on one unit, then size the sample to ~target_s of wall time
     a = draw(1, 1)
     t0 = time.perf_counter()
-    oracle.prefill_sequential(*a, per_key=(w.gate == "per_key"), nthreads=1)
+    oracle.prefill_sequential(*a, per_key=(w.gate == "per_key"), nthreads=1, order=order)
     t1 = time.perf_counter() - t0
     per_unit_parallel = t1 / threads
     n = max(threads, int(target_s / max(per_unit_parallel, 1e-6)) // threads * threads)
@@ -304,7 +309,7 @@ def oracle_sample(w, target_s=15.0):
     threads = min(threads, n)
     a = draw(n, 2)
     t0 = time.perf_counter()
-    oracle.prefill_sequential(*a, per_key=(w.gate == "per_key"), nthreads=threads)
+    oracle.prefill_sequential(*a, per_key=(w.gate == "per_key"), nthreads=threads, order=order)
     dt = time.perf_counter() - t0
     tok_loops = n * L / w.H          # a token*loop needs all H heads
     desc = (f"{n} of {w.units} (loop, batch, head) units of {w.name}, L={L}, fp64 sequential "
@@ -320,15 +325,15 @@ def reference_arm(args, world, rank):
     vals = []
     desc = threads = None
     for _ in range(args.warmup):
-        oracle_sample(w, target_s=2.0)
+        oracle_sample(w, target_s=2.0, order=args.order)
     for _ in range(args.steps):
-        v, threads, desc = oracle_sample(w, target_s=max(2.0, 20.0 / max(args.steps, 1)))
+        v, threads, desc = oracle_sample(w, target_s=max(2.0, 20.0 / max(args.steps, 1)), order=args.order)
         vals.append(v)
     value = statistics.median(vals)
     line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": config_of(w, args.gpus),
+            "data": "synthetic", "config": config_of(w, args.gpus, args.order),
             "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -339,9 +344,10 @@ def metric_of(w):
     return f"looped GDR prefill tokens*loops/s ({w.name})", "tokens*loops/s"
 
 
-def config_of(w, n_gpus):
+def config_of(w, n_gpus, order="delta_first"):
+    gate = w.gate if w.gate != "per_key" or order == "delta_first" else "per_key, decay first"
     return {"workload": w.name, "T": w.T, "B": w.B, "H": w.H, "L": w.L, "d_k": w.d, "d_v": w.d,
-            "gate": w.gate, "chunk": 32 if w.gate == "per_key" else 64, "io_dtype": w.dtype,
+            "gate": gate, "chunk": 32 if w.gate == "per_key" else 64, "io_dtype": w.dtype,
             "state_dtype": "f32",
             "parallelism": f"replicas x{n_gpus} (independent head-units, no collective)",
             "l2": "inputs larger than L2 (no flush needed)"}
@@ -355,6 +361,8 @@ def main():
     ap.add_argument("--workload", default="gdn_prefill",
                     choices=["gdn_prefill", "kda_prefill", "long_gdn"])
     ap.add_argument("--impl", default="lt2", choices=["lt2", "reference"])
+    ap.add_argument("--order", default="delta_first", choices=["delta_first", "decay_first"],
+                    help="order of the per-key factors (per-key workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
@@ -372,7 +380,7 @@ def main():
     metric, unit = metric_of(w)
     peaks, peak_src = load_peaks()
 
-    x, o, S, dims, step = prefill_case(w, "cuda")
+    x, o, S, dims, step = prefill_case(w, "cuda", args.order)
     sampler = ClockSampler(local) if rank == 0 else None
     ms = timed(step, args.steps, args.warmup, world, sampler)
     if lt2.lt2_gdr_last_device_error() != lt2.LT2_OK:
@@ -406,7 +414,7 @@ def main():
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-            "config": config_of(w, world), "roofline": roofline,
+            "config": config_of(w, world, args.order), "roofline": roofline,
             "gpu_launches": args.steps * w.T}
     if clocks:
         line["clocks"] = clocks
@@ -432,7 +440,7 @@ def main():
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, threads, desc = oracle_sample(w)
+        v, threads, desc = oracle_sample(w, order=args.order)
         line["cpu_baseline"] = {"value": v, "unit": unit, "cores": threads, "kind": "oracle",
                                 "sample": desc}
 

@@ -26,6 +26,7 @@ LT2_DTYPE_F32 = 0
 LT2_DTYPE_BF16 = 1
 LT2_GATE_SCALAR = 0
 LT2_GATE_PER_KEY = 1
+LT2_GATE_PER_KEY_DECAY_FIRST = 2
 LT2_ALGO_AUTO = 0
 LT2_ALGO_TENSOR_CORE = 1
 LT2_ALGO_CUDA_CORE = 2
@@ -155,7 +156,17 @@ def _out_torch_dtype(in_dtype, out):
     return torch.float32 if out == "f32" else torch.bfloat16
 
 
-def _dims_from(q, v, alpha, per_key, algo, out=None):
+def _gate(per_key, order):
+    """lt2_gate for a gating and an order of the per-key factors ("delta_first", the equation
+    as printed, or "decay_first"); the order does not matter for scalar gating."""
+    if order not in ("delta_first", "decay_first"):
+        raise ValueError(f"order must be 'delta_first' or 'decay_first', got {order!r}")
+    if not per_key:
+        return LT2_GATE_SCALAR
+    return LT2_GATE_PER_KEY_DECAY_FIRST if order == "decay_first" else LT2_GATE_PER_KEY
+
+
+def _dims_from(q, v, alpha, per_key, algo, out=None, order="delta_first"):
     import torch
     if q.dim() != 5 or v.dim() != 5:
         raise ValueError("q, k, v must be [T, B, H, L, d]")
@@ -166,16 +177,16 @@ def _dims_from(q, v, alpha, per_key, algo, out=None):
         raise ValueError(f"unsupported dtype {q.dtype}")
     if per_key is None:
         per_key = alpha.dim() == 5
-    return make_dims(T, B, H, L, dk, dv, dt, LT2_GATE_PER_KEY if per_key else LT2_GATE_SCALAR,
-                     algo, _OUT[out])
+    return make_dims(T, B, H, L, dk, dv, dt, _gate(per_key, order), algo, _OUT[out])
 
 
 def prefill(q, k, v, alpha, beta, S0=None, per_key=None, algo=LT2_ALGO_AUTO, o=None,
-            S_out=None, out=None, stream=None):
+            S_out=None, out=None, stream=None, order="delta_first"):
     """Run the looped prefill on CUDA tensors; returns (o, S_out).  ``out`` selects the
-    storage type of o: None/"same" (as the inputs), "f32" or "bf16"."""
+    storage type of o: None/"same" (as the inputs), "f32" or "bf16"; ``order`` the order of
+    the per-key factors ("delta_first" as printed, or "decay_first")."""
     import torch
-    dims = _dims_from(q, v, alpha, per_key, algo, out)
+    dims = _dims_from(q, v, alpha, per_key, algo, out, order)
     if o is None:
         o = torch.empty(v.shape, dtype=_out_torch_dtype(q.dtype, out), device=v.device)
     if S_out is None:
@@ -189,15 +200,14 @@ def prefill(q, k, v, alpha, beta, S0=None, per_key=None, algo=LT2_ALGO_AUTO, o=N
     return o, S_out
 
 
-def decode(q, k, v, alpha, beta, S, per_key=None, o=None, out=None, stream=None):
+def decode(q, k, v, alpha, beta, S, per_key=None, o=None, out=None, stream=None, order="delta_first"):
     """One decode token per (loop, batch, head); q/k/v [T,B,H,d]; S updated in place."""
     import torch
     per_key = (alpha.dim() == 4) if per_key is None else per_key
     T, B, H, dk = q.shape
     dv = v.shape[-1]
     dt = {torch.float32: LT2_DTYPE_F32, torch.bfloat16: LT2_DTYPE_BF16}[q.dtype]
-    dims = make_dims(T, B, H, 1, dk, dv, dt, LT2_GATE_PER_KEY if per_key else LT2_GATE_SCALAR,
-                     out_dtype=_OUT[out])
+    dims = make_dims(T, B, H, 1, dk, dv, dt, _gate(per_key, order), out_dtype=_OUT[out])
     if o is None:
         o = torch.empty(v.shape, dtype=_out_torch_dtype(q.dtype, out), device=v.device)
     st = lt2_gdr_decode(dims, q, k, v, alpha, beta, S, o, stream)

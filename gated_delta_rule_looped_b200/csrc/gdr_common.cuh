@@ -28,6 +28,7 @@ struct LoopSlice {
     int dk;
     int dv;
     int per_key;
+    int decay_first;     // per-key gating applied as (I - beta k k^T) Diag(alpha)
     int out_bf16;        // o stored as bf16 (else fp32)
     unsigned int* err;   // device status word
 };

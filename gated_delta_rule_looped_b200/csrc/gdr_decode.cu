@@ -11,6 +11,11 @@
 // (alpha.q)^T S) come from ONE read of S: each state is streamed through HBM exactly once
 // (64 KiB read + 64 KiB written for d = 128), which is the whole cost of the step.
 //
+// Per-key gating in the decay-first order, A = (I - beta k k^T) Diag(alpha):
+//
+//   e   = (alpha . k)^T S,   S' = Diag(alpha) S - beta k e + beta k v^T
+//   o   = S^T (alpha . q) - beta (q . k) e + beta (q . k) v
+//
 // Mapping: one CTA of 256 threads per head-unit.  Warp w owns the contiguous rows
 // [w*dk/8, (w+1)*dk/8); lane c owns columns 4c..4c+3 (one 16-byte access per row), so
 // every warp-wide access touches whole 128-byte lines.  The per-column partial sums are
@@ -21,7 +26,7 @@
 
 namespace lt2 {
 
-template <typename T, typename To>
+template <typename T, typename To, bool kDecayFirst>
 __global__ void __launch_bounds__(256, 2) gdr_decode_kernel(LoopSlice p, int use_pdl)
 {
     (void)use_pdl;
@@ -91,7 +96,7 @@ __global__ void __launch_bounds__(256, 2) gdr_decode_kernel(LoopSlice p, int use
         if (m < rpw && active) {
             const int r = r0 + m;
             s[m] = ld_stream_f4(S + (int64_t)r * dv + col);
-            const float kr = sk[r], ar = saq[r];
+            const float kr = kDecayFirst ? sk[r] * sa[r] : sk[r], ar = saq[r];
             e.x += kr * s[m].x; e.y += kr * s[m].y; e.z += kr * s[m].z; e.w += kr * s[m].w;
             f.x += ar * s[m].x; f.y += ar * s[m].y; f.z += ar * s[m].z; f.w += ar * s[m].w;
         }
@@ -120,16 +125,23 @@ __global__ void __launch_bounds__(256, 2) gdr_decode_kernel(LoopSlice p, int use
             const float bk = beta * sk[r];
             const float ar = sa[r];
             float4 n;
-            n.x = ar * (s[m].x - bk * E.x) + bk * vv.x;
-            n.y = ar * (s[m].y - bk * E.y) + bk * vv.y;
-            n.z = ar * (s[m].z - bk * E.z) + bk * vv.z;
-            n.w = ar * (s[m].w - bk * E.w) + bk * vv.w;
+            if (kDecayFirst) {
+                n.x = ar * s[m].x + bk * (vv.x - E.x);
+                n.y = ar * s[m].y + bk * (vv.y - E.y);
+                n.z = ar * s[m].z + bk * (vv.z - E.z);
+                n.w = ar * s[m].w + bk * (vv.w - E.w);
+            } else {
+                n.x = ar * (s[m].x - bk * E.x) + bk * vv.x;
+                n.y = ar * (s[m].y - bk * E.y) + bk * vv.y;
+                n.z = ar * (s[m].z - bk * E.z) + bk * vv.z;
+                n.w = ar * (s[m].w - bk * E.w) + bk * vv.w;
+            }
             st_stream_f4(S + (int64_t)r * dv + col, n);
         }
     }
 
     if (w == 0) {
-        const float c1 = beta * s_aqk, c2 = beta * s_qk;
+        const float c1 = beta * (kDecayFirst ? s_qk : s_aqk), c2 = beta * s_qk;
         To* o = static_cast<To*>(p.o) + u * dv + col;
         o[0] = from_f32<To>(F.x - c1 * E.x + c2 * vv.x);
         o[1] = from_f32<To>(F.y - c1 * E.y + c2 * vv.y);
@@ -153,12 +165,21 @@ cudaError_t launch_decode(const LoopSlice& s, int dtype_bf16, cudaStream_t strea
     cfg.numAttrs = 1;
     const int use_pdl = pdl ? 1 : 0;
     using bf = __nv_bfloat16;
-    if (dtype_bf16) {
-        if (s.out_bf16) return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<bf, bf>, s, use_pdl);
-        return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<bf, float>, s, use_pdl);
+    // one instance per input type, output type and order of the per-key factors
+    if (s.decay_first) {
+        if (dtype_bf16) {
+            if (s.out_bf16) return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<bf, bf, true>, s, use_pdl);
+            return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<bf, float, true>, s, use_pdl);
+        }
+        if (s.out_bf16) return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<float, bf, true>, s, use_pdl);
+        return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<float, float, true>, s, use_pdl);
     }
-    if (s.out_bf16) return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<float, bf>, s, use_pdl);
-    return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<float, float>, s, use_pdl);
+    if (dtype_bf16) {
+        if (s.out_bf16) return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<bf, bf, false>, s, use_pdl);
+        return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<bf, float, false>, s, use_pdl);
+    }
+    if (s.out_bf16) return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<float, bf, false>, s, use_pdl);
+    return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<float, float, false>, s, use_pdl);
 }
 
 }  // namespace lt2

@@ -28,6 +28,7 @@ struct TcCall {
     int64_t units_per_loop;  // B * H
     int64_t L;               // >= 1
     int out_bf16;
+    int decay_first;         // per-key gating as (I - beta k k^T) Diag(alpha)
     unsigned int* err;
 };
 // Scalar gating: 64-token chunks.  Per-key gating: 32-token chunks in the e-form (chunks whose

@@ -34,6 +34,13 @@
 // where sq = sqrt(P_31) per key and Bv, Be are the Gram tiles below: Kv = sq Bv, Ke = sq Be, so
 // the fp32 state in TMEM is kept scaled by sq (per key, i.e. per TMEM column) around MMA_C.
 //
+// Decay-first order (A_t = (I - beta_t k_t k_t^T) Diag(alpha_t), the other reading of the
+// per-key equation): e_r = k_r^T Diag(alpha_r) S_{r-1}, and token s's delta term decays like its
+// write term, so the same system holds with Gamma_r in place of Gamma_{r-1} on the k_r side
+// (K^, and M_ke, M_kv) and Gamma_s^{-1} in place of Gamma_{s-1}^{-1} on the e side (M_ke, N_qe,
+// Ke): M_ke = M_kv, N_qe = N_qv, Ke = Kv.  In the tiles below that is K^_t = P_t k_t,
+// Kt_t = F_t k_t and Be_t = Bv_t; everything else is unchanged.
+//
 // CTA = one (loop, batch, head) unit, 16 warps:
 //   warp 0       TMA producer (and TMEM allocation)
 //   warps 1-3    conversion of tokens 0-10 / 11-21 / 22-31: per-key decay factors, the six
@@ -290,6 +297,7 @@ __device__ __forceinline__ float4 chunk_products(const float* alpha_c, int w, in
 // running products of local_products.  The warp starting at token 0 writes sq of every key to
 // `sq_out`; the return value says whether every F_t of the warp's tokens lies in
 // [kFactorMin, kFactorMax].
+template <bool decay_first>
 __device__ __forceinline__ bool convert_kqv(uint32_t st, uint32_t gram, const float* alpha_c, float bl, float4 Ph,
                                             float4 Pt, int t_begin, int t_end, int lane, uint8_t* sbase, uint32_t sb,
                                             float* sq_out)
@@ -320,12 +328,12 @@ __device__ __forceinline__ bool convert_kqv(uint32_t st, uint32_t gram, const fl
         const uint2 vb = *vp;
         const float4 Pn = mul4(Ph, lp), Fn = mul4(Pn, isq), Rn = rcp4(Fn);
         ok = ok && in_factor_range(Fn);
-        *kp = pack4_scaled(k, P);                                               // K^ (in place)
+        *kp = pack4_scaled(k, decay_first ? Pn : P);                            // K^ (in place)
         *qp = pack4_scaled(q, Pn);                                              // Q^ (in place)
         *vp = make_uint2(pack_half2(bf16_lo(vb.x), bf16_hi(vb.x)), pack_half2(bf16_lo(vb.y), bf16_hi(vb.y)));
-        *reinterpret_cast<uint2*>(gp + off) = pack4_scaled(k, F);               // Kt
+        *reinterpret_cast<uint2*>(gp + off) = pack4_scaled(k, decay_first ? Fn : F);               // Kt
         *reinterpret_cast<uint2*>(gp + off + 4096) = pack4_scaled(q, Fn);       // Qt
-        *reinterpret_cast<uint2*>(bve + off) = pack4_scaled(k, scale4(R, b));   // Be
+        *reinterpret_cast<uint2*>(bve + off) = pack4_scaled(k, scale4(decay_first ? Rn : R, b));   // Be
         *reinterpret_cast<uint2*>(bve + off + 4096) = pack4_scaled(k, scale4(Rn, b));   // Bv
         P = Pn;
         F = Fn;
@@ -493,6 +501,8 @@ struct ExactIn {
     void* o;
     int out_bf16;
 };
+// decay_first: (I - beta k k^T) Diag(alpha), e = (alpha . k)^T S, S <- Diag(alpha) S + beta k (v - e)
+template <bool decay_first>
 __device__ __noinline__ void exact_chunk(uint32_t tm_s, ExactIn p, int64_t row0, int n, int j)
 {
     #pragma unroll 1
@@ -512,10 +522,16 @@ __device__ __noinline__ void exact_chunk(uint32_t tm_s, ExactIn p, int64_t row0,
             for (int d8 = 0; d8 < 64; d8 += 8) {
                 const uint4 kw = *reinterpret_cast<const uint4*>(kr + 64 * h + d8);
                 const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w};
+                float4 a0 = make_float4(1.f, 1.f, 1.f, 1.f), a1 = a0;
+                if (decay_first) {   // e = (alpha . k)^T S
+                    a0 = *reinterpret_cast<const float4*>(ar + 64 * h + d8);
+                    a1 = *reinterpret_cast<const float4*>(ar + 64 * h + d8 + 4);
+                }
+                const float aa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
                 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    e = fmaf(bf16_lo(kk[u]), sv[d8 + 2 * u], e);
-                    e = fmaf(bf16_hi(kk[u]), sv[d8 + 2 * u + 1], e);
+                    e = fmaf(bf16_lo(kk[u]) * aa[2 * u], sv[d8 + 2 * u], e);
+                    e = fmaf(bf16_hi(kk[u]) * aa[2 * u + 1], sv[d8 + 2 * u + 1], e);
                 }
             }
         }
@@ -538,8 +554,13 @@ __device__ __noinline__ void exact_chunk(uint32_t tm_s, ExactIn p, int64_t row0,
                     const float k0 = bf16_lo(kk[u]), k1 = bf16_hi(kk[u]);
                     float& s0 = sv[d8 + 2 * u];
                     float& s1 = sv[d8 + 2 * u + 1];
-                    s0 = aa[2 * u] * (s0 - b * k0 * e) + b * k0 * vj;
-                    s1 = aa[2 * u + 1] * (s1 - b * k1 * e) + b * k1 * vj;
+                    if (decay_first) {
+                        s0 = aa[2 * u] * s0 + b * k0 * (vj - e);
+                        s1 = aa[2 * u + 1] * s1 + b * k1 * (vj - e);
+                    } else {
+                        s0 = aa[2 * u] * (s0 - b * k0 * e) + b * k0 * vj;
+                        s1 = aa[2 * u + 1] * (s1 - b * k1 * e) + b * k1 * vj;
+                    }
                     o = fmaf(bf16_lo(qq[u]), s0, o);
                     o = fmaf(bf16_hi(qq[u]), s1, o);
                 }
@@ -595,6 +616,7 @@ __device__ __noinline__ int issue_gram_of(int k, uint32_t sb, uint32_t tmem, int
     return 1;
 }
 
+template <bool kDecayFirst>
 __global__ void __launch_bounds__(kThreads, 1)
 gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -725,8 +747,8 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             float4 Ph;
             const float4 Pt = chunk_products(alpha_c, w, lane, Ph);
             Gates* gs = gate(s);
-            const bool in_range = convert_kqv(st, sb + OFF_GRAM + (c & 1) * GRAM_BUF, alpha_c, bl, Ph, Pt,
-                                              t_begin, t_end, lane, sbase, sb, gs->sq);
+            const bool in_range = convert_kqv<kDecayFirst>(st, sb + OFF_GRAM + (c & 1) * GRAM_BUF, alpha_c, bl, Ph, Pt,
+                                                           t_begin, t_end, lane, sbase, sb, gs->sq);
             if (lane == 0) gs->in_range[w] = in_range ? 1 : 0;
             fence_proxy_async_smem();
             __syncwarp();
@@ -924,7 +946,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 // --- out-of-range chunk: the definition, token by token, on the fp32 state (the
                 // first half of the chain's warps; every key of a column takes part in k^T S) ---
                 if (h == 0)
-                    exact_chunk(tmem + TM_S + lane_addr, ExactIn{p.q, p.k, p.v, p.alpha, p.beta, p.o, p.out_bf16},
+                    exact_chunk<kDecayFirst>(tmem + TM_S + lane_addr, ExactIn{p.q, p.k, p.v, p.alpha, p.beta, p.o, p.out_bf16},
                                 static_cast<int64_t>(ug) * L + t0, n, j);
                 tc_fence_before();
                 // keep every hand-off in step: the stage and the [X; Z] stage are released
@@ -989,7 +1011,9 @@ cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream)
         return cudaErrorInvalidValue;
     CUtensorMap ma;
     if (!make_f32_map_3d(&ma, call.alpha, units, call.L, kC)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(gdr_prefill_kda_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    // one instance per order of the per-key factors
+    const auto kernel = call.decay_first ? gdr_prefill_kda_tc_kernel<true> : gdr_prefill_kda_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess) return e;
     for (int64_t tau = 0; tau < call.T; ++tau) {
@@ -1016,7 +1040,7 @@ cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream)
         attr[0].val.programmaticStreamSerializationAllowed = tau > 0 ? 1 : 0;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, gdr_prefill_kda_tc_kernel, mq, mk, mv, call.out_bf16 ? mo : mv, ma, p);
+        e = cudaLaunchKernelEx(&cfg, kernel, mq, mk, mv, call.out_bf16 ? mo : mv, ma, p);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

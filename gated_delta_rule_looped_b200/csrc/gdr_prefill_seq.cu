@@ -8,6 +8,12 @@
 //   S  <- Diag(alpha_t) (S - beta_t k_t e_t) + beta_t k_t v_t^T
 //   o_t = f_t - beta_t ((alpha_t . q_t) . k_t) e_t + beta_t (q_t . k_t) v_t   (= S_t^T q_t)
 //
+// With per-key gating in the decay-first order, A_t = (I - beta_t k_t k_t^T) Diag(alpha_t):
+//
+//   e_t = (alpha_t . k_t)^T S,  f_t = (alpha_t . q_t)^T S
+//   S  <- Diag(alpha_t) S - beta_t k_t e_t + beta_t k_t v_t^T
+//   o_t = f_t - beta_t (q_t . k_t) e_t + beta_t (q_t . k_t) v_t
+//
 // This path serves fp32 inputs (where bf16 tensor cores cannot meet a 1e-4 tolerance) and
 // every shape the tensor-core kernel does not cover.  Columns of S evolve independently
 // (A_t acts from the left), so the grid is (head-unit, 32-column slice of d_v).  Inside a
@@ -109,7 +115,8 @@ __global__ void __launch_bounds__(256) gdr_prefill_seq_kernel(LoopSlice p, int u
             #pragma unroll
             for (int m = 0; m < 16; ++m) {
                 if (m < rpw) {
-                    e += kr[m] * s[m];
+                    const float ke = p.decay_first ? kr[m] * sa[tt * dk + r0 + m] : kr[m];
+                    e += ke * s[m];
                     f += qr[m] * s[m];
                 }
             }
@@ -131,11 +138,12 @@ __global__ void __launch_bounds__(256) gdr_prefill_seq_kernel(LoopSlice p, int u
                 if (m < rpw) {
                     const float a = p.per_key ? sa[tt * dk + r0 + m] : sa[tt];
                     const float bk = bt * kr[m];
-                    s[m] = a * (s[m] - bk * E) + bk * vc;
+                    s[m] = p.decay_first ? a * s[m] - bk * E + bk * vc : a * (s[m] - bk * E) + bk * vc;
                 }
             }
+            const float qke = p.decay_first ? sqk[tt] : saqk[tt];
             if (w == 0 && active)
-                o[(t0 + tt) * dv + j0 + c] = from_f32<To>(F - bt * saqk[tt] * E + bt * sqk[tt] * vc);
+                o[(t0 + tt) * dv + j0 + c] = from_f32<To>(F - bt * qke * E + bt * sqk[tt] * vc);
         }
     }
 

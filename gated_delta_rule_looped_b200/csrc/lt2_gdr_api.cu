@@ -66,6 +66,12 @@ bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.hi > a.l
 
 constexpr int64_t kMaxDim = int64_t(1) << 31;
 
+// Per-key gating in either order of the per-key factors.
+bool is_per_key(const lt2_gdr_dims* d)
+{
+    return d->gate == LT2_GATE_PER_KEY || d->gate == LT2_GATE_PER_KEY_DECAY_FIRST;
+}
+
 bool out_is_bf16(const lt2_gdr_dims* d)
 {
     return d->out_dtype == LT2_OUT_BF16 || (d->out_dtype == LT2_OUT_SAME && d->dtype == LT2_DTYPE_BF16);
@@ -88,7 +94,7 @@ lt2_status validate_dims(const lt2_gdr_dims* d, Sizes* sz)
         d->dk >= kMaxDim || d->dv >= kMaxDim)
         return LT2_ERR_INVALID_ARGUMENT;
     if (d->dtype != LT2_DTYPE_F32 && d->dtype != LT2_DTYPE_BF16) return LT2_ERR_INVALID_ARGUMENT;
-    if (d->gate != LT2_GATE_SCALAR && d->gate != LT2_GATE_PER_KEY) return LT2_ERR_INVALID_ARGUMENT;
+    if (d->gate != LT2_GATE_SCALAR && !is_per_key(d)) return LT2_ERR_INVALID_ARGUMENT;
     if (d->algo < LT2_ALGO_AUTO || d->algo > LT2_ALGO_CUDA_CORE) return LT2_ERR_INVALID_ARGUMENT;
     if (d->out_dtype < LT2_OUT_SAME || d->out_dtype > LT2_OUT_BF16) return LT2_ERR_INVALID_ARGUMENT;
     if (d->dk > 128 || d->dv > 128 || (d->dk % 8) != 0 || (d->dv % 8) != 0)
@@ -102,7 +108,7 @@ lt2_status validate_dims(const lt2_gdr_dims* d, Sizes* sz)
     sz->per_loop = d->B * d->H;
     sz->qk = (int64_t)(tok * d->dk);
     sz->vo = (int64_t)(tok * d->dv);
-    sz->al = (int64_t)(d->gate == LT2_GATE_PER_KEY ? tok * d->dk : tok);
+    sz->al = (int64_t)(is_per_key(d) ? tok * d->dk : tok);
     sz->be = (int64_t)tok;
     sz->st = (int64_t)(units * d->dk * d->dv);
     sz->esz = d->dtype == LT2_DTYPE_BF16 ? 2 : 4;
@@ -121,7 +127,7 @@ bool tensor_ok(const void* p, int64_t count)
 bool use_tensor_core(const lt2_gdr_dims* d)
 {
     const bool ok = lt2::prefill_tc_supports(d->dtype == LT2_DTYPE_BF16, (int)d->dk, (int)d->dv,
-                                             d->gate == LT2_GATE_PER_KEY);
+                                             is_per_key(d));
     if (d->algo == LT2_ALGO_CUDA_CORE) return false;
     return ok;
 }
@@ -132,7 +138,7 @@ lt2::LoopSlice loop_slice(const lt2_gdr_dims* d, const Sizes& sz, int64_t tau,
                           unsigned int* err)
 {
     const int64_t U = sz.per_loop, L = d->L, dk = d->dk, dv = d->dv;
-    const int64_t na = d->gate == LT2_GATE_PER_KEY ? dk : 1;
+    const int64_t na = is_per_key(d) ? dk : 1;
     lt2::LoopSlice s;
     s.q = static_cast<const char*>(q) + tau * U * L * dk * sz.esz;
     s.k = static_cast<const char*>(k) + tau * U * L * dk * sz.esz;
@@ -146,7 +152,8 @@ lt2::LoopSlice loop_slice(const lt2_gdr_dims* d, const Sizes& sz, int64_t tau,
     s.L = L;
     s.dk = (int)dk;
     s.dv = (int)dv;
-    s.per_key = d->gate == LT2_GATE_PER_KEY;
+    s.per_key = is_per_key(d) ? 1 : 0;
+    s.decay_first = d->gate == LT2_GATE_PER_KEY_DECAY_FIRST ? 1 : 0;
     s.out_bf16 = out_is_bf16(d) ? 1 : 0;
     s.err = err;
     return s;
@@ -172,7 +179,7 @@ lt2_status lt2_gdr_prefill(const lt2_gdr_dims* dims, const void* q, const void* 
     if (st != LT2_OK) return st;
     if (dims->algo == LT2_ALGO_TENSOR_CORE &&
         !lt2::prefill_tc_supports(dims->dtype == LT2_DTYPE_BF16, (int)dims->dk, (int)dims->dv,
-                                  dims->gate == LT2_GATE_PER_KEY))
+                                  is_per_key(dims)))
         return LT2_ERR_UNSUPPORTED;
     if (!tensor_ok(q, sz.qk) || !tensor_ok(k, sz.qk) || !tensor_ok(v, sz.vo) ||
         !tensor_ok(alpha, sz.al) || !tensor_ok(beta, sz.be) || !tensor_ok(o, sz.vo))
@@ -220,9 +227,10 @@ lt2_status lt2_gdr_prefill(const lt2_gdr_dims* dims, const void* q, const void* 
         call.units_per_loop = sz.per_loop;
         call.L = dims->L;
         call.out_bf16 = out_is_bf16(dims) ? 1 : 0;
+        call.decay_first = dims->gate == LT2_GATE_PER_KEY_DECAY_FIRST ? 1 : 0;
         call.err = err;
-        cudaError_t e = dims->gate == LT2_GATE_PER_KEY ? lt2::launch_prefill_kda_tc_all(call, s)
-                                                       : lt2::launch_prefill_tc_all(call, s);
+        cudaError_t e = is_per_key(dims) ? lt2::launch_prefill_kda_tc_all(call, s)
+                                         : lt2::launch_prefill_tc_all(call, s);
         if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "prefill (tensor core)");
         return LT2_OK;

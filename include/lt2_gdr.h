@@ -19,7 +19,7 @@
  *   q, k     [T][B][H][L][dk]    dtype of dims->dtype
  *   v        [T][B][H][L][dv]    dtype of dims->dtype
  *   o        [T][B][H][L][dv]    dims->out_dtype (default: same as dims->dtype)
- *   alpha    [T][B][H][L] fp32 (LT2_GATE_SCALAR) or [T][B][H][L][dk] fp32 (LT2_GATE_PER_KEY)
+ *   alpha    [T][B][H][L] fp32 (LT2_GATE_SCALAR) or [T][B][H][L][dk] fp32 (both per-key gates)
  *   beta     [T][B][H][L] fp32
  *   S0, S_out, S  [T][B][H][dk][dv] fp32 (d_v fastest)
  * Decode uses the same layouts with L = 1.
@@ -76,7 +76,16 @@ typedef enum lt2_out_dtype {
     LT2_OUT_F32 = 1,
     LT2_OUT_BF16 = 2
 } lt2_out_dtype;
-typedef enum lt2_gate { LT2_GATE_SCALAR = 0, LT2_GATE_PER_KEY = 1 } lt2_gate;
+/* Gating.  PER_KEY is the equation as printed, A_t = Diag(alpha_t)(I - beta_t k_t k_t^T): the
+ * delta step, then the per-key decay.  PER_KEY_DECAY_FIRST takes the other reading of the same
+ * symbols, A_t = (I - beta_t k_t k_t^T) Diag(alpha_t): the decay, then the delta step on the
+ * decayed state (the order a right-multiplying convention for S gives).  Both take alpha as a
+ * d_k vector per token; for a scalar alpha the two are the same matrix. */
+typedef enum lt2_gate {
+    LT2_GATE_SCALAR = 0,
+    LT2_GATE_PER_KEY = 1,
+    LT2_GATE_PER_KEY_DECAY_FIRST = 2
+} lt2_gate;
 
 /* Prefill algorithm selector (lt2_gdr_dims.algo).  AUTO picks the tensor-core kernel
  * whenever it supports the shape.  The others force one path (for testing). */

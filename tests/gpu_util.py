@@ -17,14 +17,14 @@ def to_np(x):
     return None if x is None else x.detach().to("cpu", torch.float64).numpy()
 
 
-def oracle_prefill(x, per_key, units=None):
+def oracle_prefill(x, per_key, units=None, order="delta_first"):
     """fp64 oracle on (a subset of) the head-units of input dict x.  ``units`` is a list of
     (tau, b, h) triples, or None for all."""
     sel = (lambda t: t) if units is None else (lambda t: torch.stack([t[u] for u in units]))
     S0 = None if x.get("S0") is None else to_np(sel(x["S0"]))
     return oracle.prefill_sequential(to_np(sel(x["q"])), to_np(sel(x["k"])), to_np(sel(x["v"])),
                                      to_np(sel(x["alpha"])), to_np(sel(x["beta"])), S0=S0,
-                                     per_key=per_key)
+                                     per_key=per_key, order=order)
 
 
 def check(name, got, ref, tol):
@@ -37,10 +37,10 @@ def to_device(x, device="cuda"):
     return {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
 
 
-def run_prefill(x, per_key, algo=lt2.LT2_ALGO_AUTO, S0=None, out="f32"):
+def run_prefill(x, per_key, algo=lt2.LT2_ALGO_AUTO, S0=None, out="f32", order="delta_first"):
     o, S = lt2.prefill(x["q"], x["k"], x["v"], x["alpha"], x["beta"],
                        S0=x.get("S0") if S0 is None else S0, per_key=per_key, algo=algo,
-                       out=out)
+                       out=out, order=order)
     torch.cuda.synchronize()
     assert lt2.lt2_gdr_last_device_error() == lt2.LT2_OK
     return o, S
