@@ -160,3 +160,21 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(lt2, "_LIB", None)
     with pytest.raises(ImportError):
         lt2.lib()
+
+
+@pytest.mark.parametrize("gate", [lt2.LT2_GATE_PER_KEY, lt2.LT2_GATE_PER_KEY_DECAY_FIRST])
+def test_per_key_gates_take_per_key_alpha(L, gate):
+    # alpha of either per-key gate holds T*B*H*L*dk floats: an o placed past the scalar extent
+    # (T*B*H*L floats) but inside the per-key one overlaps it
+    a = addrs(4)[3]
+    tok = 2 * 1 * 2 * 64
+    assert call_prefill(D(gate=gate), o=a + tok * 4 + 64) == lt2.LT2_ERR_INVALID_ARGUMENT
+    assert call_prefill(D(gate=gate, T=0)) == lt2.LT2_OK
+
+
+def test_order_names_checked():
+    assert lt2._gate(True, "decay_first") == lt2.LT2_GATE_PER_KEY_DECAY_FIRST
+    assert lt2._gate(True, "delta_first") == lt2.LT2_GATE_PER_KEY
+    assert lt2._gate(False, "decay_first") == lt2.LT2_GATE_SCALAR
+    with pytest.raises(ValueError):
+        lt2._gate(True, "decay_last")
