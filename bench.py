@@ -1,6 +1,7 @@
 """Benchmark of the looped gated-delta-rule mixer on B200: tokens*loops/s and roofline fraction.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gdn_prefill]
+                    [--order delta_first|decay_first]     # per-key workloads: order of the factors
     python bench.py --impl reference ...        # the fp64 CPU oracle, timed on the host
 
 One step = one looped prefill over the workload's whole batch (all T loops, every chunk

@@ -22,11 +22,12 @@ def _units(w, n, seed):
     return sorted(picks)
 
 
-def _check_sampled(x, o32, S, units, per_key, S0=None):
+def _check_sampled(x, o32, S, units, per_key, S0=None, order="delta_first"):
     sel = lambda t: torch.stack([t[u] for u in units])
     o_ref, S_ref = oracle.prefill_sequential(
         to_np(sel(x["q"])), to_np(sel(x["k"])), to_np(sel(x["v"])), to_np(sel(x["alpha"])),
-        to_np(sel(x["beta"])), S0=None if S0 is None else to_np(sel(S0)), per_key=per_key)
+        to_np(sel(x["beta"])), S0=None if S0 is None else to_np(sel(S0)), per_key=per_key,
+        order=order)
     check("o (sampled units)", sel(o32), o_ref, TOL["bf16"])
     check("S_T (sampled units)", sel(S), S_ref, TOL["bf16"])
     return o_ref, S_ref
@@ -45,6 +46,18 @@ def test_full_size_prefill(name, nunits):
     assert torch.equal(S16, S)
     assert torch.isfinite(o32).all() and torch.isfinite(S).all()
     _check_sampled(x, o32, S, _units(w, nunits, seed=1), per_key)
+
+
+def test_full_size_prefill_decay_first():
+    # the per-key workload in the other order of the per-key factors (bench --order decay_first)
+    w = inputs.workload("kda_prefill")
+    x = inputs.make_inputs(w, seed=0, device="cuda")
+    o32, S = lt2.prefill(x["q"], x["k"], x["v"], x["alpha"], x["beta"], per_key=True, out="f32",
+                         order="decay_first")
+    torch.cuda.synchronize()
+    assert lt2.lt2_gdr_last_device_error() == lt2.LT2_OK
+    assert torch.isfinite(o32).all() and torch.isfinite(S).all()
+    _check_sampled(x, o32, S, _units(w, 4, seed=4), True, order="decay_first")
 
 
 def test_full_size_long_overwrite_invariant():
