@@ -134,10 +134,12 @@ def prefill_dense(q, k, v, alpha, beta, S0=None, per_key=False, nthreads=0, orde
 
 def prefill_chunked(q, k, v, alpha, beta, S0=None, per_key=False, chunk=64, form="e",
                     nthreads=0, order="delta_first"):
-    """Chunk-parallel rewriting; ``form`` is "u" (scalar gating only) or "e" (either)."""
+    """Chunk-parallel rewriting; ``form`` is "u" (scalar gating only), "wy" (the u-form with
+    T = (I + A)^{-1} written out, one product with S0 per chunk; scalar gating only) or "e"
+    (either gating)."""
     g = _gate_code(per_key, order)
     q, k, v, alpha, beta, S0, o, S, U, L, dk, dv = _prep(q, k, v, alpha, beta, S0, per_key)
-    f = {"u": 0, "e": 1}[form]
+    f = {"u": 0, "e": 1, "wy": 2}[form]
     rc = _lib().gdr_ref_chunked(U, L, dk, dv, g, int(chunk), f, _ptr(q), _ptr(k),
                                 _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(o), _ptr(S),
                                 int(nthreads))

@@ -327,6 +327,111 @@ static void chunked_unit_uform(int64_t L, int64_t dk, int64_t dv, int64_t C,
 /* Exported entry points.  Each runs every head-unit independently (OpenMP over units).  */
 /* Return 0 on success, -1 on bad arguments, -2 on allocation failure.                   */
 /* ------------------------------------------------------------------------------------ */
+/* ------------------------------------------------------------------------------------ */
+/* The u-form in its WY arrangement (scalar gating).  With T = (I + A)^{-1} written out,  */
+/* the state-independent products U_v = T V, W = T diag(g) K and Q' = diag(g) Q - P W      */
+/* (P_rs = beta_s (g_r/g_s) q_r.k_s for s <= r) leave one product with S0 per chunk:      */
+/*                                                                                        */
+/*   U = U_v - W S0,   O = Q' S0 + P U_v,   S_n = g_{n-1} S0 + sum_s beta_s (g_{n-1}/g_s) k_s u_s^T */
+/* ------------------------------------------------------------------------------------ */
+static int chunked_unit_wyform(int64_t L, int64_t dk, int64_t dv, int64_t C,
+                               const double* q, const double* k, const double* v,
+                               const double* alpha, const double* beta, const double* S0,
+                               double* o, double* S, double* Snew)
+{
+    double* A = (double*)calloc((size_t)(C * C), sizeof(double));
+    double* T = (double*)calloc((size_t)(C * C), sizeof(double));
+    double* P = (double*)calloc((size_t)(C * C), sizeof(double));
+    double* Uv = (double*)malloc(sizeof(double) * C * dv);
+    double* U = (double*)malloc(sizeof(double) * C * dv);
+    double* W = (double*)malloc(sizeof(double) * C * dk);
+    double* Qp = (double*)malloc(sizeof(double) * C * dk);
+    if (!A || !T || !P || !Uv || !U || !W || !Qp) {
+        free(A); free(T); free(P); free(Uv); free(U); free(W); free(Qp);
+        return -1;
+    }
+    if (S0) memcpy(S, S0, sizeof(double) * dk * dv);
+    else    memset(S, 0, sizeof(double) * dk * dv);
+
+    for (int64_t t0 = 0; t0 < L; t0 += C) {
+        const int64_t n = (L - t0 < C) ? (L - t0) : C;
+        const double* kc = k + t0 * dk;
+        const double* qc = q + t0 * dk;
+        const double* vc = v + t0 * dv;
+        const double* bc = beta + t0;
+
+        /* A (s < r) and P (s <= r) */
+        for (int64_t r = 0; r < n; ++r)
+            for (int64_t s = 0; s <= r; ++s) {
+                double kk = 0.0, qk = 0.0;
+                for (int64_t i = 0; i < dk; ++i) {
+                    kk += kc[r * dk + i] * kc[s * dk + i];
+                    qk += qc[r * dk + i] * kc[s * dk + i];
+                }
+                const double f = bc[s] * decay(alpha, 0, t0, r, s, 0, dk);
+                A[r * C + s] = s < r ? f * kk : 0.0;
+                P[r * C + s] = f * qk;
+            }
+        /* T = (I + A)^{-1}, unit lower triangular: T_rs = -sum_{s<=m<r} A_rm T_ms */
+        for (int64_t r = 0; r < n; ++r) {
+            T[r * C + r] = 1.0;
+            for (int64_t s = 0; s < r; ++s) {
+                double acc = 0.0;
+                for (int64_t m = s; m < r; ++m) acc += A[r * C + m] * T[m * C + s];
+                T[r * C + s] = -acc;
+            }
+        }
+        /* U_v = T V,  W = T diag(g) K */
+        for (int64_t r = 0; r < n; ++r) {
+            for (int64_t j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int64_t s = 0; s <= r; ++s) acc += T[r * C + s] * vc[s * dv + j];
+                Uv[r * dv + j] = acc;
+            }
+            for (int64_t i = 0; i < dk; ++i) {
+                double acc = 0.0;
+                for (int64_t s = 0; s <= r; ++s)
+                    acc += T[r * C + s] * decay(alpha, 0, t0, s, -1, 0, dk) * kc[s * dk + i];
+                W[r * dk + i] = acc;
+            }
+        }
+        /* Q' = diag(g) Q - P W */
+        for (int64_t r = 0; r < n; ++r) {
+            const double g = decay(alpha, 0, t0, r, -1, 0, dk);
+            for (int64_t i = 0; i < dk; ++i) {
+                double acc = g * qc[r * dk + i];
+                for (int64_t s = 0; s <= r; ++s) acc -= P[r * C + s] * W[s * dk + i];
+                Qp[r * dk + i] = acc;
+            }
+        }
+        /* the one product with S0: U = U_v - W S0, O = Q' S0 + P U_v */
+        for (int64_t r = 0; r < n; ++r)
+            for (int64_t j = 0; j < dv; ++j) {
+                double ws = 0.0, qs = 0.0;
+                for (int64_t i = 0; i < dk; ++i) {
+                    ws += W[r * dk + i] * S[IDX2(i, j, dv)];
+                    qs += Qp[r * dk + i] * S[IDX2(i, j, dv)];
+                }
+                U[r * dv + j] = Uv[r * dv + j] - ws;
+                double pu = 0.0;
+                for (int64_t s = 0; s <= r; ++s) pu += P[r * C + s] * Uv[s * dv + j];
+                o[(t0 + r) * dv + j] = qs + pu;
+            }
+        /* S_n = g_{n-1} S0 + sum_s beta_s (g_{n-1}/g_s) k_s u_s^T */
+        const double gn = decay(alpha, 0, t0, n - 1, -1, 0, dk);
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t j = 0; j < dv; ++j) {
+                double acc = gn * S[IDX2(i, j, dv)];
+                for (int64_t s = 0; s < n; ++s)
+                    acc += bc[s] * decay(alpha, 0, t0, n - 1, s, 0, dk) * kc[s * dk + i] * U[s * dv + j];
+                Snew[IDX2(i, j, dv)] = acc;
+            }
+        memcpy(S, Snew, sizeof(double) * dk * dv);
+    }
+    free(A); free(T); free(P); free(Uv); free(U); free(W); free(Qp);
+    return 0;
+}
+
 #define UNIT_PTRS(u)                                                                     \
     const double* qu = q + (u) * L * dk;                                                 \
     const double* ku = k + (u) * L * dk;                                                 \
@@ -389,14 +494,15 @@ int gdr_ref_dense(int64_t U, int64_t L, int64_t dk, int64_t dv, int per_key,
     return failed ? -2 : 0;
 }
 
-/* form: 0 = u-form (scalar gating only), 1 = e-form (either gating). */
+/* form: 0 = u-form (scalar gating only), 1 = e-form (either gating), 2 = u-form in its WY
+   arrangement (scalar gating only). */
 int gdr_ref_chunked(int64_t U, int64_t L, int64_t dk, int64_t dv, int per_key, int64_t C,
                     int form, const double* q, const double* k, const double* v,
                     const double* alpha, const double* beta, const double* S0,
                     double* o, double* S_out, int nthreads)
 {
     if (U < 0 || L < 0 || dk <= 0 || dv <= 0 || C <= 0) return -1;
-    if (form == 0 && per_key) return -1;
+    if ((form == 0 || form == 2) && per_key) return -1;
     int failed = 0;
     const int nt = set_threads(nthreads);
     #pragma omp parallel for schedule(dynamic, 1) num_threads(nt) reduction(|:failed)
@@ -411,7 +517,9 @@ int gdr_ref_chunked(int64_t U, int64_t L, int64_t dk, int64_t dv, int per_key, i
             failed |= 1;
             continue;
         }
-        if (form == 0)
+        if (form == 2)
+            failed |= chunked_unit_wyform(L, dk, dv, C, qu, ku, vu, au, bu, s0u, ou, su, Sn) != 0;
+        else if (form == 0)
             chunked_unit_uform(L, dk, dv, C, qu, ku, vu, au, bu, s0u, ou, su, E, M1, Sn);
         else
             chunked_unit_eform(L, dk, dv, per_key, C, qu, ku, vu, au, bu, s0u, ou, su, E, M1, M2, Sn);

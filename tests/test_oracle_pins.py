@@ -33,6 +33,7 @@ def test_sequential_dense_twin_agree(per_key, order):
 @pytest.mark.parametrize("C", [1, 2, 8, 16, 64])
 @pytest.mark.parametrize("L", [1, 5, 63, 64, 65, 200])
 @pytest.mark.parametrize("per_key,form,order", [(False, "u", "delta_first"), (False, "e", "delta_first"),
+                                                (False, "wy", "delta_first"),
                                                 (True, "e", "delta_first"), (True, "e", "decay_first")])
 def test_chunked_equals_sequential(C, L, per_key, form, order):
     # P4: the chunk-parallel rewriting used by the GPU equals the token-by-token equation.
