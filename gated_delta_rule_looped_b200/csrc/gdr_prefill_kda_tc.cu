@@ -21,8 +21,9 @@
 // tiles Kt, Qt and Be, Bv that carry e^{G - R} and e^{R - G} around a per-key reference
 // R = G_31 / 2; Be and Bv also serve the state update (Kv = sq Bv, Ke = sq Be, sq = e^{G_31/2}).
 // The tiles stay in range while a key decays by at most e^-19 over the chunk.  A chunk beyond
-// that (or with any alpha outside (0, 1]) is instead run token by token, exactly, on the fp32
-// state in TMEM.
+// that (or with any alpha <= 0, a reset) is instead run token by token, exactly, on the fp32
+// state in TMEM.  A growing alpha > 1 stays on the tensor cores while the state and the tiles
+// remain inside fp16.
 //
 // With the solve X = [T; N_qe T], T = (I + M_ke)^{-1}, and Z = X M_kv - [0; N_qv]:
 //   [E; -(O - Q^ S)] = X (K^ S) + Z V,

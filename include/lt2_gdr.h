@@ -40,8 +40,10 @@
  *   The tensor-core chunked prefills serve bf16 inputs with dk = dv = 128, for scalar gating
  *   (64-token chunks) and per-key gating (32-token chunks); every other supported shape runs
  *   on the CUDA-core path.  With per-key gating, a chunk in which some key decays by more than
- *   ~e^-19, or with any alpha outside (0, 1], is evaluated token by token inside the same
- *   kernel (exact, slower); alpha is expected in (0, 1] and |q|, |k| entries of order 1.
+ *   ~e^-19, or with any alpha <= 0 (a reset), is evaluated token by token inside the same
+ *   kernel (exact, slower).  The tensor-core paths take their operands in fp16: alpha is
+ *   expected in (0, 1] (a growing alpha > 1 works while the state stays below ~3e4 in
+ *   magnitude), with |q|, |k| entries of order 1.
  *   fp32 inputs: dk, dv multiples of 8 up to 128 (CUDA-core fp32 arithmetic throughout).
  *   bf16 inputs: dk, dv multiples of 8 up to 128.
  *   Any L >= 0 (a ragged final chunk is fine; L = 0 copies S0 to S_out).

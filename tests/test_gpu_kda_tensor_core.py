@@ -105,3 +105,21 @@ def test_kda_tc_in_place_resume_and_bf16_output():
                          out="bf16")
     torch.cuda.synchronize()
     assert torch.equal(o16, o32.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("order", ["delta_first", "decay_first"])
+def test_kda_tc_alpha_above_one(order):
+    # mild growth (alpha > 1 on a few tokens, the state and every tile staying well inside fp16)
+    # runs on the tensor cores, in either order
+    w = inputs.workload("kda_prefill", T=1, B=1, H=2, L=200, s0="normal")
+    x = inputs.make_inputs(w, seed=47)
+    a = x["alpha"].clone()
+    a[..., 64:72, :] = 1.5
+    a[..., 130:140, :7] = 1.02
+    x["alpha"] = a
+    x = to_device(x)
+    o, S = run_prefill(x, per_key=True, algo=TC, order=order)
+    o_ref, S_ref = oracle_prefill(x, True, order=order)
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    check("o", o, o_ref, TOL["bf16"])
+    check("S_T", S, S_ref, TOL["bf16"])
