@@ -114,10 +114,7 @@ def make_inputs(w, seed=0, device="cpu", q_equals_k_on_subset=False):
                 pos = torch.randperm(L, generator=gen, device=device)[:n_sel]
                 subset[t, b, pos] = True
             m = subset[t][:, None, :].expand(B, H, L)
-            if w.gate == "per_key":
-                alpha[t][m] = 1.0
-            else:
-                alpha[t][m] = 1.0
+            alpha[t][m] = 1.0          # per-key: the whole d_k vector of the position
             beta[t][m] = 1.0
             if q_equals_k_on_subset:
                 q[t][m] = k[t][m]
