@@ -180,6 +180,36 @@ def _dims_from(q, v, alpha, per_key, algo, out=None, order="delta_first"):
     return make_dims(T, B, H, L, dk, dv, dt, _gate(per_key, order), algo, _OUT[out])
 
 
+def _check(name, t, shape, dtype, device):
+    """A tensor handed to the library by pointer: on ``device``, contiguous, of the given shape
+    and dtype (the C ABI reads raw row-major memory and cannot tell)."""
+    if t is None:
+        return
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _check_call(q, k, v, alpha, beta, states, o, per_key, out):
+    """Validate the tensors of a prefill ([T,B,H,L,d]) or decode ([T,B,H,d]) call."""
+    import torch
+    lead, dk, dv = tuple(q.shape[:-1]), q.shape[-1], v.shape[-1]
+    dev = q.device
+    _check("q", q, q.shape, q.dtype, dev)
+    _check("k", k, q.shape, q.dtype, dev)
+    _check("v", v, lead + (dv,), q.dtype, dev)
+    _check("alpha", alpha, lead + ((dk,) if per_key else ()), torch.float32, dev)
+    _check("beta", beta, lead, torch.float32, dev)
+    for name, S in states:
+        _check(name, S, tuple(q.shape[:3]) + (dk, dv), torch.float32, dev)
+    _check("o", o, lead + (dv,), _out_torch_dtype(q.dtype, out), dev)
+
+
 def prefill(q, k, v, alpha, beta, S0=None, per_key=None, algo=LT2_ALGO_AUTO, o=None,
             S_out=None, out=None, stream=None, order="delta_first"):
     """Run the looped prefill on CUDA tensors; returns (o, S_out).  ``out`` selects the
@@ -187,6 +217,7 @@ def prefill(q, k, v, alpha, beta, S0=None, per_key=None, algo=LT2_ALGO_AUTO, o=N
     the per-key factors ("delta_first" as printed, or "decay_first")."""
     import torch
     dims = _dims_from(q, v, alpha, per_key, algo, out, order)
+    _check_call(q, k, v, alpha, beta, [("S0", S0), ("S_out", S_out)], o, dims.gate != LT2_GATE_SCALAR, out)
     if o is None:
         o = torch.empty(v.shape, dtype=_out_torch_dtype(q.dtype, out), device=v.device)
     if S_out is None:
@@ -208,6 +239,7 @@ def decode(q, k, v, alpha, beta, S, per_key=None, o=None, out=None, stream=None,
     dv = v.shape[-1]
     dt = {torch.float32: LT2_DTYPE_F32, torch.bfloat16: LT2_DTYPE_BF16}[q.dtype]
     dims = make_dims(T, B, H, 1, dk, dv, dt, _gate(per_key, order), out_dtype=_OUT[out])
+    _check_call(q, k, v, alpha, beta, [("S", S)], o, per_key, out)
     if o is None:
         o = torch.empty(v.shape, dtype=_out_torch_dtype(q.dtype, out), device=v.device)
     st = lt2_gdr_decode(dims, q, k, v, alpha, beta, S, o, stream)

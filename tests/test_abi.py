@@ -178,3 +178,15 @@ def test_order_names_checked():
     assert lt2._gate(False, "decay_first") == lt2.LT2_GATE_SCALAR
     with pytest.raises(ValueError):
         lt2._gate(True, "decay_last")
+
+
+def test_binding_rejects_tensors_it_cannot_pass_by_pointer():
+    # the convenience layer checks device, contiguity, shape and dtype before calling the ABI
+    import torch
+    q = torch.zeros((1, 1, 1, 4, 128), dtype=torch.bfloat16)
+    a = torch.ones((1, 1, 1, 4), dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA"):
+        lt2.prefill(q, q, q, a, a)
+    with pytest.raises(ValueError, match="CUDA"):
+        lt2.decode(q[..., 0, :], q[..., 0, :], q[..., 0, :], a[..., 0], a[..., 0],
+                   torch.zeros((1, 1, 1, 128, 128)))
