@@ -289,7 +289,8 @@ def run_decode(world, steps, warmup):
 
 def oracle_sample(w, target_s=15.0, order="delta_first"):
     """Time the fp64 oracle on a bounded sample of workload w's head-units on this host.
-    Returns (tokens*loops per second, threads used, description)."""
+    Returns (tokens*loops per second, threads used, description, single-thread figure): the
+    last is one head-unit on one thread, extrapolated to tokens*loops/s."""
     import oracle
     cores = len(os.sched_getaffinity(0))
     threads = oracle.threads(cores)
@@ -315,7 +316,9 @@ def oracle_sample(w, target_s=15.0, order="delta_first"):
     tok_loops = n * L / w.H          # a token*loop needs all H heads
     desc = (f"{n} of {w.units} (loop, batch, head) units of {w.name}, L={L}, fp64 sequential "
             f"oracle, OpenMP over units")
-    return tok_loops / dt, threads, desc
+    single = {"value": L / w.H / t1, "unit": "tokens*loops/s", "threads": 1,
+              "note": "one head-unit on one thread, extrapolated to the workload"}
+    return tok_loops / dt, threads, desc, single
 
 
 def reference_arm(args, world, rank):
@@ -325,10 +328,11 @@ def reference_arm(args, world, rank):
         return
     vals = []
     desc = threads = None
+    single = None
     for _ in range(args.warmup):
         oracle_sample(w, target_s=2.0, order=args.order)
     for _ in range(args.steps):
-        v, threads, desc = oracle_sample(w, target_s=max(2.0, 20.0 / max(args.steps, 1)), order=args.order)
+        v, threads, desc, single = oracle_sample(w, target_s=max(2.0, 20.0 / max(args.steps, 1)), order=args.order)
         vals.append(v)
     value = statistics.median(vals)
     line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
@@ -336,7 +340,7 @@ def reference_arm(args, world, rank):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config_of(w, args.gpus, args.order),
             "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
-                             "sample": desc},
+                             "sample": desc, "single_thread": single},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -441,9 +445,9 @@ def main():
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, threads, desc = oracle_sample(w, order=args.order)
+        v, threads, desc, single = oracle_sample(w, order=args.order)
         line["cpu_baseline"] = {"value": v, "unit": unit, "cores": threads, "kind": "oracle",
-                                "sample": desc}
+                                "sample": desc, "single_thread": single}
 
     if rank == 0:
         print(json.dumps(line), flush=True)
