@@ -7,7 +7,7 @@ import oracle
 
 TOL = {"f32": 1e-4, "bf16": 2e-2}   # max|gpu - ref| / rms(ref), per output tensor
 
-# Parity is judged on an fp32 copy of o: the final rounding of o to bf16 alone can reach
+# Parity is checked on an fp32 copy of o: the final rounding of o to bf16 alone can reach
 # 2^-8 |o|, i.e. ~2e-2 of rms(o) at the largest |o| of a big tensor, whatever the kernel
 # does.  The bf16 output is checked separately to be exactly the fp32 output rounded to
 # nearest-even.
