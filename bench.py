@@ -1,20 +1,23 @@
 """Benchmark of the looped gated-delta-rule mixer on B200: tokens*loops/s and roofline fraction.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gdn_prefill]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long_gdn]
+                    [--extras gdn_prefill,kda_prefill,decode | none]
                     [--order delta_first|decay_first]     # per-key workloads: order of the factors
     python bench.py --impl reference ...        # the fp64 CPU oracle, timed on the host
 
-One step = one looped prefill over the workload's whole batch (all T loops, every chunk
-step: gates, Gram products, solve, state GEMMs, outputs), through the C ABI, with inputs
-already resident in HBM.  Rank 0 prints one JSON line.  With N > 1 (torchrun, one process
-per GPU) every rank runs its own replica of the workload: the (loop, batch, head) units are
-independent recurrences, so the path shards with no collective (weak scaling); the only
-communication is the timing barrier and the max over ranks.
+The headline (`metric`, `value`, `ms_per_step`, `config`, `roofline`, `e2e`, `cpu_baseline`) is
+the long-context scalar-gated prefill `long_gdn` (T=8, B=1, H=32, L=65536, d=128), the largest
+workload that fits one GPU.  One step = one looped prefill over the workload's whole batch (all
+T loops, every chunk step: gates, Gram products, solve, state GEMMs, outputs) through the C ABI,
+with inputs already resident in HBM.  The other timed workloads ride along as keys of the same
+JSON line, each with its own `ms_per_step`, `value`, `roofline`, `cpu_baseline`, `clocks` and
+`gpu_launches`: `gdn_prefill` (T4 B4 H16 L8192, scalar gating), `kda_prefill` (T4 B2 H16
+L16384, per-key gating) and `decode` (one decode token for T4 B256 H16 from a 4096-token state).
 
-Extra keys: "decode" (one decode step of the decode workload, timed the same way),
-"roofline" (dominant kernel against MEASURED_PEAKS.json), "e2e" (same metric with host
-buffers and the copies inside the timed region), "cpu_baseline" (the oracle on a bounded
-sample), "clocks" (nvidia-smi sampled during the timed region), "gpu_launches".
+With N > 1 (torchrun, one process per GPU) every rank runs its own replica of each workload: the
+(loop, batch, head) units are independent recurrences, so the path shards with no collective
+(weak scaling); the only communication is the timing barrier and the max over ranks.  Rank 0
+prints one JSON line.
 """
 import argparse
 import hashlib
@@ -27,7 +30,6 @@ import sys
 import threading
 import time
 
-import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -37,9 +39,13 @@ import gated_delta_rule_looped_b200 as lt2  # noqa: E402
 from gated_delta_rule_looped_b200 import dist as gdist  # noqa: E402
 from gated_delta_rule_looped_b200 import inputs  # noqa: E402
 
-# Algorithmic work per token-head (chunk 64, d = 128; scalar gating): three d x d state
-# products 6d^2, the four chunk-local products 8*64*d, the 64x64 solve 64^2/3, counted as
-# dense multiply-adds (2 flops each); bytes: q, k, v in + o out (bf16) + alpha + beta (fp32).
+HEADLINE = "long_gdn"
+EXTRAS = ("gdn_prefill", "kda_prefill", "decode")
+
+# Algorithmic work per token-head (d = 128), counted as dense multiply-adds (2 flops each).
+# Scalar gating, 64-token chunks: three d x d state products 6d^2, the four chunk-local
+# products 8*64*d, the 64x64 solve 64^2/3.  Per-key gating (e-form): 8d^2 + 16*64*d + 64^2/3.
+# Bytes: q, k, v in + o out (bf16) + alpha (fp32 scalar or d_k vector) + beta (fp32).
 FLOP_PER_TOKEN_HEAD = {"scalar": 6 * 128 ** 2 + 8 * 64 * 128 + 64 ** 2 // 3,
                        "per_key": 8 * 128 ** 2 + 16 * 64 * 128 + 64 ** 2 // 3}
 BYTES_PER_TOKEN_HEAD = {"scalar": 3 * 256 + 256 + 4 + 4, "per_key": 3 * 256 + 256 + 512 + 4}
@@ -47,10 +53,15 @@ BYTES_PER_TOKEN_HEAD = {"scalar": 3 * 256 + 256 + 4 + 4, "per_key": 3 * 256 + 25
 BYTES_PER_DECODE_UNIT = 2 * 128 * 128 * 4 + 4 * 256 + 8
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Public B200 figures, reported beside the measured ones: ~8 TB/s HBM3e, 2.25 PFLOP/s dense
+# bf16/fp16.
+NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = [os.path.join(ROOT, "gated_delta_rule_looped_b200", "csrc", f)
-                  for f in ("gdr_prefill_tc.cu", "gdr_prefill_kda_tc.cu", "gdr_decode.cu", "sm100_primitives.cuh")]
+
+KERNELS = {"scalar": ("gdr_prefill_tc_kernel", "gdr_prefill_tc.cu"),
+           "per_key": ("gdr_prefill_kda_tc_kernel", "gdr_prefill_kda_tc.cu"),
+           "decode": ("gdr_decode_kernel", "gdr_decode.cu")}
 
 
 def kernel_sources(name, csrc=None):
@@ -107,16 +118,19 @@ def traffic_for(kernel, source, bytes_launch=None, path=None):
     return t * bytes_launch / a, f"scaled from the capture on {e.get('workload')} by algorithmic bytes per launch"
 
 
-# ---- clocks during the timed region ------------------------------------------------------
+# ---- clocks during the timed regions ---------------------------------------------------------
 
 class ClockSampler:
+    """nvidia-smi sampled every 100 ms for the whole run; each timed region marks its wall-clock
+    window, and `summary` reduces the samples that fall inside a set of windows."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, device_index):
         self.samples = []
-        self.window = None
+        self.windows = {}
         self.proc = None
         try:
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
@@ -138,33 +152,33 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
 
-    def mark(self, t0, t1):
-        self.window = (t0, t1)
+    def mark(self, name, t0, t1):
+        self.windows.setdefault(name, []).append((t0, t1))
 
     def stop(self):
         if self.proc is None:
-            return None
+            return
         time.sleep(0.25)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
+
+    def summary(self, names=None):
+        """Median SM clock, max clock and the throttle reasons seen inside the windows of the
+        named regions (all regions when `names` is None)."""
+        wins = [w for n, ws in self.windows.items() if names is None or n in names for w in ws]
         rows = [s for (ts, s) in self.samples
-                if self.window and self.window[0] - 0.05 <= ts <= self.window[1] + 0.15]
-        if not rows:
-            rows = [s for (_, s) in self.samples]
-        if not rows:
-            return None
+                if any(a - 0.05 <= ts <= b + 0.15 for a, b in wins)]
         sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
             try:
                 sm.append(float(r[1]))
                 mx.append(float(r[2]))
             except (ValueError, IndexError):
                 continue
-            for n, v in zip(names, r[5:9]):
+            for n, v in zip(self.REASONS, r[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         if not sm:
@@ -192,7 +206,7 @@ def max_over_ranks(x, world):
 
 # ---- timed regions -----------------------------------------------------------------------
 
-def timed(fn, steps, warmup, world, sampler=None):
+def timed(fn, steps, warmup, world, sampler=None, name="step"):
     """W untimed steps, then K steps between a barrier + synchronize on both sides; device
     time from CUDA events on the launching stream, max over ranks."""
     for _ in range(warmup):
@@ -212,9 +226,15 @@ def timed(fn, steps, warmup, world, sampler=None):
     w1 = time.time()
     barrier(world)
     if sampler is not None:
-        sampler.mark(w0, w1)
+        sampler.mark(name, w0, w1)
     ms = e0.elapsed_time(e1) / max(steps, 1)
     return max_over_ranks(ms, world)
+
+
+def check_device_status(where):
+    st = lt2.lt2_gdr_last_device_error()
+    if st != lt2.LT2_OK:
+        raise RuntimeError(f"{lt2.lt2_status_string(st)} reported by the device during {where}")
 
 
 def gate_of(w, order):
@@ -239,20 +259,71 @@ def prefill_case(w, device, order="delta_first"):
     return x, o, S, dims, step
 
 
+def tensor_roofline(gate, units_per_launch, L, launch_s, peaks, peak_src):
+    """The prefill kernel of one loop launch against the tensor and HBM peaks (measured, and the
+    public B200 figures beside them)."""
+    kernel, source = KERNELS[gate]
+    flops_launch = units_per_launch * L * FLOP_PER_TOKEN_HEAD[gate]
+    bytes_launch = units_per_launch * L * BYTES_PER_TOKEN_HEAD[gate]
+    achieved_tf = flops_launch / launch_s / 1e12
+    achieved_gbs = bytes_launch / launch_s / 1e9
+    traffic, traffic_note = traffic_for(kernel, source, bytes_launch)
+    r = {"bound": "tensor", "kernel": kernel, "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
+         "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"], "traffic": traffic,
+         "peak_source": f"{peak_src} bf16 dense burst (fp16 operands run at the same rate)",
+         "nominal": {"peak": NOMINAL_PEAKS["bf16_tflops"],
+                     "frac": achieved_tf / NOMINAL_PEAKS["bf16_tflops"]},
+         "algorithmic_per_launch": {"flop": flops_launch, "bytes": bytes_launch},
+         "hbm": {"achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                 "frac": achieved_gbs / peaks["hbm_gbs"],
+                 "nominal": {"peak": NOMINAL_PEAKS["hbm_gbs"],
+                             "frac": achieved_gbs / NOMINAL_PEAKS["hbm_gbs"]}},
+         "launch_time": "step time / T launches (the T loop launches of a step run back to back "
+                        "and overlap through programmatic dependent launch)"}
+    if traffic_note:
+        r["traffic_note"] = traffic_note
+    return r
+
+
+def run_prefill(w, args, world, sampler, peaks, peak_src, keep=False):
+    """Time workload w's looped prefill.  Returns (entry dict, the case when `keep`)."""
+    case = prefill_case(w, "cuda", args.order)
+    step = case[-1]
+    ms = timed(step, args.steps, args.warmup, world, sampler, w.name)
+    check_device_status(w.name)
+    launch_s = ms * 1e-3 / w.T
+    entry = {"metric": metric_of(w)[0], "value": gdist.whole_job_rate(w.T * w.B * w.L, world, ms),
+             "unit": "tokens*loops/s", "ms_per_step": ms, "steps": args.steps,
+             "config": config_of(w, world, args.order),
+             "roofline": tensor_roofline(w.gate, w.B * w.H, w.L, launch_s, peaks, peak_src),
+             "gpu_launches": args.steps * w.T}
+    if sampler is not None:
+        entry["clocks"] = sampler.summary([w.name])
+    if keep:
+        return entry, case
+    del case
+    torch.cuda.empty_cache()
+    return entry, None
+
+
 def run_e2e(w, x, dims, steps, warmup, world):
     """Same metric through the C ABI with host buffers: every step copies the inputs from
     pinned host memory, runs the prefill and reads o and the final state back."""
-    host = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "alpha", "beta")}
-    dev = {n: torch.empty_like(x[n]) for n in host}
+    names = ("q", "k", "v", "alpha", "beta")
+    host = {}
+    for n in names:
+        host[n] = torch.empty(x[n].shape, dtype=x[n].dtype, pin_memory=True)
+        host[n].copy_(x[n])
+    dev = {n: torch.empty_like(x[n]) for n in names}
     o_d = torch.empty(x["v"].shape, dtype=torch.bfloat16, device="cuda")
     S_d = torch.empty((w.T, w.B, w.H, w.d, w.d), dtype=torch.float32, device="cuda")
-    o_h = torch.empty(o_d.shape, dtype=o_d.dtype).pin_memory()
-    S_h = torch.empty(S_d.shape, dtype=S_d.dtype).pin_memory()
+    o_h = torch.empty(o_d.shape, dtype=o_d.dtype, pin_memory=True)
+    S_h = torch.empty(S_d.shape, dtype=S_d.dtype, pin_memory=True)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = o_h.numel() * o_h.element_size() + S_h.numel() * S_h.element_size()
 
     def step():
-        for n in host:
+        for n in names:
             dev[n].copy_(host[n], non_blocking=True)
         st = lt2.lt2_gdr_prefill(dims, dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"],
                                  None, o_d, S_d, None, 0)
@@ -264,75 +335,142 @@ def run_e2e(w, x, dims, steps, warmup, world):
     return ms, h2d, d2h
 
 
-def run_decode(world, steps, warmup):
+def run_decode(args, world, sampler, peaks, peak_src):
+    """One decode step of the decode workload (T4 B256 H16) from the state a 4096-token prefill
+    leaves; the state is updated in place, step after step."""
     w = inputs.workload("decode")
     dev = "cuda"
     hist = inputs.decode_history(w, seed=0, device=dev)
     S = torch.empty((w.T, w.B, w.H, w.d, w.d), dtype=torch.float32, device=dev)
     lt2.prefill(hist["q"], hist["k"], hist["v"], hist["alpha"], hist["beta"], per_key=False, S_out=S)
     del hist
+    torch.cuda.empty_cache()
     x = inputs.make_decode_step(w, seed=0, step=0, device=dev)
     o = torch.empty(x["v"].shape, dtype=torch.bfloat16, device=dev)
     dims = lt2.make_dims(w.T, w.B, w.H, 1, w.d, w.d, lt2.LT2_DTYPE_BF16, lt2.LT2_GATE_SCALAR)
+    S_host = S[0, 0, :8].to("cpu")      # a few units' state for the CPU baseline
 
     def step():
         st = lt2.lt2_gdr_decode(dims, x["q"], x["k"], x["v"], x["alpha"], x["beta"], S, o)
         if st != lt2.LT2_OK:
             raise lt2.Lt2Error(st, "lt2_gdr_decode")
-    ms = timed(step, steps, warmup, world)
+    nsteps = max(10, args.steps)
+    ms = timed(step, nsteps, args.warmup, world, sampler, "decode")
+    check_device_status("decode")
     units_per_launch = w.B * w.H
     launch_s = ms * 1e-3 / w.T
-    return w, ms, units_per_launch, launch_s
+    dbytes = units_per_launch * BYTES_PER_DECODE_UNIT
+    gbs = dbytes / launch_s / 1e9
+    kernel, source = KERNELS["decode"]
+    entry = {"metric": "looped GDR decode tokens*loops/s (decode)",
+             "value": w.T * w.B * world / (ms * 1e-3), "unit": "tokens*loops/s",
+             "ms_per_step": ms, "steps": nsteps,
+             "config": {"workload": "decode", "T": w.T, "B": w.B, "H": w.H, "d_k": w.d, "d_v": w.d,
+                        "gate": "scalar", "io_dtype": "bf16", "state_dtype": "f32",
+                        "state": "fp32, from a 4096-token prefill, updated in place each step",
+                        "l2": "1 GiB state read and written per step (larger than L2)"},
+             "roofline": {"bound": "hbm", "kernel": kernel, "achieved": gbs, "peak": peaks["hbm_gbs"],
+                          "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                          "traffic": traffic_for(kernel, source)[0],
+                          "peak_source": f"{peak_src} HBM copy",
+                          "nominal": {"peak": NOMINAL_PEAKS["hbm_gbs"],
+                                      "frac": gbs / NOMINAL_PEAKS["hbm_gbs"]},
+                          "algorithmic_per_launch": {"bytes": dbytes}},
+             "gpu_launches": nsteps * w.T}
+    if sampler is not None:
+        entry["clocks"] = sampler.summary(["decode"])
+    xs = {n: x[n][0, 0, :8].to("cpu") for n in ("q", "k", "v", "alpha", "beta")}
+    del S, x, o
+    torch.cuda.empty_cache()
+    return entry, (w, xs, S_host)
 
 
 # ---- CPU oracle (reported baseline / reference arm) -----------------------------------------
 
-def oracle_sample(w, target_s=15.0, order="delta_first"):
-    """Time the fp64 oracle on a bounded sample of workload w's head-units on this host.
-    Returns (tokens*loops per second, threads used, description, single-thread figure): the
-    last is one head-unit on one thread, extrapolated to tokens*loops/s."""
+def oracle_sample(w, target_s=8.0, order="delta_first"):
+    """Time the fp64 oracle on a bounded sample of workload w on this host: a calibration on
+    one head-unit (one thread, a prefix of at most 1024 tokens) sizes a sample of whole or
+    leading-prefix head-units, one per thread, to about `target_s` of wall time.  Returns
+    (tokens*loops per second, threads used, description, single-thread figure): the last is
+    the calibration, one head-unit on one thread, extrapolated to tokens*loops/s."""
     import oracle
     cores = len(os.sched_getaffinity(0))
     threads = oracle.threads(cores)
-    L = w.L
+    per_key = w.gate == "per_key"
 
-    def draw(nunits, seed):
+    def draw(nunits, L, seed):
         ws = inputs.workload(w.name, T=1, B=1, H=nunits, L=L)
         x = inputs.make_inputs(ws, seed=seed, device="cpu")
         return [x[n].to(torch.float64).numpy() for n in ("q", "k", "v", "alpha", "beta")]
-    # calibrate on one unit, then size the sample to ~target_s of wall time
-    a = draw(1, 1)
+    L_cal = min(w.L, 1024)
+    a = draw(1, L_cal, 1)
     t0 = time.perf_counter()
-    oracle.prefill_sequential(*a, per_key=(w.gate == "per_key"), nthreads=1, order=order)
-    t1 = time.perf_counter() - t0
-    per_unit_parallel = t1 / threads
-    n = max(threads, int(target_s / max(per_unit_parallel, 1e-6)) // threads * threads)
-    n = max(1, min(n, w.units, 64))
+    oracle.prefill_sequential(*a, per_key=per_key, nthreads=1, order=order)
+    per_token = (time.perf_counter() - t0) / L_cal
+    L = int(min(w.L, max(64, target_s / max(per_token, 1e-9))))
+    n = min(threads, w.units)
+    if L == w.L:
+        # whole sequences fit: as many rounds of `threads` units as the target allows
+        rounds = max(1, int(target_s / max(per_token * w.L, 1e-9)))
+        n = min(w.units, 64, threads * rounds)
     threads = min(threads, n)
-    a = draw(n, 2)
+    a = draw(n, L, 2)
     t0 = time.perf_counter()
-    oracle.prefill_sequential(*a, per_key=(w.gate == "per_key"), nthreads=threads, order=order)
+    oracle.prefill_sequential(*a, per_key=per_key, nthreads=threads, order=order)
     dt = time.perf_counter() - t0
     tok_loops = n * L / w.H          # a token*loop needs all H heads
-    desc = (f"{n} of {w.units} (loop, batch, head) units of {w.name}, L={L}, fp64 sequential "
-            f"oracle, OpenMP over units")
-    single = {"value": L / w.H / t1, "unit": "tokens*loops/s", "threads": 1,
-              "note": "one head-unit on one thread, extrapolated to the workload"}
+    span = f"all {w.L} tokens" if L == w.L else f"the first {L} of {w.L} tokens"
+    desc = (f"{n} of {w.units} (loop, batch, head) units of {w.name}, {span} each, fp64 "
+            f"sequential oracle, OpenMP over units")
+    single = {"value": 1.0 / (per_token * w.H), "unit": "tokens*loops/s", "threads": 1,
+              "note": f"one head-unit of {L_cal} tokens on one thread, extrapolated to the workload"}
     return tok_loops / dt, threads, desc, single
 
 
+def oracle_decode_sample(w, xs, S_host, target_s=4.0):
+    """Time the fp64 oracle's decode step on this host: the first units of the decode workload
+    (their q, k, v, alpha, beta and prefilled state), repeated to about `target_s`."""
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    threads = oracle.threads(cores)
+    f64 = {n: t.to(torch.float64).numpy() for n, t in xs.items()}
+    S = S_host.to(torch.float64).numpy()
+    n = S.shape[0]
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.decode_step(f64["q"], f64["k"], f64["v"], f64["alpha"], f64["beta"], S,
+                           nthreads=min(threads, n))
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= target_s or reps >= 100000:
+            break
+    units_per_s = reps * n / dt
+    desc = (f"decode step of {n} of {w.units} head-units (their prefilled fp32 state), repeated "
+            f"{reps} times, fp64 oracle")
+    return units_per_s / w.H, min(threads, n), desc
+
+
+def cpu_entry(w, order, target_s):
+    v, threads, desc, single = oracle_sample(w, target_s=target_s, order=order)
+    return {"value": v, "unit": "tokens*loops/s", "cores": threads, "kind": "oracle",
+            "sample": desc, "single_thread": single}
+
+
 def reference_arm(args, world, rank):
+    """The oracle, as it stands, timed on the host cores on the headline workload: each step a
+    bounded sample sized so that the whole --steps/--warmup run ends within a few minutes."""
     w = inputs.workload(args.workload)
     metric, unit = metric_of(w)
     if rank != 0:
         return
+    per_step = min(8.0, max(1.0, 150.0 / max(args.steps + args.warmup, 1)))
     vals = []
-    desc = threads = None
-    single = None
+    desc = threads = single = None
     for _ in range(args.warmup):
-        oracle_sample(w, target_s=2.0, order=args.order)
+        oracle_sample(w, target_s=min(per_step, 2.0), order=args.order)
     for _ in range(args.steps):
-        v, threads, desc, single = oracle_sample(w, target_s=max(2.0, 20.0 / max(args.steps, 1)), order=args.order)
+        v, threads, desc, single = oracle_sample(w, target_s=per_step, order=args.order)
         vals.append(v)
     value = statistics.median(vals)
     line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
@@ -351,28 +489,38 @@ def metric_of(w):
 
 def config_of(w, n_gpus, order="delta_first"):
     gate = w.gate if w.gate != "per_key" or order == "delta_first" else "per_key, decay first"
-    return {"workload": w.name, "T": w.T, "B": w.B, "H": w.H, "L": w.L, "d_k": w.d, "d_v": w.d,
-            "gate": gate, "chunk": 32 if w.gate == "per_key" else 64, "io_dtype": w.dtype,
-            "state_dtype": "f32",
-            "parallelism": f"replicas x{n_gpus} (independent head-units, no collective)",
-            "l2": "inputs larger than L2 (no flush needed)"}
+    c = {"workload": w.name, "T": w.T, "B": w.B, "H": w.H, "L": w.L, "d_k": w.d, "d_v": w.d,
+         "gate": gate, "chunk": 32 if w.gate == "per_key" else 64, "io_dtype": w.dtype,
+         "state_dtype": "f32",
+         "parallelism": f"replicas x{n_gpus} (independent head-units, no collective)",
+         "l2": "inputs larger than L2 (no flush needed)"}
+    if w.overwrite_frac:
+        c["overwrites"] = f"alpha = beta = 1 on {w.overwrite_frac:.0%} of the positions"
+    return c
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="gdn_prefill",
-                    choices=["gdn_prefill", "kda_prefill", "long_gdn"])
+    ap.add_argument("--workload", default=HEADLINE,
+                    choices=["gdn_prefill", "kda_prefill", "long_gdn"],
+                    help="headline workload")
+    ap.add_argument("--extras", default=",".join(EXTRAS),
+                    help="comma-separated workloads timed beside the headline, or 'none'")
     ap.add_argument("--impl", default="lt2", choices=["lt2", "reference"])
     ap.add_argument("--order", default="delta_first", choices=["delta_first", "decay_first"],
                     help="order of the per-key factors (per-key workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-decode", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    extras = [] if args.extras in ("", "none") else [e for e in args.extras.split(",") if e]
+    for e in extras:
+        if e not in EXTRAS and e != HEADLINE:
+            ap.error(f"unknown extra workload {e!r}")
+    extras = [e for e in extras if e != args.workload]
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
@@ -381,74 +529,49 @@ def main():
 
     world, rank, local = dist_setup(args.gpus)
     lt2.lib()
-    w = inputs.workload(args.workload)
-    metric, unit = metric_of(w)
     peaks, peak_src = load_peaks()
-
-    x, o, S, dims, step = prefill_case(w, "cuda", args.order)
     sampler = ClockSampler(local) if rank == 0 else None
-    ms = timed(step, args.steps, args.warmup, world, sampler)
-    if lt2.lt2_gdr_last_device_error() != lt2.LT2_OK:
-        raise RuntimeError("device-side timeout during the benchmark")
-    clocks = sampler.stop() if sampler else None
-    tok_loops = w.T * w.B * w.L * world
-    value = gdist.whole_job_rate(w.T * w.B * w.L, world, ms)
+    cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
 
-    gate = w.gate
-    units_per_launch = w.B * w.H
-    launch_s = ms * 1e-3 / w.T
-    flops_launch = units_per_launch * w.L * FLOP_PER_TOKEN_HEAD[gate]
-    bytes_launch = units_per_launch * w.L * BYTES_PER_TOKEN_HEAD[gate]
-    kernel, source = (("gdr_prefill_tc_kernel", "gdr_prefill_tc.cu") if gate == "scalar"
-                      else ("gdr_prefill_kda_tc_kernel", "gdr_prefill_kda_tc.cu"))
-    achieved_tf = flops_launch / launch_s / 1e12
-    peak_tf = peaks["bf16_tflops"]
-    traffic, traffic_note = traffic_for(kernel, source, bytes_launch)
-    roofline = {"bound": "tensor", "kernel": kernel, "achieved": achieved_tf, "peak": peak_tf,
-                "unit": "TFLOP/s", "frac": achieved_tf / peak_tf,
-                "traffic": traffic,
-                "peak_source": f"{peak_src} bf16 dense (fp16 operands run at the same rate)",
-                "algorithmic_per_launch": {"flop": flops_launch, "bytes": bytes_launch},
-                "hbm": {"achieved": bytes_launch / launch_s / 1e9, "peak": peaks["hbm_gbs"],
-                        "unit": "GB/s", "frac": bytes_launch / launch_s / 1e9 / peaks["hbm_gbs"]},
-                "launch_time": "step time / T launches (the T loop launches of a step run back "
-                               "to back and overlap through programmatic dependent launch)"}
-    if traffic_note:
-        roofline["traffic_note"] = traffic_note
-
-    line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-            "config": config_of(w, world, args.order), "roofline": roofline,
-            "gpu_launches": args.steps * w.T}
-    if clocks:
-        line["clocks"] = clocks
-
-    if not args.no_decode:
-        wd, dms, dunits, dlaunch_s = run_decode(world, max(10, args.steps // 4), args.warmup)
-        dbytes = dunits * BYTES_PER_DECODE_UNIT
-        gbs = dbytes / dlaunch_s / 1e9
-        line["decode"] = {"metric": "looped GDR decode tokens*loops/s (decode)",
-                          "value": wd.T * wd.B * world / (dms * 1e-3), "unit": "tokens*loops/s",
-                          "ms_per_step": dms,
-                          "config": {"workload": "decode", "T": wd.T, "B": wd.B, "H": wd.H,
-                                     "d": wd.d, "state": "fp32, from a 4096-token prefill"},
-                          "roofline": {"bound": "hbm", "kernel": "gdr_decode_kernel",
-                                       "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                       "frac": gbs / peaks["hbm_gbs"],
-                                       "traffic": traffic_for("gdr_decode_kernel", "gdr_decode.cu")[0],
-                                       "peak_source": f"{peak_src} HBM copy"}}
-
+    # ---- headline ----
+    w = inputs.workload(args.workload)
+    head, case = run_prefill(w, args, world, sampler, peaks, peak_src, keep=not args.no_e2e)
+    line = {"metric": head["metric"], "value": head["value"], "unit": head["unit"], "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic", "config": head["config"], "roofline": head["roofline"],
+            "gpu_launches": head["gpu_launches"]}
     if not args.no_e2e:
-        ems, h2d, d2h = run_e2e(w, x, dims, max(3, args.steps // 20), args.warmup, world)
-        line["e2e"] = {"value": tok_loops / (ems * 1e-3), "unit": unit, "ms_per_step": ems,
-                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        x, _, _, dims, _ = case
+        ems, h2d, d2h = run_e2e(w, x, dims, 3, 1, world)
+        line["e2e"] = {"value": gdist.whole_job_rate(w.T * w.B * w.L, world, ems),
+                       "unit": head["unit"], "ms_per_step": ems, "steps": 3,
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "workload": w.name}
+        del case, x
+        torch.cuda.empty_cache()
+    if cpu:
+        line["cpu_baseline"] = cpu_entry(w, args.order, target_s=10.0)
 
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, threads, desc, single = oracle_sample(w, order=args.order)
-        line["cpu_baseline"] = {"value": v, "unit": unit, "cores": threads, "kind": "oracle",
-                                "sample": desc, "single_thread": single}
+    # ---- the other workloads, each with its own timing, roofline and baseline ----
+    for name in extras:
+        if name == "decode":
+            entry, (wd, xs, S_host) = run_decode(args, world, sampler, peaks, peak_src)
+            if cpu:
+                v, threads, desc = oracle_decode_sample(wd, xs, S_host)
+                entry["cpu_baseline"] = {"value": v, "unit": "tokens*loops/s", "cores": threads,
+                                         "kind": "oracle", "sample": desc}
+        else:
+            we = inputs.workload(name)
+            entry, _ = run_prefill(we, args, world, sampler, peaks, peak_src)
+            if cpu:
+                entry["cpu_baseline"] = cpu_entry(we, args.order, target_s=6.0)
+        line[name] = entry
 
+    if sampler is not None:
+        sampler.stop()
+        line["clocks"] = sampler.summary([w.name])
+        line["clocks_all_regions"] = sampler.summary()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -21,6 +21,7 @@ LT2_ERR_UNSUPPORTED = 2
 LT2_ERR_WORKSPACE = 3
 LT2_ERR_CUDA = 4
 LT2_ERR_DEVICE_TIMEOUT = 5
+LT2_ERR_RANGE = 6
 
 LT2_DTYPE_F32 = 0
 LT2_DTYPE_BF16 = 1
@@ -185,6 +186,8 @@ def _check(name, t, shape, dtype, device):
     and dtype (the C ABI reads raw row-major memory and cannot tell)."""
     if t is None:
         return
+    if not hasattr(t, "is_cuda"):
+        raise TypeError(f"{name} must be a torch tensor, got {type(t).__name__}")
     if not t.is_cuda or t.device != device:
         raise ValueError(f"{name} must be a CUDA tensor on {device}, got {t.device}")
     if not t.is_contiguous():
@@ -195,11 +198,21 @@ def _check(name, t, shape, dtype, device):
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
 
 
+def _require_cuda(q):
+    if not getattr(q, "is_cuda", False):
+        raise ValueError(f"q must be a CUDA tensor, got {getattr(q, 'device', type(q).__name__)}")
+
+
 def _check_call(q, k, v, alpha, beta, states, o, per_key, out):
-    """Validate the tensors of a prefill ([T,B,H,L,d]) or decode ([T,B,H,d]) call."""
+    """Validate the tensors of a prefill ([T,B,H,L,d]) or decode ([T,B,H,d]) call: all on q's
+    device, which must also be the current device (the library launches on the current one)."""
     import torch
     lead, dk, dv = tuple(q.shape[:-1]), q.shape[-1], v.shape[-1]
     dev = q.device
+    if dev.type != "cuda":
+        raise ValueError(f"q must be a CUDA tensor, got {dev}")
+    if dev.index != torch.cuda.current_device():
+        raise ValueError(f"q is on {dev} but the current device is cuda:{torch.cuda.current_device()}")
     _check("q", q, q.shape, q.dtype, dev)
     _check("k", k, q.shape, q.dtype, dev)
     _check("v", v, lead + (dv,), q.dtype, dev)
@@ -214,7 +227,16 @@ def prefill(q, k, v, alpha, beta, S0=None, per_key=None, algo=LT2_ALGO_AUTO, o=N
             S_out=None, out=None, stream=None, order="delta_first"):
     """Run the looped prefill on CUDA tensors; returns (o, S_out).  ``out`` selects the
     storage type of o: None/"same" (as the inputs), "f32" or "bf16"; ``order`` the order of
-    the per-key factors ("delta_first" as printed, or "decay_first")."""
+    the per-key factors ("delta_first" as printed, or "decay_first").  The call runs on the
+    tensors' device (made current for its duration), on ``stream`` or that device's current
+    stream."""
+    import torch
+    _require_cuda(q)
+    with torch.cuda.device(q.device):
+        return _prefill(q, k, v, alpha, beta, S0, per_key, algo, o, S_out, out, stream, order)
+
+
+def _prefill(q, k, v, alpha, beta, S0, per_key, algo, o, S_out, out, stream, order):
     import torch
     dims = _dims_from(q, v, alpha, per_key, algo, out, order)
     _check_call(q, k, v, alpha, beta, [("S0", S0), ("S_out", S_out)], o, dims.gate != LT2_GATE_SCALAR, out)
@@ -232,7 +254,15 @@ def prefill(q, k, v, alpha, beta, S0=None, per_key=None, algo=LT2_ALGO_AUTO, o=N
 
 
 def decode(q, k, v, alpha, beta, S, per_key=None, o=None, out=None, stream=None, order="delta_first"):
-    """One decode token per (loop, batch, head); q/k/v [T,B,H,d]; S updated in place."""
+    """One decode token per (loop, batch, head); q/k/v [T,B,H,d]; S updated in place.  Runs
+    on the tensors' device (made current for the call)."""
+    import torch
+    _require_cuda(q)
+    with torch.cuda.device(q.device):
+        return _decode(q, k, v, alpha, beta, S, per_key, o, out, stream, order)
+
+
+def _decode(q, k, v, alpha, beta, S, per_key, o, out, stream, order):
     import torch
     per_key = (alpha.dim() == 4) if per_key is None else per_key
     T, B, H, dk = q.shape

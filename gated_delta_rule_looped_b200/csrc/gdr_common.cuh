@@ -7,10 +7,13 @@
 
 namespace lt2 {
 
-// Device-side status word written by bounded waits (see lt2_gdr_last_device_error).
+// Device-side status word (bit flags, see lt2_gdr_last_device_error): a bounded wait ran
+// out; a tensor-core path produced a non-finite output or state (its fp16 operands out of
+// range, or non-finite inputs).
 enum : unsigned int {
     kDevOk = 0u,
     kDevTimeout = 1u,
+    kDevRange = 2u,
 };
 
 // Per-launch view of one loop's slice: base pointers already offset to loop tau.

@@ -59,6 +59,7 @@
 
 #include "gdr_common.cuh"
 #include "gdr_launch.h"
+#include "gdr_nvtx.h"
 #include "gdr_tc_common.cuh"
 #include "gdr_tma_host.h"
 #include "sm100_primitives.cuh"
@@ -479,15 +480,19 @@ __device__ __forceinline__ void state_update(uint32_t tm_s, uint32_t tm_sh, cons
 }
 
 // Chain thread (d_v column j, keys 32 piece .. + 63): that part of column j of the final state,
-// f (.) TM_S (nullptr: 1), to S_out.
-__device__ __noinline__ void store_final_state_scaled(uint32_t tm_s, float* so, const float* f, int piece)
+// f (.) TM_S (nullptr: 1), to S_out.  Returns false if any entry is not finite.
+__device__ __noinline__ bool store_final_state_scaled(uint32_t tm_s, float* so, const float* f, int piece)
 {
-    {
-        float v[64];
-        tmem_load_2x32(tm_s + 32 * piece, tm_s + 32 * piece + 32, v);
-        #pragma unroll
-        for (int d = 0; d < 64; ++d) so[(32 * piece + d) * kD] = f ? v[d] * f[32 * piece + d] : v[d];
+    bool fin = true;
+    float v[64];
+    tmem_load_2x32(tm_s + 32 * piece, tm_s + 32 * piece + 32, v);
+    #pragma unroll
+    for (int d = 0; d < 64; ++d) {
+        const float x = f ? v[d] * f[32 * piece + d] : v[d];
+        fin &= is_finite(x);
+        so[(32 * piece + d) * kD] = x;
     }
+    return fin;
 }
 
 // Chain thread j: the chunk's n tokens run one at a time on column j of the fp32 state in
@@ -501,11 +506,13 @@ struct ExactIn {
     const float* beta;
     void* o;
     int out_bf16;
+    unsigned int* err;      // status word: a non-finite output is flagged there
 };
 // decay_first: (I - beta k k^T) Diag(alpha), e = (alpha . k)^T S, S <- Diag(alpha) S + beta k (v - e)
 template <bool decay_first>
 __device__ __noinline__ void exact_chunk(uint32_t tm_s, ExactIn p, int64_t row0, int n, int j)
 {
+    bool fin = true;
     #pragma unroll 1
     for (int t = 0; t < n; ++t) {
         const int64_t row = row0 + t;
@@ -570,22 +577,32 @@ __device__ __noinline__ void exact_chunk(uint32_t tm_s, ExactIn p, int64_t row0,
             tmem_st32(tm_s + 64 * h + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
             tmem_wait_st();
         }
+        fin &= is_finite(o);
         if (p.out_bf16)
             static_cast<__nv_bfloat16*>(p.o)[row * kD + j] = __float2bfloat16_rn(o);
         else
             static_cast<float*>(p.o)[row * kD + j] = o;
     }
+    if (!fin) atomicOr(p.err, kDevRange);
 }
 
 // Chain thread j, fp32 output: o[r][j] = (Q^ S)_rj - B_rj for tokens r = r0 .. r0 + 15 below n
 // (tm_qs and tm_b address token r0).
-__device__ __noinline__ void store_o_f32(uint32_t tm_qs, uint32_t tm_b, float* o, int r0, int n)
+// Returns false if any of them is not finite.
+__device__ __noinline__ bool store_o_f32(uint32_t tm_qs, uint32_t tm_b, float* o, int r0, int n)
 {
     float qp[32];
     tmem_load_2x16(tm_qs, tm_b, qp);
+    bool fin = true;
     #pragma unroll
-    for (int r = 0; r < 16; ++r)
-        if (r0 + r < n) o[(r0 + r) * kD] = qp[r] - qp[16 + r];
+    for (int r = 0; r < 16; ++r) {
+        const float ov = qp[r] - qp[16 + r];
+        if (r0 + r < n) {
+            fin &= is_finite(ov);
+            o[(r0 + r) * kD] = ov;
+        }
+    }
+    return fin;
 }
 
 // Gram [Kt; Qt; -] [Be; Bv]^T (M = 128, N = 64, K = 128) into TMEM, Be and Bv from the chunk
@@ -920,16 +937,24 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                     __syncwarp();
                 }
                 // --- while MMA_C runs: o = Q^ S - (the -O' half of MMA_B), tokens 16h .. + 15 ---
+                // (a non-finite output is flagged where it is found: rows past L are finite too,
+                // from zero inputs, so a flag means a real output went out of range)
                 if (!p.out_bf16) {
-                    store_o_f32(tmem + TM_AB + lane_addr + 32 + 16 * h, tmem + TM_B + lane_addr + 32 + 16 * h,
-                                static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, 16 * h, n);
+                    if (!store_o_f32(tmem + TM_AB + lane_addr + 32 + 16 * h, tmem + TM_B + lane_addr + 32 + 16 * h,
+                                     static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, 16 * h, n))
+                        atomicOr(err, kDevRange);
                 } else {
                     float qp[32];
                     tmem_load_2x16(tmem + TM_AB + lane_addr + 32 + 16 * h, tmem + TM_B + lane_addr + 32 + 16 * h, qp);
                     uint8_t* ost = sbase + OFF_OST + (j >> 6) * 4096 + (j & 63) * 2 + 16 * h * 128;
+                    bool bad = false;
                     #pragma unroll
-                    for (int r = 0; r < 16; ++r)
-                        *reinterpret_cast<__nv_bfloat16*>(ost + r * 128) = __float2bfloat16_rn(qp[r] - qp[16 + r]);
+                    for (int r = 0; r < 16; ++r) {
+                        const float ov = qp[r] - qp[16 + r];
+                        bad |= !is_finite(ov);
+                        *reinterpret_cast<__nv_bfloat16*>(ost + r * 128) = __float2bfloat16_rn(ov);
+                    }
+                    if (bad) atomicOr(err, kDevRange);
                     fence_proxy_async_smem();
                 }
                 // MMA_C done, and the next chunk's gates written
@@ -947,8 +972,9 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 // --- out-of-range chunk: the definition, token by token, on the fp32 state (the
                 // first half of the chain's warps; every key of a column takes part in k^T S) ---
                 if (h == 0)
-                    exact_chunk<kDecayFirst>(tmem + TM_S + lane_addr, ExactIn{p.q, p.k, p.v, p.alpha, p.beta, p.o, p.out_bf16},
-                                static_cast<int64_t>(ug) * L + t0, n, j);
+                    exact_chunk<kDecayFirst>(tmem + TM_S + lane_addr,
+                                             ExactIn{p.q, p.k, p.v, p.alpha, p.beta, p.o, p.out_bf16, err},
+                                             static_cast<int64_t>(ug) * L + t0, n, j);
                 tc_fence_before();
                 // keep every hand-off in step: the stage and the [X; Z] stage are released
                 // once their producers are done with them, the output epilogue is released
@@ -966,9 +992,9 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             // TM_S holds S' / sq after a tensor-core chunk, S' itself after an exact one
             const float* f_sh = exact ? nullptr : gs->sq;
             if (last) {
-                if (p.S_out)
-                    store_final_state_scaled(tmem + TM_S + lane_addr, p.S_out + static_cast<int64_t>(ug) * kD * kD + j, f_sh,
-                                             2 * h);
+                if (p.S_out && !store_final_state_scaled(tmem + TM_S + lane_addr,
+                                                         p.S_out + static_cast<int64_t>(ug) * kD * kD + j, f_sh, 2 * h))
+                    atomicOr(err, kDevRange);
                 drain_needed = 0;
             } else {
                 const Gates* g1 = gate(s1);
@@ -1018,6 +1044,7 @@ cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream)
                                          static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess) return e;
     for (int64_t tau = 0; tau < call.T; ++tau) {
+        NvtxRange loop_range("lt2 prefill loop (tensor core, per-key gating)");
         Params p;
         p.q = static_cast<const __nv_bfloat16*>(call.q);
         p.k = static_cast<const __nv_bfloat16*>(call.k);

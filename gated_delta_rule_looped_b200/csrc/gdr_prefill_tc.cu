@@ -51,6 +51,7 @@
 
 #include "gdr_common.cuh"
 #include "gdr_launch.h"
+#include "gdr_nvtx.h"
 #include "gdr_tc_common.cuh"
 #include "gdr_tma_host.h"
 #include "sm100_primitives.cuh"
@@ -190,8 +191,10 @@ __device__ __noinline__ void load_initial_state(uint32_t tm_s, uint32_t tm_sh, c
 }
 
 // Output thread j, fp32 output: o[r][j] = g_r (Q S)_rj + (P T X)_rj for the chunk's n tokens.
-__device__ __noinline__ void store_o_f32(uint32_t tm_qs, uint32_t tm_ptx, const float* gam, float* o, int n)
+// Returns false if any of them is not finite.
+__device__ __noinline__ bool store_o_f32(uint32_t tm_qs, uint32_t tm_ptx, const float* gam, float* o, int n)
 {
+    bool fin = true;
     #pragma unroll 1
     for (int piece = 0; piece < 2; ++piece) {
         float qp[64];
@@ -199,9 +202,14 @@ __device__ __noinline__ void store_o_f32(uint32_t tm_qs, uint32_t tm_ptx, const 
         #pragma unroll
         for (int e = 0; e < 32; ++e) {
             const int r = 32 * piece + e;
-            if (r < n) o[r * kD] = gam[r] * qp[e] + qp[32 + e];
+            const float ov = gam[r] * qp[e] + qp[32 + e];
+            if (r < n) {
+                fin &= is_finite(ov);
+                o[r * kD] = ov;
+            }
         }
     }
+    return fin;
 }
 
 // Prep thread t, chunks whose decay e^{-G} is not representable: row r of -A (t < 64) or of P
@@ -211,7 +219,8 @@ __device__ __noinline__ void gram_epilogue_unfactored(uint32_t tm_row, const Gat
                                                       uint8_t* dst_ptr, uint32_t dst, float* adiag_row)
 {
     const int lim = is_a ? r : r + 1;
-    const float sg = is_a ? -1.f : 1.f;
+    // the sign of the decay ratio is the product of the signs of gam_r and gam_s
+    const float sg = copysignf(1.f, gs->gam[r]) * (is_a ? -1.f : 1.f);
     const float Gr = gs->G[r];
     #pragma unroll 1
     for (int ch = 0; ch < 8; ++ch) {
@@ -220,7 +229,8 @@ __device__ __noinline__ void gram_epilogue_unfactored(uint32_t tm_row, const Gat
         #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const int sc = 8 * ch + e;
-            v[e] = (sc < lim) ? sg * gs->beta[sc] * __expf(Gr - gs->G[sc]) * v[e] : 0.f;
+            const float ss = gs->beta[sc] * copysignf(1.f, gs->gam[sc]);
+            v[e] = (sc < lim) ? sg * ss * __expf(Gr - gs->G[sc]) * v[e] : 0.f;
         }
         if (is_a && (ch >> 1) == (r >> 4)) {
             #pragma unroll
@@ -348,13 +358,18 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 Gates* gs = gate(s);
                 const int64_t t0 = static_cast<int64_t>(c) * kC;
                 float g[2], b[2];
+                uint32_t negs[2];
                 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
                     const int64_t tok = t0 + lane + 32 * i;
                     const bool valid = tok < L;
                     const float a = valid ? p.alpha[ug * L + tok] : 1.f;
                     b[i] = valid ? p.beta[ug * L + tok] : 0.f;
-                    g[i] = __logf(fmaxf(a, 1e-30f));
+                    // alpha = |alpha| * sign: the magnitudes go through the log-domain prefix
+                    // sums, the signs through a parity count (alpha = 0 is taken as 1e-30, a
+                    // reset to within 1e-30 of the state)
+                    g[i] = __logf(fmaxf(fabsf(a), 1e-30f));
+                    negs[i] = __ballot_sync(0xffffffffu, a < 0.f);
                 }
                 // inclusive prefix sums over the 64 tokens
                 #pragma unroll
@@ -367,18 +382,31 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
                 g[1] += __shfl_sync(0xffffffffu, g[0], 31);
                 const float GC = __shfl_sync(0xffffffffu, g[1], 31);
-                const bool safe = GC > -80.f;
+                // the factored decay e^{G_r} e^{-G_s} needs both factors representable
+                float gmin = fminf(g[0], g[1]), gmax = fmaxf(g[0], g[1]);
+                #pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    gmin = fminf(gmin, __shfl_xor_sync(0xffffffffu, gmin, off));
+                    gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, off));
+                }
+                const bool safe = gmin > -80.f && gmax < 80.f;
+                // sign of the product of the alphas up to token r: parity of the negatives
+                const uint32_t upto = 0xffffffffu >> (31 - lane);
+                const float sgn[2] = {(__popc(negs[0] & upto) & 1) ? -1.f : 1.f,
+                                      ((__popc(negs[0]) + __popc(negs[1] & upto)) & 1) ? -1.f : 1.f};
+                const float sgnC = ((__popc(negs[0]) + __popc(negs[1])) & 1) ? -1.f : 1.f;
                 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
                     const int r = lane + 32 * i;
                     gs->G[r] = g[i];
-                    gs->gam[r] = __expf(g[i]);
-                    gs->bein[r] = safe ? b[i] * __expf(-g[i]) : 0.f;
+                    // the sign of gam[r] (also kept by a zero) is the sign of the product
+                    gs->gam[r] = sgn[i] * __expf(g[i]);
+                    gs->bein[r] = safe ? sgn[i] * b[i] * __expf(-g[i]) : 0.f;
                     gs->beta[r] = b[i];
-                    gs->bgc[r] = b[i] * __expf(GC - g[i]);
+                    gs->bgc[r] = sgnC * sgn[i] * b[i] * __expf(GC - g[i]);
                 }
                 if (lane == 0) {
-                    gs->gC = __expf(GC);
+                    gs->gC = sgnC * __expf(GC);
                     gs->safe = safe ? 1 : 0;
                 }
                 __syncwarp();
@@ -618,8 +646,11 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (!ok) break;
             tc_fence_after();
             if (last) {
-                if (p.S_out)
-                    store_final_state(tmem + TM_S + lane_addr, p.S_out + static_cast<int64_t>(ug) * kD * kD + j);
+                if (p.S_out) {
+                    const bool sfin = store_final_state(tmem + TM_S + lane_addr,
+                                                        p.S_out + static_cast<int64_t>(ug) * kD * kD + j);
+                    if (__any_sync(0xffffffffu, !sfin) && lane == 0) atomicOr(err, kDevRange);
+                }
                 drain_needed = 0;
             } else {
                 const float gn = gate(s1)->gC;
@@ -651,6 +682,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const int j = threadIdx.x - 384;            // TMEM lane = d_v index
         const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
         Group grp{NB_OUT, 128, j == 0, okflags + 4, 0, abort_flag, err};
+        bool fin = true;                             // every output so far is finite
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;
             if (j == 0) bulk_wait_read_all();        // the staging tile is free again
@@ -661,8 +693,8 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (!p.out_bf16) {
                 // fp32 output: plain stores, done before the TMEM columns are released
                 const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
-                store_o_f32(tmem + TM_AB + lane_addr + 64, tmem + TM_B + lane_addr + 64, gs->gam,
-                            static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, n);
+                fin &= store_o_f32(tmem + TM_AB + lane_addr + 64, tmem + TM_B + lane_addr + 64, gs->gam,
+                                   static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, n);
                 tc_fence_before();
                 grp.sync();
                 if (j == 0) {
@@ -685,10 +717,13 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 #pragma unroll
                 for (int e4 = 0; e4 < 32; e4 += 4) {
                     const float4 g4 = *reinterpret_cast<const float4*>(gam + e4);
-                    *reinterpret_cast<__nv_bfloat16*>(orow + (e4 + 0) * 128) = __float2bfloat16_rn(g4.x * qp[e4 + 0] + qp[32 + e4 + 0]);
-                    *reinterpret_cast<__nv_bfloat16*>(orow + (e4 + 1) * 128) = __float2bfloat16_rn(g4.y * qp[e4 + 1] + qp[32 + e4 + 1]);
-                    *reinterpret_cast<__nv_bfloat16*>(orow + (e4 + 2) * 128) = __float2bfloat16_rn(g4.z * qp[e4 + 2] + qp[32 + e4 + 2]);
-                    *reinterpret_cast<__nv_bfloat16*>(orow + (e4 + 3) * 128) = __float2bfloat16_rn(g4.w * qp[e4 + 3] + qp[32 + e4 + 3]);
+                    const float ov[4] = {g4.x * qp[e4 + 0] + qp[32 + e4 + 0], g4.y * qp[e4 + 1] + qp[32 + e4 + 1],
+                                         g4.z * qp[e4 + 2] + qp[32 + e4 + 2], g4.w * qp[e4 + 3] + qp[32 + e4 + 3]};
+                    #pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        fin &= is_finite(ov[u]);
+                        *reinterpret_cast<__nv_bfloat16*>(orow + (e4 + u) * 128) = __float2bfloat16_rn(ov[u]);
+                    }
                 }
             }
             tc_fence_before();
@@ -703,6 +738,9 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
         }
         if (j == 0) bulk_wait_all();     // every output tile written before the CTA exits
+        // rows past L of the last chunk are finite too (zero inputs), so a flag here means a
+        // real output went out of range
+        if (__any_sync(0xffffffffu, !fin) && lane == 0) atomicOr(err, kDevRange);
     }
 
     tc_fence_before();
@@ -738,6 +776,7 @@ cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
                                          static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess) return e;
     for (int64_t tau = 0; tau < call.T; ++tau) {
+        NvtxRange loop_range("lt2 prefill loop (tensor core, scalar gating)");
         Params p;
         p.alpha = call.alpha;
         p.beta = call.beta;

@@ -201,16 +201,25 @@ __device__ __forceinline__ void convert_tile(uint32_t base, int n16, int lane, L
     }
 }
 
-// Chain thread j: column j of the final state (row j of S^T in TMEM) to S_out.
-static __device__ __noinline__ void store_final_state(uint32_t tm_s, float* so)
+// False for an infinity or a NaN.
+__device__ __forceinline__ bool is_finite(float x) { return fabsf(x) <= 3.402823466e38f; }
+
+// Chain thread j: column j of the final state (row j of S^T in TMEM) to S_out.  Returns false
+// if any entry is not finite.
+static __device__ __noinline__ bool store_final_state(uint32_t tm_s, float* so)
 {
+    bool fin = true;
     #pragma unroll 1
     for (int piece = 0; piece < 4; piece += 2) {
         float v[64];
         tmem_load_2x32(tm_s + 32 * piece, tm_s + 32 * piece + 32, v);
         #pragma unroll
-        for (int d = 0; d < 64; ++d) so[(32 * piece + d) * kD] = v[d];
+        for (int d = 0; d < 64; ++d) {
+            fin &= is_finite(v[d]);
+            so[(32 * piece + d) * kD] = v[d];
+        }
     }
+    return fin;
 }
 
 }  // namespace tcc

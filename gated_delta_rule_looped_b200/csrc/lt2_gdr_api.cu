@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <initializer_list>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -10,12 +11,20 @@
 
 #include "gdr_common.cuh"
 #include "gdr_launch.h"
+#include "gdr_nvtx.h"
 #include "lt2_gdr.h"
 
 namespace {
 
-// Status word of bounded in-kernel waits; one instance per device that loads the library.
-__device__ unsigned int g_lt2_device_status = 0u;
+// Status word of the kernels on this device (bit flags, see gdr_common.cuh), followed by the
+// slot that lt2_gdr_last_device_error() swaps it into; one instance per device that loads the
+// library, shared by every call on that device.
+__device__ unsigned int g_lt2_device_status[2] = {0u, 0u};
+
+// Reads the status word and clears it in one atomic step, leaving the old value in word 1.
+__global__ void take_status_kernel(unsigned int* w) { w[1] = atomicExch(&w[0], 0u); }
+
+using lt2::NvtxRange;
 
 thread_local char t_cuda_error[256] = {0};
 
@@ -113,7 +122,31 @@ lt2_status validate_dims(const lt2_gdr_dims* d, Sizes* sz)
     sz->st = (int64_t)(units * d->dk * d->dv);
     sz->esz = d->dtype == LT2_DTYPE_BF16 ? 2 : 4;
     sz->osz = out_is_bf16(d) ? 2 : 4;
-    if (sz->units > 0 && sz->per_loop >= kMaxDim) return LT2_ERR_UNSUPPORTED;
+    // Head-units are indexed with 32-bit integers inside the kernels (grid size, the first
+    // unit of a loop, TMA coordinates).
+    if (sz->units >= kMaxDim) return LT2_ERR_UNSUPPORTED;
+    return LT2_OK;
+}
+
+// Every non-null pointer must address device memory of the current device: kernels launch
+// on the current device, and the tensor maps of the tensor-core path would otherwise cover
+// another GPU's memory.
+lt2_status on_current_device(std::initializer_list<const void*> ptrs)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    for (const void* p : ptrs) {
+        if (!p) continue;
+        cudaPointerAttributes a;
+        e = cudaPointerGetAttributes(&a, p);
+        if (e != cudaSuccess) {
+            (void)cudaGetLastError();      // not a pointer CUDA knows (the error is not sticky)
+            return LT2_ERR_INVALID_ARGUMENT;
+        }
+        const bool device_mem = a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+        if (!device_mem || a.device != dev) return LT2_ERR_INVALID_ARGUMENT;
+    }
     return LT2_OK;
 }
 
@@ -206,7 +239,10 @@ lt2_status lt2_gdr_prefill(const lt2_gdr_dims* dims, const void* q, const void* 
             return LT2_ERR_INVALID_ARGUMENT;
     }
     if (sz.units == 0) return LT2_OK;
+    st = on_current_device({q, k, v, alpha, beta, S0, o, S_out, workspace});
+    if (st != LT2_OK) return st;
 
+    NvtxRange range("lt2_gdr_prefill");
     unsigned int* err = nullptr;
     st = status_word(&err);
     if (st != LT2_OK) return st;
@@ -240,6 +276,7 @@ lt2_status lt2_gdr_prefill(const lt2_gdr_dims* dims, const void* q, const void* 
         // Loop 0 waits for all earlier work on the stream; later loops may start as soon as
         // the previous loop's grid is running (the loops share no data).
         const bool pdl = tau > 0;
+        NvtxRange loop_range("lt2 prefill loop (cuda core)");
         cudaError_t e = lt2::launch_prefill_seq(ls, dims->dtype == LT2_DTYPE_BF16, s, pdl);
         if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "prefill (cuda core)");
@@ -266,12 +303,16 @@ lt2_status lt2_gdr_decode(const lt2_gdr_dims* dims, const void* q, const void* k
     for (const Range& r : rin)
         if (overlap(ro, r) || overlap(rs, r)) return LT2_ERR_INVALID_ARGUMENT;
     if (sz.units == 0) return LT2_OK;
+    st = on_current_device({q, k, v, alpha, beta, S, o});
+    if (st != LT2_OK) return st;
 
+    NvtxRange range("lt2_gdr_decode");
     unsigned int* err = nullptr;
     st = status_word(&err);
     if (st != LT2_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     for (int64_t tau = 0; tau < dims->T; ++tau) {
+        NvtxRange loop_range("lt2 decode loop");
         lt2::LoopSlice ls = loop_slice(dims, sz, tau, q, k, v, alpha, beta, nullptr, o, S, err);
         cudaError_t e = lt2::launch_decode(ls, dims->dtype == LT2_DTYPE_BF16, s, tau > 0);
         if (e == cudaSuccess) e = cudaGetLastError();
@@ -285,14 +326,21 @@ lt2_status lt2_gdr_last_device_error(void)
     unsigned int* p = nullptr;
     lt2_status st = status_word(&p);
     if (st != LT2_OK) return st;
+    // Every stream of the device, blocking or not, has finished its work before the word is
+    // read; the read and the clear are one atomic exchange on the device, so a flag that a
+    // kernel raises concurrently (another thread's work) is never lost, only left for the
+    // next call.
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    take_status_kernel<<<1, 1, 0, 0>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "take device status");
     unsigned int h = 0;
-    cudaError_t e = cudaMemcpy(&h, p, sizeof(h), cudaMemcpyDeviceToHost);
+    e = cudaMemcpy(&h, p + 1, sizeof(h), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e, "read device status");
-    if (h == lt2::kDevOk) return LT2_OK;
-    const unsigned int zero = 0;
-    e = cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice);
-    if (e != cudaSuccess) return cuda_fail(e, "clear device status");
-    return LT2_ERR_DEVICE_TIMEOUT;
+    if (h & lt2::kDevTimeout) return LT2_ERR_DEVICE_TIMEOUT;
+    if (h & lt2::kDevRange) return LT2_ERR_RANGE;
+    return LT2_OK;
 }
 
 const char* lt2_status_string(lt2_status s)
@@ -304,12 +352,13 @@ const char* lt2_status_string(lt2_status s)
         case LT2_ERR_WORKSPACE: return "LT2_ERR_WORKSPACE";
         case LT2_ERR_CUDA: return "LT2_ERR_CUDA";
         case LT2_ERR_DEVICE_TIMEOUT: return "LT2_ERR_DEVICE_TIMEOUT";
+        case LT2_ERR_RANGE: return "LT2_ERR_RANGE";
     }
     return "LT2_STATUS_UNKNOWN";
 }
 
 const char* lt2_last_cuda_error_string(void) { return t_cuda_error; }
 
-int lt2_gdr_version(void) { return 100; }
+int lt2_gdr_version(void) { return 200; }
 
 }  // extern "C"

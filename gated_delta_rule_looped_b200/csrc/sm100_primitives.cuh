@@ -352,7 +352,6 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
     return r;
 }
 
-// Two bf16 in one 32-bit word -> two floats (exact).
 // Approximate reciprocal (one MUFU instruction, relative error ~2^-22; denormals flush to 0).
 __device__ __forceinline__ float rcp_approx(float x)
 {
@@ -382,6 +381,7 @@ __device__ __forceinline__ float half_hi(uint32_t h2)
 {
     return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
 }
+// The two bf16 halves of a 32-bit word (low half = lower element index) as floats, exactly.
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 

@@ -24,17 +24,24 @@
  *   S0, S_out, S  [T][B][H][dk][dv] fp32 (d_v fastest)
  * Decode uses the same layouts with L = 1.
  *
- * Ownership and execution.  Every pointer is a DEVICE pointer owned by the caller (the
- * library never allocates, frees or synchronises on these entry points).  Work is enqueued
- * on `stream` (a cudaStream_t; NULL = legacy default stream) of the current device and
- * completes asynchronously.  The T loops are launched back to back on that stream with no
- * host synchronisation.
+ * Ownership and execution.  Every pointer is a DEVICE pointer owned by the caller, in memory
+ * of the CURRENT device (cudaGetDevice); the library never allocates, frees or synchronises on
+ * the compute entry points.  Work is enqueued on `stream` (a cudaStream_t of the current
+ * device; NULL = legacy default stream) and completes asynchronously.  The T loops are
+ * launched back to back on that stream with no host synchronisation.
  *
- * Errors.  Argument validation happens before any launch and returns synchronously.  A
- * failed launch returns LT2_ERR_CUDA (the CUDA error text is available from
- * lt2_last_cuda_error_string()).  Waits inside kernels are bounded: a wait that runs out
- * makes the kernel record LT2_ERR_DEVICE_TIMEOUT in a device-side status word and return;
- * lt2_gdr_last_device_error() reads (and clears) it.  No C++ exception crosses the ABI.
+ * Errors.  Argument validation happens before any launch and returns synchronously: a pointer
+ * that is not device memory of the current device is LT2_ERR_INVALID_ARGUMENT.  A failed
+ * launch returns LT2_ERR_CUDA (the CUDA error text is available from
+ * lt2_last_cuda_error_string()).  Conditions found while the kernels run are recorded as bit
+ * flags in one status word per device, shared by every call on that device, and read (and
+ * cleared) by lt2_gdr_last_device_error():
+ *   - waits inside kernels are bounded; a wait that runs out makes the kernel record
+ *     LT2_ERR_DEVICE_TIMEOUT, release what it holds and return;
+ *   - a tensor-core prefill whose output or final state is not finite (its fp16 operands went
+ *     out of range, or an input was not finite) records LT2_ERR_RANGE; the results of that
+ *     call are then not valid, and LT2_ALGO_CUDA_CORE computes the same call in fp32.
+ * No C++ exception crosses the ABI.
  *
  * Supported set.
  *   The tensor-core chunked prefills serve bf16 inputs with dk = dv = 128, for scalar gating
@@ -43,7 +50,9 @@
  *   ~e^-19, or with any alpha <= 0 (a reset), is evaluated token by token inside the same
  *   kernel (exact, slower).  The tensor-core paths take their operands in fp16: alpha is
  *   expected in (0, 1] (a growing alpha > 1 works while the state stays below ~3e4 in
- *   magnitude), with |q|, |k| entries of order 1.
+ *   magnitude), with |q|, |k| entries of order 1.  Outside that range the call records
+ *   LT2_ERR_RANGE instead of returning silent infinities.  Scalar gating takes any real alpha
+ *   (alpha = 0 is a reset; a negative alpha flips the sign of the decayed state).
  *   fp32 inputs: dk, dv multiples of 8 up to 128 (CUDA-core fp32 arithmetic throughout).
  *   bf16 inputs: dk, dv multiples of 8 up to 128.
  *   Any L >= 0 (a ragged final chunk is fine; L = 0 copies S0 to S_out).
@@ -66,7 +75,8 @@ typedef enum lt2_status {
     LT2_ERR_UNSUPPORTED = 2,      /* valid but outside the supported set above            */
     LT2_ERR_WORKSPACE = 3,        /* workspace smaller than lt2_gdr_prefill_workspace_bytes */
     LT2_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed                   */
-    LT2_ERR_DEVICE_TIMEOUT = 5    /* a bounded in-kernel wait ran out (see header comment)  */
+    LT2_ERR_DEVICE_TIMEOUT = 5,   /* a bounded in-kernel wait ran out (see header comment)  */
+    LT2_ERR_RANGE = 6             /* a tensor-core path produced non-finite results         */
 } lt2_status;
 
 typedef enum lt2_dtype { LT2_DTYPE_F32 = 0, LT2_DTYPE_BF16 = 1 } lt2_dtype;
@@ -112,16 +122,30 @@ typedef struct lt2_gdr_dims {
 } lt2_gdr_dims;
 
 /*
- * Bytes of device workspace lt2_gdr_prefill needs for `dims` (0 when none).  Pure host
- * function; returns 0 for invalid dims as well.
+ * Bytes of device workspace lt2_gdr_prefill needs for `dims` (0 when none; every path of this
+ * version keeps its intermediates on chip, so it is 0 for every valid `dims`).  Pure host
+ * function, no CUDA call; returns 0 for invalid dims as well.
  */
 size_t lt2_gdr_prefill_workspace_bytes(const lt2_gdr_dims* dims);
 
 /*
- * Chunked prefill over all T loops (the displayed equation over L tokens, for every
- * (loop, batch, head)).  Writes every o_t and, if S_out is non-NULL, the state after the
- * last token.  S0 == NULL means a zero initial state.  `workspace` may be NULL when
- * lt2_gdr_prefill_workspace_bytes(dims) is 0.
+ * Prefill: the recurrence of "LT2 transformer looped a tempo lineare", section "Sostituire il
+ * motore", displayed equation, over all L tokens of every (loop, batch, head), for all T
+ * loops of section "Profondita presa in prestito", each loop with its own q/k/v, S0 and final
+ * state.  Writes every o_t = S_t^T q_t and, if S_out is non-NULL, the state after the last
+ * token.
+ *   dims       problem sizes, dtypes, gating, algorithm (host pointer, read during the call)
+ *   q, k, v    inputs in the layouts above (device, read only)
+ *   alpha      decay: [T][B][H][L] fp32 for LT2_GATE_SCALAR, [T][B][H][L][dk] per key
+ *   beta       write strength [T][B][H][L] fp32
+ *   S0         initial states, or NULL for zero states
+ *   o          outputs, dims->out_dtype (device, written; must not alias an input)
+ *   S_out      final states, or NULL (may equal S0 exactly: in-place resume)
+ *   workspace  device scratch of lt2_gdr_prefill_workspace_bytes(dims) bytes (NULL when 0)
+ *   stream     cudaStream_t of the current device
+ * Returns LT2_OK once the launches are enqueued; LT2_ERR_INVALID_ARGUMENT, _UNSUPPORTED or
+ * _WORKSPACE before any launch; LT2_ERR_CUDA if a launch failed.  Device-side conditions come
+ * later from lt2_gdr_last_device_error().
  */
 lt2_status lt2_gdr_prefill(const lt2_gdr_dims* dims,
                            const void* q, const void* k, const void* v,
@@ -132,9 +156,12 @@ lt2_status lt2_gdr_prefill(const lt2_gdr_dims* dims,
                            void* stream);
 
 /*
- * One decode token per (loop, batch, head): dims->L must be 1.  S is read and replaced in
- * place by the state after the token; o receives o = S_new^T q.  Each state is streamed
- * through HBM once (read once, written once).
+ * Decode: one step of the same recurrence ("LT2 transformer looped a tempo lineare", section
+ * "Sostituire il motore", displayed equation) for one new token per (loop, batch, head);
+ * dims->L must be 1 and dims->algo is ignored.  S [T][B][H][dk][dv] fp32 is read and replaced
+ * in place by the state after the token; o receives o = S_new^T q.  Each state is streamed
+ * through HBM once (read once, written once).  q, k, v, alpha, beta, o: the layouts above with
+ * L = 1; o must alias neither S nor an input.  Same return convention as lt2_gdr_prefill.
  */
 lt2_status lt2_gdr_decode(const lt2_gdr_dims* dims,
                           const void* q, const void* k, const void* v,
@@ -143,20 +170,25 @@ lt2_status lt2_gdr_decode(const lt2_gdr_dims* dims,
                           void* stream);
 
 /*
- * Status word written by bounded in-kernel waits on the CURRENT device.  Blocks until all
- * previously issued work on the device has finished (it reads device memory), returns
- * LT2_ERR_DEVICE_TIMEOUT if any kernel gave up on a wait since the last call (and clears
- * the word), LT2_OK otherwise, or LT2_ERR_CUDA if the read itself failed.
+ * The device-side status word of the CURRENT device (not an operation of the pages: the
+ * library's own failure reporting).  Synchronises the device (every stream), then reads and
+ * clears the word in one atomic exchange.  Returns LT2_ERR_DEVICE_TIMEOUT if a kernel gave up
+ * on a bounded wait since the last read, else LT2_ERR_RANGE if a tensor-core prefill produced
+ * non-finite results, else LT2_OK; LT2_ERR_CUDA if the synchronisation or the read failed.
+ * The word is shared by every call on the device, from any thread or stream: a flag belongs
+ * to whichever work ran since the previous read.
  */
 lt2_status lt2_gdr_last_device_error(void);
 
-/* Static, human-readable name of a status code. */
+/* Static, human-readable name of a status code (library bookkeeping, no counterpart on the
+ * pages; never NULL). */
 const char* lt2_status_string(lt2_status status);
 
-/* Text of the last CUDA error seen by this library on the calling thread ("" if none). */
+/* Text of the last CUDA error seen by this library on the calling thread ("" if none;
+ * library bookkeeping, no counterpart on the pages). */
 const char* lt2_last_cuda_error_string(void);
 
-/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH (library bookkeeping). */
 int lt2_gdr_version(void);
 
 #ifdef __cplusplus

@@ -43,10 +43,10 @@ def test_exports_every_declared_symbol(L):
 def test_status_strings(L):
     for code, name in [(0, "LT2_OK"), (1, "LT2_ERR_INVALID_ARGUMENT"), (2, "LT2_ERR_UNSUPPORTED"),
                        (3, "LT2_ERR_WORKSPACE"), (4, "LT2_ERR_CUDA"),
-                       (5, "LT2_ERR_DEVICE_TIMEOUT")]:
+                       (5, "LT2_ERR_DEVICE_TIMEOUT"), (6, "LT2_ERR_RANGE")]:
         assert lt2.lt2_status_string(code) == name
     assert lt2.lt2_status_string(99) == "LT2_STATUS_UNKNOWN"
-    assert L.lt2_gdr_version() >= 100
+    assert L.lt2_gdr_version() >= 200
 
 
 def test_dims_struct_layout():

@@ -15,8 +15,12 @@ pytestmark = pytest.mark.gpu
 
 
 def _units(w, n, seed):
+    """The first and last head-units, one unit of every loop (each loop is its own launch, and
+    the later launches run on the second wave of CTAs), then random units up to n."""
     rng = np.random.default_rng(seed)
     picks = {(w.T - 1, w.B - 1, w.H - 1), (0, 0, 0)}
+    for tau in range(w.T):
+        picks.add((tau, int(rng.integers(w.B)), int(rng.integers(w.H))))
     while len(picks) < n:
         picks.add((int(rng.integers(w.T)), int(rng.integers(w.B)), int(rng.integers(w.H))))
     return sorted(picks)
