@@ -350,60 +350,67 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // ================= gates (warp 1), conversion of K / Q / V (warps 1 / 2 / 3), Gram ===
         uint32_t gram_issuer = 0;
         int gram_issued = 0;
+        // warp 1: alpha and beta of the next chunk are loaded one chunk ahead, so the latency of
+        // the global loads hides behind this chunk's gates, conversion and Gram issue
+        float a_nx[2] = {1.f, 1.f}, b_nx[2] = {0.f, 0.f};
+        auto load_gate_inputs = [&](int cn) {
+            #pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int64_t tok = static_cast<int64_t>(cn) * kC + lane + 32 * i;
+                const bool valid = cn < nchunks && tok < L;
+                a_nx[i] = valid ? p.alpha[ug * L + tok] : 1.f;
+                b_nx[i] = valid ? p.beta[ug * L + tok] : 0.f;
+            }
+        };
+        if (warp == 1) load_gate_inputs(0);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;
             const uint32_t ph = (c / kStages) & 1;
             if (warp == 1) {
                 if (!mbar_wait(bar_addr(sb, B_GATE_EMPTY + s), ph ^ 1, abort_flag, err, kTimeoutNs)) break;
                 Gates* gs = gate(s);
-                const int64_t t0 = static_cast<int64_t>(c) * kC;
-                float g[2], b[2];
-                uint32_t negs[2];
-                #pragma unroll
+                const float a_cur[2] = {a_nx[0], a_nx[1]}, b_cur[2] = {b_nx[0], b_nx[1]};
+                load_gate_inputs(c + 1);
+                // alpha = |alpha| * sign: the magnitudes go through log-domain prefix sums, the
+                // signs through a parity count of the negatives (alpha = 0 is taken as 1e-30, a
+                // reset to within 1e-30 of the state).  Pass 1, one row of 32 tokens at a time:
+                // G_r and the sign of the product up to r (kept in gam[r] for pass 2).
+                float carry = 0.f;
+                uint32_t negs_before = 0;
+                bool in_range = true;                   // every |G_r| < 80
+                #pragma unroll 1
                 for (int i = 0; i < 2; ++i) {
-                    const int64_t tok = t0 + lane + 32 * i;
-                    const bool valid = tok < L;
-                    const float a = valid ? p.alpha[ug * L + tok] : 1.f;
-                    b[i] = valid ? p.beta[ug * L + tok] : 0.f;
-                    // alpha = |alpha| * sign: the magnitudes go through the log-domain prefix
-                    // sums, the signs through a parity count (alpha = 0 is taken as 1e-30, a
-                    // reset to within 1e-30 of the state)
-                    g[i] = __logf(fmaxf(fabsf(a), 1e-30f));
-                    negs[i] = __ballot_sync(0xffffffffu, a < 0.f);
-                }
-                // inclusive prefix sums over the 64 tokens
-                #pragma unroll
-                for (int i = 0; i < 2; ++i) {
+                    const float a = i ? a_cur[1] : a_cur[0];
+                    float g = __logf(fmaxf(fabsf(a), 1e-30f));
                     #pragma unroll
                     for (int off = 1; off < 32; off <<= 1) {
-                        const float y = __shfl_up_sync(0xffffffffu, g[i], off);
-                        if (lane >= off) g[i] += y;
+                        const float y = __shfl_up_sync(0xffffffffu, g, off);
+                        if (lane >= off) g += y;
                     }
-                }
-                g[1] += __shfl_sync(0xffffffffu, g[0], 31);
-                const float GC = __shfl_sync(0xffffffffu, g[1], 31);
-                // the factored decay e^{G_r} e^{-G_s} needs both factors representable
-                float gmin = fminf(g[0], g[1]), gmax = fmaxf(g[0], g[1]);
-                #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) {
-                    gmin = fminf(gmin, __shfl_xor_sync(0xffffffffu, gmin, off));
-                    gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, off));
-                }
-                const bool safe = gmin > -80.f && gmax < 80.f;
-                // sign of the product of the alphas up to token r: parity of the negatives
-                const uint32_t upto = 0xffffffffu >> (31 - lane);
-                const float sgn[2] = {(__popc(negs[0] & upto) & 1) ? -1.f : 1.f,
-                                      ((__popc(negs[0]) + __popc(negs[1] & upto)) & 1) ? -1.f : 1.f};
-                const float sgnC = ((__popc(negs[0]) + __popc(negs[1])) & 1) ? -1.f : 1.f;
-                #pragma unroll
-                for (int i = 0; i < 2; ++i) {
+                    g += carry;
+                    carry = __shfl_sync(0xffffffffu, g, 31);
+                    const uint32_t neg = __ballot_sync(0xffffffffu, a < 0.f);
+                    const uint32_t upto = 0xffffffffu >> (31 - lane);
                     const int r = lane + 32 * i;
-                    gs->G[r] = g[i];
-                    // the sign of gam[r] (also kept by a zero) is the sign of the product
-                    gs->gam[r] = sgn[i] * __expf(g[i]);
-                    gs->bein[r] = safe ? sgn[i] * b[i] * __expf(-g[i]) : 0.f;
-                    gs->beta[r] = b[i];
-                    gs->bgc[r] = sgnC * sgn[i] * b[i] * __expf(GC - g[i]);
+                    gs->G[r] = g;
+                    gs->gam[r] = ((negs_before + __popc(neg & upto)) & 1) ? -1.f : 1.f;
+                    gs->beta[r] = i ? b_cur[1] : b_cur[0];
+                    negs_before += __popc(neg);
+                    in_range &= fabsf(g) < 80.f;
+                }
+                // the factored decay e^{G_r} e^{-G_s} needs both factors representable
+                const bool safe = __all_sync(0xffffffffu, in_range);
+                const float GC = carry;
+                const float sgnC = (negs_before & 1) ? -1.f : 1.f;
+                __syncwarp();
+                // pass 2: the decay factors (the sign of gam[r], kept by a zero, is the sign of
+                // the product of the alphas up to token r)
+                #pragma unroll 1
+                for (int r = lane; r < kC; r += 32) {
+                    const float g = gs->G[r], sg = gs->gam[r], bb = gs->beta[r];
+                    gs->gam[r] = sg * __expf(g);
+                    gs->bein[r] = safe ? sg * bb * __expf(-g) : 0.f;
+                    gs->bgc[r] = sgnC * sg * bb * __expf(GC - g);
                 }
                 if (lane == 0) {
                     gs->gC = sgnC * __expf(GC);
