@@ -22,6 +22,7 @@ LT2_ERR_WORKSPACE = 3
 LT2_ERR_CUDA = 4
 LT2_ERR_DEVICE_TIMEOUT = 5
 LT2_ERR_RANGE = 6
+LT2_ERR_DEVICE_CHECK = 7
 
 LT2_DTYPE_F32 = 0
 LT2_DTYPE_BF16 = 1
@@ -74,26 +75,38 @@ def lib():
             raise ImportError(
                 f"{LIB_PATH} is missing: build it with "
                 "`python -m gated_delta_rule_looped_b200.build` (no fallback exists)")
-        L = ctypes.CDLL(LIB_PATH)
-        vp, fp = ctypes.c_void_p, ctypes.c_void_p
-        dims_p = ctypes.POINTER(lt2_gdr_dims)
-        L.lt2_gdr_prefill_workspace_bytes.argtypes = [dims_p]
-        L.lt2_gdr_prefill_workspace_bytes.restype = ctypes.c_size_t
-        L.lt2_gdr_prefill.argtypes = [dims_p, vp, vp, vp, fp, fp, fp, vp, fp, vp,
-                                      ctypes.c_size_t, vp]
-        L.lt2_gdr_prefill.restype = ctypes.c_int
-        L.lt2_gdr_decode.argtypes = [dims_p, vp, vp, vp, fp, fp, fp, vp, vp]
-        L.lt2_gdr_decode.restype = ctypes.c_int
-        L.lt2_gdr_last_device_error.argtypes = []
-        L.lt2_gdr_last_device_error.restype = ctypes.c_int
-        L.lt2_status_string.argtypes = [ctypes.c_int]
-        L.lt2_status_string.restype = ctypes.c_char_p
-        L.lt2_last_cuda_error_string.argtypes = []
-        L.lt2_last_cuda_error_string.restype = ctypes.c_char_p
-        L.lt2_gdr_version.argtypes = []
-        L.lt2_gdr_version.restype = ctypes.c_int
-        _LIB = L
+        _LIB = load_library(LIB_PATH)
     return _LIB
+
+
+def load_library(path):
+    """A build of the library at ``path`` with the argument types of include/lt2_gdr.h declared
+    (the tests load the debug build, liblt2gdr_debug.so, this way; it also declares the hooks of
+    include/lt2_gdr_debug.h when the build exports them)."""
+    L = ctypes.CDLL(path)
+    vp, fp = ctypes.c_void_p, ctypes.c_void_p
+    dims_p = ctypes.POINTER(lt2_gdr_dims)
+    L.lt2_gdr_prefill_workspace_bytes.argtypes = [dims_p]
+    L.lt2_gdr_prefill_workspace_bytes.restype = ctypes.c_size_t
+    L.lt2_gdr_prefill.argtypes = [dims_p, vp, vp, vp, fp, fp, fp, vp, fp, vp,
+                                  ctypes.c_size_t, vp]
+    L.lt2_gdr_prefill.restype = ctypes.c_int
+    L.lt2_gdr_decode.argtypes = [dims_p, vp, vp, vp, fp, fp, fp, vp, vp]
+    L.lt2_gdr_decode.restype = ctypes.c_int
+    L.lt2_gdr_last_device_error.argtypes = []
+    L.lt2_gdr_last_device_error.restype = ctypes.c_int
+    L.lt2_status_string.argtypes = [ctypes.c_int]
+    L.lt2_status_string.restype = ctypes.c_char_p
+    L.lt2_last_cuda_error_string.argtypes = []
+    L.lt2_last_cuda_error_string.restype = ctypes.c_char_p
+    L.lt2_gdr_version.argtypes = []
+    L.lt2_gdr_version.restype = ctypes.c_int
+    if hasattr(L, "lt2_debug_set_skip_chunk"):
+        L.lt2_debug_set_skip_chunk.argtypes = [ctypes.c_int, ctypes.c_int]
+        L.lt2_debug_set_skip_chunk.restype = ctypes.c_int
+        L.lt2_debug_wait_timeout_ns.argtypes = []
+        L.lt2_debug_wait_timeout_ns.restype = ctypes.c_uint64
+    return L
 
 
 def make_dims(T, B, H, L, dk, dv, dtype=LT2_DTYPE_BF16, gate=LT2_GATE_SCALAR,

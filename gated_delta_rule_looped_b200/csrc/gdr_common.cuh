@@ -9,12 +9,26 @@ namespace lt2 {
 
 // Device-side status word (bit flags, see lt2_gdr_last_device_error): a bounded wait ran
 // out; a tensor-core path produced a non-finite output or state (its fp16 operands out of
-// range, or non-finite inputs).
+// range, or non-finite inputs); a debug build's index check failed.
 enum : unsigned int {
     kDevOk = 0u,
     kDevTimeout = 1u,
     kDevRange = 2u,
+    kDevCheck = 4u,
 };
+
+// Device-side invariant checks of the debug build (LT2_DEBUG): a failed check records kDevCheck
+// in the status word and yields false, so that the caller skips the access; nothing traps.  In
+// the product build the check compiles to `true`.
+#ifdef LT2_DEBUG
+__device__ __forceinline__ bool dbg_ok(bool cond, unsigned int* err)
+{
+    if (!cond) atomicOr(err, kDevCheck);
+    return cond;
+}
+#else
+__device__ __forceinline__ constexpr bool dbg_ok(bool, unsigned int*) { return true; }
+#endif
 
 // Per-launch view of one loop's slice: base pointers already offset to loop tau.
 struct LoopSlice {

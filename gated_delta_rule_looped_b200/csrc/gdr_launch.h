@@ -38,4 +38,10 @@ cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream);
 bool prefill_kda_tc_supports(int dtype_bf16, int dk, int dv);
 cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream);
 
+#ifdef LT2_DEBUG
+// Fault injection of the debug build: the producer of every later launch stops before `chunk`.
+cudaError_t debug_set_skip_chunk_scalar(int chunk);
+cudaError_t debug_set_skip_chunk_per_key(int chunk);
+#endif
+
 }  // namespace lt2

@@ -180,9 +180,16 @@ struct Params {
     float* S_out;              // nullable
     int64_t L;
     int unit0;
+    int units_total;           // T*B*H (the extent of the tensor maps' unit axis)
     int out_bf16;
     unsigned int* err;
 };
+
+#ifdef LT2_DEBUG
+// Fault injection of the debug build: the producer stops before this chunk (-1: never), so its
+// copies never arrive and the waits for them run out.
+__device__ int g_debug_skip_chunk = -1;
+#endif
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t base, uint32_t i) { return base + OFF_BAR + 8u * i; }
 
@@ -663,11 +670,16 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + OFF_TMEM_SLOT);
+    // every TMEM column this CTA addresses lies inside its allocation
+    if (threadIdx.x == 0) dbg_ok((tmem & 0xFFFFu) + TM_COLS <= 512u && (tmem >> 16) == 0u, err);
 
     if (warp == 0) {
         // ================= TMA producer =================
         int issued = 0;
         for (int c = 0; c < nchunks; ++c) {
+#ifdef LT2_DEBUG
+            if (c == g_debug_skip_chunk) break;
+#endif
             const int s = c % kStages;
             const uint32_t ph = ((c / kStages) & 1) ^ 1;
             int free_ok = 0;
@@ -676,7 +688,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                           mbar_wait(bar_addr(sb, B_AL_EMPTY + (c & 1)), ((c >> 1) & 1) ^ 1, abort_flag, err, kTimeoutNs);
             if (!__shfl_sync(0xffffffffu, free_ok, 0)) break;
             uint32_t leader;
-            if (elect_one(leader)) {
+            if (elect_one(leader) && dbg_ok(c * kC < L && ug < p.units_total, err)) {
                 const uint32_t fb = bar_addr(sb, B_FULL + s);
                 mbar_arrive_expect_tx(fb, STAGE_TX);
                 const uint32_t st = sb + OFF_STG + s * STAGE_BYTES;
@@ -923,7 +935,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 ph_s ^= 1u;
                 if (!ok) break;
                 tc_fence_after();
-                if (leader && p.out_bf16) {
+                if (leader && p.out_bf16 && dbg_ok(t0 < L && ug < p.units_total, err)) {
                     tma_store_3d(&tm_o, sb + OFF_OST, 0, static_cast<int32_t>(t0), ug);
                     tma_store_3d(&tm_o, sb + OFF_OST + 4096, 64, static_cast<int32_t>(t0), ug);
                     bulk_commit_group();
@@ -1016,6 +1028,7 @@ cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream)
         p.S_out = call.S_out;
         p.L = call.L;
         p.unit0 = static_cast<int>(tau * call.units_per_loop);
+        p.units_total = static_cast<int>(units);
         p.out_bf16 = call.out_bf16;
         p.err = call.err;
         cudaLaunchConfig_t cfg = {};
@@ -1035,3 +1048,12 @@ cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream)
 }
 
 }  // namespace lt2
+
+#ifdef LT2_DEBUG
+namespace lt2 {
+cudaError_t debug_set_skip_chunk_per_key(int chunk)
+{
+    return cudaMemcpyToSymbol(kda::g_debug_skip_chunk, &chunk, sizeof(chunk));
+}
+}  // namespace lt2
+#endif

@@ -150,9 +150,16 @@ struct Params {
     float* S_out;          // nullable
     int64_t L;
     int unit0;             // first unit of this loop in the flattened [T*B*H] order
+    int units_total;       // T*B*H (the extent of the tensor maps' unit axis)
     int out_bf16;
     unsigned int* err;
 };
+
+#ifdef LT2_DEBUG
+// Fault injection of the debug build: the producer stops before this chunk (-1: never), so its
+// copies never arrive and the waits for them run out.
+__device__ int g_debug_skip_chunk = -1;
+#endif
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t base, uint32_t i) { return base + OFF_BAR + 8u * i; }
 
@@ -315,18 +322,23 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + OFF_TMEM_SLOT);
+    // every TMEM column this CTA addresses lies inside its allocation
+    if (threadIdx.x == 0) dbg_ok((tmem & 0xFFFFu) + TM_COLS <= 512u && (tmem >> 16) == 0u, err);
 
     if (warp == 0) {
         // ================= TMA producer =================
         int issued = 0;
         for (int c = 0; c < nchunks; ++c) {
+#ifdef LT2_DEBUG
+            if (c == g_debug_skip_chunk) break;
+#endif
             const int s = c % kStages;
             const uint32_t ph = ((c / kStages) & 1) ^ 1;
             int free_ok = 0;
             if (lane == 0) free_ok = mbar_wait(bar_addr(sb, B_EMPTY + s), ph, abort_flag, err, kTimeoutNs);
             if (!__shfl_sync(0xffffffffu, free_ok, 0)) break;
             uint32_t leader;
-            if (elect_one(leader)) {
+            if (elect_one(leader) && dbg_ok(c * kC < L && ug < p.units_total, err)) {
                 const uint32_t fb = bar_addr(sb, B_FULL + s);
                 mbar_arrive_expect_tx(fb, STAGE_BYTES);
                 const uint32_t st = sb + OFF_KQV + s * STAGE_BYTES;
@@ -427,7 +439,8 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             for (int panel = 0; panel < 2; ++panel) {
                 const uint32_t src = warp == 3 ? st + KQ_BYTES + panel * 8192
                                                : st + (warp - 1) * 8192 + panel * 16384;
-                convert_tile(src, 512, lane, lds, sts);
+                if (dbg_ok(src >= sb + OFF_KQV && src + 8192 <= sb + OFF_KQV + kStages * STAGE_BYTES, err))
+                    convert_tile(src, 512, lane, lds, sts);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -475,6 +488,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const float gr = gs->gam[r];
             const bool safe = gs->safe != 0;
             const uint32_t dst = is_a ? as : ps;
+            dbg_ok(dst >= sb + OFF_AS && dst + 8192 <= sb + OFF_ADIAG && r < kC, err);
             if (safe) {
                 // A is kept negated (the solve only accumulates).  Entries on or above the
                 // diagonal (s >= r in A, s > r in P) are never read, apart from the diagonal P
@@ -739,8 +753,10 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (j == 0) {
                 mbar_arrive(bar_addr(sb, B_O_DONE));
                 mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
-                tma_store_3d(&tm_o, sb + OFF_OST, 0, static_cast<int32_t>(t0), ug);
-                tma_store_3d(&tm_o, sb + OFF_OST + 8192, 64, static_cast<int32_t>(t0), ug);
+                if (dbg_ok(t0 < L && ug < p.units_total, err)) {
+                    tma_store_3d(&tm_o, sb + OFF_OST, 0, static_cast<int32_t>(t0), ug);
+                    tma_store_3d(&tm_o, sb + OFF_OST + 8192, 64, static_cast<int32_t>(t0), ug);
+                }
                 bulk_commit_group();
             }
         }
@@ -792,6 +808,7 @@ cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
         p.S_out = call.S_out;
         p.L = call.L;
         p.unit0 = static_cast<int>(tau * call.units_per_loop);
+        p.units_total = static_cast<int>(units);
         p.out_bf16 = call.out_bf16;
         p.err = call.err;
         cudaLaunchConfig_t cfg = {};
@@ -812,3 +829,12 @@ cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
 }
 
 }  // namespace lt2
+
+#ifdef LT2_DEBUG
+namespace lt2 {
+cudaError_t debug_set_skip_chunk_scalar(int chunk)
+{
+    return cudaMemcpyToSymbol(tc::g_debug_skip_chunk, &chunk, sizeof(chunk));
+}
+}  // namespace lt2
+#endif

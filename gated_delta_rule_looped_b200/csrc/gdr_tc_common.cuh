@@ -16,7 +16,12 @@ namespace tcc {
 using namespace sm100;
 
 constexpr int kD = 128;                          // d_k = d_v
-constexpr uint64_t kWaitTimeoutNs = 4000000000ull;   // bound of every mbarrier wait (4 s)
+// Bound of every mbarrier wait: 4 s in the product build; the debug build (LT2_DEBUG) shortens it
+// so that its fault-injection test ends in milliseconds.
+#ifndef LT2_WAIT_TIMEOUT_NS
+#define LT2_WAIT_TIMEOUT_NS 4000000000ull
+#endif
+constexpr uint64_t kWaitTimeoutNs = LT2_WAIT_TIMEOUT_NS;
 constexpr int kAdiagRow = 17;                    // fp32 diagonal blocks: rows padded to 17
 
 __device__ __forceinline__ void named_sync(int id, int nthreads)

@@ -340,6 +340,7 @@ lt2_status lt2_gdr_last_device_error(void)
     if (e != cudaSuccess) return cuda_fail(e, "read device status");
     if (h & lt2::kDevTimeout) return LT2_ERR_DEVICE_TIMEOUT;
     if (h & lt2::kDevRange) return LT2_ERR_RANGE;
+    if (h & lt2::kDevCheck) return LT2_ERR_DEVICE_CHECK;
     return LT2_OK;
 }
 
@@ -353,6 +354,7 @@ const char* lt2_status_string(lt2_status s)
         case LT2_ERR_CUDA: return "LT2_ERR_CUDA";
         case LT2_ERR_DEVICE_TIMEOUT: return "LT2_ERR_DEVICE_TIMEOUT";
         case LT2_ERR_RANGE: return "LT2_ERR_RANGE";
+        case LT2_ERR_DEVICE_CHECK: return "LT2_ERR_DEVICE_CHECK";
     }
     return "LT2_STATUS_UNKNOWN";
 }
@@ -362,3 +364,27 @@ const char* lt2_last_cuda_error_string(void) { return t_cuda_error; }
 int lt2_gdr_version(void) { return 200; }
 
 }  // extern "C"
+
+#ifdef LT2_DEBUG
+#include "lt2_gdr_debug.h"
+#include "gdr_tc_common.cuh"
+
+extern "C" {
+
+lt2_status lt2_debug_set_skip_chunk(int kernel, int chunk)
+{
+    if (chunk < -1) return LT2_ERR_INVALID_ARGUMENT;
+    cudaError_t e;
+    if (kernel == LT2_DEBUG_SCALAR_TC)
+        e = lt2::debug_set_skip_chunk_scalar(chunk);
+    else if (kernel == LT2_DEBUG_PER_KEY_TC)
+        e = lt2::debug_set_skip_chunk_per_key(chunk);
+    else
+        return LT2_ERR_INVALID_ARGUMENT;
+    return e == cudaSuccess ? LT2_OK : cuda_fail(e, "lt2_debug_set_skip_chunk");
+}
+
+uint64_t lt2_debug_wait_timeout_ns(void) { return lt2::tcc::kWaitTimeoutNs; }
+
+}  // extern "C"
+#endif

@@ -76,7 +76,8 @@ typedef enum lt2_status {
     LT2_ERR_WORKSPACE = 3,        /* workspace smaller than lt2_gdr_prefill_workspace_bytes */
     LT2_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed                   */
     LT2_ERR_DEVICE_TIMEOUT = 5,   /* a bounded in-kernel wait ran out (see header comment)  */
-    LT2_ERR_RANGE = 6             /* a tensor-core path produced non-finite results         */
+    LT2_ERR_RANGE = 6,            /* a tensor-core path produced non-finite results         */
+    LT2_ERR_DEVICE_CHECK = 7      /* a debug build's device-side check failed (lt2_gdr_debug.h) */
 } lt2_status;
 
 typedef enum lt2_dtype { LT2_DTYPE_F32 = 0, LT2_DTYPE_BF16 = 1 } lt2_dtype;
@@ -174,7 +175,9 @@ lt2_status lt2_gdr_decode(const lt2_gdr_dims* dims,
  * library's own failure reporting).  Synchronises the device (every stream), then reads and
  * clears the word in one atomic exchange.  Returns LT2_ERR_DEVICE_TIMEOUT if a kernel gave up
  * on a bounded wait since the last read, else LT2_ERR_RANGE if a tensor-core prefill produced
- * non-finite results, else LT2_OK; LT2_ERR_CUDA if the synchronisation or the read failed.
+ * non-finite results, else LT2_ERR_DEVICE_CHECK if a device-side check of the debug build failed
+ * (never in the product build), else LT2_OK; LT2_ERR_CUDA if the synchronisation or the read
+ * failed.
  * The word is shared by every call on the device, from any thread or stream: a flag belongs
  * to whichever work ran since the previous read.
  */

@@ -21,15 +21,15 @@ def L():
     return lt2.lib()
 
 
-def _declared_functions():
-    names = set()
-    for fn in os.listdir(HEADER_DIR):
-        if fn.endswith(".h"):
-            with open(os.path.join(HEADER_DIR, fn)) as f:
-                text = f.read()
-            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-            names |= set(re.findall(r"\b(lt2_\w+)\s*\(", text))
-    return names
+def _declared_functions(header="lt2_gdr.h"):
+    with open(os.path.join(HEADER_DIR, header)) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return set(re.findall(r"\b(lt2_\w+)\s*\(", text))
+
+
+def test_headers_are_the_product_and_the_debug_header():
+    assert sorted(f for f in os.listdir(HEADER_DIR) if f.endswith(".h")) == ["lt2_gdr.h", "lt2_gdr_debug.h"]
 
 
 def test_exports_every_declared_symbol(L):
@@ -40,10 +40,26 @@ def test_exports_every_declared_symbol(L):
         assert hasattr(L, name), f"{name} not exported"
 
 
+def test_debug_library_exports_both_headers_and_product_only_its_own():
+    if lbuild.needs_build(debug=True):
+        lbuild.build(debug=True)
+    D = ctypes.CDLL(lbuild.DEBUG_LIB)
+    debug_only = _declared_functions("lt2_gdr_debug.h")
+    assert debug_only == {"lt2_debug_set_skip_chunk", "lt2_debug_wait_timeout_ns"}
+    for name in _declared_functions() | debug_only:
+        assert hasattr(D, name), f"{name} not exported by the debug library"
+    P = ctypes.CDLL(lbuild.LIB)
+    for name in debug_only:
+        assert not hasattr(P, name), f"the product library exports the test hook {name}"
+    D.lt2_debug_wait_timeout_ns.restype = ctypes.c_uint64
+    assert 0 < D.lt2_debug_wait_timeout_ns() <= 100_000_000     # milliseconds, not seconds
+
+
 def test_status_strings(L):
     for code, name in [(0, "LT2_OK"), (1, "LT2_ERR_INVALID_ARGUMENT"), (2, "LT2_ERR_UNSUPPORTED"),
                        (3, "LT2_ERR_WORKSPACE"), (4, "LT2_ERR_CUDA"),
-                       (5, "LT2_ERR_DEVICE_TIMEOUT"), (6, "LT2_ERR_RANGE")]:
+                       (5, "LT2_ERR_DEVICE_TIMEOUT"), (6, "LT2_ERR_RANGE"),
+                       (7, "LT2_ERR_DEVICE_CHECK")]:
         assert lt2.lt2_status_string(code) == name
     assert lt2.lt2_status_string(99) == "LT2_STATUS_UNKNOWN"
     assert L.lt2_gdr_version() >= 200
