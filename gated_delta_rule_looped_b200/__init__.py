@@ -40,7 +40,9 @@ LT2_OUT_BF16 = 2
 EXPORTS = (
     "lt2_gdr_prefill_workspace_bytes",
     "lt2_gdr_prefill",
+    "lt2_gdr_prefill_fused",
     "lt2_gdr_decode",
+    "lt2_gdr_decode_fused",
     "lt2_gdr_last_device_error",
     "lt2_status_string",
     "lt2_last_cuda_error_string",
@@ -53,6 +55,18 @@ class lt2_gdr_dims(ctypes.Structure):
                 ("L", ctypes.c_int64), ("dk", ctypes.c_int64), ("dv", ctypes.c_int64),
                 ("dtype", ctypes.c_int32), ("gate", ctypes.c_int32), ("algo", ctypes.c_int32),
                 ("out_dtype", ctypes.c_int32)]
+
+
+class lt2_gdr_fused(ctypes.Structure):
+    """The fused prologue and output gate (include/lt2_gdr.h); all zero selects none."""
+    _fields_ = [("qk_l2norm", ctypes.c_int32), ("gate_logits", ctypes.c_int32),
+                ("alpha_scale", ctypes.c_float), ("reserved", ctypes.c_int32),
+                ("z", ctypes.c_void_p)]
+
+
+def make_fused(qk_l2norm=False, gate_logits=False, alpha_scale=1.0, z=None):
+    """An lt2_gdr_fused; ``z`` is a tensor (its data pointer is taken), an address or None."""
+    return lt2_gdr_fused(int(bool(qk_l2norm)), int(bool(gate_logits)), float(alpha_scale), 0, _p(z))
 
 
 class Lt2Error(RuntimeError):
@@ -82,7 +96,8 @@ def lib():
 def load_library(path):
     """A build of the library at ``path`` with the argument types of include/lt2_gdr.h declared
     (the tests load the debug build, liblt2gdr_debug.so, this way; it also declares the hooks of
-    include/lt2_gdr_debug.h when the build exports them)."""
+    include/lt2_gdr_debug.h when the build exports them, and loads builds that predate the fused
+    entry points)."""
     L = ctypes.CDLL(path)
     vp, fp = ctypes.c_void_p, ctypes.c_void_p
     dims_p = ctypes.POINTER(lt2_gdr_dims)
@@ -93,6 +108,13 @@ def load_library(path):
     L.lt2_gdr_prefill.restype = ctypes.c_int
     L.lt2_gdr_decode.argtypes = [dims_p, vp, vp, vp, fp, fp, fp, vp, vp]
     L.lt2_gdr_decode.restype = ctypes.c_int
+    if hasattr(L, "lt2_gdr_prefill_fused"):
+        fused_p = ctypes.POINTER(lt2_gdr_fused)
+        L.lt2_gdr_prefill_fused.argtypes = [dims_p, fused_p, vp, vp, vp, fp, fp, fp, vp, fp, vp,
+                                            ctypes.c_size_t, vp]
+        L.lt2_gdr_prefill_fused.restype = ctypes.c_int
+        L.lt2_gdr_decode_fused.argtypes = [dims_p, fused_p, vp, vp, vp, fp, fp, fp, vp, vp]
+        L.lt2_gdr_decode_fused.restype = ctypes.c_int
     L.lt2_gdr_last_device_error.argtypes = []
     L.lt2_gdr_last_device_error.restype = ctypes.c_int
     L.lt2_status_string.argtypes = [ctypes.c_int]
@@ -148,6 +170,19 @@ def lt2_gdr_prefill(dims, q, k, v, alpha, beta, S0, o, S_out, workspace=None,
 def lt2_gdr_decode(dims, q, k, v, alpha, beta, S, o, stream=None):
     return lib().lt2_gdr_decode(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(alpha), _p(beta),
                                 _p(S), _p(o), _stream(stream))
+
+
+def lt2_gdr_prefill_fused(dims, fused, q, k, v, alpha, beta, S0, o, S_out, workspace=None,
+                          workspace_bytes=0, stream=None):
+    return lib().lt2_gdr_prefill_fused(ctypes.byref(dims), None if fused is None else ctypes.byref(fused),
+                                       _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(o),
+                                       _p(S_out), _p(workspace), int(workspace_bytes), _stream(stream))
+
+
+def lt2_gdr_decode_fused(dims, fused, q, k, v, alpha, beta, S, o, stream=None):
+    return lib().lt2_gdr_decode_fused(ctypes.byref(dims), None if fused is None else ctypes.byref(fused),
+                                      _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S), _p(o),
+                                      _stream(stream))
 
 
 def lt2_gdr_last_device_error():
@@ -237,22 +272,28 @@ def _check_call(q, k, v, alpha, beta, states, o, per_key, out):
 
 
 def prefill(q, k, v, alpha, beta, S0=None, per_key=None, algo=LT2_ALGO_AUTO, o=None,
-            S_out=None, out=None, stream=None, order="delta_first"):
+            S_out=None, out=None, stream=None, order="delta_first", qk_l2norm=False,
+            gate_logits=False, alpha_scale=1.0, z=None):
     """Run the looped prefill on CUDA tensors; returns (o, S_out).  ``out`` selects the
     storage type of o: None/"same" (as the inputs), "f32" or "bf16"; ``order`` the order of
-    the per-key factors ("delta_first" as printed, or "decay_first").  The call runs on the
-    tensors' device (made current for its duration), on ``stream`` or that device's current
-    stream."""
+    the per-key factors ("delta_first" as printed, or "decay_first").  ``qk_l2norm``,
+    ``gate_logits``/``alpha_scale`` and ``z`` select the fused prologue and output gate
+    (lt2_gdr_prefill_fused).  The call runs on the tensors' device (made current for its
+    duration), on ``stream`` or that device's current stream."""
     import torch
     _require_cuda(q)
+    fused = None
+    if qk_l2norm or gate_logits or z is not None:
+        fused = make_fused(qk_l2norm, gate_logits, alpha_scale, z)
     with torch.cuda.device(q.device):
-        return _prefill(q, k, v, alpha, beta, S0, per_key, algo, o, S_out, out, stream, order)
+        return _prefill(q, k, v, alpha, beta, S0, per_key, algo, o, S_out, out, stream, order, fused, z)
 
 
-def _prefill(q, k, v, alpha, beta, S0, per_key, algo, o, S_out, out, stream, order):
+def _prefill(q, k, v, alpha, beta, S0, per_key, algo, o, S_out, out, stream, order, fused=None, z=None):
     import torch
     dims = _dims_from(q, v, alpha, per_key, algo, out, order)
     _check_call(q, k, v, alpha, beta, [("S0", S0), ("S_out", S_out)], o, dims.gate != LT2_GATE_SCALAR, out)
+    _check("z", z, v.shape, q.dtype, q.device)
     if o is None:
         o = torch.empty(v.shape, dtype=_out_torch_dtype(q.dtype, out), device=v.device)
     if S_out is None:
@@ -260,22 +301,30 @@ def _prefill(q, k, v, alpha, beta, S0, per_key, algo, o, S_out, out, stream, ord
                             dtype=torch.float32, device=q.device)
     ws_bytes = lt2_gdr_prefill_workspace_bytes(dims)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device) if ws_bytes else None
-    st = lt2_gdr_prefill(dims, q, k, v, alpha, beta, S0, o, S_out, ws, ws_bytes, stream)
+    if fused is None:
+        st = lt2_gdr_prefill(dims, q, k, v, alpha, beta, S0, o, S_out, ws, ws_bytes, stream)
+    else:
+        st = lt2_gdr_prefill_fused(dims, fused, q, k, v, alpha, beta, S0, o, S_out, ws, ws_bytes, stream)
     if st != LT2_OK:
         raise Lt2Error(st, "lt2_gdr_prefill")
     return o, S_out
 
 
-def decode(q, k, v, alpha, beta, S, per_key=None, o=None, out=None, stream=None, order="delta_first"):
-    """One decode token per (loop, batch, head); q/k/v [T,B,H,d]; S updated in place.  Runs
-    on the tensors' device (made current for the call)."""
+def decode(q, k, v, alpha, beta, S, per_key=None, o=None, out=None, stream=None, order="delta_first",
+           qk_l2norm=False, gate_logits=False, alpha_scale=1.0, z=None):
+    """One decode token per (loop, batch, head); q/k/v [T,B,H,d]; S updated in place.  The
+    fused prologue and output gate as in ``prefill``.  Runs on the tensors' device (made
+    current for the call)."""
     import torch
     _require_cuda(q)
+    fused = None
+    if qk_l2norm or gate_logits or z is not None:
+        fused = make_fused(qk_l2norm, gate_logits, alpha_scale, z)
     with torch.cuda.device(q.device):
-        return _decode(q, k, v, alpha, beta, S, per_key, o, out, stream, order)
+        return _decode(q, k, v, alpha, beta, S, per_key, o, out, stream, order, fused, z)
 
 
-def _decode(q, k, v, alpha, beta, S, per_key, o, out, stream, order):
+def _decode(q, k, v, alpha, beta, S, per_key, o, out, stream, order, fused=None, z=None):
     import torch
     per_key = (alpha.dim() == 4) if per_key is None else per_key
     T, B, H, dk = q.shape
@@ -283,9 +332,13 @@ def _decode(q, k, v, alpha, beta, S, per_key, o, out, stream, order):
     dt = {torch.float32: LT2_DTYPE_F32, torch.bfloat16: LT2_DTYPE_BF16}[q.dtype]
     dims = make_dims(T, B, H, 1, dk, dv, dt, _gate(per_key, order), out_dtype=_OUT[out])
     _check_call(q, k, v, alpha, beta, [("S", S)], o, per_key, out)
+    _check("z", z, v.shape, q.dtype, q.device)
     if o is None:
         o = torch.empty(v.shape, dtype=_out_torch_dtype(q.dtype, out), device=v.device)
-    st = lt2_gdr_decode(dims, q, k, v, alpha, beta, S, o, stream)
+    if fused is None:
+        st = lt2_gdr_decode(dims, q, k, v, alpha, beta, S, o, stream)
+    else:
+        st = lt2_gdr_decode_fused(dims, fused, q, k, v, alpha, beta, S, o, stream)
     if st != LT2_OK:
         raise Lt2Error(st, "lt2_gdr_decode")
     return o

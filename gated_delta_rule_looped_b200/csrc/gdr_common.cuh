@@ -48,7 +48,35 @@ struct LoopSlice {
     int decay_first;     // per-key gating applied as (I - beta k k^T) Diag(alpha)
     int out_bf16;        // o stored as bf16 (else fp32)
     unsigned int* err;   // device status word
+    // fused prologue and output gate (all zero: none)
+    int qk_norm;         // q, k raw: normalise every row to unit L2 norm
+    int gate_logits;     // alpha, beta hold logits: alpha = exp(-softplus(a) c), beta = sigmoid(b)
+    float alpha_scale;   // c
+    const void* z;       // output gate logits (layout and dtype of v), or null
 };
+
+// The fused prologue and output gate, in fp32: the same formulas on every path.
+__device__ __forceinline__ float sigmoid_f32(float x) { return 1.f / (1.f + expf(-x)); }
+__device__ __forceinline__ float softplus_f32(float x) { return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))); }
+__device__ __forceinline__ float alpha_from_logit(float a, float c) { return expf(-softplus_f32(a) * c); }
+// 1 / max(sqrt(ss), 1e-12) for a row's sum of squares ss
+__device__ __forceinline__ float inv_l2(float ss) { return 1.f / fmaxf(sqrtf(ss), 1e-12f); }
+// The same three with the hardware approximations (relative errors 2^-11 to 2^-21), for the
+// tensor-core paths, whose operands are fp16 anyway: a short instruction footprint matters
+// more there than the last bits.
+// sigmoid(x) = (1 + tanh(x / 2)) / 2 with the hardware tanh (relative error ~2^-11, below the
+// fp16 operands' own rounding): three instructions
+__device__ __forceinline__ float sigmoid_fast(float x)
+{
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+    return fmaf(0.5f, t, 0.5f);
+}
+__device__ __forceinline__ float alpha_from_logit_fast(float a, float c)
+{
+    return __expf(-(fmaxf(a, 0.f) + __logf(1.f + __expf(-fabsf(a)))) * c);
+}
+__device__ __forceinline__ float inv_l2_fast(float ss) { return rsqrtf(fmaxf(ss, 1e-24f)); }
 
 template <typename T> __device__ __forceinline__ float to_f32(T x);
 template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }

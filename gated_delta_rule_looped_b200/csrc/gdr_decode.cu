@@ -20,13 +20,16 @@
 // [w*dk/8, (w+1)*dk/8); lane c owns columns 4c..4c+3 (one 16-byte access per row), so
 // every warp-wide access touches whole 128-byte lines.  The per-column partial sums are
 // combined across the 8 warps through shared memory; the update is applied in registers
-// and written back with streaming stores.
+// and written back with streaming stores.  The fused prologue (q, k normalised to unit L2
+// norm; alpha, beta from logits) and output gate (o <- sigmoid(z) o) have their own instances.
 #include "gdr_common.cuh"
 #include "gdr_launch.h"
 
 namespace lt2 {
 
-template <typename T, typename To, bool kDecayFirst>
+// kFused: the instance with the fused prologue and output gate (lt2_gdr_fused); the plain
+// instances compile exactly as without them.
+template <typename T, typename To, bool kDecayFirst, bool kFused>
 __global__ void __launch_bounds__(256, 2) gdr_decode_kernel(LoopSlice p, int use_pdl)
 {
     (void)use_pdl;
@@ -48,14 +51,49 @@ __global__ void __launch_bounds__(256, 2) gdr_decode_kernel(LoopSlice p, int use
     const T* q = static_cast<const T*>(p.q) + u * dk;
     const T* k = static_cast<const T*>(p.k) + u * dk;
     const T* v = static_cast<const T*>(p.v) + u * dv;
-    const float beta = p.beta[u];
-    const float a_scalar = p.per_key ? 0.f : p.alpha[u];
+    float beta = p.beta[u];
+    float a_scalar = p.per_key ? 0.f : p.alpha[u];
+    float iq = 1.f, ik = 1.f;          // inverse L2 norms of q and k (fused prologue)
+    if (kFused) {
+        if (p.gate_logits) {
+            beta = sigmoid_f32(beta);
+            if (!p.per_key) a_scalar = alpha_from_logit(a_scalar, p.alpha_scale);
+        }
+        if (p.qk_norm) {
+            float nq = 0.f, nk = 0.f;
+            for (int i = threadIdx.x; i < dk; i += blockDim.x) {
+                const float qi = to_f32(q[i]), ki = to_f32(k[i]);
+                nq += qi * qi;
+                nk += ki * ki;
+            }
+            #pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                nq += __shfl_xor_sync(0xffffffffu, nq, off);
+                nk += __shfl_xor_sync(0xffffffffu, nk, off);
+            }
+            if (lane == 0) {
+                red_e[1][w] = nq;
+                red_f[1][w] = nk;
+            }
+            __syncthreads();
+            nq = 0.f;
+            nk = 0.f;
+            #pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                nq += red_e[1][i];
+                nk += red_f[1][i];
+            }
+            iq = inv_l2(nq);
+            ik = inv_l2(nk);
+        }
+    }
 
     float qk_part = 0.f, aqk_part = 0.f;
     for (int i = threadIdx.x; i < dk; i += blockDim.x) {
-        const float a = p.per_key ? p.alpha[u * dk + i] : a_scalar;
-        const float qi = to_f32(q[i]);
-        const float ki = to_f32(k[i]);
+        float a = p.per_key ? p.alpha[u * dk + i] : a_scalar;
+        if (kFused && p.per_key && p.gate_logits) a = alpha_from_logit(a, p.alpha_scale);
+        const float qi = kFused ? to_f32(q[i]) * iq : to_f32(q[i]);
+        const float ki = kFused ? to_f32(k[i]) * ik : to_f32(k[i]);
         sk[i] = ki;
         sa[i] = a;
         saq[i] = a * qi;
@@ -143,11 +181,33 @@ __global__ void __launch_bounds__(256, 2) gdr_decode_kernel(LoopSlice p, int use
     if (w == 0) {
         const float c1 = beta * (kDecayFirst ? s_qk : s_aqk), c2 = beta * s_qk;
         To* o = static_cast<To*>(p.o) + u * dv + col;
-        o[0] = from_f32<To>(F.x - c1 * E.x + c2 * vv.x);
-        o[1] = from_f32<To>(F.y - c1 * E.y + c2 * vv.y);
-        o[2] = from_f32<To>(F.z - c1 * E.z + c2 * vv.z);
-        o[3] = from_f32<To>(F.w - c1 * E.w + c2 * vv.w);
+        float4 ov = make_float4(F.x - c1 * E.x + c2 * vv.x, F.y - c1 * E.y + c2 * vv.y,
+                                F.z - c1 * E.z + c2 * vv.z, F.w - c1 * E.w + c2 * vv.w);
+        if (kFused && p.z) {            // the fused output gate
+            const T* z = static_cast<const T*>(p.z) + u * dv + col;
+            ov.x *= sigmoid_f32(to_f32(z[0]));
+            ov.y *= sigmoid_f32(to_f32(z[1]));
+            ov.z *= sigmoid_f32(to_f32(z[2]));
+            ov.w *= sigmoid_f32(to_f32(z[3]));
+        }
+        o[0] = from_f32<To>(ov.x);
+        o[1] = from_f32<To>(ov.y);
+        o[2] = from_f32<To>(ov.z);
+        o[3] = from_f32<To>(ov.w);
     }
+}
+
+template <bool kDecayFirst, bool kFused>
+static cudaError_t launch_decode_typed(const cudaLaunchConfig_t& cfg, const LoopSlice& s, int dtype_bf16,
+                                       int use_pdl)
+{
+    using bf = __nv_bfloat16;
+    if (dtype_bf16) {
+        if (s.out_bf16) return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<bf, bf, kDecayFirst, kFused>, s, use_pdl);
+        return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<bf, float, kDecayFirst, kFused>, s, use_pdl);
+    }
+    if (s.out_bf16) return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<float, bf, kDecayFirst, kFused>, s, use_pdl);
+    return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<float, float, kDecayFirst, kFused>, s, use_pdl);
 }
 
 cudaError_t launch_decode(const LoopSlice& s, int dtype_bf16, cudaStream_t stream, bool pdl)
@@ -164,22 +224,13 @@ cudaError_t launch_decode(const LoopSlice& s, int dtype_bf16, cudaStream_t strea
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const int use_pdl = pdl ? 1 : 0;
-    using bf = __nv_bfloat16;
-    // one instance per input type, output type and order of the per-key factors
-    if (s.decay_first) {
-        if (dtype_bf16) {
-            if (s.out_bf16) return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<bf, bf, true>, s, use_pdl);
-            return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<bf, float, true>, s, use_pdl);
-        }
-        if (s.out_bf16) return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<float, bf, true>, s, use_pdl);
-        return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<float, float, true>, s, use_pdl);
-    }
-    if (dtype_bf16) {
-        if (s.out_bf16) return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<bf, bf, false>, s, use_pdl);
-        return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<bf, float, false>, s, use_pdl);
-    }
-    if (s.out_bf16) return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<float, bf, false>, s, use_pdl);
-    return cudaLaunchKernelEx(&cfg, gdr_decode_kernel<float, float, false>, s, use_pdl);
+    // one instance per input type, output type, order of the per-key factors and fusion
+    const bool fused = s.qk_norm || s.gate_logits || s.z;
+    if (s.decay_first)
+        return fused ? launch_decode_typed<true, true>(cfg, s, dtype_bf16, use_pdl)
+                     : launch_decode_typed<true, false>(cfg, s, dtype_bf16, use_pdl);
+    return fused ? launch_decode_typed<false, true>(cfg, s, dtype_bf16, use_pdl)
+                 : launch_decode_typed<false, false>(cfg, s, dtype_bf16, use_pdl);
 }
 
 }  // namespace lt2

@@ -30,7 +30,18 @@ struct TcCall {
     int out_bf16;
     int decay_first;         // per-key gating as (I - beta k k^T) Diag(alpha)
     unsigned int* err;
+    int qk_norm;             // fused prologue and output gate, as in LoopSlice
+    int gate_logits;
+    float alpha_scale;
+    const void* z;
 };
+// The fused steps of a call as the template argument of the tensor-core kernels' instances.
+enum FuseBits : int { kFuseNorm = 1, kFuseLogits = 2, kFuseGate = 4 };
+inline int fuse_bits(const TcCall& c)
+{
+    return (c.qk_norm ? kFuseNorm : 0) | (c.gate_logits ? kFuseLogits : 0) | (c.z ? kFuseGate : 0);
+}
+
 // Scalar gating: 64-token chunks.  Per-key gating: 32-token chunks in the e-form (chunks whose
 // per-key decay is out of the tensor-core range run token by token inside the same kernel).
 bool prefill_tc_supports(int dtype_bf16, int dk, int dv, int per_key);

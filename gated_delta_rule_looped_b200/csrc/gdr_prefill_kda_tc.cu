@@ -183,6 +183,11 @@ struct Params {
     int units_total;           // T*B*H (the extent of the tensor maps' unit axis)
     int out_bf16;
     unsigned int* err;
+    // fused prologue and output gate (used by the instances that compile the step in)
+    int qk_norm;
+    int gate_logits;
+    float alpha_scale;
+    const __nv_bfloat16* z;    // [units_total][L][128] output gate logits, or null
 };
 
 #ifdef LT2_DEBUG
@@ -229,7 +234,9 @@ __device__ __forceinline__ bool in_factor_range(float4 f)
 
 // Row t of the chunk's alpha (t in [t_begin, t_end)) becomes prod_{t_begin <= u <= t} alpha_u,
 // alpha taken as 1 past the chunk's last token n - 1.
-__device__ __forceinline__ void local_products(float* alpha_c, int n, int t_begin, int t_end, int lane)
+// With kLogits (the fused prologue) the rows hold logits a, and alpha = exp(-softplus(a) c).
+template <bool kLogits>
+__device__ __forceinline__ void local_products(float* alpha_c, int n, int t_begin, int t_end, int lane, float c)
 {
     float4 p = make_float4(1.f, 1.f, 1.f, 1.f);
     #pragma unroll 1
@@ -237,8 +244,12 @@ __device__ __forceinline__ void local_products(float* alpha_c, int n, int t_begi
         float4* row = reinterpret_cast<float4*>(alpha_c + t4 * kD + 4 * lane);
         float4 a[4];
         #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 4; ++i) {
             a[i] = t4 + i < n && t4 + i < t_end ? row[i * (kD / 4)] : make_float4(1.f, 1.f, 1.f, 1.f);
+            if (kLogits && t4 + i < n)
+                a[i] = make_float4(alpha_from_logit_fast(a[i].x, c), alpha_from_logit_fast(a[i].y, c),
+                                   alpha_from_logit_fast(a[i].z, c), alpha_from_logit_fast(a[i].w, c));
+        }
         #pragma unroll
         for (int i = 0; i < 4; ++i) {
             p = mul4(p, a[i]);
@@ -266,7 +277,9 @@ __device__ __forceinline__ float4 chunk_products(const float* alpha_c, int w, in
 // running products of local_products.  The warp starting at token 0 writes sq of every key to
 // `sq_out`; the return value says whether every F_t of the warp's tokens lies in
 // [kFactorMin, kFactorMax].
-template <bool decay_first>
+// kNorm (the fused prologue): every k and q row is divided by its L2 norm first (the warp holds
+// the whole row, four keys a lane).
+template <bool decay_first, bool kNorm>
 __device__ __forceinline__ bool convert_kqv(uint32_t st, uint32_t gram, const float* alpha_c, float bl, float4 Ph,
                                             float4 Pt, int t_begin, int t_end, int lane, uint8_t* sbase, uint32_t sb,
                                             float* sq_out)
@@ -293,7 +306,18 @@ __device__ __forceinline__ bool convert_kqv(uint32_t st, uint32_t gram, const fl
         uint2* kp = reinterpret_cast<uint2*>(kq + off);
         uint2* qp = reinterpret_cast<uint2*>(kq + off + 4096);
         uint2* vp = reinterpret_cast<uint2*>(vt + off);
-        const float4 k = unpack4_bf16(*kp), q = unpack4_bf16(*qp);
+        float4 k = unpack4_bf16(*kp), q = unpack4_bf16(*qp);
+        if (kNorm) {
+            float nk = k.x * k.x + k.y * k.y + k.z * k.z + k.w * k.w;
+            float nq = q.x * q.x + q.y * q.y + q.z * q.z + q.w * q.w;
+            #pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                nk += __shfl_xor_sync(0xffffffffu, nk, off);
+                nq += __shfl_xor_sync(0xffffffffu, nq, off);
+            }
+            k = scale4(k, inv_l2_fast(nk));
+            q = scale4(q, inv_l2_fast(nq));
+        }
         const uint2 vb = *vp;
         const float4 Pn = mul4(Ph, lp), Fn = mul4(Pn, isq), Rn = rcp4(Fn);
         ok = ok && in_factor_range(Fn);
@@ -474,19 +498,44 @@ struct ExactIn {
     void* o;
     int out_bf16;
     unsigned int* err;      // status word: a non-finite output is flagged there
+    int qk_norm;            // the fused prologue and output gate (instances with kF != 0)
+    int gate_logits;
+    float alpha_scale;
+    const __nv_bfloat16* z;
 };
 // decay_first: (I - beta k k^T) Diag(alpha), e = (alpha . k)^T S, S <- Diag(alpha) S + beta k (v - e)
-template <bool decay_first>
+// kF (FuseBits): alpha and beta from logits, k and q divided by their L2 norms, o times sigmoid(z).
+template <bool decay_first, int kF>
 __device__ __noinline__ void exact_chunk(uint32_t tm_s, ExactIn p, int64_t row0, int n, int j)
 {
-    bool fin = true;
     #pragma unroll 1
     for (int t = 0; t < n; ++t) {
         const int64_t row = row0 + t;
         const __nv_bfloat16* kr = p.k + row * kD;
         const __nv_bfloat16* qr = p.q + row * kD;
         const float* ar = p.alpha + row * kD;
-        const float b = p.beta[row];
+        float b = p.beta[row];
+        float ik = 1.f, iq = 1.f;           // inverse L2 norms of k and q (fused prologue)
+        {
+            if (kF & kFuseLogits) b = sigmoid_fast(b);
+            if (kF & kFuseNorm) {
+                float nk = 0.f, nq = 0.f;
+                #pragma unroll 1
+                for (int d8 = 0; d8 < kD; d8 += 8) {
+                    const uint4 kw = *reinterpret_cast<const uint4*>(kr + d8);
+                    const uint4 qw = *reinterpret_cast<const uint4*>(qr + d8);
+                    const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w}, qq[4] = {qw.x, qw.y, qw.z, qw.w};
+                    #pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        nk = fmaf(bf16_lo(kk[u]), bf16_lo(kk[u]), fmaf(bf16_hi(kk[u]), bf16_hi(kk[u]), nk));
+                        nq = fmaf(bf16_lo(qq[u]), bf16_lo(qq[u]), fmaf(bf16_hi(qq[u]), bf16_hi(qq[u]), nq));
+                    }
+                }
+                ik = inv_l2_fast(nk);
+                iq = inv_l2_fast(nq);
+            }
+        }
+        auto alpha_at = [&](float a) { return (kF & kFuseLogits) ? alpha_from_logit_fast(a, p.alpha_scale) : a; };
         const float vj = __bfloat162float(p.v[row * kD + j]);
         float e = 0.f;
         #pragma unroll 1
@@ -502,11 +551,15 @@ __device__ __noinline__ void exact_chunk(uint32_t tm_s, ExactIn p, int64_t row0,
                     a0 = *reinterpret_cast<const float4*>(ar + 64 * h + d8);
                     a1 = *reinterpret_cast<const float4*>(ar + 64 * h + d8 + 4);
                 }
+                if ((kF & kFuseLogits) && decay_first) {
+                    a0 = make_float4(alpha_at(a0.x), alpha_at(a0.y), alpha_at(a0.z), alpha_at(a0.w));
+                    a1 = make_float4(alpha_at(a1.x), alpha_at(a1.y), alpha_at(a1.z), alpha_at(a1.w));
+                }
                 const float aa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
                 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    e = fmaf(bf16_lo(kk[u]) * aa[2 * u], sv[d8 + 2 * u], e);
-                    e = fmaf(bf16_hi(kk[u]) * aa[2 * u + 1], sv[d8 + 2 * u + 1], e);
+                    e = fmaf(bf16_lo(kk[u]) * ik * aa[2 * u], sv[d8 + 2 * u], e);
+                    e = fmaf(bf16_hi(kk[u]) * ik * aa[2 * u + 1], sv[d8 + 2 * u + 1], e);
                 }
             }
         }
@@ -519,14 +572,18 @@ __device__ __noinline__ void exact_chunk(uint32_t tm_s, ExactIn p, int64_t row0,
             for (int d8 = 0; d8 < 64; d8 += 8) {
                 const uint4 kw = *reinterpret_cast<const uint4*>(kr + 64 * h + d8);
                 const uint4 qw = *reinterpret_cast<const uint4*>(qr + 64 * h + d8);
-                const float4 a0 = *reinterpret_cast<const float4*>(ar + 64 * h + d8);
-                const float4 a1 = *reinterpret_cast<const float4*>(ar + 64 * h + d8 + 4);
+                float4 a0 = *reinterpret_cast<const float4*>(ar + 64 * h + d8);
+                float4 a1 = *reinterpret_cast<const float4*>(ar + 64 * h + d8 + 4);
+                if (kF & kFuseLogits) {
+                    a0 = make_float4(alpha_at(a0.x), alpha_at(a0.y), alpha_at(a0.z), alpha_at(a0.w));
+                    a1 = make_float4(alpha_at(a1.x), alpha_at(a1.y), alpha_at(a1.z), alpha_at(a1.w));
+                }
                 const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w};
                 const uint32_t qq[4] = {qw.x, qw.y, qw.z, qw.w};
                 const float aa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
                 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const float k0 = bf16_lo(kk[u]), k1 = bf16_hi(kk[u]);
+                    const float k0 = bf16_lo(kk[u]) * ik, k1 = bf16_hi(kk[u]) * ik;
                     float& s0 = sv[d8 + 2 * u];
                     float& s1 = sv[d8 + 2 * u + 1];
                     if (decay_first) {
@@ -536,40 +593,36 @@ __device__ __noinline__ void exact_chunk(uint32_t tm_s, ExactIn p, int64_t row0,
                         s0 = aa[2 * u] * (s0 - b * k0 * e) + b * k0 * vj;
                         s1 = aa[2 * u + 1] * (s1 - b * k1 * e) + b * k1 * vj;
                     }
-                    o = fmaf(bf16_lo(qq[u]), s0, o);
-                    o = fmaf(bf16_hi(qq[u]), s1, o);
+                    o = fmaf(bf16_lo(qq[u]) * iq, s0, o);
+                    o = fmaf(bf16_hi(qq[u]) * iq, s1, o);
                 }
             }
             tmem_st32(tm_s + 64 * h, *reinterpret_cast<float(*)[32]>(sv));
             tmem_st32(tm_s + 64 * h + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
             tmem_wait_st();
         }
-        fin &= is_finite(o);
+        if (kF & kFuseGate) o *= sigmoid_fast(__bfloat162float(p.z[row * kD + j]));
         if (p.out_bf16)
             static_cast<__nv_bfloat16*>(p.o)[row * kD + j] = __float2bfloat16_rn(o);
         else
             static_cast<float*>(p.o)[row * kD + j] = o;
     }
-    if (!fin) atomicOr(p.err, kDevRange);
 }
 
 // Chain thread j, fp32 output: o[r][j] = (Q^ S)_rj - B_rj for tokens r = r0 .. r0 + 15 below n
-// (tm_qs and tm_b address token r0).
-// Returns false if any of them is not finite.
-__device__ __noinline__ bool store_o_f32(uint32_t tm_qs, uint32_t tm_b, float* o, int r0, int n)
+// (tm_qs and tm_b address token r0), times sigmoid(z[r][j]) when z (column j of the chunk's
+// output gate logits) is given.
+__device__ __noinline__ void store_o_f32(uint32_t tm_qs, uint32_t tm_b, float* o, int r0, int n,
+                                         const __nv_bfloat16* z)
 {
     float qp[32];
     tmem_load_2x16(tm_qs, tm_b, qp);
-    bool fin = true;
     #pragma unroll
     for (int r = 0; r < 16; ++r) {
-        const float ov = qp[r] - qp[16 + r];
-        if (r0 + r < n) {
-            fin &= is_finite(ov);
-            o[(r0 + r) * kD] = ov;
-        }
+        float ov = qp[r] - qp[16 + r];
+        if (z && r0 + r < n) ov *= sigmoid_fast(__bfloat162float(z[(r0 + r) * kD]));
+        if (r0 + r < n) o[(r0 + r) * kD] = ov;
     }
-    return fin;
 }
 
 // Gram [Kt; Qt; -] [Be; Bv]^T (M = 128, N = 64, K = 128) into TMEM, Be and Bv from the chunk
@@ -601,7 +654,11 @@ __device__ __noinline__ int issue_gram_of(int k, uint32_t sb, uint32_t tmem, int
     return 1;
 }
 
-template <bool kDecayFirst>
+// kF (FuseBits): the fused steps this instance compiles in -- alpha, beta from logits; k, q rows
+// normalised to unit L2 norm while they are converted; the output gate (o <- sigmoid(z) o, z read
+// from L1, where the chain prefetches it at the top of the chunk).  One instance per combination,
+// so that a call carries the code of the steps it uses only; kF = 0 compiles exactly as without.
+template <bool kDecayFirst, int kF>
 __global__ void __launch_bounds__(kThreads, 1)
 gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -726,18 +783,25 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
             // beta of token `lane` of this chunk: the load is issued before the waits below, which
             // hide its latency
-            const float bl = lane < n ? p.beta[static_cast<int64_t>(ug) * L + t0 + lane] : 0.f;
+            float bl = lane < n ? p.beta[static_cast<int64_t>(ug) * L + t0 + lane] : 0.f;
+            if ((kF & kFuseLogits) && lane < n) bl = sigmoid_fast(bl);
             if (!grp.wait(bar_addr(sb, B_FULL + s), ph, bar_addr(sb, B_GATE_EMPTY + s), ph ^ 1,
                           bar_addr(sb, B_AL_FULL + (c & 1)), (c >> 1) & 1))
                 break;
             if (!grp.wait(bar_addr(sb, B_GFREE + (c & 1)), ((c >> 1) & 1) ^ 1)) break;
             float* alpha_c = reinterpret_cast<float*>(sbase + OFF_ALPHA + (c & 1) * ALPHA_STAGE);
-            local_products(alpha_c, n, t_begin, t_end, lane);
+            if (kF & kFuseLogits)
+                local_products<true>(alpha_c, n, t_begin, t_end, lane, p.alpha_scale);
+            else
+                local_products<false>(alpha_c, n, t_begin, t_end, lane, 0.f);
             grp.sync();
             float4 Ph;
             const float4 Pt = chunk_products(alpha_c, w, lane, Ph);
             Gates* gs = gate(s);
-            const bool in_range = convert_kqv<kDecayFirst>(st, sb + OFF_GRAM + (c & 1) * GRAM_BUF, alpha_c, bl, Ph, Pt,
+            // (written as a select between the two instances: the plain kernel's register
+            // allocation, measured, is better this way)
+            const bool in_range = ((kF & kFuseNorm) && p.qk_norm ? convert_kqv<kDecayFirst, true> : convert_kqv<kDecayFirst, false>)(
+                                                           st, sb + OFF_GRAM + (c & 1) * GRAM_BUF, alpha_c, bl, Ph, Pt,
                                                            t_begin, t_end, lane, sbase, sb, gs->sq);
             if (lane == 0) gs->in_range[w] = in_range ? 1 : 0;
             fence_proxy_async_smem();
@@ -818,6 +882,12 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             const bool exact = !gates_in_range(gs);
             const bool last = c + 1 == nchunks;
             const int s1 = (c + 1) % kStages;
+            if ((kF & kFuseGate) && j < 2 * n) {
+                // the chunk's output gate logits (n rows of 256 bytes, two lines a row) into L1,
+                // for the output epilogue that runs under MMA_C
+                const __nv_bfloat16* zl = p.z + (static_cast<int64_t>(ug) * L + t0 + (j >> 1)) * kD + (j & 1) * 64;
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(zl));
+            }
             if (!exact) {
                 // --- MMA_A: (K^ S, Q^ S)^T = S^T [K^; Q^]^T ---
                 grp.sync();
@@ -909,24 +979,25 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                     __syncwarp();
                 }
                 // --- while MMA_C runs: o = Q^ S - (the -O' half of MMA_B), tokens 16h .. + 15 ---
-                // (a non-finite output is flagged where it is found: rows past L are finite too,
-                // from zero inputs, so a flag means a real output went out of range)
+                // (out-of-range operands are flagged through the final state: a state that left
+                // the fp16 range carries infinities or NaNs to the end of the sequence)
                 if (!p.out_bf16) {
-                    if (!store_o_f32(tmem + TM_AB + lane_addr + 32 + 16 * h, tmem + TM_B + lane_addr + 32 + 16 * h,
-                                     static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, 16 * h, n))
-                        atomicOr(err, kDevRange);
+                    store_o_f32(tmem + TM_AB + lane_addr + 32 + 16 * h, tmem + TM_B + lane_addr + 32 + 16 * h,
+                                     static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, 16 * h, n,
+                                     (kF & kFuseGate) ? p.z + (static_cast<int64_t>(ug) * L + t0) * kD + j : nullptr);
                 } else {
                     float qp[32];
                     tmem_load_2x16(tmem + TM_AB + lane_addr + 32 + 16 * h, tmem + TM_B + lane_addr + 32 + 16 * h, qp);
                     uint8_t* ost = sbase + OFF_OST + (j >> 6) * 4096 + (j & 63) * 2 + 16 * h * 128;
-                    bool bad = false;
+                    // the fused output gate: column j of the chunk's logits, prefetched to L1
+                    const __nv_bfloat16* zc = (kF & kFuseGate) ? p.z + (static_cast<int64_t>(ug) * L + t0 + 16 * h) * kD + j
+                                                            : nullptr;
                     #pragma unroll
                     for (int r = 0; r < 16; ++r) {
-                        const float ov = qp[r] - qp[16 + r];
-                        bad |= !is_finite(ov);
+                        float ov = qp[r] - qp[16 + r];
+                        if ((kF & kFuseGate) && 16 * h + r < n) ov *= sigmoid_fast(__bfloat162float(zc[r * kD]));
                         *reinterpret_cast<__nv_bfloat16*>(ost + r * 128) = __float2bfloat16_rn(ov);
                     }
-                    if (bad) atomicOr(err, kDevRange);
                     fence_proxy_async_smem();
                 }
                 // MMA_C done, and the next chunk's gates written
@@ -944,9 +1015,10 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 // --- out-of-range chunk: the definition, token by token, on the fp32 state (the
                 // first half of the chain's warps; every key of a column takes part in k^T S) ---
                 if (h == 0)
-                    exact_chunk<kDecayFirst>(tmem + TM_S + lane_addr,
-                                             ExactIn{p.q, p.k, p.v, p.alpha, p.beta, p.o, p.out_bf16, err},
-                                             static_cast<int64_t>(ug) * L + t0, n, j);
+                    exact_chunk<kDecayFirst, kF>(tmem + TM_S + lane_addr,
+                                                     ExactIn{p.q, p.k, p.v, p.alpha, p.beta, p.o, p.out_bf16, err,
+                                                             p.qk_norm, p.gate_logits, p.alpha_scale, p.z},
+                                                     static_cast<int64_t>(ug) * L + t0, n, j);
                 tc_fence_before();
                 // keep every hand-off in step: the stage and the [X; Z] stage are released
                 // once their producers are done with them, the output epilogue is released
@@ -1010,8 +1082,16 @@ cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream)
         return cudaErrorInvalidValue;
     CUtensorMap ma;
     if (!make_f32_map_3d(&ma, call.alpha, units, call.L, kC)) return cudaErrorInvalidValue;
-    // one instance per order of the per-key factors
-    const auto kernel = call.decay_first ? gdr_prefill_kda_tc_kernel<true> : gdr_prefill_kda_tc_kernel<false>;
+    // one instance per order of the per-key factors and combination of fused steps
+    using K = decltype(&gdr_prefill_kda_tc_kernel<false, 0>);
+    static const K kernels[2][8] = {
+        {gdr_prefill_kda_tc_kernel<false, 0>, gdr_prefill_kda_tc_kernel<false, 1>, gdr_prefill_kda_tc_kernel<false, 2>,
+         gdr_prefill_kda_tc_kernel<false, 3>, gdr_prefill_kda_tc_kernel<false, 4>, gdr_prefill_kda_tc_kernel<false, 5>,
+         gdr_prefill_kda_tc_kernel<false, 6>, gdr_prefill_kda_tc_kernel<false, 7>},
+        {gdr_prefill_kda_tc_kernel<true, 0>, gdr_prefill_kda_tc_kernel<true, 1>, gdr_prefill_kda_tc_kernel<true, 2>,
+         gdr_prefill_kda_tc_kernel<true, 3>, gdr_prefill_kda_tc_kernel<true, 4>, gdr_prefill_kda_tc_kernel<true, 5>,
+         gdr_prefill_kda_tc_kernel<true, 6>, gdr_prefill_kda_tc_kernel<true, 7>}};
+    const K kernel = kernels[call.decay_first ? 1 : 0][fuse_bits(call)];
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess) return e;
@@ -1031,6 +1111,10 @@ cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream)
         p.units_total = static_cast<int>(units);
         p.out_bf16 = call.out_bf16;
         p.err = call.err;
+        p.qk_norm = call.qk_norm;
+        p.gate_logits = call.gate_logits;
+        p.alpha_scale = call.alpha_scale;
+        p.z = static_cast<const __nv_bfloat16*>(call.z);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(call.units_per_loop), 1, 1);
         cfg.blockDim = dim3(kThreads, 1, 1);

@@ -14,6 +14,10 @@
 //   S  <- Diag(alpha_t) S - beta_t k_t e_t + beta_t k_t v_t^T
 //   o_t = f_t - beta_t (q_t . k_t) e_t + beta_t (q_t . k_t) v_t
 //
+// The fused prologue and output gate (lt2_gdr_fused) run here too: q and k rows normalised to
+// unit L2 norm, alpha = exp(-softplus(a) c) and beta = sigmoid(b) from logits when the tile is
+// staged, and o_t <- sigmoid(z_t) o_t when it is written.
+//
 // This path serves fp32 inputs (where bf16 tensor cores cannot meet a 1e-4 tolerance) and
 // every shape the tensor-core kernel does not cover.  Columns of S evolve independently
 // (A_t acts from the left), so the grid is (head-unit, 32-column slice of d_v).  Inside a
@@ -73,31 +77,57 @@ __global__ void __launch_bounds__(256) gdr_prefill_seq_kernel(LoopSlice p, int u
     for (int64_t t0 = 0; t0 < p.L; t0 += kTile) {
         const int nt = (p.L - t0 < kTile) ? (int)(p.L - t0) : kTile;
         __syncthreads();   // previous tile fully consumed
+        // k, q (raw), alpha and beta of the tile; with gate logits, alpha = exp(-softplus(a) c)
+        // and beta = sigmoid(b) (the fused prologue)
         for (int idx = threadIdx.x; idx < nt * dk; idx += blockDim.x) {
             const int tt = idx / dk, i = idx - tt * dk;
             const int64_t g = (t0 + tt) * dk + i;
-            const float a = p.per_key ? al[g] : al[t0 + tt];
             sk[tt * dk + i] = to_f32(k[g]);
-            saq[tt * dk + i] = a * to_f32(q[g]);
-            if (p.per_key) sa[tt * dk + i] = a;
+            saq[tt * dk + i] = to_f32(q[g]);
+            if (p.per_key) sa[tt * dk + i] = p.gate_logits ? alpha_from_logit(al[g], p.alpha_scale) : al[g];
         }
         for (int idx = threadIdx.x; idx < nt * kCols; idx += blockDim.x) {
             const int tt = idx / kCols, j = idx - tt * kCols;
             sv[idx] = (j < ncol) ? to_f32(v[(t0 + tt) * dv + j0 + j]) : 0.f;
         }
         if (threadIdx.x < nt) {
-            sb[threadIdx.x] = be[t0 + threadIdx.x];
-            if (!p.per_key) sa[threadIdx.x] = al[t0 + threadIdx.x];
+            const float b = be[t0 + threadIdx.x];
+            sb[threadIdx.x] = p.gate_logits ? sigmoid_f32(b) : b;
+            if (!p.per_key) {
+                const float a = al[t0 + threadIdx.x];
+                sa[threadIdx.x] = p.gate_logits ? alpha_from_logit(a, p.alpha_scale) : a;
+            }
         }
         __syncthreads();
-        // q.k and (alpha.q).k per token: one warp per token, lanes over channels.
+        // per token, one warp over the channels: the fused L2 normalisation of q and k, then
+        // q.k, alpha . q and (alpha.q).k
         for (int tt = w; tt < nt; tt += 8) {
+            float* kt = sk + tt * dk;
+            float* qt = saq + tt * dk;
+            if (p.qk_norm) {
+                float nq = 0.f, nk = 0.f;
+                for (int i = c; i < dk; i += 32) {
+                    nq += qt[i] * qt[i];
+                    nk += kt[i] * kt[i];
+                }
+                #pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    nq += __shfl_xor_sync(0xffffffffu, nq, off);
+                    nk += __shfl_xor_sync(0xffffffffu, nk, off);
+                }
+                const float iq = inv_l2(nq), ik = inv_l2(nk);
+                for (int i = c; i < dk; i += 32) {
+                    qt[i] *= iq;
+                    kt[i] *= ik;
+                }
+            }
             float a = 0.f, b = 0.f;
             for (int i = c; i < dk; i += 32) {
-                const int64_t g = (t0 + tt) * dk + i;
-                const float kq = to_f32(q[g]) * sk[tt * dk + i];
+                const float al_i = p.per_key ? sa[tt * dk + i] : sa[tt];
+                const float kq = qt[i] * kt[i];
+                qt[i] *= al_i;
                 a += kq;
-                b += saq[tt * dk + i] * sk[tt * dk + i];
+                b += qt[i] * kt[i];
             }
             #pragma unroll
             for (int off = 16; off > 0; off >>= 1) {
@@ -142,8 +172,12 @@ __global__ void __launch_bounds__(256) gdr_prefill_seq_kernel(LoopSlice p, int u
                 }
             }
             const float qke = p.decay_first ? sqk[tt] : saqk[tt];
-            if (w == 0 && active)
-                o[(t0 + tt) * dv + j0 + c] = from_f32<To>(F - bt * qke * E + bt * sqk[tt] * vc);
+            if (w == 0 && active) {
+                float ov = F - bt * qke * E + bt * sqk[tt] * vc;
+                if (p.z)        // the fused output gate
+                    ov *= sigmoid_f32(to_f32(static_cast<const T*>(p.z)[(u * p.L + t0 + tt) * dv + j0 + c]));
+                o[(t0 + tt) * dv + j0 + c] = from_f32<To>(ov);
+            }
         }
     }
 

@@ -116,7 +116,8 @@ enum Bar : uint32_t {
     B_O_READY = 24,    // output epilogue may read its TMEM columns
     B_O_DONE = 25,     // output epilogue has read them
     B_DRAIN = 26,      // [2] drain on abort (chain, Gram issuer)
-    B_COUNT = 28
+    B_Z = 28,          // output gate logits of a chunk landed in the staging tile (fused instance)
+    B_COUNT = 29
 };
 constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + B_COUNT * 8;        // tcgen05.alloc result
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 16;
@@ -153,6 +154,10 @@ struct Params {
     int units_total;       // T*B*H (the extent of the tensor maps' unit axis)
     int out_bf16;
     unsigned int* err;
+    // fused prologue and output gate (used by the instances that compile the step in)
+    int qk_norm;
+    int gate_logits;
+    float alpha_scale;
 };
 
 #ifdef LT2_DEBUG
@@ -197,9 +202,11 @@ __device__ __noinline__ void load_initial_state(uint32_t tm_s, uint32_t tm_sh, c
     tmem_wait_st();
 }
 
-// Output thread j, fp32 output: o[r][j] = g_r (Q S)_rj + (P T X)_rj for the chunk's n tokens.
-// Returns false if any of them is not finite.
-__device__ __noinline__ bool store_o_f32(uint32_t tm_qs, uint32_t tm_ptx, const float* gam, float* o, int n)
+// Output thread j, fp32 output: o[r][j] = g_r (Q S)_rj + (P T X)_rj for the chunk's n tokens,
+// times sigmoid(z[r][j]) when `zst` points at column j of the output gate logits in the staging
+// tile (rows 128 bytes apart).  Returns false if any of them is not finite.
+__device__ __noinline__ bool store_o_f32(uint32_t tm_qs, uint32_t tm_ptx, const float* gam, float* o, int n,
+                                         const uint8_t* zst)
 {
     bool fin = true;
     #pragma unroll 1
@@ -209,7 +216,8 @@ __device__ __noinline__ bool store_o_f32(uint32_t tm_qs, uint32_t tm_ptx, const 
         #pragma unroll
         for (int e = 0; e < 32; ++e) {
             const int r = 32 * piece + e;
-            const float ov = gam[r] * qp[e] + qp[32 + e];
+            float ov = gam[r] * qp[e] + qp[32 + e];
+            if (zst) ov *= sigmoid_fast(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(zst + r * 128)));
             if (r < n) {
                 fin &= is_finite(ov);
                 o[r * kD] = ov;
@@ -247,10 +255,16 @@ __device__ __noinline__ void gram_epilogue_unfactored(uint32_t tm_row, const Gat
     }
 }
 
+// kF: the fused steps this instance compiles in (bits of FuseBits): q, k rows normalised to unit
+// L2 norm while they are converted to fp16; alpha, beta from logits in the gate warp; the output
+// gate (the logits z of a chunk are loaded by TMA into the o staging tile, and o <- sigmoid(z) o
+// is applied as the tile is written).  One instance per combination, so that a call carries the
+// code of the steps it uses only; kF = 0 compiles exactly as without them.
+template <int kF>
 __global__ void __launch_bounds__(kThreads, 1)
 gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                      Params p, int use_pdl)
+                      const __grid_constant__ CUtensorMap tm_z, Params p, int use_pdl)
 {
     (void)use_pdl;
     allow_next_loop_to_start();
@@ -299,6 +313,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         mbar_init(bar_addr(sb, B_S_FULL), 1);
         mbar_init(bar_addr(sb, B_O_READY), 1);
         mbar_init(bar_addr(sb, B_O_DONE), 1);
+        mbar_init(bar_addr(sb, B_Z), 1);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -309,6 +324,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
             prefetch_tmap(&tm_o);
+            if (kF & kFuseGate) prefetch_tmap(&tm_z);
         }
     }
     if (warp >= 4 && warp < 8) {
@@ -392,7 +408,10 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 bool in_range = true;                   // every |G_r| < 80
                 #pragma unroll 1
                 for (int i = 0; i < 2; ++i) {
-                    const float a = i ? a_cur[1] : a_cur[0];
+                    float a = i ? a_cur[1] : a_cur[0];
+                    // (past the sequence end alpha = 1 and beta = 0 already: no logits there)
+                    const bool valid = static_cast<int64_t>(c) * kC + lane + 32 * i < L;
+                    if ((kF & kFuseLogits) && valid) a = alpha_from_logit_fast(a, p.alpha_scale);
                     float g = __logf(fmaxf(fabsf(a), 1e-30f));
                     #pragma unroll
                     for (int off = 1; off < 32; off <<= 1) {
@@ -406,7 +425,8 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     const int r = lane + 32 * i;
                     gs->G[r] = g;
                     gs->gam[r] = ((negs_before + __popc(neg & upto)) & 1) ? -1.f : 1.f;
-                    gs->beta[r] = i ? b_cur[1] : b_cur[0];
+                    const float bb = i ? b_cur[1] : b_cur[0];
+                    gs->beta[r] = (kF & kFuseLogits) && valid ? sigmoid_fast(bb) : bb;
                     negs_before += __popc(neg);
                     in_range &= fabsf(g) < 80.f;
                 }
@@ -435,12 +455,24 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const uint32_t st = sb + OFF_KQV + s * STAGE_BYTES;
             // K panels (warp 1) at +0 and +16 KB, Q panels (warp 2) at +8 and +24 KB, both V panels
             // (warp 3) at +32 KB: one copy of the conversion loop for all three
-            #pragma unroll 1
-            for (int panel = 0; panel < 2; ++panel) {
-                const uint32_t src = warp == 3 ? st + KQ_BYTES + panel * 8192
-                                               : st + (warp - 1) * 8192 + panel * 16384;
-                if (dbg_ok(src >= sb + OFF_KQV && src + 8192 <= sb + OFF_KQV + kStages * STAGE_BYTES, err))
-                    convert_tile(src, 512, lane, lds, sts);
+            if (kF & kFuseNorm) {
+                // Q (warp 2) and K (warp 3): every row divided by its L2 norm on the way to fp16;
+                // warp 1, which also computes the gates and issues the Gram, takes V instead
+                if (warp == 1) {
+                    #pragma unroll 1
+                    for (int panel = 0; panel < 2; ++panel) convert_tile(st + KQ_BYTES + panel * 8192, 512, lane, lds, sts);
+                } else {
+                    const uint32_t t = warp == 2 ? st + 8192 : st;
+                    convert_rows_l2(t, t + 16384, lane, lds, sts);
+                }
+            } else {
+                #pragma unroll 1
+                for (int panel = 0; panel < 2; ++panel) {
+                    const uint32_t src = warp == 3 ? st + KQ_BYTES + panel * 8192
+                                                   : st + (warp - 1) * 8192 + panel * 16384;
+                    if (dbg_ok(src >= sb + OFF_KQV && src + 8192 <= sb + OFF_KQV + kStages * STAGE_BYTES, err))
+                        convert_tile(src, 512, lane, lds, sts);
+                }
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -706,16 +738,28 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         bool fin = true;                             // every output so far is finite
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;
+            const int64_t t0 = static_cast<int64_t>(c) * kC;
             if (j == 0) bulk_wait_read_all();        // the staging tile is free again
-            if (!grp.wait(bar_addr(sb, B_O_READY), c & 1)) break;
+            constexpr bool gated = (kF & kFuseGate) != 0;
+            if (gated && j == 0) {
+                // the output gate logits of this chunk, into the staging tile the outputs are
+                // written to (the same two 64 x 64 boxes; rows past L read as 0)
+                const uint32_t zb = bar_addr(sb, B_Z);
+                mbar_arrive_expect_tx(zb, 16384);
+                tma_load_3d(sb + OFF_OST, &tm_z, 0, static_cast<int32_t>(t0), ug, zb);
+                tma_load_3d(sb + OFF_OST + 8192, &tm_z, 64, static_cast<int32_t>(t0), ug, zb);
+            }
+            if (!(gated ? grp.wait(bar_addr(sb, B_O_READY), c & 1, bar_addr(sb, B_Z), c & 1)
+                        : grp.wait(bar_addr(sb, B_O_READY), c & 1)))
+                break;
             tc_fence_after();
             const Gates* gs = gate(s);
-            const int64_t t0 = static_cast<int64_t>(c) * kC;
             if (!p.out_bf16) {
                 // fp32 output: plain stores, done before the TMEM columns are released
                 const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
                 fin &= store_o_f32(tmem + TM_AB + lane_addr + 64, tmem + TM_B + lane_addr + 64, gs->gam,
-                                   static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, n);
+                                   static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, n,
+                                   gated ? sbase + OFF_OST + (j >> 6) * 8192 + (j & 63) * 2 : nullptr);
                 tc_fence_before();
                 grp.sync();
                 if (j == 0) {
@@ -738,12 +782,14 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 #pragma unroll
                 for (int e4 = 0; e4 < 32; e4 += 4) {
                     const float4 g4 = *reinterpret_cast<const float4*>(gam + e4);
-                    const float ov[4] = {g4.x * qp[e4 + 0] + qp[32 + e4 + 0], g4.y * qp[e4 + 1] + qp[32 + e4 + 1],
-                                         g4.z * qp[e4 + 2] + qp[32 + e4 + 2], g4.w * qp[e4 + 3] + qp[32 + e4 + 3]};
+                    float ov[4] = {g4.x * qp[e4 + 0] + qp[32 + e4 + 0], g4.y * qp[e4 + 1] + qp[32 + e4 + 1],
+                                   g4.z * qp[e4 + 2] + qp[32 + e4 + 2], g4.w * qp[e4 + 3] + qp[32 + e4 + 3]};
                     #pragma unroll
                     for (int u = 0; u < 4; ++u) {
+                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(orow + (e4 + u) * 128);
+                        if (gated) ov[u] *= sigmoid_fast(__bfloat162float(*dst));     // z, then o in place
                         fin &= is_finite(ov[u]);
-                        *reinterpret_cast<__nv_bfloat16*>(orow + (e4 + u) * 128) = __float2bfloat16_rn(ov[u]);
+                        *dst = __float2bfloat16_rn(ov[u]);
                     }
                 }
             }
@@ -787,15 +833,24 @@ cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
     using namespace tc;
     if (call.units_per_loop == 0 || call.T == 0) return cudaSuccess;
     const int64_t units = call.T * call.units_per_loop;
-    CUtensorMap mq, mk, mv, mo;
+    CUtensorMap mq, mk, mv, mo, mz;
     const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
     if (!make_bf16_map_3d(&mq, call.q, units, call.L, kC, sw) || !make_bf16_map_3d(&mk, call.k, units, call.L, kC, sw) ||
         !make_bf16_map_3d(&mv, call.v, units, call.L, kC, sw))
         return cudaErrorInvalidValue;
-    // o (bf16 output only): plain row-major tile, written by the TMA store from shared memory
+    // o (bf16 output only): plain row-major tile, written by the TMA store from shared memory;
+    // the output gate logits z (fused) are read into the same tile the same way
     if (call.out_bf16 && !make_bf16_map_3d(&mo, call.o, units, call.L, kC, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(gdr_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (call.z && !make_bf16_map_3d(&mz, call.z, units, call.L, kC, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    const int fb = fuse_bits(call);
+    using K = decltype(&gdr_prefill_tc_kernel<0>);
+    static const K kernels[8] = {gdr_prefill_tc_kernel<0>, gdr_prefill_tc_kernel<1>, gdr_prefill_tc_kernel<2>,
+                                 gdr_prefill_tc_kernel<3>, gdr_prefill_tc_kernel<4>, gdr_prefill_tc_kernel<5>,
+                                 gdr_prefill_tc_kernel<6>, gdr_prefill_tc_kernel<7>};
+    const K kernel = kernels[fb];
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess) return e;
     for (int64_t tau = 0; tau < call.T; ++tau) {
@@ -811,6 +866,9 @@ cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
         p.units_total = static_cast<int>(units);
         p.out_bf16 = call.out_bf16;
         p.err = call.err;
+        p.qk_norm = call.qk_norm;
+        p.gate_logits = call.gate_logits;
+        p.alpha_scale = call.alpha_scale;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(call.units_per_loop), 1, 1);
         cfg.blockDim = dim3(kThreads, 1, 1);
@@ -822,7 +880,8 @@ cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         const int use_pdl = tau > 0 ? 1 : 0;
-        e = cudaLaunchKernelEx(&cfg, gdr_prefill_tc_kernel, mq, mk, mv, call.out_bf16 ? mo : mv, p, use_pdl);
+        // unused maps are passed as copies of a valid one (never dereferenced)
+        e = cudaLaunchKernelEx(&cfg, kernel, mq, mk, mv, call.out_bf16 ? mo : mv, call.z ? mz : mv, p, use_pdl);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

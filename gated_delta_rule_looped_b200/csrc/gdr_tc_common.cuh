@@ -8,6 +8,7 @@
 
 #include <cstdint>
 
+#include "gdr_common.cuh"
 #include "sm100_primitives.cuh"
 
 namespace lt2 {
@@ -208,6 +209,52 @@ __device__ __forceinline__ void convert_tile(uint32_t base, int n16, int lane, L
 
 // False for an infinity or a NaN.
 __device__ __forceinline__ bool is_finite(float x) { return fabsf(x) <= 3.402823466e38f; }
+
+// bf16 -> fp16, in place, of a 64-row tile held as two 64 x 64 panels (columns 0-63 at p0,
+// 64-127 at p1, 128-byte swizzled rows), every row divided by its L2 norm on the way (the fused
+// normalisation of q and k): lane l owns rows l and l + 32.  Pass 1 sums the squares of the row
+// in fp32, pass 2 rescales and converts; each pass loads a panel's eight vectors together.
+template <typename LdFn, typename StFn>
+__device__ __forceinline__ void convert_rows_l2(uint32_t p0, uint32_t p1, int lane, LdFn lds, StFn sts)
+{
+    #pragma unroll 1
+    for (int rr = 0; rr < 2; ++rr) {
+        const uint32_t r = static_cast<uint32_t>(lane + 32 * rr);
+        float ss = 0.f;
+        #pragma unroll 1
+        for (int pn = 0; pn < 2; ++pn) {
+            uint4 w[8];
+            #pragma unroll
+            for (uint32_t c = 0; c < 8; ++c) w[c] = lds(sw128(pn ? p1 : p0, r, c));
+            #pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint32_t ws[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+                #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float lo = bf16_lo(ws[e]), hi = bf16_hi(ws[e]);
+                    ss = fmaf(lo, lo, ss);
+                    ss = fmaf(hi, hi, ss);
+                }
+            }
+        }
+        const float inv = inv_l2_fast(ss);
+        #pragma unroll 1
+        for (int pn = 0; pn < 2; ++pn) {
+            uint4 w[8];
+            #pragma unroll
+            for (uint32_t c = 0; c < 8; ++c) w[c] = lds(sw128(pn ? p1 : p0, r, c));
+            #pragma unroll
+            for (uint32_t c = 0; c < 8; ++c) {
+                uint4 h;
+                h.x = pack_half2(bf16_lo(w[c].x) * inv, bf16_hi(w[c].x) * inv);
+                h.y = pack_half2(bf16_lo(w[c].y) * inv, bf16_hi(w[c].y) * inv);
+                h.z = pack_half2(bf16_lo(w[c].z) * inv, bf16_hi(w[c].z) * inv);
+                h.w = pack_half2(bf16_lo(w[c].w) * inv, bf16_hi(w[c].w) * inv);
+                sts(sw128(pn ? p1 : p0, r, c), h);
+            }
+        }
+    }
+}
 
 // Chain thread j: column j of the final state (row j of S^T in TMEM) to S_out.  Returns false
 // if any entry is not finite.

@@ -165,10 +165,33 @@ bool use_tensor_core(const lt2_gdr_dims* d)
     return ok;
 }
 
+// The fused prologue and output gate of a call: a zeroed struct when `f` is null.
+lt2_gdr_fused fused_or_none(const lt2_gdr_fused* f)
+{
+    lt2_gdr_fused none;
+    std::memset(&none, 0, sizeof(none));
+    return f ? *f : none;
+}
+
+lt2_status validate_fused(const lt2_gdr_fused& f, const Sizes& sz, const void* o, const float* S_out)
+{
+    if (f.reserved != 0) return LT2_ERR_INVALID_ARGUMENT;
+    if ((f.qk_l2norm != 0 && f.qk_l2norm != 1) || (f.gate_logits != 0 && f.gate_logits != 1))
+        return LT2_ERR_INVALID_ARGUMENT;
+    if (f.gate_logits && !(f.alpha_scale >= 0.f && f.alpha_scale <= 3.4e38f)) return LT2_ERR_INVALID_ARGUMENT;
+    if (f.z) {
+        if (!aligned16(f.z)) return LT2_ERR_INVALID_ARGUMENT;
+        const Range rz = range_of(f.z, sz.vo * sz.esz);
+        if (overlap(rz, range_of(o, sz.vo * sz.osz))) return LT2_ERR_INVALID_ARGUMENT;
+        if (S_out && overlap(rz, range_of(S_out, sz.st * 4))) return LT2_ERR_INVALID_ARGUMENT;
+    }
+    return LT2_OK;
+}
+
 lt2::LoopSlice loop_slice(const lt2_gdr_dims* d, const Sizes& sz, int64_t tau,
                           const void* q, const void* k, const void* v, const float* alpha,
                           const float* beta, const float* S0, void* o, float* S_out,
-                          unsigned int* err)
+                          unsigned int* err, const lt2_gdr_fused& f)
 {
     const int64_t U = sz.per_loop, L = d->L, dk = d->dk, dv = d->dv;
     const int64_t na = is_per_key(d) ? dk : 1;
@@ -189,6 +212,10 @@ lt2::LoopSlice loop_slice(const lt2_gdr_dims* d, const Sizes& sz, int64_t tau,
     s.decay_first = d->gate == LT2_GATE_PER_KEY_DECAY_FIRST ? 1 : 0;
     s.out_bf16 = out_is_bf16(d) ? 1 : 0;
     s.err = err;
+    s.qk_norm = f.qk_l2norm;
+    s.gate_logits = f.gate_logits;
+    s.alpha_scale = f.alpha_scale;
+    s.z = f.z ? static_cast<const char*>(f.z) + tau * U * L * dv * sz.esz : nullptr;
     return s;
 }
 
@@ -207,9 +234,19 @@ lt2_status lt2_gdr_prefill(const lt2_gdr_dims* dims, const void* q, const void* 
                            const float* alpha, const float* beta, const float* S0, void* o,
                            float* S_out, void* workspace, size_t workspace_bytes, void* stream)
 {
+    return lt2_gdr_prefill_fused(dims, nullptr, q, k, v, alpha, beta, S0, o, S_out, workspace,
+                                 workspace_bytes, stream);
+}
+
+lt2_status lt2_gdr_prefill_fused(const lt2_gdr_dims* dims, const lt2_gdr_fused* fused, const void* q,
+                                 const void* k, const void* v, const float* alpha, const float* beta,
+                                 const float* S0, void* o, float* S_out, void* workspace,
+                                 size_t workspace_bytes, void* stream)
+{
     Sizes sz;
     lt2_status st = validate_dims(dims, &sz);
     if (st != LT2_OK) return st;
+    const lt2_gdr_fused f = fused_or_none(fused);
     if (dims->algo == LT2_ALGO_TENSOR_CORE &&
         !lt2::prefill_tc_supports(dims->dtype == LT2_DTYPE_BF16, (int)dims->dk, (int)dims->dv,
                                   is_per_key(dims)))
@@ -238,8 +275,10 @@ lt2_status lt2_gdr_prefill(const lt2_gdr_dims* dims, const void* q, const void* 
         if (S0 && S0 != S_out && overlap(rs, range_of(S0, sz.st * 4)))
             return LT2_ERR_INVALID_ARGUMENT;
     }
+    st = validate_fused(f, sz, o, S_out);
+    if (st != LT2_OK) return st;
     if (sz.units == 0) return LT2_OK;
-    st = on_current_device({q, k, v, alpha, beta, S0, o, S_out, workspace});
+    st = on_current_device({q, k, v, alpha, beta, S0, o, S_out, workspace, f.z});
     if (st != LT2_OK) return st;
 
     NvtxRange range("lt2_gdr_prefill");
@@ -265,6 +304,10 @@ lt2_status lt2_gdr_prefill(const lt2_gdr_dims* dims, const void* q, const void* 
         call.out_bf16 = out_is_bf16(dims) ? 1 : 0;
         call.decay_first = dims->gate == LT2_GATE_PER_KEY_DECAY_FIRST ? 1 : 0;
         call.err = err;
+        call.qk_norm = f.qk_l2norm;
+        call.gate_logits = f.gate_logits;
+        call.alpha_scale = f.alpha_scale;
+        call.z = f.z;
         cudaError_t e = is_per_key(dims) ? lt2::launch_prefill_kda_tc_all(call, s)
                                          : lt2::launch_prefill_tc_all(call, s);
         if (e == cudaSuccess) e = cudaGetLastError();
@@ -272,7 +315,7 @@ lt2_status lt2_gdr_prefill(const lt2_gdr_dims* dims, const void* q, const void* 
         return LT2_OK;
     }
     for (int64_t tau = 0; tau < dims->T; ++tau) {
-        const lt2::LoopSlice ls = loop_slice(dims, sz, tau, q, k, v, alpha, beta, S0, o, S_out, err);
+        const lt2::LoopSlice ls = loop_slice(dims, sz, tau, q, k, v, alpha, beta, S0, o, S_out, err, f);
         // Loop 0 waits for all earlier work on the stream; later loops may start as soon as
         // the previous loop's grid is running (the loops share no data).
         const bool pdl = tau > 0;
@@ -287,9 +330,17 @@ lt2_status lt2_gdr_prefill(const lt2_gdr_dims* dims, const void* q, const void* 
 lt2_status lt2_gdr_decode(const lt2_gdr_dims* dims, const void* q, const void* k, const void* v,
                           const float* alpha, const float* beta, float* S, void* o, void* stream)
 {
+    return lt2_gdr_decode_fused(dims, nullptr, q, k, v, alpha, beta, S, o, stream);
+}
+
+lt2_status lt2_gdr_decode_fused(const lt2_gdr_dims* dims, const lt2_gdr_fused* fused, const void* q,
+                                const void* k, const void* v, const float* alpha, const float* beta,
+                                float* S, void* o, void* stream)
+{
     Sizes sz;
     lt2_status st = validate_dims(dims, &sz);
     if (st != LT2_OK) return st;
+    const lt2_gdr_fused f = fused_or_none(fused);
     if (dims->L != 1) return LT2_ERR_INVALID_ARGUMENT;
     if (!tensor_ok(q, sz.qk) || !tensor_ok(k, sz.qk) || !tensor_ok(v, sz.vo) ||
         !tensor_ok(alpha, sz.al) || !tensor_ok(beta, sz.be) || !tensor_ok(o, sz.vo) ||
@@ -302,8 +353,10 @@ lt2_status lt2_gdr_decode(const lt2_gdr_dims* dims, const void* q, const void* k
     if (overlap(ro, rs)) return LT2_ERR_INVALID_ARGUMENT;
     for (const Range& r : rin)
         if (overlap(ro, r) || overlap(rs, r)) return LT2_ERR_INVALID_ARGUMENT;
+    st = validate_fused(f, sz, o, S);
+    if (st != LT2_OK) return st;
     if (sz.units == 0) return LT2_OK;
-    st = on_current_device({q, k, v, alpha, beta, S, o});
+    st = on_current_device({q, k, v, alpha, beta, S, o, f.z});
     if (st != LT2_OK) return st;
 
     NvtxRange range("lt2_gdr_decode");
@@ -313,7 +366,7 @@ lt2_status lt2_gdr_decode(const lt2_gdr_dims* dims, const void* q, const void* k
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     for (int64_t tau = 0; tau < dims->T; ++tau) {
         NvtxRange loop_range("lt2 decode loop");
-        lt2::LoopSlice ls = loop_slice(dims, sz, tau, q, k, v, alpha, beta, nullptr, o, S, err);
+        lt2::LoopSlice ls = loop_slice(dims, sz, tau, q, k, v, alpha, beta, nullptr, o, S, err, f);
         cudaError_t e = lt2::launch_decode(ls, dims->dtype == LT2_DTYPE_BF16, s, tau > 0);
         if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "decode");

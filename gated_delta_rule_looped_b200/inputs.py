@@ -137,3 +137,24 @@ def make_decode_step(w, seed=0, step=0, device="cpu"):
 def decode_history(w, seed=0, device="cpu"):
     """The prefill inputs (L = w.history tokens) whose final state seeds the decode."""
     return make_inputs(replace(w, L=w.history, overwrite_frac=0.0), seed=seed, device=device)
+
+
+def make_raw_inputs(w, seed=0, device="cpu"):
+    """The raw projections of the fused prologue and output gate for workload ``w``: q, k and the
+    output gate logits z ~ N(0,1) in w's dtype (q and k NOT normalised), and N(0,1) logits a (the
+    shape of alpha: [T,B,H,L] or [T,B,H,L,d]) and b ([T,B,H,L]) in fp32; v ~ N(0,1); S0 as in
+    make_inputs.  Drawn in the order q, k, v, z, a, b, then S0."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    T, B, H, L, d = w.T, w.B, w.H, w.L, w.d
+    dt = w.torch_dtype
+    shape = (T, B, H, L, d)
+    q = _normal(shape, gen, device).to(dt)
+    k = _normal(shape, gen, device).to(dt)
+    v = _normal(shape, gen, device).to(dt)
+    z = _normal(shape, gen, device).to(dt)
+    a = _normal((T, B, H, L, d) if w.gate == "per_key" else (T, B, H, L), gen, device)
+    b = _normal((T, B, H, L), gen, device)
+    S0 = _normal((T, B, H, d, d), gen, device) if w.s0 == "normal" else None
+    return {"q": q, "k": k, "v": v, "z": z, "a": a, "b": b, "S0": S0}

@@ -123,6 +123,25 @@ typedef struct lt2_gdr_dims {
 } lt2_gdr_dims;
 
 /*
+ * The steps on either side of the mixer, fused into its kernels: the prologue that
+ * turns a layer's raw projections into the recurrence's inputs, and the sigmoid output gate of
+ * "LT2 transformer looped a tempo lineare", section "Dove il quadro si incrina" (a sigmoid gate
+ * inside the loop keeps the state norm under control; the wispaper.ai blog, section "Critical
+ * Insight: The Attention Sink Mitigation", calls it an SDPA output gate).  A zeroed struct
+ * selects none of them, which is exactly lt2_gdr_prefill / lt2_gdr_decode.
+ */
+typedef struct lt2_gdr_fused {
+    int32_t qk_l2norm;     /* 1: q and k are raw; every (token, head) row is divided by
+                              max(||row||_2, 1e-12) inside the kernels before it is used        */
+    int32_t gate_logits;   /* 1: alpha and beta hold logits a, b (same layouts as alpha, beta):
+                              beta = sigmoid(b), alpha = exp(-softplus(a) * alpha_scale)       */
+    float alpha_scale;     /* c of the alpha formula above (used when gate_logits = 1)          */
+    int32_t reserved;      /* must be 0                                                          */
+    const void* z;         /* output gate logits, dims->dtype, layout of v ([T][B][H][L][dv]);
+                              NULL = no gate.  Else every output is o <- sigmoid(z) * o          */
+} lt2_gdr_fused;
+
+/*
  * Bytes of device workspace lt2_gdr_prefill needs for `dims` (0 when none; every path of this
  * version keeps its intermediates on chip, so it is 0 for every valid `dims`).  Pure host
  * function, no CUDA call; returns 0 for invalid dims as well.
@@ -157,6 +176,22 @@ lt2_status lt2_gdr_prefill(const lt2_gdr_dims* dims,
                            void* stream);
 
 /*
+ * lt2_gdr_prefill with the fused prologue and output gate that `fused` selects (NULL or a zeroed
+ * struct: exactly lt2_gdr_prefill).  q, k, alpha and beta then hold the raw values the struct
+ * describes, and z, when given, must not alias o.  Every path of lt2_gdr_prefill fuses the steps
+ * into its own kernels: nothing extra is written to or read back from global memory.
+ * LT2_ERR_INVALID_ARGUMENT for reserved != 0, a flag other than 0 or 1, a non-finite or
+ * negative alpha_scale, a misaligned z or a z that overlaps o.
+ */
+lt2_status lt2_gdr_prefill_fused(const lt2_gdr_dims* dims, const lt2_gdr_fused* fused,
+                                 const void* q, const void* k, const void* v,
+                                 const float* alpha, const float* beta,
+                                 const float* S0,
+                                 void* o, float* S_out,
+                                 void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/*
  * Decode: one step of the same recurrence ("LT2 transformer looped a tempo lineare", section
  * "Sostituire il motore", displayed equation) for one new token per (loop, batch, head);
  * dims->L must be 1 and dims->algo is ignored.  S [T][B][H][dk][dv] fp32 is read and replaced
@@ -169,6 +204,14 @@ lt2_status lt2_gdr_decode(const lt2_gdr_dims* dims,
                           const float* alpha, const float* beta,
                           float* S, void* o,
                           void* stream);
+
+/* lt2_gdr_decode with the fused prologue and output gate of `fused` (as lt2_gdr_prefill_fused,
+ * with L = 1). */
+lt2_status lt2_gdr_decode_fused(const lt2_gdr_dims* dims, const lt2_gdr_fused* fused,
+                                const void* q, const void* k, const void* v,
+                                const float* alpha, const float* beta,
+                                float* S, void* o,
+                                void* stream);
 
 /*
  * The device-side status word of the CURRENT device (not an operation of the pages: the

@@ -206,3 +206,45 @@ def test_binding_rejects_tensors_it_cannot_pass_by_pointer():
     with pytest.raises(ValueError, match="CUDA"):
         lt2.decode(q[..., 0, :], q[..., 0, :], q[..., 0, :], a[..., 0], a[..., 0],
                    torch.zeros((1, 1, 1, 128, 128)))
+
+
+# ---- the fused entry points: their descriptor is validated before any launch ----------------
+
+def call_prefill_fused(dims, fused, **over):
+    q, k, v, a, b, s0, o, so = addrs(8)
+    args = dict(q=q, k=k, v=v, alpha=a, beta=b, S0=s0, o=o, S_out=so)
+    args.update(over)
+    return lt2.lt2_gdr_prefill_fused(dims, fused, args["q"], args["k"], args["v"], args["alpha"],
+                                     args["beta"], args["S0"], args["o"], args["S_out"], None, 0, 0)
+
+
+def test_fused_descriptor_layout():
+    assert ctypes.sizeof(lt2.lt2_gdr_fused) == 24
+    assert lt2.lt2_gdr_fused.z.offset == 16
+
+
+@pytest.mark.parametrize("field,value", [("reserved", 1), ("qk_l2norm", 2), ("gate_logits", -1)])
+def test_fused_bad_fields_rejected(L, field, value):
+    f = lt2.make_fused(True, True, 0.1)
+    setattr(f, field, value)
+    assert call_prefill_fused(D(), f) == lt2.LT2_ERR_INVALID_ARGUMENT
+
+
+@pytest.mark.parametrize("scale", [-0.5, float("nan"), float("inf")])
+def test_fused_bad_alpha_scale_rejected(L, scale):
+    assert call_prefill_fused(D(), lt2.make_fused(False, True, scale)) == lt2.LT2_ERR_INVALID_ARGUMENT
+
+
+def test_fused_z_checked(L):
+    q, k, v, a, b, s0, o, so = addrs(8)
+    assert call_prefill_fused(D(), lt2.make_fused(z=o + 64)) == lt2.LT2_ERR_INVALID_ARGUMENT     # overlaps o
+    assert call_prefill_fused(D(), lt2.make_fused(z=BASE + 9 * SPAN + 4)) == lt2.LT2_ERR_INVALID_ARGUMENT  # misaligned
+    dims = D(L=1)
+    assert lt2.lt2_gdr_decode_fused(dims, lt2.make_fused(z=o), q, k, v, a, b, s0, o, 0) == \
+        lt2.LT2_ERR_INVALID_ARGUMENT
+
+
+def test_fused_null_descriptor_is_the_plain_call(L):
+    # validation runs the same way: a bad dims fails identically with and without a descriptor
+    bad = D(dk=0)
+    assert call_prefill_fused(bad, None) == call_prefill(bad) == lt2.LT2_ERR_INVALID_ARGUMENT
