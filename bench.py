@@ -12,7 +12,9 @@ T loops, every chunk step: gates, Gram products, solve, state GEMMs, outputs) th
 with inputs already resident in HBM.  The other timed workloads ride along as keys of the same
 JSON line, each with its own `ms_per_step`, `value`, `roofline`, `cpu_baseline`, `clocks` and
 `gpu_launches`: `gdn_prefill` (T4 B4 H16 L8192, scalar gating), `kda_prefill` (T4 B2 H16
-L16384, per-key gating) and `decode` (one decode token for T4 B256 H16 from a 4096-token state).
+L16384, per-key gating), `decode` (one decode token for T4 B256 H16 from a 4096-token state) and
+`fused_gdn_prefill` (gdn_prefill through lt2_gdr_prefill_fused with raw inputs, against the same
+steps run as separate passes).
 
 With N > 1 (torchrun, one process per GPU) every rank runs its own replica of each workload: the
 (loop, batch, head) units are independent recurrences, so the path shards with no collective
@@ -40,7 +42,7 @@ from gated_delta_rule_looped_b200 import dist as gdist  # noqa: E402
 from gated_delta_rule_looped_b200 import inputs  # noqa: E402
 
 HEADLINE = "long_gdn"
-EXTRAS = ("gdn_prefill", "kda_prefill", "decode")
+EXTRAS = ("gdn_prefill", "kda_prefill", "decode", "fused_gdn_prefill")
 
 # Algorithmic work per token-head (d = 128), counted as dense multiply-adds (2 flops each).
 # Scalar gating, 64-token chunks: three d x d state products 6d^2, the four chunk-local
@@ -306,6 +308,61 @@ def run_prefill(w, args, world, sampler, peaks, peak_src, keep=False):
     return entry, None
 
 
+# The fused prologue and output gate (lt2_gdr_prefill_fused), per token-head: the step reads raw
+# q, k, v (bf16), the gate logits a, b (fp32) and the output gate logits z (bf16) and writes o
+# (bf16).  Run as separate passes around the plain mixer, the same steps move: q, k read and
+# written back normalised (4 x 256), a, b read and alpha, beta written (4 x 4), the mixer's own
+# bytes, and o, z read and o written back gated (3 x 256).
+FUSED_BYTES_PER_TOKEN_HEAD = 3 * 256 + 4 + 4 + 256 + 256
+UNFUSED_BYTES_PER_TOKEN_HEAD = 4 * 256 + 4 * 4 + BYTES_PER_TOKEN_HEAD["scalar"] + 3 * 256
+
+
+def run_fused(args, world, sampler, peaks, peak_src, alpha_scale=0.1):
+    """The gdn_prefill workload through lt2_gdr_prefill_fused with raw inputs (every fused step),
+    against the same steps as separate passes around the plain call (torch elementwise ops for
+    the prologue and the gate, the library's plain prefill for the mixer)."""
+    w = inputs.workload("gdn_prefill")
+    r = inputs.make_raw_inputs(w, seed=0, device="cuda")
+    o = torch.empty(r["v"].shape, dtype=torch.bfloat16, device="cuda")
+    S = torch.empty((w.T, w.B, w.H, w.d, w.d), dtype=torch.float32, device="cuda")
+
+    def fused():
+        lt2.prefill(r["q"], r["k"], r["v"], r["a"], r["b"], per_key=False, o=o, S_out=S, qk_l2norm=True,
+                    gate_logits=True, alpha_scale=alpha_scale, z=r["z"])
+
+    def unfused():
+        qn = (r["q"].float() * torch.rsqrt((r["q"].float() ** 2).sum(-1, keepdim=True).clamp_min(1e-24))).to(torch.bfloat16)
+        kn = (r["k"].float() * torch.rsqrt((r["k"].float() ** 2).sum(-1, keepdim=True).clamp_min(1e-24))).to(torch.bfloat16)
+        al = torch.exp(-torch.nn.functional.softplus(r["a"]) * alpha_scale)
+        be = torch.sigmoid(r["b"])
+        lt2.prefill(qn, kn, r["v"], al, be, per_key=False, o=o, S_out=S)
+        o.copy_((o.float() * torch.sigmoid(r["z"].float())).to(torch.bfloat16))
+    ms = timed(fused, args.steps, args.warmup, world, sampler, "fused_gdn_prefill")
+    check_device_status("fused_gdn_prefill")
+    ms_unfused = timed(unfused, max(3, args.steps // 4), args.warmup, world)
+    tokheads = w.T * w.B * w.H * w.L
+    entry = {"metric": "looped GDR prefill tokens*loops/s, fused prologue and output gate (gdn_prefill)",
+             "value": gdist.whole_job_rate(w.T * w.B * w.L, world, ms), "unit": "tokens*loops/s",
+             "ms_per_step": ms, "steps": args.steps,
+             "config": dict(config_of(w, world), fused="q/k L2 norm, alpha/beta from logits, sigmoid output gate",
+                            alpha_scale=alpha_scale),
+             "bytes_per_token_head": {"fused": FUSED_BYTES_PER_TOKEN_HEAD,
+                                      "unfused_passes": UNFUSED_BYTES_PER_TOKEN_HEAD},
+             "hbm": {"achieved": tokheads * FUSED_BYTES_PER_TOKEN_HEAD / (ms * 1e-3) / 1e9,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": tokheads * FUSED_BYTES_PER_TOKEN_HEAD / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "peak_source": f"{peak_src} HBM copy"},
+             "unfused_passes": {"ms_per_step": ms_unfused,
+                                "note": "the same steps as separate passes: torch elementwise prologue and "
+                                        "output gate around the library's plain prefill"},
+             "gpu_launches": args.steps * w.T}
+    if sampler is not None:
+        entry["clocks"] = sampler.summary(["fused_gdn_prefill"])
+    del r, o, S
+    torch.cuda.empty_cache()
+    return entry
+
+
 def run_e2e(w, x, dims, steps, warmup, world):
     """Same metric through the C ABI with host buffers: every step copies the inputs from
     pinned host memory, runs the prefill and reads o and the final state back."""
@@ -555,7 +612,9 @@ def main():
 
     # ---- the other workloads, each with its own timing, roofline and baseline ----
     for name in extras:
-        if name == "decode":
+        if name == "fused_gdn_prefill":
+            entry = run_fused(args, world, sampler, peaks, peak_src)
+        elif name == "decode":
             entry, (wd, xs, S_host) = run_decode(args, world, sampler, peaks, peak_src)
             if cpu:
                 v, threads, desc = oracle_decode_sample(wd, xs, S_host)
