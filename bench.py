@@ -42,7 +42,7 @@ from gated_delta_rule_looped_b200 import dist as gdist  # noqa: E402
 from gated_delta_rule_looped_b200 import inputs  # noqa: E402
 
 HEADLINE = "long_gdn"
-EXTRAS = ("gdn_prefill", "kda_prefill", "decode", "fused_gdn_prefill")
+EXTRAS = ("gdn_prefill", "kda_prefill", "decode", "fused_gdn_prefill", "swa_prefill")
 
 # Algorithmic work per token-head (d = 128), counted as dense multiply-adds (2 flops each).
 # Scalar gating, 64-token chunks: three d x d state products 6d^2, the four chunk-local
@@ -63,7 +63,8 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 
 KERNELS = {"scalar": ("gdr_prefill_tc_kernel", "gdr_prefill_tc.cu"),
            "per_key": ("gdr_prefill_kda_tc_kernel", "gdr_prefill_kda_tc.cu"),
-           "decode": ("gdr_decode_kernel", "gdr_decode.cu")}
+           "decode": ("gdr_decode_kernel", "gdr_decode.cu"),
+           "swa": ("swa_prefill_tc_kernel", "swa_prefill_tc.cu")}
 
 
 def kernel_sources(name, csrc=None):
@@ -363,6 +364,82 @@ def run_fused(args, world, sampler, peaks, peak_src, alpha_scale=0.1):
     return entry
 
 
+def swa_pairs(L, window):
+    """(query, key) pairs inside the windows of one unit: sum over t of min(t + 1, w)."""
+    w = min(window, L)
+    return w * (w + 1) // 2 + (L - w) * w
+
+
+def run_swa(args, world, sampler, peaks, peak_src):
+    """The sliding-window mixer (lt2_swa_prefill) on the swa_prefill workload, all T loops in one
+    launch.  Algorithmic work: 4 d flops per (query, key) pair inside a window (q.k and p v, 2 d
+    each); bytes: q, k, v read and o written once (4 x 256 per token-head, bf16)."""
+    w = inputs.swa_workload("swa_prefill")
+    x = inputs.make_swa_inputs(w, seed=0, device="cuda")
+    o = torch.empty_like(x["q"])
+    dims = lt2.lt2_swa_dims(w.T, w.B, w.H, w.L, w.d, w.window, 0.0, lt2.LT2_DTYPE_BF16, lt2.LT2_ALGO_AUTO,
+                            lt2.LT2_OUT_SAME)
+
+    def step():
+        st = lt2.lt2_swa_prefill(dims, x["q"], x["k"], x["v"], o)
+        if st != lt2.LT2_OK:
+            raise lt2.Lt2Error(st, "lt2_swa_prefill")
+    ms = timed(step, args.steps, args.warmup, world, sampler, "swa_prefill")
+    check_device_status("swa_prefill")
+    launch_s = ms * 1e-3
+    flops = w.units * swa_pairs(w.L, w.window) * 4 * w.d
+    nbytes = w.units * w.L * 4 * 2 * w.d
+    kernel, source = KERNELS["swa"]
+    traffic, traffic_note = traffic_for(kernel, source, nbytes)
+    tf = flops / launch_s / 1e12
+    gbs = nbytes / launch_s / 1e9
+    roof = {"bound": "tensor", "kernel": kernel, "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": tf / peaks["bf16_tflops"], "traffic": traffic,
+            "peak_source": f"{peak_src} bf16 dense burst",
+            "nominal": {"peak": NOMINAL_PEAKS["bf16_tflops"], "frac": tf / NOMINAL_PEAKS["bf16_tflops"]},
+            "algorithmic_per_launch": {"flop": flops, "bytes": nbytes,
+                                       "note": "4 d flops per (query, key) pair inside a window; the "
+                                               "kernel also multiplies the masked part of its 64-key "
+                                               "blocks, not counted"},
+            "hbm": {"achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"]}}
+    if traffic_note:
+        roof["traffic_note"] = traffic_note
+    entry = {"metric": "looped sliding-window attention prefill tokens*loops/s (swa_prefill)",
+             "value": gdist.whole_job_rate(w.T * w.B * w.L, world, ms), "unit": "tokens*loops/s",
+             "ms_per_step": ms, "steps": args.steps,
+             "config": {"workload": w.name, "T": w.T, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "window": w.window,
+                        "io_dtype": w.dtype, "scale": "1/sqrt(d)",
+                        "parallelism": f"replicas x{world} (independent units, no collective)",
+                        "l2": "inputs larger than L2 (no flush needed)"},
+             "roofline": roof, "gpu_launches": args.steps}
+    if sampler is not None:
+        entry["clocks"] = sampler.summary(["swa_prefill"])
+    del x, o
+    torch.cuda.empty_cache()
+    return entry
+
+
+def oracle_swa_sample(target_s=5.0):
+    """Time the fp64 oracle of the sliding-window mixer on this host (one thread): one whole unit
+    of swa_prefill, repeated until about `target_s` has passed."""
+    from oracle import swa as oswa
+    w = inputs.swa_workload("swa_prefill")
+    ws = inputs.swa_workload("swa_prefill", T=1, B=1, H=1)
+    x = {n: t.to(torch.float64).numpy()[0, 0, 0] for n, t in inputs.make_swa_inputs(ws, seed=1).items()}
+    rows, reps, L = 0, 0, w.L
+    t0 = time.perf_counter()
+    while True:
+        oswa.prefill(x["q"][:L], x["k"][:L], x["v"][:L], w.window)
+        rows += L
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= target_s or reps >= 100:
+            break
+    desc = (f"one (loop, batch, head) unit of swa_prefill, all {L} tokens, {reps} times; fp64 oracle, "
+            f"one query at a time")
+    return rows / dt / w.H, 1, desc
+
+
 def run_e2e(w, x, dims, steps, warmup, world):
     """Same metric through the C ABI with host buffers: every step copies the inputs from
     pinned host memory, runs the prefill and reads o and the final state back."""
@@ -614,6 +691,12 @@ def main():
     for name in extras:
         if name == "fused_gdn_prefill":
             entry = run_fused(args, world, sampler, peaks, peak_src)
+        elif name == "swa_prefill":
+            entry = run_swa(args, world, sampler, peaks, peak_src)
+            if cpu:
+                v, threads, desc = oracle_swa_sample()
+                entry["cpu_baseline"] = {"value": v, "unit": "tokens*loops/s", "cores": threads,
+                                         "kind": "oracle", "sample": desc}
         elif name == "decode":
             entry, (wd, xs, S_host) = run_decode(args, world, sampler, peaks, peak_src)
             if cpu:

@@ -43,6 +43,7 @@ EXPORTS = (
     "lt2_gdr_prefill_fused",
     "lt2_gdr_decode",
     "lt2_gdr_decode_fused",
+    "lt2_swa_prefill",
     "lt2_gdr_last_device_error",
     "lt2_status_string",
     "lt2_last_cuda_error_string",
@@ -62,6 +63,14 @@ class lt2_gdr_fused(ctypes.Structure):
     _fields_ = [("qk_l2norm", ctypes.c_int32), ("gate_logits", ctypes.c_int32),
                 ("alpha_scale", ctypes.c_float), ("reserved", ctypes.c_int32),
                 ("z", ctypes.c_void_p)]
+
+
+class lt2_swa_dims(ctypes.Structure):
+    """Sizes of a sliding-window attention prefill (include/lt2_gdr.h)."""
+    _fields_ = [("T", ctypes.c_int64), ("B", ctypes.c_int64), ("H", ctypes.c_int64),
+                ("L", ctypes.c_int64), ("d", ctypes.c_int64), ("window", ctypes.c_int64),
+                ("scale", ctypes.c_float), ("dtype", ctypes.c_int32), ("algo", ctypes.c_int32),
+                ("out_dtype", ctypes.c_int32)]
 
 
 def make_fused(qk_l2norm=False, gate_logits=False, alpha_scale=1.0, z=None):
@@ -115,6 +124,9 @@ def load_library(path):
         L.lt2_gdr_prefill_fused.restype = ctypes.c_int
         L.lt2_gdr_decode_fused.argtypes = [dims_p, fused_p, vp, vp, vp, fp, fp, fp, vp, vp]
         L.lt2_gdr_decode_fused.restype = ctypes.c_int
+    if hasattr(L, "lt2_swa_prefill"):
+        L.lt2_swa_prefill.argtypes = [ctypes.POINTER(lt2_swa_dims), vp, vp, vp, vp, vp]
+        L.lt2_swa_prefill.restype = ctypes.c_int
     L.lt2_gdr_last_device_error.argtypes = []
     L.lt2_gdr_last_device_error.restype = ctypes.c_int
     L.lt2_status_string.argtypes = [ctypes.c_int]
@@ -183,6 +195,10 @@ def lt2_gdr_decode_fused(dims, fused, q, k, v, alpha, beta, S, o, stream=None):
     return lib().lt2_gdr_decode_fused(ctypes.byref(dims), None if fused is None else ctypes.byref(fused),
                                       _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S), _p(o),
                                       _stream(stream))
+
+
+def lt2_swa_prefill(dims, q, k, v, o, stream=None):
+    return lib().lt2_swa_prefill(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(o), _stream(stream))
 
 
 def lt2_gdr_last_device_error():
@@ -342,3 +358,32 @@ def _decode(q, k, v, alpha, beta, S, per_key, o, out, stream, order, fused=None,
     if st != LT2_OK:
         raise Lt2Error(st, "lt2_gdr_decode")
     return o
+
+
+def swa_prefill(q, k, v, window, scale=None, algo=LT2_ALGO_AUTO, o=None, out=None, stream=None):
+    """Sliding-window attention over [T, B, H, L, d] CUDA tensors (lt2_swa_prefill): every token
+    attends to itself and the window - 1 tokens before it; ``scale`` multiplies q.k (None:
+    1/sqrt(d)).  Returns o, of the inputs' dtype or ``out`` ("f32" / "bf16")."""
+    import torch
+    _require_cuda(q)
+    if q.dim() != 5:
+        raise ValueError("q, k, v must be [T, B, H, L, d]")
+    dt = {torch.float32: LT2_DTYPE_F32, torch.bfloat16: LT2_DTYPE_BF16}.get(q.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    if scale is not None and not scale > 0:
+        raise ValueError("scale must be positive (None selects 1/sqrt(d))")
+    with torch.cuda.device(q.device):
+        dev = q.device
+        for name, t in (("q", q), ("k", k), ("v", v)):
+            _check(name, t, q.shape, q.dtype, dev)
+        odt = _out_torch_dtype(q.dtype, out)
+        _check("o", o, q.shape, odt, dev)
+        if o is None:
+            o = torch.empty(q.shape, dtype=odt, device=dev)
+        T, B, H, L, d = q.shape
+        dims = lt2_swa_dims(T, B, H, L, d, int(window), 0.0 if scale is None else float(scale), dt, algo, _OUT[out])
+        st = lt2_swa_prefill(dims, q, k, v, o, stream)
+        if st != LT2_OK:
+            raise Lt2Error(st, "lt2_swa_prefill")
+        return o

@@ -49,6 +49,28 @@ cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream);
 bool prefill_kda_tc_supports(int dtype_bf16, int dk, int dv);
 cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream);
 
+// Sliding-window attention prefill, every unit of every loop in one launch.
+struct SwaCall {
+    const void* q;
+    const void* k;
+    const void* v;
+    void* o;
+    int64_t units;     // T * B * H
+    int64_t L;         // >= 1
+    int64_t d;
+    int64_t window;    // >= 1
+    float scale;       // > 0 after defaulting
+    int dtype_bf16;
+    int out_bf16;
+    unsigned int* err;
+};
+// Tensor cores (bf16, d = 128): 128 queries per CTA, keys in blocks of 64, two CTAs per SM.
+bool swa_tc_supports(int dtype_bf16, int d);
+cudaError_t launch_swa_tc(const SwaCall& c, cudaStream_t stream);
+// CUDA cores (fp32 arithmetic, d <= 256): one warp per query.
+bool swa_cc_supports(int dtype_bf16, int d);
+cudaError_t launch_swa_cc(const SwaCall& c, cudaStream_t stream);
+
 #ifdef LT2_DEBUG
 // Fault injection of the debug build: the producer of every later launch stops before `chunk`.
 cudaError_t debug_set_skip_chunk_scalar(int chunk);

@@ -4,6 +4,7 @@
 
 #include <atomic>
 #include <initializer_list>
+#include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -374,6 +375,61 @@ lt2_status lt2_gdr_decode_fused(const lt2_gdr_dims* dims, const lt2_gdr_fused* f
     return LT2_OK;
 }
 
+lt2_status lt2_swa_prefill(const lt2_swa_dims* d, const void* q, const void* k, const void* v, void* o,
+                           void* stream)
+{
+    if (!d) return LT2_ERR_INVALID_ARGUMENT;
+    if (d->T < 0 || d->B < 0 || d->H < 0 || d->L < 0 || d->d < 1 || d->window < 1) return LT2_ERR_INVALID_ARGUMENT;
+    if (d->T >= kMaxDim || d->B >= kMaxDim || d->H >= kMaxDim || d->L >= kMaxDim) return LT2_ERR_INVALID_ARGUMENT;
+    if (d->dtype != LT2_DTYPE_F32 && d->dtype != LT2_DTYPE_BF16) return LT2_ERR_INVALID_ARGUMENT;
+    if (d->algo < LT2_ALGO_AUTO || d->algo > LT2_ALGO_CUDA_CORE) return LT2_ERR_INVALID_ARGUMENT;
+    if (d->out_dtype < LT2_OUT_SAME || d->out_dtype > LT2_OUT_BF16) return LT2_ERR_INVALID_ARGUMENT;
+    if (!(d->scale >= 0.f && d->scale <= 3.4e38f)) return LT2_ERR_INVALID_ARGUMENT;
+    const int bf16 = d->dtype == LT2_DTYPE_BF16 ? 1 : 0;
+    const int out_bf16 = d->out_dtype == LT2_OUT_BF16 || (d->out_dtype == LT2_OUT_SAME && bf16) ? 1 : 0;
+    if (d->d > 256) return LT2_ERR_UNSUPPORTED;
+    const __int128 units = (__int128)d->T * d->B * d->H;
+    const __int128 elems = units * d->L * d->d;
+    if (elems > ((__int128)1 << 62)) return LT2_ERR_INVALID_ARGUMENT;
+    const bool tc_ok = lt2::swa_tc_supports(bf16, (int)d->d);
+    if (d->algo == LT2_ALGO_TENSOR_CORE && !tc_ok) return LT2_ERR_UNSUPPORTED;
+    const bool tc = tc_ok && d->algo != LT2_ALGO_CUDA_CORE;
+    // grid sizes: units x query blocks of 128 (tensor cores) or queries / 4 (CUDA cores) < 2^31
+    if (tc ? units * ((d->L + 127) / 128) >= kMaxDim : units * d->L / 4 >= kMaxDim) return LT2_ERR_UNSUPPORTED;
+    const int64_t n = (int64_t)elems;
+    const int esz = bf16 ? 2 : 4, osz = out_bf16 ? 2 : 4;
+    if (!tensor_ok(q, n) || !tensor_ok(k, n) || !tensor_ok(v, n) || !tensor_ok(o, n)) return LT2_ERR_INVALID_ARGUMENT;
+    const Range ro = range_of(o, n * osz);
+    for (const void* in : {q, k, v})
+        if (overlap(ro, range_of(in, n * esz))) return LT2_ERR_INVALID_ARGUMENT;
+    if (n == 0) return LT2_OK;
+    lt2_status st = on_current_device({q, k, v, o});
+    if (st != LT2_OK) return st;
+
+    NvtxRange range("lt2_swa_prefill");
+    unsigned int* err = nullptr;
+    st = status_word(&err);
+    if (st != LT2_OK) return st;
+    lt2::SwaCall c;
+    c.q = q;
+    c.k = k;
+    c.v = v;
+    c.o = o;
+    c.units = (int64_t)units;
+    c.L = d->L;
+    c.d = d->d;
+    c.window = d->window < d->L ? d->window : d->L;
+    c.scale = d->scale > 0.f ? d->scale : 1.f / std::sqrt((float)d->d);
+    c.dtype_bf16 = bf16;
+    c.out_bf16 = out_bf16;
+    c.err = err;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = tc ? lt2::launch_swa_tc(c, s) : lt2::launch_swa_cc(c, s);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, tc ? "sliding-window prefill (tensor core)" : "sliding-window prefill (cuda core)");
+    return LT2_OK;
+}
+
 lt2_status lt2_gdr_last_device_error(void)
 {
     unsigned int* p = nullptr;
@@ -414,7 +470,7 @@ const char* lt2_status_string(lt2_status s)
 
 const char* lt2_last_cuda_error_string(void) { return t_cuda_error; }
 
-int lt2_gdr_version(void) { return 200; }
+int lt2_gdr_version(void) { return 210; }
 
 }  // extern "C"
 

@@ -11,6 +11,7 @@ Workloads (all synthetic; the pages run no public benchmark for this path):
   kda_prefill  T=4  B=2   H=16 L=16384  d=128  bf16 q/k/v, per-key alpha (a d_k vector)
   decode       T=4  B=256 H=16 L=1      d=128  bf16 q/k/v, state from a 4096-token prefill
   long_gdn     T=8  B=1   H=32 L=65536  d=128  bf16, alpha=beta=1 on 1% of the positions
+  swa_prefill  T=4  B=4   H=16 L=8192   d=128  bf16 q/k/v, sliding window w=512 (the other mixer)
 
 Distributions: q, k ~ N(0,1) then L2-normalised per (token, head) in fp32 (then cast);
 v ~ N(0,1); beta = sigmoid(N(0,1)); alpha = exp(-softplus(N(0,1)) * 0.1) except tiny_fp32
@@ -158,3 +159,46 @@ def make_raw_inputs(w, seed=0, device="cpu"):
     b = _normal((T, B, H, L), gen, device)
     S0 = _normal((T, B, H, d, d), gen, device) if w.s0 == "normal" else None
     return {"q": q, "k": k, "v": v, "z": z, "a": a, "b": b, "S0": S0}
+
+
+@dataclass(frozen=True)
+class SwaWorkload:
+    """A sliding-window attention prefill: T loops x B x H units of L tokens, head width d."""
+    name: str
+    T: int
+    B: int
+    H: int
+    L: int
+    d: int
+    window: int
+    dtype: str = "bf16"
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    @property
+    def units(self):
+        return self.T * self.B * self.H
+
+
+SWA_WORKLOADS = {
+    "swa_prefill": SwaWorkload("swa_prefill", 4, 4, 16, 8192, 128, 512),
+}
+
+
+def swa_workload(name, **overrides):
+    return replace(SWA_WORKLOADS[name], **overrides) if overrides else SWA_WORKLOADS[name]
+
+
+def make_swa_inputs(w, seed=0, device="cpu"):
+    """q, k, v ~ N(0,1) [T,B,H,L,d] in w's dtype (drawn in fp32 in that order, then cast): with
+    the default scale 1/sqrt(d) the scores q.k/sqrt(d) are ~N(0,1)."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    shape = (w.T, w.B, w.H, w.L, w.d)
+    q = _normal(shape, gen, device).to(w.torch_dtype)
+    k = _normal(shape, gen, device).to(w.torch_dtype)
+    v = _normal(shape, gen, device).to(w.torch_dtype)
+    return {"q": q, "k": k, "v": v}

@@ -123,7 +123,7 @@ typedef struct lt2_gdr_dims {
 } lt2_gdr_dims;
 
 /*
- * The steps on either side of the mixer, fused into its kernels (SURVEY f1): the prologue that
+ * The steps on either side of the mixer, fused into its kernels: the prologue that
  * turns a layer's raw projections into the recurrence's inputs, and the sigmoid output gate of
  * "LT2 transformer looped a tempo lineare", section "Dove il quadro si incrina" (a sigmoid gate
  * inside the loop keeps the state norm under control; the wispaper.ai blog, section "Critical
@@ -212,6 +212,47 @@ lt2_status lt2_gdr_decode_fused(const lt2_gdr_dims* dims, const lt2_gdr_fused* f
                                 const float* alpha, const float* beta,
                                 float* S, void* o,
                                 void* stream);
+
+/*
+ * The other mixer of "LT2 transformer looped a tempo lineare", section "Sostituire il motore":
+ * sliding-window (sparse) attention, every token looking at the w most recent positions, itself
+ * included; section "Il giro trasforma il calcolo in contesto": repeated over T loops, the window
+ * reaches back O(T w) tokens.  For every (loop, batch, head) unit and token t,
+ *     o_t = sum_{s = max(0, t-w+1) .. t} softmax_s(scale * q_t . k_s) v_s.
+ * The pages give no formula; this is the plainest reading (the softmax over the window of scaled
+ * dot products, scale = 1/sqrt(d) by default).  As for the linear mixer, every loop comes with its
+ * own q, k, v: the T loops of one call are independent.
+ */
+typedef struct lt2_swa_dims {
+    int64_t T;         /* loops                                                            */
+    int64_t B;         /* batch                                                            */
+    int64_t H;         /* heads                                                            */
+    int64_t L;         /* tokens per sequence                                              */
+    int64_t d;         /* head width (q, k and v): 1..256                                  */
+    int64_t window;    /* w >= 1 (w >= L is causal softmax attention)                      */
+    float scale;       /* multiplies q . k; 0 selects 1/sqrt(d)                            */
+    int32_t dtype;     /* lt2_dtype of q, k and v                                          */
+    int32_t algo;      /* lt2_algo: TENSOR_CORE = tcgen05/TMA kernel (bf16, d = 128 only),
+                          CUDA_CORE = fp32 arithmetic, one warp per query; AUTO picks the
+                          tensor-core kernel when it supports the shape                    */
+    int32_t out_dtype; /* lt2_out_dtype of o                                               */
+} lt2_swa_dims;
+
+/*
+ * Sliding-window prefill over all L tokens of every unit, all T loops in one call.
+ *   q, k, v    [T][B][H][L][d], dims->dtype, contiguous (device, read only)
+ *   o          [T][B][H][L][d], dims->out_dtype (device, written; must not alias an input)
+ *   stream     cudaStream_t of the current device
+ * Nothing is allocated; no workspace.  Returns LT2_OK once the launch is enqueued;
+ * LT2_ERR_INVALID_ARGUMENT (a NULL or misaligned pointer, a size out of range, window < 1, a
+ * negative or non-finite scale, o overlapping an input) or LT2_ERR_UNSUPPORTED (a forced
+ * algorithm that does not take the shape, or the device pointers not on the current device)
+ * before any launch; LT2_ERR_CUDA if the launch failed.  A bounded wait that gave up is reported
+ * by lt2_gdr_last_device_error().
+ */
+lt2_status lt2_swa_prefill(const lt2_swa_dims* dims,
+                           const void* q, const void* k, const void* v,
+                           void* o, void* stream);
 
 /*
  * The device-side status word of the CURRENT device (not an operation of the pages: the

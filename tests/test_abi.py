@@ -248,3 +248,65 @@ def test_fused_null_descriptor_is_the_plain_call(L):
     # validation runs the same way: a bad dims fails identically with and without a descriptor
     bad = D(dk=0)
     assert call_prefill_fused(bad, None) == call_prefill(bad) == lt2.LT2_ERR_INVALID_ARGUMENT
+
+
+# ---- the sliding-window mixer (lt2_swa_prefill) ------------------------------------------------
+
+def SD(**kw):
+    base = dict(T=2, B=1, H=2, L=64, d=32, window=8, scale=0.0, dtype=lt2.LT2_DTYPE_F32,
+                algo=lt2.LT2_ALGO_AUTO, out_dtype=lt2.LT2_OUT_SAME)
+    base.update(kw)
+    return lt2.lt2_swa_dims(**base)
+
+
+def call_swa(dims, **over):
+    q, k, v, o = addrs(4)
+    args = dict(q=q, k=k, v=v, o=o)
+    args.update(over)
+    return lt2.lt2_swa_prefill(dims, args["q"], args["k"], args["v"], args["o"], 0)
+
+
+def test_swa_dims_struct_layout():
+    assert ctypes.sizeof(lt2.lt2_swa_dims) == 6 * 8 + 4 * 4
+    assert lt2.lt2_swa_dims.scale.offset == 48
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(window=0), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(window=-3), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(d=0), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(L=-1), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(scale=-1.0), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(scale=float("nan")), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(scale=float("inf")), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(dtype=5), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(algo=7), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(out_dtype=3), lt2.LT2_ERR_INVALID_ARGUMENT),
+    (dict(d=257), lt2.LT2_ERR_UNSUPPORTED),
+    (dict(algo=lt2.LT2_ALGO_TENSOR_CORE), lt2.LT2_ERR_UNSUPPORTED),                           # fp32
+    (dict(algo=lt2.LT2_ALGO_TENSOR_CORE, dtype=lt2.LT2_DTYPE_BF16, d=64), lt2.LT2_ERR_UNSUPPORTED),
+    (dict(T=1 << 30, B=1 << 30, H=1 << 30), lt2.LT2_ERR_INVALID_ARGUMENT),
+])
+def test_swa_bad_dims(L, kw, status):
+    assert call_swa(SD(**kw)) == status
+
+
+def test_swa_null_dims_rejected(L):
+    assert L.lt2_swa_prefill(None, 1 << 40, 1 << 40, 1 << 40, 1 << 41, None) == lt2.LT2_ERR_INVALID_ARGUMENT
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "o"])
+def test_swa_null_or_misaligned_pointer_rejected(L, field):
+    assert call_swa(SD(), **{field: None}) == lt2.LT2_ERR_INVALID_ARGUMENT
+    assert call_swa(SD(), **{field: BASE + 20 * SPAN + 8}) == lt2.LT2_ERR_INVALID_ARGUMENT
+
+
+def test_swa_aliasing_rejected(L):
+    q, k, v, o = addrs(4)
+    assert call_swa(SD(), o=q) == lt2.LT2_ERR_INVALID_ARGUMENT
+    assert call_swa(SD(), o=v + 256) == lt2.LT2_ERR_INVALID_ARGUMENT
+
+
+def test_swa_empty_problem_is_a_noop(L):
+    assert call_swa(SD(T=0)) == lt2.LT2_OK
+    assert call_swa(SD(L=0), q=None, k=None, v=None, o=None) == lt2.LT2_OK
