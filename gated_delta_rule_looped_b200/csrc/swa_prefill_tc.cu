@@ -18,8 +18,13 @@
 // and at the end o = O / l.  Operands are bf16 (as the inputs; P rounded to bf16), accumulation
 // fp32 in tensor memory.
 //
-// Warps: 0 TMA producer (Q once, then K/V blocks through a two-stage ring), 1 MMA issuer,
-// 2-5 softmax (one query row per thread; the warp's TMEM lane quadrant is warp % 4) and output.
+// Warps: 0 TMA producer (Q once, then K and V blocks through two-stage rings of their own: a K
+// stage is free again as soon as Q K^T is done with it), 1 MMA issuer, 2-5 softmax (one query
+// row per thread; the warp's TMEM lane quadrant is warp % 4) and output.  The producer and the
+// issuer are single threads: every wait and every issue happens in lane 0, and the other 31 lanes
+// of those warps park at one __syncwarp until the end -- a lane-0 wait followed by a warp-wide
+// shuffle or sync costs several hundred cycles of reconvergence per step, which is more than the
+// tensor-core time of a block.
 // About 97 KB of shared memory and 256 TMEM columns per CTA, so two CTAs share an SM and one's
 // softmax runs under the other's MMAs.  Every mbarrier wait is bounded as in the prefills of the
 // linear mixer; on a timeout the CTA records it, drains its copies and MMAs, frees TMEM and exits.
@@ -45,29 +50,31 @@ constexpr int kThreads = 192;          // 6 warps
 constexpr uint64_t kTimeoutNs = kWaitTimeoutNs;
 
 // Shared memory (offsets from a 1024-byte aligned base), 128-byte swizzled panels of 64 bf16
-// columns: Q [2 panels][128 rows] (reused as the o staging tile at the end), and two stages of
-// K [2 panels][64 rows] and V [2 panels][64 rows].
+// columns: Q [2 panels][128 rows] (reused as the o staging tile at the end), and two-stage rings
+// of K [2 panels][64 rows] and of V [2 panels][64 rows].
 constexpr uint32_t Q_PANEL = kBM * 128;                 // 16 KB
 constexpr uint32_t KV_PANEL = kBN * 128;                // 8 KB
+constexpr uint32_t KV_STAGE = 2 * KV_PANEL;             // one K or V block
 constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_KV = OFF_Q + 2 * Q_PANEL;
-constexpr uint32_t STAGE = 4 * KV_PANEL;                // K panels, then V panels
-constexpr uint32_t OFF_BAR = OFF_KV + 2 * STAGE;
+constexpr uint32_t OFF_K = OFF_Q + 2 * Q_PANEL;
+constexpr uint32_t OFF_V = OFF_K + 2 * KV_STAGE;
+constexpr uint32_t OFF_BAR = OFF_V + 2 * KV_STAGE;
 enum Bar : uint32_t {
     B_Q = 0,          // Q landed
-    B_KV_FULL = 1,    // [2] K and V of a stage landed
-    B_KV_EMPTY = 3,   // [2] the MMAs are done with a stage
-    B_S_FULL = 5,     // S = Q K^T done
-    B_S_FREE = 6,     // the softmax warps have read S
-    B_P_FULL = 7,     // P written (and O rescaled when needed)
-    B_PV_DONE = 8,    // O += P V done
-    B_DRAIN = 9,      // [2] drain on abort (MMA issuer, producer)
-    B_COUNT = 11
+    B_K_FULL = 1,     // [2] K of a stage landed
+    B_K_EMPTY = 3,    // [2] Q K^T is done with a K stage
+    B_V_FULL = 5,     // [2] V of a stage landed
+    B_V_EMPTY = 7,    // [2] O += P V is done with a V stage
+    B_S_FULL = 9,     // S = Q K^T done
+    B_S_FREE = 10,    // the softmax warps have read S
+    B_P_FULL = 11,    // P written (and O rescaled when needed)
+    B_PV_DONE = 12,   // O += P V done
+    B_DRAIN = 13,     // drain on abort (MMA issuer)
+    B_COUNT = 14
 };
 constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + B_COUNT * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 16;
-constexpr uint32_t OFF_OKFLAG = OFF_ABORT + 16;         // [2] wait outcomes of the softmax group
-constexpr uint32_t SMEM_USED = OFF_OKFLAG + 16;
+constexpr uint32_t SMEM_USED = OFF_ABORT + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 
 // TMEM columns (lane = query row)
@@ -77,6 +84,26 @@ constexpr uint32_t TM_O = 128;         // O, fp32 (128 columns)
 constexpr uint32_t TM_COLS = 256;
 
 constexpr int NB_SOFT = 1;             // named barrier of the softmax warps
+constexpr int kSoftThreads = 128;
+
+// The softmax warps wait together: every thread polls the mbarrier itself (no lane waits while
+// the rest of its warp idles, so no reconvergence on the way out), then one barrier reduction
+// makes the outcome the group's -- if any thread gave up (timeout or abort), all of them see it
+// and leave the pipeline at the same step.
+struct SoftGroup {
+    volatile int* abort_flag;
+    unsigned int* err;
+    __device__ bool wait(uint32_t bar, uint32_t parity) const
+    {
+        const bool mine = mbar_wait(bar, parity, abort_flag, err, kTimeoutNs);
+        uint32_t all;
+        asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                     "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                     : "=r"(all) : "r"(mine ? 1u : 0u), "r"(NB_SOFT), "r"(kSoftThreads) : "memory");
+        return all != 0;
+    }
+    __device__ void sync() const { named_sync(NB_SOFT, kSoftThreads); }
+};
 
 // Instruction descriptor, kind::f16 with bf16 A and B, fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn)
@@ -163,7 +190,6 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t sb = (raw + 1023u) & ~1023u;
     uint8_t* sbase = smem_raw + (sb - raw);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + OFF_ABORT);
-    volatile int* okflags = reinterpret_cast<volatile int*>(sbase + OFF_OKFLAG);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -179,16 +205,8 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
-        mbar_init(bar_addr(sb, B_Q), 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(bar_addr(sb, B_KV_FULL + s), 1);
-            mbar_init(bar_addr(sb, B_KV_EMPTY + s), 1);
-            mbar_init(bar_addr(sb, B_DRAIN + s), 1);
-        }
-        mbar_init(bar_addr(sb, B_S_FULL), 1);
-        mbar_init(bar_addr(sb, B_S_FREE), 1);
-        mbar_init(bar_addr(sb, B_P_FULL), 1);
-        mbar_init(bar_addr(sb, B_PV_DONE), 1);
+        for (uint32_t b = 0; b < B_COUNT; ++b)
+            mbar_init(bar_addr(sb, b), b == B_S_FREE || b == B_P_FULL ? kSoftThreads : 1);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -208,100 +226,107 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (threadIdx.x == 0) dbg_ok((tmem & 0xFFFFu) + TM_COLS <= 512u && (tmem >> 16) == 0u, err);
 
     if (warp == 0) {
-        // ================= TMA producer: Q, then the K/V blocks of the window =================
-        int issued = 0;
-        uint32_t leader;
-        if (elect_one(leader)) {
+        // ================= TMA producer (one thread): Q, then K and V of the window =================
+        // K_j is released by Q K_j^T and V_j only by O += P_j V_j, one block later, so each ring
+        // advances on its own: step j issues K_j (once Q K_{j-2}^T is done), then V_{j-1} (once
+        // O += P_{j-3} V_{j-3} is done) -- the order in which the MMAs free their stages.
+        if (lane == 0) {
             const uint32_t qbar = bar_addr(sb, B_Q);
             mbar_arrive_expect_tx(qbar, 2 * Q_PANEL);
             tma_load_3d(sb + OFF_Q, &tm_q, 0, i0, unit, qbar);
             tma_load_3d(sb + OFF_Q + Q_PANEL, &tm_q, 64, i0, unit, qbar);
+            int k_issued = 0, v_issued = 0;
+            auto load = [&](bool is_v, int j) -> bool {
+                const int s = j & 1;
+                const uint32_t empty = bar_addr(sb, (is_v ? B_V_EMPTY : B_K_EMPTY) + s);
+                if (!mbar_wait(empty, ((j >> 1) & 1) ^ 1, abort_flag, err, kTimeoutNs)) return false;
+                const int32_t y = (j_first + j) * kBN;
+                if (dbg_ok(y < L && unit < p.units, err)) {
+                    const uint32_t fb = bar_addr(sb, (is_v ? B_V_FULL : B_K_FULL) + s);
+                    const uint32_t st = sb + (is_v ? OFF_V : OFF_K) + s * KV_STAGE;
+                    mbar_arrive_expect_tx(fb, KV_STAGE);
+                    tma_load_3d(st, is_v ? &tm_v : &tm_k, 0, y, unit, fb);
+                    tma_load_3d(st + KV_PANEL, is_v ? &tm_v : &tm_k, 64, y, unit, fb);
+                }
+                return true;
+            };
+            for (int j = 0; j <= nblk; ++j) {
+                if (j < nblk) {
+                    if (!load(false, j)) break;
+                    k_issued = j + 1;
+                }
+                if (j > 0) {
+                    if (!load(true, j - 1)) break;
+                    v_issued = j;
+                }
+            }
+            if (*abort_flag) {
+                // the copies in flight land before the CTA's memory goes away
+                mbar_wait(qbar, 0, abort_flag, err, kTimeoutNs / 4);
+                for (int j = k_issued - 2 < 0 ? 0 : k_issued - 2; j < k_issued; ++j)
+                    mbar_wait(bar_addr(sb, B_K_FULL + (j & 1)), (j >> 1) & 1, abort_flag, err, kTimeoutNs / 4);
+                for (int j = v_issued - 2 < 0 ? 0 : v_issued - 2; j < v_issued; ++j)
+                    mbar_wait(bar_addr(sb, B_V_FULL + (j & 1)), (j >> 1) & 1, abort_flag, err, kTimeoutNs / 4);
+            }
         }
         __syncwarp();
-        for (int idx = 0; idx < nblk; ++idx) {
-            const int s = idx & 1;
-            int free_ok = 0;
-            if (lane == 0) free_ok = mbar_wait(bar_addr(sb, B_KV_EMPTY + s), ((idx >> 1) & 1) ^ 1, abort_flag, err, kTimeoutNs);
-            if (!__shfl_sync(0xffffffffu, free_ok, 0)) break;
-            const int32_t y = (j_first + idx) * kBN;
-            if (elect_one(leader) && dbg_ok(y < L && unit < p.units, err)) {
-                const uint32_t fb = bar_addr(sb, B_KV_FULL + s);
-                mbar_arrive_expect_tx(fb, STAGE);
-                const uint32_t st = sb + OFF_KV + s * STAGE;
-                tma_load_3d(st, &tm_k, 0, y, unit, fb);
-                tma_load_3d(st + KV_PANEL, &tm_k, 64, y, unit, fb);
-                tma_load_3d(st + 2 * KV_PANEL, &tm_v, 0, y, unit, fb);
-                tma_load_3d(st + 3 * KV_PANEL, &tm_v, 64, y, unit, fb);
-            }
-            __syncwarp();
-            issued = idx + 1;
-        }
-        if (lane == 0 && *abort_flag) {
-            // the copies in flight land before the CTA's memory goes away
-            mbar_wait(bar_addr(sb, B_Q), 0, abort_flag, err, kTimeoutNs / 4);
-            for (int idx = issued - 2 < 0 ? 0 : issued - 2; idx < issued; ++idx)
-                mbar_wait(bar_addr(sb, B_KV_FULL + (idx & 1)), (idx >> 1) & 1, abort_flag, err, kTimeoutNs / 4);
-        }
     } else if (warp == 1) {
-        // ================= MMA issuer =================
-        uint32_t issuer = 0;
-        bool issued_any = false;
-        int qok = 0;
-        if (lane == 0) qok = mbar_wait(bar_addr(sb, B_Q), 0, abort_flag, err, kTimeoutNs);
-        bool ok = __shfl_sync(0xffffffffu, qok, 0) != 0;
-        // O += P V of block idx, once the softmax warps have written P
-        auto issue_pv = [&](int idx) -> bool {
-            int pok = 0;
-            if (lane == 0) pok = mbar_wait(bar_addr(sb, B_P_FULL), idx & 1, abort_flag, err, kTimeoutNs);
-            if (!__shfl_sync(0xffffffffu, pok, 0)) return false;
-            tc_fence_after();
-            if (elect_one(issuer)) {
-                const uint32_t vt = sb + OFF_KV + (idx & 1) * STAGE + 2 * KV_PANEL;
+        // ================= MMA issuer (one thread) =================
+        if (lane == 0) {
+            bool issued_any = false;
+            bool ok = mbar_wait(bar_addr(sb, B_Q), 0, abort_flag, err, kTimeoutNs);
+            // O += P_j V_j, once the softmax warps have written P_j and V_j has landed
+            auto issue_pv = [&](int j) -> bool {
+                if (!mbar_wait(bar_addr(sb, B_V_FULL + (j & 1)), (j >> 1) & 1, abort_flag, err, kTimeoutNs) ||
+                    !mbar_wait(bar_addr(sb, B_P_FULL), j & 1, abort_flag, err, kTimeoutNs))
+                    return false;
+                tc_fence_after();
+                const uint32_t vt = sb + OFF_V + (j & 1) * KV_STAGE;
+                #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     umma_f16_tmem_a(tmem + TM_O, tmem + TM_P + 8 * k, smem_desc_sw128(vt + k * 2048, KV_PANEL, 1024),
-                                    ID_PV, (idx > 0 || k > 0) ? 1u : 0u);
+                                    ID_PV, (j > 0 || k > 0) ? 1u : 0u);
                 umma_commit(bar_addr(sb, B_PV_DONE));
-                umma_commit(bar_addr(sb, B_KV_EMPTY + (idx & 1)));
-            }
-            __syncwarp();
-            return true;
-        };
-        for (int idx = 0; ok && idx < nblk; ++idx) {
-            const int s = idx & 1;
-            int kok = 0;
-            if (lane == 0)
-                kok = mbar_wait(bar_addr(sb, B_KV_FULL + s), (idx >> 1) & 1, abort_flag, err, kTimeoutNs) &&
-                      (idx == 0 || mbar_wait(bar_addr(sb, B_S_FREE), (idx - 1) & 1, abort_flag, err, kTimeoutNs));
-            if (!__shfl_sync(0xffffffffu, kok, 0)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            if (elect_one(issuer)) {
-                const uint32_t kt = sb + OFF_KV + s * STAGE;
+                umma_commit(bar_addr(sb, B_V_EMPTY + (j & 1)));
+                return true;
+            };
+            for (int j = 0; ok && j < nblk; ++j) {
+                // S = Q K_j^T into the single S buffer, once the softmax warps have read S_{j-1}
+                if (!mbar_wait(bar_addr(sb, B_K_FULL + (j & 1)), (j >> 1) & 1, abort_flag, err, kTimeoutNs) ||
+                    (j > 0 && !mbar_wait(bar_addr(sb, B_S_FREE), (j - 1) & 1, abort_flag, err, kTimeoutNs))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t kt = sb + OFF_K + (j & 1) * KV_STAGE;
+                #pragma unroll
                 for (int k = 0; k < 8; ++k)
                     umma_f16(tmem + TM_S, smem_desc_sw128(sb + OFF_Q + (k >> 2) * Q_PANEL + (k & 3) * 32, 16, 1024),
                              smem_desc_sw128(kt + (k >> 2) * KV_PANEL + (k & 3) * 32, 16, 1024), ID_QK, k > 0);
                 umma_commit(bar_addr(sb, B_S_FULL));
+                umma_commit(bar_addr(sb, B_K_EMPTY + (j & 1)));
+                issued_any = true;
+                if (j > 0 && !issue_pv(j - 1)) ok = false;
             }
-            __syncwarp();
-            issued_any = true;
-            if (idx > 0 && !issue_pv(idx - 1)) ok = false;
+            if (ok) ok = issue_pv(nblk - 1);
+            if (issued_any && !ok) {
+                // every MMA this thread issued completes before TMEM is released
+                umma_commit(bar_addr(sb, B_DRAIN));
+                mbar_wait(bar_addr(sb, B_DRAIN), 0, abort_flag, err, kTimeoutNs / 4);
+            }
         }
-        if (ok) ok = issue_pv(nblk - 1);
-        if (lane == issuer && issued_any && !ok) {
-            // every MMA this thread issued completes before TMEM is released
-            umma_commit(bar_addr(sb, B_DRAIN + 0));
-            mbar_wait(bar_addr(sb, B_DRAIN + 0), 0, abort_flag, err, kTimeoutNs / 4);
-        }
+        __syncwarp();
     } else {
         // ================= softmax and output (query row r, TMEM lane r) =================
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;
         const int64_t qi = static_cast<int64_t>(i0) + r;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
-        Group grp{NB_SOFT, 128, warp == 2 && lane == 0, okflags, 0, abort_flag, err};
-        const int64_t lo = qi - p.window + 1;                // first key of this row's window
+        const SoftGroup grp{abort_flag, err};
+        const bool leader = warp == 2 && lane == 0;
+        // this row's window relative to the CTA's first query: keys i0 + rel, rel in [wlo, whi]
+        const int64_t wlo = static_cast<int64_t>(r) - p.window + 1;
+        const int64_t whi = r < L - i0 ? r : L - 1 - i0;
         float m = -INFINITY, l = 0.f;                        // running maximum (log2 units), sum
         bool ok = true;
         for (int idx = 0; idx < nblk; ++idx) {
@@ -313,33 +338,44 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             float x[64];
             tmem_load_2x32(tmem + TM_S + lane_addr, tmem + TM_S + lane_addr + 32, x);
             tc_fence_before();
-            grp.sync();
-            if (grp.leader) mbar_arrive(bar_addr(sb, B_S_FREE));     // the next Q K^T may overwrite S
-            // the window, causality and the sequence end; log2-scaled scores
-            const int64_t kb = static_cast<int64_t>(j_first + idx) * kBN;
-            float bm = -INFINITY;
-            #pragma unroll
-            for (int c = 0; c < kBN; ++c) {
-                const int64_t key = kb + c;
-                const bool valid = key <= qi && key >= lo && key < L;
-                x[c] = valid ? x[c] * p.xscale : -INFINITY;
-                bm = fmaxf(bm, x[c]);
+            mbar_arrive(bar_addr(sb, B_S_FREE));             // all 128 read: the next Q K^T may overwrite S
+            // the window, causality and the sequence end as a column range [c_lo, c_hi] of this
+            // block; blocks inside every window of the warp skip the mask
+            const int64_t kb = static_cast<int64_t>(j_first + idx) * kBN - i0;
+            const int c_lo = static_cast<int>(wlo - kb < 0 ? 0 : (wlo - kb > kBN ? kBN : wlo - kb));
+            const int c_hi = static_cast<int>(whi - kb < -1 ? -1 : (whi - kb > kBN - 1 ? kBN - 1 : whi - kb));
+            if (!__all_sync(0xffffffffu, c_lo == 0 && c_hi == kBN - 1)) {
+                #pragma unroll
+                for (int c = 0; c < kBN; ++c) x[c] = c >= c_lo && c <= c_hi ? x[c] : -INFINITY;
             }
+            float mx[8];
+            #pragma unroll
+            for (int j = 0; j < 8; ++j) mx[j] = fmaxf(x[j], x[j + 8]);
+            #pragma unroll
+            for (int c = 16; c < kBN; c += 8) {
+                #pragma unroll
+                for (int j = 0; j < 8; ++j) mx[j] = fmaxf(mx[j], x[c + j]);
+            }
+            const float bm = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * p.xscale;
             // raise the row's reference maximum only when the block exceeds it by more than 8
             // (so P <= 2^8); O and l then shrink by 2^(m - m_new)
             const bool raise = bm > m + 8.f;
             const float mnew = raise ? bm : m;
             const float corr = raise && m != -INFINITY ? ex2_approx(m - mnew) : 1.f;
+            // p = 2^(x xscale - m); a masked score (-inf) gives 0, and a row that has seen no key
+            // yet (m = -inf) subtracts 0 instead
+            const float msub = mnew == -INFINITY ? 0.f : mnew;
             uint32_t pk[32];
-            float ps = 0.f;
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
             #pragma unroll
             for (int e = 0; e < 32; ++e) {
-                const float p0 = x[2 * e] == -INFINITY ? 0.f : ex2_approx(x[2 * e] - mnew);
-                const float p1 = x[2 * e + 1] == -INFINITY ? 0.f : ex2_approx(x[2 * e + 1] - mnew);
+                const float p0 = ex2_approx(fmaf(x[2 * e], p.xscale, -msub));
+                const float p1 = ex2_approx(fmaf(x[2 * e + 1], p.xscale, -msub));
                 pk[e] = pack_bf16x2(p0, p1);
-                ps += bf16_lo(pk[e]) + bf16_hi(pk[e]);           // the sum of what the MMA multiplies
+                ps[e & 3] += p0 + p1;
             }
-            l = l * corr + ps;
+            l = l * corr + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
             m = mnew;
             // P is single-buffered and O may need rescaling: the previous O += P V must be done
             if (idx > 0 && !grp.wait(bar_addr(sb, B_PV_DONE), (idx - 1) & 1)) {
@@ -352,8 +388,7 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tmem_st16(tmem + TM_P + lane_addr + 16, *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
             tmem_wait_st();
             tc_fence_before();
-            grp.sync();
-            if (grp.leader) mbar_arrive(bar_addr(sb, B_P_FULL));
+            mbar_arrive(bar_addr(sb, B_P_FULL));
         }
         // o = O / l after the last O += P V
         if (ok && grp.wait(bar_addr(sb, B_PV_DONE), (nblk - 1) & 1)) {
@@ -367,7 +402,7 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 // are clipped by the store
                 fence_proxy_async_smem();
                 grp.sync();
-                if (grp.leader) {
+                if (leader) {
                     if (dbg_ok(i0 < L && unit < p.units, err)) {
                         tma_store_3d(&tm_o, sb + OFF_Q, 0, i0, unit);
                         tma_store_3d(&tm_o, sb + OFF_Q + Q_PANEL, 64, i0, unit);

@@ -7,12 +7,12 @@ T loops the window reaches back O(T w) tokens.
 
 Tolerance, from the arithmetic: o_t is a convex combination of the v_s of its window, so every
 error is measured against max|v| of the call (not rms(o), which shrinks as the window widens while
-the first rows of a sequence stay as large as v).  The tensor-core kernel rounds each weight
-p_s = 2^(x_s - m) to bf16 (relative error <= 2^-9) and divides by the sum of the rounded weights:
-the result is the exact average under weights each off by <= 2^-8 of itself, hence within
-2^-8 max|v| of o_t; fp32 accumulation and the approximate exp2 (relative error ~2^-22) add far
-less.  The bar is twice that bound, 2^-7 max|v|, checked on an fp32 copy of o (the bf16 output is
-checked to be that copy rounded to nearest).  The CUDA-core path computes in fp32 with expf and is
+the first rows of a sequence stay as large as v).  The tensor-core kernel multiplies each
+weight p_s = 2^(x_s - m) rounded to bf16 (relative error <= 2^-9) and divides by the fp32 sum of
+the unrounded weights: o_t is off by sum_s w_s eps_s v_s with |eps_s| <= 2^-9, at most
+2^-9 max|v|; fp32 accumulation and the approximate exp2 (relative error ~2^-22) add far less.
+The bar, 2^-7 max|v|, leaves a margin of 4 over that bound; it is checked on an fp32 copy of o
+(the bf16 output is checked to be that copy rounded to nearest).  The CUDA-core path computes in fp32 with expf and is
 held to the library's fp32 bar, 1e-4 max|v|.
 """
 import numpy as np
