@@ -148,8 +148,7 @@ enum Bar : uint32_t {
 };
 constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + B_COUNT * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 16;
-constexpr uint32_t OFF_OKFLAG = OFF_ABORT + 16;
-static_assert(OFF_OKFLAG + 32 <= OFF_BAR + BAR_BYTES, "barrier area too small");
+static_assert(OFF_ABORT + 16 <= OFF_BAR + BAR_BYTES, "barrier area too small");
 
 constexpr int NB_PREP = 1, NB_CHAIN = 2, NB_CONV = 3;
 
@@ -671,7 +670,6 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
     const uint32_t sb = (raw + 1023u) & ~1023u;
     uint8_t* sbase = smem_raw + (sb - raw);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + OFF_ABORT);
-    volatile int* okflags = reinterpret_cast<volatile int*>(sbase + OFF_OKFLAG);
     auto gate = [&](int s) -> Gates* { return reinterpret_cast<Gates*>(sbase + OFF_GATES + s * GATE_STAGE); };
     auto sts = [&](uint32_t addr, uint4 v) { *reinterpret_cast<uint4*>(sbase + (addr - sb)) = v; };
 
@@ -773,8 +771,8 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         // ================= conversion (warps 1-3): decay factors, K/Q/V tiles =================
         const int w = warp - 1;
         const int t_begin = conv_begin(w), t_end = conv_begin(w + 1);
-        // one leader waits for the chunk's inputs; the conversion warps leave the loop together
-        Group grp{NB_CONV, 32 * kConv, warp == 1 && lane == 0, okflags + 4, 0, abort_flag, err};
+        // the conversion warps wait for the chunk's inputs together and leave the loop together
+        Group grp{NB_CONV, 32 * kConv, warp == 1 && lane == 0, abort_flag, err};
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;
             const uint32_t ph = (c / kStages) & 1;
@@ -817,7 +815,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         const int t = threadIdx.x - 128;
         const int q = warp - 4;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-        Group grp{NB_PREP, 128, t == 0, okflags + 0, 0, abort_flag, err};
+        Group grp{NB_PREP, 128, t == 0, abort_flag, err};
         float* adiag = reinterpret_cast<float*>(sbase + OFF_ADIAG);
         uint32_t gram_issuer = 0;
         int gram_issued = 0;
@@ -854,7 +852,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         const int h = (warp - 8) >> 2;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
         const bool leader = warp == 8 && lane == 0;
-        Group grp{NB_CHAIN, 256, leader, okflags + 2, 0, abort_flag, err};
+        Group grp{NB_CHAIN, 256, leader, abort_flag, err};
         bool ok = nchunks > 0;
         uint32_t ph_a = 0, ph_b = 0, ph_s = 0;
         if (ok) ok = grp.wait(bar_addr(sb, B_GATE_FULL + 0), 0);

@@ -42,10 +42,10 @@
 //                warp-level mma.sync), P T; writes [T; PT] for MMA_B
 //   warps 8-11   the S-dependent chain (its first thread issues MMA_A, MMA_B, MMA_C)
 //   warps 12-15  output epilogue: o = g (Q S) + P T X from TMEM to global memory
-// Every wait on an mbarrier is bounded (see mbar_wait) and made by one thread per group;
-// the group then meets at a named barrier and reads the outcome from shared memory, so a
-// timeout leaves every thread of the group on the same path.  On a timeout the CTA records
-// it in the device status word, drains its in-flight copies and MMAs, frees TMEM and exits.
+// Every wait on an mbarrier is bounded (see mbar_wait); a group's threads all poll and then
+// agree on the outcome through one barrier reduction, so a timeout leaves every thread of the
+// group on the same path.  On a timeout the CTA records it in the device status word, drains
+// its in-flight copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -121,7 +121,6 @@ enum Bar : uint32_t {
 };
 constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + B_COUNT * 8;        // tcgen05.alloc result
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 16;
-constexpr uint32_t OFF_OKFLAG = OFF_ABORT + 16;                  // [3 groups][2] wait outcomes
 
 // Named barriers (bar.sync ids; 0 is __syncthreads).
 constexpr int NB_PREP = 1;             // warps 4-7
@@ -274,7 +273,6 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t sb = (raw + 1023u) & ~1023u;        // 1024-aligned base (swizzle atoms)
     uint8_t* sbase = smem_raw + (sb - raw);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + OFF_ABORT);
-    volatile int* okflags = reinterpret_cast<volatile int*>(sbase + OFF_OKFLAG);
     auto gate = [&](int s) -> Gates* {
         return reinterpret_cast<Gates*>(sbase + OFF_GATES + s * GATE_STAGE);
     };
@@ -503,7 +501,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const int t = threadIdx.x - 128;            // 0..127 = TMEM lane
         const int q = warp - 4;                     // warp within the group
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-        Group grp{NB_PREP, 128, t == 0, okflags + 0, 0, abort_flag, err};
+        Group grp{NB_PREP, 128, t == 0, abort_flag, err};
         const uint32_t as = sb + OFF_AS, ps = sb + OFF_PS;
         float* adiag = reinterpret_cast<float*>(sbase + OFF_ADIAG);
         for (int c = 0; c < nchunks; ++c) {
@@ -577,7 +575,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const int j = threadIdx.x - 256;            // 0..127 = TMEM lane = d_v index
         const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
         const bool leader = j == 0;
-        Group grp{NB_CHAIN, 128, leader, okflags + 2, 0, abort_flag, err};
+        Group grp{NB_CHAIN, 128, leader, abort_flag, err};
         bool ok = nchunks > 0;
         // initial state: S0^T (fp32 in TMEM, pre-scaled by the first chunk's decay; fp16 copy)
         if (ok) ok = grp.wait(bar_addr(sb, B_GATE_FULL + 0), 0);
@@ -734,7 +732,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // ================= output epilogue: o = g (Q S) + P T X =================
         const int j = threadIdx.x - 384;            // TMEM lane = d_v index
         const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-        Group grp{NB_OUT, 128, j == 0, okflags + 4, 0, abort_flag, err};
+        Group grp{NB_OUT, 128, j == 0, abort_flag, err};
         bool fin = true;                             // every output so far is finite
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;

@@ -30,31 +30,30 @@ __device__ __forceinline__ void named_sync(int id, int nthreads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// A group of warps that waits through one leader: the leader makes the bounded waits, the
-// group meets at its named barrier and every thread reads the outcome.  Two outcome slots
-// alternate, so the leader never overwrites a slot another thread has yet to read.
+// A group of warps that waits together: every thread polls the mbarrier itself, then one
+// barrier reduction (bar.red.and) over the group's named barrier makes the outcome the group's --
+// if any thread gave up (timeout or abort) all of them see it, so the group always leaves a
+// pipeline at the same step.  (A single polling leader with the rest parked at the named barrier
+// costs the leader's warp a reconvergence per wait.)  `leader` names the one thread that makes
+// the group's single arrivals.
 struct Group {
     int nb;             // named barrier id
     int nthreads;
     bool leader;
-    volatile int* slots;
-    uint32_t k;
     volatile int* abort_flag;
     unsigned int* err;
 
     __device__ bool wait(uint32_t bar0, uint32_t par0, uint32_t bar1 = 0, uint32_t par1 = 0,
                          uint32_t bar2 = 0, uint32_t par2 = 0)
     {
-        volatile int* slot = slots + (k & 1u);
-        ++k;
-        if (leader) {
-            bool ok = mbar_wait(bar0, par0, abort_flag, err, kWaitTimeoutNs);
-            if (ok && bar1) ok = mbar_wait(bar1, par1, abort_flag, err, kWaitTimeoutNs);
-            if (ok && bar2) ok = mbar_wait(bar2, par2, abort_flag, err, kWaitTimeoutNs);
-            *slot = ok ? 1 : 0;
-        }
-        named_sync(nb, nthreads);
-        return *slot != 0;
+        bool ok = mbar_wait(bar0, par0, abort_flag, err, kWaitTimeoutNs);
+        if (ok && bar1) ok = mbar_wait(bar1, par1, abort_flag, err, kWaitTimeoutNs);
+        if (ok && bar2) ok = mbar_wait(bar2, par2, abort_flag, err, kWaitTimeoutNs);
+        uint32_t all;
+        asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                     "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                     : "=r"(all) : "r"(ok ? 1u : 0u), "r"(nb), "r"(nthreads) : "memory");
+        return all != 0;
     }
     __device__ void sync() { named_sync(nb, nthreads); }
 };

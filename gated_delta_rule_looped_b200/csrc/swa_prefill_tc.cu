@@ -86,24 +86,6 @@ constexpr uint32_t TM_COLS = 256;
 constexpr int NB_SOFT = 1;             // named barrier of the softmax warps
 constexpr int kSoftThreads = 128;
 
-// The softmax warps wait together: every thread polls the mbarrier itself (no lane waits while
-// the rest of its warp idles, so no reconvergence on the way out), then one barrier reduction
-// makes the outcome the group's -- if any thread gave up (timeout or abort), all of them see it
-// and leave the pipeline at the same step.
-struct SoftGroup {
-    volatile int* abort_flag;
-    unsigned int* err;
-    __device__ bool wait(uint32_t bar, uint32_t parity) const
-    {
-        const bool mine = mbar_wait(bar, parity, abort_flag, err, kTimeoutNs);
-        uint32_t all;
-        asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-                     "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-                     : "=r"(all) : "r"(mine ? 1u : 0u), "r"(NB_SOFT), "r"(kSoftThreads) : "memory");
-        return all != 0;
-    }
-    __device__ void sync() const { named_sync(NB_SOFT, kSoftThreads); }
-};
 
 // Instruction descriptor, kind::f16 with bf16 A and B, fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn)
@@ -322,8 +304,8 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const int r = 32 * q4 + lane;
         const int64_t qi = static_cast<int64_t>(i0) + r;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
-        const SoftGroup grp{abort_flag, err};
         const bool leader = warp == 2 && lane == 0;
+        Group grp{NB_SOFT, kSoftThreads, leader, abort_flag, err};
         // this row's window relative to the CTA's first query: keys i0 + rel, rel in [wlo, whi]
         const int64_t wlo = static_cast<int64_t>(r) - p.window + 1;
         const int64_t whi = r < L - i0 ? r : L - 1 - i0;
