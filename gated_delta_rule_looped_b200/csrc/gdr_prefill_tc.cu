@@ -35,12 +35,14 @@
 // magnitudes involved (|x| in [2^-14, 2^15]), so the inputs are not rounded again.
 //
 // CTA = one (loop, batch, head) unit, 16 warps:
-//   warp 0       TMA producer (and TMEM allocation)
+//   warp 0       TMEM allocation, TMA producer and issuer of the chain's MMAs (MMA_A, MMA_B,
+//                MMA_C): one loop that waits for each MMA's operands and issues it
 //   warp 1       chunk gates, fp16 conversion of K, and the Gram MMA [K; Q] K^T
 //   warps 2, 3   fp16 conversion of Q and of V
 //   warps 4-7    "prep": Gram epilogue, the 64x64 triangular solve (16x16 blocks with
 //                warp-level mma.sync), P T; writes [T; PT] for MMA_B
-//   warps 8-11   the S-dependent chain (its first thread issues MMA_A, MMA_B, MMA_C)
+//   warps 8-11   the S-dependent chain: each thread arrives on a 128-count barrier once its
+//                part of an MMA operand is in TMEM, and the issuer starts the MMA
 //   warps 12-15  output epilogue: o = g (Q S) + P T X from TMEM to global memory
 // Every wait on an mbarrier is bounded (see mbar_wait); a group's threads all poll and then
 // agree on the outcome through one barrier reduction, so a timeout leaves every thread of the
@@ -117,7 +119,10 @@ enum Bar : uint32_t {
     B_O_DONE = 25,     // output epilogue has read them
     B_DRAIN = 26,      // [2] drain on abort (chain, Gram issuer)
     B_Z = 28,          // output gate logits of a chunk landed in the staging tile (fused instance)
-    B_COUNT = 29
+    B_SH_READY = 29,   // the chain wrote the fp16 state copy (initial state, then after each chunk)
+    B_Y_READY = 30,    // the chain wrote (-g K S)^T: MMA_B may go
+    B_U_READY = 31,    // the chain wrote U~^T: MMA_C may go
+    B_COUNT = 32
 };
 constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + B_COUNT * 8;        // tcgen05.alloc result
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 16;
@@ -310,8 +315,11 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         mbar_init(bar_addr(sb, B_B_FULL), 1);
         mbar_init(bar_addr(sb, B_S_FULL), 1);
         mbar_init(bar_addr(sb, B_O_READY), 1);
-        mbar_init(bar_addr(sb, B_O_DONE), 1);
+        mbar_init(bar_addr(sb, B_O_DONE), 128);          // every output thread, once it has read TMEM
         mbar_init(bar_addr(sb, B_Z), 1);
+        mbar_init(bar_addr(sb, B_SH_READY), 128);        // every chain thread
+        mbar_init(bar_addr(sb, B_Y_READY), 128);
+        mbar_init(bar_addr(sb, B_U_READY), 128);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -340,38 +348,117 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (threadIdx.x == 0) dbg_ok((tmem & 0xFFFFu) + TM_COLS <= 512u && (tmem >> 16) == 0u, err);
 
     if (warp == 0) {
-        // ================= TMA producer =================
-        int issued = 0;
-        for (int c = 0; c < nchunks; ++c) {
+        // ================= TMA producer and the chain's MMA issuer =================
+        // The whole warp runs this loop in step -- every lane makes the same bounded waits -- and
+        // one elected lane issues each batch of copies or MMAs.  Per chunk c it issues MMA_A,
+        // MMA_B and MMA_C as soon as their operands are ready, then the TMA loads of chunk
+        // c + kStages into the stage MMA_C(c) frees.  (Issued from a branch on the lane index
+        // instead, the tcgen05 operands cannot stay in uniform registers and every batch costs
+        // several hundred cycles more.)
+        {
+            uint32_t issuer = 0;
+            int loaded = 0;                          // chunks whose K/Q/V loads were issued
+            bool producing = true;
+            auto produce = [&](int cc) -> bool {
 #ifdef LT2_DEBUG
-            if (c == g_debug_skip_chunk) break;
+                if (cc == g_debug_skip_chunk) producing = false;
 #endif
-            const int s = c % kStages;
-            const uint32_t ph = ((c / kStages) & 1) ^ 1;
-            int free_ok = 0;
-            if (lane == 0) free_ok = mbar_wait(bar_addr(sb, B_EMPTY + s), ph, abort_flag, err, kTimeoutNs);
-            if (!__shfl_sync(0xffffffffu, free_ok, 0)) break;
-            uint32_t leader;
-            if (elect_one(leader) && dbg_ok(c * kC < L && ug < p.units_total, err)) {
-                const uint32_t fb = bar_addr(sb, B_FULL + s);
-                mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                if (!producing) return true;
+                const int s = cc % kStages;
+                if (!mbar_wait(bar_addr(sb, B_EMPTY + s), ((cc / kStages) & 1) ^ 1, abort_flag, err, kTimeoutNs))
+                    return false;
+                if (elect_one(issuer) && dbg_ok(cc * kC < L && ug < p.units_total, err)) {
+                    const uint32_t fb = bar_addr(sb, B_FULL + s);
+                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    const uint32_t st = sb + OFF_KQV + s * STAGE_BYTES;
+                    const int32_t y = cc * kC;
+                    tma_load_3d(st, &tm_k, 0, y, ug, fb);
+                    tma_load_3d(st + 16384, &tm_k, 64, y, ug, fb);
+                    tma_load_3d(st + 8192, &tm_q, 0, y, ug, fb);
+                    tma_load_3d(st + 24576, &tm_q, 64, y, ug, fb);
+                    tma_load_3d(st + KQ_BYTES, &tm_v, 0, y, ug, fb);
+                    tma_load_3d(st + KQ_BYTES + 8192, &tm_v, 64, y, ug, fb);
+                }
+                loaded = cc + 1;
+                return true;
+            };
+            bool ok = true;
+            for (int cc = 0; ok && cc < kStages && cc < nchunks; ++cc) ok = produce(cc);
+            bool issued_any = false;
+            for (int c = 0; ok && c < nchunks; ++c) {
+                const int s = c % kStages;
                 const uint32_t st = sb + OFF_KQV + s * STAGE_BYTES;
-                const int32_t y = c * kC;
-                tma_load_3d(st, &tm_k, 0, y, ug, fb);
-                tma_load_3d(st + 16384, &tm_k, 64, y, ug, fb);
-                tma_load_3d(st + 8192, &tm_q, 0, y, ug, fb);
-                tma_load_3d(st + 24576, &tm_q, 64, y, ug, fb);
-                tma_load_3d(st + KQ_BYTES, &tm_v, 0, y, ug, fb);
-                tma_load_3d(st + KQ_BYTES + 8192, &tm_v, 64, y, ug, fb);
+                // --- MMA_A: (KQ S)^T = S^T [K;Q]^T, once the stage is converted, the fp16 state
+                // copy written and the output epilogue done with the previous chunk's columns ---
+                if (!mbar_wait(bar_addr(sb, B_CONV + s), (c / kStages) & 1, abort_flag, err, kTimeoutNs) ||
+                    !mbar_wait(bar_addr(sb, B_SH_READY), c & 1, abort_flag, err, kTimeoutNs) ||
+                    (c > 0 && !mbar_wait(bar_addr(sb, B_O_DONE), (c - 1) & 1, abort_flag, err, kTimeoutNs))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (elect_one(issuer)) {
+                    #pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t boff = (k >> 2) * 16384 + (k & 3) * 32;
+                        umma_f16_tmem_a(tmem + TM_AB, tmem + TM_SH + 8 * k, smem_desc_sw128(st + boff, 16, 1024),
+                                        ID_TK, k > 0);
+                    }
+                    umma_commit(bar_addr(sb, B_A_FULL));
+                }
+                issued_any = true;
+                // --- MMA_B: ([T;PT] X)^T = V^T [T;PT]^T + Y^T [T;PT]^T ---
+                const int tps = c & 1;
+                if (!mbar_wait(bar_addr(sb, B_Y_READY), c & 1, abort_flag, err, kTimeoutNs) ||
+                    !mbar_wait(bar_addr(sb, B_TP_FULL + tps), (c >> 1) & 1, abort_flag, err, kTimeoutNs)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (elect_one(issuer)) {
+                    const uint32_t tp = sb + OFF_TP + tps * TP_STAGE;
+                    const uint32_t vt = st + KQ_BYTES;
+                    #pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        umma_f16(tmem + TM_B, smem_desc_sw128(vt + k * 2048, 8192, 1024),
+                                 smem_desc_sw128(tp + k * 32, 16, 1024), ID_MK, k > 0);
+                    #pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        umma_f16_tmem_a(tmem + TM_B, tmem + TM_Y + 8 * k, smem_desc_sw128(tp + k * 32, 16, 1024),
+                                        ID_TK, 1);
+                    umma_commit(bar_addr(sb, B_B_FULL));
+                    umma_commit(bar_addr(sb, B_TP_EMPTY + tps));
+                }
+                // --- MMA_C: S^T += U~^T K ---
+                if (!mbar_wait(bar_addr(sb, B_U_READY), c & 1, abort_flag, err, kTimeoutNs)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (elect_one(issuer)) {
+                    #pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        umma_f16_tmem_a(tmem + TM_S, tmem + TM_U + 8 * k,
+                                        smem_desc_sw128(st + k * 2048, 16384, 1024), ID_TM, 1);
+                    umma_commit(bar_addr(sb, B_S_FULL));
+                    umma_commit(bar_addr(sb, B_EMPTY + s));
+                    mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));     // the chain is done with chunk c's gates
+                }
+                if (c + kStages < nchunks && !produce(c + kStages)) ok = false;
             }
-            __syncwarp();
-            issued = c + 1;
+            if (issued_any && lane == issuer) {
+                // every MMA this thread issued completes before TMEM is released (the chain may
+                // have left early on an abort elsewhere)
+                umma_commit(bar_addr(sb, B_DRAIN + 0));
+                mbar_wait(bar_addr(sb, B_DRAIN + 0), 0, abort_flag, err, kTimeoutNs / 4);
+            }
+            if (!ok && lane == 0) {
+                // the copies already in flight land before the CTA's memory goes away
+                for (int cc = loaded - kStages < 0 ? 0 : loaded - kStages; cc < loaded; ++cc)
+                    mbar_wait(bar_addr(sb, B_FULL + cc % kStages), (cc / kStages) & 1, abort_flag, err, kTimeoutNs / 4);
+            }
         }
-        if (lane == 0 && *abort_flag) {
-            // let the copies already in flight land before the CTA's memory goes away
-            for (int c = issued - kStages < 0 ? 0 : issued - kStages; c < issued; ++c)
-                mbar_wait(bar_addr(sb, B_FULL + c % kStages), (c / kStages) & 1, abort_flag, err, kTimeoutNs / 4);
-        }
+        __syncwarp();
     } else if (warp < 4) {
         // ================= gates (warp 1), conversion of K / Q / V (warps 1 / 2 / 3), Gram ===
         uint32_t gram_issuer = 0;
@@ -584,34 +671,10 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                                p.S0 ? p.S0 + static_cast<int64_t>(ug) * kD * kD + j : nullptr, gate(0)->gC);
             tc_fence_before();
         }
-        uint32_t drain_needed = 0;
-        uint32_t mma_issuer = 0;
+        if (ok) mbar_arrive(bar_addr(sb, B_SH_READY));      // MMA_A of chunk 0 may read it
         for (int c = 0; ok && c < nchunks; ++c) {
             const int s = c % kStages;
-            const uint32_t ph = (c / kStages) & 1;
             const Gates* gs = gate(s);
-            const uint32_t st = sb + OFF_KQV + s * STAGE_BYTES;
-            // --- MMA_A: (KQ S)^T = S^T [K;Q]^T ---
-            grp.sync();
-            if (warp == 8) {
-                int lok = 0;
-                if (leader)
-                    lok = mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs) &&
-                          (c == 0 || mbar_wait(bar_addr(sb, B_O_DONE), (c - 1) & 1, abort_flag, err, kTimeoutNs));
-                if (__shfl_sync(0xffffffffu, lok, 0)) {
-                    tc_fence_after();
-                    if (elect_one(mma_issuer)) {
-                        for (int k = 0; k < 8; ++k) {
-                            const uint32_t boff = (k >> 2) * 16384 + (k & 3) * 32;
-                            umma_f16_tmem_a(tmem + TM_AB, tmem + TM_SH + 8 * k,
-                                            smem_desc_sw128(st + boff, 16, 1024), ID_TK, k > 0);
-                        }
-                        umma_commit(bar_addr(sb, B_A_FULL));
-                    }
-                    __syncwarp();
-                    drain_needed = 1;
-                }
-            }
             ok = grp.wait(bar_addr(sb, B_A_FULL), c & 1);
             if (!ok) break;
             tc_fence_after();
@@ -631,29 +694,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 tmem_wait_st();
             }
             tc_fence_before();
-            grp.sync();
-            // --- MMA_B: ([T;PT] X)^T = V^T [T;PT]^T + Y^T [T;PT]^T ---
-            if (warp == 8) {
-                const int tps = c & 1;
-                int tok = 0;
-                if (leader) tok = mbar_wait(bar_addr(sb, B_TP_FULL + tps), (c >> 1) & 1, abort_flag, err, kTimeoutNs);
-                if (__shfl_sync(0xffffffffu, tok, 0)) {
-                    tc_fence_after();
-                    if (elect_one(mma_issuer)) {
-                        const uint32_t tp = sb + OFF_TP + tps * TP_STAGE;
-                        const uint32_t vt = st + KQ_BYTES;
-                        for (int k = 0; k < 4; ++k)
-                            umma_f16(tmem + TM_B, smem_desc_sw128(vt + k * 2048, 8192, 1024),
-                                     smem_desc_sw128(tp + k * 32, 16, 1024), ID_MK, k > 0);
-                        for (int k = 0; k < 4; ++k)
-                            umma_f16_tmem_a(tmem + TM_B, tmem + TM_Y + 8 * k, smem_desc_sw128(tp + k * 32, 16, 1024),
-                                            ID_TK, 1);
-                        umma_commit(bar_addr(sb, B_B_FULL));
-                        umma_commit(bar_addr(sb, B_TP_EMPTY + tps));
-                    }
-                    __syncwarp();
-                }
-            }
+            mbar_arrive(bar_addr(sb, B_Y_READY));
             ok = grp.wait(bar_addr(sb, B_B_FULL), c & 1);
             if (!ok) break;
             tc_fence_after();
@@ -674,20 +715,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 tmem_wait_st();
             }
             tc_fence_before();
-            grp.sync();
-            // --- MMA_C: S^T += U~^T K ---
-            if (warp == 8) {
-                tc_fence_after();
-                if (elect_one(mma_issuer)) {
-                    for (int k = 0; k < 4; ++k)
-                        umma_f16_tmem_a(tmem + TM_S, tmem + TM_U + 8 * k, smem_desc_sw128(st + k * 2048, 16384, 1024),
-                                        ID_TM, 1);
-                    umma_commit(bar_addr(sb, B_S_FULL));
-                    umma_commit(bar_addr(sb, B_EMPTY + s));
-                    mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));     // gates of chunk c consumed
-                }
-                __syncwarp();
-            }
+            mbar_arrive(bar_addr(sb, B_U_READY));
             // --- the new state ---
             const bool last = c + 1 == nchunks;
             const int s1 = (c + 1) % kStages;
@@ -702,7 +730,6 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                                                         p.S_out + static_cast<int64_t>(ug) * kD * kD + j);
                     if (__any_sync(0xffffffffu, !sfin) && lane == 0) atomicOr(err, kDevRange);
                 }
-                drain_needed = 0;
             } else {
                 const float gn = gate(s1)->gC;
                 #pragma unroll 1
@@ -721,12 +748,8 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
                 tmem_wait_st();
                 tc_fence_before();
+                mbar_arrive(bar_addr(sb, B_SH_READY));      // MMA_A of the next chunk may read it
             }
-        }
-        if (warp == 8 && lane == mma_issuer && drain_needed && !ok) {
-            // wait for every MMA this thread issued before TMEM is released
-            umma_commit(bar_addr(sb, B_DRAIN + 0));
-            mbar_wait(bar_addr(sb, B_DRAIN + 0), 0, abort_flag, err, kTimeoutNs / 4);
         }
     } else {
         // ================= output epilogue: o = g (Q S) + P T X =================
@@ -759,43 +782,46 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                                    static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, n,
                                    gated ? sbase + OFF_OST + (j >> 6) * 8192 + (j & 63) * 2 : nullptr);
                 tc_fence_before();
+                mbar_arrive(bar_addr(sb, B_O_DONE));
                 grp.sync();
-                if (j == 0) {
-                    mbar_arrive(bar_addr(sb, B_O_DONE));
-                    mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
-                }
+                if (j == 0) mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
                 continue;
             }
-            // o[r][j] = g_r (Q S)^T[j][r] + (P T X)^T[j][r], transposed through the staging tile
-            // (a warp writes 64 contiguous bytes per token) and written by the TMA unit as two
-            // 64 x 64 boxes; rows past L are clipped
+            // o[r][j] = g_r (Q S)^T[j][r] + (P T X)^T[j][r]: all 64 tokens of column j read from
+            // TMEM and rounded into registers first, so MMA_A of the next chunk may overwrite the
+            // columns while this thread transposes them through the staging tile (a warp writes
+            // 64 contiguous bytes per token), which the TMA unit writes out as two 64 x 64 boxes;
+            // rows past L are clipped
             uint8_t* ost = sbase + OFF_OST + (j >> 6) * 8192 + (j & 63) * 2;
-            #pragma unroll 1
-            for (int piece = 0; piece < 2; ++piece) {
-                float qp[64];                        // (Q S)^T, then (P T X)^T, for 32 tokens
-                tmem_load_2x32(tmem + TM_AB + lane_addr + 64 + 32 * piece,
-                               tmem + TM_B + lane_addr + 64 + 32 * piece, qp);
-                const float* gam = gs->gam + 32 * piece;
-                uint8_t* orow = ost + piece * 32 * 128;
+            uint32_t opk[32];                        // bf16 pairs: tokens 2e, 2e + 1
+            #pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float qp[32];                        // (Q S)^T, then (P T X)^T, for 16 tokens
+                tmem_load_2x16(tmem + TM_AB + lane_addr + 64 + 16 * q, tmem + TM_B + lane_addr + 64 + 16 * q, qp);
                 #pragma unroll
-                for (int e4 = 0; e4 < 32; e4 += 4) {
-                    const float4 g4 = *reinterpret_cast<const float4*>(gam + e4);
-                    float ov[4] = {g4.x * qp[e4 + 0] + qp[32 + e4 + 0], g4.y * qp[e4 + 1] + qp[32 + e4 + 1],
-                                   g4.z * qp[e4 + 2] + qp[32 + e4 + 2], g4.w * qp[e4 + 3] + qp[32 + e4 + 3]};
-                    #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(orow + (e4 + u) * 128);
-                        if (gated) ov[u] *= sigmoid_fast(__bfloat162float(*dst));     // z, then o in place
-                        fin &= is_finite(ov[u]);
-                        *dst = __float2bfloat16_rn(ov[u]);
+                for (int e = 0; e < 16; e += 2) {
+                    const int r = 16 * q + e;
+                    const float2 g2 = *reinterpret_cast<const float2*>(&gs->gam[r]);
+                    float o0 = g2.x * qp[e] + qp[16 + e];
+                    float o1 = g2.y * qp[e + 1] + qp[16 + e + 1];
+                    if (gated) {
+                        o0 *= sigmoid_fast(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(ost + r * 128)));
+                        o1 *= sigmoid_fast(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(ost + (r + 1) * 128)));
                     }
+                    fin &= is_finite(o0) & is_finite(o1);
+                    opk[r / 2] = pack_bf16x2(o0, o1);
                 }
             }
             tc_fence_before();
+            mbar_arrive(bar_addr(sb, B_O_DONE));     // this thread is done with the TMEM columns
+            #pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                *reinterpret_cast<uint16_t*>(ost + (2 * e) * 128) = static_cast<uint16_t>(opk[e] & 0xFFFFu);
+                *reinterpret_cast<uint16_t*>(ost + (2 * e + 1) * 128) = static_cast<uint16_t>(opk[e] >> 16);
+            }
             fence_proxy_async_smem();
             grp.sync();
             if (j == 0) {
-                mbar_arrive(bar_addr(sb, B_O_DONE));
                 mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
                 if (dbg_ok(t0 < L && ug < p.units_total, err)) {
                     tma_store_3d(&tm_o, sb + OFF_OST, 0, static_cast<int32_t>(t0), ug);

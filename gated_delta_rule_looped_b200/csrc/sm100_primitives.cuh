@@ -421,6 +421,12 @@ __device__ __forceinline__ float half_hi(uint32_t h2)
 {
     return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
 }
+// Two floats rounded to nearest-even bf16, packed (lo in the low half).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
 // The two bf16 halves of a 32-bit word (low half = lower element index) as floats, exactly.
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

@@ -21,10 +21,9 @@
 // Warps: 0 TMA producer (Q once, then K and V blocks through two-stage rings of their own: a K
 // stage is free again as soon as Q K^T is done with it), 1 MMA issuer, 2-5 softmax (one query
 // row per thread; the warp's TMEM lane quadrant is warp % 4) and output.  The producer and the
-// issuer are single threads: every wait and every issue happens in lane 0, and the other 31 lanes
-// of those warps park at one __syncwarp until the end -- a lane-0 wait followed by a warp-wide
-// shuffle or sync costs several hundred cycles of reconvergence per step, which is more than the
-// tensor-core time of a block.
+// issuer warps run their loops in step -- every lane makes the same bounded waits, so no lane
+// waits alone and no reconvergence follows -- and one elected lane issues each batch of copies
+// or MMAs (from a warp-uniform branch, so the tcgen05 operands stay in uniform registers).
 // About 97 KB of shared memory and 256 TMEM columns per CTA, so two CTAs share an SM and one's
 // softmax runs under the other's MMAs.  Every mbarrier wait is bounded as in the prefills of the
 // linear mixer; on a timeout the CTA records it, drains its copies and MMAs, frees TMEM and exits.
@@ -115,12 +114,6 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
-{
-    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&h);
-}
-
 // Softmax thread (query row r): O / l to the staging tile (bf16, 128-byte swizzled like Q, for
 // the TMA store) or, with an fp32 output, straight to global memory (row `o32`, null past L).
 __device__ __noinline__ void write_output(uint32_t tm_o, float inv_l, uint32_t stage, int r, float* o32,
@@ -208,22 +201,25 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (threadIdx.x == 0) dbg_ok((tmem & 0xFFFFu) + TM_COLS <= 512u && (tmem >> 16) == 0u, err);
 
     if (warp == 0) {
-        // ================= TMA producer (one thread): Q, then K and V of the window =================
+        // ================= TMA producer: Q, then K and V of the window =================
         // K_j is released by Q K_j^T and V_j only by O += P_j V_j, one block later, so each ring
         // advances on its own: step j issues K_j (once Q K_{j-2}^T is done), then V_{j-1} (once
         // O += P_{j-3} V_{j-3} is done) -- the order in which the MMAs free their stages.
-        if (lane == 0) {
+        {
+            uint32_t leader = 0;
             const uint32_t qbar = bar_addr(sb, B_Q);
-            mbar_arrive_expect_tx(qbar, 2 * Q_PANEL);
-            tma_load_3d(sb + OFF_Q, &tm_q, 0, i0, unit, qbar);
-            tma_load_3d(sb + OFF_Q + Q_PANEL, &tm_q, 64, i0, unit, qbar);
+            if (elect_one(leader)) {
+                mbar_arrive_expect_tx(qbar, 2 * Q_PANEL);
+                tma_load_3d(sb + OFF_Q, &tm_q, 0, i0, unit, qbar);
+                tma_load_3d(sb + OFF_Q + Q_PANEL, &tm_q, 64, i0, unit, qbar);
+            }
             int k_issued = 0, v_issued = 0;
             auto load = [&](bool is_v, int j) -> bool {
                 const int s = j & 1;
                 const uint32_t empty = bar_addr(sb, (is_v ? B_V_EMPTY : B_K_EMPTY) + s);
                 if (!mbar_wait(empty, ((j >> 1) & 1) ^ 1, abort_flag, err, kTimeoutNs)) return false;
                 const int32_t y = (j_first + j) * kBN;
-                if (dbg_ok(y < L && unit < p.units, err)) {
+                if (elect_one(leader) && dbg_ok(y < L && unit < p.units, err)) {
                     const uint32_t fb = bar_addr(sb, (is_v ? B_V_FULL : B_K_FULL) + s);
                     const uint32_t st = sb + (is_v ? OFF_V : OFF_K) + s * KV_STAGE;
                     mbar_arrive_expect_tx(fb, KV_STAGE);
@@ -242,7 +238,7 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     v_issued = j;
                 }
             }
-            if (*abort_flag) {
+            if (lane == leader && *abort_flag) {
                 // the copies in flight land before the CTA's memory goes away
                 mbar_wait(qbar, 0, abort_flag, err, kTimeoutNs / 4);
                 for (int j = k_issued - 2 < 0 ? 0 : k_issued - 2; j < k_issued; ++j)
@@ -253,8 +249,9 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ================= MMA issuer (one thread) =================
-        if (lane == 0) {
+        // ================= MMA issuer =================
+        {
+            uint32_t issuer = 0;
             bool issued_any = false;
             bool ok = mbar_wait(bar_addr(sb, B_Q), 0, abort_flag, err, kTimeoutNs);
             // O += P_j V_j, once the softmax warps have written P_j and V_j has landed
@@ -263,13 +260,16 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     !mbar_wait(bar_addr(sb, B_P_FULL), j & 1, abort_flag, err, kTimeoutNs))
                     return false;
                 tc_fence_after();
-                const uint32_t vt = sb + OFF_V + (j & 1) * KV_STAGE;
-                #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    umma_f16_tmem_a(tmem + TM_O, tmem + TM_P + 8 * k, smem_desc_sw128(vt + k * 2048, KV_PANEL, 1024),
-                                    ID_PV, (j > 0 || k > 0) ? 1u : 0u);
-                umma_commit(bar_addr(sb, B_PV_DONE));
-                umma_commit(bar_addr(sb, B_V_EMPTY + (j & 1)));
+                if (elect_one(issuer)) {
+                    const uint32_t vt = sb + OFF_V + (j & 1) * KV_STAGE;
+                    #pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        umma_f16_tmem_a(tmem + TM_O, tmem + TM_P + 8 * k,
+                                        smem_desc_sw128(vt + k * 2048, KV_PANEL, 1024), ID_PV,
+                                        (j > 0 || k > 0) ? 1u : 0u);
+                    umma_commit(bar_addr(sb, B_PV_DONE));
+                    umma_commit(bar_addr(sb, B_V_EMPTY + (j & 1)));
+                }
                 return true;
             };
             for (int j = 0; ok && j < nblk; ++j) {
@@ -280,18 +280,21 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     break;
                 }
                 tc_fence_after();
-                const uint32_t kt = sb + OFF_K + (j & 1) * KV_STAGE;
-                #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    umma_f16(tmem + TM_S, smem_desc_sw128(sb + OFF_Q + (k >> 2) * Q_PANEL + (k & 3) * 32, 16, 1024),
-                             smem_desc_sw128(kt + (k >> 2) * KV_PANEL + (k & 3) * 32, 16, 1024), ID_QK, k > 0);
-                umma_commit(bar_addr(sb, B_S_FULL));
-                umma_commit(bar_addr(sb, B_K_EMPTY + (j & 1)));
+                if (elect_one(issuer)) {
+                    const uint32_t kt = sb + OFF_K + (j & 1) * KV_STAGE;
+                    #pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        umma_f16(tmem + TM_S,
+                                 smem_desc_sw128(sb + OFF_Q + (k >> 2) * Q_PANEL + (k & 3) * 32, 16, 1024),
+                                 smem_desc_sw128(kt + (k >> 2) * KV_PANEL + (k & 3) * 32, 16, 1024), ID_QK, k > 0);
+                    umma_commit(bar_addr(sb, B_S_FULL));
+                    umma_commit(bar_addr(sb, B_K_EMPTY + (j & 1)));
+                }
                 issued_any = true;
                 if (j > 0 && !issue_pv(j - 1)) ok = false;
             }
             if (ok) ok = issue_pv(nblk - 1);
-            if (issued_any && !ok) {
+            if (issued_any && !ok && lane == issuer) {
                 // every MMA this thread issued completes before TMEM is released
                 umma_commit(bar_addr(sb, B_DRAIN));
                 mbar_wait(bar_addr(sb, B_DRAIN), 0, abort_flag, err, kTimeoutNs / 4);
