@@ -23,6 +23,7 @@ LT2_ERR_CUDA = 4
 LT2_ERR_DEVICE_TIMEOUT = 5
 LT2_ERR_RANGE = 6
 LT2_ERR_DEVICE_CHECK = 7
+LT2_ERR_SEQLENS = 8
 
 LT2_DTYPE_F32 = 0
 LT2_DTYPE_BF16 = 1
@@ -43,6 +44,7 @@ EXPORTS = (
     "lt2_gdr_prefill_fused",
     "lt2_gdr_decode",
     "lt2_gdr_decode_fused",
+    "lt2_gdr_prefill_varlen",
     "lt2_swa_prefill",
     "lt2_gdr_last_device_error",
     "lt2_status_string",
@@ -124,6 +126,10 @@ def load_library(path):
         L.lt2_gdr_prefill_fused.restype = ctypes.c_int
         L.lt2_gdr_decode_fused.argtypes = [dims_p, fused_p, vp, vp, vp, fp, fp, fp, vp, vp]
         L.lt2_gdr_decode_fused.restype = ctypes.c_int
+    if hasattr(L, "lt2_gdr_prefill_varlen"):
+        L.lt2_gdr_prefill_varlen.argtypes = [dims_p, ctypes.POINTER(lt2_gdr_fused), vp, vp, vp, vp, fp, fp, fp, vp,
+                                             fp, vp, ctypes.c_size_t, vp]
+        L.lt2_gdr_prefill_varlen.restype = ctypes.c_int
     if hasattr(L, "lt2_swa_prefill"):
         L.lt2_swa_prefill.argtypes = [ctypes.POINTER(lt2_swa_dims), vp, vp, vp, vp, vp]
         L.lt2_swa_prefill.restype = ctypes.c_int
@@ -195,6 +201,13 @@ def lt2_gdr_decode_fused(dims, fused, q, k, v, alpha, beta, S, o, stream=None):
     return lib().lt2_gdr_decode_fused(ctypes.byref(dims), None if fused is None else ctypes.byref(fused),
                                       _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S), _p(o),
                                       _stream(stream))
+
+
+def lt2_gdr_prefill_varlen(dims, fused, cu_seqlens, q, k, v, alpha, beta, S0, o, S_out, workspace=None,
+                           workspace_bytes=0, stream=None):
+    return lib().lt2_gdr_prefill_varlen(ctypes.byref(dims), None if fused is None else ctypes.byref(fused),
+                                        _p(cu_seqlens), _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(o),
+                                        _p(S_out), _p(workspace), int(workspace_bytes), _stream(stream))
 
 
 def lt2_swa_prefill(dims, q, k, v, o, stream=None):
@@ -387,3 +400,50 @@ def swa_prefill(q, k, v, window, scale=None, algo=LT2_ALGO_AUTO, o=None, out=Non
         if st != LT2_OK:
             raise Lt2Error(st, "lt2_swa_prefill")
         return o
+
+
+def prefill_varlen(q, k, v, alpha, beta, cu_seqlens, S0=None, per_key=None, algo=LT2_ALGO_AUTO, o=None,
+                   S_out=None, out=None, stream=None, order="delta_first", qk_l2norm=False, gate_logits=False,
+                   alpha_scale=1.0, z=None):
+    """The looped prefill over packed sequences (lt2_gdr_prefill_varlen): q, k, v [T, H, Ntot, d],
+    alpha [T, H, Ntot] (or [..., d] per key), beta [T, H, Ntot], cu_seqlens an int64 CUDA tensor of
+    B + 1 offsets.  Returns (o [T, H, Ntot, d], S_out [T, B, H, d, d]); the other arguments as in
+    ``prefill``."""
+    import torch
+    _require_cuda(q)
+    if q.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [T, H, Ntot, d]")
+    if cu_seqlens.dtype != torch.int64 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must be a 1-D int64 tensor of B + 1 offsets")
+    fused = None
+    if qk_l2norm or gate_logits or z is not None:
+        fused = make_fused(qk_l2norm, gate_logits, alpha_scale, z)
+    with torch.cuda.device(q.device):
+        T, H, N, dk = q.shape
+        dv = v.shape[-1]
+        B = cu_seqlens.numel() - 1
+        dt = {torch.float32: LT2_DTYPE_F32, torch.bfloat16: LT2_DTYPE_BF16}.get(q.dtype)
+        if dt is None:
+            raise ValueError(f"unsupported dtype {q.dtype}")
+        if per_key is None:
+            per_key = alpha.dim() == 4
+        dims = make_dims(T, B, H, N, dk, dv, dt, _gate(per_key, order), algo, _OUT[out])
+        dev = q.device
+        _check("cu_seqlens", cu_seqlens, (B + 1,), torch.int64, dev)
+        _check("k", k, q.shape, q.dtype, dev)
+        _check("v", v, (T, H, N, dv), q.dtype, dev)
+        _check("alpha", alpha, (T, H, N) + ((dk,) if per_key else ()), torch.float32, dev)
+        _check("beta", beta, (T, H, N), torch.float32, dev)
+        _check("z", z, (T, H, N, dv), q.dtype, dev)
+        for name, S in (("S0", S0), ("S_out", S_out)):
+            _check(name, S, (T, B, H, dk, dv), torch.float32, dev)
+        odt = _out_torch_dtype(q.dtype, out)
+        _check("o", o, (T, H, N, dv), odt, dev)
+        if o is None:
+            o = torch.empty((T, H, N, dv), dtype=odt, device=dev)
+        if S_out is None:
+            S_out = torch.empty((T, B, H, dk, dv), dtype=torch.float32, device=dev)
+        st = lt2_gdr_prefill_varlen(dims, fused, cu_seqlens, q, k, v, alpha, beta, S0, o, S_out, None, 0, stream)
+        if st != LT2_OK:
+            raise Lt2Error(st, "lt2_gdr_prefill_varlen")
+        return o, S_out

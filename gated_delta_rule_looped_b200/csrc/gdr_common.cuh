@@ -15,6 +15,7 @@ enum : unsigned int {
     kDevTimeout = 1u,
     kDevRange = 2u,
     kDevCheck = 4u,
+    kDevSeqlens = 8u,   // a packed sequence's offsets are out of order or past the packed length
 };
 
 // Device-side invariant checks of the debug build (LT2_DEBUG): a failed check records kDevCheck
@@ -53,6 +54,10 @@ struct LoopSlice {
     int gate_logits;     // alpha, beta hold logits: alpha = exp(-softplus(a) c), beta = sigmoid(b)
     float alpha_scale;   // c
     const void* z;       // output gate logits (layout and dtype of v), or null
+    // packed sequences: unit u = (sequence u / H, head u % H) holds tokens cu[b] .. cu[b+1]-1 of
+    // rows [H][L] (L is then the packed length); null: every unit has its own L rows
+    const int64_t* cu = nullptr;
+    int H = 0;
 };
 
 // The fused prologue and output gate, in fp32: the same formulas on every path.

@@ -34,6 +34,10 @@ struct TcCall {
     int gate_logits;
     float alpha_scale;
     const void* z;
+    // packed sequences: device offsets [units_per_loop / H + 1] (null: fixed length L); then L
+    // is the packed length Ntot and q/k/v/o/z are [T][H][Ntot][128], alpha/beta [T][H][Ntot]
+    const int64_t* cu_seqlens = nullptr;
+    int64_t H = 0;
 };
 // The fused steps of a call as the template argument of the tensor-core kernels' instances.
 enum FuseBits : int { kFuseNorm = 1, kFuseLogits = 2, kFuseGate = 4 };

@@ -59,12 +59,24 @@ __global__ void __launch_bounds__(256) gdr_prefill_seq_kernel(LoopSlice p, int u
     float* saqk = sqk + kTile;                     // [kTile]  (alpha.q).k
     float* red = saqk + kTile;                     // [2][2][8][kCols]
 
-    const T* q = static_cast<const T*>(p.q) + u * p.L * dk;
-    const T* k = static_cast<const T*>(p.k) + u * p.L * dk;
-    const T* v = static_cast<const T*>(p.v) + u * p.L * dv;
-    const float* al = p.alpha + u * p.L * na;
-    const float* be = p.beta + u * p.L;
-    To* o = static_cast<To*>(p.o) + u * p.L * dv;
+    // the unit's first row and length: its own L rows, or a packed sequence's tokens
+    int64_t row0 = u * p.L, Lu = p.L;
+    if (p.cu) {
+        const int64_t b = u / p.H, h = u - b * p.H;
+        const int64_t c0 = p.cu[b], c1 = p.cu[b + 1];
+        if (!(0 <= c0 && c0 <= c1 && c1 <= p.L)) {
+            if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(p.err, kDevSeqlens);
+            return;
+        }
+        row0 = h * p.L + c0;
+        Lu = c1 - c0;
+    }
+    const T* q = static_cast<const T*>(p.q) + row0 * dk;
+    const T* k = static_cast<const T*>(p.k) + row0 * dk;
+    const T* v = static_cast<const T*>(p.v) + row0 * dv;
+    const float* al = p.alpha + row0 * na;
+    const float* be = p.beta + row0;
+    To* o = static_cast<To*>(p.o) + row0 * dv;
 
     const int r0 = w * rpw;
     float s[16];
@@ -74,8 +86,8 @@ __global__ void __launch_bounds__(256) gdr_prefill_seq_kernel(LoopSlice p, int u
         s[m] = (m < rpw && active && S0) ? S0[(int64_t)(r0 + m) * dv + j0 + c] : 0.f;
 
     int buf = 0;
-    for (int64_t t0 = 0; t0 < p.L; t0 += kTile) {
-        const int nt = (p.L - t0 < kTile) ? (int)(p.L - t0) : kTile;
+    for (int64_t t0 = 0; t0 < Lu; t0 += kTile) {
+        const int nt = (Lu - t0 < kTile) ? (int)(Lu - t0) : kTile;
         __syncthreads();   // previous tile fully consumed
         // k, q (raw), alpha and beta of the tile; with gate logits, alpha = exp(-softplus(a) c)
         // and beta = sigmoid(b) (the fused prologue)
@@ -175,7 +187,7 @@ __global__ void __launch_bounds__(256) gdr_prefill_seq_kernel(LoopSlice p, int u
             if (w == 0 && active) {
                 float ov = F - bt * qke * E + bt * sqk[tt] * vc;
                 if (p.z)        // the fused output gate
-                    ov *= sigmoid_f32(to_f32(static_cast<const T*>(p.z)[(u * p.L + t0 + tt) * dv + j0 + c]));
+                    ov *= sigmoid_f32(to_f32(static_cast<const T*>(p.z)[(row0 + t0 + tt) * dv + j0 + c]));
                 o[(t0 + tt) * dv + j0 + c] = from_f32<To>(ov);
             }
         }

@@ -162,6 +162,12 @@ struct Params {
     int qk_norm;
     int gate_logits;
     float alpha_scale;
+    // packed sequences (the varlen instances): q/k/v/o [T][H][Ntot][128], gates [T][H][Ntot], CTA
+    // = (sequence b, head h) of loop `loop`, tokens cu[b] .. cu[b+1]-1
+    const int64_t* cu;
+    int64_t Ntot;
+    int H;
+    int loop;
 };
 
 #ifdef LT2_DEBUG
@@ -264,7 +270,7 @@ __device__ __noinline__ void gram_epilogue_unfactored(uint32_t tm_row, const Gat
 // gate (the logits z of a chunk are loaded by TMA into the o staging tile, and o <- sigmoid(z) o
 // is applied as the tile is written).  One instance per combination, so that a call carries the
 // code of the steps it uses only; kF = 0 compiles exactly as without them.
-template <int kF>
+template <int kF, bool kVar>
 __global__ void __launch_bounds__(kThreads, 1)
 gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -289,10 +295,26 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t L = p.L;
-    const int nchunks = static_cast<int>((L + kC - 1) / kC);
-    const int ug = p.unit0 + blockIdx.x;               // global head-unit index
+    const int ug = p.unit0 + blockIdx.x;               // global head-unit index (states)
     unsigned int* err = p.err;
+    // Where the unit's tokens live: the TMA unit coordinate zc, the first row y0 and the length L
+    // of the unit, and the element index gbase of its first token in the gate arrays (and, times
+    // 128, in o).  Packed sequences take them from the offsets; a bad pair of offsets is reported
+    // and the CTA does nothing.
+    int32_t zc = ug;
+    int64_t y0 = 0, L = p.L, gbase = static_cast<int64_t>(ug) * p.L;
+    bool seq_ok = true;
+    if constexpr (kVar) {
+        const int b = blockIdx.x / p.H, h = blockIdx.x - b * p.H;
+        const int64_t c0 = p.cu[b], c1 = p.cu[b + 1];
+        seq_ok = 0 <= c0 && c0 <= c1 && c1 <= p.Ntot;
+        if (!seq_ok && threadIdx.x == 0) atomicOr(err, kDevSeqlens);
+        zc = p.loop * p.H + h;
+        y0 = seq_ok ? c0 : 0;
+        L = seq_ok ? c1 - c0 : 0;
+        gbase = static_cast<int64_t>(zc) * p.Ntot + y0;
+    }
+    const int nchunks = static_cast<int>((L + kC - 1) / kC);
 
     // ---- set-up: barriers, TMEM ----
     if (threadIdx.x == 0) {
@@ -367,17 +389,17 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 const int s = cc % kStages;
                 if (!mbar_wait(bar_addr(sb, B_EMPTY + s), ((cc / kStages) & 1) ^ 1, abort_flag, err, kTimeoutNs))
                     return false;
-                if (elect_one(issuer) && dbg_ok(cc * kC < L && ug < p.units_total, err)) {
+                if (elect_one(issuer) && dbg_ok(cc * kC < L && zc < p.units_total, err)) {
                     const uint32_t fb = bar_addr(sb, B_FULL + s);
                     mbar_arrive_expect_tx(fb, STAGE_BYTES);
                     const uint32_t st = sb + OFF_KQV + s * STAGE_BYTES;
-                    const int32_t y = cc * kC;
-                    tma_load_3d(st, &tm_k, 0, y, ug, fb);
-                    tma_load_3d(st + 16384, &tm_k, 64, y, ug, fb);
-                    tma_load_3d(st + 8192, &tm_q, 0, y, ug, fb);
-                    tma_load_3d(st + 24576, &tm_q, 64, y, ug, fb);
-                    tma_load_3d(st + KQ_BYTES, &tm_v, 0, y, ug, fb);
-                    tma_load_3d(st + KQ_BYTES + 8192, &tm_v, 64, y, ug, fb);
+                    const int32_t y = static_cast<int32_t>(y0 + cc * kC);
+                    tma_load_3d(st, &tm_k, 0, y, zc, fb);
+                    tma_load_3d(st + 16384, &tm_k, 64, y, zc, fb);
+                    tma_load_3d(st + 8192, &tm_q, 0, y, zc, fb);
+                    tma_load_3d(st + 24576, &tm_q, 64, y, zc, fb);
+                    tma_load_3d(st + KQ_BYTES, &tm_v, 0, y, zc, fb);
+                    tma_load_3d(st + KQ_BYTES + 8192, &tm_v, 64, y, zc, fb);
                 }
                 loaded = cc + 1;
                 return true;
@@ -471,8 +493,8 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             for (int i = 0; i < 2; ++i) {
                 const int64_t tok = static_cast<int64_t>(cn) * kC + lane + 32 * i;
                 const bool valid = cn < nchunks && tok < L;
-                a_nx[i] = valid ? p.alpha[ug * L + tok] : 1.f;
-                b_nx[i] = valid ? p.beta[ug * L + tok] : 0.f;
+                a_nx[i] = valid ? p.alpha[gbase + tok] : 1.f;
+                b_nx[i] = valid ? p.beta[gbase + tok] : 0.f;
             }
         };
         if (warp == 1) load_gate_inputs(0);
@@ -557,6 +579,22 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                                                    : st + (warp - 1) * 8192 + panel * 16384;
                     if (dbg_ok(src >= sb + OFF_KQV && src + 8192 <= sb + OFF_KQV + kStages * STAGE_BYTES, err))
                         convert_tile(src, 512, lane, lds, sts);
+                }
+            }
+            if constexpr (kVar) {
+                const int64_t nrow = L - static_cast<int64_t>(c) * kC;
+                if (nrow < kC) {
+                    // rows past a packed sequence's end hold the next sequence's tokens: zeroed,
+                    // as the tensor map's fill leaves them for fixed lengths (this warp's tile:
+                    // 0 K, 1 Q, 2 V; two 64-row panels of 64 vectors of 16 bytes per 8 rows)
+                    __syncwarp();
+                    const int which = (kF & kFuseNorm) ? (warp == 1 ? 2 : warp == 2 ? 1 : 0) : warp - 1;
+                    const uint32_t p0 = which == 2 ? st + KQ_BYTES : st + which * 8192;
+                    const uint32_t pstride = which == 2 ? 8192 : 16384;
+                    for (int i = lane; i < 1024; i += 32) {
+                        if (((i & 511) >> 3) >= nrow)
+                            sts(p0 + (i >> 9) * pstride + (i & 511) * 16, make_uint4(0u, 0u, 0u, 0u));
+                    }
                 }
             }
             fence_proxy_async_smem();
@@ -664,6 +702,13 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const bool leader = j == 0;
         Group grp{NB_CHAIN, 128, leader, abort_flag, err};
         bool ok = nchunks > 0;
+        if constexpr (kVar) {
+            // an empty packed sequence: the state passes through unchanged
+            if (nchunks == 0 && seq_ok && p.S_out) {
+                const int64_t base = static_cast<int64_t>(ug) * kD * kD + j;
+                for (int i = 0; i < kD; ++i) p.S_out[base + i * kD] = p.S0 ? p.S0[base + i * kD] : 0.f;
+            }
+        }
         // initial state: S0^T (fp32 in TMEM, pre-scaled by the first chunk's decay; fp16 copy)
         if (ok) ok = grp.wait(bar_addr(sb, B_GATE_FULL + 0), 0);
         if (ok) {
@@ -767,8 +812,8 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 // written to (the same two 64 x 64 boxes; rows past L read as 0)
                 const uint32_t zb = bar_addr(sb, B_Z);
                 mbar_arrive_expect_tx(zb, 16384);
-                tma_load_3d(sb + OFF_OST, &tm_z, 0, static_cast<int32_t>(t0), ug, zb);
-                tma_load_3d(sb + OFF_OST + 8192, &tm_z, 64, static_cast<int32_t>(t0), ug, zb);
+                tma_load_3d(sb + OFF_OST, &tm_z, 0, static_cast<int32_t>(y0 + t0), zc, zb);
+                tma_load_3d(sb + OFF_OST + 8192, &tm_z, 64, static_cast<int32_t>(y0 + t0), zc, zb);
             }
             if (!(gated ? grp.wait(bar_addr(sb, B_O_READY), c & 1, bar_addr(sb, B_Z), c & 1)
                         : grp.wait(bar_addr(sb, B_O_READY), c & 1)))
@@ -779,7 +824,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 // fp32 output: plain stores, done before the TMEM columns are released
                 const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
                 fin &= store_o_f32(tmem + TM_AB + lane_addr + 64, tmem + TM_B + lane_addr + 64, gs->gam,
-                                   static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, n,
+                                   static_cast<float*>(p.o) + (gbase + t0) * kD + j, n,
                                    gated ? sbase + OFF_OST + (j >> 6) * 8192 + (j & 63) * 2 : nullptr);
                 tc_fence_before();
                 mbar_arrive(bar_addr(sb, B_O_DONE));
@@ -808,7 +853,12 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         o0 *= sigmoid_fast(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(ost + r * 128)));
                         o1 *= sigmoid_fast(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(ost + (r + 1) * 128)));
                     }
-                    fin &= is_finite(o0) & is_finite(o1);
+                    if constexpr (kVar) {
+                        // rows past the sequence end hold the next sequence's tokens: not outputs
+                        fin &= (r >= L - t0 || is_finite(o0)) & (r + 1 >= L - t0 || is_finite(o1));
+                    } else {
+                        fin &= is_finite(o0) & is_finite(o1);
+                    }
                     opk[r / 2] = pack_bf16x2(o0, o1);
                 }
             }
@@ -821,11 +871,24 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             fence_proxy_async_smem();
             grp.sync();
-            if (j == 0) {
+            if (kVar && t0 + kC > L) {
+                // a packed sequence's last, partial chunk: the rows past its end belong to the next
+                // sequence, so the n rows are copied out by plain 16-byte stores (both 64-column
+                // halves of a row: 16 pieces), not by the two box stores
+                const int n = static_cast<int>(L - t0);
+                __nv_bfloat16* orow0 = static_cast<__nv_bfloat16*>(p.o) + (gbase + t0) * kD;
+                for (int i = j; i < n * 16; i += 128) {
+                    const int r = i >> 4, part = i & 15;
+                    const uint4 w = *reinterpret_cast<const uint4*>(sbase + OFF_OST + (part >> 3) * 8192 + r * 128 +
+                                                                    (part & 7) * 16);
+                    *reinterpret_cast<uint4*>(orow0 + static_cast<int64_t>(r) * kD + (part >> 3) * 64 + (part & 7) * 8) = w;
+                }
+                if (j == 0) mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
+            } else if (j == 0) {
                 mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
-                if (dbg_ok(t0 < L && ug < p.units_total, err)) {
-                    tma_store_3d(&tm_o, sb + OFF_OST, 0, static_cast<int32_t>(t0), ug);
-                    tma_store_3d(&tm_o, sb + OFF_OST + 8192, 64, static_cast<int32_t>(t0), ug);
+                if (dbg_ok(t0 < L && zc < p.units_total, err)) {
+                    tma_store_3d(&tm_o, sb + OFF_OST, 0, static_cast<int32_t>(y0 + t0), zc);
+                    tma_store_3d(&tm_o, sb + OFF_OST + 8192, 64, static_cast<int32_t>(y0 + t0), zc);
                 }
                 bulk_commit_group();
             }
@@ -856,24 +919,32 @@ cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
 {
     using namespace tc;
     if (call.units_per_loop == 0 || call.T == 0) return cudaSuccess;
+    const bool var = call.cu_seqlens != nullptr;
+    // TMA unit axis and row extent: [T*B*H][L] for fixed lengths, [T*H][Ntot] for packed sequences
     const int64_t units = call.T * call.units_per_loop;
+    const int64_t map_units = var ? call.T * call.H : units;
     CUtensorMap mq, mk, mv, mo, mz;
     const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
-    if (!make_bf16_map_3d(&mq, call.q, units, call.L, kC, sw) || !make_bf16_map_3d(&mk, call.k, units, call.L, kC, sw) ||
-        !make_bf16_map_3d(&mv, call.v, units, call.L, kC, sw))
+    if (!make_bf16_map_3d(&mq, call.q, map_units, call.L, kC, sw) ||
+        !make_bf16_map_3d(&mk, call.k, map_units, call.L, kC, sw) ||
+        !make_bf16_map_3d(&mv, call.v, map_units, call.L, kC, sw))
         return cudaErrorInvalidValue;
     // o (bf16 output only): plain row-major tile, written by the TMA store from shared memory;
     // the output gate logits z (fused) are read into the same tile the same way
-    if (call.out_bf16 && !make_bf16_map_3d(&mo, call.o, units, call.L, kC, CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (call.out_bf16 && !make_bf16_map_3d(&mo, call.o, map_units, call.L, kC, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    if (call.z && !make_bf16_map_3d(&mz, call.z, units, call.L, kC, CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (call.z && !make_bf16_map_3d(&mz, call.z, map_units, call.L, kC, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     const int fb = fuse_bits(call);
-    using K = decltype(&gdr_prefill_tc_kernel<0>);
-    static const K kernels[8] = {gdr_prefill_tc_kernel<0>, gdr_prefill_tc_kernel<1>, gdr_prefill_tc_kernel<2>,
-                                 gdr_prefill_tc_kernel<3>, gdr_prefill_tc_kernel<4>, gdr_prefill_tc_kernel<5>,
-                                 gdr_prefill_tc_kernel<6>, gdr_prefill_tc_kernel<7>};
-    const K kernel = kernels[fb];
+    using K = decltype(&gdr_prefill_tc_kernel<0, false>);
+    static const K kernels[2][8] = {
+        {gdr_prefill_tc_kernel<0, false>, gdr_prefill_tc_kernel<1, false>, gdr_prefill_tc_kernel<2, false>,
+         gdr_prefill_tc_kernel<3, false>, gdr_prefill_tc_kernel<4, false>, gdr_prefill_tc_kernel<5, false>,
+         gdr_prefill_tc_kernel<6, false>, gdr_prefill_tc_kernel<7, false>},
+        {gdr_prefill_tc_kernel<0, true>, gdr_prefill_tc_kernel<1, true>, gdr_prefill_tc_kernel<2, true>,
+         gdr_prefill_tc_kernel<3, true>, gdr_prefill_tc_kernel<4, true>, gdr_prefill_tc_kernel<5, true>,
+         gdr_prefill_tc_kernel<6, true>, gdr_prefill_tc_kernel<7, true>}};
+    const K kernel = kernels[var ? 1 : 0][fb];
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess) return e;
@@ -887,12 +958,16 @@ cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
         p.S_out = call.S_out;
         p.L = call.L;
         p.unit0 = static_cast<int>(tau * call.units_per_loop);
-        p.units_total = static_cast<int>(units);
+        p.units_total = static_cast<int>(map_units);
         p.out_bf16 = call.out_bf16;
         p.err = call.err;
         p.qk_norm = call.qk_norm;
         p.gate_logits = call.gate_logits;
         p.alpha_scale = call.alpha_scale;
+        p.cu = call.cu_seqlens;
+        p.Ntot = call.L;
+        p.H = static_cast<int>(call.H);
+        p.loop = static_cast<int>(tau);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(call.units_per_loop), 1, 1);
         cfg.blockDim = dim3(kThreads, 1, 1);

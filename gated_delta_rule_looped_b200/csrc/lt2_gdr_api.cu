@@ -129,6 +129,22 @@ lt2_status validate_dims(const lt2_gdr_dims* d, Sizes* sz)
     return LT2_OK;
 }
 
+// Element counts of a packed-sequence call: dims->B sequences whose tokens are packed along
+// dims->L = Ntot; q/k/v/o [T][H][Ntot][d], gates [T][H][Ntot](x dk), states [T][B][H][dk][dv].
+lt2_status validate_varlen_dims(const lt2_gdr_dims* d, Sizes* sz)
+{
+    lt2_status st = validate_dims(d, sz);
+    if (st != LT2_OK) return st;
+    const __int128 rows = (__int128)d->T * d->H * d->L;      // packed token-heads
+    if (rows * 128 > ((__int128)1 << 62)) return LT2_ERR_INVALID_ARGUMENT;
+    sz->qk = (int64_t)(rows * d->dk);
+    sz->vo = (int64_t)(rows * d->dv);
+    sz->al = (int64_t)(is_per_key(d) ? rows * d->dk : rows);
+    sz->be = (int64_t)rows;
+    if (d->T * d->H >= kMaxDim) return LT2_ERR_UNSUPPORTED;   // TMA unit axis, 32-bit
+    return LT2_OK;
+}
+
 // Every non-null pointer must address device memory of the current device: kernels launch
 // on the current device, and the tensor maps of the tensor-core path would otherwise cover
 // another GPU's memory.
@@ -328,6 +344,98 @@ lt2_status lt2_gdr_prefill_fused(const lt2_gdr_dims* dims, const lt2_gdr_fused* 
     return LT2_OK;
 }
 
+lt2_status lt2_gdr_prefill_varlen(const lt2_gdr_dims* dims, const lt2_gdr_fused* fused, const int64_t* cu_seqlens,
+                                  const void* q, const void* k, const void* v, const float* alpha,
+                                  const float* beta, const float* S0, void* o, float* S_out, void* workspace,
+                                  size_t workspace_bytes, void* stream)
+{
+    (void)workspace;
+    (void)workspace_bytes;
+    Sizes sz;
+    lt2_status st = validate_varlen_dims(dims, &sz);
+    if (st != LT2_OK) return st;
+    const lt2_gdr_fused f = fused_or_none(fused);
+    const bool tc_ok = !is_per_key(dims) &&
+                       lt2::prefill_tc_supports(dims->dtype == LT2_DTYPE_BF16, (int)dims->dk, (int)dims->dv, 0);
+    if (dims->algo == LT2_ALGO_TENSOR_CORE && !tc_ok) return LT2_ERR_UNSUPPORTED;
+    if (sz.units == 0) return LT2_OK;
+    if (cu_seqlens == nullptr || (reinterpret_cast<uintptr_t>(cu_seqlens) & 7u) != 0) return LT2_ERR_INVALID_ARGUMENT;
+    if (!tensor_ok(q, sz.qk) || !tensor_ok(k, sz.qk) || !tensor_ok(v, sz.vo) || !tensor_ok(alpha, sz.al) ||
+        !tensor_ok(beta, sz.be) || !tensor_ok(o, sz.vo))
+        return LT2_ERR_INVALID_ARGUMENT;
+    if ((S0 && !aligned16(S0)) || (S_out && !aligned16(S_out))) return LT2_ERR_INVALID_ARGUMENT;
+    const Range ro = range_of(o, sz.vo * sz.osz);
+    const Range rin[6] = {range_of(q, sz.qk * sz.esz), range_of(k, sz.qk * sz.esz), range_of(v, sz.vo * sz.esz),
+                          range_of(alpha, sz.al * 4), range_of(beta, sz.be * 4),
+                          range_of(cu_seqlens, (dims->B + 1) * 8)};
+    for (const Range& r : rin)
+        if (overlap(ro, r)) return LT2_ERR_INVALID_ARGUMENT;
+    if (S0 && overlap(ro, range_of(S0, sz.st * 4))) return LT2_ERR_INVALID_ARGUMENT;
+    if (S_out) {
+        const Range rs = range_of(S_out, sz.st * 4);
+        if (overlap(rs, ro)) return LT2_ERR_INVALID_ARGUMENT;
+        for (const Range& r : rin)
+            if (overlap(rs, r)) return LT2_ERR_INVALID_ARGUMENT;
+        if (S0 && S0 != S_out && overlap(rs, range_of(S0, sz.st * 4))) return LT2_ERR_INVALID_ARGUMENT;
+    }
+    st = validate_fused(f, sz, o, S_out);
+    if (st != LT2_OK) return st;
+    st = on_current_device({q, k, v, alpha, beta, S0, o, S_out, f.z, cu_seqlens});
+    if (st != LT2_OK) return st;
+
+    NvtxRange range("lt2_gdr_prefill_varlen");
+    unsigned int* err = nullptr;
+    st = status_word(&err);
+    if (st != LT2_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (tc_ok && dims->algo != LT2_ALGO_CUDA_CORE && dims->L > 0) {
+        lt2::TcCall call;
+        call.q = q;
+        call.k = k;
+        call.v = v;
+        call.alpha = alpha;
+        call.beta = beta;
+        call.S0 = S0;
+        call.o = o;
+        call.S_out = S_out;
+        call.T = dims->T;
+        call.units_per_loop = sz.per_loop;
+        call.L = dims->L;
+        call.out_bf16 = out_is_bf16(dims) ? 1 : 0;
+        call.decay_first = 0;
+        call.err = err;
+        call.qk_norm = f.qk_l2norm;
+        call.gate_logits = f.gate_logits;
+        call.alpha_scale = f.alpha_scale;
+        call.z = f.z;
+        call.cu_seqlens = cu_seqlens;
+        call.H = dims->H;
+        cudaError_t e = lt2::launch_prefill_tc_all(call, s);
+        if (e == cudaSuccess) e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "prefill varlen (tensor core)");
+        return LT2_OK;
+    }
+    const int64_t rows = dims->H * dims->L;                  // packed token-heads of one loop
+    const int64_t na = is_per_key(dims) ? dims->dk : 1;
+    for (int64_t tau = 0; tau < dims->T; ++tau) {
+        lt2::LoopSlice ls = loop_slice(dims, sz, tau, q, k, v, alpha, beta, S0, o, S_out, err, f);
+        ls.q = static_cast<const char*>(q) + tau * rows * dims->dk * sz.esz;
+        ls.k = static_cast<const char*>(k) + tau * rows * dims->dk * sz.esz;
+        ls.v = static_cast<const char*>(v) + tau * rows * dims->dv * sz.esz;
+        ls.alpha = alpha + tau * rows * na;
+        ls.beta = beta + tau * rows;
+        ls.o = static_cast<char*>(o) + tau * rows * dims->dv * sz.osz;
+        ls.z = f.z ? static_cast<const char*>(f.z) + tau * rows * dims->dv * sz.esz : nullptr;
+        ls.cu = cu_seqlens;
+        ls.H = static_cast<int>(dims->H);
+        NvtxRange loop_range("lt2 prefill varlen loop (cuda core)");
+        cudaError_t e = lt2::launch_prefill_seq(ls, dims->dtype == LT2_DTYPE_BF16, s, tau > 0);
+        if (e == cudaSuccess) e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "prefill varlen (cuda core)");
+    }
+    return LT2_OK;
+}
+
 lt2_status lt2_gdr_decode(const lt2_gdr_dims* dims, const void* q, const void* k, const void* v,
                           const float* alpha, const float* beta, float* S, void* o, void* stream)
 {
@@ -448,6 +556,7 @@ lt2_status lt2_gdr_last_device_error(void)
     e = cudaMemcpy(&h, p + 1, sizeof(h), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e, "read device status");
     if (h & lt2::kDevTimeout) return LT2_ERR_DEVICE_TIMEOUT;
+    if (h & lt2::kDevSeqlens) return LT2_ERR_SEQLENS;
     if (h & lt2::kDevRange) return LT2_ERR_RANGE;
     if (h & lt2::kDevCheck) return LT2_ERR_DEVICE_CHECK;
     return LT2_OK;
@@ -464,13 +573,14 @@ const char* lt2_status_string(lt2_status s)
         case LT2_ERR_DEVICE_TIMEOUT: return "LT2_ERR_DEVICE_TIMEOUT";
         case LT2_ERR_RANGE: return "LT2_ERR_RANGE";
         case LT2_ERR_DEVICE_CHECK: return "LT2_ERR_DEVICE_CHECK";
+        case LT2_ERR_SEQLENS: return "LT2_ERR_SEQLENS";
     }
     return "LT2_STATUS_UNKNOWN";
 }
 
 const char* lt2_last_cuda_error_string(void) { return t_cuda_error; }
 
-int lt2_gdr_version(void) { return 210; }
+int lt2_gdr_version(void) { return 220; }
 
 }  // extern "C"
 

@@ -77,7 +77,8 @@ typedef enum lt2_status {
     LT2_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed                   */
     LT2_ERR_DEVICE_TIMEOUT = 5,   /* a bounded in-kernel wait ran out (see header comment)  */
     LT2_ERR_RANGE = 6,            /* a tensor-core path produced non-finite results         */
-    LT2_ERR_DEVICE_CHECK = 7      /* a debug build's device-side check failed (lt2_gdr_debug.h) */
+    LT2_ERR_DEVICE_CHECK = 7,     /* a debug build's device-side check failed (lt2_gdr_debug.h) */
+    LT2_ERR_SEQLENS = 8           /* packed-sequence offsets out of order or past the packed length */
 } lt2_status;
 
 typedef enum lt2_dtype { LT2_DTYPE_F32 = 0, LT2_DTYPE_BF16 = 1 } lt2_dtype;
@@ -192,6 +193,36 @@ lt2_status lt2_gdr_prefill_fused(const lt2_gdr_dims* dims, const lt2_gdr_fused* 
                                  void* stream);
 
 /*
+ * The same prefill over packed sequences of different lengths ("varlen" batches: the pages batch
+ * sequences but give no layout; this is the plainest packed one).  dims->B is the number of
+ * sequences and dims->L the packed length Ntot; sequence b holds tokens cu_seqlens[b] ..
+ * cu_seqlens[b+1]-1 of every (loop, head).  Each (loop, sequence, head) is an independent
+ * recurrence, exactly as a separate lt2_gdr_prefill call on that sequence would compute it.
+ *   cu_seqlens  int64 [B+1] (device, 8-byte aligned, read only): 0 <= cu[b] <= cu[b+1] <= Ntot;
+ *               offsets out of that order are reported as LT2_ERR_SEQLENS by
+ *               lt2_gdr_last_device_error() and their sequences left unwritten
+ *   q, k, z     [T][H][Ntot][dk] (z: [T][H][Ntot][dv]), dims->dtype
+ *   v, o        [T][H][Ntot][dv]
+ *   alpha       [T][H][Ntot] fp32 for scalar gating, [T][H][Ntot][dk] per key; beta [T][H][Ntot]
+ *   S0, S_out   [T][B][H][dk][dv] fp32, as for lt2_gdr_prefill (an empty sequence passes S0,
+ *               or zeros, to S_out)
+ *   fused       as lt2_gdr_prefill_fused (NULL: none)
+ * Scalar gating with bf16 inputs and d = 128 runs on the tensor-core kernel (each CTA reads its
+ * sequence's rows; the rows of a partial last chunk that belong to the next sequence are masked
+ * out); every other case runs on the CUDA-core path.  LT2_ALGO_TENSOR_CORE with per-key gating
+ * returns LT2_ERR_UNSUPPORTED.  No workspace is used (workspace may be NULL).  Same return
+ * convention as lt2_gdr_prefill.
+ */
+lt2_status lt2_gdr_prefill_varlen(const lt2_gdr_dims* dims, const lt2_gdr_fused* fused,
+                                  const int64_t* cu_seqlens,
+                                  const void* q, const void* k, const void* v,
+                                  const float* alpha, const float* beta,
+                                  const float* S0,
+                                  void* o, float* S_out,
+                                  void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/*
  * Decode: one step of the same recurrence ("LT2 transformer looped a tempo lineare", section
  * "Sostituire il motore", displayed equation) for one new token per (loop, batch, head);
  * dims->L must be 1 and dims->algo is ignored.  S [T][B][H][dk][dv] fp32 is read and replaced
@@ -258,10 +289,10 @@ lt2_status lt2_swa_prefill(const lt2_swa_dims* dims,
  * The device-side status word of the CURRENT device (not an operation of the pages: the
  * library's own failure reporting).  Synchronises the device (every stream), then reads and
  * clears the word in one atomic exchange.  Returns LT2_ERR_DEVICE_TIMEOUT if a kernel gave up
- * on a bounded wait since the last read, else LT2_ERR_RANGE if a tensor-core prefill produced
- * non-finite results, else LT2_ERR_DEVICE_CHECK if a device-side check of the debug build failed
- * (never in the product build), else LT2_OK; LT2_ERR_CUDA if the synchronisation or the read
- * failed.
+ * on a bounded wait since the last read, else LT2_ERR_SEQLENS if a packed-sequence call met bad
+ * offsets, else LT2_ERR_RANGE if a tensor-core prefill produced non-finite results, else
+ * LT2_ERR_DEVICE_CHECK if a device-side check of the debug build failed (never in the product
+ * build), else LT2_OK; LT2_ERR_CUDA if the synchronisation or the read failed.
  * The word is shared by every call on the device, from any thread or stream: a flag belongs
  * to whichever work ran since the previous read.
  */

@@ -310,3 +310,37 @@ def test_swa_aliasing_rejected(L):
 def test_swa_empty_problem_is_a_noop(L):
     assert call_swa(SD(T=0)) == lt2.LT2_OK
     assert call_swa(SD(L=0), q=None, k=None, v=None, o=None) == lt2.LT2_OK
+
+
+# ---- packed sequences (lt2_gdr_prefill_varlen) ---------------------------------------------
+
+def call_varlen(dims, cu=BASE + 30 * SPAN, **over):
+    q, k, v, a, b, s0, o, so = addrs(8)
+    args = dict(q=q, k=k, v=v, alpha=a, beta=b, S0=s0, o=o, S_out=so)
+    args.update(over)
+    return lt2.lt2_gdr_prefill_varlen(dims, None, cu, args["q"], args["k"], args["v"], args["alpha"], args["beta"],
+                                      args["S0"], args["o"], args["S_out"], None, 0, 0)
+
+
+def test_varlen_offsets_checked(L):
+    assert call_varlen(D(), cu=None) == lt2.LT2_ERR_INVALID_ARGUMENT
+    assert call_varlen(D(), cu=BASE + 30 * SPAN + 4) == lt2.LT2_ERR_INVALID_ARGUMENT     # not 8-byte aligned
+    q = addrs(1)[0]
+    assert call_varlen(D(), o=q + 64) == lt2.LT2_ERR_INVALID_ARGUMENT                    # o inside q
+    assert call_varlen(D(), cu=addrs(7)[6] + 16) == lt2.LT2_ERR_INVALID_ARGUMENT        # offsets inside o
+
+
+def test_varlen_per_key_has_no_tensor_core_path(L):
+    d = D(dtype=lt2.LT2_DTYPE_BF16, dk=128, dv=128, gate=lt2.LT2_GATE_PER_KEY, algo=lt2.LT2_ALGO_TENSOR_CORE)
+    assert call_varlen(d) == lt2.LT2_ERR_UNSUPPORTED
+
+
+def test_varlen_bad_dims_and_empty(L):
+    assert call_varlen(D(dk=0)) == lt2.LT2_ERR_INVALID_ARGUMENT
+    assert call_varlen(D(T=0)) == lt2.LT2_OK
+    assert L.lt2_gdr_prefill_varlen(None, None, BASE, 1, 1, 1, 1, 1, None, 1, None, None, 0, None) == \
+        lt2.LT2_ERR_INVALID_ARGUMENT
+
+
+def test_seqlens_status_has_a_name(L):
+    assert lt2.lt2_status_string(lt2.LT2_ERR_SEQLENS) == "LT2_ERR_SEQLENS"
