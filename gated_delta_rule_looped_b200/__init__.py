@@ -45,6 +45,8 @@ EXPORTS = (
     "lt2_gdr_decode",
     "lt2_gdr_decode_fused",
     "lt2_gdr_prefill_varlen",
+    "lt2_gdr_backward_workspace_bytes",
+    "lt2_gdr_backward",
     "lt2_swa_prefill",
     "lt2_gdr_last_device_error",
     "lt2_status_string",
@@ -130,6 +132,12 @@ def load_library(path):
         L.lt2_gdr_prefill_varlen.argtypes = [dims_p, ctypes.POINTER(lt2_gdr_fused), vp, vp, vp, vp, fp, fp, fp, vp,
                                              fp, vp, ctypes.c_size_t, vp]
         L.lt2_gdr_prefill_varlen.restype = ctypes.c_int
+    if hasattr(L, "lt2_gdr_backward"):
+        L.lt2_gdr_backward_workspace_bytes.argtypes = [dims_p]
+        L.lt2_gdr_backward_workspace_bytes.restype = ctypes.c_size_t
+        L.lt2_gdr_backward.argtypes = [dims_p, vp, vp, vp, fp, fp, fp, vp, fp, fp, fp, fp, fp, fp, fp, vp,
+                                       ctypes.c_size_t, vp]
+        L.lt2_gdr_backward.restype = ctypes.c_int
     if hasattr(L, "lt2_swa_prefill"):
         L.lt2_swa_prefill.argtypes = [ctypes.POINTER(lt2_swa_dims), vp, vp, vp, vp, vp]
         L.lt2_swa_prefill.restype = ctypes.c_int
@@ -208,6 +216,17 @@ def lt2_gdr_prefill_varlen(dims, fused, cu_seqlens, q, k, v, alpha, beta, S0, o,
     return lib().lt2_gdr_prefill_varlen(ctypes.byref(dims), None if fused is None else ctypes.byref(fused),
                                         _p(cu_seqlens), _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(o),
                                         _p(S_out), _p(workspace), int(workspace_bytes), _stream(stream))
+
+
+def lt2_gdr_backward_workspace_bytes(dims):
+    return lib().lt2_gdr_backward_workspace_bytes(ctypes.byref(dims))
+
+
+def lt2_gdr_backward(dims, q, k, v, alpha, beta, S0, dO, dS_L, dq, dk, dv, dalpha, dbeta, dS0, workspace=None,
+                     workspace_bytes=0, stream=None):
+    return lib().lt2_gdr_backward(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(dO),
+                                  _p(dS_L), _p(dq), _p(dk), _p(dv), _p(dalpha), _p(dbeta), _p(dS0), _p(workspace),
+                                  int(workspace_bytes), _stream(stream))
 
 
 def lt2_swa_prefill(dims, q, k, v, o, stream=None):
@@ -447,3 +466,27 @@ def prefill_varlen(q, k, v, alpha, beta, cu_seqlens, S0=None, per_key=None, algo
         if st != LT2_OK:
             raise Lt2Error(st, "lt2_gdr_prefill_varlen")
         return o, S_out
+
+
+def backward(q, k, v, alpha, beta, dO, S0=None, dS_L=None, per_key=None, order="delta_first", stream=None):
+    """Gradients of sum(dO * o) + sum(dS_L * S_out) of ``prefill`` (lt2_gdr_backward), fp32:
+    returns a dict dq, dk, dv, dalpha, dbeta, dS0.  The workspace is allocated with torch."""
+    import torch
+    _require_cuda(q)
+    with torch.cuda.device(q.device):
+        dims = _dims_from(q, v, alpha, per_key, LT2_ALGO_AUTO, None, order)
+        pk = dims.gate != LT2_GATE_SCALAR
+        _check_call(q, k, v, alpha, beta, [("S0", S0), ("dS_L", dS_L)], None, pk, None)
+        _check("dO", dO, v.shape, q.dtype, q.device)
+        dev = q.device
+        f32 = dict(dtype=torch.float32, device=dev)
+        g = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(q.shape, **f32), "dv": torch.empty(v.shape, **f32),
+             "dalpha": torch.empty(alpha.shape, **f32), "dbeta": torch.empty(beta.shape, **f32),
+             "dS0": torch.empty(tuple(q.shape[:3]) + (q.shape[-1], v.shape[-1]), **f32)}
+        ws_bytes = lt2_gdr_backward_workspace_bytes(dims)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+        st = lt2_gdr_backward(dims, q, k, v, alpha, beta, S0, dO, dS_L, g["dq"], g["dk"], g["dv"], g["dalpha"],
+                              g["dbeta"], g["dS0"], ws, ws_bytes, stream)
+        if st != LT2_OK:
+            raise Lt2Error(st, "lt2_gdr_backward")
+        return g

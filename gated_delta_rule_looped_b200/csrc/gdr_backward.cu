@@ -1,0 +1,321 @@
+// gdr_backward.cu -- backward pass of the looped gated delta rule on CUDA cores (fp32).
+//
+// The forward recurrence ("LT2 transformer looped a tempo lineare", section "Sostituire il
+// motore", displayed equation), per (loop, batch, head) unit and token t:
+//     printed order:      e = S_{t-1}^T k,  P = S_{t-1} - beta k e^T,  S_t = Diag(alpha) P + beta k v^T
+//     decay-first order:  R = Diag(alpha) S_{t-1},  e = R^T k,  S_t = R - beta k e^T + beta k v^T
+//     o_t = S_t^T q_t
+// The pages train looped models but give no training kernel; this is the plain reverse-mode
+// derivative of the recurrence.  For upstream gradients dO_t and dS_L, a sweep from t = L down to
+// 1 carries G = dLoss/dS_t:
+//     G += q_t dO_t^T;  dq_t = S_t dO_t
+//     printed:      dP = Diag(alpha) G;  dv = beta G^T k;  dbeta = (G^T k).v - (dP^T k).e
+//                   dk = beta G v - beta (S_{t-1} (dP^T k) + dP e);  dalpha = rowsum(G * P)
+//                   G <- dP - beta k (dP^T k)^T
+//     decay-first:  kG = G^T k;  dR = G - beta k kG^T;  dv = beta kG;  dbeta = kG.(v - e)
+//                   dk = beta G (v - e) - beta R kG;  dalpha = rowsum(dR * S_{t-1});  G <- Diag(alpha) dR
+// and dS_0 = G at the end (scalar alpha: dalpha sums over the rows too).
+//
+// The columns of S evolve independently given the token's k, alpha, beta (e_j only reads column
+// j), so a block takes one unit and a slice of 32 columns of d_v, like the token-sequential
+// prefill: warp w holds rows w*dk/8 .. of the slice, lane c column j0 + c.  The reverse sweep
+// needs S_{t-1} and S_t at every t, newest first:
+//   phase A  runs the forward over the whole sequence and keeps the state at the start of every
+//            64-token chunk (a checkpoint) in the workspace;
+//   phase B  takes the chunks from the last: it recomputes the chunk's states from its checkpoint
+//            into the workspace, then sweeps the chunk backwards.
+// Per token the three column sums the step needs (k^T S_{t-1} or k^T R, k^T G, k^T Diag(alpha) G)
+// come from one shared-memory reduction; the row sums (dq, dk, dalpha) are warp reductions whose
+// slice partials are added into the fp32 outputs with atomics (zeroed first by this library).
+// dv and dS_0 belong to one block each and are stored directly.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "gdr_common.cuh"
+#include "gdr_launch.h"
+#include "gdr_nvtx.h"
+
+namespace lt2 {
+namespace bw {
+
+constexpr int kCols = 32;          // columns of d_v per block
+constexpr int kThreads = 256;      // 8 warps
+constexpr int kChunk = 64;         // tokens between checkpoints
+constexpr int kMaxRows = 16;       // dk / 8 rows per warp, dk <= 128
+
+__device__ __forceinline__ float ld(const float* p) { return *p; }
+__device__ __forceinline__ float ld(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+__device__ __forceinline__ float warp_sum(float x)
+{
+    #pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+}
+
+struct Params {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* alpha;
+    const float* beta;
+    const float* S0;       // nullable
+    const void* dO;
+    const float* dSL;      // nullable
+    float* dq;             // [units][L][dk], accumulated (zeroed first)
+    float* gdk;            // dk, accumulated
+    float* gdv;            // dv [units][L][dv], stored
+    float* dalpha;         // [units][L] or [units][L][dk], accumulated
+    float* dbeta;          // [units][L], accumulated
+    float* dS0;            // nullable, stored
+    float* ws;             // per block: checkpoints, then the states of one chunk
+    int64_t units;
+    int64_t L;
+    int dk;
+    int dv;
+    int per_key;
+    int decay_first;
+};
+
+// Workspace floats per block: ceil(L / 64) checkpoints and the 65 states of one chunk, dk x 32 each.
+__host__ __device__ inline int64_t ws_floats_per_block(int64_t L, int dk)
+{
+    return ((L + kChunk - 1) / kChunk + kChunk + 1) * static_cast<int64_t>(dk) * kCols;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
+{
+    __shared__ float red[2][3][8][kCols];
+    const int dk = p.dk, dv = p.dv, rpw = dk >> 3;
+    const int w = threadIdx.x >> 5, c = threadIdx.x & 31;
+    const int j0 = blockIdx.y * kCols;
+    const int ncol = min(kCols, dv - j0);
+    const bool active = c < ncol;
+    const int j = j0 + c;
+    const int64_t u = blockIdx.x, L = p.L;
+    const int r0 = w * rpw;
+    const int na = p.per_key ? dk : 1;
+
+    const T* q = static_cast<const T*>(p.q) + u * L * dk;
+    const T* k = static_cast<const T*>(p.k) + u * L * dk;
+    const T* v = static_cast<const T*>(p.v) + u * L * dv;
+    const T* dO = static_cast<const T*>(p.dO) + u * L * dv;
+    const float* al = p.alpha + u * L * na;
+    const float* be = p.beta + u * L;
+    float* ws = p.ws + (u * gridDim.y + blockIdx.y) * ws_floats_per_block(L, dk);
+    const int nck = static_cast<int>((L + kChunk - 1) / kChunk);
+    float* ck = ws;                                             // [nck][dk][32]
+    float* st = ws + static_cast<int64_t>(nck) * dk * kCols;   // [65][dk][32]
+    auto at = [&](float* base, int idx, int m) -> float& { return base[(static_cast<int64_t>(idx) * dk + r0 + m) * kCols + c]; };
+
+    // one forward step of the recurrence on this thread's part of the state
+    auto step = [&](float (&s)[kMaxRows], int64_t t, int buf) {
+        float kr[kMaxRows], ar[kMaxRows];
+        const float b = be[t];
+        #pragma unroll
+        for (int m = 0; m < kMaxRows; ++m) {
+            kr[m] = m < rpw ? ld(k + t * dk + r0 + m) : 0.f;
+            ar[m] = m < rpw ? (p.per_key ? al[t * dk + r0 + m] : al[t]) : 1.f;
+        }
+        float pe = 0.f;
+        #pragma unroll
+        for (int m = 0; m < kMaxRows; ++m) pe += kr[m] * (p.decay_first ? ar[m] * s[m] : s[m]);
+        red[buf][0][w][c] = pe;
+        __syncthreads();
+        float e = 0.f;
+        #pragma unroll
+        for (int ww = 0; ww < 8; ++ww) e += red[buf][0][ww][c];
+        const float vj = active ? ld(v + t * dv + j) : 0.f;
+        #pragma unroll
+        for (int m = 0; m < kMaxRows; ++m) {
+            if (p.decay_first) s[m] = ar[m] * s[m] + b * kr[m] * (vj - e);
+            else s[m] = ar[m] * (s[m] - b * kr[m] * e) + b * kr[m] * vj;
+        }
+    };
+
+    // ---- phase A: forward, checkpoints at the chunk starts ----
+    float s[kMaxRows];
+    const float* S0 = p.S0 ? p.S0 + u * static_cast<int64_t>(dk) * dv : nullptr;
+    #pragma unroll
+    for (int m = 0; m < kMaxRows; ++m) s[m] = (m < rpw && active && S0) ? S0[static_cast<int64_t>(r0 + m) * dv + j] : 0.f;
+    for (int64_t t = 0; t < L; ++t) {
+        if (t % kChunk == 0) {
+            #pragma unroll
+            for (int m = 0; m < kMaxRows; ++m)
+                if (m < rpw) at(ck, static_cast<int>(t / kChunk), m) = s[m];
+        }
+        step(s, t, static_cast<int>(t & 1));
+    }
+    __syncthreads();                                   // the reduction buffers are reused below
+
+    // ---- phase B: chunks from the last, each recomputed, then swept backwards ----
+    float G[kMaxRows];
+    const float* dSL = p.dSL ? p.dSL + u * static_cast<int64_t>(dk) * dv : nullptr;
+    #pragma unroll
+    for (int m = 0; m < kMaxRows; ++m) G[m] = (m < rpw && active && dSL) ? dSL[static_cast<int64_t>(r0 + m) * dv + j] : 0.f;
+    for (int ci = nck - 1; ci >= 0; --ci) {
+        const int64_t t0 = static_cast<int64_t>(ci) * kChunk;
+        const int n = static_cast<int>(L - t0 < kChunk ? L - t0 : kChunk);
+        #pragma unroll
+        for (int m = 0; m < kMaxRows; ++m) {
+            s[m] = m < rpw ? at(ck, ci, m) : 0.f;
+            if (m < rpw) at(st, 0, m) = s[m];
+        }
+        for (int tau = 0; tau < n; ++tau) {
+            step(s, t0 + tau, tau & 1);
+            #pragma unroll
+            for (int m = 0; m < kMaxRows; ++m)
+                if (m < rpw) at(st, tau + 1, m) = s[m];
+        }
+        __syncthreads();
+        for (int tau = n - 1; tau >= 0; --tau) {
+            const int64_t t = t0 + tau;
+            const int buf = tau & 1;
+            float sp[kMaxRows], sc[kMaxRows], kr[kMaxRows], ar[kMaxRows];
+            const float b = be[t];
+            const float vj = active ? ld(v + t * dv + j) : 0.f;
+            const float oj = active ? ld(dO + t * dv + j) : 0.f;
+            #pragma unroll
+            for (int m = 0; m < kMaxRows; ++m) {
+                const bool on = m < rpw;
+                sp[m] = on ? at(st, tau, m) : 0.f;
+                sc[m] = on ? at(st, tau + 1, m) : 0.f;
+                kr[m] = on ? ld(k + t * dk + r0 + m) : 0.f;
+                ar[m] = on ? (p.per_key ? al[t * dk + r0 + m] : al[t]) : 1.f;
+                const float qr = on ? ld(q + t * dk + r0 + m) : 0.f;
+                G[m] += qr * oj;                       // from o_t = S_t^T q_t
+            }
+            // dq_t = S_t dO_t: row sums over this slice's columns
+            #pragma unroll
+            for (int m = 0; m < kMaxRows; ++m) {
+                if (m >= rpw) break;
+                const float x = warp_sum(sc[m] * oj);
+                if (c == 0) atomicAdd(p.dq + (u * L + t) * dk + r0 + m, x);
+            }
+            // the column sums of this step, one reduction: e, k^T G, k^T Diag(alpha) G
+            float pe = 0.f, pg = 0.f, pd = 0.f;
+            #pragma unroll
+            for (int m = 0; m < kMaxRows; ++m) {
+                pe += kr[m] * (p.decay_first ? ar[m] * sp[m] : sp[m]);
+                pg += kr[m] * G[m];
+                pd += kr[m] * ar[m] * G[m];
+            }
+            red[buf][0][w][c] = pe;
+            red[buf][1][w][c] = pg;
+            red[buf][2][w][c] = pd;
+            __syncthreads();
+            float e = 0.f, kG = 0.f, kdP = 0.f;
+            #pragma unroll
+            for (int ww = 0; ww < 8; ++ww) {
+                e += red[buf][0][ww][c];
+                kG += red[buf][1][ww][c];
+                kdP += red[buf][2][ww][c];
+            }
+            if (active) p.gdv[(u * L + t) * dv + j] = b * kG;
+            // dbeta: column terms summed over the slice
+            const float tb = active ? (p.decay_first ? kG * (vj - e) : kG * vj - kdP * e) : 0.f;
+            if (w == 0) {
+                const float x = warp_sum(tb);
+                if (c == 0) atomicAdd(p.dbeta + u * L + t, x);
+            }
+            float dal_sum = 0.f;
+            #pragma unroll
+            for (int m = 0; m < kMaxRows; ++m) {
+                if (m >= rpw) break;
+                float dkx, dax;
+                if (p.decay_first) {
+                    const float R = ar[m] * sp[m];
+                    const float dR = G[m] - b * kr[m] * kG;
+                    dkx = b * G[m] * (vj - e) - b * R * kG;
+                    dax = dR * sp[m];
+                    G[m] = ar[m] * dR;
+                } else {
+                    const float P = sp[m] - b * kr[m] * e;
+                    const float dP = ar[m] * G[m];
+                    dkx = b * G[m] * vj - b * (sp[m] * kdP + dP * e);
+                    dax = G[m] * P;
+                    G[m] = dP - b * kr[m] * kdP;
+                }
+                if (!active) dkx = dax = 0.f;
+                const float dks = warp_sum(dkx);
+                if (c == 0) atomicAdd(p.gdk + (u * L + t) * dk + r0 + m, dks);
+                if (p.per_key) {
+                    const float das = warp_sum(dax);
+                    if (c == 0) atomicAdd(p.dalpha + (u * L + t) * dk + r0 + m, das);
+                } else {
+                    dal_sum += dax;
+                }
+            }
+            if (!p.per_key) {
+                const float x = warp_sum(dal_sum);
+                if (c == 0) atomicAdd(p.dalpha + u * L + t, x);
+            }
+        }
+        __syncthreads();
+    }
+    if (p.dS0 && active) {
+        float* o = p.dS0 + u * static_cast<int64_t>(dk) * dv;
+        #pragma unroll
+        for (int m = 0; m < kMaxRows; ++m)
+            if (m < rpw) o[static_cast<int64_t>(r0 + m) * dv + j] = G[m];
+    }
+}
+
+__global__ void zero_kernel(float* x, int64_t n)
+{
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        x[i] = 0.f;
+}
+
+}  // namespace bw
+
+size_t backward_workspace_bytes(int64_t units, int64_t L, int dk, int dv)
+{
+    const int64_t slices = (dv + bw::kCols - 1) / bw::kCols;
+    return static_cast<size_t>(units * slices * bw::ws_floats_per_block(L, dk) * 4);
+}
+
+cudaError_t launch_backward(const BwCall& c, cudaStream_t stream)
+{
+    using namespace bw;
+    if (c.units == 0) return cudaSuccess;
+    NvtxRange range("lt2 backward (cuda core)");
+    const int64_t na = c.per_key ? c.dk : 1;
+    const int64_t zn[4] = {c.units * c.L * c.dk, c.units * c.L * c.dk, c.units * c.L * na, c.units * c.L};
+    float* zp[4] = {c.dq, c.dk_out, c.dalpha, c.dbeta};
+    for (int i = 0; i < 4; ++i) {
+        if (zn[i] == 0) continue;
+        const int64_t blocks = (zn[i] + 255) / 256 < 4096 ? (zn[i] + 255) / 256 : 4096;
+        zero_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(zp[i], zn[i]);
+    }
+    Params p;
+    p.q = c.q;
+    p.k = c.k;
+    p.v = c.v;
+    p.alpha = c.alpha;
+    p.beta = c.beta;
+    p.S0 = c.S0;
+    p.dO = c.dO;
+    p.dSL = c.dSL;
+    p.dq = c.dq;
+    p.gdk = c.dk_out;
+    p.gdv = c.dv_out;
+    p.dalpha = c.dalpha;
+    p.dbeta = c.dbeta;
+    p.dS0 = c.dS0;
+    p.ws = c.ws;
+    p.units = c.units;
+    p.L = c.L;
+    p.dk = c.dk;
+    p.dv = c.dv;
+    p.per_key = c.per_key;
+    p.decay_first = c.decay_first;
+    const dim3 grid(static_cast<unsigned>(c.units), static_cast<unsigned>((c.dv + kCols - 1) / kCols), 1);
+    if (c.dtype_bf16) gdr_backward_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(p);
+    else gdr_backward_kernel<float><<<grid, kThreads, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace lt2

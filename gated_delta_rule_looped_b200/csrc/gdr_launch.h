@@ -75,6 +75,35 @@ cudaError_t launch_swa_tc(const SwaCall& c, cudaStream_t stream);
 bool swa_cc_supports(int dtype_bf16, int d);
 cudaError_t launch_swa_cc(const SwaCall& c, cudaStream_t stream);
 
+// Backward pass on CUDA cores (fp32 arithmetic; q/k/v/dO fp32 or bf16, gradients fp32), every
+// unit of every loop in one launch (units = T * B * H).
+struct BwCall {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* alpha;
+    const float* beta;
+    const float* S0;       // nullable
+    const void* dO;
+    const float* dSL;      // nullable
+    float* dq;
+    float* dk_out;
+    float* dv_out;
+    float* dalpha;
+    float* dbeta;
+    float* dS0;            // nullable
+    float* ws;
+    int64_t units;
+    int64_t L;
+    int dk;
+    int dv;
+    int per_key;
+    int decay_first;
+    int dtype_bf16;
+};
+size_t backward_workspace_bytes(int64_t units, int64_t L, int dk, int dv);
+cudaError_t launch_backward(const BwCall& c, cudaStream_t stream);
+
 #ifdef LT2_DEBUG
 // Fault injection of the debug build: the producer of every later launch stops before `chunk`.
 cudaError_t debug_set_skip_chunk_scalar(int chunk);

@@ -436,6 +436,78 @@ lt2_status lt2_gdr_prefill_varlen(const lt2_gdr_dims* dims, const lt2_gdr_fused*
     return LT2_OK;
 }
 
+size_t lt2_gdr_backward_workspace_bytes(const lt2_gdr_dims* dims)
+{
+    Sizes sz;
+    if (validate_dims(dims, &sz) != LT2_OK) return 0;
+    return lt2::backward_workspace_bytes(sz.units, dims->L, (int)dims->dk, (int)dims->dv);
+}
+
+lt2_status lt2_gdr_backward(const lt2_gdr_dims* dims, const void* q, const void* k, const void* v,
+                            const float* alpha, const float* beta, const float* S0, const void* dO,
+                            const float* dS_L, float* dq, float* dk, float* dv, float* dalpha, float* dbeta,
+                            float* dS0, void* workspace, size_t workspace_bytes, void* stream)
+{
+    Sizes sz;
+    lt2_status st = validate_dims(dims, &sz);
+    if (st != LT2_OK) return st;
+    if (dims->algo == LT2_ALGO_TENSOR_CORE) return LT2_ERR_UNSUPPORTED;
+    if (sz.units == 0) return LT2_OK;
+    if (!tensor_ok(q, sz.qk) || !tensor_ok(k, sz.qk) || !tensor_ok(v, sz.vo) || !tensor_ok(alpha, sz.al) ||
+        !tensor_ok(beta, sz.be) || !tensor_ok(dO, sz.vo) || !tensor_ok(dq, sz.qk) || !tensor_ok(dk, sz.qk) ||
+        !tensor_ok(dv, sz.vo) || !tensor_ok(dalpha, sz.al) || !tensor_ok(dbeta, sz.be))
+        return LT2_ERR_INVALID_ARGUMENT;
+    if ((S0 && !aligned16(S0)) || (dS_L && !aligned16(dS_L)) || (dS0 && !aligned16(dS0)))
+        return LT2_ERR_INVALID_ARGUMENT;
+    const size_t need = lt2_gdr_backward_workspace_bytes(dims);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+        return LT2_ERR_WORKSPACE;
+    // the gradients are written: none may overlap an input, another gradient or the workspace
+    const Range rin[8] = {range_of(q, sz.qk * sz.esz), range_of(k, sz.qk * sz.esz), range_of(v, sz.vo * sz.esz),
+                          range_of(alpha, sz.al * 4), range_of(beta, sz.be * 4), range_of(dO, sz.vo * sz.esz),
+                          range_of(S0, S0 ? sz.st * 4 : 0), range_of(dS_L, dS_L ? sz.st * 4 : 0)};
+    const Range rout[7] = {range_of(dq, sz.qk * 4), range_of(dk, sz.qk * 4), range_of(dv, sz.vo * 4),
+                           range_of(dalpha, sz.al * 4), range_of(dbeta, sz.be * 4),
+                           range_of(dS0, dS0 ? sz.st * 4 : 0), range_of(workspace, (int64_t)need)};
+    for (int a = 0; a < 7; ++a) {
+        for (const Range& r : rin)
+            if (overlap(rout[a], r)) return LT2_ERR_INVALID_ARGUMENT;
+        for (int b = a + 1; b < 7; ++b)
+            if (overlap(rout[a], rout[b])) return LT2_ERR_INVALID_ARGUMENT;
+    }
+    st = on_current_device({q, k, v, alpha, beta, S0, dO, dS_L, dq, dk, dv, dalpha, dbeta, dS0, workspace});
+    if (st != LT2_OK) return st;
+
+    NvtxRange range("lt2_gdr_backward");
+    lt2::BwCall c;
+    c.q = q;
+    c.k = k;
+    c.v = v;
+    c.alpha = alpha;
+    c.beta = beta;
+    c.S0 = S0;
+    c.dO = dO;
+    c.dSL = dS_L;
+    c.dq = dq;
+    c.dk_out = dk;
+    c.dv_out = dv;
+    c.dalpha = dalpha;
+    c.dbeta = dbeta;
+    c.dS0 = dS0;
+    c.ws = static_cast<float*>(workspace);
+    c.units = sz.units;
+    c.L = dims->L;
+    c.dk = (int)dims->dk;
+    c.dv = (int)dims->dv;
+    c.per_key = is_per_key(dims) ? 1 : 0;
+    c.decay_first = dims->gate == LT2_GATE_PER_KEY_DECAY_FIRST ? 1 : 0;
+    c.dtype_bf16 = dims->dtype == LT2_DTYPE_BF16 ? 1 : 0;
+    cudaError_t e = lt2::launch_backward(c, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "backward (cuda core)");
+    return LT2_OK;
+}
+
 lt2_status lt2_gdr_decode(const lt2_gdr_dims* dims, const void* q, const void* k, const void* v,
                           const float* alpha, const float* beta, float* S, void* o, void* stream)
 {

@@ -223,6 +223,41 @@ lt2_status lt2_gdr_prefill_varlen(const lt2_gdr_dims* dims, const lt2_gdr_fused*
                                   void* stream);
 
 /*
+ * Bytes of device workspace lt2_gdr_backward needs for `dims` (0 for invalid dims): per
+ * (unit, 32-column slice of d_v), a checkpoint of the state every 64 tokens and the 65 states of
+ * one chunk, fp32.  Pure host function, no CUDA call.
+ */
+size_t lt2_gdr_backward_workspace_bytes(const lt2_gdr_dims* dims);
+
+/*
+ * Backward pass of lt2_gdr_prefill (training; the pages train looped models but give no training
+ * kernel): the gradients of loss = sum(dO * o) + sum(dS_L * S_out) with respect to every input of
+ * the recurrence of "LT2 transformer looped a tempo lineare", section "Sostituire il motore",
+ * displayed equation, for every (loop, batch, head) unit.  The reverse-mode derivative of each
+ * line of the token step, swept from the last token to the first with the states recomputed from
+ * 64-token checkpoints (no forward activations are needed from the caller).  fp32 arithmetic on
+ * CUDA cores, every gating and order of lt2_gdr_dims (dims->algo: AUTO or CUDA_CORE;
+ * TENSOR_CORE returns LT2_ERR_UNSUPPORTED; out_dtype is ignored).
+ *   q, k, v, alpha, beta, S0   the forward call's inputs (layouts and dtypes of lt2_gdr_prefill)
+ *   dO          upstream gradient of o, [T][B][H][L][dv], dims->dtype (device, read only)
+ *   dS_L        upstream gradient of S_out, [T][B][H][dk][dv] fp32, or NULL for zero
+ *   dq, dk      [T][B][H][L][dk] fp32 (device, written)
+ *   dv          [T][B][H][L][dv] fp32
+ *   dalpha      fp32, the layout of alpha; dbeta [T][B][H][L] fp32
+ *   dS0         [T][B][H][dk][dv] fp32, or NULL (not wanted)
+ *   workspace   lt2_gdr_backward_workspace_bytes(dims) bytes of device scratch (16-byte aligned)
+ * No gradient may overlap an input, another gradient or the workspace.  Same return convention
+ * as lt2_gdr_prefill (LT2_ERR_WORKSPACE for a missing or short workspace).
+ */
+lt2_status lt2_gdr_backward(const lt2_gdr_dims* dims,
+                            const void* q, const void* k, const void* v,
+                            const float* alpha, const float* beta, const float* S0,
+                            const void* dO, const float* dS_L,
+                            float* dq, float* dk, float* dv, float* dalpha, float* dbeta, float* dS0,
+                            void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/*
  * Decode: one step of the same recurrence ("LT2 transformer looped a tempo lineare", section
  * "Sostituire il motore", displayed equation) for one new token per (loop, batch, head);
  * dims->L must be 1 and dims->algo is ignored.  S [T][B][H][dk][dv] fp32 is read and replaced

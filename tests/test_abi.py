@@ -344,3 +344,35 @@ def test_varlen_bad_dims_and_empty(L):
 
 def test_seqlens_status_has_a_name(L):
     assert lt2.lt2_status_string(lt2.LT2_ERR_SEQLENS) == "LT2_ERR_SEQLENS"
+
+
+# ---- backward (lt2_gdr_backward) ------------------------------------------------------------
+
+def call_backward(dims, ws=BASE + 40 * SPAN, ws_bytes=None, **over):
+    a = addrs(16)
+    names = ["q", "k", "v", "alpha", "beta", "S0", "dO", "dS_L", "dq", "dk", "dv", "dalpha", "dbeta", "dS0"]
+    args = dict(zip(names, a))
+    args.update(over)
+    if ws_bytes is None:
+        ws_bytes = lt2.lt2_gdr_backward_workspace_bytes(dims)
+    return lt2.lt2_gdr_backward(dims, *(args[n] for n in names), ws, ws_bytes, 0)
+
+
+def test_backward_workspace_query(L):
+    d = D(L=150)
+    units, chunks, slices = 2 * 1 * 2, 3, 1                      # d = 32: one 32-column slice
+    assert lt2.lt2_gdr_backward_workspace_bytes(d) == units * slices * (chunks + 65) * 32 * 32 * 4
+    assert L.lt2_gdr_backward_workspace_bytes(None) == 0
+
+
+def test_backward_validation(L):
+    assert call_backward(D(dk=0)) == lt2.LT2_ERR_INVALID_ARGUMENT
+    assert call_backward(D(algo=lt2.LT2_ALGO_TENSOR_CORE)) == lt2.LT2_ERR_UNSUPPORTED
+    assert call_backward(D(), ws=None) == lt2.LT2_ERR_WORKSPACE
+    assert call_backward(D(), ws_bytes=16) == lt2.LT2_ERR_WORKSPACE
+    assert call_backward(D(), dq=None) == lt2.LT2_ERR_INVALID_ARGUMENT
+    q = addrs(1)[0]
+    assert call_backward(D(), dq=q) == lt2.LT2_ERR_INVALID_ARGUMENT          # a gradient over an input
+    dk = addrs(10)[9]
+    assert call_backward(D(), dv=dk + 64) == lt2.LT2_ERR_INVALID_ARGUMENT    # two gradients overlap
+    assert call_backward(D(T=0)) == lt2.LT2_OK
