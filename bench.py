@@ -32,6 +32,7 @@ import sys
 import threading
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -42,7 +43,7 @@ from gated_delta_rule_looped_b200 import dist as gdist  # noqa: E402
 from gated_delta_rule_looped_b200 import inputs  # noqa: E402
 
 HEADLINE = "long_gdn"
-EXTRAS = ("gdn_prefill", "kda_prefill", "decode", "fused_gdn_prefill", "swa_prefill")
+EXTRAS = ("gdn_prefill", "kda_prefill", "decode", "fused_gdn_prefill", "swa_prefill", "backward_gdn")
 
 # Algorithmic work per token-head (d = 128), counted as dense multiply-adds (2 flops each).
 # Scalar gating, 64-token chunks: three d x d state products 6d^2, the four chunk-local
@@ -419,6 +420,80 @@ def run_swa(args, world, sampler, peaks, peak_src):
     return entry
 
 
+# Backward pass, per token-head (d_k = d_v = d): the gradient step reads S_{t-1} and S_t and does
+# about 20 d^2 flops (G += q dO^T, dq = S dO, three column sums, the dk and dalpha row sums, the
+# update of G), and the states it needs cost one forward step, 4 d^2, to recompute.
+BW_FLOP_PER_TOKEN_HEAD = 24 * 128 * 128
+# fp32 CUDA-core peak of the part: 148 SMs x 128 fp32 lanes x 2 flops (FMA) x 1.965 GHz
+FP32_ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def run_backward(args, world, sampler):
+    """The backward pass (lt2_gdr_backward, CUDA cores, fp32) on gdn_prefill's shape: gradients of
+    every input for upstream gradients of o and of the final state, workspace preallocated."""
+    w = inputs.workload("gdn_prefill")
+    x = inputs.make_inputs(w, seed=0, device="cuda")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1)
+    dO = torch.randn(x["v"].shape, generator=g, device="cuda").to(torch.bfloat16)
+    dSL = torch.randn((w.T, w.B, w.H, w.d, w.d), generator=g, device="cuda")
+    dims = lt2.make_dims(w.T, w.B, w.H, w.L, w.d, w.d, lt2.LT2_DTYPE_BF16, lt2.LT2_GATE_SCALAR)
+    f32 = dict(dtype=torch.float32, device="cuda")
+    out = [torch.empty(x["q"].shape, **f32), torch.empty(x["q"].shape, **f32), torch.empty(x["v"].shape, **f32),
+           torch.empty(x["alpha"].shape, **f32), torch.empty(x["beta"].shape, **f32), torch.empty(dSL.shape, **f32)]
+    ws_bytes = lt2.lt2_gdr_backward_workspace_bytes(dims)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+
+    def step():
+        st = lt2.lt2_gdr_backward(dims, x["q"], x["k"], x["v"], x["alpha"], x["beta"], None, dO, dSL, *out, ws,
+                                  ws_bytes)
+        if st != lt2.LT2_OK:
+            raise lt2.Lt2Error(st, "lt2_gdr_backward")
+    steps = max(3, min(args.steps, 5))
+    ms = timed(step, steps, args.warmup, world, sampler, "backward_gdn")
+    check_device_status("backward_gdn")
+    tokheads = w.T * w.B * w.H * w.L
+    tf = tokheads * BW_FLOP_PER_TOKEN_HEAD / (ms * 1e-3) / 1e12
+    entry = {"metric": "looped GDR backward tokens*loops/s (gdn_prefill shape)",
+             "value": gdist.whole_job_rate(w.T * w.B * w.L, world, ms), "unit": "tokens*loops/s",
+             "ms_per_step": ms, "steps": steps,
+             "config": dict(config_of(w, world), **{"pass": "backward", "workspace_bytes": ws_bytes}),
+             "roofline": {"bound": "alu", "kernel": "gdr_backward_kernel", "achieved": tf,
+                          "peak": FP32_ALU_PEAK_TFLOPS, "unit": "TFLOP/s", "frac": tf / FP32_ALU_PEAK_TFLOPS,
+                          "traffic": None,
+                          "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz",
+                          "algorithmic_per_launch": {"flop": tokheads * BW_FLOP_PER_TOKEN_HEAD,
+                                                     "note": "24 d^2 per token-head: the gradient step and "
+                                                             "one recomputed forward step"}},
+             "gpu_launches": steps * 5}
+    if sampler is not None:
+        entry["clocks"] = sampler.summary(["backward_gdn"])
+    del x, out, ws, dO, dSL
+    torch.cuda.empty_cache()
+    return entry
+
+
+def oracle_backward_sample(target_s=4.0):
+    """Time the fp64 backward oracle on this host (one thread): one head-unit of gdn_prefill's
+    shape, a prefix of its tokens growing until about `target_s` has passed."""
+    from oracle import backward as obw
+    w = inputs.workload("gdn_prefill")
+    L = 64
+    while True:
+        ws = inputs.workload("gdn_prefill", T=1, B=1, H=1, L=L)
+        x = {n: t.to(torch.float64).numpy() for n, t in inputs.make_inputs(ws, seed=1).items() if t is not None
+             and n != "subset"}
+        dO = np.random.default_rng(0).normal(size=x["v"].shape)
+        t0 = time.perf_counter()
+        obw.backward(x["q"], x["k"], x["v"], x["alpha"], x["beta"], dO)
+        dt = time.perf_counter() - t0
+        if dt >= target_s / 4 or L >= w.L:
+            break
+        L *= 2
+    desc = f"one (loop, batch, head) unit of gdn_prefill's shape, the first {L} tokens, fp64 backward oracle"
+    return L / dt / w.H, 1, desc
+
+
 def oracle_swa_sample(target_s=5.0):
     """Time the fp64 oracle of the sliding-window mixer on this host (one thread): one whole unit
     of swa_prefill, repeated until about `target_s` has passed."""
@@ -691,6 +766,12 @@ def main():
     for name in extras:
         if name == "fused_gdn_prefill":
             entry = run_fused(args, world, sampler, peaks, peak_src)
+        elif name == "backward_gdn":
+            entry = run_backward(args, world, sampler)
+            if cpu:
+                v, threads, desc = oracle_backward_sample()
+                entry["cpu_baseline"] = {"value": v, "unit": "tokens*loops/s", "cores": threads,
+                                         "kind": "oracle", "sample": desc}
         elif name == "swa_prefill":
             entry = run_swa(args, world, sampler, peaks, peak_src)
             if cpu:
