@@ -47,6 +47,7 @@ EXPORTS = (
     "lt2_gdr_prefill_varlen",
     "lt2_gdr_backward_workspace_bytes",
     "lt2_gdr_backward",
+    "lt2_gdr_backward_static",
     "lt2_swa_prefill",
     "lt2_gdr_last_device_error",
     "lt2_status_string",
@@ -138,6 +139,9 @@ def load_library(path):
         L.lt2_gdr_backward.argtypes = [dims_p, vp, vp, vp, fp, fp, fp, vp, fp, fp, fp, fp, fp, fp, fp, vp,
                                        ctypes.c_size_t, vp]
         L.lt2_gdr_backward.restype = ctypes.c_int
+    if hasattr(L, "lt2_gdr_backward_static"):
+        L.lt2_gdr_backward_static.argtypes = [dims_p, vp, vp, vp, fp, fp, fp, vp, fp, fp, fp, fp, fp, fp, fp, vp]
+        L.lt2_gdr_backward_static.restype = ctypes.c_int
     if hasattr(L, "lt2_swa_prefill"):
         L.lt2_swa_prefill.argtypes = [ctypes.POINTER(lt2_swa_dims), vp, vp, vp, vp, vp]
         L.lt2_swa_prefill.restype = ctypes.c_int
@@ -227,6 +231,13 @@ def lt2_gdr_backward(dims, q, k, v, alpha, beta, S0, dO, dS_L, dq, dk, dv, dalph
     return lib().lt2_gdr_backward(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(dO),
                                   _p(dS_L), _p(dq), _p(dk), _p(dv), _p(dalpha), _p(dbeta), _p(dS0), _p(workspace),
                                   int(workspace_bytes), _stream(stream))
+
+
+def lt2_gdr_backward_static(dims, q, k, v, alpha, beta, S0, dO, dS_L, dq, dk, dv, dalpha, dbeta, dS0,
+                            stream=None):
+    return lib().lt2_gdr_backward_static(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0),
+                                         _p(dO), _p(dS_L), _p(dq), _p(dk), _p(dv), _p(dalpha), _p(dbeta),
+                                         _p(dS0), _stream(stream))
 
 
 def lt2_swa_prefill(dims, q, k, v, o, stream=None):

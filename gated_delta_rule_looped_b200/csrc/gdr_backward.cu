@@ -31,6 +31,9 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "gdr_common.cuh"
 #include "gdr_launch.h"
 #include "gdr_nvtx.h"
@@ -262,6 +265,16 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
     }
 }
 
+// Scratch of the allocation-free entry point (lt2_gdr_backward_static): a fixed 64 MiB array in
+// device memory, reserved on every GPU that loads this library until the process exits.  For
+// callers that may not allocate device memory themselves: a host program whose device memory is
+// all handed out by someone else's allocator, or a service that must not call cudaMalloc once it
+// is serving (the call can block the device).  Every call of that entry point on a device uses
+// this one array, so calls that overlap on the GPU -- from two streams or two host threads --
+// overwrite each other's scratch and must be serialised by the caller.
+constexpr size_t kStaticScratchBytes = size_t(64) << 20;
+static __device__ __align__(256) float g_static_scratch[kStaticScratchBytes / sizeof(float)];
+
 __global__ void zero_kernel(float* x, int64_t n)
 {
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
@@ -270,6 +283,36 @@ __global__ void zero_kernel(float* x, int64_t n)
 }
 
 }  // namespace bw
+
+size_t backward_static_scratch_bytes() { return bw::kStaticScratchBytes; }
+
+// The device address of the static scratch on the current device.  In host code the array's name
+// is only a host-side stand-in, so the address comes from cudaGetSymbolAddress, once per device
+// with that device current, and is cached.
+cudaError_t backward_static_scratch(float** out)
+{
+    constexpr int kMaxDevices = 64;
+    static std::atomic<float*> cache[kMaxDevices];
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    float* p = cache[dev].load(std::memory_order_acquire);
+    if (!p) {
+        std::lock_guard<std::mutex> lock(mu);
+        p = cache[dev].load(std::memory_order_acquire);
+        if (!p) {
+            void* addr = nullptr;
+            e = cudaGetSymbolAddress(&addr, bw::g_static_scratch);
+            if (e != cudaSuccess) return e;
+            p = static_cast<float*>(addr);
+            cache[dev].store(p, std::memory_order_release);
+        }
+    }
+    *out = p;
+    return cudaSuccess;
+}
 
 size_t backward_workspace_bytes(int64_t units, int64_t L, int dk, int dv)
 {

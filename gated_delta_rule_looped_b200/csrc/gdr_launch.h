@@ -102,6 +102,10 @@ struct BwCall {
     int dtype_bf16;
 };
 size_t backward_workspace_bytes(int64_t units, int64_t L, int dk, int dv);
+// The fixed scratch array of the allocation-free backward entry point: its size, and its device
+// address on the current device (looked up on the first call on each device).
+size_t backward_static_scratch_bytes();
+cudaError_t backward_static_scratch(float** out);
 cudaError_t launch_backward(const BwCall& c, cudaStream_t stream);
 
 #ifdef LT2_DEBUG

@@ -508,6 +508,25 @@ lt2_status lt2_gdr_backward(const lt2_gdr_dims* dims, const void* q, const void*
     return LT2_OK;
 }
 
+lt2_status lt2_gdr_backward_static(const lt2_gdr_dims* dims, const void* q, const void* k, const void* v,
+                                   const float* alpha, const float* beta, const float* S0, const void* dO,
+                                   const float* dS_L, float* dq, float* dk, float* dv, float* dalpha,
+                                   float* dbeta, float* dS0, void* stream)
+{
+    Sizes sz;
+    lt2_status st = validate_dims(dims, &sz);
+    if (st != LT2_OK) return st;
+    if (sz.units == 0) return lt2_gdr_backward(dims, q, k, v, alpha, beta, S0, dO, dS_L, dq, dk, dv, dalpha,
+                                               dbeta, dS0, nullptr, 0, stream);
+    const size_t need = lt2_gdr_backward_workspace_bytes(dims);
+    if (need > lt2::backward_static_scratch_bytes()) return LT2_ERR_WORKSPACE;
+    float* scratch = nullptr;
+    const cudaError_t e = lt2::backward_static_scratch(&scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress (static backward scratch)");
+    return lt2_gdr_backward(dims, q, k, v, alpha, beta, S0, dO, dS_L, dq, dk, dv, dalpha, dbeta, dS0, scratch,
+                            lt2::backward_static_scratch_bytes(), stream);
+}
+
 lt2_status lt2_gdr_decode(const lt2_gdr_dims* dims, const void* q, const void* k, const void* v,
                           const float* alpha, const float* beta, float* S, void* o, void* stream)
 {

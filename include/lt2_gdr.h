@@ -258,6 +258,30 @@ lt2_status lt2_gdr_backward(const lt2_gdr_dims* dims,
                             void* stream);
 
 /*
+ * lt2_gdr_backward without a workspace argument, for callers that cannot allocate device memory:
+ * a program whose device memory is handed out entirely by a host application's or framework's own
+ * allocator, or a service that must not call cudaMalloc while it serves (the call can block the
+ * whole device).  This entry point allocates nothing: its scratch is a fixed 64 MiB array of
+ * device memory inside the library, reserved on every GPU that loads the library until the
+ * process exits.  (The paper has no counterpart: this is the library's own arrangement.)
+ *   Arguments, layouts and results: exactly those of lt2_gdr_backward.
+ *   Limit: a problem whose lt2_gdr_backward_workspace_bytes(dims) exceeds 64 MiB (67108864 bytes)
+ *          returns LT2_ERR_WORKSPACE before any launch; for d_k = d_v = 128 that is 12 (loop,
+ *          batch, head) units of 1,024 tokens, or 5 units of 8,192.
+ *   Set-up: the first call on each device looks up the array's device address (with that device
+ *          current) and keeps it; make that first call before any stream capture.
+ *   Sharing: every call on a device uses the same array.  Nothing in it has to start at zero
+ *          (a call writes each word before it reads it), but calls that overlap on the GPU, from
+ *          two streams or two host threads, race on it: serialise them.
+ */
+lt2_status lt2_gdr_backward_static(const lt2_gdr_dims* dims,
+                                   const void* q, const void* k, const void* v,
+                                   const float* alpha, const float* beta, const float* S0,
+                                   const void* dO, const float* dS_L,
+                                   float* dq, float* dk, float* dv, float* dalpha, float* dbeta, float* dS0,
+                                   void* stream);
+
+/*
  * Decode: one step of the same recurrence ("LT2 transformer looped a tempo lineare", section
  * "Sostituire il motore", displayed equation) for one new token per (loop, batch, head);
  * dims->L must be 1 and dims->algo is ignored.  S [T][B][H][dk][dv] fp32 is read and replaced
