@@ -501,3 +501,68 @@ def backward(q, k, v, alpha, beta, dO, S0=None, dS_L=None, per_key=None, order="
         if st != LT2_OK:
             raise Lt2Error(st, "lt2_gdr_backward")
         return g
+
+
+def prefill_host(q, k, v, alpha, beta, o, S_out, S0=None, per_key=None, order="delta_first", device=None,
+                 slots=2):
+    """The looped prefill on inputs that live in pinned host memory, with o and S_out written back
+    to pinned host tensors: the loops run one at a time through ``slots`` device buffers on three
+    streams, so that the host-to-device copy of loop tau + 1, the call on loop tau (lt2_gdr_prefill
+    with T = 1) and the device-to-host copy of loop tau - 1 overlap (PCIe moves data both ways at
+    once).  Device memory: ``slots`` loops' inputs and outputs.  The work is enqueued behind the
+    current stream of ``device`` and that stream waits for all of it, so the caller synchronises as
+    usual.  Shapes as in ``prefill``; q ... S_out are host tensors (pinned for the copies to
+    overlap)."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
+    if q.is_cuda:
+        raise ValueError("prefill_host takes host tensors; use prefill for device tensors")
+    T = q.shape[0]
+    with torch.cuda.device(dev):
+        cur = torch.cuda.current_stream()
+        s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        for st in (s_in, s_run, s_out):
+            st.wait_stream(cur)
+        ins = ("q", "k", "v", "alpha", "beta") + (("S0",) if S0 is not None else ())
+        host = dict(q=q, k=k, v=v, alpha=alpha, beta=beta, S0=S0)
+        buf = [{n: torch.empty(host[n].shape[1:], dtype=host[n].dtype, device=dev) for n in ins} for _ in range(slots)]
+        obuf = [(torch.empty(o.shape[1:], dtype=o.dtype, device=dev),
+                 torch.empty(S_out.shape[1:], dtype=S_out.dtype, device=dev)) for _ in range(slots)]
+        in_free = [None] * slots      # the call on the slot's previous loop is done with its inputs
+        out_free = [None] * slots     # the slot's previous outputs have reached the host
+        out_kind = "same" if o.dtype == q.dtype else ("f32" if o.dtype == torch.float32 else "bf16")
+        for tau in range(T):
+            sl = tau % slots
+            with torch.cuda.stream(s_in):
+                if in_free[sl] is not None:
+                    s_in.wait_event(in_free[sl])
+                for n in ins:
+                    buf[sl][n].copy_(host[n][tau], non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(s_in)
+            with torch.cuda.stream(s_run):
+                s_run.wait_event(ready)
+                if out_free[sl] is not None:
+                    s_run.wait_event(out_free[sl])
+                b = buf[sl]
+                prefill(b["q"][None], b["k"][None], b["v"][None], b["alpha"][None], b["beta"][None],
+                        S0=b["S0"][None] if S0 is not None else None, per_key=per_key, o=obuf[sl][0][None],
+                        S_out=obuf[sl][1][None], out=out_kind, stream=s_run, order=order)
+                done = torch.cuda.Event()
+                done.record(s_run)
+                in_free[sl] = done
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done)
+                o[tau].copy_(obuf[sl][0], non_blocking=True)
+                S_out[tau].copy_(obuf[sl][1], non_blocking=True)
+                back = torch.cuda.Event()
+                back.record(s_out)
+                out_free[sl] = back
+        cur.wait_stream(s_out)
+        cur.wait_stream(s_run)
+        # the slot buffers stay alive until the streams are done with them
+        for t in [x for b in buf for x in b.values()] + [x for pair in obuf for x in pair]:
+            t.record_stream(s_in)
+            t.record_stream(s_run)
+            t.record_stream(s_out)
+    return o, S_out

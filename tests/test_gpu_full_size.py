@@ -113,3 +113,19 @@ def test_full_size_decode():
                                       to_np(sel(step["beta"])), S_hist)
     check("decode o (sampled units)", sel(o), o_ref, TOL["bf16"])
     check("decode S (sampled units)", sel(S_dec), S_ref, TOL["bf16"])
+
+
+@pytest.mark.gpu
+def test_prefill_host_equals_device_prefill():
+    # inputs in pinned host memory, loops streamed through two device slots with the copies
+    # overlapped: the same numbers as the device call, bit for bit
+    w = inputs.workload("gdn_prefill", T=3, B=1, H=2, L=200, s0="normal")
+    x = inputs.make_inputs(w, seed=4, device="cuda")
+    o_ref, S_ref = lt2.prefill(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S0=x["S0"], per_key=False)
+    h = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "alpha", "beta", "S0")}
+    o_h = torch.empty(o_ref.shape, dtype=o_ref.dtype).pin_memory()
+    S_h = torch.empty(S_ref.shape, dtype=S_ref.dtype).pin_memory()
+    lt2.prefill_host(h["q"], h["k"], h["v"], h["alpha"], h["beta"], o_h, S_h, S0=h["S0"])
+    torch.cuda.synchronize()
+    assert lt2.lt2_gdr_last_device_error() == lt2.LT2_OK
+    assert torch.equal(o_h, o_ref.cpu()) and torch.equal(S_h, S_ref.cpu())
