@@ -24,8 +24,10 @@
 //            64-token chunk (a checkpoint) in the workspace;
 //   phase B  takes the chunks from the last: it recomputes the chunk's states from its checkpoint
 //            into the workspace, then sweeps the chunk backwards.
-// Per token the three column sums the step needs (k^T S_{t-1} or k^T R, k^T G, k^T Diag(alpha) G)
-// come from one shared-memory reduction; the row sums (dq, dk, dalpha) are warp reductions whose
+// A chunk's inputs are staged in shared memory once per phase.  Per token the three column sums
+// the step needs (k^T S_{t-1} or k^T R, k^T G, k^T Diag(alpha) G) come from one shared-memory
+// reduction, and the sweep reuses S_{t-1} of token t+1 as S_t of token t and loads the next
+// S_{t-1} one token ahead; the row sums (dq, dk, dalpha) are warp reductions whose
 // slice partials are added into the fp32 outputs with atomics (zeroed first by this library).
 // dv and dS_0 belong to one block each and are stored directly.
 #include <cuda_bf16.h>
@@ -54,6 +56,28 @@ __device__ __forceinline__ float warp_sum(float x)
     #pragma unroll
     for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
     return x;
+}
+
+// Sums over the 32 lanes of a warp of 16 values per lane at once (recursive halving: 16 shuffles
+// instead of 16 x 5).  On return lane l holds the total of row row16(l); lanes l and l ^ 1 hold
+// the same row.
+__device__ __forceinline__ float rows_sum16(float (&v)[16], int lane)
+{
+    #pragma unroll
+    for (int half = 8, off = 16; half >= 1; half >>= 1, off >>= 1) {
+        const bool upper = (lane & off) != 0;
+        #pragma unroll
+        for (int i = 0; i < half; ++i) {
+            const float send = upper ? v[i] : v[i + half];
+            const float keep = upper ? v[i + half] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+__device__ __forceinline__ int row16(int lane)
+{
+    return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
 }
 
 struct Params {
@@ -86,10 +110,18 @@ __host__ __device__ inline int64_t ws_floats_per_block(int64_t L, int dk)
     return ((L + kChunk - 1) / kChunk + kChunk + 1) * static_cast<int64_t>(dk) * kCols;
 }
 
+// Shared memory of a block: one chunk's inputs in fp32 (k, q, alpha rows, beta, and the slice's v
+// and dO columns) and the reduction buffers.
+__host__ __device__ inline size_t smem_bytes(int dk, int per_key)
+{
+    const size_t na = per_key ? dk : 1;
+    return (static_cast<size_t>(kChunk) * (2 * dk + na + 1 + 2 * kCols) + 2 * 3 * 8 * kCols) * sizeof(float);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
 {
-    __shared__ float red[2][3][8][kCols];
+    extern __shared__ __align__(16) float smem[];
     const int dk = p.dk, dv = p.dv, rpw = dk >> 3;
     const int w = threadIdx.x >> 5, c = threadIdx.x & 31;
     const int j0 = blockIdx.y * kCols;
@@ -99,6 +131,13 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
     const int64_t u = blockIdx.x, L = p.L;
     const int r0 = w * rpw;
     const int na = p.per_key ? dk : 1;
+    float* sk = smem;                              // [64][dk]
+    float* sq = sk + kChunk * dk;                  // [64][dk]
+    float* sa = sq + kChunk * dk;                  // [64][na]
+    float* sbe = sa + kChunk * na;                 // [64]
+    float* sv = sbe + kChunk;                      // [64][32]
+    float* sdo = sv + kChunk * kCols;              // [64][32]
+    float (*red)[3][8][kCols] = reinterpret_cast<float (*)[3][8][kCols]>(sdo + kChunk * kCols);
 
     const T* q = static_cast<const T*>(p.q) + u * L * dk;
     const T* k = static_cast<const T*>(p.k) + u * L * dk;
@@ -112,28 +151,44 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
     float* st = ws + static_cast<int64_t>(nck) * dk * kCols;   // [65][dk][32]
     auto at = [&](float* base, int idx, int m) -> float& { return base[(static_cast<int64_t>(idx) * dk + r0 + m) * kCols + c]; };
 
-    // one forward step of the recurrence on this thread's part of the state
-    auto step = [&](float (&s)[kMaxRows], int64_t t, int buf) {
-        float kr[kMaxRows], ar[kMaxRows];
-        const float b = be[t];
-        #pragma unroll
-        for (int m = 0; m < kMaxRows; ++m) {
-            kr[m] = m < rpw ? ld(k + t * dk + r0 + m) : 0.f;
-            ar[m] = m < rpw ? (p.per_key ? al[t * dk + r0 + m] : al[t]) : 1.f;
+    // the inputs of tokens t0 .. t0+n-1 into shared memory (q and dO only for the reverse sweep)
+    auto load_chunk = [&](int64_t t0, int n, bool with_q) {
+        __syncthreads();                                        // the previous chunk is consumed
+        for (int i = threadIdx.x; i < n * dk; i += kThreads) {
+            sk[i] = ld(k + t0 * dk + i);
+            if (with_q) sq[i] = ld(q + t0 * dk + i);
         }
+        for (int i = threadIdx.x; i < n * na; i += kThreads) sa[i] = al[t0 * na + i];
+        for (int i = threadIdx.x; i < n; i += kThreads) sbe[i] = be[t0 + i];
+        for (int i = threadIdx.x; i < n * kCols; i += kThreads) {
+            const int tt = i / kCols, cc = i - tt * kCols;
+            const bool on = j0 + cc < dv;
+            sv[i] = on ? ld(v + (t0 + tt) * dv + j0 + cc) : 0.f;
+            if (with_q) sdo[i] = on ? ld(dO + (t0 + tt) * dv + j0 + cc) : 0.f;
+        }
+        __syncthreads();
+    };
+    auto arow = [&](int tau, int m) -> float { return p.per_key ? sa[tau * dk + r0 + m] : sa[tau]; };
+
+    // one forward step of the recurrence (token tau of the loaded chunk) on this thread's state
+    auto step = [&](float (&s)[kMaxRows], int tau, int buf) {
+        const float b = sbe[tau];
         float pe = 0.f;
         #pragma unroll
-        for (int m = 0; m < kMaxRows; ++m) pe += kr[m] * (p.decay_first ? ar[m] * s[m] : s[m]);
+        for (int m = 0; m < kMaxRows; ++m)
+            if (m < rpw) pe += sk[tau * dk + r0 + m] * (p.decay_first ? arow(tau, m) * s[m] : s[m]);
         red[buf][0][w][c] = pe;
         __syncthreads();
         float e = 0.f;
         #pragma unroll
         for (int ww = 0; ww < 8; ++ww) e += red[buf][0][ww][c];
-        const float vj = active ? ld(v + t * dv + j) : 0.f;
+        const float vj = sv[tau * kCols + c];
         #pragma unroll
         for (int m = 0; m < kMaxRows; ++m) {
-            if (p.decay_first) s[m] = ar[m] * s[m] + b * kr[m] * (vj - e);
-            else s[m] = ar[m] * (s[m] - b * kr[m] * e) + b * kr[m] * vj;
+            if (m >= rpw) break;
+            const float kr = sk[tau * dk + r0 + m], ar = arow(tau, m);
+            if (p.decay_first) s[m] = ar * s[m] + b * kr * (vj - e);
+            else s[m] = ar * (s[m] - b * kr * e) + b * kr * vj;
         }
     };
 
@@ -142,15 +197,15 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
     const float* S0 = p.S0 ? p.S0 + u * static_cast<int64_t>(dk) * dv : nullptr;
     #pragma unroll
     for (int m = 0; m < kMaxRows; ++m) s[m] = (m < rpw && active && S0) ? S0[static_cast<int64_t>(r0 + m) * dv + j] : 0.f;
-    for (int64_t t = 0; t < L; ++t) {
-        if (t % kChunk == 0) {
-            #pragma unroll
-            for (int m = 0; m < kMaxRows; ++m)
-                if (m < rpw) at(ck, static_cast<int>(t / kChunk), m) = s[m];
-        }
-        step(s, t, static_cast<int>(t & 1));
+    for (int ci = 0; ci < nck; ++ci) {
+        const int64_t t0 = static_cast<int64_t>(ci) * kChunk;
+        const int n = static_cast<int>(L - t0 < kChunk ? L - t0 : kChunk);
+        #pragma unroll
+        for (int m = 0; m < kMaxRows; ++m)
+            if (m < rpw) at(ck, ci, m) = s[m];
+        load_chunk(t0, n, false);
+        for (int tau = 0; tau < n; ++tau) step(s, tau, tau & 1);
     }
-    __syncthreads();                                   // the reduction buffers are reused below
 
     // ---- phase B: chunks from the last, each recomputed, then swept backwards ----
     float G[kMaxRows];
@@ -160,49 +215,58 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
     for (int ci = nck - 1; ci >= 0; --ci) {
         const int64_t t0 = static_cast<int64_t>(ci) * kChunk;
         const int n = static_cast<int>(L - t0 < kChunk ? L - t0 : kChunk);
+        load_chunk(t0, n, true);
         #pragma unroll
         for (int m = 0; m < kMaxRows; ++m) {
             s[m] = m < rpw ? at(ck, ci, m) : 0.f;
             if (m < rpw) at(st, 0, m) = s[m];
         }
         for (int tau = 0; tau < n; ++tau) {
-            step(s, t0 + tau, tau & 1);
-            #pragma unroll
-            for (int m = 0; m < kMaxRows; ++m)
-                if (m < rpw) at(st, tau + 1, m) = s[m];
+            step(s, tau, tau & 1);
+            if (tau + 1 < n) {                                  // S_t of the last token stays in s
+                #pragma unroll
+                for (int m = 0; m < kMaxRows; ++m)
+                    if (m < rpw) at(st, tau + 1, m) = s[m];
+            }
         }
         __syncthreads();
+        // S_t arrives from the previous step (S_{t-1} of token t+1); S_{t-1} is loaded one token ahead
+        float sc[kMaxRows], sp[kMaxRows];
+        #pragma unroll
+        for (int m = 0; m < kMaxRows; ++m) {
+            sc[m] = s[m];
+            sp[m] = m < rpw ? at(st, n - 1, m) : 0.f;
+        }
         for (int tau = n - 1; tau >= 0; --tau) {
-            const int64_t t = t0 + tau;
             const int buf = tau & 1;
-            float sp[kMaxRows], sc[kMaxRows], kr[kMaxRows], ar[kMaxRows];
-            const float b = be[t];
-            const float vj = active ? ld(v + t * dv + j) : 0.f;
-            const float oj = active ? ld(dO + t * dv + j) : 0.f;
+            const int64_t t = t0 + tau;
+            float spn[kMaxRows];                               // S_{t-2}, for the next token
             #pragma unroll
-            for (int m = 0; m < kMaxRows; ++m) {
-                const bool on = m < rpw;
-                sp[m] = on ? at(st, tau, m) : 0.f;
-                sc[m] = on ? at(st, tau + 1, m) : 0.f;
-                kr[m] = on ? ld(k + t * dk + r0 + m) : 0.f;
-                ar[m] = on ? (p.per_key ? al[t * dk + r0 + m] : al[t]) : 1.f;
-                const float qr = on ? ld(q + t * dk + r0 + m) : 0.f;
-                G[m] += qr * oj;                       // from o_t = S_t^T q_t
-            }
+            for (int m = 0; m < kMaxRows; ++m) spn[m] = (m < rpw && tau > 0) ? at(st, tau - 1, m) : 0.f;
+            const float b = sbe[tau];
+            const float vj = sv[tau * kCols + c];
+            const float oj = sdo[tau * kCols + c];
+            #pragma unroll
+            for (int m = 0; m < kMaxRows; ++m)
+                if (m < rpw) G[m] += sq[tau * dk + r0 + m] * oj;   // from o_t = S_t^T q_t
             // dq_t = S_t dO_t: row sums over this slice's columns
-            #pragma unroll
-            for (int m = 0; m < kMaxRows; ++m) {
-                if (m >= rpw) break;
-                const float x = warp_sum(sc[m] * oj);
-                if (c == 0) atomicAdd(p.dq + (u * L + t) * dk + r0 + m, x);
+            {
+                float x[kMaxRows];
+                #pragma unroll
+                for (int m = 0; m < kMaxRows; ++m) x[m] = m < rpw ? sc[m] * oj : 0.f;
+                const float tot = rows_sum16(x, c);
+                const int m = row16(c);
+                if (!(c & 1) && m < rpw) atomicAdd(p.dq + (u * L + t) * dk + r0 + m, tot);
             }
             // the column sums of this step, one reduction: e, k^T G, k^T Diag(alpha) G
             float pe = 0.f, pg = 0.f, pd = 0.f;
             #pragma unroll
             for (int m = 0; m < kMaxRows; ++m) {
-                pe += kr[m] * (p.decay_first ? ar[m] * sp[m] : sp[m]);
-                pg += kr[m] * G[m];
-                pd += kr[m] * ar[m] * G[m];
+                if (m >= rpw) break;
+                const float kr = sk[tau * dk + r0 + m], ar = arow(tau, m);
+                pe += kr * (p.decay_first ? ar * sp[m] : sp[m]);
+                pg += kr * G[m];
+                pd += kr * ar * G[m];
             }
             red[buf][0][w][c] = pe;
             red[buf][1][w][c] = pg;
@@ -222,40 +286,48 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
                 const float x = warp_sum(tb);
                 if (c == 0) atomicAdd(p.dbeta + u * L + t, x);
             }
-            float dal_sum = 0.f;
+            float dkx[kMaxRows], dax[kMaxRows];
             #pragma unroll
             for (int m = 0; m < kMaxRows; ++m) {
-                if (m >= rpw) break;
-                float dkx, dax;
+                dkx[m] = dax[m] = 0.f;
+                if (m >= rpw) continue;
+                const float kr = sk[tau * dk + r0 + m], ar = arow(tau, m);
                 if (p.decay_first) {
-                    const float R = ar[m] * sp[m];
-                    const float dR = G[m] - b * kr[m] * kG;
-                    dkx = b * G[m] * (vj - e) - b * R * kG;
-                    dax = dR * sp[m];
-                    G[m] = ar[m] * dR;
+                    const float R = ar * sp[m];
+                    const float dR = G[m] - b * kr * kG;
+                    dkx[m] = b * G[m] * (vj - e) - b * R * kG;
+                    dax[m] = dR * sp[m];
+                    G[m] = ar * dR;
                 } else {
-                    const float P = sp[m] - b * kr[m] * e;
-                    const float dP = ar[m] * G[m];
-                    dkx = b * G[m] * vj - b * (sp[m] * kdP + dP * e);
-                    dax = G[m] * P;
-                    G[m] = dP - b * kr[m] * kdP;
+                    const float P = sp[m] - b * kr * e;
+                    const float dP = ar * G[m];
+                    dkx[m] = b * G[m] * vj - b * (sp[m] * kdP + dP * e);
+                    dax[m] = G[m] * P;
+                    G[m] = dP - b * kr * kdP;
                 }
-                if (!active) dkx = dax = 0.f;
-                const float dks = warp_sum(dkx);
-                if (c == 0) atomicAdd(p.gdk + (u * L + t) * dk + r0 + m, dks);
+                if (!active) dkx[m] = dax[m] = 0.f;
+            }
+            {
+                const int m = row16(c);
+                const float dks = rows_sum16(dkx, c);
+                if (!(c & 1) && m < rpw) atomicAdd(p.gdk + (u * L + t) * dk + r0 + m, dks);
                 if (p.per_key) {
-                    const float das = warp_sum(dax);
-                    if (c == 0) atomicAdd(p.dalpha + (u * L + t) * dk + r0 + m, das);
+                    const float das = rows_sum16(dax, c);
+                    if (!(c & 1) && m < rpw) atomicAdd(p.dalpha + (u * L + t) * dk + r0 + m, das);
                 } else {
-                    dal_sum += dax;
+                    float dal_sum = 0.f;
+                    #pragma unroll
+                    for (int mm = 0; mm < kMaxRows; ++mm) dal_sum += dax[mm];
+                    const float x = warp_sum(dal_sum);
+                    if (c == 0) atomicAdd(p.dalpha + u * L + t, x);
                 }
             }
-            if (!p.per_key) {
-                const float x = warp_sum(dal_sum);
-                if (c == 0) atomicAdd(p.dalpha + u * L + t, x);
+            #pragma unroll
+            for (int m = 0; m < kMaxRows; ++m) {
+                sc[m] = sp[m];
+                sp[m] = spn[m];
             }
         }
-        __syncthreads();
     }
     if (p.dS0 && active) {
         float* o = p.dS0 + u * static_cast<int64_t>(dk) * dv;
@@ -356,8 +428,11 @@ cudaError_t launch_backward(const BwCall& c, cudaStream_t stream)
     p.per_key = c.per_key;
     p.decay_first = c.decay_first;
     const dim3 grid(static_cast<unsigned>(c.units), static_cast<unsigned>((c.dv + kCols - 1) / kCols), 1);
-    if (c.dtype_bf16) gdr_backward_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(p);
-    else gdr_backward_kernel<float><<<grid, kThreads, 0, stream>>>(p);
+    const size_t smem = smem_bytes(c.dk, c.per_key);
+    auto kernel = c.dtype_bf16 ? gdr_backward_kernel<__nv_bfloat16> : gdr_backward_kernel<float>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kernel<<<grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
