@@ -58,6 +58,11 @@ constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + 2 * Q_PANEL;
 constexpr uint32_t OFF_V = OFF_K + 2 * KV_STAGE;
 constexpr uint32_t OFF_BAR = OFF_V + 2 * KV_STAGE;
+// P_FULL and PV_DONE come in pairs (even and odd blocks): the softmax warps may run a block ahead of
+// the MMA issuer, and with one barrier of each the waiter could then see two phases complete at
+// once and misread the parity.  Each of a pair completes once every two blocks, at most one phase
+// ahead of its waiter (Q K_{j+2}^T, which the softmax of block j+2 needs, is issued after
+// O += P_j V_j).
 enum Bar : uint32_t {
     B_Q = 0,          // Q landed
     B_K_FULL = 1,     // [2] K of a stage landed
@@ -66,10 +71,10 @@ enum Bar : uint32_t {
     B_V_EMPTY = 7,    // [2] O += P V is done with a V stage
     B_S_FULL = 9,     // S = Q K^T done
     B_S_FREE = 10,    // the softmax warps have read S
-    B_P_FULL = 11,    // P written (and O rescaled when needed)
-    B_PV_DONE = 12,   // O += P V done
-    B_DRAIN = 13,     // drain on abort (MMA issuer)
-    B_COUNT = 14
+    B_P_FULL = 11,    // [2] P_j written (and O rescaled when needed), for even and odd j
+    B_PV_DONE = 13,   // [2] O += P_j V_j done, for even and odd j
+    B_DRAIN = 15,     // drain on abort (MMA issuer)
+    B_COUNT = 16
 };
 constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + B_COUNT * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 16;
@@ -78,7 +83,8 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 
 // TMEM columns (lane = query row)
 constexpr uint32_t TM_S = 0;           // S, fp32 (64 columns)
-constexpr uint32_t TM_P = 64;          // P, bf16 pairs (32 columns): A operand of O += P V
+constexpr uint32_t TM_P = 64;          // P_j, bf16 pairs, two buffers of 32 columns (j even, odd):
+                                       // the A operand of O += P_j V_j
 constexpr uint32_t TM_O = 128;         // O, fp32 (128 columns)
 constexpr uint32_t TM_COLS = 256;
 
@@ -181,7 +187,7 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         for (uint32_t b = 0; b < B_COUNT; ++b)
-            mbar_init(bar_addr(sb, b), b == B_S_FREE || b == B_P_FULL ? kSoftThreads : 1);
+            mbar_init(bar_addr(sb, b), b == B_S_FREE || b == B_P_FULL || b == B_P_FULL + 1 ? kSoftThreads : 1);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -257,17 +263,17 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // O += P_j V_j, once the softmax warps have written P_j and V_j has landed
             auto issue_pv = [&](int j) -> bool {
                 if (!mbar_wait(bar_addr(sb, B_V_FULL + (j & 1)), (j >> 1) & 1, abort_flag, err, kTimeoutNs) ||
-                    !mbar_wait(bar_addr(sb, B_P_FULL), j & 1, abort_flag, err, kTimeoutNs))
+                    !mbar_wait(bar_addr(sb, B_P_FULL + (j & 1)), (j >> 1) & 1, abort_flag, err, kTimeoutNs))
                     return false;
                 tc_fence_after();
                 if (elect_one(issuer)) {
                     const uint32_t vt = sb + OFF_V + (j & 1) * KV_STAGE;
                     #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        umma_f16_tmem_a(tmem + TM_O, tmem + TM_P + 8 * k,
+                        umma_f16_tmem_a(tmem + TM_O, tmem + TM_P + 32 * (j & 1) + 8 * k,
                                         smem_desc_sw128(vt + k * 2048, KV_PANEL, 1024), ID_PV,
                                         (j > 0 || k > 0) ? 1u : 0u);
-                    umma_commit(bar_addr(sb, B_PV_DONE));
+                    umma_commit(bar_addr(sb, B_PV_DONE + (j & 1)));
                     umma_commit(bar_addr(sb, B_V_EMPTY + (j & 1)));
                 }
                 return true;
@@ -362,21 +368,32 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             l = l * corr + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
             m = mnew;
-            // P is single-buffered and O may need rescaling: the previous O += P V must be done
-            if (idx > 0 && !grp.wait(bar_addr(sb, B_PV_DONE), (idx - 1) & 1)) {
+            // P is double-buffered: P_idx takes the buffer of P_{idx-2}, free once O += P_{idx-2} V
+            // is done (barrier idx & 1 completes once every two blocks: phase (idx - 2) / 2)
+            if (idx >= 2 && !grp.wait(bar_addr(sb, B_PV_DONE + (idx & 1)), ((idx - 2) >> 1) & 1)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            if (__any_sync(0xffffffffu, corr != 1.f)) rescale_o(tmem + TM_O + lane_addr, corr);
-            tmem_st16(tmem + TM_P + lane_addr, *reinterpret_cast<uint32_t(*)[16]>(pk));
-            tmem_st16(tmem + TM_P + lane_addr + 16, *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
+            if (__any_sync(0xffffffffu, corr != 1.f)) {
+                // a raised maximum rescales O, so the latest O += P V (block idx - 1) must be done;
+                // only this warp waits (a timeout raises the CTA's abort, which the group's next
+                // wait sees)
+                if (idx >= 1)
+                    mbar_wait(bar_addr(sb, B_PV_DONE + ((idx - 1) & 1)), ((idx - 1) >> 1) & 1, abort_flag, err,
+                              kTimeoutNs);
+                tc_fence_after();
+                rescale_o(tmem + TM_O + lane_addr, corr);
+            }
+            const uint32_t tp = tmem + TM_P + 32 * (idx & 1) + lane_addr;
+            tmem_st16(tp, *reinterpret_cast<uint32_t(*)[16]>(pk));
+            tmem_st16(tp + 16, *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar_addr(sb, B_P_FULL));
+            mbar_arrive(bar_addr(sb, B_P_FULL + (idx & 1)));
         }
         // o = O / l after the last O += P V
-        if (ok && grp.wait(bar_addr(sb, B_PV_DONE), (nblk - 1) & 1)) {
+        if (ok && grp.wait(bar_addr(sb, B_PV_DONE + ((nblk - 1) & 1)), ((nblk - 1) >> 1) & 1)) {
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
             float* o32 = !p.out_bf16 && qi < L ? static_cast<float*>(p.o) + (static_cast<int64_t>(unit) * L + qi) * 128
