@@ -643,10 +643,8 @@ __device__ __forceinline__ void issue_gram(uint32_t sb, uint32_t tmem, uint32_t 
 __device__ __noinline__ int issue_gram_of(int k, uint32_t sb, uint32_t tmem, int lane, volatile int* abort_flag,
                                           unsigned int* err, uint32_t& issuer)
 {
-    int gok = 0;
-    if (lane == 0)
-        gok = mbar_wait(bar_addr(sb, B_CONV + k % kStages), (k / kStages) & 1, abort_flag, err, kTimeoutNs);
-    if (!__shfl_sync(0xffffffffu, gok, 0)) return 0;
+    const bool gok = mbar_wait(bar_addr(sb, B_CONV + k % kStages), (k / kStages) & 1, abort_flag, err, kTimeoutNs);
+    if (!__all_sync(0xffffffffu, gok)) return 0;
     tc_fence_after();
     if (elect_one(issuer)) issue_gram(sb, tmem, sb + OFF_STG + (k % kStages) * STAGE_BYTES, k & 1);
     __syncwarp();
@@ -892,10 +890,8 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 if (leader && pend_gate >= 0) mbar_arrive(bar_addr(sb, B_GATE_EMPTY + pend_gate));
                 pend_gate = -1;
                 if (warp == 8) {
-                    int lok = 0;
-                    if (leader)
-                        lok = mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs);
-                    if (__shfl_sync(0xffffffffu, lok, 0)) {
+                    const bool lok = mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs);
+                    if (__all_sync(0xffffffffu, lok)) {
                         tc_fence_after();
                         if (elect_one(mma_issuer)) {
                             for (int k = 0; k < 8; ++k) {
@@ -927,9 +923,8 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 grp.sync();
                 // --- MMA_B: ([E; -O'])^T = V^T Z^T + (K^ S)^T X^T ---
                 if (warp == 8) {
-                    int tok = 0;
-                    if (leader) tok = mbar_wait(bar_addr(sb, B_TP_FULL + tps), (c >> 1) & 1, abort_flag, err, kTimeoutNs);
-                    if (__shfl_sync(0xffffffffu, tok, 0)) {
+                    const bool tok = mbar_wait(bar_addr(sb, B_TP_FULL + tps), (c >> 1) & 1, abort_flag, err, kTimeoutNs);
+                    if (__all_sync(0xffffffffu, tok)) {
                         tc_fence_after();
                         if (elect_one(mma_issuer)) {
                             for (int k = 0; k < 2; ++k)

@@ -603,11 +603,10 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (warp == 1) {
                 // Gram products of this chunk, once all of its tiles are in fp16 and the prep
                 // group has read the previous chunk's
-                int gram_ok = 0;
-                if (lane == 0)
-                    gram_ok = mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs) &&
-                              (c == 0 || mbar_wait(bar_addr(sb, B_G_EMPTY), (c - 1) & 1, abort_flag, err, kTimeoutNs));
-                if (__shfl_sync(0xffffffffu, gram_ok, 0)) {
+                const bool gram_ok =
+                    mbar_wait(bar_addr(sb, B_CONV + s), ph, abort_flag, err, kTimeoutNs) &&
+                    (c == 0 || mbar_wait(bar_addr(sb, B_G_EMPTY), (c - 1) & 1, abort_flag, err, kTimeoutNs));
+                if (__all_sync(0xffffffffu, gram_ok)) {
                     tc_fence_after();
                     if (elect_one(gram_issuer)) issue_gram(sb, tmem, s);
                     __syncwarp();
