@@ -320,8 +320,13 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const int64_t whi = r < L - i0 ? r : L - 1 - i0;
         float m = -INFINITY, l = 0.f;                        // running maximum (log2 units), sum
         bool ok = true;
+        // Inside the loop the softmax warps meet at no group barrier: every wait is a warp's own
+        // (all its lanes poll), so no warp waits for the slowest one.  A failed wait raises the
+        // abort flag and takes its warp out of the loop; the other warps' waits then run out or
+        // see the flag, and every thread meets the others once, at the consensus after the loop.
         for (int idx = 0; idx < nblk; ++idx) {
-            if (!grp.wait(bar_addr(sb, B_S_FULL), idx & 1)) {
+            const bool got = mbar_wait(bar_addr(sb, B_S_FULL), idx & 1, abort_flag, err, kTimeoutNs);
+            if (!__all_sync(0xffffffffu, got)) {
                 ok = false;
                 break;
             }
@@ -370,10 +375,8 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             m = mnew;
             // P is double-buffered: P_idx takes the buffer of P_{idx-2}, free once O += P_{idx-2} V
             // is done (barrier idx & 1 completes once every two blocks: phase (idx - 2) / 2)
-            if (idx >= 2 && !grp.wait(bar_addr(sb, B_PV_DONE + (idx & 1)), ((idx - 2) >> 1) & 1)) {
-                ok = false;
-                break;
-            }
+            if (idx >= 2)
+                mbar_wait(bar_addr(sb, B_PV_DONE + (idx & 1)), ((idx - 2) >> 1) & 1, abort_flag, err, kTimeoutNs);
             tc_fence_after();
             if (__any_sync(0xffffffffu, corr != 1.f)) {
                 // a raised maximum rescales O, so the latest O += P V (block idx - 1) must be done;
@@ -393,7 +396,13 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             mbar_arrive(bar_addr(sb, B_P_FULL + (idx & 1)));
         }
         // o = O / l after the last O += P V
-        if (ok && grp.wait(bar_addr(sb, B_PV_DONE + ((nblk - 1) & 1)), ((nblk - 1) >> 1) & 1)) {
+        const bool mine =
+            ok && mbar_wait(bar_addr(sb, B_PV_DONE + ((nblk - 1) & 1)), ((nblk - 1) >> 1) & 1, abort_flag, err, kTimeoutNs);
+        uint32_t all;
+        asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                     "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                     : "=r"(all) : "r"(mine ? 1u : 0u), "r"(NB_SOFT), "r"(kSoftThreads) : "memory");
+        if (all) {
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
             float* o32 = !p.out_bf16 && qi < L ? static_cast<float*>(p.o) + (static_cast<int64_t>(unit) * L + qi) * 128
