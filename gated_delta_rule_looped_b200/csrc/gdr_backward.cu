@@ -29,7 +29,9 @@
 // reduction, and the sweep reuses S_{t-1} of token t+1 as S_t of token t and loads the next
 // S_{t-1} one token ahead; the row sums (dq, dk, dalpha) are warp reductions whose
 // slice partials are added into the fp32 outputs with atomics (zeroed first by this library).
-// dv and dS_0 belong to one block each and are stored directly.
+// dv and dS_0 belong to one block each and are stored directly.  The kernel is instantiated per
+// input type, order and gating, with d_k = 128 fixed at compile time (the rows of a warp then move
+// as float4; any other d_k is read at run time), so no per-element branch stays in the token loops.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -47,9 +49,6 @@ constexpr int kCols = 32;          // columns of d_v per block
 constexpr int kThreads = 256;      // 8 warps
 constexpr int kChunk = 64;         // tokens between checkpoints
 constexpr int kMaxRows = 16;       // dk / 8 rows per warp, dk <= 128
-
-__device__ __forceinline__ float ld(const float* p) { return *p; }
-__device__ __forceinline__ float ld(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
 __device__ __forceinline__ float warp_sum(float x)
 {
@@ -118,11 +117,59 @@ __host__ __device__ inline size_t smem_bytes(int dk, int per_key)
     return (static_cast<size_t>(kChunk) * (2 * dk + na + 1 + 2 * kCols) + 2 * 3 * 8 * kCols) * sizeof(float);
 }
 
-template <typename T>
+// 8 consecutive elements of a row (16-byte aligned) into shared memory as fp32
+__device__ __forceinline__ void ld8(const float* src, float* dst)
+{
+    const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+    reinterpret_cast<float4*>(dst)[0] = a;
+    reinterpret_cast<float4*>(dst)[1] = b;
+}
+__device__ __forceinline__ void ld8(const __nv_bfloat16* src, float* dst)
+{
+    const uint4 r = __ldg(reinterpret_cast<const uint4*>(src));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r);
+    const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
+    const float2 f2 = __bfloat1622float2(h[2]), f3 = __bfloat1622float2(h[3]);
+    reinterpret_cast<float4*>(dst)[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
+    reinterpret_cast<float4*>(dst)[1] = make_float4(f2.x, f2.y, f3.x, f3.y);
+}
+__device__ __forceinline__ void zero8(float* dst)
+{
+    reinterpret_cast<float4*>(dst)[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    reinterpret_cast<float4*>(dst)[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// This thread's rows of one shared-memory row vector: with kRpw a multiple of 4 (d_k = 32, 64,
+// 96, 128) the rows r0 .. r0 + kRpw - 1 are 16-byte aligned and move as float4; otherwise one by one.
+template <int kRpw>
+__device__ __forceinline__ void lds_rows(const float* src, float (&dst)[kMaxRows], int rpw)
+{
+    if constexpr (kRpw > 0 && kRpw % 4 == 0) {
+        #pragma unroll
+        for (int m = 0; m < kRpw; m += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(src + m);
+            dst[m] = x.x;
+            dst[m + 1] = x.y;
+            dst[m + 2] = x.z;
+            dst[m + 3] = x.w;
+        }
+        #pragma unroll
+        for (int m = kRpw; m < kMaxRows; ++m) dst[m] = 0.f;
+    } else {
+        #pragma unroll
+        for (int m = 0; m < kMaxRows; ++m) dst[m] = m < rpw ? src[m] : 0.f;
+    }
+}
+
+// One block = one unit and one 32-column slice of d_v.  kRpw = d_k / 8 when the launch knows it
+// (16: d_k = 128), 0 for any d_k (a multiple of 8, <= 128) read at run time; kDF: decay-first
+// order; kPK: per-key alpha.
+template <typename T, int kRpw, bool kDF, bool kPK>
 __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
 {
     extern __shared__ __align__(16) float smem[];
-    const int dk = p.dk, dv = p.dv, rpw = dk >> 3;
+    const int dk = kRpw > 0 ? 8 * kRpw : p.dk, dv = p.dv, rpw = kRpw > 0 ? kRpw : dk >> 3;
     const int w = threadIdx.x >> 5, c = threadIdx.x & 31;
     const int j0 = blockIdx.y * kCols;
     const int ncol = min(kCols, dv - j0);
@@ -130,7 +177,7 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
     const int j = j0 + c;
     const int64_t u = blockIdx.x, L = p.L;
     const int r0 = w * rpw;
-    const int na = p.per_key ? dk : 1;
+    const int na = kPK ? dk : 1;                  // alpha values per token: d_k (per key) or 1
     float* sk = smem;                              // [64][dk]
     float* sq = sk + kChunk * dk;                  // [64][dk]
     float* sa = sq + kChunk * dk;                  // [64][na]
@@ -147,48 +194,64 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
     const float* be = p.beta + u * L;
     float* ws = p.ws + (u * gridDim.y + blockIdx.y) * ws_floats_per_block(L, dk);
     const int nck = static_cast<int>((L + kChunk - 1) / kChunk);
-    float* ck = ws;                                             // [nck][dk][32]
-    float* st = ws + static_cast<int64_t>(nck) * dk * kCols;   // [65][dk][32]
-    auto at = [&](float* base, int idx, int m) -> float& { return base[(static_cast<int64_t>(idx) * dk + r0 + m) * kCols + c]; };
+    // this thread's element (row r0 + m, column c) of checkpoint / chunk state idx: base[idx * stride + m * 32]
+    const int64_t stride = static_cast<int64_t>(dk) * kCols;
+    float* ck = ws + r0 * kCols + c;                                       // [nck][dk][32]
+    float* st = ws + static_cast<int64_t>(nck) * stride + r0 * kCols + c;  // [65][dk][32]
 
-    // the inputs of tokens t0 .. t0+n-1 into shared memory (q and dO only for the reverse sweep)
+    // the inputs of tokens t0 .. t0+n-1 into shared memory (q and dO only for the reverse sweep);
+    // every tensor is 16-byte aligned and d_k, d_v are multiples of 8, so rows move 8 elements at a time
     auto load_chunk = [&](int64_t t0, int n, bool with_q) {
         __syncthreads();                                        // the previous chunk is consumed
-        for (int i = threadIdx.x; i < n * dk; i += kThreads) {
-            sk[i] = ld(k + t0 * dk + i);
-            if (with_q) sq[i] = ld(q + t0 * dk + i);
+        const int pieces = n * dk / 8;
+        for (int i = threadIdx.x; i < pieces; i += kThreads) {
+            ld8(k + t0 * dk + 8 * i, sk + 8 * i);
+            if (with_q) ld8(q + t0 * dk + 8 * i, sq + 8 * i);
         }
-        for (int i = threadIdx.x; i < n * na; i += kThreads) sa[i] = al[t0 * na + i];
+        if constexpr (kPK) {
+            for (int i = threadIdx.x; i < pieces; i += kThreads) ld8(al + t0 * dk + 8 * i, sa + 8 * i);
+        } else {
+            for (int i = threadIdx.x; i < n; i += kThreads) sa[i] = al[t0 + i];
+        }
         for (int i = threadIdx.x; i < n; i += kThreads) sbe[i] = be[t0 + i];
-        for (int i = threadIdx.x; i < n * kCols; i += kThreads) {
-            const int tt = i / kCols, cc = i - tt * kCols;
-            const bool on = j0 + cc < dv;
-            sv[i] = on ? ld(v + (t0 + tt) * dv + j0 + cc) : 0.f;
-            if (with_q) sdo[i] = on ? ld(dO + (t0 + tt) * dv + j0 + cc) : 0.f;
+        for (int i = threadIdx.x; i < n * (kCols / 8); i += kThreads) {
+            const int tt = i / (kCols / 8), cc = (i % (kCols / 8)) * 8;
+            if (j0 + cc < dv) {                                 // a piece lies wholly inside d_v or outside
+                ld8(v + (t0 + tt) * dv + j0 + cc, sv + tt * kCols + cc);
+                if (with_q) ld8(dO + (t0 + tt) * dv + j0 + cc, sdo + tt * kCols + cc);
+            } else {
+                zero8(sv + tt * kCols + cc);
+                if (with_q) zero8(sdo + tt * kCols + cc);
+            }
         }
         __syncthreads();
     };
-    auto arow = [&](int tau, int m) -> float { return p.per_key ? sa[tau * dk + r0 + m] : sa[tau]; };
 
     // one forward step of the recurrence (token tau of the loaded chunk) on this thread's state
     auto step = [&](float (&s)[kMaxRows], int tau, int buf) {
         const float b = sbe[tau];
+        float kr[kMaxRows], ar[kMaxRows];
+        lds_rows<kRpw>(sk + tau * dk + r0, kr, rpw);
+        if constexpr (kPK) lds_rows<kRpw>(sa + tau * dk + r0, ar, rpw);
+        const float a0 = kPK ? 0.f : sa[tau];
         float pe = 0.f;
         #pragma unroll
         for (int m = 0; m < kMaxRows; ++m)
-            if (m < rpw) pe += sk[tau * dk + r0 + m] * (p.decay_first ? arow(tau, m) * s[m] : s[m]);
+            if (m < rpw) pe += kr[m] * ((kDF && kPK) ? ar[m] * s[m] : s[m]);
+        if (kDF && !kPK) pe *= a0;
         red[buf][0][w][c] = pe;
         __syncthreads();
         float e = 0.f;
         #pragma unroll
         for (int ww = 0; ww < 8; ++ww) e += red[buf][0][ww][c];
         const float vj = sv[tau * kCols + c];
+        const float bd = b * (vj - e), bv = b * vj, be_ = b * e;
         #pragma unroll
         for (int m = 0; m < kMaxRows; ++m) {
             if (m >= rpw) break;
-            const float kr = sk[tau * dk + r0 + m], ar = arow(tau, m);
-            if (p.decay_first) s[m] = ar * s[m] + b * kr * (vj - e);
-            else s[m] = ar * (s[m] - b * kr * e) + b * kr * vj;
+            const float ar_ = kPK ? ar[m] : a0;
+            if (kDF) s[m] = ar_ * s[m] + kr[m] * bd;
+            else s[m] = ar_ * (s[m] - kr[m] * be_) + kr[m] * bv;
         }
     };
 
@@ -200,9 +263,10 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
     for (int ci = 0; ci < nck; ++ci) {
         const int64_t t0 = static_cast<int64_t>(ci) * kChunk;
         const int n = static_cast<int>(L - t0 < kChunk ? L - t0 : kChunk);
+        float* cp = ck + ci * stride;
         #pragma unroll
         for (int m = 0; m < kMaxRows; ++m)
-            if (m < rpw) at(ck, ci, m) = s[m];
+            if (m < rpw) cp[m * kCols] = s[m];
         load_chunk(t0, n, false);
         for (int tau = 0; tau < n; ++tau) step(s, tau, tau & 1);
     }
@@ -216,39 +280,57 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
         const int64_t t0 = static_cast<int64_t>(ci) * kChunk;
         const int n = static_cast<int>(L - t0 < kChunk ? L - t0 : kChunk);
         load_chunk(t0, n, true);
-        #pragma unroll
-        for (int m = 0; m < kMaxRows; ++m) {
-            s[m] = m < rpw ? at(ck, ci, m) : 0.f;
-            if (m < rpw) at(st, 0, m) = s[m];
+        {
+            const float* cp = ck + ci * stride;
+            #pragma unroll
+            for (int m = 0; m < kMaxRows; ++m) {
+                s[m] = m < rpw ? cp[m * kCols] : 0.f;
+                if (m < rpw) st[m * kCols] = s[m];
+            }
         }
         for (int tau = 0; tau < n; ++tau) {
             step(s, tau, tau & 1);
             if (tau + 1 < n) {                                  // S_t of the last token stays in s
+                float* sp_ = st + (tau + 1) * stride;
                 #pragma unroll
                 for (int m = 0; m < kMaxRows; ++m)
-                    if (m < rpw) at(st, tau + 1, m) = s[m];
+                    if (m < rpw) sp_[m * kCols] = s[m];
             }
         }
         __syncthreads();
         // S_t arrives from the previous step (S_{t-1} of token t+1); S_{t-1} is loaded one token ahead
         float sc[kMaxRows], sp[kMaxRows];
-        #pragma unroll
-        for (int m = 0; m < kMaxRows; ++m) {
-            sc[m] = s[m];
-            sp[m] = m < rpw ? at(st, n - 1, m) : 0.f;
+        {
+            const float* sp_ = st + (n - 1) * stride;
+            #pragma unroll
+            for (int m = 0; m < kMaxRows; ++m) {
+                sc[m] = s[m];
+                sp[m] = m < rpw ? sp_[m * kCols] : 0.f;
+            }
         }
         for (int tau = n - 1; tau >= 0; --tau) {
             const int buf = tau & 1;
             const int64_t t = t0 + tau;
             float spn[kMaxRows];                               // S_{t-2}, for the next token
-            #pragma unroll
-            for (int m = 0; m < kMaxRows; ++m) spn[m] = (m < rpw && tau > 0) ? at(st, tau - 1, m) : 0.f;
+            {
+                const float* sp_ = st + (tau > 0 ? tau - 1 : 0) * stride;
+                #pragma unroll
+                for (int m = 0; m < kMaxRows; ++m) spn[m] = (m < rpw && tau > 0) ? sp_[m * kCols] : 0.f;
+            }
             const float b = sbe[tau];
             const float vj = sv[tau * kCols + c];
             const float oj = sdo[tau * kCols + c];
-            #pragma unroll
-            for (int m = 0; m < kMaxRows; ++m)
-                if (m < rpw) G[m] += sq[tau * dk + r0 + m] * oj;   // from o_t = S_t^T q_t
+            float kr[kMaxRows], ar[kMaxRows];
+            lds_rows<kRpw>(sk + tau * dk + r0, kr, rpw);
+            if constexpr (kPK) lds_rows<kRpw>(sa + tau * dk + r0, ar, rpw);
+            const float a0 = kPK ? 0.f : sa[tau];
+            {
+                float qr[kMaxRows];
+                lds_rows<kRpw>(sq + tau * dk + r0, qr, rpw);
+                #pragma unroll
+                for (int m = 0; m < kMaxRows; ++m)
+                    if (m < rpw) G[m] += qr[m] * oj;           // from o_t = S_t^T q_t
+            }
             // dq_t = S_t dO_t: row sums over this slice's columns
             {
                 float x[kMaxRows];
@@ -259,59 +341,64 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
                 if (!(c & 1) && m < rpw) atomicAdd(p.dq + (u * L + t) * dk + r0 + m, tot);
             }
             // the column sums of this step, one reduction: e, k^T G, k^T Diag(alpha) G
+            // (with a scalar alpha the third is alpha k^T G, and e of the decay-first order alpha k^T S)
             float pe = 0.f, pg = 0.f, pd = 0.f;
             #pragma unroll
             for (int m = 0; m < kMaxRows; ++m) {
                 if (m >= rpw) break;
-                const float kr = sk[tau * dk + r0 + m], ar = arow(tau, m);
-                pe += kr * (p.decay_first ? ar * sp[m] : sp[m]);
-                pg += kr * G[m];
-                pd += kr * ar * G[m];
+                pe += kr[m] * ((kDF && kPK) ? ar[m] * sp[m] : sp[m]);
+                pg += kr[m] * G[m];
+                if (kPK) pd += kr[m] * ar[m] * G[m];
             }
+            if (kDF && !kPK) pe *= a0;
             red[buf][0][w][c] = pe;
             red[buf][1][w][c] = pg;
-            red[buf][2][w][c] = pd;
+            if (kPK) red[buf][2][w][c] = pd;
             __syncthreads();
             float e = 0.f, kG = 0.f, kdP = 0.f;
             #pragma unroll
             for (int ww = 0; ww < 8; ++ww) {
                 e += red[buf][0][ww][c];
                 kG += red[buf][1][ww][c];
-                kdP += red[buf][2][ww][c];
+                if (kPK) kdP += red[buf][2][ww][c];
             }
+            if (!kPK) kdP = a0 * kG;
             if (active) p.gdv[(u * L + t) * dv + j] = b * kG;
             // dbeta: column terms summed over the slice
-            const float tb = active ? (p.decay_first ? kG * (vj - e) : kG * vj - kdP * e) : 0.f;
+            const float tb = active ? (kDF ? kG * (vj - e) : kG * vj - kdP * e) : 0.f;
             if (w == 0) {
                 const float x = warp_sum(tb);
                 if (c == 0) atomicAdd(p.dbeta + u * L + t, x);
             }
             float dkx[kMaxRows], dax[kMaxRows];
-            #pragma unroll
-            for (int m = 0; m < kMaxRows; ++m) {
-                dkx[m] = dax[m] = 0.f;
-                if (m >= rpw) continue;
-                const float kr = sk[tau * dk + r0 + m], ar = arow(tau, m);
-                if (p.decay_first) {
-                    const float R = ar * sp[m];
-                    const float dR = G[m] - b * kr * kG;
-                    dkx[m] = b * G[m] * (vj - e) - b * R * kG;
-                    dax[m] = dR * sp[m];
-                    G[m] = ar * dR;
-                } else {
-                    const float P = sp[m] - b * kr * e;
-                    const float dP = ar * G[m];
-                    dkx[m] = b * G[m] * vj - b * (sp[m] * kdP + dP * e);
-                    dax[m] = G[m] * P;
-                    G[m] = dP - b * kr * kdP;
+            {
+                const float bkG = b * kG, bkdP = b * kdP, bd = b * (vj - e), bv = b * vj, bE = b * e;
+                #pragma unroll
+                for (int m = 0; m < kMaxRows; ++m) {
+                    dkx[m] = dax[m] = 0.f;
+                    if (m >= rpw) continue;
+                    const float ar_ = kPK ? ar[m] : a0;
+                    if (kDF) {
+                        const float R = ar_ * sp[m];
+                        const float dR = G[m] - kr[m] * bkG;
+                        dkx[m] = G[m] * bd - R * bkG;
+                        dax[m] = dR * sp[m];
+                        G[m] = ar_ * dR;
+                    } else {
+                        const float P = sp[m] - kr[m] * bE;
+                        const float dP = ar_ * G[m];
+                        dkx[m] = G[m] * bv - (sp[m] * bkdP + dP * bE);
+                        dax[m] = G[m] * P;
+                        G[m] = dP - kr[m] * bkdP;
+                    }
+                    if (!active) dkx[m] = dax[m] = 0.f;
                 }
-                if (!active) dkx[m] = dax[m] = 0.f;
             }
             {
                 const int m = row16(c);
                 const float dks = rows_sum16(dkx, c);
                 if (!(c & 1) && m < rpw) atomicAdd(p.gdk + (u * L + t) * dk + r0 + m, dks);
-                if (p.per_key) {
+                if constexpr (kPK) {
                     const float das = rows_sum16(dax, c);
                     if (!(c & 1) && m < rpw) atomicAdd(p.dalpha + (u * L + t) * dk + r0 + m, das);
                 } else {
@@ -429,7 +516,18 @@ cudaError_t launch_backward(const BwCall& c, cudaStream_t stream)
     p.decay_first = c.decay_first;
     const dim3 grid(static_cast<unsigned>(c.units), static_cast<unsigned>((c.dv + kCols - 1) / kCols), 1);
     const size_t smem = smem_bytes(c.dk, c.per_key);
-    auto kernel = c.dtype_bf16 ? gdr_backward_kernel<__nv_bfloat16> : gdr_backward_kernel<float>;
+    // [bf16][d_k == 128][decay-first][per-key]
+    using Kernel = void (*)(Params);
+    static const Kernel kernels[2][2][2][2] = {
+        {{{gdr_backward_kernel<float, 0, false, false>, gdr_backward_kernel<float, 0, false, true>},
+          {gdr_backward_kernel<float, 0, true, false>, gdr_backward_kernel<float, 0, true, true>}},
+         {{gdr_backward_kernel<float, 16, false, false>, gdr_backward_kernel<float, 16, false, true>},
+          {gdr_backward_kernel<float, 16, true, false>, gdr_backward_kernel<float, 16, true, true>}}},
+        {{{gdr_backward_kernel<__nv_bfloat16, 0, false, false>, gdr_backward_kernel<__nv_bfloat16, 0, false, true>},
+          {gdr_backward_kernel<__nv_bfloat16, 0, true, false>, gdr_backward_kernel<__nv_bfloat16, 0, true, true>}},
+         {{gdr_backward_kernel<__nv_bfloat16, 16, false, false>, gdr_backward_kernel<__nv_bfloat16, 16, false, true>},
+          {gdr_backward_kernel<__nv_bfloat16, 16, true, false>, gdr_backward_kernel<__nv_bfloat16, 16, true, true>}}}};
+    const Kernel kernel = kernels[c.dtype_bf16 ? 1 : 0][c.dk == 128 ? 1 : 0][c.decay_first ? 1 : 0][c.per_key ? 1 : 0];
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kernel<<<grid, kThreads, smem, stream>>>(p);
