@@ -17,21 +17,25 @@
 // and dS_0 = G at the end (scalar alpha: dalpha sums over the rows too).
 //
 // The columns of S evolve independently given the token's k, alpha, beta (e_j only reads column
-// j), so a block takes one unit and a slice of 32 columns of d_v, like the token-sequential
-// prefill: warp w holds rows w*dk/8 .. of the slice, lane c column j0 + c.  The reverse sweep
-// needs S_{t-1} and S_t at every t, newest first:
+// j), so a block takes one unit and a slice of 32 columns of d_v, and each warp four whole columns
+// of it: lane 4 g + c holds rows g*dk/8 .. (g+1)*dk/8 - 1 of column j0 + 4 w + c.  Every column sum
+// a step needs (k^T S_{t-1} or k^T R, k^T G, k^T Diag(alpha) G) is then a sum over the 8 row groups
+// of one warp -- three shuffles, no block barrier -- and the warps run their columns' recurrences
+// independently.  The reverse sweep needs S_{t-1} and S_t at every t, newest first:
 //   phase A  runs the forward over the whole sequence and keeps the state at the start of every
-//            64-token chunk (a checkpoint) in the workspace;
+//            32-token chunk (a checkpoint) in the workspace;
 //   phase B  takes the chunks from the last: it recomputes the chunk's states from its checkpoint
 //            into the workspace, then sweeps the chunk backwards.
-// A chunk's inputs are staged in shared memory once per phase.  Per token the three column sums
-// the step needs (k^T S_{t-1} or k^T R, k^T G, k^T Diag(alpha) G) come from one shared-memory
-// reduction, and the sweep reuses S_{t-1} of token t+1 as S_t of token t and loads the next
-// S_{t-1} one token ahead; the row sums (dq, dk, dalpha) are warp reductions whose
-// slice partials are added into the fp32 outputs with atomics (zeroed first by this library).
-// dv and dS_0 belong to one block each and are stored directly.  The kernel is instantiated per
-// input type, order and gating, with d_k = 128 fixed at compile time (the rows of a warp then move
-// as float4; any other d_k is read at run time), so no per-element branch stays in the token loops.
+// The workspace is thread-major (element m of thread i of a state at [m][i]): each thread reads
+// back only what it wrote, in coalesced rows.  A chunk's inputs are staged in shared memory once
+// per phase; the sweep reuses S_{t-1} of token t+1 as S_t of token t and loads the next S_{t-1}
+// one token ahead.  The row sums (dq, dk and the per-key dalpha: sums over the slice's 32
+// columns) are summed over a warp's 4 columns with shuffles, parked per warp in shared memory, and
+// every few tokens added over the 8 warps and into the fp32 outputs with atomics (zeroed first by
+// this library), as are the dbeta and scalar dalpha terms.  dv and dS_0 belong to one block each
+// and are stored directly.  The kernel is instantiated per input type, order and gating, with
+// d_k = 128 fixed at compile time (the rows of a thread then move as float4; any other d_k is read
+// at run time), so no per-element branch stays in the token loops.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -46,9 +50,15 @@ namespace lt2 {
 namespace bw {
 
 constexpr int kCols = 32;          // columns of d_v per block
-constexpr int kThreads = 256;      // 8 warps
-constexpr int kChunk = 64;         // tokens between checkpoints
-constexpr int kMaxRows = 16;       // dk / 8 rows per warp, dk <= 128
+constexpr int kThreads = 256;      // 8 warps, 4 columns each
+constexpr int kChunk = 32;         // tokens between checkpoints, staged in shared memory at once
+constexpr int kMaxRows = 16;       // dk / 8 rows per thread, dk <= 128
+
+// Tokens whose row-sum partials wait in shared memory before they are added up and written
+// (fewer with a per-key alpha, which adds a third row sum).
+__host__ __device__ constexpr int flush_tokens(bool per_key) { return per_key ? 4 : 8; }
+// Floats per warp row of the row-sum partials: d_k plus one pad per 32 rows (no bank conflicts)
+__host__ __device__ constexpr int part_stride(int dk) { return dk + 4; }
 
 __device__ __forceinline__ float warp_sum(float x)
 {
@@ -57,14 +67,23 @@ __device__ __forceinline__ float warp_sum(float x)
     return x;
 }
 
-// Sums over the 32 lanes of a warp of 16 values per lane at once (recursive halving: 16 shuffles
-// instead of 16 x 5).  On return lane l holds the total of row row16(l); lanes l and l ^ 1 hold
-// the same row.
-__device__ __forceinline__ float rows_sum16(float (&v)[16], int lane)
+// A column sum over all d_k rows: the 8 row groups of a column are lanes c, c + 4, ..., c + 28.
+__device__ __forceinline__ float sum_row_groups(float x)
+{
+    x += __shfl_xor_sync(0xffffffffu, x, 4);
+    x += __shfl_xor_sync(0xffffffffu, x, 8);
+    x += __shfl_xor_sync(0xffffffffu, x, 16);
+    return x;
+}
+
+// Row sums over a warp's 4 columns (lanes 4 g .. 4 g + 3) of 16 values per lane at once, by
+// recursive halving (12 shuffles instead of 16 x 2).  On return v[i], i < 4, holds the sum of row
+// (c & 1) * 8 + (c & 2) * 2 + i of the thread's rows, c = lane & 3.
+__device__ __forceinline__ void sum_cols4(float (&v)[kMaxRows], int c)
 {
     #pragma unroll
-    for (int half = 8, off = 16; half >= 1; half >>= 1, off >>= 1) {
-        const bool upper = (lane & off) != 0;
+    for (int half = 8, off = 1; half >= 4; half >>= 1, off <<= 1) {
+        const bool upper = (c & off) != 0;
         #pragma unroll
         for (int i = 0; i < half; ++i) {
             const float send = upper ? v[i] : v[i + half];
@@ -72,11 +91,6 @@ __device__ __forceinline__ float rows_sum16(float (&v)[16], int lane)
             v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
         }
     }
-    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
-}
-__device__ __forceinline__ int row16(int lane)
-{
-    return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
 }
 
 struct Params {
@@ -103,18 +117,21 @@ struct Params {
     int decay_first;
 };
 
-// Workspace floats per block: ceil(L / 64) checkpoints and the 65 states of one chunk, dk x 32 each.
+// Workspace floats per block: ceil(L / 32) checkpoints and the 33 states of one chunk, dk x 32 each.
 __host__ __device__ inline int64_t ws_floats_per_block(int64_t L, int dk)
 {
     return ((L + kChunk - 1) / kChunk + kChunk + 1) * static_cast<int64_t>(dk) * kCols;
 }
 
 // Shared memory of a block: one chunk's inputs in fp32 (k, q, alpha rows, beta, and the slice's v
-// and dO columns) and the reduction buffers.
+// and dO columns), the row-sum partials [dq, dk(, dalpha)][token][warp][row] and the per-warp
+// dbeta and scalar dalpha terms [token][warp].
 __host__ __device__ inline size_t smem_bytes(int dk, int per_key)
 {
     const size_t na = per_key ? dk : 1;
-    return (static_cast<size_t>(kChunk) * (2 * dk + na + 1 + 2 * kCols) + 2 * 3 * 8 * kCols) * sizeof(float);
+    const size_t f = flush_tokens(per_key != 0), ng = per_key ? 3 : 2;
+    return (static_cast<size_t>(kChunk) * (2 * dk + na + 1 + 2 * kCols) + ng * f * 8 * part_stride(dk) + 2 * f * 8) *
+           sizeof(float);
 }
 
 // 8 consecutive elements of a row (16-byte aligned) into shared memory as fp32
@@ -166,25 +183,29 @@ __device__ __forceinline__ void lds_rows(const float* src, float (&dst)[kMaxRows
 // (16: d_k = 128), 0 for any d_k (a multiple of 8, <= 128) read at run time; kDF: decay-first
 // order; kPK: per-key alpha.
 template <typename T, int kRpw, bool kDF, bool kPK>
-__global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
+__global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
 {
+    constexpr int kF = flush_tokens(kPK);
+    constexpr int kNg = kPK ? 3 : 2;               // row sums: dq, dk (and the per-key dalpha)
     extern __shared__ __align__(16) float smem[];
     const int dk = kRpw > 0 ? 8 * kRpw : p.dk, dv = p.dv, rpw = kRpw > 0 ? kRpw : dk >> 3;
-    const int w = threadIdx.x >> 5, c = threadIdx.x & 31;
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, g = lane >> 2, cg = lane & 3;
     const int j0 = blockIdx.y * kCols;
-    const int ncol = min(kCols, dv - j0);
-    const bool active = c < ncol;
-    const int j = j0 + c;
+    const int jl = 4 * w + cg, j = j0 + jl;        // this thread's column (in the slice, in d_v)
+    const bool active = j < dv;
     const int64_t u = blockIdx.x, L = p.L;
-    const int r0 = w * rpw;
-    const int na = kPK ? dk : 1;                  // alpha values per token: d_k (per key) or 1
-    float* sk = smem;                              // [64][dk]
-    float* sq = sk + kChunk * dk;                  // [64][dk]
-    float* sa = sq + kChunk * dk;                  // [64][na]
-    float* sbe = sa + kChunk * na;                 // [64]
-    float* sv = sbe + kChunk;                      // [64][32]
-    float* sdo = sv + kChunk * kCols;              // [64][32]
-    float (*red)[3][8][kCols] = reinterpret_cast<float (*)[3][8][kCols]>(sdo + kChunk * kCols);
+    const int r0 = g * rpw;                        // first of this thread's rows
+    const int na = kPK ? dk : 1;
+    const int ps = part_stride(dk);
+    float* sk = smem;                              // [32][dk]
+    float* sq = sk + kChunk * dk;                  // [32][dk]
+    float* sa = sq + kChunk * dk;                  // [32][na]
+    float* sbe = sa + kChunk * na;                 // [32]
+    float* sv = sbe + kChunk;                      // [32][32]
+    float* sdo = sv + kChunk * kCols;              // [32][32]
+    float* part = sdo + kChunk * kCols;            // [kNg][kF][8][ps]
+    float* pbe = part + kNg * kF * 8 * ps;         // [kF][8]
+    float* pal = pbe + kF * 8;                     // [kF][8] (scalar alpha)
 
     const T* q = static_cast<const T*>(p.q) + u * L * dk;
     const T* k = static_cast<const T*>(p.k) + u * L * dk;
@@ -192,29 +213,28 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
     const T* dO = static_cast<const T*>(p.dO) + u * L * dv;
     const float* al = p.alpha + u * L * na;
     const float* be = p.beta + u * L;
-    float* ws = p.ws + (u * gridDim.y + blockIdx.y) * ws_floats_per_block(L, dk);
     const int nck = static_cast<int>((L + kChunk - 1) / kChunk);
-    // this thread's element (row r0 + m, column c) of checkpoint / chunk state idx: base[idx * stride + m * 32]
-    const int64_t stride = static_cast<int64_t>(dk) * kCols;
-    float* ck = ws + r0 * kCols + c;                                       // [nck][dk][32]
-    float* st = ws + static_cast<int64_t>(nck) * stride + r0 * kCols + c;  // [65][dk][32]
+    // element m of this thread in checkpoint idx: ck[idx * sst + m * 256] (likewise st)
+    const int64_t sst = static_cast<int64_t>(rpw) * kThreads;
+    float* ck = p.ws + (u * gridDim.y + blockIdx.y) * ws_floats_per_block(L, dk) + tid;
+    float* st = ck + nck * sst;                    // [33] states of the chunk being swept
 
     // the inputs of tokens t0 .. t0+n-1 into shared memory (q and dO only for the reverse sweep);
     // every tensor is 16-byte aligned and d_k, d_v are multiples of 8, so rows move 8 elements at a time
     auto load_chunk = [&](int64_t t0, int n, bool with_q) {
         __syncthreads();                                        // the previous chunk is consumed
         const int pieces = n * dk / 8;
-        for (int i = threadIdx.x; i < pieces; i += kThreads) {
+        for (int i = tid; i < pieces; i += kThreads) {
             ld8(k + t0 * dk + 8 * i, sk + 8 * i);
             if (with_q) ld8(q + t0 * dk + 8 * i, sq + 8 * i);
         }
         if constexpr (kPK) {
-            for (int i = threadIdx.x; i < pieces; i += kThreads) ld8(al + t0 * dk + 8 * i, sa + 8 * i);
+            for (int i = tid; i < pieces; i += kThreads) ld8(al + t0 * dk + 8 * i, sa + 8 * i);
         } else {
-            for (int i = threadIdx.x; i < n; i += kThreads) sa[i] = al[t0 + i];
+            for (int i = tid; i < n; i += kThreads) sa[i] = al[t0 + i];
         }
-        for (int i = threadIdx.x; i < n; i += kThreads) sbe[i] = be[t0 + i];
-        for (int i = threadIdx.x; i < n * (kCols / 8); i += kThreads) {
+        for (int i = tid; i < n; i += kThreads) sbe[i] = be[t0 + i];
+        for (int i = tid; i < n * (kCols / 8); i += kThreads) {
             const int tt = i / (kCols / 8), cc = (i % (kCols / 8)) * 8;
             if (j0 + cc < dv) {                                 // a piece lies wholly inside d_v or outside
                 ld8(v + (t0 + tt) * dv + j0 + cc, sv + tt * kCols + cc);
@@ -228,7 +248,7 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
     };
 
     // one forward step of the recurrence (token tau of the loaded chunk) on this thread's state
-    auto step = [&](float (&s)[kMaxRows], int tau, int buf) {
+    auto step = [&](float (&s)[kMaxRows], int tau) {
         const float b = sbe[tau];
         float kr[kMaxRows], ar[kMaxRows];
         lds_rows<kRpw>(sk + tau * dk + r0, kr, rpw);
@@ -239,12 +259,8 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
         for (int m = 0; m < kMaxRows; ++m)
             if (m < rpw) pe += kr[m] * ((kDF && kPK) ? ar[m] * s[m] : s[m]);
         if (kDF && !kPK) pe *= a0;
-        red[buf][0][w][c] = pe;
-        __syncthreads();
-        float e = 0.f;
-        #pragma unroll
-        for (int ww = 0; ww < 8; ++ww) e += red[buf][0][ww][c];
-        const float vj = sv[tau * kCols + c];
+        const float e = sum_row_groups(pe);
+        const float vj = sv[tau * kCols + jl];
         const float bd = b * (vj - e), bv = b * vj, be_ = b * e;
         #pragma unroll
         for (int m = 0; m < kMaxRows; ++m) {
@@ -255,6 +271,46 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
         }
     };
 
+    // a warp's row sums over its 4 columns (16 per thread) into the partials of gradient gi, token slot sl
+    auto park_rows = [&](float (&x)[kMaxRows], int gi, int sl) {
+        sum_cols4(x, cg);
+        float* dst = part + ((gi * kF + sl) * 8 + w) * ps;
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int m = (cg & 1) * 8 + (cg & 2) * 2 + i;
+            const int r = r0 + m;
+            if (m < rpw) dst[r + (r >> 5)] = x[i];
+        }
+    };
+
+    // tokens tg0 .. tg0 + cnt - 1 (slots 0 .. cnt - 1): partials summed over the 8 warps, added to the outputs
+    auto flush = [&](int64_t tg0, int cnt) {
+        __syncthreads();                                        // every warp has parked its partials
+        const int half = tid >> 7, r = tid & 127;
+        if (r < dk) {
+            for (int gs = half; gs < kNg * cnt; gs += 2) {
+                const int gi = gs / cnt, sl = gs - gi * cnt;
+                const float* src = part + ((gi * kF + sl) * 8) * ps + r + (r >> 5);
+                float x = 0.f;
+                #pragma unroll
+                for (int ww = 0; ww < 8; ++ww) x += src[ww * ps];
+                float* out = gi == 0 ? p.dq : (gi == 1 ? p.gdk : p.dalpha);
+                atomicAdd(out + (u * L + tg0 + sl) * dk + r, x);
+            }
+        }
+        if (tid < cnt) {
+            float xb = 0.f, xa = 0.f;
+            #pragma unroll
+            for (int ww = 0; ww < 8; ++ww) {
+                xb += pbe[tid * 8 + ww];
+                if (!kPK) xa += pal[tid * 8 + ww];
+            }
+            atomicAdd(p.dbeta + u * L + tg0 + tid, xb);
+            if (!kPK) atomicAdd(p.dalpha + u * L + tg0 + tid, xa);
+        }
+        __syncthreads();                                        // the partials are free again
+    };
+
     // ---- phase A: forward, checkpoints at the chunk starts ----
     float s[kMaxRows];
     const float* S0 = p.S0 ? p.S0 + u * static_cast<int64_t>(dk) * dv : nullptr;
@@ -263,12 +319,12 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
     for (int ci = 0; ci < nck; ++ci) {
         const int64_t t0 = static_cast<int64_t>(ci) * kChunk;
         const int n = static_cast<int>(L - t0 < kChunk ? L - t0 : kChunk);
-        float* cp = ck + ci * stride;
+        float* cp = ck + ci * sst;
         #pragma unroll
         for (int m = 0; m < kMaxRows; ++m)
-            if (m < rpw) cp[m * kCols] = s[m];
+            if (m < rpw) cp[m * kThreads] = s[m];
         load_chunk(t0, n, false);
-        for (int tau = 0; tau < n; ++tau) step(s, tau, tau & 1);
+        for (int tau = 0; tau < n; ++tau) step(s, tau);
     }
 
     // ---- phase B: chunks from the last, each recomputed, then swept backwards ----
@@ -281,45 +337,43 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
         const int n = static_cast<int>(L - t0 < kChunk ? L - t0 : kChunk);
         load_chunk(t0, n, true);
         {
-            const float* cp = ck + ci * stride;
+            const float* cp = ck + ci * sst;
             #pragma unroll
             for (int m = 0; m < kMaxRows; ++m) {
-                s[m] = m < rpw ? cp[m * kCols] : 0.f;
-                if (m < rpw) st[m * kCols] = s[m];
+                s[m] = m < rpw ? cp[m * kThreads] : 0.f;
+                if (m < rpw) st[m * kThreads] = s[m];
             }
         }
         for (int tau = 0; tau < n; ++tau) {
-            step(s, tau, tau & 1);
+            step(s, tau);
             if (tau + 1 < n) {                                  // S_t of the last token stays in s
-                float* sp_ = st + (tau + 1) * stride;
+                float* sp_ = st + (tau + 1) * sst;
                 #pragma unroll
                 for (int m = 0; m < kMaxRows; ++m)
-                    if (m < rpw) sp_[m * kCols] = s[m];
+                    if (m < rpw) sp_[m * kThreads] = s[m];
             }
         }
-        __syncthreads();
         // S_t arrives from the previous step (S_{t-1} of token t+1); S_{t-1} is loaded one token ahead
         float sc[kMaxRows], sp[kMaxRows];
         {
-            const float* sp_ = st + (n - 1) * stride;
+            const float* sp_ = st + (n - 1) * sst;
             #pragma unroll
             for (int m = 0; m < kMaxRows; ++m) {
                 sc[m] = s[m];
-                sp[m] = m < rpw ? sp_[m * kCols] : 0.f;
+                sp[m] = m < rpw ? sp_[m * kThreads] : 0.f;
             }
         }
         for (int tau = n - 1; tau >= 0; --tau) {
-            const int buf = tau & 1;
-            const int64_t t = t0 + tau;
+            const int sl = tau % kF;                            // this token's slot among the parked partials
             float spn[kMaxRows];                               // S_{t-2}, for the next token
             {
-                const float* sp_ = st + (tau > 0 ? tau - 1 : 0) * stride;
+                const float* sp_ = st + (tau > 0 ? tau - 1 : 0) * sst;
                 #pragma unroll
-                for (int m = 0; m < kMaxRows; ++m) spn[m] = (m < rpw && tau > 0) ? sp_[m * kCols] : 0.f;
+                for (int m = 0; m < kMaxRows; ++m) spn[m] = (m < rpw && tau > 0) ? sp_[m * kThreads] : 0.f;
             }
             const float b = sbe[tau];
-            const float vj = sv[tau * kCols + c];
-            const float oj = sdo[tau * kCols + c];
+            const float vj = sv[tau * kCols + jl];
+            const float oj = sdo[tau * kCols + jl];
             float kr[kMaxRows], ar[kMaxRows];
             lds_rows<kRpw>(sk + tau * dk + r0, kr, rpw);
             if constexpr (kPK) lds_rows<kRpw>(sa + tau * dk + r0, ar, rpw);
@@ -331,16 +385,14 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
                 for (int m = 0; m < kMaxRows; ++m)
                     if (m < rpw) G[m] += qr[m] * oj;           // from o_t = S_t^T q_t
             }
-            // dq_t = S_t dO_t: row sums over this slice's columns
+            // dq_t = S_t dO_t: row sums over the slice's columns
             {
                 float x[kMaxRows];
                 #pragma unroll
                 for (int m = 0; m < kMaxRows; ++m) x[m] = m < rpw ? sc[m] * oj : 0.f;
-                const float tot = rows_sum16(x, c);
-                const int m = row16(c);
-                if (!(c & 1) && m < rpw) atomicAdd(p.dq + (u * L + t) * dk + r0 + m, tot);
+                park_rows(x, 0, sl);
             }
-            // the column sums of this step, one reduction: e, k^T G, k^T Diag(alpha) G
+            // the column sums of this step: e, k^T G, k^T Diag(alpha) G
             // (with a scalar alpha the third is alpha k^T G, and e of the decay-first order alpha k^T S)
             float pe = 0.f, pg = 0.f, pd = 0.f;
             #pragma unroll
@@ -351,25 +403,18 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
                 if (kPK) pd += kr[m] * ar[m] * G[m];
             }
             if (kDF && !kPK) pe *= a0;
-            red[buf][0][w][c] = pe;
-            red[buf][1][w][c] = pg;
-            if (kPK) red[buf][2][w][c] = pd;
-            __syncthreads();
-            float e = 0.f, kG = 0.f, kdP = 0.f;
-            #pragma unroll
-            for (int ww = 0; ww < 8; ++ww) {
-                e += red[buf][0][ww][c];
-                kG += red[buf][1][ww][c];
-                if (kPK) kdP += red[buf][2][ww][c];
+            const float e = sum_row_groups(pe);
+            const float kG = sum_row_groups(pg);
+            const float kdP = kPK ? sum_row_groups(pd) : a0 * kG;
+            if (active && g == 0) p.gdv[(u * L + t0 + tau) * dv + j] = b * kG;
+            // dbeta: column terms summed over the warp's columns, parked per warp
+            {
+                float tb = active ? (kDF ? kG * (vj - e) : kG * vj - kdP * e) : 0.f;
+                tb += __shfl_xor_sync(0xffffffffu, tb, 1);
+                tb += __shfl_xor_sync(0xffffffffu, tb, 2);
+                if (lane == 0) pbe[sl * 8 + w] = tb;
             }
-            if (!kPK) kdP = a0 * kG;
-            if (active) p.gdv[(u * L + t) * dv + j] = b * kG;
-            // dbeta: column terms summed over the slice
-            const float tb = active ? (kDF ? kG * (vj - e) : kG * vj - kdP * e) : 0.f;
-            if (w == 0) {
-                const float x = warp_sum(tb);
-                if (c == 0) atomicAdd(p.dbeta + u * L + t, x);
-            }
+            // (a column past d_v has S = 0, G = 0 and v = dO = 0 throughout, so its terms are 0)
             float dkx[kMaxRows], dax[kMaxRows];
             {
                 const float bkG = b * kG, bkdP = b * kdP, bd = b * (vj - e), bv = b * vj, bE = b * e;
@@ -391,24 +436,19 @@ __global__ void __launch_bounds__(kThreads) gdr_backward_kernel(Params p)
                         dax[m] = G[m] * P;
                         G[m] = dP - kr[m] * bkdP;
                     }
-                    if (!active) dkx[m] = dax[m] = 0.f;
                 }
             }
-            {
-                const int m = row16(c);
-                const float dks = rows_sum16(dkx, c);
-                if (!(c & 1) && m < rpw) atomicAdd(p.gdk + (u * L + t) * dk + r0 + m, dks);
-                if constexpr (kPK) {
-                    const float das = rows_sum16(dax, c);
-                    if (!(c & 1) && m < rpw) atomicAdd(p.dalpha + (u * L + t) * dk + r0 + m, das);
-                } else {
-                    float dal_sum = 0.f;
-                    #pragma unroll
-                    for (int mm = 0; mm < kMaxRows; ++mm) dal_sum += dax[mm];
-                    const float x = warp_sum(dal_sum);
-                    if (c == 0) atomicAdd(p.dalpha + u * L + t, x);
-                }
+            park_rows(dkx, 1, sl);
+            if constexpr (kPK) {
+                park_rows(dax, 2, sl);
+            } else {
+                float dal_sum = 0.f;
+                #pragma unroll
+                for (int mm = 0; mm < kMaxRows; ++mm) dal_sum += dax[mm];
+                const float x = warp_sum(dal_sum);
+                if (lane == 0) pal[sl * 8 + w] = x;
             }
+            if (sl == 0) flush(t0 + tau, min(kF, n - tau));
             #pragma unroll
             for (int m = 0; m < kMaxRows; ++m) {
                 sc[m] = sp[m];

@@ -224,7 +224,7 @@ lt2_status lt2_gdr_prefill_varlen(const lt2_gdr_dims* dims, const lt2_gdr_fused*
 
 /*
  * Bytes of device workspace lt2_gdr_backward needs for `dims` (0 for invalid dims): per
- * (unit, 32-column slice of d_v), a checkpoint of the state every 64 tokens and the 65 states of
+ * (unit, 32-column slice of d_v), a checkpoint of the state every 32 tokens and the 33 states of
  * one chunk, fp32.  Pure host function, no CUDA call.
  */
 size_t lt2_gdr_backward_workspace_bytes(const lt2_gdr_dims* dims);
@@ -266,8 +266,8 @@ lt2_status lt2_gdr_backward(const lt2_gdr_dims* dims,
  * process exits.  (The paper has no counterpart: this is the library's own arrangement.)
  *   Arguments, layouts and results: exactly those of lt2_gdr_backward.
  *   Limit: a problem whose lt2_gdr_backward_workspace_bytes(dims) exceeds 64 MiB (67108864 bytes)
- *          returns LT2_ERR_WORKSPACE before any launch; for d_k = d_v = 128 that is 12 (loop,
- *          batch, head) units of 1,024 tokens, or 5 units of 8,192.
+ *          returns LT2_ERR_WORKSPACE before any launch; for d_k = d_v = 128 that is 15 (loop,
+ *          batch, head) units of 1,024 tokens, or 3 units of 8,192.
  *   Set-up: the first call on each device looks up the array's device address (with that device
  *          current) and keeps it; make that first call before any stream capture.
  *   Sharing: every call on a device uses the same array.  Nothing in it has to start at zero

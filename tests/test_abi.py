@@ -360,8 +360,9 @@ def call_backward(dims, ws=BASE + 40 * SPAN, ws_bytes=None, **over):
 
 def test_backward_workspace_query(L):
     d = D(L=150)
-    units, chunks, slices = 2 * 1 * 2, 3, 1                      # d = 32: one 32-column slice
-    assert lt2.lt2_gdr_backward_workspace_bytes(d) == units * slices * (chunks + 65) * 32 * 32 * 4
+    units, chunks, slices = 2 * 1 * 2, 5, 1                      # d = 32: one 32-column slice
+    # a checkpoint every 32 tokens (ceil(150 / 32) = 5) and the 33 states of one chunk, d_k x 32 fp32 each
+    assert lt2.lt2_gdr_backward_workspace_bytes(d) == units * slices * (chunks + 33) * 32 * 32 * 4
     assert L.lt2_gdr_backward_workspace_bytes(None) == 0
 
 
