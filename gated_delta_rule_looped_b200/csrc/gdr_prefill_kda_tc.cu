@@ -57,6 +57,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "gdr_common.cuh"
 #include "gdr_launch.h"
 #include "gdr_nvtx.h"
@@ -188,6 +190,15 @@ struct Params {
     float alpha_scale;
     const __nv_bfloat16* z;    // [units_total][L][128] output gate logits, or null
 };
+// The packed-sequence instances' parameters: q/k/v/o/z/alpha [T][H][L][128], beta [T][H][L] with L
+// the packed length; CTA = (sequence b, head h) of loop `loop`, tokens cu[b] .. cu[b+1]-1.  (A
+// separate type, so that the fixed-length instances keep their parameter block as it was.)
+struct ParamsVar : Params {
+    const int64_t* cu;
+    int H;
+    int loop;
+};
+template <bool kVar> using KdaParams = typename std::conditional<kVar, ParamsVar, Params>::type;
 
 #ifdef LT2_DEBUG
 // Fault injection of the debug build: the producer stops before this chunk (-1: never), so its
@@ -505,7 +516,7 @@ struct ExactIn {
 // decay_first: (I - beta k k^T) Diag(alpha), e = (alpha . k)^T S, S <- Diag(alpha) S + beta k (v - e)
 // kF (FuseBits): alpha and beta from logits, k and q divided by their L2 norms, o times sigmoid(z).
 template <bool decay_first, int kF>
-__device__ __noinline__ void exact_chunk(uint32_t tm_s, ExactIn p, int64_t row0, int n, int j)
+__device__ __forceinline__ void exact_body(uint32_t tm_s, const ExactIn& p, int64_t row0, int n, int j)
 {
     #pragma unroll 1
     for (int t = 0; t < n; ++t) {
@@ -608,6 +619,25 @@ __device__ __noinline__ void exact_chunk(uint32_t tm_s, ExactIn p, int64_t row0,
     }
 }
 
+// Two entry points with the same body.  The fixed-length kernels pass the inputs as one struct by
+// value: measured the lightest call for their register allocation.  The packed-sequence kernels,
+// whose parameter block is longer, pass them one by one: with that block, the struct passed by
+// value arrived wrong in a measured build.
+template <bool decay_first, int kF>
+__device__ __noinline__ void exact_chunk(uint32_t tm_s, ExactIn p, int64_t row0, int n, int j)
+{
+    exact_body<decay_first, kF>(tm_s, p, row0, n, j);
+}
+template <bool decay_first, int kF>
+__device__ __noinline__ void exact_chunk_args(uint32_t tm_s, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                                             const __nv_bfloat16* v, const float* alpha, const float* beta, void* o,
+                                             int out_bf16, int qk_norm, int gate_logits, float alpha_scale,
+                                             const __nv_bfloat16* z, int64_t row0, int n, int j)
+{
+    const ExactIn p{q, k, v, alpha, beta, o, out_bf16, nullptr, qk_norm, gate_logits, alpha_scale, z};
+    exact_body<decay_first, kF>(tm_s, p, row0, n, j);
+}
+
 // Chain thread j, fp32 output: o[r][j] = (Q^ S)_rj - B_rj for tokens r = r0 .. r0 + 15 below n
 // (tm_qs and tm_b address token r0), times sigmoid(z[r][j]) when z (column j of the chunk's
 // output gate logits) is given.
@@ -655,11 +685,11 @@ __device__ __noinline__ int issue_gram_of(int k, uint32_t sb, uint32_t tmem, int
 // normalised to unit L2 norm while they are converted; the output gate (o <- sigmoid(z) o, z read
 // from L1, where the chain prefetches it at the top of the chunk).  One instance per combination,
 // so that a call carries the code of the steps it uses only; kF = 0 compiles exactly as without.
-template <bool kDecayFirst, int kF>
+template <bool kDecayFirst, int kF, bool kVar>
 __global__ void __launch_bounds__(kThreads, 1)
 gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                          const __grid_constant__ CUtensorMap tm_a, Params p)
+                          const __grid_constant__ CUtensorMap tm_a, KdaParams<kVar> p)
 {
     allow_next_loop_to_start();
 
@@ -673,10 +703,32 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t L = p.L;
-    const int nchunks = static_cast<int>((L + kC - 1) / kC);
-    const int ug = p.unit0 + blockIdx.x;
+    const int ug = p.unit0 + blockIdx.x;             // global head-unit index (states)
     unsigned int* err = p.err;
+    // Where the unit's tokens live.  Fixed lengths: unit ug of the tensor maps, rows ug * L + t.
+    // Packed sequences: the TMA unit coordinate zv of (loop, head), the sequence's first row y0 and
+    // length, and the row index gbase of its first token in the gate, o and z arrays; a bad pair
+    // of offsets is reported and the CTA does nothing.
+    struct Where { int32_t zv; int64_t y0, len, gbase; bool ok; };
+    const Where wh = [&]() -> Where {
+        if constexpr (kVar) {
+            const int b = blockIdx.x / p.H, hd = blockIdx.x - b * p.H;
+            const int64_t c0 = p.cu[b], c1 = p.cu[b + 1];
+            const bool ok = 0 <= c0 && c0 <= c1 && c1 <= p.L;
+            if (!ok && threadIdx.x == 0) atomicOr(p.err, kDevSeqlens);
+            const int32_t zv = p.loop * p.H + hd;
+            return Where{zv, ok ? c0 : 0, ok ? c1 - c0 : 0, static_cast<int64_t>(zv) * p.L + (ok ? c0 : 0), ok};
+        } else {
+            return Where{ug, 0, p.L, 0, true};
+        }
+    }();
+    const int64_t L = wh.len;
+    const int32_t zc = kVar ? wh.zv : ug;
+    const bool seq_ok = wh.ok;
+    // row index of token t0 of the unit in the gate, o and z arrays; its TMA row coordinate
+    auto row_of = [&](int64_t t0) -> int64_t { return kVar ? wh.gbase + t0 : static_cast<int64_t>(ug) * L + t0; };
+    auto tma_row = [&](int64_t t0) -> int32_t { return static_cast<int32_t>(kVar ? wh.y0 + t0 : t0); };
+    const int nchunks = static_cast<int>((L + kC - 1) / kC);
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -741,20 +793,20 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                           mbar_wait(bar_addr(sb, B_AL_EMPTY + (c & 1)), ((c >> 1) & 1) ^ 1, abort_flag, err, kTimeoutNs);
             if (!__shfl_sync(0xffffffffu, free_ok, 0)) break;
             uint32_t leader;
-            if (elect_one(leader) && dbg_ok(c * kC < L && ug < p.units_total, err)) {
+            if (elect_one(leader) && dbg_ok(c * kC < L && zc < p.units_total, err)) {
                 const uint32_t fb = bar_addr(sb, B_FULL + s);
                 mbar_arrive_expect_tx(fb, STAGE_TX);
                 const uint32_t st = sb + OFF_STG + s * STAGE_BYTES;
-                const int32_t y = c * kC;
-                tma_load_3d(st + ST_KQ, &tm_k, 0, y, ug, fb);
-                tma_load_3d(st + ST_KQ + 8192, &tm_k, 64, y, ug, fb);
-                tma_load_3d(st + ST_KQ + 4096, &tm_q, 0, y, ug, fb);
-                tma_load_3d(st + ST_KQ + 8192 + 4096, &tm_q, 64, y, ug, fb);
-                tma_load_3d(st + ST_V, &tm_v, 0, y, ug, fb);
-                tma_load_3d(st + ST_V + 4096, &tm_v, 64, y, ug, fb);
+                const int32_t y = tma_row(static_cast<int64_t>(c) * kC);
+                tma_load_3d(st + ST_KQ, &tm_k, 0, y, zc, fb);
+                tma_load_3d(st + ST_KQ + 8192, &tm_k, 64, y, zc, fb);
+                tma_load_3d(st + ST_KQ + 4096, &tm_q, 0, y, zc, fb);
+                tma_load_3d(st + ST_KQ + 8192 + 4096, &tm_q, 64, y, zc, fb);
+                tma_load_3d(st + ST_V, &tm_v, 0, y, zc, fb);
+                tma_load_3d(st + ST_V + 4096, &tm_v, 64, y, zc, fb);
                 const uint32_t ab = bar_addr(sb, B_AL_FULL + (c & 1));
                 mbar_arrive_expect_tx(ab, ALPHA_STAGE);
-                tma_load_3d(sb + OFF_ALPHA + (c & 1) * ALPHA_STAGE, &tm_a, 0, y, ug, ab);
+                tma_load_3d(sb + OFF_ALPHA + (c & 1) * ALPHA_STAGE, &tm_a, 0, y, zc, ab);
             }
             __syncwarp();
             issued = c + 1;
@@ -779,7 +831,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
             // beta of token `lane` of this chunk: the load is issued before the waits below, which
             // hide its latency
-            float bl = lane < n ? p.beta[static_cast<int64_t>(ug) * L + t0 + lane] : 0.f;
+            float bl = lane < n ? p.beta[row_of(t0) + lane] : 0.f;
             if ((kF & kFuseLogits) && lane < n) bl = sigmoid_fast(bl);
             if (!grp.wait(bar_addr(sb, B_FULL + s), ph, bar_addr(sb, B_GATE_EMPTY + s), ph ^ 1,
                           bar_addr(sb, B_AL_FULL + (c & 1)), (c >> 1) & 1))
@@ -796,6 +848,9 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             Gates* gs = gate(s);
             // (written as a select between the two instances: the plain kernel's register
             // allocation, measured, is better this way)
+            // (packed sequences: the rows of a last, partial chunk past n hold the next sequence's
+            // tokens; with beta = 0 and alpha = 1 there they reach only their own rows of E and o,
+            // never the state or the rows below n, exactly as the zero rows of fixed lengths do)
             const bool in_range = ((kF & kFuseNorm) && p.qk_norm ? convert_kqv<kDecayFirst, true> : convert_kqv<kDecayFirst, false>)(
                                                            st, sb + OFF_GRAM + (c & 1) * GRAM_BUF, alpha_c, bl, Ph, Pt,
                                                            t_begin, t_end, lane, sbase, sb, gs->sq);
@@ -852,6 +907,13 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         const bool leader = warp == 8 && lane == 0;
         Group grp{NB_CHAIN, 256, leader, abort_flag, err};
         bool ok = nchunks > 0;
+        if constexpr (kVar) {
+            // an empty packed sequence: the state passes through unchanged (keys 64 h .. + 63)
+            if (nchunks == 0 && seq_ok && p.S_out) {
+                const int64_t base = static_cast<int64_t>(ug) * kD * kD + j;
+                for (int i = 64 * h; i < 64 * h + 64; ++i) p.S_out[base + i * kD] = p.S0 ? p.S0[base + i * kD] : 0.f;
+            }
+        }
         uint32_t ph_a = 0, ph_b = 0, ph_s = 0;
         if (ok) ok = grp.wait(bar_addr(sb, B_GATE_FULL + 0), 0);
         if (ok) {
@@ -881,7 +943,7 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             if ((kF & kFuseGate) && j < 2 * n) {
                 // the chunk's output gate logits (n rows of 256 bytes, two lines a row) into L1,
                 // for the output epilogue that runs under MMA_C
-                const __nv_bfloat16* zl = p.z + (static_cast<int64_t>(ug) * L + t0 + (j >> 1)) * kD + (j & 1) * 64;
+                const __nv_bfloat16* zl = p.z + (row_of(t0) + (j >> 1)) * kD + (j & 1) * 64;
                 asm volatile("prefetch.global.L1 [%0];" ::"l"(zl));
             }
             if (!exact) {
@@ -976,19 +1038,18 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 // the fp16 range carries infinities or NaNs to the end of the sequence)
                 if (!p.out_bf16) {
                     store_o_f32(tmem + TM_AB + lane_addr + 32 + 16 * h, tmem + TM_B + lane_addr + 32 + 16 * h,
-                                     static_cast<float*>(p.o) + (static_cast<int64_t>(ug) * L + t0) * kD + j, 16 * h, n,
-                                     (kF & kFuseGate) ? p.z + (static_cast<int64_t>(ug) * L + t0) * kD + j : nullptr);
+                                     static_cast<float*>(p.o) + row_of(t0) * kD + j, 16 * h, n,
+                                     (kF & kFuseGate) ? p.z + row_of(t0) * kD + j : nullptr);
                 } else {
                     float qp[32];
                     tmem_load_2x16(tmem + TM_AB + lane_addr + 32 + 16 * h, tmem + TM_B + lane_addr + 32 + 16 * h, qp);
                     uint8_t* ost = sbase + OFF_OST + (j >> 6) * 4096 + (j & 63) * 2 + 16 * h * 128;
                     // the fused output gate: column j of the chunk's logits, prefetched to L1
-                    const __nv_bfloat16* zc = (kF & kFuseGate) ? p.z + (static_cast<int64_t>(ug) * L + t0 + 16 * h) * kD + j
-                                                            : nullptr;
+                    const __nv_bfloat16* zr = (kF & kFuseGate) ? p.z + (row_of(t0) + 16 * h) * kD + j : nullptr;
                     #pragma unroll
                     for (int r = 0; r < 16; ++r) {
                         float ov = qp[r] - qp[16 + r];
-                        if ((kF & kFuseGate) && 16 * h + r < n) ov *= sigmoid_fast(__bfloat162float(zc[r * kD]));
+                        if ((kF & kFuseGate) && 16 * h + r < n) ov *= sigmoid_fast(__bfloat162float(zr[r * kD]));
                         *reinterpret_cast<__nv_bfloat16*>(ost + r * 128) = __float2bfloat16_rn(ov);
                     }
                     fence_proxy_async_smem();
@@ -999,25 +1060,50 @@ gdr_prefill_kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                 ph_s ^= 1u;
                 if (!ok) break;
                 tc_fence_after();
-                if (leader && p.out_bf16 && dbg_ok(t0 < L && ug < p.units_total, err)) {
-                    tma_store_3d(&tm_o, sb + OFF_OST, 0, static_cast<int32_t>(t0), ug);
-                    tma_store_3d(&tm_o, sb + OFF_OST + 4096, 64, static_cast<int32_t>(t0), ug);
+                if (kVar && t0 + kC > L) {
+                    // a packed sequence's last, partial chunk: the rows past its end belong to the
+                    // next sequence, so its n rows leave by plain 16-byte stores (both 64-column
+                    // halves of a row: 16 pieces), not by the two box stores
+                    if (p.out_bf16) {
+                        __nv_bfloat16* orow0 = static_cast<__nv_bfloat16*>(p.o) + row_of(t0) * kD;
+                        for (int i = threadIdx.x - 256; i < n * 16; i += 256) {
+                            const int r = i >> 4, part = i & 15;
+                            const uint4 w = *reinterpret_cast<const uint4*>(sbase + OFF_OST + (part >> 3) * 4096 +
+                                                                            r * 128 + (part & 7) * 16);
+                            *reinterpret_cast<uint4*>(orow0 + static_cast<int64_t>(r) * kD + (part >> 3) * 64 +
+                                                      (part & 7) * 8) = w;
+                        }
+                    }
+                } else if (leader && p.out_bf16 && dbg_ok(t0 < L && zc < p.units_total, err)) {
+                    tma_store_3d(&tm_o, sb + OFF_OST, 0, tma_row(t0), zc);
+                    tma_store_3d(&tm_o, sb + OFF_OST + 4096, 64, tma_row(t0), zc);
                     bulk_commit_group();
                 }
             } else {
                 // --- out-of-range chunk: the definition, token by token, on the fp32 state (the
                 // first half of the chain's warps; every key of a column takes part in k^T S) ---
-                if (h == 0)
-                    exact_chunk<kDecayFirst, kF>(tmem + TM_S + lane_addr,
+                // The state's keys 64-127 were written by the second half (the initial state or the
+                // last update): the group barrier orders those TMEM stores before these loads.
+                grp.sync();
+                tc_fence_after();
+                if (h == 0) {
+                    if constexpr (kVar)
+                        exact_chunk_args<kDecayFirst, kF>(tmem + TM_S + lane_addr, p.q, p.k, p.v, p.alpha, p.beta,
+                                                          p.o, p.out_bf16, p.qk_norm, p.gate_logits, p.alpha_scale,
+                                                          p.z, row_of(t0), n, j);
+                    else
+                        exact_chunk<kDecayFirst, kF>(tmem + TM_S + lane_addr,
                                                      ExactIn{p.q, p.k, p.v, p.alpha, p.beta, p.o, p.out_bf16, err,
                                                              p.qk_norm, p.gate_logits, p.alpha_scale, p.z},
-                                                     static_cast<int64_t>(ug) * L + t0, n, j);
+                                                     row_of(t0), n, j);
+                }
                 tc_fence_before();
                 // keep every hand-off in step: the stage and the [X; Z] stage are released
                 // once their producers are done with them, the output epilogue is released
                 ok = grp.wait(bar_addr(sb, B_CONV + s), ph, bar_addr(sb, B_TP_FULL + tps), (c >> 1) & 1,
                               last ? 0u : bar_addr(sb, B_GATE_FULL + s1), ((c + 1) / kStages) & 1);
                 if (!ok) break;
+                tc_fence_after();                       // the first half's TMEM stores, for the update
                 if (leader) {
                     mbar_arrive(bar_addr(sb, B_EMPTY + s));
                     mbar_arrive(bar_addr(sb, B_TP_EMPTY + tps));
@@ -1061,36 +1147,33 @@ bool prefill_kda_tc_supports(int dtype_bf16, int dk, int dv)
     return dtype_bf16 && dk == kda::kD && dv == kda::kD;
 }
 
-cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream)
+namespace kda {
+namespace {
+// One launch per loop of the instance for this layout, order of the per-key factors and
+// combination of fused steps (kVar: packed sequences, the ParamsVar block).  Internal linkage: a
+// template's static table would otherwise be one object per process, shared with any other copy
+// of this library loaded alongside (the debug build), whose kernels are not this library's.
+template <bool kVar>
+cudaError_t launch_loops(const TcCall& call, int64_t map_units, const CUtensorMap& mq, const CUtensorMap& mk,
+                         const CUtensorMap& mv, const CUtensorMap& mo, const CUtensorMap& ma, cudaStream_t stream)
 {
-    using namespace kda;
-    if (call.units_per_loop == 0 || call.T == 0) return cudaSuccess;
-    const int64_t units = call.T * call.units_per_loop;
-    CUtensorMap mq, mk, mv, mo;
-    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
-    if (!make_bf16_map_3d(&mq, call.q, units, call.L, kC, sw) || !make_bf16_map_3d(&mk, call.k, units, call.L, kC, sw) ||
-        !make_bf16_map_3d(&mv, call.v, units, call.L, kC, sw))
-        return cudaErrorInvalidValue;
-    if (call.out_bf16 && !make_bf16_map_3d(&mo, call.o, units, call.L, kC, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
-    CUtensorMap ma;
-    if (!make_f32_map_3d(&ma, call.alpha, units, call.L, kC)) return cudaErrorInvalidValue;
-    // one instance per order of the per-key factors and combination of fused steps
-    using K = decltype(&gdr_prefill_kda_tc_kernel<false, 0>);
+    using K = decltype(&gdr_prefill_kda_tc_kernel<false, 0, kVar>);
     static const K kernels[2][8] = {
-        {gdr_prefill_kda_tc_kernel<false, 0>, gdr_prefill_kda_tc_kernel<false, 1>, gdr_prefill_kda_tc_kernel<false, 2>,
-         gdr_prefill_kda_tc_kernel<false, 3>, gdr_prefill_kda_tc_kernel<false, 4>, gdr_prefill_kda_tc_kernel<false, 5>,
-         gdr_prefill_kda_tc_kernel<false, 6>, gdr_prefill_kda_tc_kernel<false, 7>},
-        {gdr_prefill_kda_tc_kernel<true, 0>, gdr_prefill_kda_tc_kernel<true, 1>, gdr_prefill_kda_tc_kernel<true, 2>,
-         gdr_prefill_kda_tc_kernel<true, 3>, gdr_prefill_kda_tc_kernel<true, 4>, gdr_prefill_kda_tc_kernel<true, 5>,
-         gdr_prefill_kda_tc_kernel<true, 6>, gdr_prefill_kda_tc_kernel<true, 7>}};
+        {gdr_prefill_kda_tc_kernel<false, 0, kVar>, gdr_prefill_kda_tc_kernel<false, 1, kVar>,
+         gdr_prefill_kda_tc_kernel<false, 2, kVar>, gdr_prefill_kda_tc_kernel<false, 3, kVar>,
+         gdr_prefill_kda_tc_kernel<false, 4, kVar>, gdr_prefill_kda_tc_kernel<false, 5, kVar>,
+         gdr_prefill_kda_tc_kernel<false, 6, kVar>, gdr_prefill_kda_tc_kernel<false, 7, kVar>},
+        {gdr_prefill_kda_tc_kernel<true, 0, kVar>, gdr_prefill_kda_tc_kernel<true, 1, kVar>,
+         gdr_prefill_kda_tc_kernel<true, 2, kVar>, gdr_prefill_kda_tc_kernel<true, 3, kVar>,
+         gdr_prefill_kda_tc_kernel<true, 4, kVar>, gdr_prefill_kda_tc_kernel<true, 5, kVar>,
+         gdr_prefill_kda_tc_kernel<true, 6, kVar>, gdr_prefill_kda_tc_kernel<true, 7, kVar>}};
     const K kernel = kernels[call.decay_first ? 1 : 0][fuse_bits(call)];
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess) return e;
     for (int64_t tau = 0; tau < call.T; ++tau) {
         NvtxRange loop_range("lt2 prefill loop (tensor core, per-key gating)");
-        Params p;
+        KdaParams<kVar> p;
         p.q = static_cast<const __nv_bfloat16*>(call.q);
         p.k = static_cast<const __nv_bfloat16*>(call.k);
         p.v = static_cast<const __nv_bfloat16*>(call.v);
@@ -1101,13 +1184,18 @@ cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream)
         p.S_out = call.S_out;
         p.L = call.L;
         p.unit0 = static_cast<int>(tau * call.units_per_loop);
-        p.units_total = static_cast<int>(units);
+        p.units_total = static_cast<int>(map_units);
         p.out_bf16 = call.out_bf16;
         p.err = call.err;
         p.qk_norm = call.qk_norm;
         p.gate_logits = call.gate_logits;
         p.alpha_scale = call.alpha_scale;
         p.z = static_cast<const __nv_bfloat16*>(call.z);
+        if constexpr (kVar) {
+            p.cu = call.cu_seqlens;
+            p.H = static_cast<int>(call.H);
+            p.loop = static_cast<int>(tau);
+        }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(call.units_per_loop), 1, 1);
         cfg.blockDim = dim3(kThreads, 1, 1);
@@ -1118,10 +1206,36 @@ cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream)
         attr[0].val.programmaticStreamSerializationAllowed = tau > 0 ? 1 : 0;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, kernel, mq, mk, mv, call.out_bf16 ? mo : mv, ma, p);
+        e = cudaLaunchKernelEx(&cfg, kernel, mq, mk, mv, mo, ma, p);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
+}
+}  // namespace
+}  // namespace kda
+
+cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream)
+{
+    using namespace kda;
+    if (call.units_per_loop == 0 || call.T == 0) return cudaSuccess;
+    const bool var = call.cu_seqlens != nullptr;
+    // TMA unit axis and row extent: [T*B*H][L] for fixed lengths, [T*H][Ntot] for packed sequences
+    const int64_t units = call.T * call.units_per_loop;
+    const int64_t map_units = var ? call.T * call.H : units;
+    CUtensorMap mq, mk, mv, mo;
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!make_bf16_map_3d(&mq, call.q, map_units, call.L, kC, sw) ||
+        !make_bf16_map_3d(&mk, call.k, map_units, call.L, kC, sw) ||
+        !make_bf16_map_3d(&mv, call.v, map_units, call.L, kC, sw))
+        return cudaErrorInvalidValue;
+    if (call.out_bf16 && !make_bf16_map_3d(&mo, call.o, map_units, call.L, kC, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    CUtensorMap ma;
+    if (!make_f32_map_3d(&ma, call.alpha, map_units, call.L, kC)) return cudaErrorInvalidValue;
+    // (o's map is only read with bf16 output; a copy of a valid map stands in otherwise)
+    const CUtensorMap& mo_or = call.out_bf16 ? mo : mv;
+    return var ? launch_loops<true>(call, map_units, mq, mk, mv, mo_or, ma, stream)
+               : launch_loops<false>(call, map_units, mq, mk, mv, mo_or, ma, stream);
 }
 
 }  // namespace lt2

@@ -355,8 +355,8 @@ lt2_status lt2_gdr_prefill_varlen(const lt2_gdr_dims* dims, const lt2_gdr_fused*
     lt2_status st = validate_varlen_dims(dims, &sz);
     if (st != LT2_OK) return st;
     const lt2_gdr_fused f = fused_or_none(fused);
-    const bool tc_ok = !is_per_key(dims) &&
-                       lt2::prefill_tc_supports(dims->dtype == LT2_DTYPE_BF16, (int)dims->dk, (int)dims->dv, 0);
+    const bool tc_ok = lt2::prefill_tc_supports(dims->dtype == LT2_DTYPE_BF16, (int)dims->dk, (int)dims->dv,
+                                                is_per_key(dims));
     if (dims->algo == LT2_ALGO_TENSOR_CORE && !tc_ok) return LT2_ERR_UNSUPPORTED;
     if (sz.units == 0) return LT2_OK;
     if (cu_seqlens == nullptr || (reinterpret_cast<uintptr_t>(cu_seqlens) & 7u) != 0) return LT2_ERR_INVALID_ARGUMENT;
@@ -402,7 +402,7 @@ lt2_status lt2_gdr_prefill_varlen(const lt2_gdr_dims* dims, const lt2_gdr_fused*
         call.units_per_loop = sz.per_loop;
         call.L = dims->L;
         call.out_bf16 = out_is_bf16(dims) ? 1 : 0;
-        call.decay_first = 0;
+        call.decay_first = dims->gate == LT2_GATE_PER_KEY_DECAY_FIRST ? 1 : 0;
         call.err = err;
         call.qk_norm = f.qk_l2norm;
         call.gate_logits = f.gate_logits;
@@ -410,7 +410,8 @@ lt2_status lt2_gdr_prefill_varlen(const lt2_gdr_dims* dims, const lt2_gdr_fused*
         call.z = f.z;
         call.cu_seqlens = cu_seqlens;
         call.H = dims->H;
-        cudaError_t e = lt2::launch_prefill_tc_all(call, s);
+        cudaError_t e = is_per_key(dims) ? lt2::launch_prefill_kda_tc_all(call, s)
+                                         : lt2::launch_prefill_tc_all(call, s);
         if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "prefill varlen (tensor core)");
         return LT2_OK;

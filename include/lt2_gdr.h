@@ -207,11 +207,11 @@ lt2_status lt2_gdr_prefill_fused(const lt2_gdr_dims* dims, const lt2_gdr_fused* 
  *   S0, S_out   [T][B][H][dk][dv] fp32, as for lt2_gdr_prefill (an empty sequence passes S0,
  *               or zeros, to S_out)
  *   fused       as lt2_gdr_prefill_fused (NULL: none)
- * Scalar gating with bf16 inputs and d = 128 runs on the tensor-core kernel (each CTA reads its
- * sequence's rows; the rows of a partial last chunk that belong to the next sequence are masked
- * out); every other case runs on the CUDA-core path.  LT2_ALGO_TENSOR_CORE with per-key gating
- * returns LT2_ERR_UNSUPPORTED.  No workspace is used (workspace may be NULL).  Same return
- * convention as lt2_gdr_prefill.
+ * bf16 inputs with d = 128 run on the tensor-core kernels, scalar or per-key gating, either
+ * order (each CTA reads its sequence's rows; the rows of a partial last chunk that belong to the
+ * next sequence are masked out and its outputs are written row by row); every other case runs on
+ * the CUDA-core path.  No workspace is used (workspace may be NULL).  Same return convention as
+ * lt2_gdr_prefill.
  */
 lt2_status lt2_gdr_prefill_varlen(const lt2_gdr_dims* dims, const lt2_gdr_fused* fused,
                                   const int64_t* cu_seqlens,

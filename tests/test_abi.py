@@ -330,9 +330,12 @@ def test_varlen_offsets_checked(L):
     assert call_varlen(D(), cu=addrs(7)[6] + 16) == lt2.LT2_ERR_INVALID_ARGUMENT        # offsets inside o
 
 
-def test_varlen_per_key_has_no_tensor_core_path(L):
-    d = D(dtype=lt2.LT2_DTYPE_BF16, dk=128, dv=128, gate=lt2.LT2_GATE_PER_KEY, algo=lt2.LT2_ALGO_TENSOR_CORE)
-    assert call_varlen(d) == lt2.LT2_ERR_UNSUPPORTED
+def test_varlen_tensor_core_needs_bf16_and_d128(L):
+    # both gatings have a tensor-core varlen path for bf16 inputs at d = 128, and only there
+    for gate in (lt2.LT2_GATE_SCALAR, lt2.LT2_GATE_PER_KEY, lt2.LT2_GATE_PER_KEY_DECAY_FIRST):
+        for over in (dict(dtype=lt2.LT2_DTYPE_F32, dk=128, dv=128), dict(dtype=lt2.LT2_DTYPE_BF16, dk=64, dv=64)):
+            d = D(gate=gate, algo=lt2.LT2_ALGO_TENSOR_CORE, **over)
+            assert call_varlen(d) == lt2.LT2_ERR_UNSUPPORTED
 
 
 def test_varlen_bad_dims_and_empty(L):

@@ -98,15 +98,78 @@ def test_tensor_core_leaves_rows_outside_the_sequences_alone():
     assert torch.equal(outs["bf16"][:, :, :73], outs["f32"][:, :, :73].to(torch.bfloat16))
 
 
-@pytest.mark.parametrize("order", ["delta_first", "decay_first"])
-def test_per_key_runs_on_the_cuda_core_path(order):
-    x = _x([5, 40, 0, 33], seed=5, gate="per_key")
-    o, S = _run(x, per_key=True, order=order)
+# the per-key kernel works in 32-token chunks: lengths around one and several of them
+LENS_PK = [1, 31, 32, 33, 100, 0, 70, 7]
+ORDERS = ["delta_first", "decay_first"]
+
+
+@pytest.mark.parametrize("order", ORDERS)
+@pytest.mark.parametrize("algo", [TC, CC])
+def test_per_key_bf16_matches_oracle(algo, order):
+    x = _x(LENS_PK, seed=5, gate="per_key")
+    o, S = _run(x, algo, per_key=True, order=order)
     o_ref, S_ref = _ref(x, per_key=True, order=order)
     check("o (per-key varlen)", o, o_ref, TOL["bf16"])
     check("S_T (per-key varlen)", S, S_ref, TOL["bf16"])
-    with pytest.raises(lt2.Lt2Error):
-        _run(x, TC, per_key=True, order=order)
+
+
+@pytest.mark.parametrize("order", ORDERS)
+def test_per_key_tensor_core_bf16_output_is_rounded_fp32_output(order):
+    x = _x(LENS_PK, seed=9, gate="per_key")
+    o32, S32 = _run(x, TC, out="f32", per_key=True, order=order)
+    o16, S16 = _run(x, TC, out="bf16", per_key=True, order=order)
+    assert torch.equal(o16, o32.to(torch.bfloat16)) and torch.equal(S16, S32)
+
+
+@pytest.mark.parametrize("order", ORDERS)
+def test_per_key_tensor_core_equal_lengths_equal_the_fixed_layout(order):
+    # B sequences of one length (4 chunks and a ragged 22-token tail) through the packed call give
+    # the fixed-layout call's numbers
+    T, B, H, L = 2, 3, 2, 150
+    x = _x([L] * B, seed=10, T=T, H=H, gate="per_key")
+    o, S = _run(x, TC, out="bf16", per_key=True, order=order)
+    unpack = lambda t: t.reshape(T, H, B, L, *t.shape[3:]).transpose(1, 2).contiguous()
+    of, Sf = lt2.prefill(unpack(x["q"]), unpack(x["k"]), unpack(x["v"]), unpack(x["alpha"]), unpack(x["beta"]),
+                         S0=x["S0"], per_key=True, algo=TC, out="bf16", order=order)
+    torch.cuda.synchronize()
+    assert torch.equal(unpack(o), of) and torch.equal(S, Sf)
+
+
+def test_per_key_tensor_core_leaves_rows_outside_the_sequences_alone():
+    lens = [40, 0, 3]
+    x = _x(lens + [30], seed=11, gate="per_key")
+    x["cu"] = x["cu"][:-1].contiguous()                      # the last 30 rows belong to no sequence
+    x["S0"] = x["S0"][:, :3].contiguous()
+    outs = {}
+    for dt, name in ((torch.float32, "f32"), (torch.bfloat16, "bf16")):
+        o = torch.full(x["v"].shape, 7.0, dtype=dt, device="cuda")
+        lt2.prefill_varlen(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["cu"], S0=x["S0"], algo=TC, o=o,
+                           out=name, per_key=True)
+        torch.cuda.synchronize()
+        assert lt2.lt2_gdr_last_device_error() == lt2.LT2_OK
+        assert torch.all(o[:, :, 43:] == 7.0)
+        outs[name] = o
+    o_ref, _ = _ref(x, per_key=True)
+    check("o (per-key sequences)", outs["f32"][:, :, :43], o_ref[:, :, :43], TOL["bf16"])
+    assert torch.equal(outs["bf16"][:, :, :43], outs["f32"][:, :, :43].to(torch.bfloat16))
+
+
+def test_per_key_fused_steps_on_packed_sequences():
+    lens = [50, 1, 32, 29]
+    N, T, H = sum(lens), 2, 2
+    w = inputs.workload("kda_prefill", T=T, B=1, H=H, L=N)
+    r = inputs.make_raw_inputs(w, seed=12, device="cuda")
+    x = {n: r[n][:, 0].contiguous() for n in ("q", "k", "v", "z", "a", "b")}
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int64, device="cuda")
+    for algo in (TC, CC):
+        o, S = lt2.prefill_varlen(x["q"], x["k"], x["v"], x["a"], x["b"], cu, algo=algo, out="f32", per_key=True,
+                                  qk_l2norm=True, gate_logits=True, alpha_scale=0.1, z=x["z"])
+        torch.cuda.synchronize()
+        assert lt2.lt2_gdr_last_device_error() == lt2.LT2_OK
+        o_ref, S_ref = ovarlen.prefill(*(to_np(x[n]) for n in ("q", "k", "v", "a", "b")), to_np(cu), per_key=True,
+                                       raw=dict(z=to_np(x["z"]), alpha_scale=0.1))
+        check(f"o (per-key fused varlen, algo {algo})", o, o_ref, TOL["bf16"])
+        check(f"S_T (per-key fused varlen, algo {algo})", S, S_ref, TOL["bf16"])
 
 
 @pytest.mark.parametrize("gate", ["scalar", "per_key"])
@@ -136,15 +199,17 @@ def test_fused_steps_on_packed_sequences():
         check(f"S_T (fused varlen, algo {algo})", S, S_ref, TOL["bf16"])
 
 
+@pytest.mark.parametrize("gate", ["scalar", "per_key"])
 @pytest.mark.parametrize("algo", [TC, CC])
-def test_bad_offsets_are_reported(algo):
-    x = _x([10, 20, 30], seed=8)
+def test_bad_offsets_are_reported(algo, gate):
+    pk = gate == "per_key"
+    x = _x([10, 20, 30], seed=8, gate=gate)
     x["cu"] = torch.tensor([0, 20, 10, 60], dtype=torch.int64, device="cuda")     # out of order
-    lt2.prefill_varlen(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["cu"], S0=x["S0"], algo=algo)
+    lt2.prefill_varlen(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["cu"], S0=x["S0"], algo=algo, per_key=pk)
     torch.cuda.synchronize()
     assert lt2.lt2_gdr_last_device_error() == lt2.LT2_ERR_SEQLENS
     # and the context is fine afterwards
     x["cu"] = torch.tensor([0, 10, 30, 60], dtype=torch.int64, device="cuda")
-    o, S = _run(x, algo)
-    o_ref, S_ref = _ref(x)
+    o, S = _run(x, algo, per_key=pk)
+    o_ref, S_ref = _ref(x, per_key=pk)
     check("o (after bad offsets)", o, o_ref, TOL["bf16"])
