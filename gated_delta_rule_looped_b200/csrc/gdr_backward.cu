@@ -394,14 +394,18 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
             }
             // the column sums of this step: e, k^T G, k^T Diag(alpha) G
             // (with a scalar alpha the third is alpha k^T G, and e of the decay-first order alpha k^T S)
-            float pe = 0.f, pg = 0.f, pd = 0.f;
+            // (scalar alpha: gs = G . S_{t-1} over the thread's rows gives its dalpha term without a
+            // per-element product: sum G P = gs - b e pg, sum dR S_{t-1} = gs - b kG ks)
+            float pe = 0.f, pg = 0.f, pd = 0.f, gs = 0.f;
             #pragma unroll
             for (int m = 0; m < kMaxRows; ++m) {
                 if (m >= rpw) break;
                 pe += kr[m] * ((kDF && kPK) ? ar[m] * sp[m] : sp[m]);
                 pg += kr[m] * G[m];
                 if (kPK) pd += kr[m] * ar[m] * G[m];
+                if (!kPK) gs += G[m] * sp[m];
             }
+            const float ks = pe;                        // k^T S_{t-1} over the thread's rows
             if (kDF && !kPK) pe *= a0;
             const float e = sum_row_groups(pe);
             const float kG = sum_row_groups(pg);
@@ -427,13 +431,12 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
                         const float R = ar_ * sp[m];
                         const float dR = G[m] - kr[m] * bkG;
                         dkx[m] = G[m] * bd - R * bkG;
-                        dax[m] = dR * sp[m];
+                        if (kPK) dax[m] = dR * sp[m];
                         G[m] = ar_ * dR;
                     } else {
-                        const float P = sp[m] - kr[m] * bE;
                         const float dP = ar_ * G[m];
                         dkx[m] = G[m] * bv - (sp[m] * bkdP + dP * bE);
-                        dax[m] = G[m] * P;
+                        if (kPK) dax[m] = G[m] * (sp[m] - kr[m] * bE);
                         G[m] = dP - kr[m] * bkdP;
                     }
                 }
@@ -442,9 +445,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
             if constexpr (kPK) {
                 park_rows(dax, 2, sl);
             } else {
-                float dal_sum = 0.f;
-                #pragma unroll
-                for (int mm = 0; mm < kMaxRows; ++mm) dal_sum += dax[mm];
+                const float dal_sum = kDF ? gs - b * kG * ks : gs - b * e * pg;
                 const float x = warp_sum(dal_sum);
                 if (lane == 0) pal[sl * 8 + w] = x;
             }
