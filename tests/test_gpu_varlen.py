@@ -135,6 +135,21 @@ def test_per_key_tensor_core_equal_lengths_equal_the_fixed_layout(order):
     assert torch.equal(unpack(o), of) and torch.equal(S, Sf)
 
 
+@pytest.mark.parametrize("order", ORDERS)
+def test_per_key_tensor_core_exact_chunks_on_packed_sequences(order):
+    # alpha^6 puts most chunks beyond the fp16 tile range (run token by token inside the kernel)
+    # and a zeroed alpha row is a reset: the packed instances' exact path, at every position of a
+    # sequence (first chunk, middle, a partial last chunk)
+    x = _x([100, 33, 0, 64, 7], seed=13, gate="per_key")
+    x["alpha"] = x["alpha"].double().pow(6.0).float()
+    x["alpha"][:, :, 40, :] = 0.0
+    x["alpha"][:, :, 120, 3] = 0.0
+    o, S = _run(x, TC, per_key=True, order=order)
+    o_ref, S_ref = _ref(x, per_key=True, order=order)
+    check("o (per-key varlen, exact chunks)", o, o_ref, TOL["bf16"])
+    check("S_T (per-key varlen, exact chunks)", S, S_ref, TOL["bf16"])
+
+
 def test_per_key_tensor_core_leaves_rows_outside_the_sequences_alone():
     lens = [40, 0, 3]
     x = _x(lens + [30], seed=11, gate="per_key")
