@@ -18,7 +18,8 @@
 //
 // Mapping: one CTA of 256 threads per head-unit.  Warp w owns the contiguous rows
 // [w*dk/8, (w+1)*dk/8); lane c owns columns 4c..4c+3 (one 16-byte access per row), so
-// every warp-wide access touches whole 128-byte lines.  The per-column partial sums are
+// every warp-wide access touches whole 128-byte lines; a thread issues its state loads before it
+// reads the token's vectors, so the two latencies overlap.  The per-column partial sums are
 // combined across the 8 warps through shared memory; the update is applied in registers
 // and written back with streaming stores.  The fused prologue (q, k normalised to unit L2
 // norm; alpha, beta from logits) and output gate (o <- sigmoid(z) o) have their own instances.
@@ -47,6 +48,17 @@ __global__ void __launch_bounds__(256, 2) gdr_decode_kernel(LoopSlice p, int use
     const int dk = p.dk, dv = p.dv;
     const int rpw = dk >> 3;
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // The state first: its loads (16 per thread) are in flight while the token's vectors are read
+    // and reduced, instead of after them.
+    float* S = p.S_out + u * (int64_t)dk * dv;
+    const bool active = lane * 4 < dv;
+    const int col = lane * 4;
+    const int r0 = w * rpw;
+    float4 s[16];
+    #pragma unroll
+    for (int m = 0; m < 16; ++m)
+        if (m < rpw && active) s[m] = ld_stream_f4(S + (int64_t)(r0 + m) * dv + col);
 
     const T* q = static_cast<const T*>(p.q) + u * dk;
     const T* k = static_cast<const T*>(p.k) + u * dk;
@@ -121,19 +133,12 @@ __global__ void __launch_bounds__(256, 2) gdr_decode_kernel(LoopSlice p, int use
     }
     __syncthreads();
 
-    float* S = p.S_out + u * (int64_t)dk * dv;
-    const bool active = lane * 4 < dv;
-    const int col = lane * 4;
-    const int r0 = w * rpw;
-
-    float4 s[16];
     float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
     float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
     #pragma unroll
     for (int m = 0; m < 16; ++m) {
         if (m < rpw && active) {
             const int r = r0 + m;
-            s[m] = ld_stream_f4(S + (int64_t)r * dv + col);
             const float kr = kDecayFirst ? sk[r] * sa[r] : sk[r], ar = saq[r];
             e.x += kr * s[m].x; e.y += kr * s[m].y; e.z += kr * s[m].z; e.w += kr * s[m].w;
             f.x += ar * s[m].x; f.y += ar * s[m].y; f.z += ar * s[m].z; f.w += ar * s[m].w;
