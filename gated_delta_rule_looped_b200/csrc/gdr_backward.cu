@@ -134,18 +134,27 @@ __host__ __device__ inline size_t smem_bytes(int dk, int per_key)
            sizeof(float);
 }
 
-// 8 consecutive elements of a row (16-byte aligned) into shared memory as fp32
-__device__ __forceinline__ void ld8(const float* src, float* dst)
+// 8 consecutive elements of a row (16-byte aligned) into shared memory as fp32, in two halves:
+// a thread issues all its loads before it stores any of them.
+template <typename T> struct Raw8;
+template <> struct Raw8<float> { float4 a, b; };
+template <> struct Raw8<__nv_bfloat16> { uint4 a; };
+__device__ __forceinline__ Raw8<float> raw8_load(const float* src)
 {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(src));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
-    reinterpret_cast<float4*>(dst)[0] = a;
-    reinterpret_cast<float4*>(dst)[1] = b;
+    return Raw8<float>{__ldg(reinterpret_cast<const float4*>(src)), __ldg(reinterpret_cast<const float4*>(src) + 1)};
 }
-__device__ __forceinline__ void ld8(const __nv_bfloat16* src, float* dst)
+__device__ __forceinline__ Raw8<__nv_bfloat16> raw8_load(const __nv_bfloat16* src)
 {
-    const uint4 r = __ldg(reinterpret_cast<const uint4*>(src));
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r);
+    return Raw8<__nv_bfloat16>{__ldg(reinterpret_cast<const uint4*>(src))};
+}
+__device__ __forceinline__ void raw8_store(const Raw8<float>& r, float* dst)
+{
+    reinterpret_cast<float4*>(dst)[0] = r.a;
+    reinterpret_cast<float4*>(dst)[1] = r.b;
+}
+__device__ __forceinline__ void raw8_store(const Raw8<__nv_bfloat16>& r, float* dst)
+{
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r.a);
     const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
     const float2 f2 = __bfloat1622float2(h[2]), f3 = __bfloat1622float2(h[3]);
     reinterpret_cast<float4*>(dst)[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
@@ -221,24 +230,55 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
 
     // the inputs of tokens t0 .. t0+n-1 into shared memory (q and dO only for the reverse sweep);
     // every tensor is 16-byte aligned and d_k, d_v are multiples of 8, so rows move 8 elements at a time
+    // A thread's pieces: rows of k, q (and per-key alpha) at most 2 (i0, i1), one v / dO piece,
+    // one beta and one scalar alpha.  All are loaded before the barrier that frees the previous
+    // chunk's buffers, so their latency overlaps the wait for the other warps.
+    static_assert(kChunk * 128 / 8 <= 2 * kThreads && kChunk * (kCols / 8) <= kThreads, "chunk pieces per thread");
     auto load_chunk = [&](int64_t t0, int n, bool with_q) {
-        __syncthreads();                                        // the previous chunk is consumed
         const int pieces = n * dk / 8;
-        for (int i = tid; i < pieces; i += kThreads) {
-            ld8(k + t0 * dk + 8 * i, sk + 8 * i);
-            if (with_q) ld8(q + t0 * dk + 8 * i, sq + 8 * i);
+        const int i0 = tid, i1 = tid + kThreads;
+        Raw8<T> k0{}, k1{}, q0{}, q1{}, v0{}, o0{};
+        Raw8<float> a0{}, a1{};
+        float as = 1.f, bs = 0.f;
+        if (i0 < pieces) {
+            k0 = raw8_load(k + t0 * dk + 8 * i0);
+            if (with_q) q0 = raw8_load(q + t0 * dk + 8 * i0);
+            if constexpr (kPK) a0 = raw8_load(al + t0 * dk + 8 * i0);
         }
-        if constexpr (kPK) {
-            for (int i = tid; i < pieces; i += kThreads) ld8(al + t0 * dk + 8 * i, sa + 8 * i);
-        } else {
-            for (int i = tid; i < n; i += kThreads) sa[i] = al[t0 + i];
+        if (i1 < pieces) {
+            k1 = raw8_load(k + t0 * dk + 8 * i1);
+            if (with_q) q1 = raw8_load(q + t0 * dk + 8 * i1);
+            if constexpr (kPK) a1 = raw8_load(al + t0 * dk + 8 * i1);
         }
-        for (int i = tid; i < n; i += kThreads) sbe[i] = be[t0 + i];
-        for (int i = tid; i < n * (kCols / 8); i += kThreads) {
-            const int tt = i / (kCols / 8), cc = (i % (kCols / 8)) * 8;
-            if (j0 + cc < dv) {                                 // a piece lies wholly inside d_v or outside
-                ld8(v + (t0 + tt) * dv + j0 + cc, sv + tt * kCols + cc);
-                if (with_q) ld8(dO + (t0 + tt) * dv + j0 + cc, sdo + tt * kCols + cc);
+        if (tid < n) {
+            if constexpr (!kPK) as = al[t0 + tid];
+            bs = be[t0 + tid];
+        }
+        const int tt = tid / (kCols / 8), cc = (tid % (kCols / 8)) * 8;
+        const bool vpiece = tid < n * (kCols / 8), vin = vpiece && j0 + cc < dv;   // wholly inside d_v or outside
+        if (vin) {
+            v0 = raw8_load(v + (t0 + tt) * dv + j0 + cc);
+            if (with_q) o0 = raw8_load(dO + (t0 + tt) * dv + j0 + cc);
+        }
+        __syncthreads();                                        // the previous chunk is consumed
+        if (i0 < pieces) {
+            raw8_store(k0, sk + 8 * i0);
+            if (with_q) raw8_store(q0, sq + 8 * i0);
+            if constexpr (kPK) raw8_store(a0, sa + 8 * i0);
+        }
+        if (i1 < pieces) {
+            raw8_store(k1, sk + 8 * i1);
+            if (with_q) raw8_store(q1, sq + 8 * i1);
+            if constexpr (kPK) raw8_store(a1, sa + 8 * i1);
+        }
+        if (tid < n) {
+            if constexpr (!kPK) sa[tid] = as;
+            sbe[tid] = bs;
+        }
+        if (vpiece) {
+            if (vin) {
+                raw8_store(v0, sv + tt * kCols + cc);
+                if (with_q) raw8_store(o0, sdo + tt * kCols + cc);
             } else {
                 zero8(sv + tt * kCols + cc);
                 if (with_q) zero8(sdo + tt * kCols + cc);
@@ -335,15 +375,15 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
     for (int ci = nck - 1; ci >= 0; --ci) {
         const int64_t t0 = static_cast<int64_t>(ci) * kChunk;
         const int n = static_cast<int>(L - t0 < kChunk ? L - t0 : kChunk);
-        load_chunk(t0, n, true);
         {
-            const float* cp = ck + ci * sst;
+            const float* cp = ck + ci * sst;                    // (in flight while the inputs load)
             #pragma unroll
-            for (int m = 0; m < kMaxRows; ++m) {
-                s[m] = m < rpw ? cp[m * kThreads] : 0.f;
-                if (m < rpw) st[m * kThreads] = s[m];
-            }
+            for (int m = 0; m < kMaxRows; ++m) s[m] = m < rpw ? cp[m * kThreads] : 0.f;
         }
+        load_chunk(t0, n, true);
+        #pragma unroll
+        for (int m = 0; m < kMaxRows; ++m)
+            if (m < rpw) st[m * kThreads] = s[m];
         for (int tau = 0; tau < n; ++tau) {
             step(s, tau);
             if (tau + 1 < n) {                                  // S_t of the last token stays in s
