@@ -213,8 +213,9 @@ __device__ __noinline__ void load_initial_state(uint32_t tm_s, uint32_t tm_sh, c
 }
 
 // Output thread j, fp32 output: o[r][j] = g_r (Q S)_rj + (P T X)_rj for the chunk's n tokens,
-// times sigmoid(z[r][j]) when `zst` points at column j of the output gate logits in the staging
-// tile (rows 128 bytes apart).  Returns false if any of them is not finite.
+// times sigmoid(z[r][j]) when `zst` points at column j of the output gate in the staging tile
+// (rows 128 bytes apart; the gate already taken through the sigmoid, fp16).  Returns false if any
+// of them is not finite.
 __device__ __noinline__ bool store_o_f32(uint32_t tm_qs, uint32_t tm_ptx, const float* gam, float* o, int n,
                                          const uint8_t* zst)
 {
@@ -227,7 +228,7 @@ __device__ __noinline__ bool store_o_f32(uint32_t tm_qs, uint32_t tm_ptx, const 
         for (int e = 0; e < 32; ++e) {
             const int r = 32 * piece + e;
             float ov = gam[r] * qp[e] + qp[32 + e];
-            if (zst) ov *= sigmoid_fast(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(zst + r * 128)));
+            if (zst) ov *= __half2float(*reinterpret_cast<const __half*>(zst + r * 128));
             if (r < n) {
                 fin &= is_finite(ov);
                 o[r * kD] = ov;
@@ -814,9 +815,18 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 tma_load_3d(sb + OFF_OST, &tm_z, 0, static_cast<int32_t>(y0 + t0), zc, zb);
                 tma_load_3d(sb + OFF_OST + 8192, &tm_z, 64, static_cast<int32_t>(y0 + t0), zc, zb);
             }
-            if (!(gated ? grp.wait(bar_addr(sb, B_O_READY), c & 1, bar_addr(sb, B_Z), c & 1)
-                        : grp.wait(bar_addr(sb, B_O_READY), c & 1)))
-                break;
+            if constexpr (gated) {
+                // sigmoid(z) of this thread's column, in place as fp16, while the chain is still
+                // working on the chunk: the output's own wait below is then free of MUFU work
+                if (!grp.wait(bar_addr(sb, B_Z), c & 1)) break;
+                uint8_t* zcol = sbase + OFF_OST + (j >> 6) * 8192 + (j & 63) * 2;
+                #pragma unroll 8
+                for (int r = 0; r < kC; ++r) {
+                    const float zr = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(zcol + r * 128));
+                    *reinterpret_cast<__half*>(zcol + r * 128) = __float2half_rn(sigmoid_fast(zr));
+                }
+            }
+            if (!grp.wait(bar_addr(sb, B_O_READY), c & 1)) break;
             tc_fence_after();
             const Gates* gs = gate(s);
             if (!p.out_bf16) {
@@ -848,9 +858,9 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     const float2 g2 = *reinterpret_cast<const float2*>(&gs->gam[r]);
                     float o0 = g2.x * qp[e] + qp[16 + e];
                     float o1 = g2.y * qp[e + 1] + qp[16 + e + 1];
-                    if (gated) {
-                        o0 *= sigmoid_fast(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(ost + r * 128)));
-                        o1 *= sigmoid_fast(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(ost + (r + 1) * 128)));
+                    if (gated) {                     // sigmoid(z), fp16, from the staging tile
+                        o0 *= __half2float(*reinterpret_cast<const __half*>(ost + r * 128));
+                        o1 *= __half2float(*reinterpret_cast<const __half*>(ost + (r + 1) * 128));
                     }
                     if constexpr (kVar) {
                         // rows past the sequence end hold the next sequence's tokens: not outputs
