@@ -38,6 +38,9 @@ struct TcCall {
     // is the packed length Ntot and q/k/v/o/z are [T][H][Ntot][128], alpha/beta [T][H][Ntot]
     const int64_t* cu_seqlens = nullptr;
     int64_t H = 0;
+    // scratch for the balanced schedule of the scalar kernel (one flag per unit), or null
+    void* workspace = nullptr;
+    size_t workspace_bytes = 0;
 };
 // The fused steps of a call as the template argument of the tensor-core kernels' instances.
 enum FuseBits : int { kFuseNorm = 1, kFuseLogits = 2, kFuseGate = 4 };
@@ -49,6 +52,8 @@ inline int fuse_bits(const TcCall& c)
 // Scalar gating: 64-token chunks.  Per-key gating: 32-token chunks in the e-form (chunks whose
 // per-key decay is out of the tensor-core range run token by token inside the same kernel).
 bool prefill_tc_supports(int dtype_bf16, int dk, int dv, int per_key);
+// Workspace bytes of the scalar tensor-core prefill's balanced schedule: one flag per unit.
+size_t prefill_tc_flag_bytes(int64_t units);
 cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream);
 bool prefill_kda_tc_supports(int dtype_bf16, int dk, int dv);
 cudaError_t launch_prefill_kda_tc_all(const TcCall& call, cudaStream_t stream);

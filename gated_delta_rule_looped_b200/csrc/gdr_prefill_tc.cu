@@ -126,6 +126,12 @@ enum Bar : uint32_t {
 };
 constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + B_COUNT * 8;        // tcgen05.alloc result
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 16;
+// Balanced launches: this CTA's segments (count, then {unit, first chunk, end chunk, flags}).
+constexpr int kMaxSeg = 8;
+constexpr uint32_t OFF_SEGS = OFF_ABORT + 16;
+static_assert(OFF_SEGS + 16 + kMaxSeg * 16 <= OFF_BAR + BAR_BYTES, "barrier area too small");
+constexpr int kSegIn = 1;              // the segment's first state is handed over (flag, then S_out)
+constexpr int kSegOut = 2;             // the segment's last state is handed on (S_out, then flag)
 
 // Named barriers (bar.sync ids; 0 is __syncthreads).
 constexpr int NB_PREP = 1;             // warps 4-7
@@ -168,7 +174,35 @@ struct Params {
     int64_t Ntot;
     int H;
     int loop;
+    // balanced launches (one launch for every loop): the units' chunks laid end to end, bal_per_cta
+    // of them per CTA; a unit split between two CTAs hands its state over through S_out, and
+    // bal_flags[unit] (zeroed before the launch) says when
+    int bal_units;
+    int bal_chunks;
+    int bal_per_cta;
+    unsigned int* bal_flags;
 };
+
+// Bounded wait for a handoff flag set by another CTA of the same launch (acquire).
+__device__ __noinline__ bool wait_handoff(const unsigned int* f, volatile int* abort_flag, unsigned int* err)
+{
+    uint64_t t0 = 0;
+    for (uint32_t it = 1;; ++it) {
+        unsigned int v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+        if (v) return true;
+        if (*abort_flag) return false;
+        const uint64_t now = global_timer_ns();
+        if (t0 == 0) {
+            t0 = now;
+        } else if (now - t0 > kWaitTimeoutNs) {
+            *abort_flag = 1;
+            atomicOr(err, 1u);
+            return false;
+        }
+        __nanosleep(200);
+    }
+}
 
 #ifdef LT2_DEBUG
 // Fault injection of the debug build: the producer stops before this chunk (-1: never), so its
@@ -271,7 +305,7 @@ __device__ __noinline__ void gram_epilogue_unfactored(uint32_t tm_row, const Gat
 // gate (the logits z of a chunk are loaded by TMA into the o staging tile, and o <- sigmoid(z) o
 // is applied as the tile is written).  One instance per combination, so that a call carries the
 // code of the steps it uses only; kF = 0 compiles exactly as without them.
-template <int kF, bool kVar>
+template <int kF, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
 gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -279,6 +313,8 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 {
     (void)use_pdl;
     allow_next_loop_to_start();
+    constexpr bool kVar = kMode == 1;       // packed sequences
+    constexpr bool kBal = kMode == 2;       // balanced: segments of units, one launch for every loop
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -315,11 +351,56 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         L = seq_ok ? c1 - c0 : 0;
         gbase = static_cast<int64_t>(zc) * p.Ntot + y0;
     }
-    const int nchunks = static_cast<int>((L + kC - 1) / kC);
+    // this CTA's chunks: one unit's, or (balanced) the range [bal_a, bal_b) of all units' chunks
+    // laid end to end
+    const int64_t bal_a = kBal ? static_cast<int64_t>(blockIdx.x) * p.bal_per_cta : 0;
+    const int64_t bal_b = kBal ? min(bal_a + p.bal_per_cta, static_cast<int64_t>(p.bal_units) * p.bal_chunks) : 0;
+    const int nchunks = kBal ? static_cast<int>(bal_b > bal_a ? bal_b - bal_a : 0) : static_cast<int>((L + kC - 1) / kC);
+    // Where chunk g of this CTA lives: its unit's TMA coordinate zc and state index unit, the
+    // unit's first row y0 and gate/o base gbase, the chunk's index c in the unit, and (balanced)
+    // whether it starts or ends its segment and how that segment's states are handed.
+    struct Loc { int32_t zc; int unit; int64_t y0, gbase; int c; bool first, last; int flags; };
+    auto loc = [&](int g) -> Loc {
+        if constexpr (kBal) {
+            const int* tab = reinterpret_cast<const int*>(sbase + OFF_SEGS);
+            const int n = tab[0];
+            int g0 = 0;
+            for (int i = 0; i < n; ++i) {
+                const int4 sg = reinterpret_cast<const int4*>(tab + 4)[i];
+                const int len = sg.z - sg.y;
+                if (g < g0 + len || i == n - 1)
+                    return Loc{sg.x, sg.x, 0, static_cast<int64_t>(sg.x) * p.L, sg.y + (g - g0), g == g0,
+                               g == g0 + len - 1, sg.w};
+                g0 += len;
+            }
+            return Loc{ug, ug, 0, 0, g, true, true, 0};   // (no segment: not reached)
+        } else {
+            return Loc{zc, ug, y0, gbase, g, g == 0, g == nchunks - 1, 0};
+        }
+    };
 
     // ---- set-up: barriers, TMEM ----
     if (threadIdx.x == 0) {
         *abort_flag = 0;
+        if constexpr (kBal) {
+            // the segments of [bal_a, bal_b), in this order: the start of a unit that the next
+            // CTA finishes (its state handed on), whole units, then the end of a unit whose start
+            // the previous CTA ran first (its state handed over)
+            const int64_t N = p.bal_chunks;
+            int* tab = reinterpret_cast<int*>(sbase + OFF_SEGS);
+            int4* segs = reinterpret_cast<int4*>(tab + 4);
+            int n = 0;
+            for (int kind = 0; kind < 3; ++kind) {
+                for (int64_t u = bal_a / N; u * N < bal_b && n < kMaxSeg; ++u) {
+                    const int c0 = static_cast<int>(bal_a > u * N ? bal_a - u * N : 0);
+                    const int c1 = static_cast<int>(bal_b - u * N < N ? bal_b - u * N : N);
+                    const int k = c0 > 0 ? 2 : (c1 < N ? 0 : 1);
+                    if (k != kind) continue;
+                    segs[n++] = make_int4(static_cast<int>(u), c0, c1, (c0 > 0 ? kSegIn : 0) | (c1 < N ? kSegOut : 0));
+                }
+            }
+            tab[0] = n;
+        }
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar_addr(sb, B_FULL + s), 1);
             mbar_init(bar_addr(sb, B_CONV + s), 3);
@@ -390,17 +471,18 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 const int s = cc % kStages;
                 if (!mbar_wait(bar_addr(sb, B_EMPTY + s), ((cc / kStages) & 1) ^ 1, abort_flag, err, kTimeoutNs))
                     return false;
-                if (elect_one(issuer) && dbg_ok(cc * kC < L && zc < p.units_total, err)) {
+                const Loc lc = loc(cc);
+                if (elect_one(issuer) && dbg_ok(lc.c * kC < L && lc.zc < p.units_total, err)) {
                     const uint32_t fb = bar_addr(sb, B_FULL + s);
                     mbar_arrive_expect_tx(fb, STAGE_BYTES);
                     const uint32_t st = sb + OFF_KQV + s * STAGE_BYTES;
-                    const int32_t y = static_cast<int32_t>(y0 + cc * kC);
-                    tma_load_3d(st, &tm_k, 0, y, zc, fb);
-                    tma_load_3d(st + 16384, &tm_k, 64, y, zc, fb);
-                    tma_load_3d(st + 8192, &tm_q, 0, y, zc, fb);
-                    tma_load_3d(st + 24576, &tm_q, 64, y, zc, fb);
-                    tma_load_3d(st + KQ_BYTES, &tm_v, 0, y, zc, fb);
-                    tma_load_3d(st + KQ_BYTES + 8192, &tm_v, 64, y, zc, fb);
+                    const int32_t y = static_cast<int32_t>(lc.y0 + lc.c * kC);
+                    tma_load_3d(st, &tm_k, 0, y, lc.zc, fb);
+                    tma_load_3d(st + 16384, &tm_k, 64, y, lc.zc, fb);
+                    tma_load_3d(st + 8192, &tm_q, 0, y, lc.zc, fb);
+                    tma_load_3d(st + 24576, &tm_q, 64, y, lc.zc, fb);
+                    tma_load_3d(st + KQ_BYTES, &tm_v, 0, y, lc.zc, fb);
+                    tma_load_3d(st + KQ_BYTES + 8192, &tm_v, 64, y, lc.zc, fb);
                 }
                 loaded = cc + 1;
                 return true;
@@ -490,12 +572,13 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // the global loads hides behind this chunk's gates, conversion and Gram issue
         float a_nx[2] = {1.f, 1.f}, b_nx[2] = {0.f, 0.f};
         auto load_gate_inputs = [&](int cn) {
+            const Loc ln = loc(cn < nchunks ? cn : 0);
             #pragma unroll
             for (int i = 0; i < 2; ++i) {
-                const int64_t tok = static_cast<int64_t>(cn) * kC + lane + 32 * i;
+                const int64_t tok = static_cast<int64_t>(ln.c) * kC + lane + 32 * i;
                 const bool valid = cn < nchunks && tok < L;
-                a_nx[i] = valid ? p.alpha[gbase + tok] : 1.f;
-                b_nx[i] = valid ? p.beta[gbase + tok] : 0.f;
+                a_nx[i] = valid ? p.alpha[ln.gbase + tok] : 1.f;
+                b_nx[i] = valid ? p.beta[ln.gbase + tok] : 0.f;
             }
         };
         if (warp == 1) load_gate_inputs(0);
@@ -514,11 +597,12 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 float carry = 0.f;
                 uint32_t negs_before = 0;
                 bool in_range = true;                   // every |G_r| < 80
+                const int64_t tok0 = static_cast<int64_t>(loc(c).c) * kC;   // the chunk's first token in its unit
                 #pragma unroll 1
                 for (int i = 0; i < 2; ++i) {
                     float a = i ? a_cur[1] : a_cur[0];
                     // (past the sequence end alpha = 1 and beta = 0 already: no logits there)
-                    const bool valid = static_cast<int64_t>(c) * kC + lane + 32 * i < L;
+                    const bool valid = tok0 + lane + 32 * i < L;
                     if ((kF & kFuseLogits) && valid) a = alpha_from_logit_fast(a, p.alpha_scale);
                     float g = __logf(fmaxf(fabsf(a), 1e-30f));
                     #pragma unroll
@@ -709,14 +793,34 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int i = 0; i < kD; ++i) p.S_out[base + i * kD] = p.S0 ? p.S0[base + i * kD] : 0.f;
             }
         }
-        // initial state: S0^T (fp32 in TMEM, pre-scaled by the first chunk's decay; fp16 copy)
-        if (ok) ok = grp.wait(bar_addr(sb, B_GATE_FULL + 0), 0);
-        if (ok) {
-            load_initial_state(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr,
-                               p.S0 ? p.S0 + static_cast<int64_t>(ug) * kD * kD + j : nullptr, gate(0)->gC);
+        // a segment's initial state: S0^T, or (balanced, the end of a unit begun by the previous
+        // CTA) the state it handed over in S_out; fp32 in TMEM, pre-scaled by the first chunk's
+        // decay, and an fp16 copy.  Chunk g's gates are in (its stage's GATE_FULL was waited).
+        auto segment_start = [&](int g) -> bool {
+            const Loc ls = loc(g);
+            const float* src = p.S0 ? p.S0 + static_cast<int64_t>(ls.unit) * kD * kD + j : nullptr;
+            if constexpr (kBal) {
+                if (ls.flags & kSegIn) {
+                    const unsigned int* f = p.bal_flags + ls.unit;
+                    const int got = leader ? (wait_handoff(f, abort_flag, err) ? 1 : 0) : 1;
+                    unsigned int all;
+                    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                                 "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                                 : "=r"(all) : "r"(got), "r"(NB_CHAIN), "r"(128) : "memory");
+                    if (!all) return false;
+                    unsigned int v;                      // (every thread acquires the handoff)
+                    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+                    (void)v;
+                    src = p.S_out + static_cast<int64_t>(ls.unit) * kD * kD + j;
+                }
+            }
+            load_initial_state(tmem + TM_S + lane_addr, tmem + TM_SH + lane_addr, src, gate(g % kStages)->gC);
             tc_fence_before();
-        }
-        if (ok) mbar_arrive(bar_addr(sb, B_SH_READY));      // MMA_A of chunk 0 may read it
+            mbar_arrive(bar_addr(sb, B_SH_READY));           // MMA_A of chunk g may read it
+            return true;
+        };
+        if (ok) ok = grp.wait(bar_addr(sb, B_GATE_FULL + 0), 0);
+        if (ok) ok = segment_start(0);
         for (int c = 0; ok && c < nchunks; ++c) {
             const int s = c % kStages;
             const Gates* gs = gate(s);
@@ -769,11 +873,27 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                                  ((c + 1) / kStages) & 1);
             if (!ok) break;
             tc_fence_after();
-            if (last) {
+            const Loc lc = loc(c);
+            if (kBal ? lc.last : last) {
+                // the segment's last state: the final state of its unit, or (balanced) the state
+                // handed on to the CTA that finishes the unit
                 if (p.S_out) {
                     const bool sfin = store_final_state(tmem + TM_S + lane_addr,
-                                                        p.S_out + static_cast<int64_t>(ug) * kD * kD + j);
+                                                        p.S_out + static_cast<int64_t>(lc.unit) * kD * kD + j);
                     if (__any_sync(0xffffffffu, !sfin) && lane == 0) atomicOr(err, kDevRange);
+                }
+                if constexpr (kBal) {
+                    if (lc.flags & kSegOut) {
+                        __threadfence();                 // this thread's column, then the flag
+                        grp.sync();
+                        if (leader)
+                            asm volatile("st.release.gpu.global.u32 [%0], %1;" :: "l"(p.bal_flags + lc.unit), "r"(1u)
+                                         : "memory");
+                    }
+                    if (!last) {
+                        ok = segment_start(c + 1);       // the next segment, from its first chunk
+                        if (!ok) break;
+                    }
                 }
             } else {
                 const float gn = gate(s1)->gC;
@@ -804,7 +924,8 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         bool fin = true;                             // every output so far is finite
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;
-            const int64_t t0 = static_cast<int64_t>(c) * kC;
+            const Loc lo = loc(c);
+            const int64_t t0 = static_cast<int64_t>(lo.c) * kC;      // the chunk's first token in its unit
             if (j == 0) bulk_wait_read_all();        // the staging tile is free again
             constexpr bool gated = (kF & kFuseGate) != 0;
             if (gated && j == 0) {
@@ -812,8 +933,8 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 // written to (the same two 64 x 64 boxes; rows past L read as 0)
                 const uint32_t zb = bar_addr(sb, B_Z);
                 mbar_arrive_expect_tx(zb, 16384);
-                tma_load_3d(sb + OFF_OST, &tm_z, 0, static_cast<int32_t>(y0 + t0), zc, zb);
-                tma_load_3d(sb + OFF_OST + 8192, &tm_z, 64, static_cast<int32_t>(y0 + t0), zc, zb);
+                tma_load_3d(sb + OFF_OST, &tm_z, 0, static_cast<int32_t>(lo.y0 + t0), lo.zc, zb);
+                tma_load_3d(sb + OFF_OST + 8192, &tm_z, 64, static_cast<int32_t>(lo.y0 + t0), lo.zc, zb);
             }
             if constexpr (gated) {
                 // sigmoid(z) of this thread's column, in place as fp16, while the chain is still
@@ -833,7 +954,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 // fp32 output: plain stores, done before the TMEM columns are released
                 const int n = static_cast<int>(L - t0 < kC ? L - t0 : kC);
                 fin &= store_o_f32(tmem + TM_AB + lane_addr + 64, tmem + TM_B + lane_addr + 64, gs->gam,
-                                   static_cast<float*>(p.o) + (gbase + t0) * kD + j, n,
+                                   static_cast<float*>(p.o) + (lo.gbase + t0) * kD + j, n,
                                    gated ? sbase + OFF_OST + (j >> 6) * 8192 + (j & 63) * 2 : nullptr);
                 tc_fence_before();
                 mbar_arrive(bar_addr(sb, B_O_DONE));
@@ -885,7 +1006,7 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 // sequence, so the n rows are copied out by plain 16-byte stores (both 64-column
                 // halves of a row: 16 pieces), not by the two box stores
                 const int n = static_cast<int>(L - t0);
-                __nv_bfloat16* orow0 = static_cast<__nv_bfloat16*>(p.o) + (gbase + t0) * kD;
+                __nv_bfloat16* orow0 = static_cast<__nv_bfloat16*>(p.o) + (lo.gbase + t0) * kD;
                 for (int i = j; i < n * 16; i += 128) {
                     const int r = i >> 4, part = i & 15;
                     const uint4 w = *reinterpret_cast<const uint4*>(sbase + OFF_OST + (part >> 3) * 8192 + r * 128 +
@@ -895,9 +1016,9 @@ gdr_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 if (j == 0) mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
             } else if (j == 0) {
                 mbar_arrive(bar_addr(sb, B_GATE_EMPTY + s));
-                if (dbg_ok(t0 < L && zc < p.units_total, err)) {
-                    tma_store_3d(&tm_o, sb + OFF_OST, 0, static_cast<int32_t>(y0 + t0), zc);
-                    tma_store_3d(&tm_o, sb + OFF_OST + 8192, 64, static_cast<int32_t>(y0 + t0), zc);
+                if (dbg_ok(t0 < L && lo.zc < p.units_total, err)) {
+                    tma_store_3d(&tm_o, sb + OFF_OST, 0, static_cast<int32_t>(lo.y0 + t0), lo.zc);
+                    tma_store_3d(&tm_o, sb + OFF_OST + 8192, 64, static_cast<int32_t>(lo.y0 + t0), lo.zc);
                 }
                 bulk_commit_group();
             }
@@ -924,6 +1045,11 @@ bool prefill_tc_supports(int dtype_bf16, int dk, int dv, int per_key)
     return dtype_bf16 && dk == tc::kD && dv == tc::kD;
 }
 
+size_t prefill_tc_flag_bytes(int64_t units)
+{
+    return static_cast<size_t>((units * 4 + 255) / 256 * 256);
+}
+
 cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
 {
     using namespace tc;
@@ -945,14 +1071,67 @@ cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
     if (call.z && !make_bf16_map_3d(&mz, call.z, map_units, call.L, kC, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     const int fb = fuse_bits(call);
-    using K = decltype(&gdr_prefill_tc_kernel<0, false>);
-    static const K kernels[2][8] = {
-        {gdr_prefill_tc_kernel<0, false>, gdr_prefill_tc_kernel<1, false>, gdr_prefill_tc_kernel<2, false>,
-         gdr_prefill_tc_kernel<3, false>, gdr_prefill_tc_kernel<4, false>, gdr_prefill_tc_kernel<5, false>,
-         gdr_prefill_tc_kernel<6, false>, gdr_prefill_tc_kernel<7, false>},
-        {gdr_prefill_tc_kernel<0, true>, gdr_prefill_tc_kernel<1, true>, gdr_prefill_tc_kernel<2, true>,
-         gdr_prefill_tc_kernel<3, true>, gdr_prefill_tc_kernel<4, true>, gdr_prefill_tc_kernel<5, true>,
-         gdr_prefill_tc_kernel<6, true>, gdr_prefill_tc_kernel<7, true>}};
+    using K = decltype(&gdr_prefill_tc_kernel<0, 0>);
+    static const K kernels[3][8] = {
+        {gdr_prefill_tc_kernel<0, 0>, gdr_prefill_tc_kernel<1, 0>, gdr_prefill_tc_kernel<2, 0>,
+         gdr_prefill_tc_kernel<3, 0>, gdr_prefill_tc_kernel<4, 0>, gdr_prefill_tc_kernel<5, 0>,
+         gdr_prefill_tc_kernel<6, 0>, gdr_prefill_tc_kernel<7, 0>},
+        {gdr_prefill_tc_kernel<0, 1>, gdr_prefill_tc_kernel<1, 1>, gdr_prefill_tc_kernel<2, 1>,
+         gdr_prefill_tc_kernel<3, 1>, gdr_prefill_tc_kernel<4, 1>, gdr_prefill_tc_kernel<5, 1>,
+         gdr_prefill_tc_kernel<6, 1>, gdr_prefill_tc_kernel<7, 1>},
+        {gdr_prefill_tc_kernel<0, 2>, gdr_prefill_tc_kernel<1, 2>, gdr_prefill_tc_kernel<2, 2>,
+         gdr_prefill_tc_kernel<3, 2>, gdr_prefill_tc_kernel<4, 2>, gdr_prefill_tc_kernel<5, 2>,
+         gdr_prefill_tc_kernel<6, 2>, gdr_prefill_tc_kernel<7, 2>}};
+    // Balanced schedule: with more units than SMs, one CTA per SM takes an equal share of all
+    // units' chunks (so no SM idles through a partial second wave); it needs S_out (a unit split
+    // between two CTAs hands its state over there) and the caller's workspace (one flag a unit).
+    int sms = 0;
+    if (!var && call.S_out && call.workspace && call.workspace_bytes >= prefill_tc_flag_bytes(units)) {
+        int dev = 0;
+        cudaError_t e0 = cudaGetDevice(&dev);
+        if (e0 == cudaSuccess) e0 = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e0 != cudaSuccess) return e0;
+    }
+    const int64_t nch = (call.L + kC - 1) / kC;
+    const int64_t per_cta = sms > 0 ? (units * nch + sms - 1) / sms : 0;
+    // (a share of per_cta chunks touches at most per_cta / nch + 2 units: kMaxSeg bounds it)
+    if (sms > 0 && units > sms && units <= INT32_MAX / nch && per_cta <= (kMaxSeg - 2) * nch) {
+        const K kernel = kernels[2][fb];
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(SMEM_BYTES));
+        if (e != cudaSuccess) return e;
+        e = cudaMemsetAsync(call.workspace, 0, prefill_tc_flag_bytes(units), stream);
+        if (e != cudaSuccess) return e;
+        NvtxRange range("lt2 prefill, all loops (tensor core, scalar gating, balanced)");
+        Params p;
+        p.alpha = call.alpha;
+        p.beta = call.beta;
+        p.S0 = call.S0;
+        p.o = call.o;
+        p.S_out = call.S_out;
+        p.L = call.L;
+        p.unit0 = 0;
+        p.units_total = static_cast<int>(map_units);
+        p.out_bf16 = call.out_bf16;
+        p.err = call.err;
+        p.qk_norm = call.qk_norm;
+        p.gate_logits = call.gate_logits;
+        p.alpha_scale = call.alpha_scale;
+        p.cu = nullptr;
+        p.Ntot = call.L;
+        p.H = 0;
+        p.loop = 0;
+        p.bal_units = static_cast<int>(units);
+        p.bal_chunks = static_cast<int>(nch);
+        p.bal_per_cta = static_cast<int>(per_cta);     // >= nch, since units > sms
+        p.bal_flags = static_cast<unsigned int*>(call.workspace);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(sms), 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = SMEM_BYTES;
+        cfg.stream = stream;
+        return cudaLaunchKernelEx(&cfg, kernel, mq, mk, mv, call.out_bf16 ? mo : mv, call.z ? mz : mv, p, 0);
+    }
     const K kernel = kernels[var ? 1 : 0][fb];
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM_BYTES));
@@ -977,6 +1156,10 @@ cudaError_t launch_prefill_tc_all(const TcCall& call, cudaStream_t stream)
         p.Ntot = call.L;
         p.H = static_cast<int>(call.H);
         p.loop = static_cast<int>(tau);
+        p.bal_units = 0;
+        p.bal_chunks = 0;
+        p.bal_per_cta = 0;
+        p.bal_flags = nullptr;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(call.units_per_loop), 1, 1);
         cfg.blockDim = dim3(kThreads, 1, 1);

@@ -244,6 +244,10 @@ size_t lt2_gdr_prefill_workspace_bytes(const lt2_gdr_dims* dims)
 {
     Sizes sz;
     if (validate_dims(dims, &sz) != LT2_OK) return 0;
+    // the scalar tensor-core prefill's balanced schedule: one flag per unit
+    if (dims->gate == LT2_GATE_SCALAR && dims->algo != LT2_ALGO_CUDA_CORE && sz.units > 0 &&
+        lt2::prefill_tc_supports(dims->dtype == LT2_DTYPE_BF16, (int)dims->dk, (int)dims->dv, 0))
+        return lt2::prefill_tc_flag_bytes(sz.units);
     return 0;
 }
 
@@ -272,11 +276,13 @@ lt2_status lt2_gdr_prefill_fused(const lt2_gdr_dims* dims, const lt2_gdr_fused* 
         !tensor_ok(alpha, sz.al) || !tensor_ok(beta, sz.be) || !tensor_ok(o, sz.vo))
         return LT2_ERR_INVALID_ARGUMENT;
     if ((S0 && !aligned16(S0)) || (S_out && !aligned16(S_out))) return LT2_ERR_INVALID_ARGUMENT;
+    // The workspace is optional: without it the scalar tensor-core prefill runs one unit per CTA.
     const size_t need = lt2_gdr_prefill_workspace_bytes(dims);
-    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+    if (workspace != nullptr && need > 0 && (workspace_bytes < need || !aligned16(workspace)))
         return LT2_ERR_WORKSPACE;
+    if (need == 0) workspace = nullptr;
     // Aliasing: o and S_out are written; neither may overlap an input or each other
-    // (S_out == S0 exactly is the documented in-place resume).
+    // (S_out == S0 exactly is the documented in-place resume); nor may the workspace.
     const Range ro = range_of(o, sz.vo * sz.osz);
     const Range rin[5] = {range_of(q, sz.qk * sz.esz), range_of(k, sz.qk * sz.esz),
                           range_of(v, sz.vo * sz.esz), range_of(alpha, sz.al * 4),
@@ -291,6 +297,14 @@ lt2_status lt2_gdr_prefill_fused(const lt2_gdr_dims* dims, const lt2_gdr_fused* 
             if (overlap(rs, r)) return LT2_ERR_INVALID_ARGUMENT;
         if (S0 && S0 != S_out && overlap(rs, range_of(S0, sz.st * 4)))
             return LT2_ERR_INVALID_ARGUMENT;
+    }
+    if (workspace) {
+        const Range rw = range_of(workspace, static_cast<int64_t>(need));
+        if (overlap(rw, ro) || (S_out && overlap(rw, range_of(S_out, sz.st * 4))) ||
+            (S0 && overlap(rw, range_of(S0, sz.st * 4))))
+            return LT2_ERR_INVALID_ARGUMENT;
+        for (const Range& r : rin)
+            if (overlap(rw, r)) return LT2_ERR_INVALID_ARGUMENT;
     }
     st = validate_fused(f, sz, o, S_out);
     if (st != LT2_OK) return st;
@@ -325,6 +339,8 @@ lt2_status lt2_gdr_prefill_fused(const lt2_gdr_dims* dims, const lt2_gdr_fused* 
         call.gate_logits = f.gate_logits;
         call.alpha_scale = f.alpha_scale;
         call.z = f.z;
+        call.workspace = workspace;
+        call.workspace_bytes = workspace_bytes;
         cudaError_t e = is_per_key(dims) ? lt2::launch_prefill_kda_tc_all(call, s)
                                          : lt2::launch_prefill_tc_all(call, s);
         if (e == cudaSuccess) e = cudaGetLastError();

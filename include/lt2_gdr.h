@@ -143,9 +143,14 @@ typedef struct lt2_gdr_fused {
 } lt2_gdr_fused;
 
 /*
- * Bytes of device workspace lt2_gdr_prefill needs for `dims` (0 when none; every path of this
- * version keeps its intermediates on chip, so it is 0 for every valid `dims`).  Pure host
- * function, no CUDA call; returns 0 for invalid dims as well.
+ * Bytes of device workspace lt2_gdr_prefill can use for `dims`: one 4-byte flag per (loop, batch,
+ * head) unit, rounded up to 256, for scalar gating with bf16 inputs and d = 128 (the tensor-core
+ * kernel); 0 otherwise and for invalid dims.  Pure host function, no CUDA call.
+ * The workspace is optional.  Given (with S_out, and more units than the GPU has SMs), the
+ * tensor-core kernel runs every loop in ONE balanced launch: one CTA per SM takes an equal share
+ * of all units' 64-token chunks, so no SM idles through a partial second wave; a unit split
+ * between two CTAs hands its state over through S_out and a flag in the workspace.  Without it,
+ * one launch per loop and one CTA per unit.  The results are the same bit for bit either way.
  */
 size_t lt2_gdr_prefill_workspace_bytes(const lt2_gdr_dims* dims);
 
@@ -162,7 +167,10 @@ size_t lt2_gdr_prefill_workspace_bytes(const lt2_gdr_dims* dims);
  *   S0         initial states, or NULL for zero states
  *   o          outputs, dims->out_dtype (device, written; must not alias an input)
  *   S_out      final states, or NULL (may equal S0 exactly: in-place resume)
- *   workspace  device scratch of lt2_gdr_prefill_workspace_bytes(dims) bytes (NULL when 0)
+ *   workspace  NULL, or device scratch of lt2_gdr_prefill_workspace_bytes(dims) bytes (16-byte
+ *              aligned, not overlapping any other argument; the library zeroes what it uses, on
+ *              `stream`).  Optional: see lt2_gdr_prefill_workspace_bytes.  Calls that overlap on
+ *              the GPU need workspaces of their own
  *   stream     cudaStream_t of the current device
  * Returns LT2_OK once the launches are enqueued; LT2_ERR_INVALID_ARGUMENT, _UNSUPPORTED or
  * _WORKSPACE before any launch; LT2_ERR_CUDA if a launch failed.  Device-side conditions come
