@@ -361,6 +361,18 @@ def call_backward(dims, ws=BASE + 40 * SPAN, ws_bytes=None, **over):
     return lt2.lt2_gdr_backward(dims, *(args[n] for n in names), ws, ws_bytes, 0)
 
 
+def test_prefill_workspace_query(L):
+    # one 4-byte flag per unit, rounded up to 256 bytes, for the scalar bf16 d = 128 tensor-core
+    # prefill (its balanced schedule); 0 for the per-key kernel and the CUDA-core path
+    d = D(dtype=lt2.LT2_DTYPE_BF16, dk=128, dv=128, T=3, B=2, H=50)
+    assert lt2.lt2_gdr_prefill_workspace_bytes(d) == (3 * 2 * 50 * 4 + 255) // 256 * 256
+    assert lt2.lt2_gdr_prefill_workspace_bytes(D(dtype=lt2.LT2_DTYPE_BF16, dk=128, dv=128,
+                                                gate=lt2.LT2_GATE_PER_KEY)) == 0
+    assert lt2.lt2_gdr_prefill_workspace_bytes(D(dtype=lt2.LT2_DTYPE_BF16, dk=128, dv=128,
+                                                algo=lt2.LT2_ALGO_CUDA_CORE)) == 0
+    assert lt2.lt2_gdr_prefill_workspace_bytes(D()) == 0                   # fp32, d = 32
+
+
 def test_backward_workspace_query(L):
     d = D(L=150)
     units, chunks, slices = 2 * 1 * 2, 5, 1                      # d = 32: one 32-column slice

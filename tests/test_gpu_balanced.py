@@ -79,3 +79,30 @@ def test_short_workspace_is_refused():
     S = torch.empty((1, 1, 150, 128, 128), device="cuda")
     st = lt2.lt2_gdr_prefill(dims, x["q"], x["k"], x["v"], x["alpha"], x["beta"], None, o, S, ws, nbytes - 16)
     assert st == lt2.LT2_ERR_WORKSPACE
+
+
+def test_balanced_from_zero_states_and_without_final_state_request():
+    # S0 = NULL (zero states); the balanced schedule needs S_out, which lt2.prefill always passes
+    w = inputs.workload("gdn_prefill", T=3, B=1, H=60, L=129)
+    x = inputs.make_inputs(w, seed=6, device="cuda")
+    dims = lt2.make_dims(w.T, w.B, w.H, w.L, w.d, w.d, lt2.LT2_DTYPE_BF16, lt2.LT2_GATE_SCALAR,
+                         out_dtype=lt2.LT2_OUT_F32)
+    nbytes = lt2.lt2_gdr_prefill_workspace_bytes(dims)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    res = []
+    for use_ws in (True, False):
+        o = torch.empty(x["v"].shape, dtype=torch.float32, device="cuda")
+        S = torch.empty((w.T, w.B, w.H, 128, 128), device="cuda")
+        _call(x, dims, o, S, None, ws if use_ws else None)
+        res.append((o, S))
+    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+    # without S_out the call runs one unit per CTA and gives the same outputs
+    o = torch.empty(x["v"].shape, dtype=torch.float32, device="cuda")
+    _call(x, dims, o, None, None, ws)
+    assert torch.equal(o, res[0][0])
+    units = [(0, 0, 0), (2, 0, 59), (1, 0, 31)]
+    x0 = dict(x, S0=None)
+    o_ref, S_ref = oracle_prefill(x0, False, units=units)
+    check("o (balanced, zero states)", torch.stack([res[0][0][u] for u in units]), o_ref, TOL["bf16"])
+    check("S_T (balanced, zero states)", torch.stack([res[0][1][u] for u in units]), S_ref, TOL["bf16"])
+
