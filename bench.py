@@ -441,6 +441,10 @@ def run_swa(args, world, sampler, peaks, peak_src):
 # about 20 d^2 flops (G += q dO^T, dq = S dO, three column sums, the dk and dalpha row sums, the
 # update of G), and the states it needs cost one forward step, 4 d^2, to recompute.
 BW_FLOP_PER_TOKEN_HEAD = 24 * 128 * 128
+# Its algorithmic bytes per token-head: q, k, v and dO in bf16, alpha and beta, and the fp32
+# gradients dq, dk, dv, dalpha and dbeta (the checkpoints and recomputed states of the workspace
+# are the design's, not the problem's).
+BW_BYTES_PER_TOKEN_HEAD = 4 * 128 * 2 + 2 * 4 + 3 * 128 * 4 + 2 * 4
 # fp32 CUDA-core peak of the part: 148 SMs x 128 fp32 lanes x 2 flops (FMA) x 1.965 GHz
 FP32_ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
@@ -471,18 +475,24 @@ def run_backward(args, world, sampler):
     check_device_status("backward_gdn")
     tokheads = w.T * w.B * w.H * w.L
     tf = tokheads * BW_FLOP_PER_TOKEN_HEAD / (ms * 1e-3) / 1e12
+    kernel, source = "gdr_backward_kernel", "gdr_backward.cu"
+    traffic, traffic_note = traffic_for(kernel, source, tokheads * BW_BYTES_PER_TOKEN_HEAD)
     entry = {"metric": "looped GDR backward tokens*loops/s (gdn_prefill shape)",
              "value": gdist.whole_job_rate(w.T * w.B * w.L, world, ms), "unit": "tokens*loops/s",
              "ms_per_step": ms, "steps": steps,
              "config": dict(config_of(w, world), **{"pass": "backward", "workspace_bytes": ws_bytes}),
-             "roofline": {"bound": "alu", "kernel": "gdr_backward_kernel", "achieved": tf,
+             "roofline": {"bound": "alu", "kernel": kernel, "achieved": tf,
                           "peak": FP32_ALU_PEAK_TFLOPS, "unit": "TFLOP/s", "frac": tf / FP32_ALU_PEAK_TFLOPS,
-                          "traffic": None,
+                          "traffic": traffic,
                           "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz",
                           "algorithmic_per_launch": {"flop": tokheads * BW_FLOP_PER_TOKEN_HEAD,
-                                                     "note": "24 d^2 per token-head: the gradient step and "
-                                                             "one recomputed forward step"}},
+                                                     "bytes": tokheads * BW_BYTES_PER_TOKEN_HEAD,
+                                                     "note": "24 d^2 flops per token-head: the gradient step "
+                                                             "and one recomputed forward step; bytes: inputs "
+                                                             "and gradients, the workspace's states not counted"}},
              "gpu_launches": steps * 5}
+    if traffic_note:
+        entry["roofline"]["traffic_note"] = traffic_note + "; the workspace's per-token states are most of it"
     if sampler is not None:
         entry["clocks"] = sampler.summary(["backward_gdn"])
     del x, out, ws, dO, dSL
