@@ -26,8 +26,9 @@
 //            32-token chunk (a checkpoint) in the workspace;
 //   phase B  takes the chunks from the last: it recomputes the chunk's states from its checkpoint
 //            into the workspace, then sweeps the chunk backwards.
-// The workspace is thread-major (element m of thread i of a state at [m][i]): each thread reads
-// back only what it wrote, in coalesced rows.  A chunk's inputs are staged in shared memory once
+// The workspace is thread-major (element m of thread i of a state at [m / 4][i][m % 4] when the
+// rows move as float4, else at [m][i]): each thread reads back only what it wrote, in coalesced
+// rows.  A chunk's inputs are staged in shared memory once
 // per phase; the sweep reuses S_{t-1} of token t+1 as S_t of token t and loads the next S_{t-1}
 // one token ahead.  The row sums (dq, dk and the per-key dalpha: sums over the slice's 32
 // columns) are summed over a warp's 4 columns with shuffles, parked per warp in shared memory, and
@@ -223,10 +224,41 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
     const float* al = p.alpha + u * L * na;
     const float* be = p.beta + u * L;
     const int nck = static_cast<int>((L + kChunk - 1) / kChunk);
-    // element m of this thread in checkpoint idx: ck[idx * sst + m * 256] (likewise st)
+    // A state in the workspace takes rpw * 256 floats.  Element m of thread i sits at [m][i], or,
+    // when the rows move as float4 (kRpw a multiple of 4), at [m / 4][i][m % 4]; either way at
+    // base + m * 256 from the thread's own base, for m a multiple of 4 in the second layout.
+    constexpr bool kVec = kRpw > 0 && kRpw % 4 == 0;
     const int64_t sst = static_cast<int64_t>(rpw) * kThreads;
-    float* ck = p.ws + (u * gridDim.y + blockIdx.y) * ws_floats_per_block(L, dk) + tid;
+    float* ck = p.ws + (u * gridDim.y + blockIdx.y) * ws_floats_per_block(L, dk) + (kVec ? 4 * tid : tid);
     float* st = ck + nck * sst;                    // [33] states of the chunk being swept
+    auto ws_store = [&](float* dst, const float (&x)[kMaxRows]) {
+        if constexpr (kVec) {
+            #pragma unroll
+            for (int m = 0; m < kRpw; m += 4)
+                *reinterpret_cast<float4*>(dst + m * kThreads) = make_float4(x[m], x[m + 1], x[m + 2], x[m + 3]);
+        } else {
+            #pragma unroll
+            for (int m = 0; m < kMaxRows; ++m)
+                if (m < rpw) dst[m * kThreads] = x[m];
+        }
+    };
+    auto ws_load = [&](float (&x)[kMaxRows], const float* src) {
+        if constexpr (kVec) {
+            #pragma unroll
+            for (int m = 0; m < kRpw; m += 4) {
+                const float4 v4 = *reinterpret_cast<const float4*>(src + m * kThreads);
+                x[m] = v4.x;
+                x[m + 1] = v4.y;
+                x[m + 2] = v4.z;
+                x[m + 3] = v4.w;
+            }
+            #pragma unroll
+            for (int m = kRpw; m < kMaxRows; ++m) x[m] = 0.f;
+        } else {
+            #pragma unroll
+            for (int m = 0; m < kMaxRows; ++m) x[m] = m < rpw ? src[m * kThreads] : 0.f;
+        }
+    };
 
     // the inputs of tokens t0 .. t0+n-1 into shared memory (q and dO only for the reverse sweep);
     // every tensor is 16-byte aligned and d_k, d_v are multiples of 8, so rows move 8 elements at a time
@@ -302,12 +334,14 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
         const float e = sum_row_groups(pe);
         const float vj = sv[tau * kCols + jl];
         const float bd = b * (vj - e), bv = b * vj, be_ = b * e;
+        const float cs = bv - a0 * be_;        // scalar alpha, printed order: a s + (b v - a b e) k
         #pragma unroll
         for (int m = 0; m < kMaxRows; ++m) {
             if (m >= rpw) break;
             const float ar_ = kPK ? ar[m] : a0;
             if (kDF) s[m] = ar_ * s[m] + kr[m] * bd;
-            else s[m] = ar_ * (s[m] - kr[m] * be_) + kr[m] * bv;
+            else if (kPK) s[m] = ar_ * (s[m] - kr[m] * be_) + kr[m] * bv;
+            else s[m] = kr[m] * cs + a0 * s[m];
         }
     };
 
@@ -359,10 +393,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
     for (int ci = 0; ci < nck; ++ci) {
         const int64_t t0 = static_cast<int64_t>(ci) * kChunk;
         const int n = static_cast<int>(L - t0 < kChunk ? L - t0 : kChunk);
-        float* cp = ck + ci * sst;
-        #pragma unroll
-        for (int m = 0; m < kMaxRows; ++m)
-            if (m < rpw) cp[m * kThreads] = s[m];
+        ws_store(ck + ci * sst, s);
         load_chunk(t0, n, false);
         for (int tau = 0; tau < n; ++tau) step(s, tau);
     }
@@ -375,42 +406,23 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
     for (int ci = nck - 1; ci >= 0; --ci) {
         const int64_t t0 = static_cast<int64_t>(ci) * kChunk;
         const int n = static_cast<int>(L - t0 < kChunk ? L - t0 : kChunk);
-        {
-            const float* cp = ck + ci * sst;                    // (in flight while the inputs load)
-            #pragma unroll
-            for (int m = 0; m < kMaxRows; ++m) s[m] = m < rpw ? cp[m * kThreads] : 0.f;
-        }
+        ws_load(s, ck + ci * sst);                              // (in flight while the inputs load)
         load_chunk(t0, n, true);
-        #pragma unroll
-        for (int m = 0; m < kMaxRows; ++m)
-            if (m < rpw) st[m * kThreads] = s[m];
+        ws_store(st, s);
         for (int tau = 0; tau < n; ++tau) {
             step(s, tau);
-            if (tau + 1 < n) {                                  // S_t of the last token stays in s
-                float* sp_ = st + (tau + 1) * sst;
-                #pragma unroll
-                for (int m = 0; m < kMaxRows; ++m)
-                    if (m < rpw) sp_[m * kThreads] = s[m];
-            }
+            if (tau + 1 < n) ws_store(st + (tau + 1) * sst, s); // S_t of the last token stays in s
         }
         // S_t arrives from the previous step (S_{t-1} of token t+1); S_{t-1} is loaded one token ahead
         float sc[kMaxRows], sp[kMaxRows];
-        {
-            const float* sp_ = st + (n - 1) * sst;
-            #pragma unroll
-            for (int m = 0; m < kMaxRows; ++m) {
-                sc[m] = s[m];
-                sp[m] = m < rpw ? sp_[m * kThreads] : 0.f;
-            }
-        }
+        #pragma unroll
+        for (int m = 0; m < kMaxRows; ++m) sc[m] = s[m];
+        ws_load(sp, st + (n - 1) * sst);
         for (int tau = n - 1; tau >= 0; --tau) {
             const int sl = tau % kF;                            // this token's slot among the parked partials
-            float spn[kMaxRows];                               // S_{t-2}, for the next token
-            {
-                const float* sp_ = st + (tau > 0 ? tau - 1 : 0) * sst;
-                #pragma unroll
-                for (int m = 0; m < kMaxRows; ++m) spn[m] = (m < rpw && tau > 0) ? sp_[m * kThreads] : 0.f;
-            }
+            // S_{t-2}, for the next token (at tau = 0 the chunk's first state again, never used)
+            float spn[kMaxRows];
+            ws_load(spn, st + (tau > 0 ? tau - 1 : 0) * sst);
             const float b = sbe[tau];
             const float vj = sv[tau * kCols + jl];
             const float oj = sdo[tau * kCols + jl];
@@ -462,22 +474,30 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
             float dkx[kMaxRows], dax[kMaxRows];
             {
                 const float bkG = b * kG, bkdP = b * kdP, bd = b * (vj - e), bv = b * vj, bE = b * e;
+                // scalar alpha: R bkG = (a bkG) S_{t-1}, and G bv - dP bE = (bv - a bE) G
+                const float abkG = a0 * bkG, cv = bv - a0 * bE;
                 #pragma unroll
                 for (int m = 0; m < kMaxRows; ++m) {
                     dkx[m] = dax[m] = 0.f;
                     if (m >= rpw) continue;
                     const float ar_ = kPK ? ar[m] : a0;
                     if (kDF) {
-                        const float R = ar_ * sp[m];
                         const float dR = G[m] - kr[m] * bkG;
-                        dkx[m] = G[m] * bd - R * bkG;
-                        if (kPK) dax[m] = dR * sp[m];
+                        if (kPK) {
+                            dkx[m] = G[m] * bd - ar_ * sp[m] * bkG;
+                            dax[m] = dR * sp[m];
+                        } else {
+                            dkx[m] = G[m] * bd - sp[m] * abkG;
+                        }
                         G[m] = ar_ * dR;
-                    } else {
+                    } else if (kPK) {
                         const float dP = ar_ * G[m];
                         dkx[m] = G[m] * bv - (sp[m] * bkdP + dP * bE);
-                        if (kPK) dax[m] = G[m] * (sp[m] - kr[m] * bE);
+                        dax[m] = G[m] * (sp[m] - kr[m] * bE);
                         G[m] = dP - kr[m] * bkdP;
+                    } else {
+                        dkx[m] = G[m] * cv - sp[m] * bkdP;
+                        G[m] = a0 * G[m] - kr[m] * bkdP;
                     }
                 }
             }
