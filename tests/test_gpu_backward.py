@@ -54,6 +54,12 @@ def test_backward_bf16_d128_matches_oracle(gate, order):
     _compare(_case(130, 128, "bf16", gate, seed=7), gate == "per_key", order)
 
 
+@pytest.mark.parametrize("gate,order", GATES)
+def test_backward_fp32_d128_matches_oracle(gate, order):
+    # fp32 inputs with d_k = 128: the compile-time instances whose workspace states move as float4
+    _compare(_case(70, 128, "f32", gate, seed=5, T=1, H=2), gate == "per_key", order)
+
+
 def test_backward_without_initial_state_or_final_gradient():
     _compare(_case(70, 64, "f32", "scalar", seed=3, s0=False, dsl=False), False, "delta_first")
 
