@@ -125,13 +125,14 @@ __host__ __device__ inline int64_t ws_floats_per_block(int64_t L, int dk)
 }
 
 // Shared memory of a block: one chunk's inputs in fp32 (k, q, alpha rows, beta, and the slice's v
-// and dO columns), the row-sum partials [dq, dk(, dalpha)][token][warp][row] and the per-warp
-// dbeta and scalar dalpha terms [token][warp].
+// and dO columns), the row-sum partials [dq, dk(, dalpha)][token][warp][row], the per-warp
+// dbeta and scalar dalpha terms [token][warp], and the column sums e of the chunk's tokens
+// [token][column] (about 111 KB with d_k = 128: two blocks per SM).
 __host__ __device__ inline size_t smem_bytes(int dk, int per_key)
 {
     const size_t na = per_key ? dk : 1;
     const size_t f = flush_tokens(per_key != 0), ng = per_key ? 3 : 2;
-    return (static_cast<size_t>(kChunk) * (2 * dk + na + 1 + 2 * kCols) + ng * f * 8 * part_stride(dk) + 2 * f * 8) *
+    return (static_cast<size_t>(kChunk) * (2 * dk + na + 1 + 3 * kCols) + ng * f * 8 * part_stride(dk) + 2 * f * 8) *
            sizeof(float);
 }
 
@@ -216,6 +217,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
     float* part = sdo + kChunk * kCols;            // [kNg][kF][8][ps]
     float* pbe = part + kNg * kF * 8 * ps;         // [kF][8]
     float* pal = pbe + kF * 8;                     // [kF][8] (scalar alpha)
+    float* se = pal + kF * 8;                      // [32][32] e of the chunk's tokens, from the recompute
 
     const T* q = static_cast<const T*>(p.q) + u * L * dk;
     const T* k = static_cast<const T*>(p.k) + u * L * dk;
@@ -320,7 +322,9 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
     };
 
     // one forward step of the recurrence (token tau of the loaded chunk) on this thread's state
-    auto step = [&](float (&s)[kMaxRows], int tau) {
+    // (keep_e: the column sum e of the token goes to se for the reverse sweep, which needs the same
+    // value, computed from the same S_{t-1} in the same order)
+    auto step = [&](float (&s)[kMaxRows], int tau, bool keep_e) {
         const float b = sbe[tau];
         float kr[kMaxRows], ar[kMaxRows];
         lds_rows<kRpw>(sk + tau * dk + r0, kr, rpw);
@@ -332,6 +336,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
             if (m < rpw) pe += kr[m] * ((kDF && kPK) ? ar[m] * s[m] : s[m]);
         if (kDF && !kPK) pe *= a0;
         const float e = sum_row_groups(pe);
+        if (keep_e && g == 0) se[tau * kCols + jl] = e;
         const float vj = sv[tau * kCols + jl];
         const float bd = b * (vj - e), bv = b * vj, be_ = b * e;
         const float cs = bv - a0 * be_;        // scalar alpha, printed order: a s + (b v - a b e) k
@@ -395,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
         const int n = static_cast<int>(L - t0 < kChunk ? L - t0 : kChunk);
         ws_store(ck + ci * sst, s);
         load_chunk(t0, n, false);
-        for (int tau = 0; tau < n; ++tau) step(s, tau);
+        for (int tau = 0; tau < n; ++tau) step(s, tau, false);
     }
 
     // ---- phase B: chunks from the last, each recomputed, then swept backwards ----
@@ -410,9 +415,10 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
         load_chunk(t0, n, true);
         ws_store(st, s);
         for (int tau = 0; tau < n; ++tau) {
-            step(s, tau);
+            step(s, tau, true);
             if (tau + 1 < n) ws_store(st + (tau + 1) * sst, s); // S_t of the last token stays in s
         }
+        __syncwarp();                                           // se is read by the warp's other lanes
         // S_t arrives from the previous step (S_{t-1} of token t+1); S_{t-1} is loaded one token ahead
         float sc[kMaxRows], sp[kMaxRows];
         #pragma unroll
@@ -448,18 +454,20 @@ __global__ void __launch_bounds__(kThreads, 2) gdr_backward_kernel(Params p)
             // (with a scalar alpha the third is alpha k^T G, and e of the decay-first order alpha k^T S)
             // (scalar alpha: gs = G . S_{t-1} over the thread's rows gives its dalpha term without a
             // per-element product: sum G P = gs - b e pg, sum dR S_{t-1} = gs - b kG ks)
+            // e comes from the recompute, except with a scalar alpha in the decay-first order, whose
+            // dalpha term needs this thread's share ks of k^T S_{t-1}
+            constexpr bool kOwnE = kDF && !kPK;
             float pe = 0.f, pg = 0.f, pd = 0.f, gs = 0.f;
             #pragma unroll
             for (int m = 0; m < kMaxRows; ++m) {
                 if (m >= rpw) break;
-                pe += kr[m] * ((kDF && kPK) ? ar[m] * sp[m] : sp[m]);
+                if (kOwnE) pe += kr[m] * sp[m];
                 pg += kr[m] * G[m];
                 if (kPK) pd += kr[m] * ar[m] * G[m];
                 if (!kPK) gs += G[m] * sp[m];
             }
-            const float ks = pe;                        // k^T S_{t-1} over the thread's rows
-            if (kDF && !kPK) pe *= a0;
-            const float e = sum_row_groups(pe);
+            const float ks = pe;                        // k^T S_{t-1} over the thread's rows (kOwnE)
+            const float e = kOwnE ? sum_row_groups(pe * a0) : se[tau * kCols + jl];
             const float kG = sum_row_groups(pg);
             const float kdP = kPK ? sum_row_groups(pd) : a0 * kG;
             if (active && g == 0) p.gdv[(u * L + t0 + tau) * dv + j] = b * kG;
